@@ -1,0 +1,763 @@
+// Causal / sliding-window flash attention, forward and backward, for head_dim 32, 64 or 128.
+//
+// The causal softmax attention of the nanochat decoder ("nanochat User Guide" §10: sliding-window
+// attention pattern; queries see keys t−w < j ≤ t).  Q/K/V/dO tiles are staged into shared memory
+// by 4-D TMA loads (128-byte swizzle, double-buffered, mbarrier completion); the products run on
+// the tensor cores as m16n8k16 bf16 MMAs with fp32 accumulation; the online softmax lives in
+// registers, with row statistics reduced over each quad by warp shuffles.  KV tiles entirely
+// outside the causal band or the window are never loaded.
+//
+//   forward     grid (q tiles of 128, H, B), 8 warps × 16 query rows; O and LSE (natural log).
+//   backward    (1) delta = rowsum(dO∘O);  (2) dK, dV: grid over 64-key tiles, loop over the query
+//               tiles that see them;  (3) dQ: grid over 64-query tiles, loop over their key tiles.
+//               No atomics: every output element is written by exactly one thread, so results are
+//               bitwise reproducible.
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "host.h"
+
+namespace gpt {
+
+namespace {
+
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+
+struct AttnArgs {
+  int B, H, T, window;  // window: effective (T for full causal)
+  float scale_log2;     // log2(e)/sqrt(Dh)
+  float scale;          // 1/sqrt(Dh)
+  uint16_t* o;          // forward output / backward dq
+  uint16_t* dk;
+  uint16_t* dv;
+  long long sb_o, sh_o, st_o;        // strides of o (fwd) or of dq/dk/dv (bwd)
+  const uint16_t* obuf;              // bwd: o
+  const uint16_t* dobuf;             // bwd: dO
+  long long sb_d, sh_d, st_d;        // strides of o/dO in the backward
+  float* lse;
+  float* delta;
+  int* status;
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Address of element (r, c) (c a multiple of 8) of a [ROWS × DH] bf16 tile in shared memory.
+// DH ≥ 64: stored as [DH/64][ROWS][64] with the TMA 128-byte swizzle (16-byte unit u of row r lives
+// at unit u ^ (r & 7)); DH = 32: plain rows of 64 bytes.  base is 1024-byte aligned.
+template <int DH, int ROWS>
+__device__ __forceinline__ uint32_t swz(uint32_t base, int r, int c) {
+  if constexpr (DH >= 64) {
+    return base + (uint32_t)((c >> 6) * ROWS * 128 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4));
+  } else {
+    return base + (uint32_t)(r * DH * 2 + ((c >> 3) << 4));
+  }
+}
+
+// Issue the TMA loads of a [ROWS × DH] tile at sequence row t0 of head (b, h).
+template <int DH, int ROWS>
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
+                                          int t0, int h, int b) {
+  if constexpr (DH >= 64) {
+#pragma unroll
+    for (int c = 0; c < DH / 64; ++c) tma_load_4d(dst + c * ROWS * 128, map, bar, c * 64, t0, h, b);
+  } else {
+    tma_load_4d(dst, map, bar, 0, t0, h, b);
+  }
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) &
+                                    ~static_cast<uintptr_t>(1023));
+}
+
+// ================================================================================================
+// forward
+// ================================================================================================
+template <int DH>
+struct FwdShape {
+  static constexpr int BMQ = 128, BNK = 64;
+  static constexpr int Q_BYTES = BMQ * DH * 2, KV_BYTES = BNK * DH * 2;
+  static constexpr int SMEM = Q_BYTES + 4 * KV_BYTES + 1024 + 64;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(256)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                    const __grid_constant__ CUtensorMap mv, const AttnArgs a) {
+  using S = FwdShape<DH>;
+  constexpr int BMQ = S::BMQ, BNK = S::BNK;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sQ = smem;
+  uint8_t* sK0 = smem + S::Q_BYTES;
+  uint8_t* sV0 = sK0 + 2 * S::KV_BYTES;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sV0 + 2 * S::KV_BYTES);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 3);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t4 = lane & 3;
+  const int qt = gridDim.x - 1 - blockIdx.x;  // longest rows first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int T = a.T, W = a.window;
+  const int q0 = qt * BMQ;
+  const int key_lo = max(0, q0 - W + 1);
+  const int key_hi = min(T, q0 + BMQ);
+  const int kv_first = key_lo / BNK;
+  const int n_kv = (key_hi - 1) / BNK - kv_first + 1;
+
+  if (tid == 0) {
+    for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bar[0], S::Q_BYTES);
+    load_tile<DH, BMQ>(sQ, &mq, &bar[0], q0, h, b);
+    for (int i = 0; i < 2 && i < n_kv; ++i) {
+      mbar_arrive_expect_tx(&bar[1 + i], 2 * S::KV_BYTES);
+      load_tile<DH, BNK>(sK0 + i * S::KV_BYTES, &mk, &bar[1 + i], (kv_first + i) * BNK, h, b);
+      load_tile<DH, BNK>(sV0 + i * S::KV_BYTES, &mv, &bar[1 + i], (kv_first + i) * BNK, h, b);
+    }
+  }
+  bool ok = mbar_wait(&bar[0], 0, abort_flag, a.status);
+
+  uint32_t qf[DH / 16][4];
+  {
+    const uint32_t base = smem_u32(sQ);
+    const int r = 16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+    for (int kk = 0; kk < DH / 16; ++kk)
+      ldsm_x4(swz<DH, BMQ>(base, r, 16 * kk + 8 * (lane >> 4)), qf[kk][0], qf[kk][1], qf[kk][2],
+              qf[kk][3]);
+  }
+
+  float o[DH / 8][4];
+#pragma unroll
+  for (int i = 0; i < DH / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+  const int row0 = q0 + 16 * warp + g;  // rows row0 and row0 + 8
+
+  for (int i = 0; i < n_kv && ok; ++i) {
+    const int buf = i & 1;
+    if (!mbar_wait(&bar[1 + buf], (i >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+    const int kv0 = (kv_first + i) * BNK;
+    const uint32_t kb = smem_u32(sK0 + buf * S::KV_BYTES);
+    const uint32_t vb = smem_u32(sV0 + buf * S::KV_BYTES);
+    float s[8][4];
+#pragma unroll
+    for (int n = 0; n < 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < DH / 16; ++kk) {
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(swz<DH, BNK>(kb, 16 * np + (lane & 7) + 8 * (lane >> 4), 16 * kk + 8 * ((lane >> 3) & 1)),
+                b0, b1, b2, b3);
+        mma16816(s[2 * np], qf[kk], b0, b1);
+        mma16816(s[2 * np + 1], qf[kk], b2, b3);
+      }
+    }
+    const bool need_mask = (kv0 + BNK - 1 > q0) || (kv0 <= q0 + BMQ - 1 - W);
+#pragma unroll
+    for (int n = 0; n < 8; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float x = s[n][e] * a.scale_log2;
+        if (need_mask) {
+          const int row = row0 + 8 * (e >> 1);
+          const int key = kv0 + 8 * n + 2 * t4 + (e & 1);
+          if (!(key <= row && key > row - W)) x = -INFINITY;
+        }
+        s[n][e] = x;
+      }
+    // online softmax (log2 domain)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int n = 0; n < 8; ++n) mx = fmaxf(mx, fmaxf(s[n][2 * r], s[n][2 * r + 1]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float mnew = fmaxf(mrow[r], mx);
+      const float muse = (mnew == -INFINITY) ? 0.f : mnew;
+      const float alpha = exp2f(mrow[r] - muse);
+      mrow[r] = mnew;
+      float ls = 0.f;
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        s[n][2 * r] = exp2f(s[n][2 * r] - muse);
+        s[n][2 * r + 1] = exp2f(s[n][2 * r + 1] - muse);
+        ls += s[n][2 * r] + s[n][2 * r + 1];
+      }
+      lrow[r] = lrow[r] * alpha + ls;
+#pragma unroll
+      for (int d = 0; d < DH / 8; ++d) {
+        o[d][2 * r] *= alpha;
+        o[d][2 * r + 1] *= alpha;
+      }
+    }
+    // O += P·V
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t pa[4];
+      pa[0] = pack_bf2(s[2 * ks][0], s[2 * ks][1]);
+      pa[1] = pack_bf2(s[2 * ks][2], s[2 * ks][3]);
+      pa[2] = pack_bf2(s[2 * ks + 1][0], s[2 * ks + 1][1]);
+      pa[3] = pack_bf2(s[2 * ks + 1][2], s[2 * ks + 1][3]);
+#pragma unroll
+      for (int dp = 0; dp < DH / 16; ++dp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(swz<DH, BNK>(vb, 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1), 16 * dp + 8 * (lane >> 4)),
+                  b0, b1, b2, b3);
+        mma16816(o[2 * dp], pa, b0, b1);
+        mma16816(o[2 * dp + 1], pa, b2, b3);
+      }
+    }
+    __syncthreads();
+    if (tid == 0 && i + 2 < n_kv) {
+      mbar_arrive_expect_tx(&bar[1 + buf], 2 * S::KV_BYTES);
+      load_tile<DH, BNK>(sK0 + buf * S::KV_BYTES, &mk, &bar[1 + buf], (kv_first + i + 2) * BNK, h, b);
+      load_tile<DH, BNK>(sV0 + buf * S::KV_BYTES, &mv, &bar[1 + buf], (kv_first + i + 2) * BNK, h, b);
+    }
+  }
+  // finalize
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    float l = lrow[r];
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    const int row = row0 + 8 * r;
+    if (row < T && ok) {
+      const float inv = 1.f / l;
+      uint16_t* orow = a.o + b * a.sb_o + h * a.sh_o + (long long)row * a.st_o;
+#pragma unroll
+      for (int d = 0; d < DH / 8; ++d)
+        *reinterpret_cast<uint32_t*>(orow + 8 * d + 2 * t4) =
+            pack_bf2(o[d][2 * r] * inv, o[d][2 * r + 1] * inv);
+      if (t4 == 0) a.lse[((long long)b * a.H + h) * T + row] = (mrow[r] + log2f(l)) * LN2;
+    }
+  }
+  if (*abort_flag && tid == 0) {
+    for (int i = 0; i < 2000; ++i) __nanosleep(1000);  // let in-flight copies land before exit
+  }
+}
+
+// ================================================================================================
+// backward (1): delta = rowsum(dO ∘ O), one warp per row
+// ================================================================================================
+__global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
+                                  float* __restrict__ delta, int B, int H, int T, int Dh,
+                                  long long sb, long long sh, long long st) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const long long rows = (long long)B * H * T;
+  if (warp >= rows) return;
+  const int t = warp % T, h = (warp / T) % H, b = warp / (T * H);
+  const long long off = b * sb + h * sh + (long long)t * st;
+  float acc = 0.f;
+  for (int j = 2 * lane; j < Dh; j += 64) {
+    const uint32_t x = *reinterpret_cast<const uint32_t*>(o + off + j);
+    const uint32_t y = *reinterpret_cast<const uint32_t*>(dout + off + j);
+    acc += bf_lo(x) * bf_lo(y) + bf_hi(x) * bf_hi(y);
+  }
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (lane == 0) delta[warp] = acc;
+}
+
+// ================================================================================================
+// backward (2): dK, dV for a 64-key tile; 4 warps × 16 keys; loop over 64-query tiles
+// ================================================================================================
+template <int DH>
+struct BwdShape {
+  static constexpr int BNK = 64, BMQ = 64;
+  static constexpr int TILE = 64 * DH * 2;
+  static constexpr int SMEM = 6 * TILE + 1024 + 64;  // K, V, 2×Q, 2×dO  (dkdv) / Q, dO, 2×K, 2×V (dq)
+};
+
+template <int DH>
+__global__ void __launch_bounds__(128)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                         const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
+                         const AttnArgs a) {
+  using S = BwdShape<DH>;
+  constexpr int BNK = S::BNK, BMQ = S::BMQ;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + S::TILE;
+  uint8_t* sQ0 = smem + 2 * S::TILE;   // 2 buffers
+  uint8_t* sD0 = smem + 4 * S::TILE;   // 2 buffers of dO
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 6 * S::TILE);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 3);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t4 = lane & 3;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int T = a.T, W = a.window;
+  const int kv0 = blockIdx.x * BNK;
+  const int q_first = kv0 / BMQ;
+  const int q_last = min(T - 1, kv0 + BNK - 1 + W - 1) / BMQ;
+  const int n_q = q_last - q_first + 1;
+  const long long bh = (long long)b * a.H + h;
+
+  if (tid == 0) {
+    for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bar[0], 2 * S::TILE);
+    load_tile<DH, BNK>(sK, &mk, &bar[0], kv0, h, b);
+    load_tile<DH, BNK>(sV, &mv, &bar[0], kv0, h, b);
+    for (int i = 0; i < 2 && i < n_q; ++i) {
+      mbar_arrive_expect_tx(&bar[1 + i], 2 * S::TILE);
+      load_tile<DH, BMQ>(sQ0 + i * S::TILE, &mq, &bar[1 + i], (q_first + i) * BMQ, h, b);
+      load_tile<DH, BMQ>(sD0 + i * S::TILE, &mdo, &bar[1 + i], (q_first + i) * BMQ, h, b);
+    }
+  }
+  bool ok = mbar_wait(&bar[0], 0, abort_flag, a.status);
+
+  float dk[DH / 8][4], dv[DH / 8][4];
+#pragma unroll
+  for (int i = 0; i < DH / 8; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dk[i][e] = dv[i][e] = 0.f;
+
+  const uint32_t kbase = smem_u32(sK), vbase = smem_u32(sV);
+  const int arow = 16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1);  // A-operand ldmatrix row
+  const int key_r0 = kv0 + 16 * warp + g;                           // keys key_r0, key_r0 + 8
+
+  for (int i = 0; i < n_q && ok; ++i) {
+    const int buf = i & 1;
+    if (!mbar_wait(&bar[1 + buf], (i >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+    const int q0 = (q_first + i) * BMQ;
+    const uint32_t qb = smem_u32(sQ0 + buf * S::TILE);
+    const uint32_t db = smem_u32(sD0 + buf * S::TILE);
+    float st[8][4], dp[8][4];
+#pragma unroll
+    for (int n = 0; n < 8; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) st[n][e] = dp[n][e] = 0.f;
+    // Sᵀ = K·Qᵀ and dPᵀ = V·dOᵀ   (16 keys × 64 queries per warp)
+#pragma unroll
+    for (int kk = 0; kk < DH / 16; ++kk) {
+      uint32_t ka[4], va[4];
+      ldsm_x4(swz<DH, BNK>(kbase, arow, 16 * kk + 8 * (lane >> 4)), ka[0], ka[1], ka[2], ka[3]);
+      ldsm_x4(swz<DH, BNK>(vbase, arow, 16 * kk + 8 * (lane >> 4)), va[0], va[1], va[2], va[3]);
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+        const int br = 16 * np + (lane & 7) + 8 * (lane >> 4);
+        const int bc = 16 * kk + 8 * ((lane >> 3) & 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(swz<DH, BMQ>(qb, br, bc), b0, b1, b2, b3);
+        mma16816(st[2 * np], ka, b0, b1);
+        mma16816(st[2 * np + 1], ka, b2, b3);
+        ldsm_x4(swz<DH, BMQ>(db, br, bc), b0, b1, b2, b3);
+        mma16816(dp[2 * np], va, b0, b1);
+        mma16816(dp[2 * np + 1], va, b2, b3);
+      }
+    }
+    // Pᵀ and dSᵀ
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      const int qa = q0 + 8 * n + 2 * t4;
+      float l2[2], dl[2];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int qq = qa + c;
+        l2[c] = (qq < T) ? a.lse[bh * T + qq] * LOG2E : 0.f;
+        dl[c] = (qq < T) ? a.delta[bh * T + qq] : 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = key_r0 + 8 * (e >> 1);
+        const int qq = qa + (e & 1);
+        const bool vis = (qq < T) && (key <= qq) && (key > qq - W);
+        const float p = vis ? exp2f(st[n][e] * a.scale_log2 - l2[e & 1]) : 0.f;
+        st[n][e] = p;
+        dp[n][e] = p * (dp[n][e] - dl[e & 1]);
+      }
+    }
+    // dV += Pᵀ·dO,  dK += dSᵀ·Q
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t pa[4], sa[4];
+      pa[0] = pack_bf2(st[2 * ks][0], st[2 * ks][1]);
+      pa[1] = pack_bf2(st[2 * ks][2], st[2 * ks][3]);
+      pa[2] = pack_bf2(st[2 * ks + 1][0], st[2 * ks + 1][1]);
+      pa[3] = pack_bf2(st[2 * ks + 1][2], st[2 * ks + 1][3]);
+      sa[0] = pack_bf2(dp[2 * ks][0], dp[2 * ks][1]);
+      sa[1] = pack_bf2(dp[2 * ks][2], dp[2 * ks][3]);
+      sa[2] = pack_bf2(dp[2 * ks + 1][0], dp[2 * ks + 1][1]);
+      sa[3] = pack_bf2(dp[2 * ks + 1][2], dp[2 * ks + 1][3]);
+#pragma unroll
+      for (int dpair = 0; dpair < DH / 16; ++dpair) {
+        const int tr = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int tc = 16 * dpair + 8 * (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(swz<DH, BMQ>(db, tr, tc), b0, b1, b2, b3);
+        mma16816(dv[2 * dpair], pa, b0, b1);
+        mma16816(dv[2 * dpair + 1], pa, b2, b3);
+        ldsm_x4_t(swz<DH, BMQ>(qb, tr, tc), b0, b1, b2, b3);
+        mma16816(dk[2 * dpair], sa, b0, b1);
+        mma16816(dk[2 * dpair + 1], sa, b2, b3);
+      }
+    }
+    __syncthreads();
+    if (tid == 0 && i + 2 < n_q) {
+      mbar_arrive_expect_tx(&bar[1 + buf], 2 * S::TILE);
+      load_tile<DH, BMQ>(sQ0 + buf * S::TILE, &mq, &bar[1 + buf], (q_first + i + 2) * BMQ, h, b);
+      load_tile<DH, BMQ>(sD0 + buf * S::TILE, &mdo, &bar[1 + buf], (q_first + i + 2) * BMQ, h, b);
+    }
+  }
+  if (ok) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int key = key_r0 + 8 * r;
+      if (key < T) {
+        const long long off = b * a.sb_o + h * a.sh_o + (long long)key * a.st_o;
+#pragma unroll
+        for (int d = 0; d < DH / 8; ++d) {
+          *reinterpret_cast<uint32_t*>(a.dk + off + 8 * d + 2 * t4) =
+              pack_bf2(dk[d][2 * r] * a.scale, dk[d][2 * r + 1] * a.scale);
+          *reinterpret_cast<uint32_t*>(a.dv + off + 8 * d + 2 * t4) =
+              pack_bf2(dv[d][2 * r], dv[d][2 * r + 1]);
+        }
+      }
+    }
+  }
+  if (*abort_flag && tid == 0) {
+    for (int i = 0; i < 2000; ++i) __nanosleep(1000);
+  }
+}
+
+// ================================================================================================
+// backward (3): dQ for a 64-query tile; 4 warps × 16 rows; loop over key tiles
+// ================================================================================================
+template <int DH>
+__global__ void __launch_bounds__(128)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                       const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
+                       const AttnArgs a) {
+  using S = BwdShape<DH>;
+  constexpr int BNK = S::BNK, BMQ = S::BMQ;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sQ = smem;
+  uint8_t* sD = smem + S::TILE;
+  uint8_t* sK0 = smem + 2 * S::TILE;  // 2 buffers
+  uint8_t* sV0 = smem + 4 * S::TILE;  // 2 buffers
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 6 * S::TILE);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 3);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t4 = lane & 3;
+  const int qt = gridDim.x - 1 - blockIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int T = a.T, W = a.window;
+  const int q0 = qt * BMQ;
+  const int key_lo = max(0, q0 - W + 1);
+  const int key_hi = min(T, q0 + BMQ);
+  const int kv_first = key_lo / BNK;
+  const int n_kv = (key_hi - 1) / BNK - kv_first + 1;
+  const long long bh = (long long)b * a.H + h;
+
+  if (tid == 0) {
+    for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bar[0], 2 * S::TILE);
+    load_tile<DH, BMQ>(sQ, &mq, &bar[0], q0, h, b);
+    load_tile<DH, BMQ>(sD, &mdo, &bar[0], q0, h, b);
+    for (int i = 0; i < 2 && i < n_kv; ++i) {
+      mbar_arrive_expect_tx(&bar[1 + i], 2 * S::TILE);
+      load_tile<DH, BNK>(sK0 + i * S::TILE, &mk, &bar[1 + i], (kv_first + i) * BNK, h, b);
+      load_tile<DH, BNK>(sV0 + i * S::TILE, &mv, &bar[1 + i], (kv_first + i) * BNK, h, b);
+    }
+  }
+  bool ok = mbar_wait(&bar[0], 0, abort_flag, a.status);
+
+  uint32_t qf[DH / 16][4], df[DH / 16][4];
+  {
+    const int r = 16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+    for (int kk = 0; kk < DH / 16; ++kk) {
+      ldsm_x4(swz<DH, BMQ>(smem_u32(sQ), r, 16 * kk + 8 * (lane >> 4)), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+      ldsm_x4(swz<DH, BMQ>(smem_u32(sD), r, 16 * kk + 8 * (lane >> 4)), df[kk][0], df[kk][1], df[kk][2], df[kk][3]);
+    }
+  }
+  const int row0 = q0 + 16 * warp + g;
+  float l2[2], dl[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int row = row0 + 8 * r;
+    l2[r] = (row < T) ? a.lse[bh * T + row] * LOG2E : 0.f;
+    dl[r] = (row < T) ? a.delta[bh * T + row] : 0.f;
+  }
+  float dq[DH / 8][4];
+#pragma unroll
+  for (int i = 0; i < DH / 8; ++i) dq[i][0] = dq[i][1] = dq[i][2] = dq[i][3] = 0.f;
+
+  for (int i = 0; i < n_kv && ok; ++i) {
+    const int buf = i & 1;
+    if (!mbar_wait(&bar[1 + buf], (i >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+    const int kv0 = (kv_first + i) * BNK;
+    const uint32_t kb = smem_u32(sK0 + buf * S::TILE);
+    const uint32_t vb = smem_u32(sV0 + buf * S::TILE);
+    float s[8][4], dp[8][4];
+#pragma unroll
+    for (int n = 0; n < 8; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[n][e] = dp[n][e] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < DH / 16; ++kk) {
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+        const int br = 16 * np + (lane & 7) + 8 * (lane >> 4);
+        const int bc = 16 * kk + 8 * ((lane >> 3) & 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(swz<DH, BNK>(kb, br, bc), b0, b1, b2, b3);
+        mma16816(s[2 * np], qf[kk], b0, b1);
+        mma16816(s[2 * np + 1], qf[kk], b2, b3);
+        ldsm_x4(swz<DH, BNK>(vb, br, bc), b0, b1, b2, b3);
+        mma16816(dp[2 * np], df[kk], b0, b1);
+        mma16816(dp[2 * np + 1], df[kk], b2, b3);
+      }
+    }
+#pragma unroll
+    for (int n = 0; n < 8; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int row = row0 + 8 * (e >> 1);
+        const int key = kv0 + 8 * n + 2 * t4 + (e & 1);
+        const bool vis = (row < T) && (key <= row) && (key > row - W);
+        const float p = vis ? exp2f(s[n][e] * a.scale_log2 - l2[e >> 1]) : 0.f;
+        dp[n][e] = p * (dp[n][e] - dl[e >> 1]);
+      }
+    // dQ += dS·K
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t sa[4];
+      sa[0] = pack_bf2(dp[2 * ks][0], dp[2 * ks][1]);
+      sa[1] = pack_bf2(dp[2 * ks][2], dp[2 * ks][3]);
+      sa[2] = pack_bf2(dp[2 * ks + 1][0], dp[2 * ks + 1][1]);
+      sa[3] = pack_bf2(dp[2 * ks + 1][2], dp[2 * ks + 1][3]);
+#pragma unroll
+      for (int dpair = 0; dpair < DH / 16; ++dpair) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(swz<DH, BNK>(kb, 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1), 16 * dpair + 8 * (lane >> 4)),
+                  b0, b1, b2, b3);
+        mma16816(dq[2 * dpair], sa, b0, b1);
+        mma16816(dq[2 * dpair + 1], sa, b2, b3);
+      }
+    }
+    __syncthreads();
+    if (tid == 0 && i + 2 < n_kv) {
+      mbar_arrive_expect_tx(&bar[1 + buf], 2 * S::TILE);
+      load_tile<DH, BNK>(sK0 + buf * S::TILE, &mk, &bar[1 + buf], (kv_first + i + 2) * BNK, h, b);
+      load_tile<DH, BNK>(sV0 + buf * S::TILE, &mv, &bar[1 + buf], (kv_first + i + 2) * BNK, h, b);
+    }
+  }
+  if (ok) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int row = row0 + 8 * r;
+      if (row < T) {
+        uint16_t* dst = a.o + b * a.sb_o + h * a.sh_o + (long long)row * a.st_o;
+#pragma unroll
+        for (int d = 0; d < DH / 8; ++d)
+          *reinterpret_cast<uint32_t*>(dst + 8 * d + 2 * t4) =
+              pack_bf2(dq[d][2 * r] * a.scale, dq[d][2 * r + 1] * a.scale);
+      }
+    }
+  }
+  if (*abort_flag && tid == 0) {
+    for (int i = 0; i < 2000; ++i) __nanosleep(1000);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// host helpers
+// ------------------------------------------------------------------------------------------------
+bool make_head_map(CUtensorMap* m, const void* base, int B, int H, int T, int Dh, long long sb,
+                   long long sh, long long st, int rows) {
+  const uint64_t dims[4] = {(uint64_t)Dh, (uint64_t)T, (uint64_t)H, (uint64_t)B};
+  const uint64_t strides[3] = {(uint64_t)st * 2, (uint64_t)sh * 2, (uint64_t)sb * 2};
+  const uint32_t box[4] = {(uint32_t)std::min(Dh, 64), (uint32_t)rows, 1, 1};
+  return encode_map_bf16(m, base, 4, dims, strides, box, Dh >= 64);
+}
+
+gpt_status check_attn(const void* p, int B, int H, int T, int Dh, long long sb, long long sh,
+                      long long st) {
+  if (!p) return GPT_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || T <= 0) return GPT_ERR_INVALID_ARG;
+  if (Dh != 32 && Dh != 64 && Dh != 128) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(p) & 15) || (sb % 8) || (sh % 8) || (st % 8))
+    return GPT_ERR_UNSUPPORTED_SHAPE;
+  if (sb <= 0 || sh <= 0 || st <= 0) return GPT_ERR_INVALID_ARG;
+  return GPT_OK;
+}
+
+template <typename K>
+gpt_status set_smem(K kern, int bytes) {
+  GPT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  return GPT_OK;
+}
+
+template <int DH>
+gpt_status launch_fwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                      const AttnArgs& a, cudaStream_t stream) {
+  static bool once = false;
+  if (!once) { GPT_TRY(set_smem(attn_fwd_kernel<DH>, FwdShape<DH>::SMEM)); once = true; }
+  attn_fwd_kernel<DH><<<grid, 256, FwdShape<DH>::SMEM, stream>>>(mq, mk, mv, a);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
+template <int DH>
+gpt_status launch_bwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                      const CUtensorMap& mdo, AttnArgs a, void* dq, cudaStream_t stream) {
+  constexpr int smem = BwdShape<DH>::SMEM;
+  static bool once = false;
+  if (!once) {
+    GPT_TRY(set_smem(attn_bwd_dkdv_kernel<DH>, smem));
+    GPT_TRY(set_smem(attn_bwd_dq_kernel<DH>, smem));
+    once = true;
+  }
+  attn_bwd_dkdv_kernel<DH><<<grid, 128, smem, stream>>>(mq, mk, mv, mdo, a);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  a.o = reinterpret_cast<uint16_t*>(dq);
+  attn_bwd_dq_kernel<DH><<<grid, 128, smem, stream>>>(mq, mk, mv, mdo, a);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
+}  // namespace
+
+gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int T, int Dh, int window, long long sbq, long long shq,
+                         long long stq, long long sbo, long long sho, long long sto, int* status,
+                         cudaStream_t stream) {
+  GPT_TRY(check_attn(q, B, H, T, Dh, sbq, shq, stq));
+  GPT_TRY(check_attn(k, B, H, T, Dh, sbq, shq, stq));
+  GPT_TRY(check_attn(v, B, H, T, Dh, sbq, shq, stq));
+  GPT_TRY(check_attn(o, B, H, T, Dh, sbo, sho, sto));
+  if (!lse) return GPT_ERR_INVALID_ARG;
+  CUtensorMap mq, mk, mv;
+  if (!make_head_map(&mq, q, B, H, T, Dh, sbq, shq, stq, 128) ||
+      !make_head_map(&mk, k, B, H, T, Dh, sbq, shq, stq, 64) ||
+      !make_head_map(&mv, v, B, H, T, Dh, sbq, shq, stq, 64))
+    return GPT_ERR_UNSUPPORTED_SHAPE;
+  AttnArgs a{};
+  a.B = B; a.H = H; a.T = T;
+  a.window = (window > 0 && window < T) ? window : T;
+  a.scale = 1.f / sqrtf((float)Dh);
+  a.scale_log2 = a.scale * LOG2E;
+  a.o = reinterpret_cast<uint16_t*>(o);
+  a.sb_o = sbo; a.sh_o = sho; a.st_o = sto;
+  a.lse = lse;
+  a.status = status;
+  dim3 grid((T + 127) / 128, H, B);
+  if (Dh == 128) GPT_TRY(launch_fwd<128>(grid, mq, mk, mv, a, stream));
+  else if (Dh == 64) GPT_TRY(launch_fwd<64>(grid, mq, mk, mv, a, stream));
+  else GPT_TRY(launch_fwd<32>(grid, mq, mk, mv, a, stream));
+  return GPT_OK;
+}
+
+gpt_status attention_bwd(const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, float* delta, void* dq, void* dk,
+                         void* dv, int B, int H, int T, int Dh, int window, long long sbq,
+                         long long shq, long long stq, long long sbo, long long sho, long long sto,
+                         int* status, cudaStream_t stream) {
+  GPT_TRY(check_attn(q, B, H, T, Dh, sbq, shq, stq));
+  GPT_TRY(check_attn(k, B, H, T, Dh, sbq, shq, stq));
+  GPT_TRY(check_attn(v, B, H, T, Dh, sbq, shq, stq));
+  GPT_TRY(check_attn(dq, B, H, T, Dh, sbq, shq, stq));
+  GPT_TRY(check_attn(dk, B, H, T, Dh, sbq, shq, stq));
+  GPT_TRY(check_attn(dv, B, H, T, Dh, sbq, shq, stq));
+  GPT_TRY(check_attn(o, B, H, T, Dh, sbo, sho, sto));
+  GPT_TRY(check_attn(dout, B, H, T, Dh, sbo, sho, sto));
+  if (!lse || !delta) return GPT_ERR_INVALID_ARG;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_head_map(&mq, q, B, H, T, Dh, sbq, shq, stq, 64) ||
+      !make_head_map(&mk, k, B, H, T, Dh, sbq, shq, stq, 64) ||
+      !make_head_map(&mv, v, B, H, T, Dh, sbq, shq, stq, 64) ||
+      !make_head_map(&mdo, dout, B, H, T, Dh, sbo, sho, sto, 64))
+    return GPT_ERR_UNSUPPORTED_SHAPE;
+  {
+    const long long rows = (long long)B * H * T;
+    const int threads = 256;
+    const long long blocks = (rows * 32 + threads - 1) / threads;
+    attn_delta_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+        reinterpret_cast<const uint16_t*>(o), reinterpret_cast<const uint16_t*>(dout), delta, B, H,
+        T, Dh, sbo, sho, sto);
+    count_launch();
+    GPT_CUDA_TRY(cudaGetLastError());
+  }
+  AttnArgs a{};
+  a.B = B; a.H = H; a.T = T;
+  a.window = (window > 0 && window < T) ? window : T;
+  a.scale = 1.f / sqrtf((float)Dh);
+  a.scale_log2 = a.scale * LOG2E;
+  a.lse = const_cast<float*>(lse);
+  a.delta = delta;
+  a.status = status;
+  a.sb_o = sbq; a.sh_o = shq; a.st_o = stq;  // dq/dk/dv share the q/k/v strides
+  dim3 grid((T + 63) / 64, H, B);
+  a.dk = reinterpret_cast<uint16_t*>(dk);
+  a.dv = reinterpret_cast<uint16_t*>(dv);
+  if (Dh == 128) GPT_TRY(launch_bwd<128>(grid, mq, mk, mv, mdo, a, dq, stream));
+  else if (Dh == 64) GPT_TRY(launch_bwd<64>(grid, mq, mk, mv, mdo, a, dq, stream));
+  else GPT_TRY(launch_bwd<32>(grid, mq, mk, mv, mdo, a, dq, stream));
+  return GPT_OK;
+}
+
+}  // namespace gpt
+
+extern "C" gpt_status gpt_attention_fwd(const void* q, const void* k, const void* v, void* o,
+                                        float* lse, int B, int H, int T, int Dh, int window,
+                                        long long sb_qkv, long long sh_qkv, long long st_qkv,
+                                        long long sb_o, long long sh_o, long long st_o,
+                                        int* status, void* stream) {
+  return gpt::attention_fwd(q, k, v, o, lse, B, H, T, Dh, window, sb_qkv, sh_qkv, st_qkv, sb_o,
+                            sh_o, st_o, status, gpt::as_stream(stream));
+}
+
+extern "C" gpt_status gpt_attention_bwd(const void* q, const void* k, const void* v, const void* o,
+                                        const void* dout, const float* lse, float* delta, void* dq,
+                                        void* dk, void* dv, int B, int H, int T, int Dh,
+                                        int window, long long sb_qkv, long long sh_qkv,
+                                        long long st_qkv, long long sb_o, long long sh_o,
+                                        long long st_o, int* status, void* stream) {
+  return gpt::attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, T, Dh, window, sb_qkv,
+                            sh_qkv, st_qkv, sb_o, sh_o, st_o, status, gpt::as_stream(stream));
+}

@@ -1,0 +1,472 @@
+// Persistent, warp-specialised bf16 GEMM on the sm_100a tcgen05 tensor cores.
+//
+//   warp 0      TMA producer: streams 128×64 A and BN×64 B tiles (128-byte swizzle) into a ring of
+//               shared-memory stages, signalling a "full" mbarrier with the transaction bytes.
+//   warp 1      MMA issuer: one thread issues tcgen05.mma (128×BN×16 per instruction) from the
+//               stage descriptors into a tensor-memory accumulator, commits each stage back to
+//               its "empty" barrier and each finished tile to an accumulator barrier.
+//   warps 2..5  epilogue: tcgen05.ld the fp32 accumulator rows (one row per thread), apply the
+//               fused epilogue (bf16 cast, residual add, ReLU², dReLU², fp32 store, or the
+//               cross-entropy statistics / gradient of the fused lm-head) and store to global.
+// Two accumulator buffers in tensor memory let the epilogue of tile i overlap the main loop of
+// tile i+1.  Tiles are scheduled persistently over min(#tiles, #SMs) CTAs.
+//
+// Operand majors: A and B may each be K-contiguous ("K-major") or M/N-contiguous ("MN-major"),
+// which covers y = x·Wᵀ (forward), dx = dy·W (activation gradient) and dW = dyᵀ·x (weight
+// gradient) without any transposed copy.
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "host.h"
+
+namespace gpt {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int GEMM_THREADS = 192;
+
+enum : int { EPI_CE_STATS = 100, EPI_CE_GRAD = 101 };
+
+struct GemmArgs {
+  int M, N, K;
+  int tiles_m, tiles_n, k_tiles;
+  void* C;
+  int ldc;
+  void* C2;
+  const uint16_t* aux;
+  int ldaux;
+  int* status;
+  CeArgs ce;
+};
+
+template <int BN>
+struct GemmShape {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+};
+
+// ------------------------------------------------------------------------------------------------
+// epilogue: one thread owns row m, columns n0 .. n0+31 of the tile (32 fp32 values in v)
+// ------------------------------------------------------------------------------------------------
+template <int EPI>
+__device__ __forceinline__ void epilogue_store(const GemmArgs& a, int m, int n0, const float* v) {
+  const bool full = (n0 + 32 <= a.N);
+  if (EPI == GPT_EPI_F32 || EPI == GPT_EPI_F32_ADD) {
+    float* c = reinterpret_cast<float*>(a.C) + (size_t)m * a.ldc + n0;
+    if (full) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        float4 o = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        if (EPI == GPT_EPI_F32_ADD) {
+          float4 p = *reinterpret_cast<const float4*>(c + j);
+          o.x += p.x; o.y += p.y; o.z += p.z; o.w += p.w;
+        }
+        *reinterpret_cast<float4*>(c + j) = o;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (n0 + j < a.N) c[j] = (EPI == GPT_EPI_F32_ADD) ? c[j] + v[j] : v[j];
+    }
+    return;
+  }
+  uint16_t* c = reinterpret_cast<uint16_t*>(a.C) + (size_t)m * a.ldc + n0;
+  if (EPI == GPT_EPI_BF16 || EPI == GPT_EPI_RESID || EPI == GPT_EPI_DRELU2) {
+    const uint16_t* x = nullptr;
+    if (EPI == GPT_EPI_RESID) x = c;
+    if (EPI == GPT_EPI_DRELU2) x = a.aux + (size_t)m * a.ldaux + n0;
+    if (full) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) {
+        float w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = v[j + e];
+        if (EPI != GPT_EPI_BF16) {
+          uint4 p = *reinterpret_cast<const uint4*>(x + j);
+          const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float lo = bf_lo(pw[e]), hi = bf_hi(pw[e]);
+            if (EPI == GPT_EPI_RESID) { w[2 * e] += lo; w[2 * e + 1] += hi; }
+            else { w[2 * e] *= 2.f * lo; w[2 * e + 1] *= 2.f * hi; }
+          }
+        }
+        uint4 o;
+        o.x = pack_bf2(w[0], w[1]); o.y = pack_bf2(w[2], w[3]);
+        o.z = pack_bf2(w[4], w[5]); o.w = pack_bf2(w[6], w[7]);
+        *reinterpret_cast<uint4*>(c + j) = o;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (n0 + j >= a.N) continue;
+        float w = v[j];
+        if (EPI == GPT_EPI_RESID) w += bf2f(x[j]);
+        if (EPI == GPT_EPI_DRELU2) w *= 2.f * bf2f(x[j]);
+        c[j] = f2bf(w);
+      }
+    }
+    return;
+  }
+  if (EPI == GPT_EPI_RELU2) {
+    uint16_t* c2 = reinterpret_cast<uint16_t*>(a.C2) + (size_t)m * a.ldc + n0;
+    if (full) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) {
+        float r[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r[e] = fmaxf(v[j + e], 0.f);
+        uint4 o, o2;
+        o.x = pack_bf2(r[0], r[1]); o.y = pack_bf2(r[2], r[3]);
+        o.z = pack_bf2(r[4], r[5]); o.w = pack_bf2(r[6], r[7]);
+        o2.x = pack_bf2(r[0] * r[0], r[1] * r[1]); o2.y = pack_bf2(r[2] * r[2], r[3] * r[3]);
+        o2.z = pack_bf2(r[4] * r[4], r[5] * r[5]); o2.w = pack_bf2(r[6] * r[6], r[7] * r[7]);
+        *reinterpret_cast<uint4*>(c + j) = o;
+        *reinterpret_cast<uint4*>(c2 + j) = o2;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (n0 + j >= a.N) continue;
+        const float r = fmaxf(v[j], 0.f);
+        c[j] = f2bf(r);
+        c2[j] = f2bf(r * r);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// the kernel
+// ------------------------------------------------------------------------------------------------
+template <int BN, bool A_MN, bool B_MN, int EPI>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const GemmArgs args) {
+  using S = GemmShape<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::STAGES * S::STAGE_BYTES);
+  uint64_t* empty = full + S::STAGES;
+  uint64_t* tfull = empty + S::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, S::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_tiles = args.tiles_m * args.tiles_n;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        const int tm = tile / args.tiles_n, tn = tile % args.tiles_n;
+        bool ok = true;
+        for (int kt = 0; kt < args.k_tiles; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, args.status)) { ok = false; break; }
+          uint8_t* sa = smem + stage * S::STAGE_BYTES;
+          uint8_t* sb = sa + S::A_BYTES;
+          mbar_arrive_expect_tx(&full[stage], S::STAGE_BYTES);
+          const int k0 = kt * BK;
+          if (!A_MN) {
+            tma_load_2d(sa, &tmA, &full[stage], k0, tm * BM);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BM / 64; ++c)
+              tma_load_2d(sa + c * 8192, &tmA, &full[stage], tm * BM + c * 64, k0);
+          }
+          if (!B_MN) {
+            tma_load_2d(sb, &tmB, &full[stage], k0, tn * BN);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_2d(sb + c * 8192, &tmB, &full[stage], tn * BN + c * 64, k0);
+          }
+          if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(BM, BN, A_MN, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, args.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        bool ok = true;
+        for (int kt = 0; kt < args.k_tiles; ++kt) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, args.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * S::STAGE_BYTES);
+          const uint32_t sb = sa + S::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = A_MN ? sdesc_sw128(sa + kk * 2048, 8192, 1024)
+                                     : sdesc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sdesc_sw128(sb + kk * 2048, 8192, 1024)
+                                     : sdesc_sw128(sb + kk * 32, 16, 1024);
+            mma_bf16_ss(d_tmem, ad, bd, idesc, (kt | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+    }
+  } else {
+    // ---------------- epilogue warps ----------------
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int tm = tile / args.tiles_n, tn = tile % args.tiles_n;
+      const int m = tm * BM + row_in_tile;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, args.status)) break;
+      tc_fence_after();
+      float run_max = -INFINITY, run_sum = 0.f;
+      int tgt = -1;
+      float lse_m = 0.f, scale = 0.f;
+      if (EPI == EPI_CE_STATS || EPI == EPI_CE_GRAD) {
+        if (m < args.M) {
+          tgt = args.ce.targets[m] - args.ce.n_offset;
+          if (EPI == EPI_CE_GRAD) {
+            lse_m = args.ce.lse[m];
+            scale = (args.ce.targets[m] >= 0) ? *args.ce.inv_n : 0.f;
+          }
+        }
+      }
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + c * 32, r);
+        tmem_ld_wait();
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        const int n0 = tn * BN + c * 32;
+        if (EPI == EPI_CE_STATS) {
+          if (m < args.M) {
+            float cm = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n0 + j < args.N) cm = fmaxf(cm, v[j]);
+            const float nm = fmaxf(run_max, cm);
+            float s = (run_max == -INFINITY) ? 0.f : run_sum * __expf(run_max - nm);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n0 + j < args.N) s += __expf(v[j] - nm);
+            run_max = nm;
+            run_sum = s;
+            if (tgt >= n0 && tgt < n0 + 32 && tgt < args.N) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (n0 + j == tgt) args.ce.ztarget[m] = v[j];
+            }
+          }
+        } else if (EPI == EPI_CE_GRAD) {
+          if (m < args.M) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float p = __expf(v[j] - lse_m);
+              v[j] = (p - ((n0 + j == tgt) ? 1.f : 0.f)) * scale;
+            }
+            epilogue_store<GPT_EPI_BF16>(args, m, n0, v);
+          }
+        } else {
+          if (m < args.M && n0 < args.N) epilogue_store<EPI>(args, m, n0, v);
+        }
+      }
+      if (EPI == EPI_CE_STATS && m < args.M) {
+        args.ce.stats[(size_t)m * args.ce.stats_ld + args.ce.stats_col0 + tn] =
+            make_float2(run_max, run_sum);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+
+  __syncwarp();
+  // After an expired wait, give copies and MMAs already in flight time to land before the shared
+  // and tensor memory they target is released.
+  if (*abort_flag && threadIdx.x == 0) {
+    for (int i = 0; i < 2000; ++i) __nanosleep(1000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, S::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------------------
+template <int BN, bool A_MN, bool B_MN, int EPI>
+static gpt_status launch_inst(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& a,
+                              cudaStream_t stream) {
+  using S = GemmShape<BN>;
+  auto kern = gemm_kernel<BN, A_MN, B_MN, EPI>;
+  static bool attr_done = false;  // per instantiation
+  if (!attr_done) {
+    GPT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      S::SMEM_BYTES));
+    attr_done = true;
+  }
+  int sms = 0;
+  GPT_TRY(device_info(&sms));
+  const int tiles = a.tiles_m * a.tiles_n;
+  const int grid = std::min(tiles, sms);
+  kern<<<grid, GEMM_THREADS, S::SMEM_BYTES, stream>>>(ma, mb, a);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
+template <int BN, bool A_MN, bool B_MN>
+static gpt_status dispatch_epi(int epi, const CUtensorMap& ma, const CUtensorMap& mb,
+                               const GemmArgs& a, cudaStream_t s) {
+  switch (epi) {
+    case GPT_EPI_BF16: return launch_inst<BN, A_MN, B_MN, GPT_EPI_BF16>(ma, mb, a, s);
+    case GPT_EPI_RESID: return launch_inst<BN, A_MN, B_MN, GPT_EPI_RESID>(ma, mb, a, s);
+    case GPT_EPI_RELU2: return launch_inst<BN, A_MN, B_MN, GPT_EPI_RELU2>(ma, mb, a, s);
+    case GPT_EPI_DRELU2: return launch_inst<BN, A_MN, B_MN, GPT_EPI_DRELU2>(ma, mb, a, s);
+    case GPT_EPI_F32: return launch_inst<BN, A_MN, B_MN, GPT_EPI_F32>(ma, mb, a, s);
+    case GPT_EPI_F32_ADD: return launch_inst<BN, A_MN, B_MN, GPT_EPI_F32_ADD>(ma, mb, a, s);
+    default: return GPT_ERR_INVALID_ARG;
+  }
+}
+
+// A operand map: K-major [M rows, K cols] box {64, 128}; MN-major [K rows, M cols] box {64, 64}.
+static bool make_operand_map(CUtensorMap* map, const void* base, bool mn_major, int mn, int K,
+                             int ld, int box_mn) {
+  uint64_t dims[2], strides[1];
+  uint32_t box[2];
+  strides[0] = (uint64_t)ld * 2;
+  if (!mn_major) {
+    dims[0] = (uint64_t)K; dims[1] = (uint64_t)mn;
+    box[0] = 64; box[1] = (uint32_t)box_mn;
+  } else {
+    dims[0] = (uint64_t)mn; dims[1] = (uint64_t)K;
+    box[0] = 64; box[1] = 64;
+  }
+  return encode_map_bf16(map, base, 2, dims, strides, box, true);
+}
+
+static gpt_status check_gemm_args(int op, int M, int N, int K, const void* A, int lda, const void* B,
+                                  int ldb, void* C, int ldc) {
+  if (!A || !B || !C) return GPT_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return GPT_ERR_INVALID_ARG;
+  if (op < GPT_GEMM_NT || op > GPT_GEMM_TN) return GPT_ERR_INVALID_ARG;
+  const int a_inner = (op == GPT_GEMM_TN) ? M : K;
+  const int b_inner = (op == GPT_GEMM_NT) ? K : N;
+  if (lda < a_inner || ldb < b_inner || ldc < N) return GPT_ERR_INVALID_ARG;
+  if ((lda % 8) || (ldb % 8) || (ldc % 8)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) |
+       reinterpret_cast<uintptr_t>(C)) & 15)
+    return GPT_ERR_UNSUPPORTED_SHAPE;
+  return GPT_OK;
+}
+
+gpt_status gemm_launch(int op, int epi, int M, int N, int K, const void* A, int lda, const void* B,
+                       int ldb, void* C, int ldc, void* C2, const void* aux, int ldaux, int* status,
+                       cudaStream_t stream) {
+  GPT_TRY(check_gemm_args(op, M, N, K, A, lda, B, ldb, C, ldc));
+  if (epi == GPT_EPI_RELU2 && !C2) return GPT_ERR_INVALID_ARG;
+  if (epi == GPT_EPI_DRELU2 && (!aux || ldaux < N || (ldaux % 8))) return GPT_ERR_INVALID_ARG;
+  const bool a_mn = (op == GPT_GEMM_TN);
+  const bool b_mn = (op != GPT_GEMM_NT);
+  const int BN = (N > 128) ? 256 : 128;
+  CUtensorMap ma, mb;
+  if (!make_operand_map(&ma, A, a_mn, M, K, lda, BM)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if (!make_operand_map(&mb, B, b_mn, N, K, ldb, BN)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  GemmArgs a{};
+  a.M = M; a.N = N; a.K = K;
+  a.tiles_m = (M + BM - 1) / BM;
+  a.tiles_n = (N + BN - 1) / BN;
+  a.k_tiles = (K + BK - 1) / BK;
+  a.C = C; a.ldc = ldc; a.C2 = C2;
+  a.aux = reinterpret_cast<const uint16_t*>(aux); a.ldaux = ldaux;
+  a.status = status;
+  if (BN == 256) {
+    if (op == GPT_GEMM_NT) return dispatch_epi<256, false, false>(epi, ma, mb, a, stream);
+    if (op == GPT_GEMM_NN) return dispatch_epi<256, false, true>(epi, ma, mb, a, stream);
+    return dispatch_epi<256, true, true>(epi, ma, mb, a, stream);
+  } else {
+    if (op == GPT_GEMM_NT) return dispatch_epi<128, false, false>(epi, ma, mb, a, stream);
+    if (op == GPT_GEMM_NN) return dispatch_epi<128, false, true>(epi, ma, mb, a, stream);
+    return dispatch_epi<128, true, true>(epi, ma, mb, a, stream);
+  }
+}
+
+int gemm_ce_tile_n() { return 256; }
+
+gpt_status gemm_ce_launch(bool grad, int M, int N, int K, const void* A, int lda, const void* B,
+                          int ldb, void* C, int ldc, const CeArgs& ce, int* status,
+                          cudaStream_t stream) {
+  GPT_TRY(check_gemm_args(GPT_GEMM_NT, M, N, K, A, lda, B, ldb, grad ? C : (void*)A, grad ? ldc : N));
+  CUtensorMap ma, mb;
+  if (!make_operand_map(&ma, A, false, M, K, lda, BM)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if (!make_operand_map(&mb, B, false, N, K, ldb, 256)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  GemmArgs a{};
+  a.M = M; a.N = N; a.K = K;
+  a.tiles_m = (M + BM - 1) / BM;
+  a.tiles_n = (N + 255) / 256;
+  a.k_tiles = (K + BK - 1) / BK;
+  a.C = C; a.ldc = ldc;
+  a.status = status;
+  a.ce = ce;
+  if (grad) return launch_inst<256, false, false, EPI_CE_GRAD>(ma, mb, a, stream);
+  return launch_inst<256, false, false, EPI_CE_STATS>(ma, mb, a, stream);
+}
+
+}  // namespace gpt
+
+extern "C" gpt_status gpt_gemm(int op, int epilogue, int M, int N, int K, const void* A, int lda,
+                               const void* B, int ldb, void* C, int ldc, void* C2,
+                               const void* aux, int ldaux, int* status, void* stream) {
+  return gpt::gemm_launch(op, epilogue, M, N, K, A, lda, B, ldb, C, ldc, C2, aux, ldaux, status,
+                          gpt::as_stream(stream));
+}

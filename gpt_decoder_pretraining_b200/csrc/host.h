@@ -1,0 +1,62 @@
+// Host-side helpers shared by the .cu files: CUDA error mapping, device properties, TMA tensor-map
+// encoding (through the runtime's driver entry point, so the library does not link libcuda).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gptstep.h"
+
+namespace gpt {
+
+#define GPT_CUDA_TRY(expr)                           \
+  do {                                               \
+    cudaError_t e_ = (expr);                         \
+    if (e_ != cudaSuccess) return GPT_ERR_CUDA;      \
+  } while (0)
+
+#define GPT_TRY(expr)                                \
+  do {                                               \
+    gpt_status s_ = (expr);                          \
+    if (s_ != GPT_OK) return s_;                     \
+  } while (0)
+
+// Multiprocessor count and sm_100 check of the current device (cached per device).
+gpt_status device_info(int* num_sms);
+
+// Encode a tiled TMA map over a bf16 tensor of `rank` dims (dims[0] contiguous).  strides_bytes
+// has rank-1 entries (byte stride of dims 1..rank-1).  128-byte swizzle when swizzle128 is set.
+// Returns false if the driver rejects the map (alignment, box size).
+bool encode_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128);
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Kernel-launch counter for reporting how many of this library's kernels a step enqueued.
+extern thread_local int64_t g_launch_count;
+inline void count_launch(int n = 1) { g_launch_count += n; }
+
+// Kernel-level launchers used by the step orchestrator (same semantics as the C entry points).
+gpt_status gemm_launch(int op, int epi, int M, int N, int K, const void* A, int lda, const void* B,
+                       int ldb, void* C, int ldc, void* C2, const void* aux, int ldaux, int* status,
+                       cudaStream_t stream);
+
+struct CeArgs {
+  const int32_t* targets;
+  int n_offset;         // vocabulary index of column 0 of this launch
+  const float* lse;     // [M]
+  const float* inv_n;   // device scalar: 1 / n_valid (0 if none)
+  float2* stats;        // [M, stats_ld] (max, sum exp) per vocabulary tile
+  int stats_ld;
+  int stats_col0;       // tile index of column 0 of this launch
+  float* ztarget;       // [M] logit of the target
+};
+// z = A·Bᵀ (A = x_f [M,K], B = W_lm rows [N,K]); CE statistics (stats/ztarget) or CE gradient
+// dz = (softmax − onehot)·inv_n stored bf16 into C [M, ldc].
+gpt_status gemm_ce_launch(bool grad, int M, int N, int K, const void* A, int lda, const void* B,
+                          int ldb, void* C, int ldc, const CeArgs& ce, int* status,
+                          cudaStream_t stream);
+int gemm_ce_tile_n();  // vocabulary columns per CE statistics tile
+
+}  // namespace gpt

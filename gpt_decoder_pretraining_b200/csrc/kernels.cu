@@ -1,0 +1,587 @@
+// Memory-bound kernels of the training step: RMSNorm, RoPE + QK-norm, embedding gather and
+// deterministic scatter, cross-entropy reductions, parameter cast.  Each is one pass over its
+// operands with 16-byte vector accesses and one warp per row.
+//
+// RMSNorm has no gain ("Introducing nanochat", Pretraining: no RMSNorm parameters):
+//   y = x·rho, rho = 1/sqrt(mean(x²) + 1e-6);  backward dx = rho·(dy − y·mean(y·dy)).
+// RoPE ("nanochat User Guide" §10: rotary positional embeddings) rotates the pairs (i, i+Dh/2) by
+// t·10000^(−2i/Dh); QK-norm (same section) is the parameter-free RMSNorm over each head.
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "host.h"
+
+namespace gpt {
+
+constexpr float NORM_EPS = 1e-6f;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) v += __shfl_xor_sync(0xffffffffu, v, s);
+  return v;
+}
+
+// ------------------------------------------------------------------------------------------------
+// RMSNorm
+// ------------------------------------------------------------------------------------------------
+__global__ void rmsnorm_fwd_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ y,
+                                   float* __restrict__ rho, int rows, int d) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * d);
+  uint4* yr = reinterpret_cast<uint4*>(y + (size_t)row * d);
+  const int nv = d >> 3;
+  float ss = 0.f;
+  for (int i = lane; i < nv; i += 32) {
+    const uint4 v = xr[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) ss += bf_lo(w[e]) * bf_lo(w[e]) + bf_hi(w[e]) * bf_hi(w[e]);
+  }
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / (float)d + NORM_EPS);
+  for (int i = lane; i < nv; i += 32) {
+    const uint4 v = xr[i];
+    uint4 o;
+    o.x = pack_bf2(bf_lo(v.x) * r, bf_hi(v.x) * r);
+    o.y = pack_bf2(bf_lo(v.y) * r, bf_hi(v.y) * r);
+    o.z = pack_bf2(bf_lo(v.z) * r, bf_hi(v.z) * r);
+    o.w = pack_bf2(bf_lo(v.w) * r, bf_hi(v.w) * r);
+    yr[i] = o;
+  }
+  if (lane == 0) rho[row] = r;
+}
+
+template <bool DY_F32>
+__device__ __forceinline__ void load8(const void* p, size_t idx, float (&v)[8]) {
+  if (DY_F32) {
+    const float4* f = reinterpret_cast<const float4*>(p) + idx * 2;
+    const float4 a = f[0], b = f[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    const uint4 u = reinterpret_cast<const uint4*>(p)[idx];
+    v[0] = bf_lo(u.x); v[1] = bf_hi(u.x); v[2] = bf_lo(u.y); v[3] = bf_hi(u.y);
+    v[4] = bf_lo(u.z); v[5] = bf_hi(u.z); v[6] = bf_lo(u.w); v[7] = bf_hi(u.w);
+  }
+}
+
+template <bool DY_F32>
+__global__ void rmsnorm_bwd_kernel(const void* __restrict__ dy, const uint16_t* __restrict__ y,
+                                   const float* __restrict__ rho, float* __restrict__ gx,
+                                   uint16_t* __restrict__ gx_bf16, int accumulate, int rows, int d) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int nv = d >> 3;
+  const size_t base = (size_t)row * nv;
+  float dot = 0.f;
+  for (int i = lane; i < nv; i += 32) {
+    float a[8], b[8];
+    load8<DY_F32>(dy, base + i, a);
+    load8<false>(y, base + i, b);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dot += a[e] * b[e];
+  }
+  dot = warp_sum(dot) / (float)d;
+  const float r = rho[row];
+  for (int i = lane; i < nv; i += 32) {
+    float a[8], b[8];
+    load8<DY_F32>(dy, base + i, a);
+    load8<false>(y, base + i, b);
+    float4* g = reinterpret_cast<float4*>(gx) + (base + i) * 2;
+    float o[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = r * (a[e] - b[e] * dot);
+    if (accumulate) {
+      const float4 p0 = g[0], p1 = g[1];
+      o[0] += p0.x; o[1] += p0.y; o[2] += p0.z; o[3] += p0.w;
+      o[4] += p1.x; o[5] += p1.y; o[6] += p1.z; o[7] += p1.w;
+    }
+    g[0] = make_float4(o[0], o[1], o[2], o[3]);
+    g[1] = make_float4(o[4], o[5], o[6], o[7]);
+    if (gx_bf16) {
+      uint4 u;
+      u.x = pack_bf2(o[0], o[1]); u.y = pack_bf2(o[2], o[3]);
+      u.z = pack_bf2(o[4], o[5]); u.w = pack_bf2(o[6], o[7]);
+      reinterpret_cast<uint4*>(gx_bf16)[base + i] = u;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// RoPE + QK-norm
+// ------------------------------------------------------------------------------------------------
+__global__ void rope_table_kernel(float* __restrict__ cs, int T, int half, int Dh) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= T * half) return;
+  const int t = idx / half, i = idx % half;
+  const double inv_freq = pow(10000.0, -2.0 * (double)i / (double)Dh);
+  const double phi = (double)t * inv_freq;
+  cs[2 * idx] = (float)cos(phi);
+  cs[2 * idx + 1] = (float)sin(phi);
+}
+
+// One warp per (token m, part ∈ {q, k}, head h); lane handles pair indices i = 2·lane + {0,1}
+// (+64 per further round) of the first half and their partners i + Dh/2.
+__global__ void rope_qknorm_fwd_kernel(uint16_t* __restrict__ qkv, float* __restrict__ rho_q,
+                                       float* __restrict__ rho_k, const float* __restrict__ cs,
+                                       int M, int T, int H, int Dh) {
+  const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= (long long)M * 2 * H) return;
+  const int h = (int)(w % H), part = (int)((w / H) % 2);
+  const long long m = w / (2 * H);
+  const int t = (int)(m % T), half = Dh >> 1, d = H * Dh;
+  uint16_t* p = qkv + m * 3 * d + part * d + h * Dh;
+  float a[2][2], b[2][2];
+  float ss = 0.f;
+  const int rounds = (half + 63) >> 6;
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    const int i = 2 * lane + 64 * rr;
+    if (rr < rounds && i < half) {
+      const uint32_t ua = *reinterpret_cast<const uint32_t*>(p + i);
+      const uint32_t ub = *reinterpret_cast<const uint32_t*>(p + i + half);
+      const float a0 = bf_lo(ua), a1 = bf_hi(ua), b0 = bf_lo(ub), b1 = bf_hi(ub);
+      const float2 c0 = *reinterpret_cast<const float2*>(cs + 2 * ((size_t)t * half + i));
+      const float2 c1 = *reinterpret_cast<const float2*>(cs + 2 * ((size_t)t * half + i + 1));
+      a[rr][0] = a0 * c0.x - b0 * c0.y;
+      b[rr][0] = a0 * c0.y + b0 * c0.x;
+      a[rr][1] = a1 * c1.x - b1 * c1.y;
+      b[rr][1] = a1 * c1.y + b1 * c1.x;
+      ss += a[rr][0] * a[rr][0] + a[rr][1] * a[rr][1] + b[rr][0] * b[rr][0] + b[rr][1] * b[rr][1];
+    }
+  }
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / (float)Dh + NORM_EPS);
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    const int i = 2 * lane + 64 * rr;
+    if (rr < rounds && i < half) {
+      *reinterpret_cast<uint32_t*>(p + i) = pack_bf2(a[rr][0] * r, a[rr][1] * r);
+      *reinterpret_cast<uint32_t*>(p + i + half) = pack_bf2(b[rr][0] * r, b[rr][1] * r);
+    }
+  }
+  if (lane == 0) (part == 0 ? rho_q : rho_k)[m * H + h] = r;
+}
+
+// Backward: g = rho·(dŷ − ŷ·mean(ŷ·dŷ)) with ŷ the stored forward output, then the inverse
+// rotation (a, b) → (a cos + b sin, −a sin + b cos).
+__global__ void rope_qknorm_bwd_kernel(uint16_t* __restrict__ dqkv, const uint16_t* __restrict__ qkv,
+                                       const float* __restrict__ rho_q, const float* __restrict__ rho_k,
+                                       const float* __restrict__ cs, int M, int T, int H, int Dh) {
+  const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= (long long)M * 2 * H) return;
+  const int h = (int)(w % H), part = (int)((w / H) % 2);
+  const long long m = w / (2 * H);
+  const int t = (int)(m % T), half = Dh >> 1, d = H * Dh;
+  const long long off = m * 3 * d + part * d + h * Dh;
+  uint16_t* g = dqkv + off;
+  const uint16_t* y = qkv + off;
+  const float r = (part == 0 ? rho_q : rho_k)[m * H + h];
+  float ga[2][2], gb[2][2], ya[2][2], yb[2][2];
+  float dot = 0.f;
+  const int rounds = (half + 63) >> 6;
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    const int i = 2 * lane + 64 * rr;
+    if (rr < rounds && i < half) {
+      const uint32_t u0 = *reinterpret_cast<const uint32_t*>(g + i);
+      const uint32_t u1 = *reinterpret_cast<const uint32_t*>(g + i + half);
+      const uint32_t v0 = *reinterpret_cast<const uint32_t*>(y + i);
+      const uint32_t v1 = *reinterpret_cast<const uint32_t*>(y + i + half);
+      ga[rr][0] = bf_lo(u0); ga[rr][1] = bf_hi(u0); gb[rr][0] = bf_lo(u1); gb[rr][1] = bf_hi(u1);
+      ya[rr][0] = bf_lo(v0); ya[rr][1] = bf_hi(v0); yb[rr][0] = bf_lo(v1); yb[rr][1] = bf_hi(v1);
+      dot += ga[rr][0] * ya[rr][0] + ga[rr][1] * ya[rr][1] + gb[rr][0] * yb[rr][0] + gb[rr][1] * yb[rr][1];
+    }
+  }
+  dot = warp_sum(dot) / (float)Dh;
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    const int i = 2 * lane + 64 * rr;
+    if (rr < rounds && i < half) {
+      float oa[2], ob[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float na = r * (ga[rr][e] - ya[rr][e] * dot);
+        const float nb = r * (gb[rr][e] - yb[rr][e] * dot);
+        const float2 c = *reinterpret_cast<const float2*>(cs + 2 * ((size_t)t * half + i + e));
+        oa[e] = na * c.x + nb * c.y;
+        ob[e] = -na * c.y + nb * c.x;
+      }
+      *reinterpret_cast<uint32_t*>(g + i) = pack_bf2(oa[0], oa[1]);
+      *reinterpret_cast<uint32_t*>(g + i + half) = pack_bf2(ob[0], ob[1]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// embedding
+// ------------------------------------------------------------------------------------------------
+__global__ void embedding_fwd_kernel(const int32_t* __restrict__ tok, const uint16_t* __restrict__ wte,
+                                     uint16_t* __restrict__ x, int M, int d, int V, int* status) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= M) return;
+  int id = tok[row];
+  if (id < 0 || id >= V) {
+    if (lane == 0) set_status(status, GPT_ERR_TOKEN_OUT_OF_RANGE);
+    id = min(max(id, 0), V - 1);
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(wte + (size_t)id * d);
+  uint4* dst = reinterpret_cast<uint4*>(x + (size_t)row * d);
+  for (int i = lane; i < (d >> 3); i += 32) dst[i] = src[i];
+}
+
+// Single-CTA bitonic sort of the keys (id << 16 | local index) of one segment of ≤ 32768 tokens,
+// then the run heads (first position of every distinct id) are compacted in ascending order.
+// Outputs: sorted keys [n], run starts [nruns + 1] (last = n), *nruns.
+constexpr int EMB_SEG = 32768;
+__global__ void __launch_bounds__(1024) embedding_sort_kernel(const int32_t* __restrict__ tok, int n,
+                                                              int V, uint32_t* __restrict__ keys_out,
+                                                              int* __restrict__ run_start,
+                                                              int* __restrict__ nruns) {
+  extern __shared__ uint32_t sk[];  // [P] keys, then [P/1024 + 1] scan scratch
+  int P = 1;
+  while (P < n) P <<= 1;
+  for (int i = threadIdx.x; i < P; i += blockDim.x) {
+    if (i < n) {
+      int id = tok[i];
+      id = min(max(id, 0), V - 1);
+      sk[i] = ((uint32_t)id << 16) | (uint32_t)i;
+    } else {
+      sk[i] = 0xFFFFFFFFu;
+    }
+  }
+  __syncthreads();
+  for (int k = 2; k <= P; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < P; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const uint32_t a = sk[i], b = sk[ixj];
+          const bool up = ((i & k) == 0);
+          if ((a > b) == up) { sk[i] = b; sk[ixj] = a; }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < n; i += blockDim.x) keys_out[i] = sk[i];
+  __syncthreads();
+  // run heads: a stable compaction with a block-wide scan over chunks of blockDim.x
+  __shared__ int warp_tot[32];
+  __shared__ int base_s;
+  if (threadIdx.x == 0) base_s = 0;
+  __syncthreads();
+  for (int c0 = 0; c0 < n; c0 += blockDim.x) {
+    const int i = c0 + threadIdx.x;
+    const int head = (i < n) && (i == 0 || (sk[i] >> 16) != (sk[i - 1] >> 16));
+    const unsigned mask = __ballot_sync(0xffffffffu, head);
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int before = __popc(mask & ((1u << lane) - 1));
+    if (lane == 0) warp_tot[wid] = __popc(mask);
+    __syncthreads();
+    int off = 0;
+    for (int w = 0; w < wid; ++w) off += warp_tot[w];
+    if (head) run_start[base_s + off + before] = i;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int tot = 0;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += warp_tot[w];
+      base_s += tot;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    run_start[base_s] = n;
+    *nruns = base_s;
+  }
+}
+
+// One CTA per run: dwte[id] += Σ over the run (ascending token index) of gx rows.  The column
+// range is split over the threads (4 floats each); rows are summed 4 at a time in a fixed order.
+__global__ void embedding_accum_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ run_start,
+                                       const int* __restrict__ nruns, const float* __restrict__ gx,
+                                       float* __restrict__ dwte, int seg0, int d) {
+  const int r = blockIdx.x;
+  if (r >= *nruns) return;
+  const int s = run_start[r], e = run_start[r + 1];
+  const int id = (int)(keys[s] >> 16);
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int i = s;
+    for (; i + 4 <= e; i += 4) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int m = seg0 + (int)(keys[i + u] & 0xFFFFu);
+        v[u] = *reinterpret_cast<const float4*>(gx + (size_t)m * d + c);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
+      }
+    }
+    for (; i < e; ++i) {
+      const int m = seg0 + (int)(keys[i] & 0xFFFFu);
+      const float4 v = *reinterpret_cast<const float4*>(gx + (size_t)m * d + c);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    float4* dst = reinterpret_cast<float4*>(dwte + (size_t)id * d + c);
+    float4 o = *dst;
+    o.x += acc.x; o.y += acc.y; o.z += acc.z; o.w += acc.w;
+    *dst = o;
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// cross-entropy reductions
+// ------------------------------------------------------------------------------------------------
+// Per row: lse = logsumexp over the vocabulary tiles' (max, Σexp) pairs; ℓ = lse − z[target]
+// (0 for ignored rows).  One warp per row.
+__global__ void ce_rows_kernel(const float2* __restrict__ stats, int ntiles, const float* __restrict__ zt,
+                               const int32_t* __restrict__ targets, int M, int V, float* __restrict__ lse,
+                               float* __restrict__ ell, int* status) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const float2* s = stats + (size_t)row * ntiles;
+  float mx = -INFINITY;
+  for (int i = lane; i < ntiles; i += 32) mx = fmaxf(mx, s[i].x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float sum = 0.f;
+  for (int i = lane; i < ntiles; i += 32) sum += s[i].y * __expf(s[i].x - mx);
+  sum = warp_sum(sum);
+  if (lane == 0) {
+    const float l = mx + logf(sum);
+    lse[row] = l;
+    const int t = targets[row];
+    if (t < -1 || t >= V) set_status(status, GPT_ERR_TOKEN_OUT_OF_RANGE);
+    ell[row] = (t >= 0 && t < V) ? (l - zt[row]) : 0.f;
+  }
+}
+
+// Single CTA: loss = Σ ℓ / n_valid in a fixed order (0 when n_valid = 0); inv_n = 1/n_valid.
+__global__ void __launch_bounds__(1024) ce_finalize_kernel(const float* __restrict__ ell,
+                                                           const int32_t* __restrict__ targets, int M,
+                                                           int V, float* __restrict__ loss,
+                                                           float* __restrict__ inv_n) {
+  __shared__ double ssum[1024];
+  __shared__ int scnt[1024];
+  double acc = 0.0;
+  int cnt = 0;
+  for (int i = threadIdx.x; i < M; i += blockDim.x) {
+    const int t = targets[i];
+    if (t >= 0 && t < V) { acc += (double)ell[i]; ++cnt; }
+  }
+  ssum[threadIdx.x] = acc;
+  scnt[threadIdx.x] = cnt;
+  __syncthreads();
+  for (int s = blockDim.x >> 1; s > 0; s >>= 1) {
+    if ((int)threadIdx.x < s) {
+      ssum[threadIdx.x] += ssum[threadIdx.x + s];
+      scnt[threadIdx.x] += scnt[threadIdx.x + s];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const int n = scnt[0];
+    *loss = n ? (float)(ssum[0] / (double)n) : 0.f;
+    *inv_n = n ? 1.f / (float)n : 0.f;
+  }
+}
+
+__global__ void cast_f32_bf16_kernel(const float* __restrict__ src, uint16_t* __restrict__ dst, size_t n) {
+  const size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (i + 4 <= n) {
+    const float4 v = *reinterpret_cast<const float4*>(src + i);
+    uint2 o;
+    o.x = pack_bf2(v.x, v.y);
+    o.y = pack_bf2(v.z, v.w);
+    *reinterpret_cast<uint2*>(dst + i) = o;
+  } else {
+    for (size_t j = i; j < n; ++j) dst[j] = f2bf(src[j]);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// launchers
+// ------------------------------------------------------------------------------------------------
+static inline unsigned blocks_for_warps(long long warps, int threads) {
+  return (unsigned)((warps * 32 + threads - 1) / threads);
+}
+
+gpt_status rmsnorm_fwd(const void* x, void* y, float* rho, int rows, int d, cudaStream_t s) {
+  if (!x || !y || !rho || rows <= 0 || d <= 0) return GPT_ERR_INVALID_ARG;
+  if (d % 8) return GPT_ERR_UNSUPPORTED_SHAPE;
+  rmsnorm_fwd_kernel<<<blocks_for_warps(rows, 256), 256, 0, s>>>(
+      reinterpret_cast<const uint16_t*>(x), reinterpret_cast<uint16_t*>(y), rho, rows, d);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
+gpt_status rmsnorm_bwd(const void* dy, int dy_f32, const void* y, const float* rho, float* gx,
+                       void* gx_bf16, int accumulate, int rows, int d, cudaStream_t s) {
+  if (!dy || !y || !rho || !gx || rows <= 0 || d <= 0) return GPT_ERR_INVALID_ARG;
+  if (d % 8) return GPT_ERR_UNSUPPORTED_SHAPE;
+  const unsigned nb = blocks_for_warps(rows, 256);
+  if (dy_f32)
+    rmsnorm_bwd_kernel<true><<<nb, 256, 0, s>>>(dy, reinterpret_cast<const uint16_t*>(y), rho, gx,
+                                                reinterpret_cast<uint16_t*>(gx_bf16), accumulate, rows, d);
+  else
+    rmsnorm_bwd_kernel<false><<<nb, 256, 0, s>>>(dy, reinterpret_cast<const uint16_t*>(y), rho, gx,
+                                                 reinterpret_cast<uint16_t*>(gx_bf16), accumulate, rows, d);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
+gpt_status rope_table(float* cs, int T, int Dh, cudaStream_t s) {
+  if (!cs || T <= 0 || Dh <= 0 || (Dh % 4)) return GPT_ERR_INVALID_ARG;
+  const int n = T * (Dh / 2);
+  rope_table_kernel<<<(n + 255) / 256, 256, 0, s>>>(cs, T, Dh / 2, Dh);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
+static gpt_status check_rope(int B, int T, int H, int Dh) {
+  if (B <= 0 || T <= 0 || H <= 0) return GPT_ERR_INVALID_ARG;
+  if (Dh != 32 && Dh != 64 && Dh != 128 && Dh != 256) return GPT_ERR_UNSUPPORTED_SHAPE;
+  return GPT_OK;
+}
+
+gpt_status rope_qknorm_fwd(void* qkv, float* rq, float* rk, const float* cs, int B, int T, int H,
+                           int Dh, cudaStream_t s) {
+  if (!qkv || !rq || !rk || !cs) return GPT_ERR_INVALID_ARG;
+  GPT_TRY(check_rope(B, T, H, Dh));
+  const long long warps = (long long)B * T * 2 * H;
+  rope_qknorm_fwd_kernel<<<blocks_for_warps(warps, 256), 256, 0, s>>>(
+      reinterpret_cast<uint16_t*>(qkv), rq, rk, cs, B * T, T, H, Dh);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
+gpt_status rope_qknorm_bwd(void* dqkv, const void* qkv, const float* rq, const float* rk,
+                           const float* cs, int B, int T, int H, int Dh, cudaStream_t s) {
+  if (!dqkv || !qkv || !rq || !rk || !cs) return GPT_ERR_INVALID_ARG;
+  GPT_TRY(check_rope(B, T, H, Dh));
+  const long long warps = (long long)B * T * 2 * H;
+  rope_qknorm_bwd_kernel<<<blocks_for_warps(warps, 256), 256, 0, s>>>(
+      reinterpret_cast<uint16_t*>(dqkv), reinterpret_cast<const uint16_t*>(qkv), rq, rk, cs, B * T,
+      T, H, Dh);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
+gpt_status embedding_fwd(const int32_t* tok, const void* wte, void* x, int M, int d, int V,
+                         int* status, cudaStream_t s) {
+  if (!tok || !wte || !x || M <= 0 || d <= 0 || V <= 0) return GPT_ERR_INVALID_ARG;
+  if (d % 8) return GPT_ERR_UNSUPPORTED_SHAPE;
+  embedding_fwd_kernel<<<blocks_for_warps(M, 256), 256, 0, s>>>(
+      tok, reinterpret_cast<const uint16_t*>(wte), reinterpret_cast<uint16_t*>(x), M, d, V, status);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
+size_t embedding_bwd_scratch_bytes(int M, int V) {
+  (void)V;
+  const int seg = std::min(M, EMB_SEG);
+  // keys [seg] + run starts [seg + 1] + nruns, 256-byte aligned pieces
+  auto al = [](size_t b) { return (b + 255) & ~(size_t)255; };
+  return al((size_t)seg * 4) + al((size_t)(seg + 1) * 4) + al(4);
+}
+
+gpt_status embedding_bwd(const int32_t* tok, const float* gx, float* dwte, int M, int d, int V,
+                         void* scratch, cudaStream_t s) {
+  if (!tok || !gx || !dwte || !scratch || M <= 0 || d <= 0 || V <= 0) return GPT_ERR_INVALID_ARG;
+  if ((d % 4) || V > 65536) return GPT_ERR_UNSUPPORTED_SHAPE;
+  auto al = [](size_t b) { return (b + 255) & ~(size_t)255; };
+  const int seg = std::min(M, EMB_SEG);
+  uint8_t* p = reinterpret_cast<uint8_t*>(scratch);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(p);
+  int* run_start = reinterpret_cast<int*>(p + al((size_t)seg * 4));
+  int* nruns = reinterpret_cast<int*>(p + al((size_t)seg * 4) + al((size_t)(seg + 1) * 4));
+  GPT_CUDA_TRY(cudaMemsetAsync(dwte, 0, (size_t)V * d * sizeof(float), s));
+  static bool attr = false;
+  if (!attr) {
+    GPT_CUDA_TRY(cudaFuncSetAttribute(embedding_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      EMB_SEG * 4));
+    attr = true;
+  }
+  for (int s0 = 0; s0 < M; s0 += EMB_SEG) {
+    const int n = std::min(EMB_SEG, M - s0);
+    int P = 1;
+    while (P < n) P <<= 1;
+    embedding_sort_kernel<<<1, 1024, (size_t)P * 4, s>>>(tok + s0, n, V, keys, run_start, nruns);
+    count_launch();
+    GPT_CUDA_TRY(cudaGetLastError());
+    const int threads = std::min(256, std::max(32, ((d / 4) + 31) / 32 * 32));
+    embedding_accum_kernel<<<n, threads, 0, s>>>(keys, run_start, nruns, gx, dwte, s0, d);
+    count_launch();
+    GPT_CUDA_TRY(cudaGetLastError());
+  }
+  return GPT_OK;
+}
+
+gpt_status ce_rows(const float2* stats, int ntiles, const float* zt, const int32_t* targets, int M,
+                   int V, float* lse, float* ell, int* status, cudaStream_t s) {
+  ce_rows_kernel<<<blocks_for_warps(M, 256), 256, 0, s>>>(stats, ntiles, zt, targets, M, V, lse, ell, status);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
+gpt_status ce_finalize(const float* ell, const int32_t* targets, int M, int V, float* loss,
+                       float* inv_n, cudaStream_t s) {
+  ce_finalize_kernel<<<1, 1024, 0, s>>>(ell, targets, M, V, loss, inv_n);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
+gpt_status cast_f32_bf16(const float* src, void* dst, size_t n, cudaStream_t s) {
+  const size_t threads = 256, per = 4;
+  const size_t blocks = (n + threads * per - 1) / (threads * per);
+  cast_f32_bf16_kernel<<<(unsigned)blocks, (unsigned)threads, 0, s>>>(src, reinterpret_cast<uint16_t*>(dst), n);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
+}  // namespace gpt
+
+extern "C" {
+gpt_status gpt_rmsnorm_fwd(const void* x, void* y, float* rho, int rows, int d, void* stream) {
+  return gpt::rmsnorm_fwd(x, y, rho, rows, d, gpt::as_stream(stream));
+}
+gpt_status gpt_rmsnorm_bwd(const void* dy, int dy_f32, const void* y, const float* rho, float* gx,
+                           void* gx_bf16, int accumulate, int rows, int d, void* stream) {
+  return gpt::rmsnorm_bwd(dy, dy_f32, y, rho, gx, gx_bf16, accumulate, rows, d, gpt::as_stream(stream));
+}
+gpt_status gpt_rope_table(float* cos_sin, int T, int Dh, void* stream) {
+  return gpt::rope_table(cos_sin, T, Dh, gpt::as_stream(stream));
+}
+gpt_status gpt_rope_qknorm_fwd(void* qkv, float* rho_q, float* rho_k, const float* cos_sin, int B,
+                               int T, int H, int Dh, void* stream) {
+  return gpt::rope_qknorm_fwd(qkv, rho_q, rho_k, cos_sin, B, T, H, Dh, gpt::as_stream(stream));
+}
+gpt_status gpt_rope_qknorm_bwd(void* dqkv, const void* qkv, const float* rho_q, const float* rho_k,
+                               const float* cos_sin, int B, int T, int H, int Dh, void* stream) {
+  return gpt::rope_qknorm_bwd(dqkv, qkv, rho_q, rho_k, cos_sin, B, T, H, Dh, gpt::as_stream(stream));
+}
+gpt_status gpt_embedding_fwd(const int32_t* tokens, const void* wte, void* x, int M, int d, int V,
+                             int* status, void* stream) {
+  return gpt::embedding_fwd(tokens, wte, x, M, d, V, status, gpt::as_stream(stream));
+}
+size_t gpt_embedding_bwd_scratch_bytes(int M, int V) { return gpt::embedding_bwd_scratch_bytes(M, V); }
+gpt_status gpt_embedding_bwd(const int32_t* tokens, const float* gx, float* dwte, int M, int d,
+                             int V, void* scratch, void* stream) {
+  return gpt::embedding_bwd(tokens, gx, dwte, M, d, V, scratch, gpt::as_stream(stream));
+}
+}

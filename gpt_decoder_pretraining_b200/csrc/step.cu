@@ -1,0 +1,434 @@
+// The training-step orchestrator behind the C ABI: parameter packing, workspace plan, and the
+// launch sequence of one forward + backward pass of the nanochat GPT decoder.
+//
+// Forward, per layer ("nanochat User Guide" §10; "Introducing nanochat", Pretraining):
+//   r1 = RMS(x) → qkv = r1·W_qkvᵀ → RoPE + QK-norm (in place) → o = attention(q̃, k̃, v)
+//   → x += o·W_oᵀ (residual epilogue) → r2 = RMS(x) → a = relu(r2·W_fcᵀ), h = a² (epilogue)
+//   → x += h·W_projᵀ (residual epilogue)
+// then x_f = RMS(x) and the fused lm-head + cross-entropy ("supa beginna nanochat",
+// Troubleshooting: mean over targets ≠ −1).  The backward pass runs the same chain in reverse with
+// an fp32 residual gradient and its bf16 copy as the GEMM operand; every weight gradient is an
+// fp32 GEMM output written straight into the caller's gradient buffer.
+
+#include <algorithm>
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+#include "host.h"
+
+namespace gpt {
+
+gpt_status rmsnorm_fwd(const void* x, void* y, float* rho, int rows, int d, cudaStream_t s);
+gpt_status rmsnorm_bwd(const void* dy, int dy_f32, const void* y, const float* rho, float* gx,
+                       void* gx_bf16, int accumulate, int rows, int d, cudaStream_t s);
+gpt_status rope_table(float* cs, int T, int Dh, cudaStream_t s);
+gpt_status rope_qknorm_fwd(void* qkv, float* rq, float* rk, const float* cs, int B, int T, int H,
+                           int Dh, cudaStream_t s);
+gpt_status rope_qknorm_bwd(void* dqkv, const void* qkv, const float* rq, const float* rk,
+                           const float* cs, int B, int T, int H, int Dh, cudaStream_t s);
+gpt_status embedding_fwd(const int32_t* tok, const void* wte, void* x, int M, int d, int V,
+                         int* status, cudaStream_t s);
+size_t embedding_bwd_scratch_bytes(int M, int V);
+gpt_status embedding_bwd(const int32_t* tok, const float* gx, float* dwte, int M, int d, int V,
+                         void* scratch, cudaStream_t s);
+gpt_status ce_rows(const float2* stats, int ntiles, const float* zt, const int32_t* targets, int M,
+                   int V, float* lse, float* ell, int* status, cudaStream_t s);
+gpt_status ce_finalize(const float* ell, const int32_t* targets, int M, int V, float* loss,
+                       float* inv_n, cudaStream_t s);
+gpt_status cast_f32_bf16(const float* src, void* dst, size_t n, cudaStream_t s);
+gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int T, int Dh, int window, long long sbq, long long shq,
+                         long long stq, long long sbo, long long sho, long long sto, int* status,
+                         cudaStream_t stream);
+gpt_status attention_bwd(const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, float* delta, void* dq, void* dk,
+                         void* dv, int B, int H, int T, int Dh, int window, long long sbq,
+                         long long shq, long long stq, long long sbo, long long sho, long long sto,
+                         int* status, cudaStream_t stream);
+
+static inline size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// ------------------------------------------------------------------------------------------------
+// configuration and packing
+// ------------------------------------------------------------------------------------------------
+static gpt_status validate(const gpt_config* c) {
+  if (!c) return GPT_ERR_INVALID_ARG;
+  if (c->depth < 0 || c->d_model <= 0 || c->n_heads <= 0 || c->head_dim <= 0 || c->d_mlp <= 0 ||
+      c->vocab <= 0 || c->seq_len <= 0 || c->batch <= 0)
+    return GPT_ERR_INVALID_ARG;
+  if (c->param_dtype != GPT_DTYPE_BF16 && c->param_dtype != GPT_DTYPE_F32) return GPT_ERR_INVALID_ARG;
+  if (c->n_heads * c->head_dim != c->d_model) return GPT_ERR_INVALID_ARG;
+  if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if ((c->d_model % 64) || (c->d_mlp % 64) || (c->vocab % 64)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if (c->vocab > 65536) return GPT_ERR_UNSUPPORTED_SHAPE;
+  const long long M = (long long)c->batch * c->seq_len;
+  if (M > (1ll << 30)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  return GPT_OK;
+}
+
+struct Layout {
+  std::vector<size_t> off;  // 2 + 4·depth
+  size_t total = 0;
+};
+
+static Layout make_layout(const gpt_config& c) {
+  Layout L;
+  const size_t d = c.d_model, F = c.d_mlp, V = c.vocab;
+  size_t pos = 0;
+  L.off.push_back(pos); pos += V * d;
+  for (int l = 0; l < c.depth; ++l) {
+    L.off.push_back(pos); pos += 3 * d * d;
+    L.off.push_back(pos); pos += d * d;
+    L.off.push_back(pos); pos += F * d;
+    L.off.push_back(pos); pos += d * F;
+  }
+  L.off.push_back(pos); pos += V * d;
+  L.total = pos;
+  return L;
+}
+
+// ------------------------------------------------------------------------------------------------
+// workspace plan
+// ------------------------------------------------------------------------------------------------
+struct Plan {
+  size_t status, rope, pshadow;
+  size_t x, xf, rhof;
+  // per layer (base + l·stride)
+  size_t r1, rho1, qkv, rq, rk, lse, o, r2, rho2, act, hsq, layer_stride;
+  // CE
+  size_t stats, zt, lse_ce, ell, inv_n, dz, dxf;
+  // backward transients
+  size_t gx, gxb, du, dr, dO, dqkv, delta, emb;
+  size_t total;
+  int vc;  // vocabulary chunk of the backward lm-head
+};
+
+}  // namespace gpt
+
+struct gpt_step {
+  gpt_config cfg;
+  std::vector<int32_t> window;
+  gpt::Layout layout;
+  gpt::Plan plan;
+  int64_t last_launches = 0;
+};
+
+namespace gpt {
+
+static Plan make_plan(const gpt_config& c, size_t n_params) {
+  Plan p{};
+  const size_t M = (size_t)c.batch * c.seq_len, d = c.d_model, F = c.d_mlp, V = c.vocab,
+               H = c.n_heads;
+  size_t pos = 0;
+  auto take = [&](size_t bytes) { size_t o = pos; pos += al256(bytes); return o; };
+  p.status = take(256);
+  p.rope = take((size_t)c.seq_len * c.head_dim * sizeof(float));
+  p.pshadow = (c.param_dtype == GPT_DTYPE_F32) ? take(n_params * 2) : 0;
+  p.x = take(M * d * 2);
+  p.xf = take(M * d * 2);
+  p.rhof = take(M * 4);
+  // per-layer saved activations
+  const size_t layer0 = pos;
+  p.r1 = take(M * d * 2) - layer0;
+  p.rho1 = take(M * 4) - layer0;
+  p.qkv = take(M * 3 * d * 2) - layer0;
+  p.rq = take(M * H * 4) - layer0;
+  p.rk = take(M * H * 4) - layer0;
+  p.lse = take(M * H * 4) - layer0;
+  p.o = take(M * d * 2) - layer0;
+  p.r2 = take(M * d * 2) - layer0;
+  p.rho2 = take(M * 4) - layer0;
+  p.act = take(M * F * 2) - layer0;
+  p.hsq = take(M * F * 2) - layer0;
+  p.layer_stride = pos - layer0;
+  pos = layer0 + p.layer_stride * (size_t)c.depth;
+  // make the per-layer offsets absolute for layer 0
+  p.r1 += layer0; p.rho1 += layer0; p.qkv += layer0; p.rq += layer0; p.rk += layer0;
+  p.lse += layer0; p.o += layer0; p.r2 += layer0; p.rho2 += layer0; p.act += layer0; p.hsq += layer0;
+  // cross-entropy
+  const int tiles = (int)((V + 255) / 256);
+  p.stats = take(M * tiles * sizeof(float2));
+  p.zt = take(M * 4);
+  p.lse_ce = take(M * 4);
+  p.ell = take(M * 4);
+  p.inv_n = take(256);
+  int vc = (int)V;
+  while ((size_t)vc * M * 2 > ((size_t)1 << 29) && vc % 128 == 0 && vc > 256) vc /= 2;
+  p.vc = vc;
+  p.dz = take(M * (size_t)vc * 2);
+  p.dxf = take(M * d * 4);
+  // backward transients
+  p.gx = take(M * d * 4);
+  p.gxb = take(M * d * 2);
+  p.du = take(M * F * 2);
+  p.dr = take(M * d * 2);
+  p.dO = take(M * d * 2);
+  p.dqkv = take(M * 3 * d * 2);
+  p.delta = take(M * H * 4);
+  p.emb = take(embedding_bwd_scratch_bytes((int)M, (int)V));
+  p.total = pos;
+  return p;
+}
+
+// ------------------------------------------------------------------------------------------------
+// the step
+// ------------------------------------------------------------------------------------------------
+static gpt_status run_step(gpt_step* st, const void* params, const int32_t* tokens,
+                           const int32_t* targets, float* loss, float* grads, uint8_t* ws,
+                           cudaStream_t s) {
+  const gpt_config& c = st->cfg;
+  const Plan& p = st->plan;
+  const Layout& L = st->layout;
+  const int B = c.batch, T = c.seq_len, M = B * T, d = c.d_model, F = c.d_mlp, V = c.vocab,
+            H = c.n_heads, Dh = c.head_dim;
+  int* status = reinterpret_cast<int*>(ws + p.status);
+  float* rope = reinterpret_cast<float*>(ws + p.rope);
+  GPT_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
+  const uint16_t* P = reinterpret_cast<const uint16_t*>(params);
+  if (c.param_dtype == GPT_DTYPE_F32) {
+    GPT_TRY(cast_f32_bf16(reinterpret_cast<const float*>(params), ws + p.pshadow, L.total, s));
+    P = reinterpret_cast<const uint16_t*>(ws + p.pshadow);
+  }
+  auto W = [&](int idx) { return P + L.off[idx]; };
+  auto G = [&](int idx) { return grads + L.off[idx]; };
+  auto at = [&](size_t off, int l) { return ws + off + (size_t)l * p.layer_stride; };
+  uint16_t* x = reinterpret_cast<uint16_t*>(ws + p.x);
+  uint16_t* xf = reinterpret_cast<uint16_t*>(ws + p.xf);
+  float* rhof = reinterpret_cast<float*>(ws + p.rhof);
+  const long long qs_b = (long long)T * 3 * d, qs_h = Dh, qs_t = 3 * d;  // q/k/v inside qkv
+  const long long os_b = (long long)T * d, os_h = Dh, os_t = d;          // o / dO
+
+  GPT_TRY(rope_table(rope, T, Dh, s));
+  GPT_TRY(embedding_fwd(tokens, W(0), x, M, d, V, status, s));
+
+  // ---------------- forward ----------------
+  for (int l = 0; l < c.depth; ++l) {
+    const int wq = 1 + 4 * l;
+    uint16_t* r1 = reinterpret_cast<uint16_t*>(at(p.r1, l));
+    float* rho1 = reinterpret_cast<float*>(at(p.rho1, l));
+    uint16_t* qkv = reinterpret_cast<uint16_t*>(at(p.qkv, l));
+    float* rq = reinterpret_cast<float*>(at(p.rq, l));
+    float* rk = reinterpret_cast<float*>(at(p.rk, l));
+    float* lse = reinterpret_cast<float*>(at(p.lse, l));
+    uint16_t* o = reinterpret_cast<uint16_t*>(at(p.o, l));
+    uint16_t* r2 = reinterpret_cast<uint16_t*>(at(p.r2, l));
+    float* rho2 = reinterpret_cast<float*>(at(p.rho2, l));
+    uint16_t* act = reinterpret_cast<uint16_t*>(at(p.act, l));
+    uint16_t* hsq = reinterpret_cast<uint16_t*>(at(p.hsq, l));
+    GPT_TRY(rmsnorm_fwd(x, r1, rho1, M, d, s));
+    GPT_TRY(gemm_launch(GPT_GEMM_NT, GPT_EPI_BF16, M, 3 * d, d, r1, d, W(wq), d, qkv, 3 * d,
+                        nullptr, nullptr, 0, status, s));
+    GPT_TRY(rope_qknorm_fwd(qkv, rq, rk, rope, B, T, H, Dh, s));
+    GPT_TRY(attention_fwd(qkv, qkv + d, qkv + 2 * d, o, lse, B, H, T, Dh, st->window[l], qs_b,
+                          qs_h, qs_t, os_b, os_h, os_t, status, s));
+    GPT_TRY(gemm_launch(GPT_GEMM_NT, GPT_EPI_RESID, M, d, d, o, d, W(wq + 1), d, x, d, nullptr,
+                        nullptr, 0, status, s));
+    GPT_TRY(rmsnorm_fwd(x, r2, rho2, M, d, s));
+    GPT_TRY(gemm_launch(GPT_GEMM_NT, GPT_EPI_RELU2, M, F, d, r2, d, W(wq + 2), d, act, F, hsq,
+                        nullptr, 0, status, s));
+    GPT_TRY(gemm_launch(GPT_GEMM_NT, GPT_EPI_RESID, M, d, F, hsq, F, W(wq + 3), F, x, d, nullptr,
+                        nullptr, 0, status, s));
+  }
+  GPT_TRY(rmsnorm_fwd(x, xf, rhof, M, d, s));
+
+  // ---------------- lm-head + cross-entropy ----------------
+  const int wlm = 1 + 4 * c.depth;
+  const int tiles = (V + 255) / 256;
+  CeArgs ce{};
+  ce.targets = targets;
+  ce.lse = reinterpret_cast<float*>(ws + p.lse_ce);
+  ce.inv_n = reinterpret_cast<float*>(ws + p.inv_n);
+  ce.stats = reinterpret_cast<float2*>(ws + p.stats);
+  ce.stats_ld = tiles;
+  ce.ztarget = reinterpret_cast<float*>(ws + p.zt);
+  ce.n_offset = 0;
+  ce.stats_col0 = 0;
+  GPT_TRY(gemm_ce_launch(false, M, V, d, xf, d, W(wlm), d, nullptr, 0, ce, status, s));
+  GPT_TRY(ce_rows(ce.stats, tiles, ce.ztarget, targets, M, V, const_cast<float*>(ce.lse),
+                  reinterpret_cast<float*>(ws + p.ell), status, s));
+  GPT_TRY(ce_finalize(reinterpret_cast<float*>(ws + p.ell), targets, M, V, loss,
+                      const_cast<float*>(ce.inv_n), s));
+  uint16_t* dz = reinterpret_cast<uint16_t*>(ws + p.dz);
+  float* dxf = reinterpret_cast<float*>(ws + p.dxf);
+  for (int c0 = 0; c0 < V; c0 += p.vc) {
+    const int n = std::min(p.vc, V - c0);
+    ce.n_offset = c0;
+    GPT_TRY(gemm_ce_launch(true, M, n, d, xf, d, W(wlm) + (size_t)c0 * d, d, dz, n, ce, status, s));
+    GPT_TRY(gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, n, d, M, dz, n, xf, d, G(wlm) + (size_t)c0 * d, d,
+                        nullptr, nullptr, 0, status, s));
+    GPT_TRY(gemm_launch(GPT_GEMM_NN, c0 == 0 ? GPT_EPI_F32 : GPT_EPI_F32_ADD, M, d, n, dz, n,
+                        W(wlm) + (size_t)c0 * d, d, dxf, d, nullptr, nullptr, 0, status, s));
+  }
+  float* gx = reinterpret_cast<float*>(ws + p.gx);
+  uint16_t* gxb = reinterpret_cast<uint16_t*>(ws + p.gxb);
+  GPT_TRY(rmsnorm_bwd(dxf, 1, xf, rhof, gx, gxb, 0, M, d, s));
+
+  // ---------------- backward ----------------
+  uint16_t* du = reinterpret_cast<uint16_t*>(ws + p.du);
+  uint16_t* dr = reinterpret_cast<uint16_t*>(ws + p.dr);
+  uint16_t* dO = reinterpret_cast<uint16_t*>(ws + p.dO);
+  uint16_t* dqkv = reinterpret_cast<uint16_t*>(ws + p.dqkv);
+  float* delta = reinterpret_cast<float*>(ws + p.delta);
+  for (int l = c.depth - 1; l >= 0; --l) {
+    const int wq = 1 + 4 * l;
+    uint16_t* r1 = reinterpret_cast<uint16_t*>(at(p.r1, l));
+    float* rho1 = reinterpret_cast<float*>(at(p.rho1, l));
+    uint16_t* qkv = reinterpret_cast<uint16_t*>(at(p.qkv, l));
+    float* rq = reinterpret_cast<float*>(at(p.rq, l));
+    float* rk = reinterpret_cast<float*>(at(p.rk, l));
+    float* lse = reinterpret_cast<float*>(at(p.lse, l));
+    uint16_t* o = reinterpret_cast<uint16_t*>(at(p.o, l));
+    uint16_t* r2 = reinterpret_cast<uint16_t*>(at(p.r2, l));
+    float* rho2 = reinterpret_cast<float*>(at(p.rho2, l));
+    uint16_t* act = reinterpret_cast<uint16_t*>(at(p.act, l));
+    uint16_t* hsq = reinterpret_cast<uint16_t*>(at(p.hsq, l));
+    // MLP
+    GPT_TRY(gemm_launch(GPT_GEMM_NN, GPT_EPI_DRELU2, M, F, d, gxb, d, W(wq + 3), F, du, F, nullptr,
+                        act, F, status, s));
+    GPT_TRY(gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, d, F, M, gxb, d, hsq, F, G(wq + 3), F, nullptr,
+                        nullptr, 0, status, s));
+    GPT_TRY(gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, F, d, M, du, F, r2, d, G(wq + 2), d, nullptr,
+                        nullptr, 0, status, s));
+    GPT_TRY(gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, F, du, F, W(wq + 2), d, dr, d, nullptr,
+                        nullptr, 0, status, s));
+    GPT_TRY(rmsnorm_bwd(dr, 0, r2, rho2, gx, gxb, 1, M, d, s));
+    // attention
+    GPT_TRY(gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, d, gxb, d, W(wq + 1), d, dO, d, nullptr,
+                        nullptr, 0, status, s));
+    GPT_TRY(gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, d, d, M, gxb, d, o, d, G(wq + 1), d, nullptr,
+                        nullptr, 0, status, s));
+    GPT_TRY(attention_bwd(qkv, qkv + d, qkv + 2 * d, o, dO, lse, delta, dqkv, dqkv + d,
+                          dqkv + 2 * d, B, H, T, Dh, st->window[l], qs_b, qs_h, qs_t, os_b, os_h,
+                          os_t, status, s));
+    GPT_TRY(rope_qknorm_bwd(dqkv, qkv, rq, rk, rope, B, T, H, Dh, s));
+    GPT_TRY(gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, 3 * d, d, M, dqkv, 3 * d, r1, d, G(wq), d,
+                        nullptr, nullptr, 0, status, s));
+    GPT_TRY(gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, 3 * d, dqkv, 3 * d, W(wq), d, dr, d,
+                        nullptr, nullptr, 0, status, s));
+    GPT_TRY(rmsnorm_bwd(dr, 0, r1, rho1, gx, gxb, 1, M, d, s));
+  }
+  GPT_TRY(embedding_bwd(tokens, gx, G(0), M, d, V, ws + p.emb, s));
+  return GPT_OK;
+}
+
+}  // namespace gpt
+
+// ================================================================================================
+// C ABI
+// ================================================================================================
+extern "C" {
+
+gpt_status gpt_param_layout(const gpt_config* cfg, size_t* offsets, size_t* total) {
+  gpt_status v = gpt::validate(cfg);
+  if (v != GPT_OK) return v;
+  if (!total) return GPT_ERR_INVALID_ARG;
+  gpt::Layout L = gpt::make_layout(*cfg);
+  if (offsets)
+    for (size_t i = 0; i < L.off.size(); ++i) offsets[i] = L.off[i];
+  *total = L.total;
+  return GPT_OK;
+}
+
+gpt_status gpt_step_create(const gpt_config* cfg, gpt_step** out) {
+  if (!out) return GPT_ERR_INVALID_ARG;
+  *out = nullptr;
+  gpt_status v = gpt::validate(cfg);
+  if (v != GPT_OK) return v;
+  gpt_step* st = new (std::nothrow) gpt_step();
+  if (!st) return GPT_ERR_INVALID_ARG;
+  st->cfg = *cfg;
+  st->window.assign(cfg->depth, 0);
+  if (cfg->window)
+    for (int l = 0; l < cfg->depth; ++l) st->window[l] = cfg->window[l];
+  st->cfg.window = nullptr;  // the copy in st->window is the one used
+  st->layout = gpt::make_layout(*cfg);
+  st->plan = gpt::make_plan(*cfg, st->layout.total);
+  *out = st;
+  return GPT_OK;
+}
+
+void gpt_step_destroy(gpt_step* step) { delete step; }
+
+gpt_status gpt_step_workspace_bytes(const gpt_step* step, size_t* bytes) {
+  if (!step || !bytes) return GPT_ERR_INVALID_ARG;
+  *bytes = step->plan.total;
+  return GPT_OK;
+}
+
+int64_t gpt_step_last_launch_count(const gpt_step* step) { return step ? step->last_launches : -1; }
+
+gpt_status gpt_step_fwd_bwd(gpt_step* step, const void* params, const int32_t* tokens,
+                            const int32_t* targets, float* loss, float* grads, void* workspace,
+                            size_t workspace_bytes, int accumulate, void* stream) {
+  if (!step || !params || !tokens || !targets || !loss || !grads || !workspace)
+    return GPT_ERR_INVALID_ARG;
+  if (accumulate != 0) return GPT_ERR_INVALID_ARG;
+  if (workspace_bytes < step->plan.total) return GPT_ERR_WORKSPACE_TOO_SMALL;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) || (reinterpret_cast<uintptr_t>(params) & 15) ||
+      (reinterpret_cast<uintptr_t>(grads) & 15))
+    return GPT_ERR_UNSUPPORTED_SHAPE;
+  int sms = 0;
+  gpt_status dv = gpt::device_info(&sms);
+  if (dv != GPT_OK) return dv;
+  const int64_t before = gpt::g_launch_count;
+  gpt_status r = gpt::run_step(step, params, tokens, targets, loss, grads,
+                               reinterpret_cast<uint8_t*>(workspace), gpt::as_stream(stream));
+  step->last_launches = gpt::g_launch_count - before;
+  return r;
+}
+
+gpt_status gpt_step_status(const gpt_step* step, const void* workspace, void* stream) {
+  if (!step || !workspace) return GPT_ERR_INVALID_ARG;
+  cudaStream_t s = gpt::as_stream(stream);
+  int* dst = reinterpret_cast<int*>(const_cast<void*>(workspace)) + step->plan.status / sizeof(int);
+  int host = 0;
+  if (cudaMemcpyAsync(&host, dst, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return GPT_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GPT_ERR_CUDA;
+  if (host != 0) {
+    if (cudaMemsetAsync(dst, 0, sizeof(int), s) != cudaSuccess) return GPT_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GPT_ERR_CUDA;
+  }
+  return static_cast<gpt_status>(host);
+}
+
+size_t gpt_lmhead_ce_scratch_bytes(int M, int d, int V) {
+  (void)d;
+  const size_t tiles = (size_t)(V + 255) / 256;
+  return gpt::al256((size_t)M * tiles * 8) + 4 * gpt::al256((size_t)M * 4) + 256 +
+         gpt::al256((size_t)M * V * 2);
+}
+
+gpt_status gpt_lmhead_ce_fwd_bwd(const void* xf, const void* wlm, const int32_t* targets, int M,
+                                 int d, int V, float* loss, float* lse, float* dx, float* dW,
+                                 void* scratch, int* status, void* stream) {
+  if (!xf || !wlm || !targets || !loss || !lse || !dx || !dW || !scratch) return GPT_ERR_INVALID_ARG;
+  if (M <= 0 || d <= 0 || V <= 0) return GPT_ERR_INVALID_ARG;
+  if ((d % 64) || (V % 64)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t s = gpt::as_stream(stream);
+  uint8_t* p = reinterpret_cast<uint8_t*>(scratch);
+  const int tiles = (V + 255) / 256;
+  gpt::CeArgs ce{};
+  ce.targets = targets;
+  ce.stats = reinterpret_cast<float2*>(p);
+  p += gpt::al256((size_t)M * tiles * 8);
+  ce.ztarget = reinterpret_cast<float*>(p); p += gpt::al256((size_t)M * 4);
+  float* ell = reinterpret_cast<float*>(p); p += gpt::al256((size_t)M * 4);
+  p += 2 * gpt::al256((size_t)M * 4);
+  ce.inv_n = reinterpret_cast<float*>(p); p += 256;
+  uint16_t* dz = reinterpret_cast<uint16_t*>(p);
+  ce.lse = lse;
+  ce.stats_ld = tiles;
+  GPT_TRY(gpt::gemm_ce_launch(false, M, V, d, xf, d, wlm, d, nullptr, 0, ce, status, s));
+  GPT_TRY(gpt::ce_rows(ce.stats, tiles, ce.ztarget, targets, M, V, lse, ell, status, s));
+  GPT_TRY(gpt::ce_finalize(ell, targets, M, V, loss, const_cast<float*>(ce.inv_n), s));
+  GPT_TRY(gpt::gemm_ce_launch(true, M, V, d, xf, d, wlm, d, dz, V, ce, status, s));
+  GPT_TRY(gpt::gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, V, d, M, dz, V, xf, d, dW, d, nullptr, nullptr,
+                           0, status, s));
+  GPT_TRY(gpt::gemm_launch(GPT_GEMM_NN, GPT_EPI_F32, M, d, V, dz, V, wlm, d, dx, d, nullptr,
+                           nullptr, 0, status, s));
+  return GPT_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,259 @@
+"""ctypes binding of libgptstep.so (argument marshalling only; every computation runs in the
+library's CUDA kernels).
+
+The names mirror the C entry points of include/gptstep.h.  Tensors are torch tensors on the
+current CUDA device; the library receives their data pointers and the current CUDA stream.  If the
+shared library is missing, loading fails loudly: there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+from .config import DTYPE_F32, GptConfig
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptstep.so")
+_lib = None
+
+GPT_OK = 0
+STATUS_NAMES = {0: "GPT_OK", -1: "GPT_ERR_INVALID_ARG", -2: "GPT_ERR_UNSUPPORTED_SHAPE",
+                -3: "GPT_ERR_WORKSPACE_TOO_SMALL", -4: "GPT_ERR_CUDA", -5: "GPT_ERR_DEVICE_TIMEOUT",
+                -6: "GPT_ERR_TOKEN_OUT_OF_RANGE", -7: "GPT_ERR_NO_DEVICE"}
+GEMM_NT, GEMM_NN, GEMM_TN = 0, 1, 2
+EPI_BF16, EPI_RESID, EPI_RELU2, EPI_DRELU2, EPI_F32, EPI_F32_ADD = 0, 1, 2, 3, 4, 5
+
+EXPORTED = [
+    "gpt_param_layout", "gpt_step_create", "gpt_step_destroy", "gpt_step_workspace_bytes",
+    "gpt_step_fwd_bwd", "gpt_step_status", "gpt_strerror", "gpt_step_last_launch_count",
+    "gpt_gemm", "gpt_rmsnorm_fwd", "gpt_rmsnorm_bwd", "gpt_rope_qknorm_fwd", "gpt_rope_qknorm_bwd",
+    "gpt_rope_table", "gpt_attention_fwd", "gpt_attention_bwd", "gpt_embedding_fwd",
+    "gpt_embedding_bwd_scratch_bytes", "gpt_embedding_bwd", "gpt_lmhead_ce_scratch_bytes",
+    "gpt_lmhead_ce_fwd_bwd",
+]
+
+
+class GptError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("depth", ctypes.c_int32), ("d_model", ctypes.c_int32), ("n_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("d_mlp", ctypes.c_int32), ("vocab", ctypes.c_int32),
+                ("seq_len", ctypes.c_int32), ("batch", ctypes.c_int32),
+                ("window", ctypes.POINTER(ctypes.c_int32)), ("param_dtype", ctypes.c_int32)]
+
+
+def lib():
+    """Load libgptstep.so (built in-tree by gpt_decoder_pretraining_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                              "`python -m gpt_decoder_pretraining_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        ll = ctypes.c_longlong
+        L.gpt_param_layout.argtypes = [ctypes.POINTER(_Config), ctypes.POINTER(sz), ctypes.POINTER(sz)]
+        L.gpt_step_create.argtypes = [ctypes.POINTER(_Config), ctypes.POINTER(vp)]
+        L.gpt_step_destroy.argtypes = [vp]
+        L.gpt_step_destroy.restype = None
+        L.gpt_step_workspace_bytes.argtypes = [vp, ctypes.POINTER(sz)]
+        L.gpt_step_fwd_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, i32, vp]
+        L.gpt_step_status.argtypes = [vp, vp, vp]
+        L.gpt_strerror.argtypes = [i32]
+        L.gpt_strerror.restype = ctypes.c_char_p
+        L.gpt_step_last_launch_count.argtypes = [vp]
+        L.gpt_step_last_launch_count.restype = ctypes.c_int64
+        L.gpt_gemm.argtypes = [i32, i32, i32, i32, i32, vp, i32, vp, i32, vp, i32, vp, vp, i32, vp, vp]
+        L.gpt_rmsnorm_fwd.argtypes = [vp, vp, vp, i32, i32, vp]
+        L.gpt_rmsnorm_bwd.argtypes = [vp, i32, vp, vp, vp, vp, i32, i32, i32, vp]
+        L.gpt_rope_qknorm_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp]
+        L.gpt_rope_qknorm_bwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
+        L.gpt_rope_table.argtypes = [vp, i32, i32, vp]
+        L.gpt_attention_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, ll, ll, ll, ll, ll, ll, vp, vp]
+        L.gpt_attention_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                        ll, ll, ll, ll, ll, ll, vp, vp]
+        L.gpt_embedding_fwd.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp]
+        L.gpt_embedding_bwd_scratch_bytes.argtypes = [i32, i32]
+        L.gpt_embedding_bwd_scratch_bytes.restype = sz
+        L.gpt_embedding_bwd.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp]
+        L.gpt_lmhead_ce_scratch_bytes.argtypes = [i32, i32, i32]
+        L.gpt_lmhead_ce_scratch_bytes.restype = sz
+        L.gpt_lmhead_ce_fwd_bwd.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+        _lib = L
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != GPT_OK:
+        raise GptError(status, what)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream():
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _cconfig(cfg: GptConfig):
+    win = (ctypes.c_int32 * max(1, cfg.depth))(*cfg.windows)
+    c = _Config(cfg.depth, cfg.d_model, cfg.n_heads, cfg.head_dim, cfg.d_mlp, cfg.vocab, cfg.seq_len,
+                cfg.batch, ctypes.cast(win, ctypes.POINTER(ctypes.c_int32)), cfg.param_dtype)
+    return c, win
+
+
+def param_layout(cfg: GptConfig):
+    """(offsets, total) of the flat parameter packing, as the library defines it."""
+    c, _keep = _cconfig(cfg)
+    n = 2 + 4 * cfg.depth
+    offs = (ctypes.c_size_t * n)()
+    total = ctypes.c_size_t(0)
+    _check(lib().gpt_param_layout(ctypes.byref(c), offs, ctypes.byref(total)), "gpt_param_layout")
+    return list(offs), int(total.value)
+
+
+class GptStep:
+    """One training step on the GPU: ``loss, grads = step(params, tokens, targets)``."""
+
+    def __init__(self, cfg: GptConfig, device=None):
+        import torch
+        self.cfg = cfg
+        c, self._win = _cconfig(cfg)
+        h = ctypes.c_void_p()
+        _check(lib().gpt_step_create(ctypes.byref(c), ctypes.byref(h)), "gpt_step_create")
+        self._h = h
+        nbytes = ctypes.c_size_t(0)
+        _check(lib().gpt_step_workspace_bytes(h, ctypes.byref(nbytes)), "gpt_step_workspace_bytes")
+        self.workspace_bytes = int(nbytes.value)
+        self.device = torch.device(device or "cuda")
+        self.workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8, device=self.device)
+        self.offsets, self.n_params = param_layout(cfg)
+        self.loss = torch.zeros(1, dtype=torch.float32, device=self.device)
+        self.grads = torch.empty(self.n_params, dtype=torch.float32, device=self.device)
+
+    def __del__(self):
+        try:
+            if getattr(self, "_h", None) is not None and _lib is not None:
+                _lib.gpt_step_destroy(self._h)
+                self._h = None
+        except Exception:
+            pass
+
+    def __call__(self, params, tokens, targets, grads=None, loss=None):
+        """Enqueue one step on the current stream; returns (loss tensor [1], grads tensor)."""
+        grads = self.grads if grads is None else grads
+        loss = self.loss if loss is None else loss
+        want = "torch.float32" if self.cfg.param_dtype == DTYPE_F32 else "torch.bfloat16"
+        if str(params.dtype) != want or params.numel() != self.n_params:
+            raise ValueError(f"params must be {want}[{self.n_params}]")
+        if tokens.dtype != targets.dtype or str(tokens.dtype) != "torch.int32":
+            raise ValueError("tokens/targets must be int32")
+        st = lib().gpt_step_fwd_bwd(self._h, params.data_ptr(), tokens.data_ptr(), targets.data_ptr(),
+                                    loss.data_ptr(), grads.data_ptr(), self.workspace.data_ptr(),
+                                    self.workspace_bytes, 0, _stream())
+        _check(st, "gpt_step_fwd_bwd")
+        return loss, grads
+
+    def status(self) -> int:
+        return int(lib().gpt_step_status(self._h, self.workspace.data_ptr(), _stream()))
+
+    def last_launch_count(self) -> int:
+        return int(lib().gpt_step_last_launch_count(self._h))
+
+
+# ------------------------------------------------------------------------------------------------
+# kernel-level calls (tensors in, tensors out); used by the unit parity tests and the benchmark
+# ------------------------------------------------------------------------------------------------
+def gemm(op: int, epi: int, A, B, C, M: int, N: int, K: int, C2=None, aux=None, status=None,
+         lda=None, ldb=None, ldc=None):
+    """C (op) A·B as defined for gpt_gemm; row strides default to the tensors' last dimension."""
+    lda = lda or A.shape[-1]
+    ldb = ldb or B.shape[-1]
+    ldc = ldc or C.shape[-1]
+    ldaux = aux.shape[-1] if aux is not None else 0
+    _check(lib().gpt_gemm(op, epi, M, N, K, A.data_ptr(), lda, B.data_ptr(), ldb, C.data_ptr(), ldc,
+                          _ptr(C2), _ptr(aux), ldaux, _ptr(status), _stream()), "gpt_gemm")
+
+
+def rmsnorm_fwd(x, y, rho):
+    rows, d = x.shape
+    _check(lib().gpt_rmsnorm_fwd(x.data_ptr(), y.data_ptr(), rho.data_ptr(), rows, d, _stream()), "rmsnorm_fwd")
+
+
+def rmsnorm_bwd(dy, y, rho, gx, gx_bf16=None, accumulate=False):
+    rows, d = y.shape
+    dy_f32 = 1 if str(dy.dtype) == "torch.float32" else 0
+    _check(lib().gpt_rmsnorm_bwd(dy.data_ptr(), dy_f32, y.data_ptr(), rho.data_ptr(), gx.data_ptr(),
+                                 _ptr(gx_bf16), int(accumulate), rows, d, _stream()), "rmsnorm_bwd")
+
+
+def rope_table(cs, T: int, Dh: int):
+    _check(lib().gpt_rope_table(cs.data_ptr(), T, Dh, _stream()), "rope_table")
+
+
+def rope_qknorm_fwd(qkv, rho_q, rho_k, cs, B, T, H, Dh):
+    _check(lib().gpt_rope_qknorm_fwd(qkv.data_ptr(), rho_q.data_ptr(), rho_k.data_ptr(), cs.data_ptr(),
+                                     B, T, H, Dh, _stream()), "rope_qknorm_fwd")
+
+
+def rope_qknorm_bwd(dqkv, qkv, rho_q, rho_k, cs, B, T, H, Dh):
+    _check(lib().gpt_rope_qknorm_bwd(dqkv.data_ptr(), qkv.data_ptr(), rho_q.data_ptr(), rho_k.data_ptr(),
+                                     cs.data_ptr(), B, T, H, Dh, _stream()), "rope_qknorm_bwd")
+
+
+def attention_fwd(q, k, v, o, lse, window: int, strides_qkv, strides_o, B, H, T, Dh, status=None):
+    _check(lib().gpt_attention_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                   B, H, T, Dh, window, *strides_qkv, *strides_o, _ptr(status), _stream()),
+           "attention_fwd")
+
+
+def attention_bwd(q, k, v, o, do, lse, delta, dq, dk, dv, window: int, strides_qkv, strides_o, B, H, T,
+                  Dh, status=None):
+    _check(lib().gpt_attention_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                   lse.data_ptr(), delta.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                   dv.data_ptr(), B, H, T, Dh, window, *strides_qkv, *strides_o,
+                                   _ptr(status), _stream()), "attention_bwd")
+
+
+def embedding_fwd(tokens, wte, x, status=None):
+    M = tokens.numel()
+    V, d = wte.shape
+    _check(lib().gpt_embedding_fwd(tokens.data_ptr(), wte.data_ptr(), x.data_ptr(), M, d, V, _ptr(status),
+                                   _stream()), "embedding_fwd")
+
+
+def embedding_bwd_scratch_bytes(M: int, V: int) -> int:
+    return int(lib().gpt_embedding_bwd_scratch_bytes(M, V))
+
+
+def embedding_bwd(tokens, gx, dwte, scratch):
+    M = tokens.numel()
+    V, d = dwte.shape
+    _check(lib().gpt_embedding_bwd(tokens.data_ptr(), gx.data_ptr(), dwte.data_ptr(), M, d, V,
+                                   scratch.data_ptr(), _stream()), "embedding_bwd")
+
+
+def lmhead_ce_scratch_bytes(M: int, d: int, V: int) -> int:
+    return int(lib().gpt_lmhead_ce_scratch_bytes(M, d, V))
+
+
+def lmhead_ce_fwd_bwd(xf, wlm, targets, loss, lse, dx, dW, scratch, status=None):
+    M, d = xf.shape
+    V = wlm.shape[0]
+    _check(lib().gpt_lmhead_ce_fwd_bwd(xf.data_ptr(), wlm.data_ptr(), targets.data_ptr(), M, d, V,
+                                       loss.data_ptr(), lse.data_ptr(), dx.data_ptr(), dW.data_ptr(),
+                                       scratch.data_ptr(), _ptr(status), _stream()), "lmhead_ce_fwd_bwd")
+
+
+def flat_to_bf16_tensor(params_f32: np.ndarray, device="cuda"):
+    """Upload bf16-exact float32 values as a torch bfloat16 tensor (exact)."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(params_f32, dtype=np.float32)).to(device).to(torch.bfloat16)

@@ -1,0 +1,192 @@
+/*
+ * gptstep.h — C ABI of libgptstep.so: one training step (forward + backward to parameter
+ * gradients) of a nanochat-style GPT decoder, computed by hand-written sm_100a CUDA kernels.
+ *
+ * The model (nanochat User Guide, §10 "How It Works"; Introducing nanochat, Pretraining section):
+ *   x0 = wte[tok]                                     (no norm after the embedding)
+ *   per layer l:  r1 = RMS(x);  [q|k|v] = r1·W_qkvᵀ;  q̃,k̃ = RMS_Dh(RoPE(q)), RMS_Dh(RoPE(k)) per head
+ *                 o = softmax(q̃k̃ᵀ/√Dh + causal/window mask)·v;   x += o·W_oᵀ
+ *                 r2 = RMS(x);  x += relu(r2·W_fcᵀ)²·W_projᵀ
+ *   x_f = RMS(x);  z = x_f·W_lmᵀ;  loss = mean over valid targets of (logsumexp(z) − z[target])
+ * RMS(x) = x/sqrt(mean(x²) + 1e-6) with no gain; RoPE base 10000 on the pairs (i, i + Dh/2);
+ * window w keeps keys t−w < j ≤ t (w ≤ 0 or w ≥ T: full causal); targets equal to −1 are ignored
+ * (supa beginna nanochat, Troubleshooting: cross_entropy with ignore_index=−1, mean reduction).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers unless a parameter says "host".  The caller owns every
+ *     buffer, including the workspace.  The library never calls cudaMalloc on the step path and keeps
+ *     no pointer after a call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Kernels are
+ *     enqueued on it; results are ready when the stream reaches that point.
+ *   - bf16 tensors are raw IEEE bfloat16 (uint16 storage).  Matrices are row-major.  A weight is
+ *     stored [out, in] and applied as y = x·Wᵀ.
+ *   - Every call returns a gpt_status.  Argument errors are reported before anything is enqueued.
+ *     Nothing aborts, throws across the ABI or traps on the device.  Problems found on the device
+ *     (token id out of range, a bounded wait that expired) are written to a status word that
+ *     gpt_step_status() / the `status` argument of the kernel-level calls report.
+ */
+#ifndef GPTSTEP_H
+#define GPTSTEP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gpt_status {
+  GPT_OK = 0,
+  GPT_ERR_INVALID_ARG = -1,        /* null pointer, non-positive size, bad enum */
+  GPT_ERR_UNSUPPORTED_SHAPE = -2,  /* a size this build cannot tile (see each call) */
+  GPT_ERR_WORKSPACE_TOO_SMALL = -3,
+  GPT_ERR_CUDA = -4,               /* a CUDA runtime call or kernel launch failed */
+  GPT_ERR_DEVICE_TIMEOUT = -5,     /* a bounded device-side wait expired; results are invalid */
+  GPT_ERR_TOKEN_OUT_OF_RANGE = -6, /* a token id outside [0, V) (or a target outside [-1, V)) */
+  GPT_ERR_NO_DEVICE = -7           /* no sm_100 device is current */
+} gpt_status;
+
+enum { GPT_DTYPE_BF16 = 0, GPT_DTYPE_F32 = 1 };
+
+/* Model and batch shape.  d_model = n_heads·head_dim.  head_dim ∈ {32, 64, 128}; d_model, d_mlp and
+ * vocab multiples of 64; seq_len ≥ 1; batch ≥ 1.  `window` is a HOST array of `depth` entries
+ * (copied by gpt_step_create; may be NULL = every layer full causal).  param_dtype selects the
+ * parameter storage: BF16 is used as is, F32 is rounded to a bf16 copy inside the workspace at every
+ * step (weights live in one dtype and are cast on the fly, nanochat User Guide "Precision"). */
+typedef struct gpt_config {
+  int32_t depth, d_model, n_heads, head_dim, d_mlp, vocab, seq_len, batch;
+  const int32_t* window;
+  int32_t param_dtype;
+} gpt_config;
+
+typedef struct gpt_step gpt_step; /* opaque host-side plan; owns no device memory */
+
+/* Flat parameter packing (element offsets, each a multiple of 64):
+ *   offsets[0]            wte   [V, d]
+ *   offsets[1 + 4l + 0]   W_qkv [3d, d]   rows q | k | v, row = part·d + head·Dh + j
+ *   offsets[1 + 4l + 1]   W_o   [d, d]
+ *   offsets[1 + 4l + 2]   W_fc  [F, d]
+ *   offsets[1 + 4l + 3]   W_proj[d, F]
+ *   offsets[1 + 4·depth]  W_lm  [V, d]
+ * `offsets` is a HOST array of 2 + 4·depth entries (may be NULL); *total gets the element count.
+ * Gradients use the same packing in fp32.  Host-only; needs no GPU. */
+gpt_status gpt_param_layout(const gpt_config* cfg, size_t* offsets, size_t* total);
+
+/* Validate cfg and build the host plan.  Host-only; needs no GPU. */
+gpt_status gpt_step_create(const gpt_config* cfg, gpt_step** out);
+void gpt_step_destroy(gpt_step* step);
+
+/* Bytes of device workspace gpt_step_fwd_bwd needs (activations kept for the backward pass,
+ * gradient scratch, statistics).  Host-only. */
+gpt_status gpt_step_workspace_bytes(const gpt_step* step, size_t* bytes);
+
+/* One training step.
+ *   params    [n_params] bf16 or fp32 (cfg.param_dtype), packing as above
+ *   tokens    [batch, seq_len] int32 in [0, V)
+ *   targets   [batch, seq_len] int32 in [0, V) or −1 (ignored)
+ *   loss      1 float: Σ_valid ℓ / n_valid, or 0 when no target is valid (grads are then 0 too)
+ *   grads     [n_params] fp32, overwritten (accumulate must be 0 in this version)
+ *   workspace ≥ gpt_step_workspace_bytes, 256-byte aligned
+ * Out-of-range ids are clamped for memory safety and flagged in the device status word. */
+gpt_status gpt_step_fwd_bwd(gpt_step* step, const void* params, const int32_t* tokens,
+                            const int32_t* targets, float* loss, float* grads, void* workspace,
+                            size_t workspace_bytes, int accumulate, void* stream);
+
+/* Synchronize `stream`, read and clear the device status word that the last step on `workspace`
+ * wrote.  Returns GPT_OK, GPT_ERR_TOKEN_OUT_OF_RANGE or GPT_ERR_DEVICE_TIMEOUT (or GPT_ERR_CUDA). */
+gpt_status gpt_step_status(const gpt_step* step, const void* workspace, void* stream);
+
+const char* gpt_strerror(int status);
+
+/* Number of kernel launches the last gpt_step_fwd_bwd enqueued (host counter, for reporting). */
+int64_t gpt_step_last_launch_count(const gpt_step* step);
+
+/* ---------------------------------------------------------------------------------------------
+ * Kernel-level entry points.  The step is built from these; they are exported for unit parity
+ * tests and for the attention-only workload.  `status` (device int, may be NULL) receives a
+ * device-side error code (0 = fine); it is only ever written with a nonzero code.
+ * --------------------------------------------------------------------------------------------- */
+
+/* Dense bf16 GEMM on the tcgen05 tensor cores, fp32 accumulation in tensor memory.
+ *   op = GPT_GEMM_NT : C[M,N] = A[M,K]·B[N,K]ᵀ      (forward projections; A, B K-contiguous)
+ *   op = GPT_GEMM_NN : C[M,N] = A[M,K]·B[K,N]       (activation gradient; B N-contiguous)
+ *   op = GPT_GEMM_TN : C[M,N] = A[K,M]ᵀ·B[K,N]      (weight gradient; A, B M/N-contiguous)
+ * lda/ldb/ldc/ldaux are row strides in elements (multiples of 8 for bf16, 4 for fp32).
+ * epilogue (what is written for each accumulator value acc at (m, n)):
+ *   GPT_EPI_BF16    C = bf16(acc)
+ *   GPT_EPI_RESID   C = bf16(C + acc)                 (C bf16, residual add in place)
+ *   GPT_EPI_RELU2   C = bf16(max(acc,0)), C2 = bf16(max(acc,0)²)   (C2 uses ldc)
+ *   GPT_EPI_DRELU2  C = bf16(acc · 2 · aux)           (aux bf16 = max(u,0) saved by RELU2)
+ *   GPT_EPI_F32     C = acc                           (C fp32)
+ *   GPT_EPI_F32_ADD C = C + acc                       (C fp32)
+ * Sizes: M, N ≥ 1; K ≥ 1 (tails are zero-filled).  Pointers 16-byte aligned. */
+enum { GPT_GEMM_NT = 0, GPT_GEMM_NN = 1, GPT_GEMM_TN = 2 };
+enum {
+  GPT_EPI_BF16 = 0, GPT_EPI_RESID = 1, GPT_EPI_RELU2 = 2, GPT_EPI_DRELU2 = 3,
+  GPT_EPI_F32 = 4, GPT_EPI_F32_ADD = 5
+};
+gpt_status gpt_gemm(int op, int epilogue, int M, int N, int K, const void* A, int lda,
+                    const void* B, int ldb, void* C, int ldc, void* C2, const void* aux,
+                    int ldaux, int* status, void* stream);
+
+/* RMSNorm forward over rows of d (bf16 in/out), y = x·rho, rho = 1/sqrt(mean(x²)+1e-6) (fp32). */
+gpt_status gpt_rmsnorm_fwd(const void* x, void* y, float* rho, int rows, int d, void* stream);
+
+/* RMSNorm backward: g = rho·(dy − y·mean(y·dy)).  dy is bf16 (dy_f32 = 0) or fp32 (dy_f32 = 1).
+ * gx (fp32 [rows,d]) receives g (accumulate = 0) or gx + g (accumulate = 1); gx_bf16 (may be NULL)
+ * receives a bf16 copy of the new gx. */
+gpt_status gpt_rmsnorm_bwd(const void* dy, int dy_f32, const void* y, const float* rho, float* gx,
+                           void* gx_bf16, int accumulate, int rows, int d, void* stream);
+
+/* RoPE + QK-norm forward on qkv [B·T, 3·H·Dh] (bf16, output of the QKV projection), in place:
+ * the q and k blocks of every head become RMS_Dh(RoPE(·, t)); v is untouched.  rho_q, rho_k fp32
+ * [B·T, H].  cos_sin: fp32 [T, Dh/2, 2] table from gpt_rope_table. */
+gpt_status gpt_rope_qknorm_fwd(void* qkv, float* rho_q, float* rho_k, const float* cos_sin, int B,
+                               int T, int H, int Dh, void* stream);
+/* Backward of the above, in place on dqkv (q and k blocks hold dq̃, dk̃ on entry, dq, dk on exit);
+ * qkv holds the forward output (q̃, k̃). */
+gpt_status gpt_rope_qknorm_bwd(void* dqkv, const void* qkv, const float* rho_q, const float* rho_k,
+                               const float* cos_sin, int B, int T, int H, int Dh, void* stream);
+/* Fill cos_sin [T, Dh/2, 2] with cos/sin of t·10000^(−2i/Dh), angles computed in fp64. */
+gpt_status gpt_rope_table(float* cos_sin, int T, int Dh, void* stream);
+
+/* Causal / sliding-window flash attention.  q, k, v, o, dq, dk, dv are bf16 tensors addressed as
+ * element (b, h, t, j) at base + b·sb + h·sh + t·st + j (strides in elements, j contiguous), one
+ * stride set per tensor group: (sb_qkv, sh_qkv, st_qkv) for q/k/v/dq/dk/dv and (sb_o, sh_o, st_o)
+ * for o/do.  lse, delta: fp32 [B, H, T].  Dh ∈ {64, 128}.  window ≤ 0 or ≥ T = full causal.
+ * lse = natural-log logsumexp of the scaled scores; delta = rowsum(dO∘O) (computed by the bwd). */
+gpt_status gpt_attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int H, int T, int Dh, int window, long long sb_qkv,
+                             long long sh_qkv, long long st_qkv, long long sb_o, long long sh_o,
+                             long long st_o, int* status, void* stream);
+gpt_status gpt_attention_bwd(const void* q, const void* k, const void* v, const void* o,
+                             const void* dout, const float* lse, float* delta, void* dq, void* dk,
+                             void* dv, int B, int H, int T, int Dh, int window, long long sb_qkv,
+                             long long sh_qkv, long long st_qkv, long long sb_o, long long sh_o,
+                             long long st_o, int* status, void* stream);
+
+/* Embedding gather x[m] = wte[tok[m]] (bf16 rows of d).  Ids outside [0, V) are clamped and
+ * flagged in *status. */
+gpt_status gpt_embedding_fwd(const int32_t* tokens, const void* wte, void* x, int M, int d, int V,
+                             int* status, void* stream);
+/* Embedding backward dwte = Σ_{m: tok[m]=v} gx[m] for every row v (fp32, rows without a token are
+ * zeroed).  Duplicate ids are summed in ascending m, so the result is deterministic.  scratch:
+ * device bytes ≥ gpt_embedding_bwd_scratch_bytes(M, V). */
+size_t gpt_embedding_bwd_scratch_bytes(int M, int V);
+gpt_status gpt_embedding_bwd(const int32_t* tokens, const float* gx, float* dwte, int M, int d,
+                             int V, void* scratch, void* stream);
+
+/* Fused lm-head + softmax cross-entropy, vocabulary processed in tiles so the [M, V] logits are
+ * never stored.  Forward: lse[m] = logsumexp_v(x_f[m]·W_lm[v]), loss = Σ_valid (lse − z[target])
+ * / n_valid.  Backward (dz = (softmax − onehot)/n_valid, rows with target −1 get 0):
+ * dx (fp32 [M,d]) = dz·W_lm and dW (fp32 [V,d]) = dzᵀ·x_f.  x_f, W_lm bf16.  scratch: device
+ * bytes ≥ gpt_lmhead_ce_scratch_bytes(M, d, V). */
+size_t gpt_lmhead_ce_scratch_bytes(int M, int d, int V);
+gpt_status gpt_lmhead_ce_fwd_bwd(const void* xf, const void* wlm, const int32_t* targets, int M,
+                                 int d, int V, float* loss, float* lse, float* dx, float* dW,
+                                 void* scratch, int* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPTSTEP_H */

@@ -1,0 +1,301 @@
+"""Kernel-level parity of the CUDA path against the oracle's definitions (needs a B200).
+
+Every call goes through the C ABI of libgptstep.so.  Inputs are seeded and bf16-exact; the
+references are the oracle's functions (or, for the GEMM, the fp64 matrix product that defines it)
+evaluated in float64 on the same values.  Sizes span several tiles and ragged tails.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import gpt_oracle as O
+from tests.gpu_util import assert_close_rel, bf16_tensor, cosine, randn, to_np
+
+pytestmark = pytest.mark.gpu
+
+S = None
+
+
+def setup_module(module):
+    global S
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from gpt_decoder_pretraining_b200 import step
+    S = step
+    S.lib()
+
+
+def _status():
+    return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+# --------------------------------------------------------------------------------------------------
+# GEMM: the three operand layouts and every epilogue
+# --------------------------------------------------------------------------------------------------
+GEMM_SHAPES = [(128, 64, 64), (296, 200, 200), (256, 520, 640), (136, 384, 96), (2048, 2560, 256)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+@pytest.mark.parametrize("op", [0, 1, 2])
+def test_gemm_layouts_bf16_and_f32(op, M, N, K):
+    rng = np.random.default_rng(M * 7 + N * 3 + K + op)
+    A = randn(rng, *( (K, M) if op == 2 else (M, K) ))
+    B = randn(rng, *( (N, K) if op == 0 else (K, N) ))
+    ref = (A.T if op == 2 else A) @ (B.T if op == 0 else B)
+    tA, tB = bf16_tensor(A), bf16_tensor(B)
+    st = _status()
+    C = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+    S.gemm(op, S.EPI_BF16, tA, tB, C, M, N, K, status=st)
+    Cf = torch.zeros(M, N, dtype=torch.float32, device="cuda")
+    S.gemm(op, S.EPI_F32, tA, tB, Cf, M, N, K, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert_close_rel(to_np(C), ref, rel=8e-3, what="bf16 out")
+    assert_close_rel(to_np(Cf), ref, rel=1e-5, cos=0.9999999, what="f32 out")
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 200, 200), (256, 520, 640)])
+def test_gemm_epilogues(M, N, K):
+    rng = np.random.default_rng(11)
+    A, B = randn(rng, M, K), randn(rng, N, K)
+    acc = A @ B.T
+    tA, tB = bf16_tensor(A), bf16_tensor(B)
+    # residual add in place
+    X = randn(rng, M, N, scale=3.0)
+    tX = bf16_tensor(X)
+    S.gemm(0, S.EPI_RESID, tA, tB, tX, M, N, K)
+    # ReLU² (relu and its square)
+    Ca = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+    Ch = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+    S.gemm(0, S.EPI_RELU2, tA, tB, Ca, M, N, K, C2=Ch)
+    # dReLU²: acc·2·aux
+    aux = np.maximum(randn(rng, M, N), 0)
+    Cd = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+    S.gemm(0, S.EPI_DRELU2, tA, tB, Cd, M, N, K, aux=bf16_tensor(aux))
+    # fp32 accumulate
+    base = rng.standard_normal((M, N)).astype(np.float32)
+    Cf = torch.from_numpy(base).cuda()
+    S.gemm(0, S.EPI_F32_ADD, tA, tB, Cf, M, N, K)
+    torch.cuda.synchronize()
+    assert_close_rel(to_np(tX), X + acc, rel=8e-3, what="resid")
+    r = np.maximum(acc, 0)
+    assert_close_rel(to_np(Ca), r, rel=8e-3, what="relu")
+    assert_close_rel(to_np(Ch), r * r, rel=8e-3, what="relu2")
+    assert_close_rel(to_np(Cd), acc * 2 * aux, rel=8e-3, what="drelu2")
+    assert_close_rel(to_np(Cf), base + acc, rel=1e-5, cos=0.9999999, what="f32 add")
+
+
+def test_gemm_rejects_bad_arguments():
+    t = torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(S.GptError):
+        S.gemm(0, S.EPI_BF16, t, t, t, 0, 64, 64)
+    with pytest.raises(S.GptError):
+        S.gemm(7, S.EPI_BF16, t, t, t, 64, 64, 64)
+    with pytest.raises(S.GptError):
+        S.gemm(0, 99, t, t, t, 64, 64, 64)
+
+
+# --------------------------------------------------------------------------------------------------
+# RMSNorm
+# --------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("rows,d", [(1, 64), (77, 768), (300, 1536)])
+def test_rmsnorm_fwd_bwd(rows, d):
+    rng = np.random.default_rng(rows + d)
+    x = randn(rng, rows, d, scale=2.0)
+    dy = randn(rng, rows, d)
+    g0 = rng.standard_normal((rows, d))
+    y_ref, rho_ref = O.rmsnorm(x)
+    tx = bf16_tensor(x)
+    ty = torch.empty_like(tx)
+    rho = torch.empty(rows, dtype=torch.float32, device="cuda")
+    S.rmsnorm_fwd(tx, ty, rho)
+    torch.cuda.synchronize()
+    assert_close_rel(to_np(ty), y_ref, rel=8e-3, what="y")
+    np.testing.assert_allclose(to_np(rho), rho_ref[:, 0], rtol=1e-5)
+    # backward with y as stored by the forward (bf16) and accumulate into g0
+    y_b = to_np(ty)
+    ref = g0 + O.rmsnorm_backward(dy, y_b, to_np(rho)[:, None])
+    gx = torch.from_numpy(g0.astype(np.float32)).cuda()
+    gxb = torch.empty(rows, d, dtype=torch.bfloat16, device="cuda")
+    S.rmsnorm_bwd(bf16_tensor(dy), ty, rho, gx, gxb, accumulate=True)
+    gx2 = torch.zeros(rows, d, dtype=torch.float32, device="cuda")
+    S.rmsnorm_bwd(torch.from_numpy(dy.astype(np.float32)).cuda(), ty, rho, gx2, None, accumulate=False)
+    torch.cuda.synchronize()
+    assert_close_rel(to_np(gx), ref, rel=1e-5, cos=0.9999999, what="gx")
+    assert_close_rel(to_np(gxb), ref, rel=8e-3, what="gx bf16")
+    assert_close_rel(to_np(gx2), ref - g0, rel=1e-5, cos=0.9999999, what="gx f32 dy")
+
+
+# --------------------------------------------------------------------------------------------------
+# RoPE + QK-norm
+# --------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("B,T,H,Dh", [(1, 5, 2, 32), (2, 130, 3, 64), (1, 257, 2, 128)])
+def test_rope_qknorm_fwd_bwd(B, T, H, Dh):
+    rng = np.random.default_rng(B * 100 + T + Dh)
+    d = H * Dh
+    qkv = randn(rng, B * T, 3 * d, scale=1.5)
+    dqkv = randn(rng, B * T, 3 * d)
+    cs = torch.empty(T * Dh, dtype=torch.float32, device="cuda")
+    S.rope_table(cs, T, Dh)
+    tq = bf16_tensor(qkv)
+    rq = torch.empty(B * T * H, dtype=torch.float32, device="cuda")
+    rk = torch.empty_like(rq)
+    S.rope_qknorm_fwd(tq, rq, rk, cs, B, T, H, Dh)
+    torch.cuda.synchronize()
+    cos, sin = O.rope_angles(T, Dh, np.float64)
+    got = to_np(tq).reshape(B, T, 3, H, Dh)
+    x = qkv.reshape(B, T, 3, H, Dh)
+    for b in range(B):
+        for part in range(2):
+            ref, rho = O.rmsnorm(O.rope(x[b, :, part], cos, sin))
+            assert_close_rel(got[b, :, part], ref, rel=1e-2, what=f"fwd part {part}")
+            r_got = to_np(rq if part == 0 else rk).reshape(B, T, H)[b]
+            np.testing.assert_allclose(r_got, rho[..., 0], rtol=2e-3)
+        assert np.array_equal(got[b, :, 2], x[b, :, 2])  # v untouched
+    # backward on the stored forward output
+    td = bf16_tensor(dqkv)
+    S.rope_qknorm_bwd(td, tq, rq, rk, cs, B, T, H, Dh)
+    torch.cuda.synchronize()
+    gd = to_np(td).reshape(B, T, 3, H, Dh)
+    dx = dqkv.reshape(B, T, 3, H, Dh)
+    for b in range(B):
+        for part in range(2):
+            yv = got[b, :, part]
+            rho = to_np(rq if part == 0 else rk).reshape(B, T, H)[b][..., None]
+            ref = O.rope_inverse(O.rmsnorm_backward(dx[b, :, part], yv, rho), cos, sin)
+            assert_close_rel(gd[b, :, part], ref, rel=1e-2, what=f"bwd part {part}")
+
+
+# --------------------------------------------------------------------------------------------------
+# attention
+# --------------------------------------------------------------------------------------------------
+ATTN_CASES = [(1, 1, 1, 64, 0), (2, 2, 63, 64, 0), (1, 2, 128, 32, 0), (2, 1, 77, 32, 9), (1, 3, 200, 128, 0), (2, 1, 200, 128, 17),
+              (1, 2, 130, 64, 1), (1, 1, 257, 128, 64), (1, 2, 128, 128, 1000)]
+
+
+@pytest.mark.parametrize("B,H,T,Dh,window", ATTN_CASES)
+def test_attention_fwd_bwd(B, H, T, Dh, window):
+    rng = np.random.default_rng(B * 1000 + H * 100 + T + Dh + window)
+    q, k, v, do = (randn(rng, B, H, T, Dh) for _ in range(4))
+    # QK-normalised inputs, as in the model
+    q = np.asarray([[O.rmsnorm(q[b, h])[0] for h in range(H)] for b in range(B)])
+    k = np.asarray([[O.rmsnorm(k[b, h])[0] for h in range(H)] for b in range(B)])
+    from gpt_decoder_pretraining_b200.inputs import round_to_bf16
+    q = round_to_bf16(q.astype(np.float32)).astype(np.float64)
+    k = round_to_bf16(k.astype(np.float32)).astype(np.float64)
+    o_ref, lse_ref = O.attention_batch_forward(q, k, v, window)
+    dq_ref, dk_ref, dv_ref = O.attention_batch_backward(q, k, v, do, window)
+    tq, tk, tv, tdo = (bf16_tensor(a) for a in (q, k, v, do))
+    strides = (H * T * Dh, T * Dh, Dh)
+    to = torch.zeros(B, H, T, Dh, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
+    st = _status()
+    S.attention_fwd(tq, tk, tv, to, lse, window, strides, strides, B, H, T, Dh, status=st)
+    dq, dk, dv = (torch.zeros_like(tq) for _ in range(3))
+    delta = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
+    S.attention_bwd(tq, tk, tv, to, tdo, lse, delta, dq, dk, dv, window, strides, strides, B, H, T, Dh,
+                    status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert_close_rel(to_np(to), o_ref, rel=2e-2, cos=0.9999, what="o")
+    np.testing.assert_allclose(to_np(lse), lse_ref, atol=2e-3)
+    assert_close_rel(to_np(dq), dq_ref, rel=3e-2, cos=0.999, what="dq")
+    assert_close_rel(to_np(dk), dk_ref, rel=3e-2, cos=0.999, what="dk")
+    assert_close_rel(to_np(dv), dv_ref, rel=3e-2, cos=0.999, what="dv")
+
+
+def test_attention_token_major_strides():
+    """q/k/v read from a [B·T, 3·H·Dh] buffer and o written to [B·T, H·Dh], as the step does."""
+    B, H, T, Dh, window = 2, 2, 96, 64, 40
+    rng = np.random.default_rng(5)
+    d = H * Dh
+    qkv = randn(rng, B * T, 3 * d)
+    tqkv = bf16_tensor(qkv)
+    to = torch.zeros(B * T, d, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
+    sq = (T * 3 * d, Dh, 3 * d)
+    so = (T * d, Dh, d)
+    S.attention_fwd(tqkv, tqkv[:, d:], tqkv[:, 2 * d:], to, lse, window, sq, so, B, H, T, Dh)
+    torch.cuda.synchronize()
+    x = qkv.reshape(B, T, 3, H, Dh).transpose(2, 0, 3, 1, 4)  # [3, B, H, T, Dh]
+    o_ref, _ = O.attention_batch_forward(x[0], x[1], x[2], window)
+    got = to_np(to).reshape(B, T, H, Dh).transpose(0, 2, 1, 3)
+    assert_close_rel(got, o_ref, rel=2e-2, what="o token-major")
+
+
+# --------------------------------------------------------------------------------------------------
+# embedding
+# --------------------------------------------------------------------------------------------------
+def test_embedding_fwd_bwd_deterministic():
+    rng = np.random.default_rng(3)
+    V, d, M = 512, 128, 3000
+    from gpt_decoder_pretraining_b200.inputs import _zipf_ids
+    tok = _zipf_ids(rng, M, V)
+    wte = randn(rng, V, d)
+    gx = rng.standard_normal((M, d)).astype(np.float32)
+    ttok = torch.from_numpy(tok).cuda()
+    x = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+    S.embedding_fwd(ttok, bf16_tensor(wte), x)
+    scratch = torch.empty(S.embedding_bwd_scratch_bytes(M, V), dtype=torch.uint8, device="cuda")
+    dw1 = torch.full((V, d), 7.0, dtype=torch.float32, device="cuda")
+    dw2 = torch.empty((V, d), dtype=torch.float32, device="cuda")
+    tg = torch.from_numpy(gx).cuda()
+    S.embedding_bwd(ttok, tg, dw1, scratch)
+    S.embedding_bwd(ttok, tg, dw2, scratch)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(x), wte[tok])
+    ref = np.zeros((V, d))
+    np.add.at(ref, tok, gx.astype(np.float64))
+    assert_close_rel(to_np(dw1), ref, rel=1e-6, cos=0.9999999, what="dwte")
+    assert torch.equal(dw1, dw2)  # bitwise reproducible
+
+
+def test_embedding_out_of_range_is_flagged_not_faulted():
+    V, d = 64, 64
+    tok = torch.tensor([0, 5, 64, -3, 63], dtype=torch.int32, device="cuda")
+    wte = torch.randn(V, d, device="cuda").to(torch.bfloat16)
+    x = torch.empty(5, d, dtype=torch.bfloat16, device="cuda")
+    st = _status()
+    S.embedding_fwd(tok, wte, x, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == -6
+    assert torch.equal(x[2], wte[63]) and torch.equal(x[3], wte[0])
+
+
+# --------------------------------------------------------------------------------------------------
+# fused lm-head + cross-entropy
+# --------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("M,d,V,ignore", [(128, 64, 2048, 0), (300, 128, 1000 // 64 * 64 + 64, 7),
+                                           (256, 64, 512, 256)])
+def test_lmhead_ce(M, d, V, ignore):
+    rng = np.random.default_rng(M + d + V)
+    xf = randn(rng, M, d)
+    w = randn(rng, V, d, scale=0.5)
+    y = rng.integers(0, V, M).astype(np.int32)
+    y[:ignore] = -1
+    z = xf @ w.T
+    lse_ref = O.logsumexp_rows(z)
+    valid = y >= 0
+    n = int(valid.sum())
+    loss_ref = float(np.sum((lse_ref - z[np.arange(M), np.maximum(y, 0)])[valid]) / n) if n else 0.0
+    dz = O.softmax_rows(z)
+    dz[np.arange(M), np.maximum(y, 0)] -= 1.0
+    dz *= (valid / max(n, 1))[:, None]
+    txf, tw = bf16_tensor(xf), bf16_tensor(w)
+    ty = torch.from_numpy(y).cuda()
+    loss = torch.zeros(1, device="cuda")
+    lse = torch.zeros(M, device="cuda")
+    dx = torch.zeros(M, d, device="cuda")
+    dW = torch.zeros(V, d, device="cuda")
+    scratch = torch.empty(S.lmhead_ce_scratch_bytes(M, d, V), dtype=torch.uint8, device="cuda")
+    S.lmhead_ce_fwd_bwd(txf, tw, ty, loss, lse, dx, dW, scratch)
+    torch.cuda.synchronize()
+    assert abs(loss.item() - loss_ref) < 2e-3
+    np.testing.assert_allclose(to_np(lse), lse_ref, atol=2e-3)
+    if n:
+        assert_close_rel(to_np(dx), dz @ w, rel=2e-2, cos=0.9999, what="dx")
+        assert_close_rel(to_np(dW), dz.T @ xf, rel=2e-2, cos=0.9999, what="dW")
+    else:
+        assert not torch.any(dx) and not torch.any(dW)
