@@ -1,0 +1,347 @@
+"""Benchmark of one GPT training step (forward + backward to parameter gradients) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config d24] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  Metric: training tokens/s of the fwd+bwd step and its MFU
+(FLOPs/token × tokens/s ÷ 2.25e15, the nominal dense-bf16 peak of one B200), FLOPs/token by the
+nanochat convention 6·(N − V·d) + 12·H·Dh·Σ_l min(w_l, T).
+
+* `value`: whole-job tokens/s with inputs already resident in HBM, timed by CUDA events on the
+  step's stream over K steps bracketed by barrier + synchronize, max over ranks.  Activations
+  (tens of GB) exceed the 126 MB L2, so no flush is needed between steps.
+* `e2e`: the same metric through the public API (GptStep) with the step's tokens/targets copied
+  from pinned host memory and the loss copied back every step, inside the timed region.
+* `roofline`: the GEMM class (the dominant kernel family) — algorithmic FLOPs ÷ its CUDA-event
+  time measured inside the timed region — against the measured sustained bf16 peak.
+* `cpu_baseline`: the CPU oracle timed on this host on a bounded sample (rank 0, N = 1).
+* N > 1 (torchrun): each rank runs an independent replica on its own batch (weak scaling); the
+  only collectives are the barrier and the max-reduction of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from gpt_decoder_pretraining_b200.config import B200_DENSE_BF16_PEAK, preset  # noqa: E402
+from gpt_decoder_pretraining_b200.inputs import make_params, make_tokens  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if any."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d.get(workload)
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": ["no samples"]}
+        # "under load": samples at or above half of the max power seen
+        pmax = max(power) if power else 0
+        loaded = [s for s, p in zip(sm, power) if p >= 0.5 * pmax] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": pmax}
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle arm
+# ------------------------------------------------------------------------------------------------
+def cpu_sample_config(cfg, tokens: int):
+    import dataclasses
+    T = min(cfg.seq_len, tokens)
+    wins = [w if (0 < w < T) else 0 for w in cfg.windows]
+    return dataclasses.replace(cfg, batch=1, seq_len=T, windows=wins)
+
+
+def time_oracle(cfg, sample_tokens: int, repeats: int = 1, warmup: int = 0, params=None):
+    """Wall times of the oracle's fp32 fwd+bwd on one row of `sample_tokens` tokens."""
+    from oracle import gpt_oracle as O
+    scfg = cpu_sample_config(cfg, sample_tokens)
+    p = params if params is not None else make_params(scfg.n_params, keep_fp32=(cfg.param_dtype == 1))
+    t, y = make_tokens(1, scfg.seq_len, scfg.vocab, scfg.token_dist)
+    times = []
+    for i in range(warmup + repeats):
+        t0 = time.perf_counter()
+        O.step(scfg, p, t, y, dtype=np.float32)
+        dt = time.perf_counter() - t0
+        if i >= warmup:
+            times.append(dt)
+    return scfg, times
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cores = cpu_cores()
+    scfg, times = time_oracle(cfg, args.cpu_sample_tokens, repeats=args.steps, warmup=args.warmup)
+    per_step = statistics.median(times)
+    value = scfg.seq_len / per_step
+    mfu = cfg.flops_per_token() * value / B200_DENSE_BF16_PEAK
+    sample = (f"one row of {scfg.seq_len} tokens of the {cfg.name} model (B=1), fp32 NumPy oracle "
+              f"fwd+bwd, median of {args.steps} after {args.warmup} warm-up")
+    line = {
+        "impl": "reference", "metric": "training tokens/sec per fwd+bwd step, 1 GPU", "value": value,
+        "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic", "mfu": mfu,
+        "config": {"workload": f"{cfg.name} GPT fwd+bwd step (CPU oracle sample)", "model": cfg.name,
+                   "global_batch": 1, "seq_len": scfg.seq_len, "parallelism": "none"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------------------
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+    from gpt_decoder_pretraining_b200.step import GptStep
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    step = GptStep(cfg, device=dev)
+    params_np = make_params(cfg.n_params, keep_fp32=(cfg.param_dtype == 1))
+    params = torch.from_numpy(params_np).to(dev)
+    if cfg.param_dtype == 0:
+        params = params.to(torch.bfloat16)
+    tok_np, tgt_np = make_tokens(cfg.batch, cfg.seq_len, cfg.vocab, cfg.token_dist, seed=1 + rank)
+    tokens = torch.from_numpy(tok_np).to(dev)
+    targets = torch.from_numpy(tgt_np).to(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # warm-up
+    for _ in range(args.warmup):
+        step(params, tokens, targets)
+    torch.cuda.synchronize(dev)
+    st = step.status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+    loss0 = float(step.loss.item())
+
+    # ---------------- timed region (device-resident inputs) ----------------
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    clocks.start()
+    time.sleep(0.3)
+    step.set_profiling(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    launches = 0
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(params, tokens, targets)
+        launches += step.last_launch_count()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    clk = clocks.stop()
+    step.set_profiling(False)
+    prof = step.profile()
+
+    # ---------------- end to end through the public API, host buffers ----------------
+    tok_h = torch.from_numpy(tok_np).pin_memory()
+    tgt_h = torch.from_numpy(tgt_np).pin_memory()
+    loss_h = torch.zeros(1, dtype=torch.float32).pin_memory()
+    tok_d, tgt_d = torch.empty_like(tokens), torch.empty_like(targets)
+    barrier()
+    torch.cuda.synchronize(dev)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        tok_d.copy_(tok_h, non_blocking=True)
+        tgt_d.copy_(tgt_h, non_blocking=True)
+        loss, _ = step(params, tok_d, tgt_d)
+        loss_h.copy_(loss, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms_e2e = f0.elapsed_time(f1) / args.steps
+
+    if world > 1:
+        t = torch.tensor([ms, ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, ms_e2e = float(t[0]), float(t[1])
+
+    tokens_step = cfg.batch * cfg.seq_len
+    value = tokens_step * world / (ms / 1e3)
+    value_e2e = tokens_step * world / (ms_e2e / 1e3)
+    fpt = cfg.flops_per_token()
+    mfu = fpt * value / (world * B200_DENSE_BF16_PEAK)
+
+    peaks, peak_src = load_peaks()
+    g_ms, g_calls, g_fl, _ = prof["gemm"]
+    achieved = (g_fl / (g_ms / 1e3)) / 1e12 if g_ms > 0 else None
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    kernels = {}
+    for name, (kms, calls, fl, by) in prof.items():
+        if calls == 0:
+            continue
+        ent = {"ms_per_step": kms / args.steps, "calls_per_step": calls // args.steps,
+               "share": kms / (ms * args.steps)}
+        if fl:
+            ent["tflops"] = fl / (kms / 1e3) / 1e12
+        if by:
+            ent["gbs"] = by / (kms / 1e3) / 1e9
+        kernels[name] = ent
+    workload = f"{cfg.name} GPT fwd+bwd step"
+    line = {
+        "metric": "training tokens/sec per fwd+bwd step, 1 GPU (MFU in 'mfu')",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,0.02) params, "
+                                   f"{cfg.token_dist} token ids)",
+        "mfu": mfu, "mfu_of_measured_sustained": fpt * value / (world * peak_sus * 1e12),
+        "flops_per_token": fpt,
+        "config": {"workload": workload, "model": cfg.name, "global_batch": cfg.batch * world,
+                   "seq_len": cfg.seq_len, "parallelism": f"replicas{world}" if world > 1 else "none",
+                   "depth": cfg.depth, "d_model": cfg.d_model, "vocab": cfg.vocab,
+                   "windows": "SSSL w=1024" if any(cfg.windows) else "full causal",
+                   "l2": "inputs larger than L2 (activations ~tens of GB), no flush"},
+        "loss_first_step": loss0,
+        "e2e": {"value": value_e2e, "unit": "tokens/s",
+                "h2d_bytes_per_step": int(tok_np.nbytes + tgt_np.nbytes), "d2h_bytes_per_step": 4},
+        "gpu_launches": int(launches),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
+                     "frac": (achieved / peak_sus) if achieved else None,
+                     "peak_source": f"bf16_tflops_sustained of {peak_src}",
+                     "kernel": "tcgen05 GEMM family (all projection, MLP and lm-head GEMMs)",
+                     "traffic": load_traffic(workload)},
+        "kernels": kernels,
+        "clocks": clk,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cores = cpu_cores()
+        scfg, times = time_oracle(cfg, args.cpu_sample_tokens, repeats=1, warmup=0, params=params_np)
+        cv = scfg.seq_len / times[0]
+        line["cpu_baseline"] = {
+            "value": cv, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"one row of {scfg.seq_len} tokens of the {cfg.name} model (B=1), fp32 NumPy "
+                      f"oracle fwd+bwd, one timed run ({times[0]:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="d24")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-sample-tokens", type=int, default=512)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    cfg = preset(args.config)
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -106,12 +106,39 @@ struct Plan {
 
 }  // namespace gpt
 
+namespace gpt {
+// Optional per-launch CUDA-event timing, by kernel class (see gpt_step_profile).
+struct Profiler {
+  struct Rec {
+    int cls;
+    double flops, bytes;
+    cudaEvent_t a, b;
+  };
+  bool on = false;
+  std::vector<cudaEvent_t> pool;
+  size_t used = 0;
+  std::vector<Rec> recs;
+  cudaEvent_t get() {
+    if (used < pool.size()) return pool[used++];
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    pool.push_back(e);
+    ++used;
+    return e;
+  }
+  ~Profiler() {
+    for (cudaEvent_t e : pool) cudaEventDestroy(e);
+  }
+};
+}  // namespace gpt
+
 struct gpt_step {
   gpt_config cfg;
   std::vector<int32_t> window;
   gpt::Layout layout;
   gpt::Plan plan;
   int64_t last_launches = 0;
+  gpt::Profiler prof;
 };
 
 namespace gpt {
@@ -174,6 +201,39 @@ static Plan make_plan(const gpt_config& c, size_t n_params) {
 // ------------------------------------------------------------------------------------------------
 // the step
 // ------------------------------------------------------------------------------------------------
+// Kernel classes reported by gpt_step_profile.
+enum { PROF_GEMM = 0, PROF_ATTN_FWD, PROF_ATTN_BWD, PROF_NORM, PROF_ROPE, PROF_EMBED, PROF_CE, PROF_N };
+
+// Run `expr` (a launcher returning gpt_status); when profiling, bracket it with CUDA events on
+// the step's stream and record its class and algorithmic FLOPs / bytes.
+#define PROF(cls, fl, by, expr)                                                          \
+  do {                                                                                   \
+    cudaEvent_t e0_ = nullptr, e1_ = nullptr;                                            \
+    if (st->prof.on) {                                                                   \
+      e0_ = st->prof.get();                                                              \
+      e1_ = st->prof.get();                                                              \
+      if (e0_) cudaEventRecord(e0_, s);                                                  \
+    }                                                                                    \
+    GPT_TRY(expr);                                                                       \
+    if (e0_ && e1_) {                                                                    \
+      cudaEventRecord(e1_, s);                                                           \
+      st->prof.recs.push_back({(cls), (double)(fl), (double)(by), e0_, e1_});            \
+    }                                                                                    \
+  } while (0)
+
+static double gemm_flops(double M, double N, double K) { return 2.0 * M * N * K; }
+
+// Σ over query rows of the keys each one attends to (causal band of width w).
+static double attn_pairs(int T, int w) {
+  const double W = (w > 0 && w < T) ? w : T;
+  double full = 0;
+  // rows t < W see t+1 keys, rows t ≥ W see W keys
+  const double a = std::min<double>(W, T);
+  full += a * (a + 1) / 2;
+  full += (T - a) * W;
+  return full;
+}
+
 static gpt_status run_step(gpt_step* st, const void* params, const int32_t* tokens,
                            const int32_t* targets, float* loss, float* grads, uint8_t* ws,
                            cudaStream_t s) {
@@ -187,7 +247,7 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
   GPT_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
   const uint16_t* P = reinterpret_cast<const uint16_t*>(params);
   if (c.param_dtype == GPT_DTYPE_F32) {
-    GPT_TRY(cast_f32_bf16(reinterpret_cast<const float*>(params), ws + p.pshadow, L.total, s));
+    PROF(PROF_CE, 0, 6.0 * L.total, cast_f32_bf16(reinterpret_cast<const float*>(params), ws + p.pshadow, L.total, s));
     P = reinterpret_cast<const uint16_t*>(ws + p.pshadow);
   }
   auto W = [&](int idx) { return P + L.off[idx]; };
@@ -199,8 +259,8 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
   const long long qs_b = (long long)T * 3 * d, qs_h = Dh, qs_t = 3 * d;  // q/k/v inside qkv
   const long long os_b = (long long)T * d, os_h = Dh, os_t = d;          // o / dO
 
-  GPT_TRY(rope_table(rope, T, Dh, s));
-  GPT_TRY(embedding_fwd(tokens, W(0), x, M, d, V, status, s));
+  PROF(PROF_ROPE, 0, (double)T * Dh * 4, rope_table(rope, T, Dh, s));
+  PROF(PROF_EMBED, 0, 4.0 * (double)M * d, embedding_fwd(tokens, W(0), x, M, d, V, status, s));
 
   // ---------------- forward ----------------
   for (int l = 0; l < c.depth; ++l) {
@@ -216,21 +276,21 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
     float* rho2 = reinterpret_cast<float*>(at(p.rho2, l));
     uint16_t* act = reinterpret_cast<uint16_t*>(at(p.act, l));
     uint16_t* hsq = reinterpret_cast<uint16_t*>(at(p.hsq, l));
-    GPT_TRY(rmsnorm_fwd(x, r1, rho1, M, d, s));
-    GPT_TRY(gemm_launch(GPT_GEMM_NT, GPT_EPI_BF16, M, 3 * d, d, r1, d, W(wq), d, qkv, 3 * d,
+    PROF(PROF_NORM, 0, 4.0 * (double)M * d + 4.0 * M, rmsnorm_fwd(x, r1, rho1, M, d, s));
+    PROF(PROF_GEMM, gemm_flops(M, 3.0 * d, d), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_BF16, M, 3 * d, d, r1, d, W(wq), d, qkv, 3 * d,
                         nullptr, nullptr, 0, status, s));
-    GPT_TRY(rope_qknorm_fwd(qkv, rq, rk, rope, B, T, H, Dh, s));
-    GPT_TRY(attention_fwd(qkv, qkv + d, qkv + 2 * d, o, lse, B, H, T, Dh, st->window[l], qs_b,
+    PROF(PROF_ROPE, 0, 8.0 * (double)M * d, rope_qknorm_fwd(qkv, rq, rk, rope, B, T, H, Dh, s));
+    PROF(PROF_ATTN_FWD, 4.0 * Dh * H * B * attn_pairs(T, st->window[l]), 0, attention_fwd(qkv, qkv + d, qkv + 2 * d, o, lse, B, H, T, Dh, st->window[l], qs_b,
                           qs_h, qs_t, os_b, os_h, os_t, status, s));
-    GPT_TRY(gemm_launch(GPT_GEMM_NT, GPT_EPI_RESID, M, d, d, o, d, W(wq + 1), d, x, d, nullptr,
+    PROF(PROF_GEMM, gemm_flops(M, d, d), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_RESID, M, d, d, o, d, W(wq + 1), d, x, d, nullptr,
                         nullptr, 0, status, s));
-    GPT_TRY(rmsnorm_fwd(x, r2, rho2, M, d, s));
-    GPT_TRY(gemm_launch(GPT_GEMM_NT, GPT_EPI_RELU2, M, F, d, r2, d, W(wq + 2), d, act, F, hsq,
+    PROF(PROF_NORM, 0, 4.0 * (double)M * d + 4.0 * M, rmsnorm_fwd(x, r2, rho2, M, d, s));
+    PROF(PROF_GEMM, gemm_flops(M, F, d), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_RELU2, M, F, d, r2, d, W(wq + 2), d, act, F, hsq,
                         nullptr, 0, status, s));
-    GPT_TRY(gemm_launch(GPT_GEMM_NT, GPT_EPI_RESID, M, d, F, hsq, F, W(wq + 3), F, x, d, nullptr,
+    PROF(PROF_GEMM, gemm_flops(M, d, F), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_RESID, M, d, F, hsq, F, W(wq + 3), F, x, d, nullptr,
                         nullptr, 0, status, s));
   }
-  GPT_TRY(rmsnorm_fwd(x, xf, rhof, M, d, s));
+  PROF(PROF_NORM, 0, 4.0 * (double)M * d + 4.0 * M, rmsnorm_fwd(x, xf, rhof, M, d, s));
 
   // ---------------- lm-head + cross-entropy ----------------
   const int wlm = 1 + 4 * c.depth;
@@ -244,25 +304,25 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
   ce.ztarget = reinterpret_cast<float*>(ws + p.zt);
   ce.n_offset = 0;
   ce.stats_col0 = 0;
-  GPT_TRY(gemm_ce_launch(false, M, V, d, xf, d, W(wlm), d, nullptr, 0, ce, status, s));
-  GPT_TRY(ce_rows(ce.stats, tiles, ce.ztarget, targets, M, V, const_cast<float*>(ce.lse),
+  PROF(PROF_GEMM, gemm_flops(M, V, d), 0, gemm_ce_launch(false, M, V, d, xf, d, W(wlm), d, nullptr, 0, ce, status, s));
+  PROF(PROF_CE, 0, (double)M * tiles * 8, ce_rows(ce.stats, tiles, ce.ztarget, targets, M, V, const_cast<float*>(ce.lse),
                   reinterpret_cast<float*>(ws + p.ell), status, s));
-  GPT_TRY(ce_finalize(reinterpret_cast<float*>(ws + p.ell), targets, M, V, loss,
+  PROF(PROF_CE, 0, 8.0 * M, ce_finalize(reinterpret_cast<float*>(ws + p.ell), targets, M, V, loss,
                       const_cast<float*>(ce.inv_n), s));
   uint16_t* dz = reinterpret_cast<uint16_t*>(ws + p.dz);
   float* dxf = reinterpret_cast<float*>(ws + p.dxf);
   for (int c0 = 0; c0 < V; c0 += p.vc) {
     const int n = std::min(p.vc, V - c0);
     ce.n_offset = c0;
-    GPT_TRY(gemm_ce_launch(true, M, n, d, xf, d, W(wlm) + (size_t)c0 * d, d, dz, n, ce, status, s));
-    GPT_TRY(gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, n, d, M, dz, n, xf, d, G(wlm) + (size_t)c0 * d, d,
+    PROF(PROF_GEMM, gemm_flops(M, n, d), 0, gemm_ce_launch(true, M, n, d, xf, d, W(wlm) + (size_t)c0 * d, d, dz, n, ce, status, s));
+    PROF(PROF_GEMM, gemm_flops(n, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, n, d, M, dz, n, xf, d, G(wlm) + (size_t)c0 * d, d,
                         nullptr, nullptr, 0, status, s));
-    GPT_TRY(gemm_launch(GPT_GEMM_NN, c0 == 0 ? GPT_EPI_F32 : GPT_EPI_F32_ADD, M, d, n, dz, n,
+    PROF(PROF_GEMM, gemm_flops(M, d, n), 0, gemm_launch(GPT_GEMM_NN, c0 == 0 ? GPT_EPI_F32 : GPT_EPI_F32_ADD, M, d, n, dz, n,
                         W(wlm) + (size_t)c0 * d, d, dxf, d, nullptr, nullptr, 0, status, s));
   }
   float* gx = reinterpret_cast<float*>(ws + p.gx);
   uint16_t* gxb = reinterpret_cast<uint16_t*>(ws + p.gxb);
-  GPT_TRY(rmsnorm_bwd(dxf, 1, xf, rhof, gx, gxb, 0, M, d, s));
+  PROF(PROF_NORM, 0, 12.0 * (double)M * d, rmsnorm_bwd(dxf, 1, xf, rhof, gx, gxb, 0, M, d, s));
 
   // ---------------- backward ----------------
   uint16_t* du = reinterpret_cast<uint16_t*>(ws + p.du);
@@ -284,31 +344,31 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
     uint16_t* act = reinterpret_cast<uint16_t*>(at(p.act, l));
     uint16_t* hsq = reinterpret_cast<uint16_t*>(at(p.hsq, l));
     // MLP
-    GPT_TRY(gemm_launch(GPT_GEMM_NN, GPT_EPI_DRELU2, M, F, d, gxb, d, W(wq + 3), F, du, F, nullptr,
+    PROF(PROF_GEMM, gemm_flops(M, F, d), 0, gemm_launch(GPT_GEMM_NN, GPT_EPI_DRELU2, M, F, d, gxb, d, W(wq + 3), F, du, F, nullptr,
                         act, F, status, s));
-    GPT_TRY(gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, d, F, M, gxb, d, hsq, F, G(wq + 3), F, nullptr,
+    PROF(PROF_GEMM, gemm_flops(d, F, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, d, F, M, gxb, d, hsq, F, G(wq + 3), F, nullptr,
                         nullptr, 0, status, s));
-    GPT_TRY(gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, F, d, M, du, F, r2, d, G(wq + 2), d, nullptr,
+    PROF(PROF_GEMM, gemm_flops(F, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, F, d, M, du, F, r2, d, G(wq + 2), d, nullptr,
                         nullptr, 0, status, s));
-    GPT_TRY(gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, F, du, F, W(wq + 2), d, dr, d, nullptr,
+    PROF(PROF_GEMM, gemm_flops(M, d, F), 0, gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, F, du, F, W(wq + 2), d, dr, d, nullptr,
                         nullptr, 0, status, s));
-    GPT_TRY(rmsnorm_bwd(dr, 0, r2, rho2, gx, gxb, 1, M, d, s));
+    PROF(PROF_NORM, 0, 14.0 * (double)M * d, rmsnorm_bwd(dr, 0, r2, rho2, gx, gxb, 1, M, d, s));
     // attention
-    GPT_TRY(gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, d, gxb, d, W(wq + 1), d, dO, d, nullptr,
+    PROF(PROF_GEMM, gemm_flops(M, d, d), 0, gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, d, gxb, d, W(wq + 1), d, dO, d, nullptr,
                         nullptr, 0, status, s));
-    GPT_TRY(gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, d, d, M, gxb, d, o, d, G(wq + 1), d, nullptr,
+    PROF(PROF_GEMM, gemm_flops(d, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, d, d, M, gxb, d, o, d, G(wq + 1), d, nullptr,
                         nullptr, 0, status, s));
-    GPT_TRY(attention_bwd(qkv, qkv + d, qkv + 2 * d, o, dO, lse, delta, dqkv, dqkv + d,
+    PROF(PROF_ATTN_BWD, 8.0 * Dh * H * B * attn_pairs(T, st->window[l]), 0, attention_bwd(qkv, qkv + d, qkv + 2 * d, o, dO, lse, delta, dqkv, dqkv + d,
                           dqkv + 2 * d, B, H, T, Dh, st->window[l], qs_b, qs_h, qs_t, os_b, os_h,
                           os_t, status, s));
-    GPT_TRY(rope_qknorm_bwd(dqkv, qkv, rq, rk, rope, B, T, H, Dh, s));
-    GPT_TRY(gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, 3 * d, d, M, dqkv, 3 * d, r1, d, G(wq), d,
+    PROF(PROF_ROPE, 0, 12.0 * (double)M * d, rope_qknorm_bwd(dqkv, qkv, rq, rk, rope, B, T, H, Dh, s));
+    PROF(PROF_GEMM, gemm_flops(3.0 * d, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, 3 * d, d, M, dqkv, 3 * d, r1, d, G(wq), d,
                         nullptr, nullptr, 0, status, s));
-    GPT_TRY(gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, 3 * d, dqkv, 3 * d, W(wq), d, dr, d,
+    PROF(PROF_GEMM, gemm_flops(M, d, 3.0 * d), 0, gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, 3 * d, dqkv, 3 * d, W(wq), d, dr, d,
                         nullptr, nullptr, 0, status, s));
-    GPT_TRY(rmsnorm_bwd(dr, 0, r1, rho1, gx, gxb, 1, M, d, s));
+    PROF(PROF_NORM, 0, 14.0 * (double)M * d, rmsnorm_bwd(dr, 0, r1, rho1, gx, gxb, 1, M, d, s));
   }
-  GPT_TRY(embedding_bwd(tokens, gx, G(0), M, d, V, ws + p.emb, s));
+  PROF(PROF_EMBED, 0, 4.0 * (double)M * d + 8.0 * V * d, embedding_bwd(tokens, gx, G(0), M, d, V, ws + p.emb, s));
   return GPT_OK;
 }
 
@@ -357,6 +417,41 @@ gpt_status gpt_step_workspace_bytes(const gpt_step* step, size_t* bytes) {
 }
 
 int64_t gpt_step_last_launch_count(const gpt_step* step) { return step ? step->last_launches : -1; }
+
+gpt_status gpt_step_set_profiling(gpt_step* step, int enable) {
+  if (!step) return GPT_ERR_INVALID_ARG;
+  step->prof.on = enable != 0;
+  return GPT_OK;
+}
+
+gpt_status gpt_step_profile(gpt_step* step, double* ms, int64_t* calls, double* flops, double* bytes,
+                            int n_classes) {
+  if (!step || n_classes <= 0) return GPT_ERR_INVALID_ARG;
+  for (int c = 0; c < n_classes; ++c) {
+    if (ms) ms[c] = 0;
+    if (calls) calls[c] = 0;
+    if (flops) flops[c] = 0;
+    if (bytes) bytes[c] = 0;
+  }
+  gpt::Profiler& P = step->prof;
+  gpt_status r = GPT_OK;
+  for (const auto& rec : P.recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(rec.b) != cudaSuccess || cudaEventElapsedTime(&t, rec.a, rec.b) != cudaSuccess) {
+      r = GPT_ERR_CUDA;
+      continue;
+    }
+    if (rec.cls < n_classes) {
+      if (ms) ms[rec.cls] += t;
+      if (calls) calls[rec.cls] += 1;
+      if (flops) flops[rec.cls] += rec.flops;
+      if (bytes) bytes[rec.cls] += rec.bytes;
+    }
+  }
+  P.recs.clear();
+  P.used = 0;
+  return r;
+}
 
 gpt_status gpt_step_fwd_bwd(gpt_step* step, const void* params, const int32_t* tokens,
                             const int32_t* targets, float* loss, float* grads, void* workspace,

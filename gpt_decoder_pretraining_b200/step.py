@@ -23,11 +23,13 @@ STATUS_NAMES = {0: "GPT_OK", -1: "GPT_ERR_INVALID_ARG", -2: "GPT_ERR_UNSUPPORTED
                 -3: "GPT_ERR_WORKSPACE_TOO_SMALL", -4: "GPT_ERR_CUDA", -5: "GPT_ERR_DEVICE_TIMEOUT",
                 -6: "GPT_ERR_TOKEN_OUT_OF_RANGE", -7: "GPT_ERR_NO_DEVICE"}
 GEMM_NT, GEMM_NN, GEMM_TN = 0, 1, 2
+PROFILE_CLASSES = ("gemm", "attn_fwd", "attn_bwd", "rmsnorm", "rope_qknorm", "embedding", "ce_reduce")
 EPI_BF16, EPI_RESID, EPI_RELU2, EPI_DRELU2, EPI_F32, EPI_F32_ADD = 0, 1, 2, 3, 4, 5
 
 EXPORTED = [
     "gpt_param_layout", "gpt_step_create", "gpt_step_destroy", "gpt_step_workspace_bytes",
     "gpt_step_fwd_bwd", "gpt_step_status", "gpt_strerror", "gpt_step_last_launch_count",
+    "gpt_step_set_profiling", "gpt_step_profile",
     "gpt_gemm", "gpt_rmsnorm_fwd", "gpt_rmsnorm_bwd", "gpt_rope_qknorm_fwd", "gpt_rope_qknorm_bwd",
     "gpt_rope_table", "gpt_attention_fwd", "gpt_attention_bwd", "gpt_embedding_fwd",
     "gpt_embedding_bwd_scratch_bytes", "gpt_embedding_bwd", "gpt_lmhead_ce_scratch_bytes",
@@ -69,6 +71,9 @@ def lib():
         L.gpt_strerror.restype = ctypes.c_char_p
         L.gpt_step_last_launch_count.argtypes = [vp]
         L.gpt_step_last_launch_count.restype = ctypes.c_int64
+        L.gpt_step_set_profiling.argtypes = [vp, i32]
+        L.gpt_step_profile.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64),
+                                       ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double), i32]
         L.gpt_gemm.argtypes = [i32, i32, i32, i32, i32, vp, i32, vp, i32, vp, i32, vp, vp, i32, vp, vp]
         L.gpt_rmsnorm_fwd.argtypes = [vp, vp, vp, i32, i32, vp]
         L.gpt_rmsnorm_bwd.argtypes = [vp, i32, vp, vp, vp, vp, i32, i32, i32, vp]
@@ -167,6 +172,19 @@ class GptStep:
 
     def last_launch_count(self) -> int:
         return int(lib().gpt_step_last_launch_count(self._h))
+
+    def set_profiling(self, on: bool):
+        _check(lib().gpt_step_set_profiling(self._h, int(bool(on))), "gpt_step_set_profiling")
+
+    def profile(self):
+        """{class: (ms, calls, flops, bytes)} accumulated since the last read (see gpt_step_profile)."""
+        n = len(PROFILE_CLASSES)
+        ms = (ctypes.c_double * n)()
+        calls = (ctypes.c_int64 * n)()
+        fl = (ctypes.c_double * n)()
+        by = (ctypes.c_double * n)()
+        _check(lib().gpt_step_profile(self._h, ms, calls, fl, by, n), "gpt_step_profile")
+        return {c: (ms[i], int(calls[i]), fl[i], by[i]) for i, c in enumerate(PROFILE_CLASSES)}
 
 
 # ------------------------------------------------------------------------------------------------

@@ -101,6 +101,18 @@ const char* gpt_strerror(int status);
 /* Number of kernel launches the last gpt_step_fwd_bwd enqueued (host counter, for reporting). */
 int64_t gpt_step_last_launch_count(const gpt_step* step);
 
+/* Per-kernel-class timing.  While enabled, every launcher call of gpt_step_fwd_bwd is bracketed
+ * by two CUDA events recorded on the step's stream.  gpt_step_profile waits for those events and
+ * returns, for each class c < n_classes, the summed milliseconds, number of calls, algorithmic
+ * FLOPs (2·M·N·K per GEMM; 4·Dh per visible query-key pair for attention forward, twice that
+ * backward) and algorithmic bytes (memory-bound kernels), then clears the record.  Classes:
+ * 0 GEMM (all projections, MLP and lm-head GEMMs), 1 attention forward, 2 attention backward,
+ * 3 RMSNorm, 4 RoPE + QK-norm, 5 embedding, 6 cross-entropy reductions and parameter cast.
+ * Any output pointer may be NULL. */
+gpt_status gpt_step_set_profiling(gpt_step* step, int enable);
+gpt_status gpt_step_profile(gpt_step* step, double* ms, int64_t* calls, double* flops,
+                            double* bytes, int n_classes);
+
 /* ---------------------------------------------------------------------------------------------
  * Kernel-level entry points.  The step is built from these; they are exported for unit parity
  * tests and for the attention-only workload.  `status` (device int, may be NULL) receives a
