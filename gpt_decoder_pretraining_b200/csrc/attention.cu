@@ -14,6 +14,7 @@
 //               bitwise reproducible.
 
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "host.h"
@@ -741,6 +742,44 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   return GPT_OK;
 }
 
+// ------------------------------------------------------------------------------------------------
+// Allocation-free attention backward: the per-row delta = rowsum(dO∘O) lives in this fixed array
+// instead of a caller-supplied buffer.  Every GPU that loads the library holds it until exit.
+// ------------------------------------------------------------------------------------------------
+constexpr long long NOALLOC_DELTA_ROWS = GPT_ATTN_BWD_NOALLOC_MAX_ROWS;
+static __device__ __align__(256) float g_noalloc_delta[NOALLOC_DELTA_ROWS];
+
+// Device address of g_noalloc_delta on the current device, looked up once per device with that
+// device current.  In host code the symbol itself is only a host-side stand-in for the array.
+static gpt_status noalloc_delta_ptr(float** out) {
+  static std::mutex mu;
+  static float* cached[64] = {nullptr};
+  int dev = 0;
+  GPT_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return GPT_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cached[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_delta) != cudaSuccess || p == nullptr) return GPT_ERR_CUDA;
+    cached[dev] = static_cast<float*>(p);
+  }
+  *out = cached[dev];
+  return GPT_OK;
+}
+
+gpt_status attention_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                 const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                 int B, int H, int T, int Dh, int window, long long sbq,
+                                 long long shq, long long stq, long long sbo, long long sho,
+                                 long long sto, int* status, cudaStream_t stream) {
+  if (B <= 0 || H <= 0 || T <= 0) return GPT_ERR_INVALID_ARG;
+  if ((long long)B * H * T > NOALLOC_DELTA_ROWS) return GPT_ERR_UNSUPPORTED_SHAPE;
+  float* delta = nullptr;
+  GPT_TRY(noalloc_delta_ptr(&delta));
+  return attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, T, Dh, window, sbq, shq, stq,
+                       sbo, sho, sto, status, stream);
+}
+
 }  // namespace gpt
 
 extern "C" gpt_status gpt_attention_fwd(const void* q, const void* k, const void* v, void* o,
@@ -760,4 +799,16 @@ extern "C" gpt_status gpt_attention_bwd(const void* q, const void* k, const void
                                         long long st_o, int* status, void* stream) {
   return gpt::attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, T, Dh, window, sb_qkv,
                             sh_qkv, st_qkv, sb_o, sh_o, st_o, status, gpt::as_stream(stream));
+}
+
+extern "C" gpt_status gpt_attention_bwd_noalloc(const void* q, const void* k, const void* v,
+                                                const void* o, const void* dout, const float* lse,
+                                                void* dq, void* dk, void* dv, int B, int H, int T,
+                                                int Dh, int window, long long sb_qkv,
+                                                long long sh_qkv, long long st_qkv, long long sb_o,
+                                                long long sh_o, long long st_o, int* status,
+                                                void* stream) {
+  return gpt::attention_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, T, Dh, window, sb_qkv,
+                                    sh_qkv, st_qkv, sb_o, sh_o, st_o, status,
+                                    gpt::as_stream(stream));
 }

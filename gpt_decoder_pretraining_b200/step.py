@@ -31,7 +31,8 @@ EXPORTED = [
     "gpt_step_fwd_bwd", "gpt_step_status", "gpt_strerror", "gpt_step_last_launch_count",
     "gpt_step_set_profiling", "gpt_step_profile",
     "gpt_gemm", "gpt_rmsnorm_fwd", "gpt_rmsnorm_bwd", "gpt_rope_qknorm_fwd", "gpt_rope_qknorm_bwd",
-    "gpt_rope_table", "gpt_attention_fwd", "gpt_attention_bwd", "gpt_embedding_fwd",
+    "gpt_rope_table", "gpt_attention_fwd", "gpt_attention_bwd", "gpt_attention_bwd_noalloc",
+    "gpt_embedding_fwd",
     "gpt_embedding_bwd_scratch_bytes", "gpt_embedding_bwd", "gpt_lmhead_ce_scratch_bytes",
     "gpt_lmhead_ce_fwd_bwd",
 ]
@@ -83,6 +84,8 @@ def lib():
         L.gpt_attention_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, ll, ll, ll, ll, ll, ll, vp, vp]
         L.gpt_attention_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                         ll, ll, ll, ll, ll, ll, vp, vp]
+        L.gpt_attention_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                                ll, ll, ll, ll, ll, ll, vp, vp]
         L.gpt_embedding_fwd.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp]
         L.gpt_embedding_bwd_scratch_bytes.argtypes = [i32, i32]
         L.gpt_embedding_bwd_scratch_bytes.restype = sz
@@ -239,6 +242,15 @@ def attention_bwd(q, k, v, o, do, lse, delta, dq, dk, dv, window: int, strides_q
                                    lse.data_ptr(), delta.data_ptr(), dq.data_ptr(), dk.data_ptr(),
                                    dv.data_ptr(), B, H, T, Dh, window, *strides_qkv, *strides_o,
                                    _ptr(status), _stream()), "attention_bwd")
+
+
+def attention_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, window: int, strides_qkv, strides_o, B, H, T,
+                          Dh, status=None):
+    """gpt_attention_bwd_noalloc: the attention backward with its scratch held inside the library."""
+    _check(lib().gpt_attention_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                           do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                           dv.data_ptr(), B, H, T, Dh, window, *strides_qkv, *strides_o,
+                                           _ptr(status), _stream()), "attention_bwd_noalloc")
 
 
 def embedding_fwd(tokens, wte, x, status=None):

@@ -177,6 +177,29 @@ gpt_status gpt_attention_bwd(const void* q, const void* k, const void* v, const 
                              long long sh_qkv, long long st_qkv, long long sb_o, long long sh_o,
                              long long st_o, int* status, void* stream);
 
+/* Attention backward that allocates nothing.  The pages have no counterpart: this is a calling
+ * convenience, not part of the method.  Arguments and results are those of gpt_attention_bwd
+ * without `delta`; the per-row rowsum(dO∘O) that the backward needs is kept in a static device
+ * array inside this library (GPT_ATTN_BWD_NOALLOC_MAX_ROWS fp32 values = 8 MiB), which every GPU
+ * that loads the library holds until the process exits.
+ * It serves callers that cannot obtain device memory where they call the backward — for example
+ * code running under a device-memory budget fixed at start-up, or inside a host framework whose own
+ * allocator owns all device memory and allows no side allocations — and therefore cannot hand
+ * gpt_attention_bwd its scratch buffer.  It calls no cudaMalloc, cudaFree or allocating routine.
+ *   - B·H·T > GPT_ATTN_BWD_NOALLOC_MAX_ROWS returns GPT_ERR_UNSUPPORTED_SHAPE; nothing is enqueued.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the one array.  Each call writes the rows it uses before reading them, so
+ *     nothing needs clearing, but calls that overlap on the GPU (unordered streams, several host
+ *     threads) race on it and give wrong results: order them on one stream. */
+#define GPT_ATTN_BWD_NOALLOC_MAX_ROWS (1ll << 21)
+gpt_status gpt_attention_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                     const void* dout, const float* lse, void* dq, void* dk,
+                                     void* dv, int B, int H, int T, int Dh, int window,
+                                     long long sb_qkv, long long sh_qkv, long long st_qkv,
+                                     long long sb_o, long long sh_o, long long st_o, int* status,
+                                     void* stream);
+
 /* Embedding gather x[m] = wte[tok[m]] (bf16 rows of d).  Ids outside [0, V) are clamped and
  * flagged in *status. */
 gpt_status gpt_embedding_fwd(const int32_t* tokens, const void* wte, void* x, int M, int d, int V,
