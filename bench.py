@@ -325,6 +325,70 @@ def run_ours(args, cfg):
     return 0
 
 
+# ------------------------------------------------------------------------------------------------
+# single-kernel workloads (GEMM shapes of the step; the causal-attention sweep)
+# ------------------------------------------------------------------------------------------------
+def run_kernel(args):
+    """Time one kernel-level call through the C ABI; prints one JSON line (not the step metric)."""
+    import torch
+    from gpt_decoder_pretraining_b200 import step as S
+    from gpt_decoder_pretraining_b200.inputs import make_attention_inputs
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    peaks, src = load_peaks()
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    if args.kernel == "gemm":
+        M, N, K = (int(x) for x in args.gemm_shape.split(","))
+        op = {"nt": 0, "nn": 1, "tn": 2}[args.gemm_op]
+        a_shape = (K, M) if op == 2 else (M, K)
+        b_shape = (N, K) if op == 0 else (K, N)
+        A = torch.randn(a_shape, device=dev, generator=g).to(torch.bfloat16)
+        B = torch.randn(b_shape, device=dev, generator=g).to(torch.bfloat16)
+        C = torch.empty(M, N, device=dev, dtype=torch.float32 if op == 2 else torch.bfloat16)
+        epi = S.EPI_F32 if op == 2 else S.EPI_BF16
+        run = lambda: S.gemm(op, epi, A, B, C, M, N, K)  # noqa: E731
+        flops = 2.0 * M * N * K
+        unit_desc = f"GEMM {args.gemm_op} M={M} N={N} K={K}"
+    else:
+        T, Dh, W = (int(x) for x in args.attn.split(","))
+        H = 8
+        Bt = max(1, (1 << 21) // (H * T))
+        q, k, v, do = (torch.from_numpy(a).to(dev).to(torch.bfloat16)
+                       for a in make_attention_inputs(Bt, H, T, Dh))
+        o = torch.empty_like(q)
+        lse = torch.empty(Bt, H, T, device=dev)
+        strides = (H * T * Dh, T * Dh, Dh)
+        dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+        delta = torch.empty(Bt, H, T, device=dev)
+        Wf = W if 0 < W < T else T
+        pairs = Wf * (Wf + 1) / 2 + (T - Wf) * Wf
+        if args.attn_pass == "fwd":
+            run = lambda: S.attention_fwd(q, k, v, o, lse, W, strides, strides, Bt, H, T, Dh)  # noqa: E731
+            flops = 4.0 * Dh * pairs * H * Bt
+        else:
+            S.attention_fwd(q, k, v, o, lse, W, strides, strides, Bt, H, T, Dh)
+            run = lambda: S.attention_bwd(q, k, v, o, do, lse, delta, dq, dk, dv, W, strides, strides,  # noqa: E731
+                                          Bt, H, T, Dh)
+            flops = 8.0 * Dh * pairs * H * Bt
+        unit_desc = f"causal attention {args.attn_pass} B={Bt} H={H} T={T} Dh={Dh} window={W or 'full'}"
+    for _ in range(max(3, args.warmup)):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    tf = flops / (ms / 1e3) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    print(json.dumps({"kernel": unit_desc, "ms": ms, "tflops": tf, "peak_burst_tflops": peak,
+                      "frac_of_burst": tf / peak, "peak_source": src, "steps": args.steps}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -334,9 +398,17 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-sample-tokens", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=["gemm", "attention"], default=None,
+                    help="time one kernel-level workload instead of the step")
+    ap.add_argument("--gemm-shape", default="32768,6144,1536")
+    ap.add_argument("--gemm-op", default="nt", choices=["nt", "nn", "tn"])
+    ap.add_argument("--attn", default="2048,128,0", help="T,Dh,window (window 0 = full causal)")
+    ap.add_argument("--attn-pass", default="fwd", choices=["fwd", "bwd"])
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.kernel:
+        return run_kernel(args)
     cfg = preset(args.config)
     if args.impl == "reference":
         return run_reference(args, cfg)

@@ -266,6 +266,291 @@ __global__ void __launch_bounds__(256)
 }
 
 // ================================================================================================
+// forward on the tcgen05 tensor cores (head_dim 64 or 128)
+//
+// One CTA owns two 128-row query tiles (a, b) of one (batch, head) and streams 128-key K/V tiles
+// through a two-stage TMA ring.  Warp roles:
+//   warps 0-3 / 4-7   softmax of tile a / tile b: each thread owns one query row (= TMEM lane)
+//   warp 8            TMA producer
+//   warp 9            MMA issuer: S_x = Q_x·K_jᵀ (A, B from shared memory) into tensor memory,
+//                     O_x += P_x·V_j with P read from tensor memory (written there by softmax)
+// Tensor memory: S_a | S_b (128 columns each; P_x overwrites the first 64 columns of S_x as packed
+// bf16 pairs) | O_a | O_b (Dh columns each).  The MMA warp orders its work as
+//   S_a(0) S_b(0) | PV_a(0) S_a(1) PV_b(0) S_b(1) | PV_a(1) S_a(2) ...
+// so the softmax of one tile overlaps the MMAs of the other.
+//
+// Softmax shift: each row uses the fixed bound c_t = ‖q_t‖·max_j‖k_j‖/√Dh ≥ every score of the
+// row (Cauchy–Schwarz) instead of a running maximum.  softmax is invariant to the shift, so
+//   p = exp(s − c_t),  l = Σ p,  O = (Σ p·v)/l,  LSE = c_t + ln l
+// is the exact softmax; p ∈ [e^{−2c_t}, 1] cannot overflow and, for c_t ≤ 40, cannot underflow.
+// With a fixed shift O never needs rescaling inside tensor memory.
+// ================================================================================================
+template <int DH>
+struct TcFwdShape {
+  static constexpr int BQ = 128, BK = 128;
+  static constexpr int Q_TILE = BQ * DH * 2;
+  static constexpr int KV_TILE = BK * DH * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = 2 * Q_TILE;
+  static constexpr int OFF_V = OFF_K + 2 * KV_TILE;
+  static constexpr int OFF_BAR = OFF_V + 2 * KV_TILE;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int THREADS = 320;
+  static constexpr int TM_S = 0;    // S_x at x·128
+  static constexpr int TM_O = 256;  // O_x at 256 + x·DH
+};
+
+// Row of the [DH/64][128][64] swizzled Q tile as fp32 sum of squares.
+template <int DH>
+__device__ __forceinline__ float q_row_sumsq(const uint8_t* tile, int r) {
+  float ss = 0.f;
+#pragma unroll
+  for (int c = 0; c < DH / 64; ++c) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint4 v = *reinterpret_cast<const uint4*>(tile + c * 128 * 128 + r * 128 + ((u ^ (r & 7)) << 4));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ss += bf_lo(w[e]) * bf_lo(w[e]) + bf_hi(w[e]) * bf_hi(w[e]);
+    }
+  }
+  return ss;
+}
+
+template <int DH>
+__global__ void __launch_bounds__(320, 1)
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                       const __grid_constant__ CUtensorMap mv, const AttnArgs a, const float* kmax,
+                       float kmax_const) {
+  using S = TcFwdShape<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
+  uint64_t* bar_q = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = bars + 3;
+  uint64_t* s_full = bars + 5;
+  uint64_t* p_full = bars + 7;
+  uint64_t* o_full = bars + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int qt = gridDim.x - 1 - blockIdx.x;  // longest rows first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int T = a.T, W = a.window;
+  const int q0 = qt * 256;
+  const int key_lo = max(0, q0 - W + 1);
+  const int key_hi = min(T, q0 + 256);
+  const int kv_first = key_lo / 128;
+  const int n_kv = (key_hi - 1) / 128 - kv_first + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+    }
+    mbar_init(o_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_q, 2 * S::Q_TILE);
+      load_tile<DH, 128>(smem + S::OFF_Q, &mq, bar_q, q0, h, b);
+      load_tile<DH, 128>(smem + S::OFF_Q + S::Q_TILE, &mq, bar_q, q0 + 128, h, b);
+      for (int j = 0; j < n_kv; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1, abort_flag, a.status)) break;
+        mbar_arrive_expect_tx(&kv_full[st], 2 * S::KV_TILE);
+        const int k0 = (kv_first + j) * 128;
+        load_tile<DH, 128>(smem + S::OFF_K + st * S::KV_TILE, &mk, &kv_full[st], k0, h, b);
+        load_tile<DH, 128>(smem + S::OFF_V + st * S::KV_TILE, &mv, &kv_full[st], k0, h, b);
+      }
+    }
+  } else if (warp == 9) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t id_o = idesc_bf16(128, DH, false, true);
+      const uint32_t qa = smem_u32(smem + S::OFF_Q);
+      const uint32_t kb0 = smem_u32(smem + S::OFF_K);
+      const uint32_t vb0 = smem_u32(smem + S::OFF_V);
+      auto issue_s = [&](int x, int j) {
+        const uint32_t q_base = qa + x * S::Q_TILE;
+        const uint32_t k_base = kb0 + (j & 1) * S::KV_TILE;
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_bf16_ss(tmem + S::TM_S + x * 128, sdesc_sw128(q_base + off, 16, 1024),
+                      sdesc_sw128(k_base + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_full[x]);
+      };
+      auto issue_pv = [&](int x, int j) {
+        const uint32_t v_base = vb0 + (j & 1) * S::KV_TILE;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + S::TM_O + x * DH, tmem + S::TM_S + x * 128 + kk * 8,
+                      sdesc_sw128(v_base + kk * 2048, 128 * 128, 1024), id_o,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(bar_q, 0, abort_flag, a.status);
+      if (ok) ok = mbar_wait(&kv_full[0], 0, abort_flag, a.status);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+      }
+      for (int j = 0; j < n_kv && ok; ++j) {
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (!mbar_wait(&p_full[x], j & 1, abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(x, j);
+          if (x == 1) tc_commit(&kv_empty[j & 1]);
+          if (j + 1 < n_kv) {
+            if (x == 0) {
+              if (!mbar_wait(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag, a.status)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            issue_s(x, j + 1);
+          }
+        }
+      }
+      tc_commit(o_full);
+    }
+  } else {
+    // ---------------- softmax warpgroups ----------------
+    const int x = warp >> 2;
+    const int quarter = warp & 3;
+    const int row = 32 * quarter + lane;
+    const int t = q0 + 128 * x + row;
+    const int tile0 = q0 + 128 * x;
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    const uint32_t s_addr = tmem + lane_off + S::TM_S + x * 128;
+    bool ok = mbar_wait(bar_q, 0, abort_flag, a.status);
+    // fixed shift c_t (log2 units)
+    const float qn = sqrtf(q_row_sumsq<DH>(smem + S::OFF_Q + x * S::Q_TILE, row));
+    const float km = kmax ? kmax[(long long)b * a.H + h] : kmax_const;
+    const float c_nat = qn * km * a.scale * 1.001f + 1e-3f;
+    if (c_nat > 40.f && t < T) set_status(a.status, GPT_ERR_NUMERIC_RANGE);
+    const float c2 = c_nat * LOG2E;
+    // l: exact sum of the weights (gives the LSE the backward pass needs); lb: sum of the bf16
+    // weights that P·V actually uses, so that O = Σ P·v / lb is a convex combination of the v rows
+    float l = 0.f, lb = 0.f;
+    for (int j = 0; j < n_kv && ok; ++j) {
+      if (!mbar_wait(&s_full[x], j & 1, abort_flag, a.status)) { ok = false; break; }
+      tc_fence_after();
+      const int kv0 = (kv_first + j) * 128;
+      const bool need_mask = (kv0 + 127 > tile0) || (kv0 <= tile0 + 127 - W);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(s_addr + 32 * c, r);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float p0 = exp2f(fmaf(__uint_as_float(r[2 * e]), a.scale_log2, -c2));
+          float p1 = exp2f(fmaf(__uint_as_float(r[2 * e + 1]), a.scale_log2, -c2));
+          if (need_mask) {
+            const int key = kv0 + 32 * c + 2 * e;
+            if (!(key <= t && key > t - W)) p0 = 0.f;
+            if (!(key + 1 <= t && key + 1 > t - W)) p1 = 0.f;
+          }
+          l += p0 + p1;
+          pk[e] = pack_bf2(p0, p1);
+          lb += bf_lo(pk[e]) + bf_hi(pk[e]);
+        }
+        tmem_st16(s_addr + 16 * c, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[x]);
+    }
+    // epilogue: O / l
+    if (ok) ok = mbar_wait(o_full, 0, abort_flag, a.status);
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.f / lb;
+      uint16_t* orow = a.o + b * a.sb_o + h * a.sh_o + (long long)t * a.st_o;
+#pragma unroll 1
+      for (int c = 0; c < DH / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + S::TM_O + x * DH + 32 * c, r);
+        tmem_ld_wait();
+        if (t < T) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 w;
+            w.x = pack_bf2(__uint_as_float(r[8 * u + 0]) * inv, __uint_as_float(r[8 * u + 1]) * inv);
+            w.y = pack_bf2(__uint_as_float(r[8 * u + 2]) * inv, __uint_as_float(r[8 * u + 3]) * inv);
+            w.z = pack_bf2(__uint_as_float(r[8 * u + 4]) * inv, __uint_as_float(r[8 * u + 5]) * inv);
+            w.w = pack_bf2(__uint_as_float(r[8 * u + 6]) * inv, __uint_as_float(r[8 * u + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + 32 * c + 8 * u) = w;
+          }
+        }
+      }
+      if (t < T) a.lse[((long long)b * a.H + h) * T + t] = (c2 + log2f(l)) * LN2;
+    }
+  }
+
+  __syncwarp();
+  if (*abort_flag && threadIdx.x == 0) {
+    for (int i = 0; i < 2000; ++i) __nanosleep(1000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+// max_t ‖k_t‖ for each (batch, head): one CTA per (h, b).
+__global__ void attn_kmax_kernel(const uint16_t* __restrict__ k, float* __restrict__ kmax, int H,
+                                 int T, int Dh, long long sb, long long sh, long long st) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  const uint16_t* base = k + b * sb + h * sh;
+  float m = 0.f;
+  for (int t = threadIdx.x; t < T; t += blockDim.x) {
+    const uint4* row = reinterpret_cast<const uint4*>(base + (long long)t * st);
+    float ss = 0.f;
+    for (int u = 0; u < Dh / 8; ++u) {
+      const uint4 v = row[u];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ss += bf_lo(w[e]) * bf_lo(w[e]) + bf_hi(w[e]) * bf_hi(w[e]);
+    }
+    m = fmaxf(m, ss);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float red[32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float r = 0.f;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) r = fmaxf(r, red[i]);
+    kmax[(long long)b * H + h] = sqrtf(r);
+  }
+}
+
+// ================================================================================================
 // backward (1): delta = rowsum(dO ∘ O), one warp per row
 // ================================================================================================
 __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
@@ -643,6 +928,19 @@ gpt_status launch_fwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, c
 }
 
 template <int DH>
+gpt_status launch_fwd_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const AttnArgs& a, const float* kmax, float kmax_const, cudaStream_t stream) {
+  using S = TcFwdShape<DH>;
+  static bool once = false;
+  if (!once) { GPT_TRY(set_smem(attn_fwd_tc_kernel<DH>, S::SMEM)); once = true; }
+  dim3 grid((a.T + 255) / 256, a.H, a.B);
+  attn_fwd_tc_kernel<DH><<<grid, S::THREADS, S::SMEM, stream>>>(mq, mk, mv, a, kmax, kmax_const);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
+template <int DH>
 gpt_status launch_bwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const CUtensorMap& mdo, AttnArgs a, void* dq, cudaStream_t stream) {
   constexpr int smem = BwdShape<DH>::SMEM;
@@ -664,10 +962,12 @@ gpt_status launch_bwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, c
 
 }  // namespace
 
+// kmax_scratch: B·H floats for max_t ‖k_t‖, or nullptr when every k row is RMS-normalised over
+// Dh (QK-norm), in which case ‖k‖ ≤ √Dh·(1 + 2⁻⁹) after bf16 rounding bounds it.
 gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                          int H, int T, int Dh, int window, long long sbq, long long shq,
                          long long stq, long long sbo, long long sho, long long sto, int* status,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, float* kmax_scratch) {
   GPT_TRY(check_attn(q, B, H, T, Dh, sbq, shq, stq));
   GPT_TRY(check_attn(k, B, H, T, Dh, sbq, shq, stq));
   GPT_TRY(check_attn(v, B, H, T, Dh, sbq, shq, stq));
@@ -687,11 +987,24 @@ gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, f
   a.sb_o = sbo; a.sh_o = sho; a.st_o = sto;
   a.lse = lse;
   a.status = status;
-  dim3 grid((T + 127) / 128, H, B);
-  if (Dh == 128) GPT_TRY(launch_fwd<128>(grid, mq, mk, mv, a, stream));
-  else if (Dh == 64) GPT_TRY(launch_fwd<64>(grid, mq, mk, mv, a, stream));
-  else GPT_TRY(launch_fwd<32>(grid, mq, mk, mv, a, stream));
-  return GPT_OK;
+  if (Dh == 32) {
+    dim3 grid((T + 127) / 128, H, B);
+    return launch_fwd<32>(grid, mq, mk, mv, a, stream);
+  }
+  CUtensorMap mq2, mk2, mv2;
+  if (!make_head_map(&mq2, q, B, H, T, Dh, sbq, shq, stq, 128) ||
+      !make_head_map(&mk2, k, B, H, T, Dh, sbq, shq, stq, 128) ||
+      !make_head_map(&mv2, v, B, H, T, Dh, sbq, shq, stq, 128))
+    return GPT_ERR_UNSUPPORTED_SHAPE;
+  const float kconst = sqrtf((float)Dh) * 1.002f;
+  if (kmax_scratch) {
+    attn_kmax_kernel<<<dim3(H, B), 256, 0, stream>>>(reinterpret_cast<const uint16_t*>(k),
+                                                    kmax_scratch, H, T, Dh, sbq, shq, stq);
+    count_launch();
+    GPT_CUDA_TRY(cudaGetLastError());
+  }
+  if (Dh == 128) return launch_fwd_tc<128>(mq2, mk2, mv2, a, kmax_scratch, kconst, stream);
+  return launch_fwd_tc<64>(mq2, mk2, mv2, a, kmax_scratch, kconst, stream);
 }
 
 gpt_status attention_bwd(const void* q, const void* k, const void* v, const void* o,
@@ -783,12 +1096,12 @@ gpt_status attention_bwd_noalloc(const void* q, const void* k, const void* v, co
 }  // namespace gpt
 
 extern "C" gpt_status gpt_attention_fwd(const void* q, const void* k, const void* v, void* o,
-                                        float* lse, int B, int H, int T, int Dh, int window,
-                                        long long sb_qkv, long long sh_qkv, long long st_qkv,
-                                        long long sb_o, long long sh_o, long long st_o,
-                                        int* status, void* stream) {
+                                        float* lse, float* kmax, int B, int H, int T, int Dh,
+                                        int window, long long sb_qkv, long long sh_qkv,
+                                        long long st_qkv, long long sb_o, long long sh_o,
+                                        long long st_o, int* status, void* stream) {
   return gpt::attention_fwd(q, k, v, o, lse, B, H, T, Dh, window, sb_qkv, sh_qkv, st_qkv, sb_o,
-                            sh_o, st_o, status, gpt::as_stream(stream));
+                            sh_o, st_o, status, gpt::as_stream(stream), kmax);
 }
 
 extern "C" gpt_status gpt_attention_bwd(const void* q, const void* k, const void* v, const void* o,

@@ -70,6 +70,7 @@ extern "C" const char* gpt_strerror(int status) {
     case GPT_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
     case GPT_ERR_TOKEN_OUT_OF_RANGE: return "token or target id out of range";
     case GPT_ERR_NO_DEVICE: return "no sm_100 device is current";
+    case GPT_ERR_NUMERIC_RANGE: return "attention score bound out of the supported range";
     default: return "unknown status";
   }
 }

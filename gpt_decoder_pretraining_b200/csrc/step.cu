@@ -40,7 +40,7 @@ gpt_status cast_f32_bf16(const float* src, void* dst, size_t n, cudaStream_t s);
 gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                          int H, int T, int Dh, int window, long long sbq, long long shq,
                          long long stq, long long sbo, long long sho, long long sto, int* status,
-                         cudaStream_t stream);
+                         cudaStream_t stream, float* kmax_scratch);
 gpt_status attention_bwd(const void* q, const void* k, const void* v, const void* o,
                          const void* dout, const float* lse, float* delta, void* dq, void* dk,
                          void* dv, int B, int H, int T, int Dh, int window, long long sbq,
@@ -281,7 +281,7 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
                         nullptr, nullptr, 0, status, s));
     PROF(PROF_ROPE, 0, 8.0 * (double)M * d, rope_qknorm_fwd(qkv, rq, rk, rope, B, T, H, Dh, s));
     PROF(PROF_ATTN_FWD, 4.0 * Dh * H * B * attn_pairs(T, st->window[l]), 0, attention_fwd(qkv, qkv + d, qkv + 2 * d, o, lse, B, H, T, Dh, st->window[l], qs_b,
-                          qs_h, qs_t, os_b, os_h, os_t, status, s));
+                          qs_h, qs_t, os_b, os_h, os_t, status, s, nullptr));
     PROF(PROF_GEMM, gemm_flops(M, d, d), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_RESID, M, d, d, o, d, W(wq + 1), d, x, d, nullptr,
                         nullptr, 0, status, s));
     PROF(PROF_NORM, 0, 4.0 * (double)M * d + 4.0 * M, rmsnorm_fwd(x, r2, rho2, M, d, s));

@@ -21,7 +21,8 @@ _lib = None
 GPT_OK = 0
 STATUS_NAMES = {0: "GPT_OK", -1: "GPT_ERR_INVALID_ARG", -2: "GPT_ERR_UNSUPPORTED_SHAPE",
                 -3: "GPT_ERR_WORKSPACE_TOO_SMALL", -4: "GPT_ERR_CUDA", -5: "GPT_ERR_DEVICE_TIMEOUT",
-                -6: "GPT_ERR_TOKEN_OUT_OF_RANGE", -7: "GPT_ERR_NO_DEVICE"}
+                -6: "GPT_ERR_TOKEN_OUT_OF_RANGE", -7: "GPT_ERR_NO_DEVICE",
+                -8: "GPT_ERR_NUMERIC_RANGE"}
 GEMM_NT, GEMM_NN, GEMM_TN = 0, 1, 2
 PROFILE_CLASSES = ("gemm", "attn_fwd", "attn_bwd", "rmsnorm", "rope_qknorm", "embedding", "ce_reduce")
 EPI_BF16, EPI_RESID, EPI_RELU2, EPI_DRELU2, EPI_F32, EPI_F32_ADD = 0, 1, 2, 3, 4, 5
@@ -81,7 +82,7 @@ def lib():
         L.gpt_rope_qknorm_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.gpt_rope_qknorm_bwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.gpt_rope_table.argtypes = [vp, i32, i32, vp]
-        L.gpt_attention_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, ll, ll, ll, ll, ll, ll, vp, vp]
+        L.gpt_attention_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, ll, ll, ll, ll, ll, ll, vp, vp]
         L.gpt_attention_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                         ll, ll, ll, ll, ll, ll, vp, vp]
         L.gpt_attention_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
@@ -230,10 +231,16 @@ def rope_qknorm_bwd(dqkv, qkv, rho_q, rho_k, cs, B, T, H, Dh):
                                      cs.data_ptr(), B, T, H, Dh, _stream()), "rope_qknorm_bwd")
 
 
-def attention_fwd(q, k, v, o, lse, window: int, strides_qkv, strides_o, B, H, T, Dh, status=None):
+def attention_fwd(q, k, v, o, lse, window: int, strides_qkv, strides_o, B, H, T, Dh, status=None,
+                  kmax=None, qk_normalized=False):
+    """Causal/window attention forward.  Unless qk_normalized, a B·H float scratch for the per-head
+    key-norm bound is allocated here (or taken from `kmax`)."""
+    import torch
+    if not qk_normalized and kmax is None:
+        kmax = torch.empty(B * H, dtype=torch.float32, device=q.device)
     _check(lib().gpt_attention_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                   B, H, T, Dh, window, *strides_qkv, *strides_o, _ptr(status), _stream()),
-           "attention_fwd")
+                                   _ptr(None if qk_normalized else kmax), B, H, T, Dh, window,
+                                   *strides_qkv, *strides_o, _ptr(status), _stream()), "attention_fwd")
 
 
 def attention_bwd(q, k, v, o, do, lse, delta, dq, dk, dv, window: int, strides_qkv, strides_o, B, H, T,

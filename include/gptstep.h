@@ -43,7 +43,8 @@ typedef enum gpt_status {
   GPT_ERR_CUDA = -4,               /* a CUDA runtime call or kernel launch failed */
   GPT_ERR_DEVICE_TIMEOUT = -5,     /* a bounded device-side wait expired; results are invalid */
   GPT_ERR_TOKEN_OUT_OF_RANGE = -6, /* a token id outside [0, V) (or a target outside [-1, V)) */
-  GPT_ERR_NO_DEVICE = -7           /* no sm_100 device is current */
+  GPT_ERR_NO_DEVICE = -7,          /* no sm_100 device is current */
+  GPT_ERR_NUMERIC_RANGE = -8       /* attention: some ‖q‖·‖k‖/√Dh exceeds 40 (see gpt_attention_fwd) */
 } gpt_status;
 
 enum { GPT_DTYPE_BF16 = 0, GPT_DTYPE_F32 = 1 };
@@ -166,9 +167,15 @@ gpt_status gpt_rope_table(float* cos_sin, int T, int Dh, void* stream);
  * element (b, h, t, j) at base + b·sb + h·sh + t·st + j (strides in elements, j contiguous), one
  * stride set per tensor group: (sb_qkv, sh_qkv, st_qkv) for q/k/v/dq/dk/dv and (sb_o, sh_o, st_o)
  * for o/do.  lse, delta: fp32 [B, H, T].  Dh ∈ {64, 128}.  window ≤ 0 or ≥ T = full causal.
- * lse = natural-log logsumexp of the scaled scores; delta = rowsum(dO∘O) (computed by the bwd). */
+ * lse = natural-log logsumexp of the scaled scores; delta = rowsum(dO∘O) (computed by the bwd).
+ * The forward shifts each row's exponentials by the Cauchy–Schwarz bound c_t = ‖q_t‖·max_j‖k_j‖/√Dh
+ * instead of a running maximum (softmax is invariant to the shift, so the result is exact); this
+ * needs c_t ≤ 40 so that no row underflows, which always holds after QK-norm (c_t ≈ √Dh) — rows
+ * beyond it set GPT_ERR_NUMERIC_RANGE in *status. */
+/* kmax: device scratch of B·H floats that receives max_t ‖k_t‖ per (b, h), or NULL when every k row
+ * is RMS-normalised over Dh (QK-norm), in which case the bound √Dh·(1 + 2⁻⁹) is used. */
 gpt_status gpt_attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
-                             int B, int H, int T, int Dh, int window, long long sb_qkv,
+                             float* kmax, int B, int H, int T, int Dh, int window, long long sb_qkv,
                              long long sh_qkv, long long st_qkv, long long sb_o, long long sh_o,
                              long long st_o, int* status, void* stream);
 gpt_status gpt_attention_bwd(const void* q, const void* k, const void* v, const void* o,

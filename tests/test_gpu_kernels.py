@@ -193,6 +193,11 @@ def test_attention_fwd_bwd(B, H, T, Dh, window):
     lse = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
     st = _status()
     S.attention_fwd(tq, tk, tv, to, lse, window, strides, strides, B, H, T, Dh, status=st)
+    # the same with the QK-norm bound instead of the measured key norms
+    to_n = torch.zeros_like(to)
+    lse_n = torch.zeros_like(lse)
+    S.attention_fwd(tq, tk, tv, to_n, lse_n, window, strides, strides, B, H, T, Dh, status=st,
+                    qk_normalized=True)
     dq, dk, dv = (torch.zeros_like(tq) for _ in range(3))
     delta = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
     S.attention_bwd(tq, tk, tv, to, tdo, lse, delta, dq, dk, dv, window, strides, strides, B, H, T, Dh,
@@ -201,9 +206,14 @@ def test_attention_fwd_bwd(B, H, T, Dh, window):
     assert int(st.item()) == 0
     assert_close_rel(to_np(to), o_ref, rel=2e-2, cos=0.9999, what="o")
     np.testing.assert_allclose(to_np(lse), lse_ref, atol=2e-3)
-    assert_close_rel(to_np(dq), dq_ref, rel=3e-2, cos=0.999, what="dq")
-    assert_close_rel(to_np(dk), dk_ref, rel=3e-2, cos=0.999, what="dk")
-    assert_close_rel(to_np(dv), dv_ref, rel=3e-2, cos=0.999, what="dv")
+    assert_close_rel(to_np(to_n), o_ref, rel=2e-2, cos=0.9999, what="o (qk-norm bound)")
+    np.testing.assert_allclose(to_np(lse_n), lse_ref, atol=2e-3)
+    # Absolute floor: O is stored in bf16 (relative rounding 2^-9), so delta = rowsum(dO∘O) and
+    # hence dS carry ~2^-9·|dO·v| ≈ 2^-9·√Dh of noise even where the exact dq is 0 (T = 1).
+    floor = 2.0 ** -9 * math.sqrt(Dh)
+    assert_close_rel(to_np(dq), dq_ref, rel=3e-2, cos=0.999, what="dq", atol=floor)
+    assert_close_rel(to_np(dk), dk_ref, rel=3e-2, cos=0.999, what="dk", atol=floor)
+    assert_close_rel(to_np(dv), dv_ref, rel=3e-2, cos=0.999, what="dv", atol=floor)
 
 
 def test_attention_token_major_strides():
