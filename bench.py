@@ -353,7 +353,7 @@ def run_kernel(args):
     else:
         T, Dh, W = (int(x) for x in args.attn.split(","))
         H = 8
-        Bt = max(1, (1 << 21) // (H * T))
+        Bt = max(1, args.attn_rows // (H * T))
         q, k, v, do = (torch.from_numpy(a).to(dev).to(torch.bfloat16)
                        for a in make_attention_inputs(Bt, H, T, Dh))
         o = torch.empty_like(q)
@@ -404,6 +404,7 @@ def main():
     ap.add_argument("--gemm-op", default="nt", choices=["nt", "nn", "tn"])
     ap.add_argument("--attn", default="2048,128,0", help="T,Dh,window (window 0 = full causal)")
     ap.add_argument("--attn-pass", default="fwd", choices=["fwd", "bwd"])
+    ap.add_argument("--attn-rows", type=int, default=1 << 21, help="batch·heads·seq of the attention workload")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

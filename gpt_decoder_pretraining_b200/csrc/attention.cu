@@ -467,8 +467,8 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          float p0 = exp2f(fmaf(__uint_as_float(r[2 * e]), a.scale_log2, -c2));
-          float p1 = exp2f(fmaf(__uint_as_float(r[2 * e + 1]), a.scale_log2, -c2));
+          float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * e]), a.scale_log2, -c2));
+          float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * e + 1]), a.scale_log2, -c2));
           if (need_mask) {
             const int key = kv0 + 32 * c + 2 * e;
             if (!(key <= t && key > t - W)) p0 = 0.f;
@@ -508,6 +508,447 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       if (t < T) a.lse[((long long)b * a.H + h) * T + t] = (c2 + log2f(l)) * LN2;
+    }
+  }
+
+  __syncwarp();
+  if (*abort_flag && threadIdx.x == 0) {
+    for (int i = 0; i < 2000; ++i) __nanosleep(1000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+// ================================================================================================
+// backward on the tcgen05 tensor cores (head_dim 64 or 128), two deterministic kernels
+//
+// dK/dV kernel: one CTA per 128-key tile; loops over the 64-query tiles that see it.
+//   Sᵀ = K·Qᵢᵀ and dPᵀ = V·dOᵢᵀ (128 keys × 64 queries, A and B from shared memory) go to tensor
+//   memory; the softmax warps (one key row per thread) form Pᵀ = exp(Sᵀ/√Dh − LSE) and
+//   dSᵀ = Pᵀ∘(dPᵀ − delta), write both back over Sᵀ / dPᵀ as packed bf16, and the MMA warp
+//   accumulates dV += Pᵀ·dOᵢ and dK += dSᵀ·Qᵢ with A read from tensor memory.
+// dQ kernel: one CTA per 128-query tile; loops over its 64-key tiles.
+//   S = Q·Kⱼᵀ, dP = dO·Vⱼᵀ; the softmax warps (one query row per thread) write dS over S and the
+//   MMA warp accumulates dQ += dS·Kⱼ.
+// S/dP buffers are double-buffered in tensor memory, so tile i+1's products run while the softmax
+// warps work on tile i.  Each output element has exactly one writer: results are reproducible.
+// ================================================================================================
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+template <int DH>
+struct TcBwdShape {
+  static constexpr int BIG = 128, SMALL = 64;          // outer tile rows, inner tile rows
+  static constexpr int BIG_TILE = BIG * DH * 2;        // one [128 × DH] bf16 tile
+  static constexpr int SMALL_TILE = SMALL * DH * 2;    // one [64 × DH] bf16 tile
+  static constexpr int STAGES = 4;                     // inner-tile ring depth (hides TMA latency)
+  static constexpr int OFF_A = 0;                      // K (dkdv) or Q (dq)
+  static constexpr int OFF_B = BIG_TILE;               // V (dkdv) or dO (dq)
+  static constexpr int OFF_STAGE = 2 * BIG_TILE;       // stages of (Q, dO) or (K, V)
+  static constexpr int STAGE_BYTES = 2 * SMALL_TILE;
+  static constexpr int OFF_RED = OFF_STAGE + STAGES * STAGE_BYTES;  // [stage][lse2 | delta][64] fp32
+  static constexpr int OFF_BAR = OFF_RED + STAGES * 128 * 4;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int THREADS = 320;  // 8 softmax warps (two per TMEM lane quarter), TMA, MMA
+  static constexpr int TM_S = 0, TM_P = 128, TM_ACC = 256;  // S[b] at b·64, dP[b] at 128 + b·64
+};
+
+// Issue one [128 × 64] product A·Bᵀ (A: 128 rows, B: 64 rows, both K-major [DH/64][rows][64]).
+template <int DH>
+__device__ __forceinline__ void mma_rows_128x64(uint32_t d_tmem, uint32_t a_base, uint32_t b_base,
+                                                uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < DH / 16; ++kk) {
+    mma_bf16_ss(d_tmem, sdesc_sw128(a_base + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024),
+                sdesc_sw128(b_base + (kk >> 2) * (64 * 128) + (kk & 3) * 32, 16, 1024), idesc,
+                kk > 0 ? 1u : 0u);
+  }
+}
+
+// D[128 × DH] (+)= A[128 × 64] (tensor memory, packed bf16) · B[64 × DH] (shared, MN-major).
+// A's 64 columns are packed as two halves of 32: half h occupies tensor-memory columns
+// 32h .. 32h+15 of the 64-column buffer (each softmax warp-half writes inside the columns it read).
+template <int DH>
+__device__ __forceinline__ void mma_acc_from_tmem(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base,
+                                                  uint32_t idesc, bool first) {
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+    mma_bf16_ts(d_tmem, a_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
+                sdesc_sw128(b_base + kk * 2048, 64 * 128, 1024), idesc, (!first || kk > 0) ? 1u : 0u);
+}
+
+template <int DH>
+__global__ void __launch_bounds__(320, 1)
+    attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                            const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
+                            const AttnArgs a) {
+  using S = TcBwdShape<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  float* red = reinterpret_cast<float*>(smem + S::OFF_RED);  // [buf][0 = lse2, 1 = delta][64]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
+  uint64_t* kv_bar = bars;
+  uint64_t* q_full = bars + 1;                // [STAGES]
+  uint64_t* q_empty = q_full + S::STAGES;     // [STAGES]
+  uint64_t* s_full = q_empty + S::STAGES;     // [2]
+  uint64_t* p_full = s_full + 2;              // [2]
+  uint64_t* done = p_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int T = a.T, W = a.window;
+  const int kv0 = blockIdx.x * 128;
+  const int q_first = kv0 / 64;
+  const int q_last = min(T - 1, kv0 + 127 + W - 1) / 64;
+  const int n_q = q_last - q_first + 1;
+  const long long bh = (long long)b * a.H + h;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_bar, 1);
+    for (int i = 0; i < S::STAGES; ++i) {
+      mbar_init(&q_full[i], 2);  // TMA transaction + the LSE/delta staging
+      mbar_init(&q_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 256);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ---------------- TMA producer (lane 0) + LSE/delta staging (all lanes) ----------------
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_bar, 2 * S::BIG_TILE);
+      load_tile<DH, 128>(smem + S::OFF_A, &mk, kv_bar, kv0, h, b);
+      load_tile<DH, 128>(smem + S::OFF_B, &mv, kv_bar, kv0, h, b);
+    }
+    for (int i = 0; i < n_q; ++i) {
+      const int st = i % S::STAGES;
+      if (!mbar_wait(&q_empty[st], ((i / S::STAGES) & 1) ^ 1, abort_flag, a.status)) break;
+      const int t0 = (q_first + i) * 64;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&q_full[st], S::STAGE_BYTES);
+        uint8_t* dst = smem + S::OFF_STAGE + st * S::STAGE_BYTES;
+        load_tile<DH, 64>(dst, &mq, &q_full[st], t0, h, b);
+        load_tile<DH, 64>(dst + S::SMALL_TILE, &mdo, &q_full[st], t0, h, b);
+      }
+      // LSE in log2 units and delta of the 64 queries: 4 values per lane
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int idx = lane + 32 * u;  // 0..63 lse, 64..127 delta
+        const int qq = t0 + (idx & 63);
+        float v = 0.f;
+        if (qq < T) v = (idx < 64) ? a.lse[bh * T + qq] * LOG2E : a.delta[bh * T + qq];
+        red[st * 128 + idx] = v;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&q_full[st]);
+    }
+  } else if (warp == 9) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
+      constexpr uint32_t id_acc = idesc_bf16(128, DH, false, true);
+      const uint32_t kb = smem_u32(smem + S::OFF_A), vb = smem_u32(smem + S::OFF_B);
+      const uint32_t stage0 = smem_u32(smem + S::OFF_STAGE);
+      bool ok = mbar_wait(kv_bar, 0, abort_flag, a.status);
+      auto issue_acc = [&](int i) {  // dV += Pᵀ·dOᵢ, dK += dSᵀ·Qᵢ
+        const int bf = i & 1;
+        const uint32_t qs = stage0 + (i % S::STAGES) * S::STAGE_BYTES;
+        mma_acc_from_tmem<DH>(tmem + S::TM_ACC, tmem + S::TM_S + bf * 64, qs + S::SMALL_TILE, id_acc, i == 0);
+        mma_acc_from_tmem<DH>(tmem + S::TM_ACC + DH, tmem + S::TM_P + bf * 64, qs, id_acc, i == 0);
+        tc_commit(&q_empty[i % S::STAGES]);
+      };
+      for (int i = 0; i < n_q && ok; ++i) {
+        const int st = i % S::STAGES, bf = i & 1;
+        if (!mbar_wait(&q_full[st], (i / S::STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t qs = stage0 + st * S::STAGE_BYTES;
+        mma_rows_128x64<DH>(tmem + S::TM_S + bf * 64, kb, qs, id_s);                  // Sᵀ
+        mma_rows_128x64<DH>(tmem + S::TM_P + bf * 64, vb, qs + S::SMALL_TILE, id_s);  // dPᵀ
+        tc_commit(&s_full[bf]);
+        if (i >= 1) {
+          if (!mbar_wait(&p_full[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+          issue_acc(i - 1);
+        }
+      }
+      if (ok && n_q >= 1) {
+        if (mbar_wait(&p_full[(n_q - 1) & 1], ((n_q - 1) >> 1) & 1, abort_flag, a.status)) {
+          tc_fence_after();
+          issue_acc(n_q - 1);
+        }
+      }
+      tc_commit(done);
+    }
+  } else {
+    // ---------------- softmax-backward warps: thread = key row, warp half = 32 of the 64 queries
+    const int quarter = warp & 3, half = warp >> 2;
+    const int kr = 32 * quarter + lane;
+    const int key = kv0 + kr;
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    bool ok = true;
+    for (int i = 0; i < n_q && ok; ++i) {
+      const int bf = i & 1;
+      const int qc = (q_first + i) * 64 + 32 * half;  // first query of this warp's 32 columns
+      if (!mbar_wait(&s_full[bf], (i >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+      tc_fence_after();
+      const int st = i % S::STAGES;
+      const float4* l2v = reinterpret_cast<const float4*>(red + st * 128 + 32 * half);
+      const float4* dlv = reinterpret_cast<const float4*>(red + st * 128 + 64 + 32 * half);
+      uint32_t rs[32], rp[32];
+      tmem_ld32(tmem + lane_off + S::TM_S + bf * 64 + 32 * half, rs);
+      tmem_ld32(tmem + lane_off + S::TM_P + bf * 64 + 32 * half, rp);
+      tmem_ld_wait();
+      // every (key, query) of the warp visible: no per-element mask
+      const int kmin = kv0 + 32 * quarter, kmax_ = kmin + 31;
+      const bool full = (kmax_ <= qc) && (kmin > qc + 31 - W) && (qc + 31 < T);
+      uint32_t pk[16], dk[16];
+#pragma unroll
+      for (int g4 = 0; g4 < 8; ++g4) {
+        const float4 L = l2v[g4], D = dlv[g4];
+        const float lv[4] = {L.x, L.y, L.z, L.w}, dv4[4] = {D.x, D.y, D.z, D.w};
+        float pv[4], sv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = 4 * g4 + u;
+          float p = ex2_approx(fmaf(__uint_as_float(rs[j]), a.scale_log2, -lv[u]));
+          if (!full) {
+            const int qq = qc + j;
+            if (!((qq < T) && (key <= qq) && (key > qq - W))) p = 0.f;
+          }
+          pv[u] = p;
+          sv[u] = p * (__uint_as_float(rp[j]) - dv4[u]);
+        }
+        pk[2 * g4] = pack_bf2(pv[0], pv[1]);
+        pk[2 * g4 + 1] = pack_bf2(pv[2], pv[3]);
+        dk[2 * g4] = pack_bf2(sv[0], sv[1]);
+        dk[2 * g4 + 1] = pack_bf2(sv[2], sv[3]);
+      }
+      // packed halves stay inside the columns this warp just read (see mma_acc_from_tmem)
+      tmem_st16(tmem + lane_off + S::TM_S + bf * 64 + 32 * half, pk);
+      tmem_st16(tmem + lane_off + S::TM_P + bf * 64 + 32 * half, dk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[bf]);
+    }
+    // epilogue: dV and dK rows of this key tile
+    if (ok) ok = mbar_wait(done, 0, abort_flag, a.status);
+    if (ok) {
+      tc_fence_after();
+      const long long off = b * a.sb_o + h * a.sh_o + (long long)key * a.st_o;
+      {
+        const int part = half;  // half 0 writes dV, half 1 writes dK
+        uint16_t* dst = (part == 0 ? a.dv : a.dk) + off;
+        const float sc = (part == 0) ? 1.f : a.scale;
+#pragma unroll 1
+        for (int c = 0; c < DH / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_off + S::TM_ACC + part * DH + 32 * c, r);
+          tmem_ld_wait();
+          if (key < T) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              uint4 w;
+              w.x = pack_bf2(__uint_as_float(r[8 * u + 0]) * sc, __uint_as_float(r[8 * u + 1]) * sc);
+              w.y = pack_bf2(__uint_as_float(r[8 * u + 2]) * sc, __uint_as_float(r[8 * u + 3]) * sc);
+              w.z = pack_bf2(__uint_as_float(r[8 * u + 4]) * sc, __uint_as_float(r[8 * u + 5]) * sc);
+              w.w = pack_bf2(__uint_as_float(r[8 * u + 6]) * sc, __uint_as_float(r[8 * u + 7]) * sc);
+              *reinterpret_cast<uint4*>(dst + 32 * c + 8 * u) = w;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  if (*abort_flag && threadIdx.x == 0) {
+    for (int i = 0; i < 2000; ++i) __nanosleep(1000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+template <int DH>
+__global__ void __launch_bounds__(320, 1)
+    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                          const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
+                          const AttnArgs a) {
+  using S = TcBwdShape<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
+  uint64_t* q_bar = bars;
+  uint64_t* kv_full = bars + 1;               // [STAGES]
+  uint64_t* kv_empty = kv_full + S::STAGES;   // [STAGES]
+  uint64_t* s_full = kv_empty + S::STAGES;    // [2]
+  uint64_t* p_full = s_full + 2;              // [2]
+  uint64_t* done = p_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int qt = gridDim.x - 1 - blockIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int T = a.T, W = a.window;
+  const int q0 = qt * 128;
+  const int key_lo = max(0, q0 - W + 1);
+  const int key_hi = min(T, q0 + 128);
+  const int kv_first = key_lo / 64;
+  const int n_kv = (key_hi - 1) / 64 - kv_first + 1;
+  const long long bh = (long long)b * a.H + h;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_bar, 1);
+    for (int i = 0; i < S::STAGES; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 256);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_bar, 2 * S::BIG_TILE);
+      load_tile<DH, 128>(smem + S::OFF_A, &mq, q_bar, q0, h, b);
+      load_tile<DH, 128>(smem + S::OFF_B, &mdo, q_bar, q0, h, b);
+      for (int j = 0; j < n_kv; ++j) {
+        const int st = j % S::STAGES;
+        if (!mbar_wait(&kv_empty[st], ((j / S::STAGES) & 1) ^ 1, abort_flag, a.status)) break;
+        mbar_arrive_expect_tx(&kv_full[st], S::STAGE_BYTES);
+        uint8_t* dst = smem + S::OFF_STAGE + st * S::STAGE_BYTES;
+        const int k0 = (kv_first + j) * 64;
+        load_tile<DH, 64>(dst, &mk, &kv_full[st], k0, h, b);
+        load_tile<DH, 64>(dst + S::SMALL_TILE, &mv, &kv_full[st], k0, h, b);
+      }
+    }
+  } else if (warp == 9) {
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
+      constexpr uint32_t id_acc = idesc_bf16(128, DH, false, true);
+      const uint32_t qb = smem_u32(smem + S::OFF_A), dob = smem_u32(smem + S::OFF_B);
+      const uint32_t stage0 = smem_u32(smem + S::OFF_STAGE);
+      bool ok = mbar_wait(q_bar, 0, abort_flag, a.status);
+      auto issue_acc = [&](int j) {  // dQ += dS·Kⱼ
+        const uint32_t ks = stage0 + (j % S::STAGES) * S::STAGE_BYTES;
+        mma_acc_from_tmem<DH>(tmem + S::TM_ACC, tmem + S::TM_S + (j & 1) * 64, ks, id_acc, j == 0);
+        tc_commit(&kv_empty[j % S::STAGES]);
+      };
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int st = j % S::STAGES, bf = j & 1;
+        if (!mbar_wait(&kv_full[st], (j / S::STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t ks = stage0 + st * S::STAGE_BYTES;
+        mma_rows_128x64<DH>(tmem + S::TM_S + bf * 64, qb, ks, id_s);                  // S
+        mma_rows_128x64<DH>(tmem + S::TM_P + bf * 64, dob, ks + S::SMALL_TILE, id_s);  // dP
+        tc_commit(&s_full[bf]);
+        if (j >= 1) {
+          if (!mbar_wait(&p_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+          issue_acc(j - 1);
+        }
+      }
+      if (ok && n_kv >= 1) {
+        if (mbar_wait(&p_full[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort_flag, a.status)) {
+          tc_fence_after();
+          issue_acc(n_kv - 1);
+        }
+      }
+      tc_commit(done);
+    }
+  } else {
+    // ---------------- softmax-backward warps: thread = query row, warp half = 32 of the 64 keys
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = 32 * quarter + lane;
+    const int t = q0 + row;
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    const float l2 = (t < T) ? a.lse[bh * T + t] * LOG2E : 0.f;
+    const float dl = (t < T) ? a.delta[bh * T + t] : 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int bf = j & 1;
+      const int k0 = (kv_first + j) * 64 + 32 * half;
+      if (!mbar_wait(&s_full[bf], (j >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+      tc_fence_after();
+      const bool need_mask = (k0 + 31 > q0 + 32 * quarter) || (k0 <= q0 + 32 * quarter + 31 - W) ||
+                             (q0 + 32 * quarter + 31 >= T);
+      uint32_t rs[32], rp[32];
+      tmem_ld32(tmem + lane_off + S::TM_S + bf * 64 + 32 * half, rs);
+      tmem_ld32(tmem + lane_off + S::TM_P + bf * 64 + 32 * half, rp);
+      tmem_ld_wait();
+      uint32_t dk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        float dv[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int kk = k0 + 2 * e + u;
+          float p = ex2_approx(fmaf(__uint_as_float(rs[2 * e + u]), a.scale_log2, -l2));
+          if (need_mask && !((t < T) && (kk <= t) && (kk > t - W))) p = 0.f;
+          dv[u] = p * (__uint_as_float(rp[2 * e + u]) - dl);
+        }
+        dk[e] = pack_bf2(dv[0], dv[1]);
+      }
+      // the packed half stays inside the columns this warp just read (see mma_acc_from_tmem)
+      tmem_st16(tmem + lane_off + S::TM_S + bf * 64 + 32 * half, dk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[bf]);
+    }
+    if (ok) ok = mbar_wait(done, 0, abort_flag, a.status);
+    if (ok) {
+      tc_fence_after();
+      uint16_t* dst = a.o + b * a.sb_o + h * a.sh_o + (long long)t * a.st_o;
+#pragma unroll 1
+      for (int c = half * (DH / 64); c < (half + 1) * (DH / 64); ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + S::TM_ACC + 32 * c, r);
+        tmem_ld_wait();
+        if (t < T) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 w;
+            w.x = pack_bf2(__uint_as_float(r[8 * u + 0]) * a.scale, __uint_as_float(r[8 * u + 1]) * a.scale);
+            w.y = pack_bf2(__uint_as_float(r[8 * u + 2]) * a.scale, __uint_as_float(r[8 * u + 3]) * a.scale);
+            w.z = pack_bf2(__uint_as_float(r[8 * u + 4]) * a.scale, __uint_as_float(r[8 * u + 5]) * a.scale);
+            w.w = pack_bf2(__uint_as_float(r[8 * u + 6]) * a.scale, __uint_as_float(r[8 * u + 7]) * a.scale);
+            *reinterpret_cast<uint4*>(dst + 32 * c + 8 * u) = w;
+          }
+        }
+      }
     }
   }
 
@@ -960,6 +1401,31 @@ gpt_status launch_bwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, c
   return GPT_OK;
 }
 
+// tcgen05 backward: maps with 128-row boxes (outer tiles) and 64-row boxes (inner tiles).
+template <int DH>
+gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[4], AttnArgs a,
+                         void* dq, cudaStream_t stream) {
+  using S = TcBwdShape<DH>;
+  static bool once = false;
+  if (!once) {
+    GPT_TRY(set_smem(attn_bwd_dkdv_tc_kernel<DH>, S::SMEM));
+    GPT_TRY(set_smem(attn_bwd_dq_tc_kernel<DH>, S::SMEM));
+    once = true;
+  }
+  // dK/dV: outer 128-key tiles (K, V with 128-row boxes), inner 64-query tiles (Q, dO 64-row boxes)
+  dim3 g1((a.T + 127) / 128, a.H, a.B);
+  attn_bwd_dkdv_tc_kernel<DH><<<g1, S::THREADS, S::SMEM, stream>>>(m64[0], m128[1], m128[2], m64[3], a);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  // dQ: outer 128-query tiles (Q, dO 128-row boxes), inner 64-key tiles (K, V 64-row boxes)
+  a.o = reinterpret_cast<uint16_t*>(dq);
+  dim3 g2((a.T + 127) / 128, a.H, a.B);
+  attn_bwd_dq_tc_kernel<DH><<<g2, S::THREADS, S::SMEM, stream>>>(m128[0], m64[1], m64[2], m128[3], a);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
 }  // namespace
 
 // kmax_scratch: B·H floats for max_t ‖k_t‖, or nullptr when every k row is RMS-normalised over
@@ -1049,9 +1515,19 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   dim3 grid((T + 63) / 64, H, B);
   a.dk = reinterpret_cast<uint16_t*>(dk);
   a.dv = reinterpret_cast<uint16_t*>(dv);
-  if (Dh == 128) GPT_TRY(launch_bwd<128>(grid, mq, mk, mv, mdo, a, dq, stream));
-  else if (Dh == 64) GPT_TRY(launch_bwd<64>(grid, mq, mk, mv, mdo, a, dq, stream));
-  else GPT_TRY(launch_bwd<32>(grid, mq, mk, mv, mdo, a, dq, stream));
+  if (Dh == 32) return launch_bwd<32>(grid, mq, mk, mv, mdo, a, dq, stream);
+  CUtensorMap m128[4], m64[4];
+  const void* src[4] = {q, k, v, dout};
+  for (int i = 0; i < 4; ++i) {
+    const bool is_o = (i == 3);
+    if (!make_head_map(&m128[i], src[i], B, H, T, Dh, is_o ? sbo : sbq, is_o ? sho : shq,
+                       is_o ? sto : stq, 128) ||
+        !make_head_map(&m64[i], src[i], B, H, T, Dh, is_o ? sbo : sbq, is_o ? sho : shq,
+                       is_o ? sto : stq, 64))
+      return GPT_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (Dh == 128) GPT_TRY(launch_bwd_tc<128>(m128, m64, a, dq, stream));
+  else GPT_TRY(launch_bwd_tc<64>(m128, m64, a, dq, stream));
   return GPT_OK;
 }
 
