@@ -1,15 +1,19 @@
-// Persistent, warp-specialised bf16 GEMM on the sm_100a tcgen05 tensor cores.
+// Persistent, warp-specialised bf16 GEMM on the sm_100a tcgen05 tensor cores, run by CTA pairs.
 //
-//   warp 0      TMA producer: streams 128×64 A and BN×64 B tiles (128-byte swizzle) into a ring of
-//               shared-memory stages, signalling a "full" mbarrier with the transaction bytes.
-//   warp 1      MMA issuer: one thread issues tcgen05.mma (128×BN×16 per instruction) from the
-//               stage descriptors into a tensor-memory accumulator, commits each stage back to
-//               its "empty" barrier and each finished tile to an accumulator barrier.
-//   warps 2..5  epilogue: tcgen05.ld the fp32 accumulator rows (one row per thread), apply the
-//               fused epilogue (bf16 cast, residual add, ReLU², dReLU², fp32 store, or the
-//               cross-entropy statistics / gradient of the fused lm-head) and store to global.
-// Two accumulator buffers in tensor memory let the epilogue of tile i overlap the main loop of
-// tile i+1.  Tiles are scheduled persistently over min(#tiles, #SMs) CTAs.
+// A cluster of two CTAs (one per SM) computes 256×256 output tiles with one `cta_group::2` MMA
+// stream: each CTA stages its own 128 rows of A and its own 128 rows (columns of C) of B, the even
+// CTA issues the MMAs, and each CTA's tensor memory receives its 128 accumulator rows.  Per SM this
+// halves the B traffic of a 128×256 single-CTA tile and leaves room for a 6-deep TMA ring.
+//
+//   warp 0      TMA producer (both CTAs): 128×64 A and 128×64 B tiles (128-byte swizzle) into the
+//               ring; every load counts its bytes on the leader CTA's "full" barrier.
+//   warp 1      MMA issuer (leader CTA only): tcgen05.mma 256×256×16 into a double-buffered
+//               accumulator; commits free the ring stage and publish the tile in both CTAs.
+//   warps 2..5  epilogue (both CTAs): tcgen05.ld one accumulator row per thread, fused epilogue
+//               (bf16 cast, residual add, ReLU², dReLU², fp32 store / add, split-K reduction, or the
+//               cross-entropy statistics / gradient of the fused lm-head), global store; then
+//               release the accumulator buffer to the leader.
+// Tiles (and K halves, for split-K) are distributed persistently over the CTA pairs.
 //
 // Operand majors: A and B may each be K-contiguous ("K-major") or M/N-contiguous ("MN-major"),
 // which covers y = x·Wᵀ (forward), dx = dy·W (activation gradient) and dW = dyᵀ·x (weight
@@ -23,15 +27,17 @@
 
 namespace gpt {
 
-constexpr int BM = 128;
+constexpr int BM = 128;   // rows per CTA (the pair covers 256)
+constexpr int BN = 256;   // columns per tile (each CTA stages 128 rows of B)
 constexpr int BK = 64;
 constexpr int GEMM_THREADS = 192;
 
-enum : int { EPI_CE_STATS = 100, EPI_CE_GRAD = 101 };
+enum : int { EPI_CE_STATS = 100, EPI_CE_GRAD = 101, EPI_F32_RED = 102 };
 
 struct GemmArgs {
   int M, N, K;
-  int tiles_m, tiles_n, k_tiles;
+  int tiles_m, tiles_n, k_tiles;  // tiles_m counts 256-row pair tiles
+  int splits;                      // split-K factor (1 or 2)
   void* C;
   int ldc;
   void* C2;
@@ -41,12 +47,11 @@ struct GemmArgs {
   CeArgs ce;
 };
 
-template <int BN>
 struct GemmShape {
-  static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int A_BYTES = BM * BK * 2;        // 16 KB
+  static constexpr int B_BYTES = (BN / 2) * BK * 2;  // 16 KB
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int STAGES = 6;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 };
@@ -57,6 +62,15 @@ struct GemmShape {
 template <int EPI>
 __device__ __forceinline__ void epilogue_store(const GemmArgs& a, int m, int n0, const float* v) {
   const bool full = (n0 + 32 <= a.N);
+  if (EPI == EPI_F32_RED) {
+    // split-K: exactly two partial sums land on a zeroed output; fp32 addition is commutative,
+    // so 0 + a + b is the same whichever half arrives first
+    float* c = reinterpret_cast<float*>(a.C) + (size_t)m * a.ldc + n0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (n0 + j < a.N) atomicAdd(c + j, v[j]);
+    return;
+  }
   if (EPI == GPT_EPI_F32 || EPI == GPT_EPI_F32_ADD) {
     float* c = reinterpret_cast<float*>(a.C) + (size_t)m * a.ldc + n0;
     if (full) {
@@ -145,11 +159,11 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, int m, int n0,
 // ------------------------------------------------------------------------------------------------
 // the kernel
 // ------------------------------------------------------------------------------------------------
-template <int BN, bool A_MN, bool B_MN, int EPI>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+template <bool A_MN, bool B_MN, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmArgs args) {
-  using S = GemmShape<BN>;
+  using S = GemmShape;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -161,6 +175,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = warp_id(), lane = lane_id();
+  const uint32_t rank = cluster_ctarank();  // 0 = leader (issues the MMAs), 1 = peer
+  const bool leader = (rank == 0);
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -168,7 +184,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 128);
+      mbar_init(&tempty[b], 2 * 128);  // epilogue threads of both CTAs
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -176,43 +192,56 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, S::TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, S::TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // barriers of both CTAs initialised before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int num_tiles = args.tiles_m * args.tiles_n;
+  const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+  const int mn_tiles = args.tiles_m * args.tiles_n;
+  const int num_units = mn_tiles * args.splits;
+  const int kt_per_split = (args.k_tiles + args.splits - 1) / args.splits;
+  auto unit_coords = [&](int u, int& tm, int& tn, int& kt0, int& kt1) {
+    const int ks = u / mn_tiles, r = u % mn_tiles;
+    tm = r / args.tiles_n;
+    tn = r % args.tiles_n;
+    kt0 = ks * kt_per_split;
+    kt1 = min(args.k_tiles, kt0 + kt_per_split);
+  };
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (both CTAs) ----------------
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        const int tm = tile / args.tiles_n, tn = tile % args.tiles_n;
+      for (int u = pair; u < num_units; u += num_pairs) {
+        int tm, tn, kt0, kt1;
+        unit_coords(u, tm, tn, kt0, kt1);
+        const int arow = tm * 2 * BM + rank * BM;        // this CTA's 128 rows of A
+        const int brow = tn * BN + rank * (BN / 2);      // this CTA's 128 rows of B
         bool ok = true;
-        for (int kt = 0; kt < args.k_tiles; ++kt) {
+        for (int kt = kt0; kt < kt1; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, args.status)) { ok = false; break; }
           uint8_t* sa = smem + stage * S::STAGE_BYTES;
           uint8_t* sb = sa + S::A_BYTES;
-          mbar_arrive_expect_tx(&full[stage], S::STAGE_BYTES);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * S::STAGE_BYTES);
           const int k0 = kt * BK;
           if (!A_MN) {
-            tma_load_2d(sa, &tmA, &full[stage], k0, tm * BM);
+            tma_load_2d_pair(sa, &tmA, &full[stage], k0, arow);
           } else {
 #pragma unroll
             for (int c = 0; c < BM / 64; ++c)
-              tma_load_2d(sa + c * 8192, &tmA, &full[stage], tm * BM + c * 64, k0);
+              tma_load_2d_pair(sa + c * 8192, &tmA, &full[stage], arow + c * 64, k0);
           }
           if (!B_MN) {
-            tma_load_2d(sb, &tmB, &full[stage], k0, tn * BN);
+            tma_load_2d_pair(sb, &tmB, &full[stage], k0, brow);
           } else {
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c)
-              tma_load_2d(sb + c * 8192, &tmB, &full[stage], tn * BN + c * 64, k0);
+            for (int c = 0; c < (BN / 2) / 64; ++c)
+              tma_load_2d_pair(sb + c * 8192, &tmB, &full[stage], brow + c * 64, k0);
           }
           if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
         }
@@ -220,19 +249,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(BM, BN, A_MN, B_MN);
+    // ---------------- MMA issuer (leader CTA) ----------------
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(2 * BM, BN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      for (int u = pair; u < num_units; u += num_pairs) {
+        int tm, tn, kt0, kt1;
+        unit_coords(u, tm, tn, kt0, kt1);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, args.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         bool ok = true;
-        for (int kt = 0; kt < args.k_tiles; ++kt) {
+        for (int kt = kt0; kt < kt1; ++kt) {
           if (!mbar_wait(&full[stage], phase, abort_flag, args.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * S::STAGE_BYTES);
@@ -243,26 +274,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                                      : sdesc_sw128(sa + kk * 32, 16, 1024);
             const uint64_t bd = B_MN ? sdesc_sw128(sb + kk * 2048, 8192, 1024)
                                      : sdesc_sw128(sb + kk * 32, 16, 1024);
-            mma_bf16_ss(d_tmem, ad, bd, idesc, (kt | kk) != 0 ? 1u : 0u);
+            mma_bf16_pair(d_tmem, ad, bd, idesc, (kt > kt0 || kk > 0) ? 1u : 0u);
           }
-          tc_commit(&empty[stage]);
+          tc_commit_pair(&empty[stage], 0x3);
           if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        tc_commit(&tfull[acc]);
+        tc_commit_pair(&tfull[acc], 0x3);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1;
       }
     }
   } else {
-    // ---------------- epilogue warps ----------------
+    // ---------------- epilogue warps (both CTAs) ----------------
     const int q = warp & 3;
     const int row_in_tile = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int tm = tile / args.tiles_n, tn = tile % args.tiles_n;
-      const int m = tm * BM + row_in_tile;
+    for (int u = pair; u < num_units; u += num_pairs) {
+      int tm, tn, kt0, kt1;
+      unit_coords(u, tm, tn, kt0, kt1);
+      const int m = tm * 2 * BM + rank * BM + row_in_tile;
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, args.status)) break;
       tc_fence_after();
       float run_max = -INFINITY, run_sum = 0.f;
@@ -293,12 +325,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             for (int j = 0; j < 32; ++j)
               if (n0 + j < args.N) cm = fmaxf(cm, v[j]);
             const float nm = fmaxf(run_max, cm);
-            float s = (run_max == -INFINITY) ? 0.f : run_sum * __expf(run_max - nm);
+            float sacc = (run_max == -INFINITY) ? 0.f : run_sum * __expf(run_max - nm);
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (n0 + j < args.N) s += __expf(v[j] - nm);
+              if (n0 + j < args.N) sacc += __expf(v[j] - nm);
             run_max = nm;
-            run_sum = s;
+            run_sum = sacc;
             if (tgt >= n0 && tgt < n0 + 32 && tgt < args.N) {
 #pragma unroll
               for (int j = 0; j < 32; ++j)
@@ -306,7 +338,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             }
           }
         } else if (EPI == EPI_CE_GRAD) {
-          if (m < args.M) {
+          if (m < args.M && n0 < args.N) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const float p = __expf(v[j] - lse_m);
@@ -323,7 +355,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             make_float2(run_max, run_sum);
       }
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      mbar_arrive_leader(&tempty[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
@@ -336,19 +368,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     for (int i = 0; i < 2000; ++i) __nanosleep(1000);
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its partner may still signal or read it
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, S::TMEM_COLS);
+  if (warp == 1) tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
 }
 
 // ------------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------------
-template <int BN, bool A_MN, bool B_MN, int EPI>
+template <bool A_MN, bool B_MN, int EPI>
 static gpt_status launch_inst(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& a,
                               cudaStream_t stream) {
-  using S = GemmShape<BN>;
-  auto kern = gemm_kernel<BN, A_MN, B_MN, EPI>;
+  using S = GemmShape;
+  auto kern = gemm_kernel<A_MN, B_MN, EPI>;
   static bool attr_done = false;  // per instantiation
   if (!attr_done) {
     GPT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -357,37 +389,39 @@ static gpt_status launch_inst(const CUtensorMap& ma, const CUtensorMap& mb, cons
   }
   int sms = 0;
   GPT_TRY(device_info(&sms));
-  const int tiles = a.tiles_m * a.tiles_n;
-  const int grid = std::min(tiles, sms);
-  kern<<<grid, GEMM_THREADS, S::SMEM_BYTES, stream>>>(ma, mb, a);
+  const int units = a.tiles_m * a.tiles_n * a.splits;
+  const int pairs = std::max(1, std::min(units, sms / 2));
+  kern<<<2 * pairs, GEMM_THREADS, S::SMEM_BYTES, stream>>>(ma, mb, a);
   count_launch();
   GPT_CUDA_TRY(cudaGetLastError());
   return GPT_OK;
 }
 
-template <int BN, bool A_MN, bool B_MN>
+template <bool A_MN, bool B_MN>
 static gpt_status dispatch_epi(int epi, const CUtensorMap& ma, const CUtensorMap& mb,
                                const GemmArgs& a, cudaStream_t s) {
   switch (epi) {
-    case GPT_EPI_BF16: return launch_inst<BN, A_MN, B_MN, GPT_EPI_BF16>(ma, mb, a, s);
-    case GPT_EPI_RESID: return launch_inst<BN, A_MN, B_MN, GPT_EPI_RESID>(ma, mb, a, s);
-    case GPT_EPI_RELU2: return launch_inst<BN, A_MN, B_MN, GPT_EPI_RELU2>(ma, mb, a, s);
-    case GPT_EPI_DRELU2: return launch_inst<BN, A_MN, B_MN, GPT_EPI_DRELU2>(ma, mb, a, s);
-    case GPT_EPI_F32: return launch_inst<BN, A_MN, B_MN, GPT_EPI_F32>(ma, mb, a, s);
-    case GPT_EPI_F32_ADD: return launch_inst<BN, A_MN, B_MN, GPT_EPI_F32_ADD>(ma, mb, a, s);
+    case GPT_EPI_BF16: return launch_inst<A_MN, B_MN, GPT_EPI_BF16>(ma, mb, a, s);
+    case GPT_EPI_RESID: return launch_inst<A_MN, B_MN, GPT_EPI_RESID>(ma, mb, a, s);
+    case GPT_EPI_RELU2: return launch_inst<A_MN, B_MN, GPT_EPI_RELU2>(ma, mb, a, s);
+    case GPT_EPI_DRELU2: return launch_inst<A_MN, B_MN, GPT_EPI_DRELU2>(ma, mb, a, s);
+    case GPT_EPI_F32: return launch_inst<A_MN, B_MN, GPT_EPI_F32>(ma, mb, a, s);
+    case GPT_EPI_F32_ADD: return launch_inst<A_MN, B_MN, GPT_EPI_F32_ADD>(ma, mb, a, s);
+    case EPI_F32_RED: return launch_inst<A_MN, B_MN, EPI_F32_RED>(ma, mb, a, s);
     default: return GPT_ERR_INVALID_ARG;
   }
 }
 
-// A operand map: K-major [M rows, K cols] box {64, 128}; MN-major [K rows, M cols] box {64, 64}.
+// Operand map for one CTA's half of a pair tile: K-major [rows, K] with box {64, 128};
+// MN-major [K rows, MN cols] with box {64, 64}.
 static bool make_operand_map(CUtensorMap* map, const void* base, bool mn_major, int mn, int K,
-                             int ld, int box_mn) {
+                             int ld) {
   uint64_t dims[2], strides[1];
   uint32_t box[2];
   strides[0] = (uint64_t)ld * 2;
   if (!mn_major) {
     dims[0] = (uint64_t)K; dims[1] = (uint64_t)mn;
-    box[0] = 64; box[1] = (uint32_t)box_mn;
+    box[0] = 64; box[1] = 128;
   } else {
     dims[0] = (uint64_t)mn; dims[1] = (uint64_t)K;
     box[0] = 64; box[1] = 64;
@@ -410,56 +444,72 @@ static gpt_status check_gemm_args(int op, int M, int N, int K, const void* A, in
   return GPT_OK;
 }
 
+static void fill_args(GemmArgs& a, int M, int N, int K, int splits) {
+  a.M = M; a.N = N; a.K = K;
+  a.tiles_m = (M + 2 * BM - 1) / (2 * BM);
+  a.tiles_n = (N + BN - 1) / BN;
+  a.k_tiles = (K + BK - 1) / BK;
+  a.splits = splits;
+}
+
 gpt_status gemm_launch(int op, int epi, int M, int N, int K, const void* A, int lda, const void* B,
                        int ldb, void* C, int ldc, void* C2, const void* aux, int ldaux, int* status,
                        cudaStream_t stream) {
   GPT_TRY(check_gemm_args(op, M, N, K, A, lda, B, ldb, C, ldc));
+  if (epi < GPT_EPI_BF16 || epi > GPT_EPI_F32_ADD) return GPT_ERR_INVALID_ARG;
   if (epi == GPT_EPI_RELU2 && !C2) return GPT_ERR_INVALID_ARG;
   if (epi == GPT_EPI_DRELU2 && (!aux || ldaux < N || (ldaux % 8))) return GPT_ERR_INVALID_ARG;
   const bool a_mn = (op == GPT_GEMM_TN);
   const bool b_mn = (op != GPT_GEMM_NT);
-  const int BN = (N > 128) ? 256 : 128;
   CUtensorMap ma, mb;
-  if (!make_operand_map(&ma, A, a_mn, M, K, lda, BM)) return GPT_ERR_UNSUPPORTED_SHAPE;
-  if (!make_operand_map(&mb, B, b_mn, N, K, ldb, BN)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if (!make_operand_map(&ma, A, a_mn, M, K, lda)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if (!make_operand_map(&mb, B, b_mn, N, K, ldb)) return GPT_ERR_UNSUPPORTED_SHAPE;
   GemmArgs a{};
-  a.M = M; a.N = N; a.K = K;
-  a.tiles_m = (M + BM - 1) / BM;
-  a.tiles_n = (N + BN - 1) / BN;
-  a.k_tiles = (K + BK - 1) / BK;
+  fill_args(a, M, N, K, 1);
   a.C = C; a.ldc = ldc; a.C2 = C2;
   a.aux = reinterpret_cast<const uint16_t*>(aux); a.ldaux = ldaux;
   a.status = status;
-  if (BN == 256) {
-    if (op == GPT_GEMM_NT) return dispatch_epi<256, false, false>(epi, ma, mb, a, stream);
-    if (op == GPT_GEMM_NN) return dispatch_epi<256, false, true>(epi, ma, mb, a, stream);
-    return dispatch_epi<256, true, true>(epi, ma, mb, a, stream);
-  } else {
-    if (op == GPT_GEMM_NT) return dispatch_epi<128, false, false>(epi, ma, mb, a, stream);
-    if (op == GPT_GEMM_NN) return dispatch_epi<128, false, true>(epi, ma, mb, a, stream);
-    return dispatch_epi<128, true, true>(epi, ma, mb, a, stream);
+  // A plain fp32 store (weight gradients: few tiles, long K) is split into two K halves when that
+  // shortens the schedule (waves of CTA pairs × k-tiles per unit); the halves add onto a zeroed
+  // output.
+  int sms = 0;
+  GPT_TRY(device_info(&sms));
+  if (epi == GPT_EPI_F32 && a.k_tiles >= 8) {
+    const long long pairs = std::max(1, sms / 2), units = (long long)a.tiles_m * a.tiles_n;
+    const long long t1 = ((units + pairs - 1) / pairs) * a.k_tiles;
+    const long long t2 = ((2 * units + pairs - 1) / pairs) * ((a.k_tiles + 1) / 2);
+    if (t2 < t1) {
+      if (ldc == N) {
+        GPT_CUDA_TRY(cudaMemsetAsync(C, 0, (size_t)M * N * sizeof(float), stream));
+      } else {
+        GPT_CUDA_TRY(cudaMemset2DAsync(C, (size_t)ldc * sizeof(float), 0, (size_t)N * sizeof(float),
+                                       M, stream));
+      }
+      a.splits = 2;
+      epi = EPI_F32_RED;
+    }
   }
+  if (op == GPT_GEMM_NT) return dispatch_epi<false, false>(epi, ma, mb, a, stream);
+  if (op == GPT_GEMM_NN) return dispatch_epi<false, true>(epi, ma, mb, a, stream);
+  return dispatch_epi<true, true>(epi, ma, mb, a, stream);
 }
 
-int gemm_ce_tile_n() { return 256; }
+int gemm_ce_tile_n() { return BN; }
 
 gpt_status gemm_ce_launch(bool grad, int M, int N, int K, const void* A, int lda, const void* B,
                           int ldb, void* C, int ldc, const CeArgs& ce, int* status,
                           cudaStream_t stream) {
   GPT_TRY(check_gemm_args(GPT_GEMM_NT, M, N, K, A, lda, B, ldb, grad ? C : (void*)A, grad ? ldc : N));
   CUtensorMap ma, mb;
-  if (!make_operand_map(&ma, A, false, M, K, lda, BM)) return GPT_ERR_UNSUPPORTED_SHAPE;
-  if (!make_operand_map(&mb, B, false, N, K, ldb, 256)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if (!make_operand_map(&ma, A, false, M, K, lda)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if (!make_operand_map(&mb, B, false, N, K, ldb)) return GPT_ERR_UNSUPPORTED_SHAPE;
   GemmArgs a{};
-  a.M = M; a.N = N; a.K = K;
-  a.tiles_m = (M + BM - 1) / BM;
-  a.tiles_n = (N + 255) / 256;
-  a.k_tiles = (K + BK - 1) / BK;
+  fill_args(a, M, N, K, 1);
   a.C = C; a.ldc = ldc;
   a.status = status;
   a.ce = ce;
-  if (grad) return launch_inst<256, false, false, EPI_CE_GRAD>(ma, mb, a, stream);
-  return launch_inst<256, false, false, EPI_CE_STATS>(ma, mb, a, stream);
+  if (grad) return launch_inst<false, false, EPI_CE_GRAD>(ma, mb, a, stream);
+  return launch_inst<false, false, EPI_CE_STATS>(ma, mb, a, stream);
 }
 
 }  // namespace gpt

@@ -121,97 +121,141 @@ __global__ void rope_table_kernel(float* __restrict__ cs, int T, int half, int D
   cs[2 * idx + 1] = (float)sin(phi);
 }
 
-// One warp per (token m, part ∈ {q, k}, head h); lane handles pair indices i = 2·lane + {0,1}
-// (+64 per further round) of the first half and their partners i + Dh/2.
-__global__ void rope_qknorm_fwd_kernel(uint16_t* __restrict__ qkv, float* __restrict__ rho_q,
-                                       float* __restrict__ rho_k, const float* __restrict__ cs,
-                                       int M, int T, int H, int Dh) {
-  const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+// One warp per token: it walks the 2H (part ∈ {q, k}, head) units of the token in batches of 8,
+// issuing all loads of a batch before using them.  Lane l holds the pairs i = 2l, 2l+1 (+64 per
+// further round) of the first half of each head and their partners i + Dh/2; the cos/sin of those
+// pairs at position t are loaded once per token.
+constexpr int ROPE_BATCH = 8;
+
+template <int ROUNDS>
+__global__ void __launch_bounds__(256) rope_qknorm_fwd_kernel(uint16_t* __restrict__ qkv, float* __restrict__ rho_q,
+                                                              float* __restrict__ rho_k, const float* __restrict__ cs,
+                                                              int M, int T, int H, int Dh) {
+  const long long m = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (w >= (long long)M * 2 * H) return;
-  const int h = (int)(w % H), part = (int)((w / H) % 2);
-  const long long m = w / (2 * H);
+  if (m >= M) return;
   const int t = (int)(m % T), half = Dh >> 1, d = H * Dh;
-  uint16_t* p = qkv + m * 3 * d + part * d + h * Dh;
-  float a[2][2], b[2][2];
-  float ss = 0.f;
-  const int rounds = (half + 63) >> 6;
+  bool act[ROUNDS];
+  float4 cw[ROUNDS];  // cos_i, sin_i, cos_{i+1}, sin_{i+1}
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
+  for (int rr = 0; rr < ROUNDS; ++rr) {
     const int i = 2 * lane + 64 * rr;
-    if (rr < rounds && i < half) {
-      const uint32_t ua = *reinterpret_cast<const uint32_t*>(p + i);
-      const uint32_t ub = *reinterpret_cast<const uint32_t*>(p + i + half);
-      const float a0 = bf_lo(ua), a1 = bf_hi(ua), b0 = bf_lo(ub), b1 = bf_hi(ub);
-      const float2 c0 = *reinterpret_cast<const float2*>(cs + 2 * ((size_t)t * half + i));
-      const float2 c1 = *reinterpret_cast<const float2*>(cs + 2 * ((size_t)t * half + i + 1));
-      a[rr][0] = a0 * c0.x - b0 * c0.y;
-      b[rr][0] = a0 * c0.y + b0 * c0.x;
-      a[rr][1] = a1 * c1.x - b1 * c1.y;
-      b[rr][1] = a1 * c1.y + b1 * c1.x;
-      ss += a[rr][0] * a[rr][0] + a[rr][1] * a[rr][1] + b[rr][0] * b[rr][0] + b[rr][1] * b[rr][1];
+    act[rr] = i < half;
+    if (act[rr]) cw[rr] = *reinterpret_cast<const float4*>(cs + 2 * ((size_t)t * half + i));
+  }
+  uint16_t* row = qkv + m * 3 * d;
+  for (int u0 = 0; u0 < 2 * H; u0 += ROPE_BATCH) {
+    uint32_t ua[ROPE_BATCH][ROUNDS], ub[ROPE_BATCH][ROUNDS];
+#pragma unroll
+    for (int k = 0; k < ROPE_BATCH; ++k) {
+      const int u = u0 + k;
+#pragma unroll
+      for (int rr = 0; rr < ROUNDS; ++rr) {
+        ua[k][rr] = ub[k][rr] = 0;
+        if (u < 2 * H && act[rr]) {
+          const uint16_t* p = row + (u / H) * d + (u % H) * Dh + 2 * lane + 64 * rr;
+          ua[k][rr] = *reinterpret_cast<const uint32_t*>(p);
+          ub[k][rr] = *reinterpret_cast<const uint32_t*>(p + half);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < ROPE_BATCH; ++k) {
+      const int u = u0 + k;
+      if (u >= 2 * H) break;  // warp-uniform
+      float a0[ROUNDS], a1[ROUNDS], b0[ROUNDS], b1[ROUNDS];
+      float ss = 0.f;
+#pragma unroll
+      for (int rr = 0; rr < ROUNDS; ++rr) {
+        const float x0 = bf_lo(ua[k][rr]), x1 = bf_hi(ua[k][rr]);
+        const float y0 = bf_lo(ub[k][rr]), y1 = bf_hi(ub[k][rr]);
+        const float4 c = cw[rr];
+        a0[rr] = x0 * c.x - y0 * c.y;
+        b0[rr] = x0 * c.y + y0 * c.x;
+        a1[rr] = x1 * c.z - y1 * c.w;
+        b1[rr] = x1 * c.w + y1 * c.z;
+        if (act[rr]) ss += a0[rr] * a0[rr] + a1[rr] * a1[rr] + b0[rr] * b0[rr] + b1[rr] * b1[rr];
+      }
+      ss = warp_sum(ss);
+      const float r = rsqrtf(ss / (float)Dh + NORM_EPS);
+      uint16_t* p = row + (u / H) * d + (u % H) * Dh + 2 * lane;
+#pragma unroll
+      for (int rr = 0; rr < ROUNDS; ++rr) {
+        if (act[rr]) {
+          *reinterpret_cast<uint32_t*>(p + 64 * rr) = pack_bf2(a0[rr] * r, a1[rr] * r);
+          *reinterpret_cast<uint32_t*>(p + 64 * rr + half) = pack_bf2(b0[rr] * r, b1[rr] * r);
+        }
+      }
+      if (lane == 0) ((u < H) ? rho_q : rho_k)[m * H + (u % H)] = r;
     }
   }
-  ss = warp_sum(ss);
-  const float r = rsqrtf(ss / (float)Dh + NORM_EPS);
-#pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const int i = 2 * lane + 64 * rr;
-    if (rr < rounds && i < half) {
-      *reinterpret_cast<uint32_t*>(p + i) = pack_bf2(a[rr][0] * r, a[rr][1] * r);
-      *reinterpret_cast<uint32_t*>(p + i + half) = pack_bf2(b[rr][0] * r, b[rr][1] * r);
-    }
-  }
-  if (lane == 0) (part == 0 ? rho_q : rho_k)[m * H + h] = r;
 }
 
 // Backward: g = rho·(dŷ − ŷ·mean(ŷ·dŷ)) with ŷ the stored forward output, then the inverse
-// rotation (a, b) → (a cos + b sin, −a sin + b cos).
-__global__ void rope_qknorm_bwd_kernel(uint16_t* __restrict__ dqkv, const uint16_t* __restrict__ qkv,
-                                       const float* __restrict__ rho_q, const float* __restrict__ rho_k,
-                                       const float* __restrict__ cs, int M, int T, int H, int Dh) {
-  const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+// rotation (a, b) → (a cos + b sin, −a sin + b cos).  Same work split as the forward.
+template <int ROUNDS>
+__global__ void __launch_bounds__(256) rope_qknorm_bwd_kernel(uint16_t* __restrict__ dqkv, const uint16_t* __restrict__ qkv,
+                                                              const float* __restrict__ rho_q, const float* __restrict__ rho_k,
+                                                              const float* __restrict__ cs, int M, int T, int H, int Dh) {
+  const long long m = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (w >= (long long)M * 2 * H) return;
-  const int h = (int)(w % H), part = (int)((w / H) % 2);
-  const long long m = w / (2 * H);
+  if (m >= M) return;
   const int t = (int)(m % T), half = Dh >> 1, d = H * Dh;
-  const long long off = m * 3 * d + part * d + h * Dh;
-  uint16_t* g = dqkv + off;
-  const uint16_t* y = qkv + off;
-  const float r = (part == 0 ? rho_q : rho_k)[m * H + h];
-  float ga[2][2], gb[2][2], ya[2][2], yb[2][2];
-  float dot = 0.f;
-  const int rounds = (half + 63) >> 6;
+  bool act[ROUNDS];
+  float4 cw[ROUNDS];
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
+  for (int rr = 0; rr < ROUNDS; ++rr) {
     const int i = 2 * lane + 64 * rr;
-    if (rr < rounds && i < half) {
-      const uint32_t u0 = *reinterpret_cast<const uint32_t*>(g + i);
-      const uint32_t u1 = *reinterpret_cast<const uint32_t*>(g + i + half);
-      const uint32_t v0 = *reinterpret_cast<const uint32_t*>(y + i);
-      const uint32_t v1 = *reinterpret_cast<const uint32_t*>(y + i + half);
-      ga[rr][0] = bf_lo(u0); ga[rr][1] = bf_hi(u0); gb[rr][0] = bf_lo(u1); gb[rr][1] = bf_hi(u1);
-      ya[rr][0] = bf_lo(v0); ya[rr][1] = bf_hi(v0); yb[rr][0] = bf_lo(v1); yb[rr][1] = bf_hi(v1);
-      dot += ga[rr][0] * ya[rr][0] + ga[rr][1] * ya[rr][1] + gb[rr][0] * yb[rr][0] + gb[rr][1] * yb[rr][1];
-    }
+    act[rr] = i < half;
+    if (act[rr]) cw[rr] = *reinterpret_cast<const float4*>(cs + 2 * ((size_t)t * half + i));
   }
-  dot = warp_sum(dot) / (float)Dh;
+  uint16_t* grow = dqkv + m * 3 * d;
+  const uint16_t* yrow = qkv + m * 3 * d;
+  for (int u0 = 0; u0 < 2 * H; u0 += ROPE_BATCH) {
+    uint32_t ga[ROPE_BATCH][ROUNDS], gb[ROPE_BATCH][ROUNDS], ya[ROPE_BATCH][ROUNDS], yb[ROPE_BATCH][ROUNDS];
+    float rh[ROPE_BATCH];
 #pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const int i = 2 * lane + 64 * rr;
-    if (rr < rounds && i < half) {
-      float oa[2], ob[2];
+    for (int k = 0; k < ROPE_BATCH; ++k) {
+      const int u = u0 + k;
+      rh[k] = 0.f;
+      if (u < 2 * H) rh[k] = ((u < H) ? rho_q : rho_k)[m * H + (u % H)];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float na = r * (ga[rr][e] - ya[rr][e] * dot);
-        const float nb = r * (gb[rr][e] - yb[rr][e] * dot);
-        const float2 c = *reinterpret_cast<const float2*>(cs + 2 * ((size_t)t * half + i + e));
-        oa[e] = na * c.x + nb * c.y;
-        ob[e] = -na * c.y + nb * c.x;
+      for (int rr = 0; rr < ROUNDS; ++rr) {
+        ga[k][rr] = gb[k][rr] = ya[k][rr] = yb[k][rr] = 0;
+        if (u < 2 * H && act[rr]) {
+          const size_t off = (u / H) * d + (u % H) * Dh + 2 * lane + 64 * rr;
+          ga[k][rr] = *reinterpret_cast<const uint32_t*>(grow + off);
+          gb[k][rr] = *reinterpret_cast<const uint32_t*>(grow + off + half);
+          ya[k][rr] = *reinterpret_cast<const uint32_t*>(yrow + off);
+          yb[k][rr] = *reinterpret_cast<const uint32_t*>(yrow + off + half);
+        }
       }
-      *reinterpret_cast<uint32_t*>(g + i) = pack_bf2(oa[0], oa[1]);
-      *reinterpret_cast<uint32_t*>(g + i + half) = pack_bf2(ob[0], ob[1]);
+    }
+#pragma unroll
+    for (int k = 0; k < ROPE_BATCH; ++k) {
+      const int u = u0 + k;
+      if (u >= 2 * H) break;
+      float dot = 0.f;
+#pragma unroll
+      for (int rr = 0; rr < ROUNDS; ++rr)
+        dot += bf_lo(ga[k][rr]) * bf_lo(ya[k][rr]) + bf_hi(ga[k][rr]) * bf_hi(ya[k][rr]) +
+               bf_lo(gb[k][rr]) * bf_lo(yb[k][rr]) + bf_hi(gb[k][rr]) * bf_hi(yb[k][rr]);
+      dot = warp_sum(dot) / (float)Dh;
+      const float r = rh[k];
+      uint16_t* p = grow + (u / H) * d + (u % H) * Dh + 2 * lane;
+#pragma unroll
+      for (int rr = 0; rr < ROUNDS; ++rr) {
+        if (!act[rr]) continue;
+        const float4 c = cw[rr];
+        const float na0 = r * (bf_lo(ga[k][rr]) - bf_lo(ya[k][rr]) * dot);
+        const float na1 = r * (bf_hi(ga[k][rr]) - bf_hi(ya[k][rr]) * dot);
+        const float nb0 = r * (bf_lo(gb[k][rr]) - bf_lo(yb[k][rr]) * dot);
+        const float nb1 = r * (bf_hi(gb[k][rr]) - bf_hi(yb[k][rr]) * dot);
+        *reinterpret_cast<uint32_t*>(p + 64 * rr) =
+            pack_bf2(na0 * c.x + nb0 * c.y, na1 * c.z + nb1 * c.w);
+        *reinterpret_cast<uint32_t*>(p + 64 * rr + half) =
+            pack_bf2(-na0 * c.y + nb0 * c.x, -na1 * c.w + nb1 * c.z);
+      }
     }
   }
 }
@@ -457,9 +501,13 @@ gpt_status rope_qknorm_fwd(void* qkv, float* rq, float* rk, const float* cs, int
                            int Dh, cudaStream_t s) {
   if (!qkv || !rq || !rk || !cs) return GPT_ERR_INVALID_ARG;
   GPT_TRY(check_rope(B, T, H, Dh));
-  const long long warps = (long long)B * T * 2 * H;
-  rope_qknorm_fwd_kernel<<<blocks_for_warps(warps, 256), 256, 0, s>>>(
-      reinterpret_cast<uint16_t*>(qkv), rq, rk, cs, B * T, T, H, Dh);
+  const long long warps = (long long)B * T;
+  if (Dh > 128)
+    rope_qknorm_fwd_kernel<2><<<blocks_for_warps(warps, 256), 256, 0, s>>>(
+        reinterpret_cast<uint16_t*>(qkv), rq, rk, cs, B * T, T, H, Dh);
+  else
+    rope_qknorm_fwd_kernel<1><<<blocks_for_warps(warps, 256), 256, 0, s>>>(
+        reinterpret_cast<uint16_t*>(qkv), rq, rk, cs, B * T, T, H, Dh);
   count_launch();
   GPT_CUDA_TRY(cudaGetLastError());
   return GPT_OK;
@@ -469,10 +517,15 @@ gpt_status rope_qknorm_bwd(void* dqkv, const void* qkv, const float* rq, const f
                            const float* cs, int B, int T, int H, int Dh, cudaStream_t s) {
   if (!dqkv || !qkv || !rq || !rk || !cs) return GPT_ERR_INVALID_ARG;
   GPT_TRY(check_rope(B, T, H, Dh));
-  const long long warps = (long long)B * T * 2 * H;
-  rope_qknorm_bwd_kernel<<<blocks_for_warps(warps, 256), 256, 0, s>>>(
-      reinterpret_cast<uint16_t*>(dqkv), reinterpret_cast<const uint16_t*>(qkv), rq, rk, cs, B * T,
-      T, H, Dh);
+  const long long warps = (long long)B * T;
+  if (Dh > 128)
+    rope_qknorm_bwd_kernel<2><<<blocks_for_warps(warps, 256), 256, 0, s>>>(
+        reinterpret_cast<uint16_t*>(dqkv), reinterpret_cast<const uint16_t*>(qkv), rq, rk, cs, B * T,
+        T, H, Dh);
+  else
+    rope_qknorm_bwd_kernel<1><<<blocks_for_warps(warps, 256), 256, 0, s>>>(
+        reinterpret_cast<uint16_t*>(dqkv), reinterpret_cast<const uint16_t*>(qkv), rq, rk, cs, B * T,
+        T, H, Dh);
   count_launch();
   GPT_CUDA_TRY(cudaGetLastError());
   return GPT_OK;
