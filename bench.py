@@ -352,7 +352,7 @@ def run_kernel(args):
         unit_desc = f"GEMM {args.gemm_op} M={M} N={N} K={K}"
     else:
         T, Dh, W = (int(x) for x in args.attn.split(","))
-        H = 8
+        H = args.attn_heads
         Bt = max(1, args.attn_rows // (H * T))
         q, k, v, do = (torch.from_numpy(a).to(dev).to(torch.bfloat16)
                        for a in make_attention_inputs(Bt, H, T, Dh))
@@ -405,6 +405,7 @@ def main():
     ap.add_argument("--attn", default="2048,128,0", help="T,Dh,window (window 0 = full causal)")
     ap.add_argument("--attn-pass", default="fwd", choices=["fwd", "bwd"])
     ap.add_argument("--attn-rows", type=int, default=1 << 21, help="batch·heads·seq of the attention workload")
+    ap.add_argument("--attn-heads", type=int, default=8)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -40,6 +40,11 @@ struct AttnArgs {
   float* lse;
   float* delta;
   int* status;
+  // optional QK-norm + RoPE backward fused into the dq / dk epilogues (rho_q == nullptr: off):
+  // q̃ = RMS_Dh(RoPE(q)), so dq = Rᵀ·rho·(dq̃ − q̃·mean(q̃·dq̃)), likewise for k
+  const float* rho_q;      // [B·T, H]
+  const float* rho_k;
+  const float* cos_sin;    // [T, Dh/2, 2]
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -580,6 +585,80 @@ __device__ __forceinline__ void mma_acc_from_tmem(uint32_t d_tmem, uint32_t a_tm
                 sdesc_sw128(b_base + kk * 2048, 64 * 128, 1024), idesc, (!first || kk > 0) ? 1u : 0u);
 }
 
+
+// Norm backward and inverse RoPE of one head row: g (fp32, DH values, in place) is the gradient of
+// ŷ = RMS_Dh(RoPE(y)); ŷ is streamed in 8-element vectors from the swizzled [DH/64][ROWS][64] tile
+// in shared memory.  On return g holds the gradient with respect to the pre-RoPE row.
+template <int ROWS>
+__device__ __forceinline__ void load_y8(const uint8_t* tile, int r, int col, float (&y)[8]) {
+  const int c = col >> 6, u = (col & 63) >> 3;
+  const uint4 v = *reinterpret_cast<const uint4*>(tile + c * ROWS * 128 + r * 128 + ((u ^ (r & 7)) << 4));
+  y[0] = bf_lo(v.x); y[1] = bf_hi(v.x); y[2] = bf_lo(v.y); y[3] = bf_hi(v.y);
+  y[4] = bf_lo(v.z); y[5] = bf_hi(v.z); y[6] = bf_lo(v.w); y[7] = bf_hi(v.w);
+}
+
+// The gradient of the head row lives in tensor memory (columns taddr .. taddr+DH−1 of this thread's
+// lane, times `scale`).  Two passes: the dot product with ŷ, then, pair chunk by pair chunk, the
+// norm backward and the inverse rotation, written as bf16 to dst (when `store`).  Must be called
+// by whole warps (tcgen05.ld is warp-wide).
+template <int DH, int ROWS>
+__device__ __forceinline__ void qknorm_rope_bwd_tmem(uint32_t taddr, float scale, const uint8_t* tile,
+                                                     int r, float rho, const float* cs_t, uint16_t* dst,
+                                                     bool store) {
+  constexpr int HALF = DH / 2;
+  float dot = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < DH / 32; ++c) {
+    uint32_t v[32];
+    tmem_ld32(taddr + 32 * c, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      float y[8];
+      load_y8<ROWS>(tile, r, 32 * c + 8 * jj, y);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dot += __uint_as_float(v[8 * jj + e]) * y[e];
+    }
+  }
+  dot = dot * scale / (float)DH;
+  const float4* cs4 = reinterpret_cast<const float4*>(cs_t);
+#pragma unroll 1
+  for (int c = 0; c < HALF / 32; ++c) {
+    uint32_t va[32], vb[32];
+    tmem_ld32(taddr + 32 * c, va);
+    tmem_ld32(taddr + HALF + 32 * c, vb);
+    tmem_ld_wait();
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j = 32 * c + 8 * jj;
+      float ya[8], yb[8], oa[8], ob[8];
+      load_y8<ROWS>(tile, r, j, ya);
+      load_y8<ROWS>(tile, r, j + HALF, yb);
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const float4 w = cs4[(j + e) / 2];  // cos_j, sin_j, cos_{j+1}, sin_{j+1}
+        const float a0 = rho * (__uint_as_float(va[8 * jj + e]) * scale - ya[e] * dot);
+        const float b0 = rho * (__uint_as_float(vb[8 * jj + e]) * scale - yb[e] * dot);
+        const float a1 = rho * (__uint_as_float(va[8 * jj + e + 1]) * scale - ya[e + 1] * dot);
+        const float b1 = rho * (__uint_as_float(vb[8 * jj + e + 1]) * scale - yb[e + 1] * dot);
+        oa[e] = a0 * w.x + b0 * w.y;
+        ob[e] = -a0 * w.y + b0 * w.x;
+        oa[e + 1] = a1 * w.z + b1 * w.w;
+        ob[e + 1] = -a1 * w.w + b1 * w.z;
+      }
+      if (store) {
+        uint4 pa, pb;
+        pa.x = pack_bf2(oa[0], oa[1]); pa.y = pack_bf2(oa[2], oa[3]);
+        pa.z = pack_bf2(oa[4], oa[5]); pa.w = pack_bf2(oa[6], oa[7]);
+        pb.x = pack_bf2(ob[0], ob[1]); pb.y = pack_bf2(ob[2], ob[3]);
+        pb.z = pack_bf2(ob[4], ob[5]); pb.w = pack_bf2(ob[6], ob[7]);
+        *reinterpret_cast<uint4*>(dst + j) = pa;
+        *reinterpret_cast<uint4*>(dst + j + HALF) = pb;
+      }
+    }
+  }
+}
+
 template <int DH>
 __global__ void __launch_bounds__(320, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
@@ -748,13 +827,18 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_before();
       mbar_arrive(&p_full[bf]);
     }
-    // epilogue: dV and dK rows of this key tile
+    // epilogue: half 0 writes the dV row, half 1 the dK row of each key
     if (ok) ok = mbar_wait(done, 0, abort_flag, a.status);
     if (ok) {
       tc_fence_after();
       const long long off = b * a.sb_o + h * a.sh_o + (long long)key * a.st_o;
-      {
-        const int part = half;  // half 0 writes dV, half 1 writes dK
+      if (half == 1 && a.rho_k != nullptr) {
+        const bool valid = key < T;
+        const float rho = valid ? a.rho_k[((long long)b * T + key) * a.H + h] : 0.f;
+        qknorm_rope_bwd_tmem<DH, 128>(tmem + lane_off + S::TM_ACC + DH, a.scale, smem + S::OFF_A, kr,
+                                      rho, a.cos_sin + (size_t)(valid ? key : 0) * DH, a.dk + off, valid);
+      } else {
+        const int part = half;
         uint16_t* dst = (part == 0 ? a.dv : a.dk) + off;
         const float sc = (part == 0) ? 1.f : a.scale;
 #pragma unroll 1
@@ -932,6 +1016,15 @@ __global__ void __launch_bounds__(320, 1)
     if (ok) {
       tc_fence_after();
       uint16_t* dst = a.o + b * a.sb_o + h * a.sh_o + (long long)t * a.st_o;
+      if (a.rho_q != nullptr) {
+        // half 0 takes the whole row: the norm backward needs all DH columns
+        if (half == 0) {
+          const bool valid = t < T;
+          const float rho = valid ? a.rho_q[((long long)b * T + t) * a.H + h] : 0.f;
+          qknorm_rope_bwd_tmem<DH, 128>(tmem + lane_off + S::TM_ACC, a.scale, smem + S::OFF_A, row, rho,
+                                        a.cos_sin + (size_t)(valid ? t : 0) * DH, dst, valid);
+        }
+      } else {
 #pragma unroll 1
       for (int c = half * (DH / 64); c < (half + 1) * (DH / 64); ++c) {
         uint32_t r[32];
@@ -948,6 +1041,7 @@ __global__ void __launch_bounds__(320, 1)
             *reinterpret_cast<uint4*>(dst + 32 * c + 8 * u) = w;
           }
         }
+      }
       }
     }
   }
@@ -996,16 +1090,18 @@ __global__ void attn_kmax_kernel(const uint16_t* __restrict__ k, float* __restri
 // ================================================================================================
 __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                                   float* __restrict__ delta, int B, int H, int T, int Dh,
-                                  long long sb, long long sh, long long st) {
+                                  long long sb, long long sh, long long st, long long sbd,
+                                  long long shd, long long std_) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const long long rows = (long long)B * H * T;
   if (warp >= rows) return;
   const int t = warp % T, h = (warp / T) % H, b = warp / (T * H);
   const long long off = b * sb + h * sh + (long long)t * st;
+  const long long offd = b * sbd + h * shd + (long long)t * std_;
   float acc = 0.f;
   for (int j = 2 * lane; j < Dh; j += 64) {
     const uint32_t x = *reinterpret_cast<const uint32_t*>(o + off + j);
-    const uint32_t y = *reinterpret_cast<const uint32_t*>(dout + off + j);
+    const uint32_t y = *reinterpret_cast<const uint32_t*>(dout + offd + j);
     acc += bf_lo(x) * bf_lo(y) + bf_hi(x) * bf_hi(y);
   }
 #pragma unroll
@@ -1473,25 +1569,29 @@ gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, f
   return launch_fwd_tc<64>(mq2, mk2, mv2, a, kmax_scratch, kconst, stream);
 }
 
+// Strides: (sbq, shq, stq) for q, k, v; (sbg, shg, stg) for dq, dk, dv; (sbo, sho, sto) for o;
+// (sbd, shd, std_) for dO.
 gpt_status attention_bwd(const void* q, const void* k, const void* v, const void* o,
                          const void* dout, const float* lse, float* delta, void* dq, void* dk,
                          void* dv, int B, int H, int T, int Dh, int window, long long sbq,
-                         long long shq, long long stq, long long sbo, long long sho, long long sto,
-                         int* status, cudaStream_t stream) {
+                         long long shq, long long stq, long long sbg, long long shg, long long stg,
+                         long long sbo, long long sho, long long sto, long long sbd, long long shd,
+                         long long std_, int* status, cudaStream_t stream, const float* rho_q,
+                         const float* rho_k, const float* cos_sin) {
   GPT_TRY(check_attn(q, B, H, T, Dh, sbq, shq, stq));
   GPT_TRY(check_attn(k, B, H, T, Dh, sbq, shq, stq));
   GPT_TRY(check_attn(v, B, H, T, Dh, sbq, shq, stq));
-  GPT_TRY(check_attn(dq, B, H, T, Dh, sbq, shq, stq));
-  GPT_TRY(check_attn(dk, B, H, T, Dh, sbq, shq, stq));
-  GPT_TRY(check_attn(dv, B, H, T, Dh, sbq, shq, stq));
+  GPT_TRY(check_attn(dq, B, H, T, Dh, sbg, shg, stg));
+  GPT_TRY(check_attn(dk, B, H, T, Dh, sbg, shg, stg));
+  GPT_TRY(check_attn(dv, B, H, T, Dh, sbg, shg, stg));
   GPT_TRY(check_attn(o, B, H, T, Dh, sbo, sho, sto));
-  GPT_TRY(check_attn(dout, B, H, T, Dh, sbo, sho, sto));
+  GPT_TRY(check_attn(dout, B, H, T, Dh, sbd, shd, std_));
   if (!lse || !delta) return GPT_ERR_INVALID_ARG;
   CUtensorMap mq, mk, mv, mdo;
   if (!make_head_map(&mq, q, B, H, T, Dh, sbq, shq, stq, 64) ||
       !make_head_map(&mk, k, B, H, T, Dh, sbq, shq, stq, 64) ||
       !make_head_map(&mv, v, B, H, T, Dh, sbq, shq, stq, 64) ||
-      !make_head_map(&mdo, dout, B, H, T, Dh, sbo, sho, sto, 64))
+      !make_head_map(&mdo, dout, B, H, T, Dh, sbd, shd, std_, 64))
     return GPT_ERR_UNSUPPORTED_SHAPE;
   {
     const long long rows = (long long)B * H * T;
@@ -1499,7 +1599,7 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
     const long long blocks = (rows * 32 + threads - 1) / threads;
     attn_delta_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
         reinterpret_cast<const uint16_t*>(o), reinterpret_cast<const uint16_t*>(dout), delta, B, H,
-        T, Dh, sbo, sho, sto);
+        T, Dh, sbo, sho, sto, sbd, shd, std_);
     count_launch();
     GPT_CUDA_TRY(cudaGetLastError());
   }
@@ -1511,7 +1611,11 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   a.lse = const_cast<float*>(lse);
   a.delta = delta;
   a.status = status;
-  a.sb_o = sbq; a.sh_o = shq; a.st_o = stq;  // dq/dk/dv share the q/k/v strides
+  a.sb_o = sbg; a.sh_o = shg; a.st_o = stg;  // strides of the dq/dk/dv outputs
+  a.rho_q = rho_q;
+  a.rho_k = rho_k;
+  a.cos_sin = cos_sin;
+  if (rho_q && (Dh == 32 || !rho_k || !cos_sin)) return GPT_ERR_INVALID_ARG;
   dim3 grid((T + 63) / 64, H, B);
   a.dk = reinterpret_cast<uint16_t*>(dk);
   a.dv = reinterpret_cast<uint16_t*>(dv);
@@ -1519,11 +1623,11 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   CUtensorMap m128[4], m64[4];
   const void* src[4] = {q, k, v, dout};
   for (int i = 0; i < 4; ++i) {
-    const bool is_o = (i == 3);
-    if (!make_head_map(&m128[i], src[i], B, H, T, Dh, is_o ? sbo : sbq, is_o ? sho : shq,
-                       is_o ? sto : stq, 128) ||
-        !make_head_map(&m64[i], src[i], B, H, T, Dh, is_o ? sbo : sbq, is_o ? sho : shq,
-                       is_o ? sto : stq, 64))
+    const bool is_do = (i == 3);
+    if (!make_head_map(&m128[i], src[i], B, H, T, Dh, is_do ? sbd : sbq, is_do ? shd : shq,
+                       is_do ? std_ : stq, 128) ||
+        !make_head_map(&m64[i], src[i], B, H, T, Dh, is_do ? sbd : sbq, is_do ? shd : shq,
+                       is_do ? std_ : stq, 64))
       return GPT_ERR_UNSUPPORTED_SHAPE;
   }
   if (Dh == 128) GPT_TRY(launch_bwd_tc<128>(m128, m64, a, dq, stream));
@@ -1566,7 +1670,8 @@ gpt_status attention_bwd_noalloc(const void* q, const void* k, const void* v, co
   float* delta = nullptr;
   GPT_TRY(noalloc_delta_ptr(&delta));
   return attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, T, Dh, window, sbq, shq, stq,
-                       sbo, sho, sto, status, stream);
+                       sbq, shq, stq, sbo, sho, sto, sbo, sho, sto, status, stream, nullptr,
+                       nullptr, nullptr);
 }
 
 }  // namespace gpt
@@ -1587,7 +1692,8 @@ extern "C" gpt_status gpt_attention_bwd(const void* q, const void* k, const void
                                         long long st_qkv, long long sb_o, long long sh_o,
                                         long long st_o, int* status, void* stream) {
   return gpt::attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, T, Dh, window, sb_qkv,
-                            sh_qkv, st_qkv, sb_o, sh_o, st_o, status, gpt::as_stream(stream));
+                            sh_qkv, st_qkv, sb_qkv, sh_qkv, st_qkv, sb_o, sh_o, st_o, sb_o, sh_o,
+                            st_o, status, gpt::as_stream(stream), nullptr, nullptr, nullptr);
 }
 
 extern "C" gpt_status gpt_attention_bwd_noalloc(const void* q, const void* k, const void* v,

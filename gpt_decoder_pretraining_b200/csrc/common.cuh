@@ -20,8 +20,11 @@ __device__ __forceinline__ uint16_t f2bf(float f) {
   __nv_bfloat16 b = __float2bfloat16_rn(f);
   return *reinterpret_cast<uint16_t*>(&b);
 }
+// Two fp32 values to a bf16 pair (lo in bits 0..15), one round-to-nearest-even conversion.
 __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
-  return (uint32_t)f2bf(lo) | ((uint32_t)f2bf(hi) << 16);
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }

@@ -32,7 +32,13 @@ constexpr int BN = 256;   // columns per tile (each CTA stages 128 rows of B)
 constexpr int BK = 64;
 constexpr int GEMM_THREADS = 192;
 
-enum : int { EPI_CE_STATS = 100, EPI_CE_GRAD = 101, EPI_F32_RED = 102 };
+enum : int {
+  EPI_CE_STATS = 100,
+  EPI_CE_GRAD = 101,
+  EPI_F32_RED = 102,
+  EPI_BF16_HEADS = 103,   // bf16 store with row m = b·T + t, column n = h·Dh + j sent to [B, H, T, Dh]
+  EPI_QKV_ROPE = 200      // + Dh: RoPE + QK-norm of the q and k heads, all three to [3][B][H][T][Dh]
+};
 
 struct GemmArgs {
   int M, N, K;
@@ -45,6 +51,11 @@ struct GemmArgs {
   int ldaux;
   int* status;
   CeArgs ce;
+  // head-major outputs (EPI_BF16_HEADS, EPI_QKV_ROPE + Dh)
+  int T, H, Dh, d;
+  const float* cs;        // [T, Dh/2, 2] cos / sin
+  float* rho_q;           // [M, H]
+  float* rho_k;
 };
 
 struct GemmShape {
@@ -309,6 +320,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           }
         }
       }
+      if constexpr (EPI > EPI_QKV_ROPE) {
+        // one head (DH columns) at a time: q and k heads get RoPE + QK-norm, v heads a plain cast
+        constexpr int DH = EPI - EPI_QKV_ROPE, HALF = DH / 2;
+        const long long bhtd = (long long)(args.M / args.T) * args.H * args.T * DH;
+        const int b = m / args.T, t = m % args.T;
+#pragma unroll 1
+        for (int hh = 0; hh < BN / DH; ++hh) {
+          const int n_head = tn * BN + hh * DH;
+          float xh[DH];
+#pragma unroll
+          for (int c = 0; c < DH / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + hh * DH + c * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) xh[c * 32 + j] = __uint_as_float(r[j]);
+          }
+          if (m >= args.M || n_head >= args.N) continue;
+          const int region = n_head / args.d;            // 0 q, 1 k, 2 v
+          const int h = (n_head % args.d) / DH;
+          if (region < 2) {
+            const float4* cs4 = reinterpret_cast<const float4*>(args.cs + (size_t)t * DH);
+            float ss = 0.f;
+#pragma unroll
+            for (int j = 0; j < HALF; j += 2) {
+              const float4 w = cs4[j / 2];  // cos_j, sin_j, cos_{j+1}, sin_{j+1}
+              const float a0 = xh[j], b0 = xh[j + HALF], a1 = xh[j + 1], b1 = xh[j + 1 + HALF];
+              xh[j] = a0 * w.x - b0 * w.y;
+              xh[j + HALF] = a0 * w.y + b0 * w.x;
+              xh[j + 1] = a1 * w.z - b1 * w.w;
+              xh[j + 1 + HALF] = a1 * w.w + b1 * w.z;
+              ss += xh[j] * xh[j] + xh[j + HALF] * xh[j + HALF] + xh[j + 1] * xh[j + 1] +
+                    xh[j + 1 + HALF] * xh[j + 1 + HALF];
+            }
+            const float rr = rsqrtf(ss / (float)DH + 1e-6f);
+#pragma unroll
+            for (int j = 0; j < DH; ++j) xh[j] *= rr;
+            (region == 0 ? args.rho_q : args.rho_k)[(size_t)m * args.H + h] = rr;
+          }
+          uint16_t* dst = reinterpret_cast<uint16_t*>(args.C) + region * bhtd +
+                          (((long long)b * args.H + h) * args.T + t) * DH;
+#pragma unroll
+          for (int j = 0; j < DH; j += 8) {
+            uint4 o;
+            o.x = pack_bf2(xh[j], xh[j + 1]);
+            o.y = pack_bf2(xh[j + 2], xh[j + 3]);
+            o.z = pack_bf2(xh[j + 4], xh[j + 5]);
+            o.w = pack_bf2(xh[j + 6], xh[j + 7]);
+            *reinterpret_cast<uint4*>(dst + j) = o;
+          }
+        }
+      } else {
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
@@ -346,9 +409,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
             }
             epilogue_store<GPT_EPI_BF16>(args, m, n0, v);
           }
+        } else if (EPI == EPI_BF16_HEADS) {
+          if (m < args.M && n0 < args.N) {
+            const int b = m / args.T, t = m % args.T, h = n0 / args.Dh, j0 = n0 % args.Dh;
+            uint16_t* dst = reinterpret_cast<uint16_t*>(args.C) +
+                            (((long long)b * args.H + h) * args.T + t) * args.Dh + j0;
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              uint4 o;
+              o.x = pack_bf2(v[j], v[j + 1]);
+              o.y = pack_bf2(v[j + 2], v[j + 3]);
+              o.z = pack_bf2(v[j + 4], v[j + 5]);
+              o.w = pack_bf2(v[j + 6], v[j + 7]);
+              *reinterpret_cast<uint4*>(dst + j) = o;
+            }
+          }
         } else {
           if (m < args.M && n0 < args.N) epilogue_store<EPI>(args, m, n0, v);
         }
+      }
       }
       if (EPI == EPI_CE_STATS && m < args.M) {
         args.ce.stats[(size_t)m * args.ce.stats_ld + args.ce.stats_col0 + tn] =
@@ -494,6 +573,43 @@ gpt_status gemm_launch(int op, int epi, int M, int N, int K, const void* A, int 
   return dispatch_epi<true, true>(epi, ma, mb, a, stream);
 }
 
+gpt_status gemm_heads_launch(int op, int M, int N, int K, const void* A, int lda, const void* B,
+                             int ldb, void* heads, int T, int H, int Dh, int* status,
+                             cudaStream_t stream) {
+  GPT_TRY(check_gemm_args(op, M, N, K, A, lda, B, ldb, heads, N));
+  if (T <= 0 || H <= 0 || Dh <= 0 || (Dh % 32) || H * Dh != N || (M % T)) return GPT_ERR_INVALID_ARG;
+  const bool a_mn = (op == GPT_GEMM_TN), b_mn = (op != GPT_GEMM_NT);
+  CUtensorMap ma, mb;
+  if (!make_operand_map(&ma, A, a_mn, M, K, lda)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if (!make_operand_map(&mb, B, b_mn, N, K, ldb)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  GemmArgs a{};
+  fill_args(a, M, N, K, 1);
+  a.C = heads; a.ldc = N; a.status = status;
+  a.T = T; a.H = H; a.Dh = Dh;
+  if (op == GPT_GEMM_NT) return launch_inst<false, false, EPI_BF16_HEADS>(ma, mb, a, stream);
+  if (op == GPT_GEMM_NN) return launch_inst<false, true, EPI_BF16_HEADS>(ma, mb, a, stream);
+  return launch_inst<true, true, EPI_BF16_HEADS>(ma, mb, a, stream);
+}
+
+gpt_status gemm_qkv_rope_launch(int M, int d, const void* A, const void* Wqkv, void* heads,
+                                float* rho_q, float* rho_k, const float* cs, int T, int H, int Dh,
+                                int* status, cudaStream_t stream) {
+  const int N = 3 * d, K = d;
+  GPT_TRY(check_gemm_args(GPT_GEMM_NT, M, N, K, A, K, Wqkv, K, heads, N));
+  if (!rho_q || !rho_k || !cs || T <= 0 || H * Dh != d || (M % T)) return GPT_ERR_INVALID_ARG;
+  if (Dh != 32 && Dh != 64 && Dh != 128) return GPT_ERR_UNSUPPORTED_SHAPE;
+  CUtensorMap ma, mb;
+  if (!make_operand_map(&ma, A, false, M, K, K)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if (!make_operand_map(&mb, Wqkv, false, N, K, K)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  GemmArgs a{};
+  fill_args(a, M, N, K, 1);
+  a.C = heads; a.ldc = N; a.status = status;
+  a.T = T; a.H = H; a.Dh = Dh; a.d = d; a.cs = cs; a.rho_q = rho_q; a.rho_k = rho_k;
+  if (Dh == 128) return launch_inst<false, false, EPI_QKV_ROPE + 128>(ma, mb, a, stream);
+  if (Dh == 64) return launch_inst<false, false, EPI_QKV_ROPE + 64>(ma, mb, a, stream);
+  return launch_inst<false, false, EPI_QKV_ROPE + 32>(ma, mb, a, stream);
+}
+
 int gemm_ce_tile_n() { return BN; }
 
 gpt_status gemm_ce_launch(bool grad, int M, int N, int K, const void* A, int lda, const void* B,
@@ -513,6 +629,14 @@ gpt_status gemm_ce_launch(bool grad, int M, int N, int K, const void* A, int lda
 }
 
 }  // namespace gpt
+
+extern "C" gpt_status gpt_qkv_proj_rope(const void* r, const void* w_qkv, void* heads, float* rho_q,
+                                        float* rho_k, const float* cos_sin, int B, int T, int H,
+                                        int Dh, int* status, void* stream) {
+  if (B <= 0 || T <= 0 || H <= 0 || Dh <= 0) return GPT_ERR_INVALID_ARG;
+  return gpt::gemm_qkv_rope_launch(B * T, H * Dh, r, w_qkv, heads, rho_q, rho_k, cos_sin, T, H, Dh,
+                                   status, gpt::as_stream(stream));
+}
 
 extern "C" gpt_status gpt_gemm(int op, int epilogue, int M, int N, int K, const void* A, int lda,
                                const void* B, int ldb, void* C, int ldc, void* C2,

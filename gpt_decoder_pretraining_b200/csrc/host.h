@@ -59,4 +59,14 @@ gpt_status gemm_ce_launch(bool grad, int M, int N, int K, const void* A, int lda
                           cudaStream_t stream);
 int gemm_ce_tile_n();  // vocabulary columns per CE statistics tile
 
+// C (row m = b·T + t, column n = h·Dh + j) stored bf16 head-major at heads[((b·H + h)·T + t)·Dh + j].
+gpt_status gemm_heads_launch(int op, int M, int N, int K, const void* A, int lda, const void* B,
+                             int ldb, void* heads, int T, int H, int Dh, int* status,
+                             cudaStream_t stream);
+// [q|k|v] = A·W_qkvᵀ with RoPE + QK-norm applied to q and k, stored head-major as
+// heads[part][b][h][t][j]; rho_q / rho_k [M, H] receive the norm factors.
+gpt_status gemm_qkv_rope_launch(int M, int d, const void* A, const void* Wqkv, void* heads,
+                                float* rho_q, float* rho_k, const float* cs, int T, int H, int Dh,
+                                int* status, cudaStream_t stream);
+
 }  // namespace gpt

@@ -193,7 +193,9 @@ __global__ void __launch_bounds__(256) rope_qknorm_fwd_kernel(uint16_t* __restri
 
 // Backward: g = rho·(dŷ − ŷ·mean(ŷ·dŷ)) with ŷ the stored forward output, then the inverse
 // rotation (a, b) → (a cos + b sin, −a sin + b cos).  Same work split as the forward.
-template <int ROUNDS>
+// Y_HEADS: the forward output ŷ is read head-major, y[part][b][h][t][j], instead of from the
+// token-major [M, 3d] rows.
+template <int ROUNDS, bool Y_HEADS>
 __global__ void __launch_bounds__(256) rope_qknorm_bwd_kernel(uint16_t* __restrict__ dqkv, const uint16_t* __restrict__ qkv,
                                                               const float* __restrict__ rho_q, const float* __restrict__ rho_k,
                                                               const float* __restrict__ cs, int M, int T, int H, int Dh) {
@@ -226,8 +228,15 @@ __global__ void __launch_bounds__(256) rope_qknorm_bwd_kernel(uint16_t* __restri
           const size_t off = (u / H) * d + (u % H) * Dh + 2 * lane + 64 * rr;
           ga[k][rr] = *reinterpret_cast<const uint32_t*>(grow + off);
           gb[k][rr] = *reinterpret_cast<const uint32_t*>(grow + off + half);
-          ya[k][rr] = *reinterpret_cast<const uint32_t*>(yrow + off);
-          yb[k][rr] = *reinterpret_cast<const uint32_t*>(yrow + off + half);
+          const uint16_t* yp;
+          if (Y_HEADS) {
+            const long long b = m / T;
+            yp = qkv + (long long)(u / H) * M * d + ((b * H + (u % H)) * T + t) * Dh + 2 * lane + 64 * rr;
+          } else {
+            yp = yrow + off;
+          }
+          ya[k][rr] = *reinterpret_cast<const uint32_t*>(yp);
+          yb[k][rr] = *reinterpret_cast<const uint32_t*>(yp + half);
         }
       }
     }
@@ -513,19 +522,36 @@ gpt_status rope_qknorm_fwd(void* qkv, float* rq, float* rk, const float* cs, int
   return GPT_OK;
 }
 
+template <bool Y_HEADS>
+static void launch_rope_bwd(void* dqkv, const void* y, const float* rq, const float* rk,
+                            const float* cs, int B, int T, int H, int Dh, cudaStream_t s) {
+  const long long warps = (long long)B * T;
+  if (Dh > 128)
+    rope_qknorm_bwd_kernel<2, Y_HEADS><<<blocks_for_warps(warps, 256), 256, 0, s>>>(
+        reinterpret_cast<uint16_t*>(dqkv), reinterpret_cast<const uint16_t*>(y), rq, rk, cs, B * T,
+        T, H, Dh);
+  else
+    rope_qknorm_bwd_kernel<1, Y_HEADS><<<blocks_for_warps(warps, 256), 256, 0, s>>>(
+        reinterpret_cast<uint16_t*>(dqkv), reinterpret_cast<const uint16_t*>(y), rq, rk, cs, B * T,
+        T, H, Dh);
+}
+
+// y_heads: the forward output is stored head-major [2][B][H][T][Dh] (q̃ then k̃).
+gpt_status rope_qknorm_bwd_heads(void* dqkv, const void* y_heads, const float* rq, const float* rk,
+                                 const float* cs, int B, int T, int H, int Dh, cudaStream_t s) {
+  if (!dqkv || !y_heads || !rq || !rk || !cs) return GPT_ERR_INVALID_ARG;
+  GPT_TRY(check_rope(B, T, H, Dh));
+  launch_rope_bwd<true>(dqkv, y_heads, rq, rk, cs, B, T, H, Dh, s);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
 gpt_status rope_qknorm_bwd(void* dqkv, const void* qkv, const float* rq, const float* rk,
                            const float* cs, int B, int T, int H, int Dh, cudaStream_t s) {
   if (!dqkv || !qkv || !rq || !rk || !cs) return GPT_ERR_INVALID_ARG;
   GPT_TRY(check_rope(B, T, H, Dh));
-  const long long warps = (long long)B * T;
-  if (Dh > 128)
-    rope_qknorm_bwd_kernel<2><<<blocks_for_warps(warps, 256), 256, 0, s>>>(
-        reinterpret_cast<uint16_t*>(dqkv), reinterpret_cast<const uint16_t*>(qkv), rq, rk, cs, B * T,
-        T, H, Dh);
-  else
-    rope_qknorm_bwd_kernel<1><<<blocks_for_warps(warps, 256), 256, 0, s>>>(
-        reinterpret_cast<uint16_t*>(dqkv), reinterpret_cast<const uint16_t*>(qkv), rq, rk, cs, B * T,
-        T, H, Dh);
+  launch_rope_bwd<false>(dqkv, qkv, rq, rk, cs, B, T, H, Dh, s);
   count_launch();
   GPT_CUDA_TRY(cudaGetLastError());
   return GPT_OK;

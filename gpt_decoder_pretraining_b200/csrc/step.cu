@@ -27,6 +27,8 @@ gpt_status rope_qknorm_fwd(void* qkv, float* rq, float* rk, const float* cs, int
                            int Dh, cudaStream_t s);
 gpt_status rope_qknorm_bwd(void* dqkv, const void* qkv, const float* rq, const float* rk,
                            const float* cs, int B, int T, int H, int Dh, cudaStream_t s);
+gpt_status rope_qknorm_bwd_heads(void* dqkv, const void* y_heads, const float* rq, const float* rk,
+                                 const float* cs, int B, int T, int H, int Dh, cudaStream_t s);
 gpt_status embedding_fwd(const int32_t* tok, const void* wte, void* x, int M, int d, int V,
                          int* status, cudaStream_t s);
 size_t embedding_bwd_scratch_bytes(int M, int V);
@@ -44,8 +46,10 @@ gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, f
 gpt_status attention_bwd(const void* q, const void* k, const void* v, const void* o,
                          const void* dout, const float* lse, float* delta, void* dq, void* dk,
                          void* dv, int B, int H, int T, int Dh, int window, long long sbq,
-                         long long shq, long long stq, long long sbo, long long sho, long long sto,
-                         int* status, cudaStream_t stream);
+                         long long shq, long long stq, long long sbg, long long shg, long long stg,
+                         long long sbo, long long sho, long long sto, long long sbd, long long shd,
+                         long long std_, int* status, cudaStream_t stream, const float* rho_q,
+                         const float* rho_k, const float* cos_sin);
 
 static inline size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
 
@@ -256,8 +260,10 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
   uint16_t* x = reinterpret_cast<uint16_t*>(ws + p.x);
   uint16_t* xf = reinterpret_cast<uint16_t*>(ws + p.xf);
   float* rhof = reinterpret_cast<float*>(ws + p.rhof);
-  const long long qs_b = (long long)T * 3 * d, qs_h = Dh, qs_t = 3 * d;  // q/k/v inside qkv
-  const long long os_b = (long long)T * d, os_h = Dh, os_t = d;          // o / dO
+  const long long qs_b = (long long)T * 3 * d, qs_h = Dh, qs_t = 3 * d;  // dq/dk/dv inside dqkv
+  const long long os_b = (long long)T * d, os_h = Dh, os_t = d;          // o (token-major)
+  const long long hs_b = (long long)H * T * Dh, hs_h = (long long)T * Dh, hs_t = Dh;  // head-major
+  const long long bhtd = (long long)B * H * T * Dh;
 
   PROF(PROF_ROPE, 0, (double)T * Dh * 4, rope_table(rope, T, Dh, s));
   PROF(PROF_EMBED, 0, 4.0 * (double)M * d, embedding_fwd(tokens, W(0), x, M, d, V, status, s));
@@ -277,11 +283,12 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
     uint16_t* act = reinterpret_cast<uint16_t*>(at(p.act, l));
     uint16_t* hsq = reinterpret_cast<uint16_t*>(at(p.hsq, l));
     PROF(PROF_NORM, 0, 4.0 * (double)M * d + 4.0 * M, rmsnorm_fwd(x, r1, rho1, M, d, s));
-    PROF(PROF_GEMM, gemm_flops(M, 3.0 * d, d), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_BF16, M, 3 * d, d, r1, d, W(wq), d, qkv, 3 * d,
-                        nullptr, nullptr, 0, status, s));
-    PROF(PROF_ROPE, 0, 8.0 * (double)M * d, rope_qknorm_fwd(qkv, rq, rk, rope, B, T, H, Dh, s));
-    PROF(PROF_ATTN_FWD, 4.0 * Dh * H * B * attn_pairs(T, st->window[l]), 0, attention_fwd(qkv, qkv + d, qkv + 2 * d, o, lse, B, H, T, Dh, st->window[l], qs_b,
-                          qs_h, qs_t, os_b, os_h, os_t, status, s, nullptr));
+    // q̃, k̃, v head-major [3][B][H][T][Dh]; RoPE + QK-norm fused into the projection epilogue
+    PROF(PROF_GEMM, gemm_flops(M, 3.0 * d, d), 0,
+         gemm_qkv_rope_launch(M, d, r1, W(wq), qkv, rq, rk, rope, T, H, Dh, status, s));
+    PROF(PROF_ATTN_FWD, 4.0 * Dh * H * B * attn_pairs(T, st->window[l]), 0,
+         attention_fwd(qkv, qkv + bhtd, qkv + 2 * bhtd, o, lse, B, H, T, Dh, st->window[l], hs_b,
+                       hs_h, hs_t, os_b, os_h, os_t, status, s, nullptr));
     PROF(PROF_GEMM, gemm_flops(M, d, d), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_RESID, M, d, d, o, d, W(wq + 1), d, x, d, nullptr,
                         nullptr, 0, status, s));
     PROF(PROF_NORM, 0, 4.0 * (double)M * d + 4.0 * M, rmsnorm_fwd(x, r2, rho2, M, d, s));
@@ -354,14 +361,19 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
                         nullptr, 0, status, s));
     PROF(PROF_NORM, 0, 14.0 * (double)M * d, rmsnorm_bwd(dr, 0, r2, rho2, gx, gxb, 1, M, d, s));
     // attention
-    PROF(PROF_GEMM, gemm_flops(M, d, d), 0, gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, d, gxb, d, W(wq + 1), d, dO, d, nullptr,
-                        nullptr, 0, status, s));
+    PROF(PROF_GEMM, gemm_flops(M, d, d), 0,
+         gemm_heads_launch(GPT_GEMM_NN, M, d, d, gxb, d, W(wq + 1), d, dO, T, H, Dh, status, s));
     PROF(PROF_GEMM, gemm_flops(d, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, d, d, M, gxb, d, o, d, G(wq + 1), d, nullptr,
                         nullptr, 0, status, s));
-    PROF(PROF_ATTN_BWD, 8.0 * Dh * H * B * attn_pairs(T, st->window[l]), 0, attention_bwd(qkv, qkv + d, qkv + 2 * d, o, dO, lse, delta, dqkv, dqkv + d,
-                          dqkv + 2 * d, B, H, T, Dh, st->window[l], qs_b, qs_h, qs_t, os_b, os_h,
-                          os_t, status, s));
-    PROF(PROF_ROPE, 0, 12.0 * (double)M * d, rope_qknorm_bwd(dqkv, qkv, rq, rk, rope, B, T, H, Dh, s));
+    PROF(PROF_ATTN_BWD, 8.0 * Dh * H * B * attn_pairs(T, st->window[l]), 0,
+         attention_bwd(qkv, qkv + bhtd, qkv + 2 * bhtd, o, dO, lse, delta, dqkv, dqkv + d,
+                       dqkv + 2 * d, B, H, T, Dh, st->window[l], hs_b, hs_h, hs_t, qs_b, qs_h,
+                       qs_t, os_b, os_h, os_t, hs_b, hs_h, hs_t, status, s,
+                       Dh == 32 ? nullptr : rq, rk, rope));
+    if (Dh == 32) {  // the mma.sync path for head_dim 32 has no fused QK-norm/RoPE backward
+      PROF(PROF_ROPE, 0, 12.0 * (double)M * d,
+           rope_qknorm_bwd_heads(dqkv, qkv, rq, rk, rope, B, T, H, Dh, s));
+    }
     PROF(PROF_GEMM, gemm_flops(3.0 * d, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, 3 * d, d, M, dqkv, 3 * d, r1, d, G(wq), d,
                         nullptr, nullptr, 0, status, s));
     PROF(PROF_GEMM, gemm_flops(M, d, 3.0 * d), 0, gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, 3 * d, dqkv, 3 * d, W(wq), d, dr, d,

@@ -31,7 +31,7 @@ EXPORTED = [
     "gpt_param_layout", "gpt_step_create", "gpt_step_destroy", "gpt_step_workspace_bytes",
     "gpt_step_fwd_bwd", "gpt_step_status", "gpt_strerror", "gpt_step_last_launch_count",
     "gpt_step_set_profiling", "gpt_step_profile",
-    "gpt_gemm", "gpt_rmsnorm_fwd", "gpt_rmsnorm_bwd", "gpt_rope_qknorm_fwd", "gpt_rope_qknorm_bwd",
+    "gpt_gemm", "gpt_qkv_proj_rope", "gpt_rmsnorm_fwd", "gpt_rmsnorm_bwd", "gpt_rope_qknorm_fwd", "gpt_rope_qknorm_bwd",
     "gpt_rope_table", "gpt_attention_fwd", "gpt_attention_bwd", "gpt_attention_bwd_noalloc",
     "gpt_embedding_fwd",
     "gpt_embedding_bwd_scratch_bytes", "gpt_embedding_bwd", "gpt_lmhead_ce_scratch_bytes",
@@ -77,6 +77,7 @@ def lib():
         L.gpt_step_profile.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64),
                                        ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double), i32]
         L.gpt_gemm.argtypes = [i32, i32, i32, i32, i32, vp, i32, vp, i32, vp, i32, vp, vp, i32, vp, vp]
+        L.gpt_qkv_proj_rope.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp]
         L.gpt_rmsnorm_fwd.argtypes = [vp, vp, vp, i32, i32, vp]
         L.gpt_rmsnorm_bwd.argtypes = [vp, i32, vp, vp, vp, vp, i32, i32, i32, vp]
         L.gpt_rope_qknorm_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp]
@@ -203,6 +204,13 @@ def gemm(op: int, epi: int, A, B, C, M: int, N: int, K: int, C2=None, aux=None, 
     ldaux = aux.shape[-1] if aux is not None else 0
     _check(lib().gpt_gemm(op, epi, M, N, K, A.data_ptr(), lda, B.data_ptr(), ldb, C.data_ptr(), ldc,
                           _ptr(C2), _ptr(aux), ldaux, _ptr(status), _stream()), "gpt_gemm")
+
+
+def qkv_proj_rope(r, w_qkv, heads, rho_q, rho_k, cs, B, T, H, Dh, status=None):
+    """gpt_qkv_proj_rope: QKV projection + RoPE + QK-norm, head-major output [3][B][H][T][Dh]."""
+    _check(lib().gpt_qkv_proj_rope(r.data_ptr(), w_qkv.data_ptr(), heads.data_ptr(), rho_q.data_ptr(),
+                                   rho_k.data_ptr(), cs.data_ptr(), B, T, H, Dh, _ptr(status), _stream()),
+           "qkv_proj_rope")
 
 
 def rmsnorm_fwd(x, y, rho):

@@ -142,6 +142,15 @@ gpt_status gpt_gemm(int op, int epilogue, int M, int N, int K, const void* A, in
                     const void* B, int ldb, void* C, int ldc, void* C2, const void* aux,
                     int ldaux, int* status, void* stream);
 
+/* Fused QKV projection with RoPE + QK-norm, the step's forward entry into attention:
+ * [q | k | v] = r·W_qkvᵀ (r bf16 [B·T, d], W_qkv bf16 [3d, d], d = H·Dh); each q and k head becomes
+ * RMS_Dh(RoPE(·, t)) as in gpt_rope_qknorm_fwd; all three are stored head-major in `heads`
+ * (bf16 [3][B][H][T][Dh]).  rho_q, rho_k fp32 [B·T, H]; cos_sin from gpt_rope_table.
+ * Dh ∈ {32, 64, 128}. */
+gpt_status gpt_qkv_proj_rope(const void* r, const void* w_qkv, void* heads, float* rho_q,
+                             float* rho_k, const float* cos_sin, int B, int T, int H, int Dh,
+                             int* status, void* stream);
+
 /* RMSNorm forward over rows of d (bf16 in/out), y = x·rho, rho = 1/sqrt(mean(x²)+1e-6) (fp32). */
 gpt_status gpt_rmsnorm_fwd(const void* x, void* y, float* rho, int rows, int d, void* stream);
 

@@ -168,6 +168,35 @@ def test_rope_qknorm_fwd_bwd(B, T, H, Dh):
             assert_close_rel(gd[b, :, part], ref, rel=1e-2, what=f"bwd part {part}")
 
 
+@pytest.mark.parametrize("B,T,H,Dh", [(1, 130, 2, 128), (2, 64, 3, 64), (1, 96, 4, 32)])
+def test_qkv_proj_rope_matches_gemm_then_rope(B, T, H, Dh):
+    """The fused projection + RoPE + QK-norm equals the oracle's rope/rmsnorm of r·W_qkvᵀ."""
+    rng = np.random.default_rng(B + T + H + Dh)
+    d = H * Dh
+    r = randn(rng, B * T, d)
+    w = randn(rng, 3 * d, d, scale=0.05)
+    cs = torch.empty(T * Dh, dtype=torch.float32, device="cuda")
+    S.rope_table(cs, T, Dh)
+    heads = torch.zeros(3, B, H, T, Dh, dtype=torch.bfloat16, device="cuda")
+    rq = torch.zeros(B * T * H, dtype=torch.float32, device="cuda")
+    rk = torch.zeros_like(rq)
+    S.qkv_proj_rope(bf16_tensor(r), bf16_tensor(w), heads, rq, rk, cs, B, T, H, Dh)
+    torch.cuda.synchronize()
+    qkv = (r @ w.T).reshape(B, T, 3, H, Dh)
+    cos, sin = O.rope_angles(T, Dh, np.float64)
+    got = to_np(heads)  # [3, B, H, T, Dh]
+    for b in range(B):
+        for part in range(3):
+            x = qkv[b, :, part]  # [T, H, Dh]
+            if part < 2:
+                ref, rho = O.rmsnorm(O.rope(x, cos, sin))
+                r_got = to_np(rq if part == 0 else rk).reshape(B, T, H)[b]
+                np.testing.assert_allclose(r_got, rho[..., 0], rtol=2e-2)
+            else:
+                ref = x
+            assert_close_rel(got[part, b].transpose(1, 0, 2), ref, rel=2e-2, what=f"part {part}")
+
+
 # --------------------------------------------------------------------------------------------------
 # attention
 # --------------------------------------------------------------------------------------------------
