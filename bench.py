@@ -178,6 +178,25 @@ def run_reference(args, cfg):
 
 
 # ------------------------------------------------------------------------------------------------
+# multi-rank bookkeeping (replicas: no collective on the data path)
+# ------------------------------------------------------------------------------------------------
+def max_over_ranks(values, world, device="cpu"):
+    """Element-wise maximum of per-rank timings (the slowest rank sets the job's time)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def whole_job_rate(units_per_rank_step, world, ms_per_step):
+    """Units all ranks processed per second: every rank does units_per_rank_step per step."""
+    return units_per_rank_step * world / (ms_per_step / 1e3)
+
+
+# ------------------------------------------------------------------------------------------------
 # GPU arm
 # ------------------------------------------------------------------------------------------------
 def run_ours(args, cfg):
@@ -258,14 +277,10 @@ def run_ours(args, cfg):
     barrier()
     ms_e2e = f0.elapsed_time(f1) / args.steps
 
-    if world > 1:
-        t = torch.tensor([ms, ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, ms_e2e = float(t[0]), float(t[1])
-
+    ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, dev)
     tokens_step = cfg.batch * cfg.seq_len
-    value = tokens_step * world / (ms / 1e3)
-    value_e2e = tokens_step * world / (ms_e2e / 1e3)
+    value = whole_job_rate(tokens_step, world, ms)
+    value_e2e = whole_job_rate(tokens_step, world, ms_e2e)
     fpt = cfg.flops_per_token()
     mfu = fpt * value / (world * B200_DENSE_BF16_PEAK)
 
@@ -360,7 +375,7 @@ def run_kernel(args):
         lse = torch.empty(Bt, H, T, device=dev)
         strides = (H * T * Dh, T * Dh, Dh)
         dq, dk, dv = (torch.empty_like(q) for _ in range(3))
-        delta = torch.empty(Bt, H, T, device=dev)
+        delta = S.attention_bwd_scratch(Bt, H, T, dev)
         Wf = W if 0 < W < T else T
         pairs = Wf * (Wf + 1) / 2 + (T - Wf) * Wf
         if args.attn_pass == "fwd":

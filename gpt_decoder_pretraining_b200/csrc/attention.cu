@@ -38,7 +38,8 @@ struct AttnArgs {
   const uint16_t* dobuf;             // bwd: dO
   long long sb_d, sh_d, st_d;        // strides of o/dO in the backward
   float* lse;
-  float* delta;
+  float* delta;  // backward: [2][B·H][Tpad] fp32 — LSE·log2(e), then rowsum(dO∘O); zero-padded
+  int Tpad;      // T rounded up to a multiple of 64
   int* status;
   // optional QK-norm + RoPE backward fused into the dq / dk epilogues (rho_q == nullptr: off):
   // q̃ = RMS_Dh(RoPE(q)), so dq = Rᵀ·rho·(dq̃ − q̃·mean(q̃·dq̃)), likewise for k
@@ -464,11 +465,14 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       const int kv0 = (kv_first + j) * 128;
       const bool need_mask = (kv0 + 127 > tile0) || (kv0 <= tile0 + 127 - W);
+      // chunk c+1 is loaded from tensor memory while chunk c is exponentiated
+      uint32_t rbuf[2][32];
+      tmem_ld32(s_addr, rbuf[0]);
+      tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(s_addr + 32 * c, r);
-        tmem_ld_wait();
+        uint32_t (&r)[32] = rbuf[c & 1];
+        if (c < 3) tmem_ld32(s_addr + 32 * (c + 1), rbuf[(c + 1) & 1]);
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -483,7 +487,9 @@ __global__ void __launch_bounds__(320, 1)
           pk[e] = pack_bf2(p0, p1);
           lb += bf_lo(pk[e]) + bf_hi(pk[e]);
         }
+        // P of chunk c overwrites S columns 16c..16c+15, all of which have been read already
         tmem_st16(s_addr + 16 * c, pk);
+        if (c < 3) tmem_ld_wait();
       }
       tmem_st_wait();
       tc_fence_before();
@@ -540,9 +546,6 @@ __global__ void __launch_bounds__(320, 1)
 // S/dP buffers are double-buffered in tensor memory, so tile i+1's products run while the softmax
 // warps work on tile i.  Each output element has exactly one writer: results are reproducible.
 // ================================================================================================
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 
 template <int DH>
 struct TcBwdShape {
@@ -663,7 +666,7 @@ template <int DH>
 __global__ void __launch_bounds__(320, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                             const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
-                            const AttnArgs a) {
+                            const __grid_constant__ CUtensorMap mpad, const AttnArgs a) {
   using S = TcBwdShape<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -690,7 +693,7 @@ __global__ void __launch_bounds__(320, 1)
   if (threadIdx.x == 0) {
     mbar_init(kv_bar, 1);
     for (int i = 0; i < S::STAGES; ++i) {
-      mbar_init(&q_full[i], 2);  // TMA transaction + the LSE/delta staging
+      mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -711,33 +714,23 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 8) {
-    // ---------------- TMA producer (lane 0) + LSE/delta staging (all lanes) ----------------
+    // ---------------- TMA producer: K, V once; per query tile Q, dO and the LSE / delta rows ----------------
     if (lane == 0) {
       mbar_arrive_expect_tx(kv_bar, 2 * S::BIG_TILE);
       load_tile<DH, 128>(smem + S::OFF_A, &mk, kv_bar, kv0, h, b);
       load_tile<DH, 128>(smem + S::OFF_B, &mv, kv_bar, kv0, h, b);
-    }
-    for (int i = 0; i < n_q; ++i) {
-      const int st = i % S::STAGES;
-      if (!mbar_wait(&q_empty[st], ((i / S::STAGES) & 1) ^ 1, abort_flag, a.status)) break;
-      const int t0 = (q_first + i) * 64;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&q_full[st], S::STAGE_BYTES);
+      const int bhrows = a.B * a.H;
+      for (int i = 0; i < n_q; ++i) {
+        const int st = i % S::STAGES;
+        if (!mbar_wait(&q_empty[st], ((i / S::STAGES) & 1) ^ 1, abort_flag, a.status)) break;
+        const int t0 = (q_first + i) * 64;
+        mbar_arrive_expect_tx(&q_full[st], S::STAGE_BYTES + 2 * 64 * 4);
         uint8_t* dst = smem + S::OFF_STAGE + st * S::STAGE_BYTES;
         load_tile<DH, 64>(dst, &mq, &q_full[st], t0, h, b);
         load_tile<DH, 64>(dst + S::SMALL_TILE, &mdo, &q_full[st], t0, h, b);
+        tma_load_2d(red + st * 128, &mpad, &q_full[st], t0, (int)bh);
+        tma_load_2d(red + st * 128 + 64, &mpad, &q_full[st], t0, bhrows + (int)bh);
       }
-      // LSE in log2 units and delta of the 64 queries: 4 values per lane
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int idx = lane + 32 * u;  // 0..63 lse, 64..127 delta
-        const int qq = t0 + (idx & 63);
-        float v = 0.f;
-        if (qq < T) v = (idx < 64) ? a.lse[bh * T + qq] * LOG2E : a.delta[bh * T + qq];
-        red[st * 128 + idx] = v;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&q_full[st]);
     }
   } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
@@ -783,18 +776,25 @@ __global__ void __launch_bounds__(320, 1)
     const int key = kv0 + kr;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     bool ok = true;
+    // the next tile's Sᵀ / dPᵀ columns are loaded before this tile is released to the MMA warp
+    uint32_t rs[32], rp[32];
+    if (n_q > 0) {
+      ok = mbar_wait(&s_full[0], 0, abort_flag, a.status);
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(tmem + lane_off + S::TM_S + 32 * half, rs);
+        tmem_ld32(tmem + lane_off + S::TM_P + 32 * half, rp);
+        tmem_ld_wait();
+      }
+    }
     for (int i = 0; i < n_q && ok; ++i) {
       const int bf = i & 1;
       const int qc = (q_first + i) * 64 + 32 * half;  // first query of this warp's 32 columns
-      if (!mbar_wait(&s_full[bf], (i >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
-      tc_fence_after();
       const int st = i % S::STAGES;
+      // already complete (the MMA warp waited on it); makes the TMA-written rows visible here
+      if (!mbar_wait(&q_full[st], (i / S::STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
       const float4* l2v = reinterpret_cast<const float4*>(red + st * 128 + 32 * half);
       const float4* dlv = reinterpret_cast<const float4*>(red + st * 128 + 64 + 32 * half);
-      uint32_t rs[32], rp[32];
-      tmem_ld32(tmem + lane_off + S::TM_S + bf * 64 + 32 * half, rs);
-      tmem_ld32(tmem + lane_off + S::TM_P + bf * 64 + 32 * half, rp);
-      tmem_ld_wait();
       // every (key, query) of the warp visible: no per-element mask
       const int kmin = kv0 + 32 * quarter, kmax_ = kmin + 31;
       const bool full = (kmax_ <= qc) && (kmin > qc + 31 - W) && (qc + 31 < T);
@@ -823,9 +823,20 @@ __global__ void __launch_bounds__(320, 1)
       // packed halves stay inside the columns this warp just read (see mma_acc_from_tmem)
       tmem_st16(tmem + lane_off + S::TM_S + bf * 64 + 32 * half, pk);
       tmem_st16(tmem + lane_off + S::TM_P + bf * 64 + 32 * half, dk);
+      const bool more = (i + 1 < n_q);
+      if (more) {
+        const int nb = (i + 1) & 1;
+        if (!mbar_wait(&s_full[nb], ((i + 1) >> 1) & 1, abort_flag, a.status)) { ok = false; }
+        if (ok) {
+          tc_fence_after();
+          tmem_ld32(tmem + lane_off + S::TM_S + nb * 64 + 32 * half, rs);
+          tmem_ld32(tmem + lane_off + S::TM_P + nb * 64 + 32 * half, rp);
+        }
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[bf]);
+      if (more && ok) tmem_ld_wait();
     }
     // epilogue: half 0 writes the dV row, half 1 the dK row of each key
     if (ok) ok = mbar_wait(done, 0, abort_flag, a.status);
@@ -979,20 +990,25 @@ __global__ void __launch_bounds__(320, 1)
     const int row = 32 * quarter + lane;
     const int t = q0 + row;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
-    const float l2 = (t < T) ? a.lse[bh * T + t] * LOG2E : 0.f;
-    const float dl = (t < T) ? a.delta[bh * T + t] : 0.f;
+    const float l2 = (t < T) ? a.delta[bh * a.Tpad + t] : 0.f;
+    const float dl = (t < T) ? a.delta[((long long)a.B * a.H + bh) * a.Tpad + t] : 0.f;
     bool ok = true;
+    // the next tile's S / dP columns are loaded before this tile is released to the MMA warp
+    uint32_t rs[32], rp[32];
+    if (n_kv > 0) {
+      ok = mbar_wait(&s_full[0], 0, abort_flag, a.status);
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(tmem + lane_off + S::TM_S + 32 * half, rs);
+        tmem_ld32(tmem + lane_off + S::TM_P + 32 * half, rp);
+        tmem_ld_wait();
+      }
+    }
     for (int j = 0; j < n_kv && ok; ++j) {
       const int bf = j & 1;
       const int k0 = (kv_first + j) * 64 + 32 * half;
-      if (!mbar_wait(&s_full[bf], (j >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
-      tc_fence_after();
       const bool need_mask = (k0 + 31 > q0 + 32 * quarter) || (k0 <= q0 + 32 * quarter + 31 - W) ||
                              (q0 + 32 * quarter + 31 >= T);
-      uint32_t rs[32], rp[32];
-      tmem_ld32(tmem + lane_off + S::TM_S + bf * 64 + 32 * half, rs);
-      tmem_ld32(tmem + lane_off + S::TM_P + bf * 64 + 32 * half, rp);
-      tmem_ld_wait();
       uint32_t dk[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
@@ -1008,9 +1024,20 @@ __global__ void __launch_bounds__(320, 1)
       }
       // the packed half stays inside the columns this warp just read (see mma_acc_from_tmem)
       tmem_st16(tmem + lane_off + S::TM_S + bf * 64 + 32 * half, dk);
+      const bool more = (j + 1 < n_kv);
+      if (more) {
+        const int nb = (j + 1) & 1;
+        if (!mbar_wait(&s_full[nb], ((j + 1) >> 1) & 1, abort_flag, a.status)) { ok = false; }
+        if (ok) {
+          tc_fence_after();
+          tmem_ld32(tmem + lane_off + S::TM_S + nb * 64 + 32 * half, rs);
+          tmem_ld32(tmem + lane_off + S::TM_P + nb * 64 + 32 * half, rp);
+        }
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[bf]);
+      if (more && ok) tmem_ld_wait();
     }
     if (ok) ok = mbar_wait(done, 0, abort_flag, a.status);
     if (ok) {
@@ -1089,24 +1116,34 @@ __global__ void attn_kmax_kernel(const uint16_t* __restrict__ k, float* __restri
 // backward (1): delta = rowsum(dO ∘ O), one warp per row
 // ================================================================================================
 __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
-                                  float* __restrict__ delta, int B, int H, int T, int Dh,
-                                  long long sb, long long sh, long long st, long long sbd,
-                                  long long shd, long long std_) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  const long long rows = (long long)B * H * T;
+                                  const float* __restrict__ lse, float* __restrict__ pad, int B,
+                                  int H, int T, int Tpad, int Dh, long long sb, long long sh,
+                                  long long st, long long sbd, long long shd, long long std_) {
+  // one warp per padded row (b, h, t < Tpad): pad[0][bh][t] = lse·log2(e), pad[1][bh][t] =
+  // rowsum(dO∘O); rows t ≥ T are zero
+  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long rows = (long long)B * H * Tpad;
   if (warp >= rows) return;
-  const int t = warp % T, h = (warp / T) % H, b = warp / (T * H);
-  const long long off = b * sb + h * sh + (long long)t * st;
-  const long long offd = b * sbd + h * shd + (long long)t * std_;
+  const int t = (int)(warp % Tpad);
+  const long long bh = warp / Tpad;
+  const int h = (int)(bh % H), b = (int)(bh / H);
   float acc = 0.f;
-  for (int j = 2 * lane; j < Dh; j += 64) {
-    const uint32_t x = *reinterpret_cast<const uint32_t*>(o + off + j);
-    const uint32_t y = *reinterpret_cast<const uint32_t*>(dout + offd + j);
-    acc += bf_lo(x) * bf_lo(y) + bf_hi(x) * bf_hi(y);
+  if (t < T) {
+    const long long off = b * sb + h * sh + (long long)t * st;
+    const long long offd = b * sbd + h * shd + (long long)t * std_;
+    for (int j = 2 * lane; j < Dh; j += 64) {
+      const uint32_t x = *reinterpret_cast<const uint32_t*>(o + off + j);
+      const uint32_t y = *reinterpret_cast<const uint32_t*>(dout + offd + j);
+      acc += bf_lo(x) * bf_lo(y) + bf_hi(x) * bf_hi(y);
+    }
   }
 #pragma unroll
   for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  if (lane == 0) delta[warp] = acc;
+  if (lane == 0) {
+    pad[warp] = (t < T) ? lse[bh * T + t] * LOG2E : 0.f;
+    pad[rows + warp] = acc;
+  }
 }
 
 // ================================================================================================
@@ -1211,8 +1248,8 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const int qq = qa + c;
-        l2[c] = (qq < T) ? a.lse[bh * T + qq] * LOG2E : 0.f;
-        dl[c] = (qq < T) ? a.delta[bh * T + qq] : 0.f;
+        l2[c] = (qq < T) ? a.delta[bh * a.Tpad + qq] : 0.f;
+        dl[c] = (qq < T) ? a.delta[((long long)a.B * a.H + bh) * a.Tpad + qq] : 0.f;
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -1340,8 +1377,8 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     const int row = row0 + 8 * r;
-    l2[r] = (row < T) ? a.lse[bh * T + row] * LOG2E : 0.f;
-    dl[r] = (row < T) ? a.delta[bh * T + row] : 0.f;
+    l2[r] = (row < T) ? a.delta[bh * a.Tpad + row] : 0.f;
+    dl[r] = (row < T) ? a.delta[((long long)a.B * a.H + bh) * a.Tpad + row] : 0.f;
   }
   float dq[DH / 8][4];
 #pragma unroll
@@ -1497,10 +1534,11 @@ gpt_status launch_bwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, c
   return GPT_OK;
 }
 
-// tcgen05 backward: maps with 128-row boxes (outer tiles) and 64-row boxes (inner tiles).
+// tcgen05 backward: maps with 128-row boxes (outer tiles) and 64-row boxes (inner tiles), and the
+// padded [2·B·H][Tpad] fp32 LSE / delta array in 64-float boxes.
 template <int DH>
-gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[4], AttnArgs a,
-                         void* dq, cudaStream_t stream) {
+gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[4],
+                         const CUtensorMap& mpad, AttnArgs a, void* dq, cudaStream_t stream) {
   using S = TcBwdShape<DH>;
   static bool once = false;
   if (!once) {
@@ -1510,7 +1548,8 @@ gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[
   }
   // dK/dV: outer 128-key tiles (K, V with 128-row boxes), inner 64-query tiles (Q, dO 64-row boxes)
   dim3 g1((a.T + 127) / 128, a.H, a.B);
-  attn_bwd_dkdv_tc_kernel<DH><<<g1, S::THREADS, S::SMEM, stream>>>(m64[0], m128[1], m128[2], m64[3], a);
+  attn_bwd_dkdv_tc_kernel<DH><<<g1, S::THREADS, S::SMEM, stream>>>(m64[0], m128[1], m128[2], m64[3],
+                                                                   mpad, a);
   count_launch();
   GPT_CUDA_TRY(cudaGetLastError());
   // dQ: outer 128-query tiles (Q, dO 128-row boxes), inner 64-key tiles (K, V 64-row boxes)
@@ -1593,13 +1632,24 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
       !make_head_map(&mv, v, B, H, T, Dh, sbq, shq, stq, 64) ||
       !make_head_map(&mdo, dout, B, H, T, Dh, sbd, shd, std_, 64))
     return GPT_ERR_UNSUPPORTED_SHAPE;
+  const int Tpad = (T + 63) / 64 * 64;
+  // the tensor-core kernels fetch the padded LSE / delta rows with TMA (64-float boxes)
+  CUtensorMap mpad;
+  if (Dh != 32) {
+    const uint64_t dims[2] = {(uint64_t)Tpad, (uint64_t)2 * B * H};
+    const uint64_t strides[1] = {(uint64_t)Tpad * 4};
+    const uint32_t box[2] = {64, 1};
+    if ((reinterpret_cast<uintptr_t>(delta) & 15) != 0 ||
+        !encode_map_f32(&mpad, delta, 2, dims, strides, box))
+      return GPT_ERR_UNSUPPORTED_SHAPE;
+  }
   {
-    const long long rows = (long long)B * H * T;
+    const long long rows = (long long)B * H * Tpad;
     const int threads = 256;
     const long long blocks = (rows * 32 + threads - 1) / threads;
     attn_delta_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
-        reinterpret_cast<const uint16_t*>(o), reinterpret_cast<const uint16_t*>(dout), delta, B, H,
-        T, Dh, sbo, sho, sto, sbd, shd, std_);
+        reinterpret_cast<const uint16_t*>(o), reinterpret_cast<const uint16_t*>(dout), lse, delta, B,
+        H, T, Tpad, Dh, sbo, sho, sto, sbd, shd, std_);
     count_launch();
     GPT_CUDA_TRY(cudaGetLastError());
   }
@@ -1610,6 +1660,7 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   a.scale_log2 = a.scale * LOG2E;
   a.lse = const_cast<float*>(lse);
   a.delta = delta;
+  a.Tpad = Tpad;
   a.status = status;
   a.sb_o = sbg; a.sh_o = shg; a.st_o = stg;  // strides of the dq/dk/dv outputs
   a.rho_q = rho_q;
@@ -1630,14 +1681,15 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
                        is_do ? std_ : stq, 64))
       return GPT_ERR_UNSUPPORTED_SHAPE;
   }
-  if (Dh == 128) GPT_TRY(launch_bwd_tc<128>(m128, m64, a, dq, stream));
-  else GPT_TRY(launch_bwd_tc<64>(m128, m64, a, dq, stream));
+  if (Dh == 128) GPT_TRY(launch_bwd_tc<128>(m128, m64, mpad, a, dq, stream));
+  else GPT_TRY(launch_bwd_tc<64>(m128, m64, mpad, a, dq, stream));
   return GPT_OK;
 }
 
 // ------------------------------------------------------------------------------------------------
-// Allocation-free attention backward: the per-row delta = rowsum(dO∘O) lives in this fixed array
-// instead of a caller-supplied buffer.  Every GPU that loads the library holds it until exit.
+// Allocation-free attention backward: the backward's per-row scratch (LSE·log2 e and
+// delta = rowsum(dO∘O), 2·B·H·⌈T/64⌉·64 floats) lives in this fixed array instead of a
+// caller-supplied buffer.  Every GPU that loads the library holds it until exit.
 // ------------------------------------------------------------------------------------------------
 constexpr long long NOALLOC_DELTA_ROWS = GPT_ATTN_BWD_NOALLOC_MAX_ROWS;
 static __device__ __align__(256) float g_noalloc_delta[NOALLOC_DELTA_ROWS];
@@ -1666,7 +1718,7 @@ gpt_status attention_bwd_noalloc(const void* q, const void* k, const void* v, co
                                  long long shq, long long stq, long long sbo, long long sho,
                                  long long sto, int* status, cudaStream_t stream) {
   if (B <= 0 || H <= 0 || T <= 0) return GPT_ERR_INVALID_ARG;
-  if ((long long)B * H * T > NOALLOC_DELTA_ROWS) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if (2ll * B * H * ((T + 63) / 64 * 64) > NOALLOC_DELTA_ROWS) return GPT_ERR_UNSUPPORTED_SHAPE;
   float* delta = nullptr;
   GPT_TRY(noalloc_delta_ptr(&delta));
   return attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, T, Dh, window, sbq, shq, stq,
@@ -1694,6 +1746,11 @@ extern "C" gpt_status gpt_attention_bwd(const void* q, const void* k, const void
   return gpt::attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, T, Dh, window, sb_qkv,
                             sh_qkv, st_qkv, sb_qkv, sh_qkv, st_qkv, sb_o, sh_o, st_o, sb_o, sh_o,
                             st_o, status, gpt::as_stream(stream), nullptr, nullptr, nullptr);
+}
+
+extern "C" size_t gpt_attention_bwd_scratch_bytes(int B, int H, int T) {
+  if (B <= 0 || H <= 0 || T <= 0) return 0;
+  return (size_t)2 * B * H * ((T + 63) / 64 * 64) * sizeof(float);
 }
 
 extern "C" gpt_status gpt_attention_bwd_noalloc(const void* q, const void* k, const void* v,

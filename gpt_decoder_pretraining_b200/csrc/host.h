@@ -30,6 +30,9 @@ gpt_status device_info(int* num_sms);
 // Returns false if the driver rejects the map (alignment, box size).
 bool encode_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                      const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128);
+// Same for an fp32 tensor, no swizzle.
+bool encode_map_f32(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box);
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 

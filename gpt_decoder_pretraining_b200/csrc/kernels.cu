@@ -352,39 +352,76 @@ __global__ void __launch_bounds__(1024) embedding_sort_kernel(const int32_t* __r
   }
 }
 
-// One CTA per run: dwte[id] += Σ over the run (ascending token index) of gx rows.  The column
-// range is split over the threads (4 floats each); rows are summed 4 at a time in a fixed order.
-__global__ void embedding_accum_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ run_start,
-                                       const int* __restrict__ nruns, const float* __restrict__ gx,
-                                       float* __restrict__ dwte, int seg0, int d) {
-  const int r = blockIdx.x;
-  if (r >= *nruns) return;
-  const int s = run_start[r], e = run_start[r + 1];
-  const int id = (int)(keys[s] >> 16);
+// Deterministic accumulation over the sorted (id, position) keys in fixed pieces of EMB_PIECE
+// consecutive keys, so that a frequent id (Zipf-hot rows) is spread over many CTAs:
+//   piece kernel  one CTA per piece; threads cover the columns (4 floats each) and walk the piece's
+//                 rows in order.  A run (equal ids) lying wholly inside the piece is written to
+//                 dwte directly; a run that crosses the piece's start goes to partial slot 0, one
+//                 that continues past its end to slot 1 (a run crossing both: slot 0).
+//   fix-up kernel one CTA per run that spans several pieces: sums slot 1 of its first piece,
+//                 slot 0 of the pieces after it, in piece order, into dwte[id].
+constexpr int EMB_PIECE = 64;
+
+__global__ void embedding_piece_kernel(const uint32_t* __restrict__ keys, int n, const float* __restrict__ gx,
+                                       float* __restrict__ dwte, float* __restrict__ partial, int seg0, int d,
+                                       int accumulate) {
+  const int p = blockIdx.x;
+  const int s = p * EMB_PIECE, e = min(n, s + EMB_PIECE);
+  const int idx_before = (s > 0) ? (int)(keys[s - 1] >> 16) : -1;
+  const int idx_after = (e < n) ? (int)(keys[e] >> 16) : -1;
   for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     int i = s;
-    for (; i + 4 <= e; i += 4) {
-      float4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int m = seg0 + (int)(keys[i + u] & 0xFFFFu);
-        v[u] = *reinterpret_cast<const float4*>(gx + (size_t)m * d + c);
+    while (i < e) {
+      const int id = (int)(keys[i] >> 16);
+      int j = i;
+      acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (; j < e && (int)(keys[j] >> 16) == id; ++j) {
+        const int m = seg0 + (int)(keys[j] & 0xFFFFu);
+        const float4 v = *reinterpret_cast<const float4*>(gx + (size_t)m * d + c);
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
       }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
+      const bool from_before = (i == s) && (id == idx_before);
+      const bool to_after = (j == e) && (id == idx_after);
+      if (!from_before && !to_after) {
+        float4* dst = reinterpret_cast<float4*>(dwte + (size_t)id * d + c);
+        if (accumulate) {
+          const float4 o = *dst;
+          acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+        }
+        *dst = acc;
+      } else {
+        const int slot = from_before ? 0 : 1;
+        *reinterpret_cast<float4*>(partial + ((size_t)p * 2 + slot) * d + c) = acc;
       }
+      i = j;
     }
-    for (; i < e; ++i) {
-      const int m = seg0 + (int)(keys[i] & 0xFFFFu);
-      const float4 v = *reinterpret_cast<const float4*>(gx + (size_t)m * d + c);
+  }
+}
+
+__global__ void embedding_fixup_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ run_start,
+                                       const int* __restrict__ nruns, const float* __restrict__ partial,
+                                       float* __restrict__ dwte, int d, int accumulate) {
+  const int r = blockIdx.x;
+  if (r >= *nruns) return;
+  const int s = run_start[r], e = run_start[r + 1];
+  const int ps = s / EMB_PIECE, pe = (e - 1) / EMB_PIECE;
+  if (ps == pe) return;  // written by its piece
+  const int id = (int)(keys[s] >> 16);
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    // the first piece holds the run's head in slot 1 (slot 0 if the run starts the piece at its
+    // first key and the previous key has another id, which makes it "not from before")
+    float4 acc = *reinterpret_cast<const float4*>(partial + ((size_t)ps * 2 + 1) * d + c);
+    for (int p = ps + 1; p <= pe; ++p) {
+      const float4 v = *reinterpret_cast<const float4*>(partial + ((size_t)p * 2 + 0) * d + c);
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
     float4* dst = reinterpret_cast<float4*>(dwte + (size_t)id * d + c);
-    float4 o = *dst;
-    o.x += acc.x; o.y += acc.y; o.z += acc.z; o.w += acc.w;
-    *dst = o;
+    if (accumulate) {
+      const float4 o = *dst;
+      acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+    }
+    *dst = acc;
   }
 }
 
@@ -568,12 +605,13 @@ gpt_status embedding_fwd(const int32_t* tok, const void* wte, void* x, int M, in
   return GPT_OK;
 }
 
-size_t embedding_bwd_scratch_bytes(int M, int V) {
+size_t embedding_bwd_scratch_bytes(int M, int d, int V) {
   (void)V;
   const int seg = std::min(M, EMB_SEG);
-  // keys [seg] + run starts [seg + 1] + nruns, 256-byte aligned pieces
+  const size_t pieces = (seg + EMB_PIECE - 1) / EMB_PIECE;
+  // keys [seg], run starts [seg + 1], nruns, partial sums [pieces][2][d]
   auto al = [](size_t b) { return (b + 255) & ~(size_t)255; };
-  return al((size_t)seg * 4) + al((size_t)(seg + 1) * 4) + al(4);
+  return al((size_t)seg * 4) + al((size_t)(seg + 1) * 4) + al(4) + al(pieces * 2 * (size_t)d * 4);
 }
 
 gpt_status embedding_bwd(const int32_t* tok, const float* gx, float* dwte, int M, int d, int V,
@@ -586,6 +624,7 @@ gpt_status embedding_bwd(const int32_t* tok, const float* gx, float* dwte, int M
   uint32_t* keys = reinterpret_cast<uint32_t*>(p);
   int* run_start = reinterpret_cast<int*>(p + al((size_t)seg * 4));
   int* nruns = reinterpret_cast<int*>(p + al((size_t)seg * 4) + al((size_t)(seg + 1) * 4));
+  float* partial = reinterpret_cast<float*>(p + al((size_t)seg * 4) + al((size_t)(seg + 1) * 4) + al(4));
   GPT_CUDA_TRY(cudaMemsetAsync(dwte, 0, (size_t)V * d * sizeof(float), s));
   static bool attr = false;
   if (!attr) {
@@ -593,6 +632,7 @@ gpt_status embedding_bwd(const int32_t* tok, const float* gx, float* dwte, int M
                                       EMB_SEG * 4));
     attr = true;
   }
+  const int threads = std::min(512, std::max(32, ((d / 4) + 31) / 32 * 32));
   for (int s0 = 0; s0 < M; s0 += EMB_SEG) {
     const int n = std::min(EMB_SEG, M - s0);
     int P = 1;
@@ -600,8 +640,13 @@ gpt_status embedding_bwd(const int32_t* tok, const float* gx, float* dwte, int M
     embedding_sort_kernel<<<1, 1024, (size_t)P * 4, s>>>(tok + s0, n, V, keys, run_start, nruns);
     count_launch();
     GPT_CUDA_TRY(cudaGetLastError());
-    const int threads = std::min(256, std::max(32, ((d / 4) + 31) / 32 * 32));
-    embedding_accum_kernel<<<n, threads, 0, s>>>(keys, run_start, nruns, gx, dwte, s0, d);
+    const int pieces = (n + EMB_PIECE - 1) / EMB_PIECE;
+    // segments after the first add onto the rows earlier segments wrote
+    const int acc = (s0 > 0) ? 1 : 0;
+    embedding_piece_kernel<<<pieces, threads, 0, s>>>(keys, n, gx, dwte, partial, s0, d, acc);
+    count_launch();
+    GPT_CUDA_TRY(cudaGetLastError());
+    embedding_fixup_kernel<<<n, threads, 0, s>>>(keys, run_start, nruns, partial, dwte, d, acc);
     count_launch();
     GPT_CUDA_TRY(cudaGetLastError());
   }
@@ -658,7 +703,9 @@ gpt_status gpt_embedding_fwd(const int32_t* tokens, const void* wte, void* x, in
                              int* status, void* stream) {
   return gpt::embedding_fwd(tokens, wte, x, M, d, V, status, gpt::as_stream(stream));
 }
-size_t gpt_embedding_bwd_scratch_bytes(int M, int V) { return gpt::embedding_bwd_scratch_bytes(M, V); }
+size_t gpt_embedding_bwd_scratch_bytes(int M, int d, int V) {
+  return gpt::embedding_bwd_scratch_bytes(M, d, V);
+}
 gpt_status gpt_embedding_bwd(const int32_t* tokens, const float* gx, float* dwte, int M, int d,
                              int V, void* scratch, void* stream) {
   return gpt::embedding_bwd(tokens, gx, dwte, M, d, V, scratch, gpt::as_stream(stream));

@@ -34,7 +34,7 @@ EXPORTED = [
     "gpt_gemm", "gpt_qkv_proj_rope", "gpt_rmsnorm_fwd", "gpt_rmsnorm_bwd", "gpt_rope_qknorm_fwd", "gpt_rope_qknorm_bwd",
     "gpt_rope_table", "gpt_attention_fwd", "gpt_attention_bwd", "gpt_attention_bwd_noalloc",
     "gpt_embedding_fwd",
-    "gpt_embedding_bwd_scratch_bytes", "gpt_embedding_bwd", "gpt_lmhead_ce_scratch_bytes",
+    "gpt_attention_bwd_scratch_bytes", "gpt_embedding_bwd_scratch_bytes", "gpt_embedding_bwd", "gpt_lmhead_ce_scratch_bytes",
     "gpt_lmhead_ce_fwd_bwd",
 ]
 
@@ -89,7 +89,9 @@ def lib():
         L.gpt_attention_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                                 ll, ll, ll, ll, ll, ll, vp, vp]
         L.gpt_embedding_fwd.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp]
-        L.gpt_embedding_bwd_scratch_bytes.argtypes = [i32, i32]
+        L.gpt_attention_bwd_scratch_bytes.argtypes = [i32, i32, i32]
+        L.gpt_attention_bwd_scratch_bytes.restype = sz
+        L.gpt_embedding_bwd_scratch_bytes.argtypes = [i32, i32, i32]
         L.gpt_embedding_bwd_scratch_bytes.restype = sz
         L.gpt_embedding_bwd.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp]
         L.gpt_lmhead_ce_scratch_bytes.argtypes = [i32, i32, i32]
@@ -251,6 +253,16 @@ def attention_fwd(q, k, v, o, lse, window: int, strides_qkv, strides_o, B, H, T,
                                    *strides_qkv, *strides_o, _ptr(status), _stream()), "attention_fwd")
 
 
+def attention_bwd_scratch_bytes(B: int, H: int, T: int) -> int:
+    return int(lib().gpt_attention_bwd_scratch_bytes(B, H, T))
+
+
+def attention_bwd_scratch(B: int, H: int, T: int, device="cuda"):
+    """A device buffer for gpt_attention_bwd's `delta` scratch."""
+    import torch
+    return torch.empty(attention_bwd_scratch_bytes(B, H, T) // 4, dtype=torch.float32, device=device)
+
+
 def attention_bwd(q, k, v, o, do, lse, delta, dq, dk, dv, window: int, strides_qkv, strides_o, B, H, T,
                   Dh, status=None):
     _check(lib().gpt_attention_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
@@ -275,8 +287,8 @@ def embedding_fwd(tokens, wte, x, status=None):
                                    _stream()), "embedding_fwd")
 
 
-def embedding_bwd_scratch_bytes(M: int, V: int) -> int:
-    return int(lib().gpt_embedding_bwd_scratch_bytes(M, V))
+def embedding_bwd_scratch_bytes(M: int, d: int, V: int) -> int:
+    return int(lib().gpt_embedding_bwd_scratch_bytes(M, d, V))
 
 
 def embedding_bwd(tokens, gx, dwte, scratch):

@@ -175,8 +175,10 @@ gpt_status gpt_rope_table(float* cos_sin, int T, int Dh, void* stream);
 /* Causal / sliding-window flash attention.  q, k, v, o, dq, dk, dv are bf16 tensors addressed as
  * element (b, h, t, j) at base + b·sb + h·sh + t·st + j (strides in elements, j contiguous), one
  * stride set per tensor group: (sb_qkv, sh_qkv, st_qkv) for q/k/v/dq/dk/dv and (sb_o, sh_o, st_o)
- * for o/do.  lse, delta: fp32 [B, H, T].  Dh ∈ {64, 128}.  window ≤ 0 or ≥ T = full causal.
- * lse = natural-log logsumexp of the scaled scores; delta = rowsum(dO∘O) (computed by the bwd).
+ * for o/do.  lse: fp32 [B, H, T], the natural-log logsumexp of the scaled scores.  Dh ∈ {32, 64,
+ * 128}.  window ≤ 0 or ≥ T = full causal.  delta: backward scratch of at least 2·B·H·⌈T/64⌉·64 fp32
+ * values (4-byte aligned, 16-byte aligned for Dh ≥ 64); the backward fills it with LSE·log2(e) and
+ * rowsum(dO∘O) per row, zero-padded to a multiple of 64 rows per (b, h).
  * The forward shifts each row's exponentials by the Cauchy–Schwarz bound c_t = ‖q_t‖·max_j‖k_j‖/√Dh
  * instead of a running maximum (softmax is invariant to the shift, so the result is exact); this
  * needs c_t ≤ 40 so that no row underflows, which always holds after QK-norm (c_t ≈ √Dh) — rows
@@ -187,6 +189,9 @@ gpt_status gpt_attention_fwd(const void* q, const void* k, const void* v, void* 
                              float* kmax, int B, int H, int T, int Dh, int window, long long sb_qkv,
                              long long sh_qkv, long long st_qkv, long long sb_o, long long sh_o,
                              long long st_o, int* status, void* stream);
+/* Bytes of the `delta` scratch that gpt_attention_bwd needs for (B, H, T): 2·B·H·⌈T/64⌉·64 fp32
+ * values.  Returns 0 for a non-positive size. */
+size_t gpt_attention_bwd_scratch_bytes(int B, int H, int T);
 gpt_status gpt_attention_bwd(const void* q, const void* k, const void* v, const void* o,
                              const void* dout, const float* lse, float* delta, void* dq, void* dk,
                              void* dv, int B, int H, int T, int Dh, int window, long long sb_qkv,
@@ -195,14 +200,15 @@ gpt_status gpt_attention_bwd(const void* q, const void* k, const void* v, const 
 
 /* Attention backward that allocates nothing.  The pages have no counterpart: this is a calling
  * convenience, not part of the method.  Arguments and results are those of gpt_attention_bwd
- * without `delta`; the per-row rowsum(dO∘O) that the backward needs is kept in a static device
- * array inside this library (GPT_ATTN_BWD_NOALLOC_MAX_ROWS fp32 values = 8 MiB), which every GPU
- * that loads the library holds until the process exits.
+ * without `delta`; the per-row scratch that the backward needs (2·B·H·⌈T/64⌉·64 fp32 values) is
+ * kept in a static device array inside this library (GPT_ATTN_BWD_NOALLOC_MAX_ROWS fp32 values =
+ * 8 MiB), which every GPU that loads the library holds until the process exits.
  * It serves callers that cannot obtain device memory where they call the backward — for example
  * code running under a device-memory budget fixed at start-up, or inside a host framework whose own
  * allocator owns all device memory and allows no side allocations — and therefore cannot hand
  * gpt_attention_bwd its scratch buffer.  It calls no cudaMalloc, cudaFree or allocating routine.
- *   - B·H·T > GPT_ATTN_BWD_NOALLOC_MAX_ROWS returns GPT_ERR_UNSUPPORTED_SHAPE; nothing is enqueued.
+ *   - 2·B·H·⌈T/64⌉·64 > GPT_ATTN_BWD_NOALLOC_MAX_ROWS returns GPT_ERR_UNSUPPORTED_SHAPE; nothing
+ *     is enqueued.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
  *     that device current); make that first call before any stream capture.
  *   - All calls share the one array.  Each call writes the rows it uses before reading them, so
@@ -221,9 +227,10 @@ gpt_status gpt_attention_bwd_noalloc(const void* q, const void* k, const void* v
 gpt_status gpt_embedding_fwd(const int32_t* tokens, const void* wte, void* x, int M, int d, int V,
                              int* status, void* stream);
 /* Embedding backward dwte = Σ_{m: tok[m]=v} gx[m] for every row v (fp32, rows without a token are
- * zeroed).  Duplicate ids are summed in ascending m, so the result is deterministic.  scratch:
- * device bytes ≥ gpt_embedding_bwd_scratch_bytes(M, V). */
-size_t gpt_embedding_bwd_scratch_bytes(int M, int V);
+ * zeroed).  Duplicate ids are summed in a fixed order (ascending m within pieces of 64 sorted
+ * tokens, pieces in order), so the result is deterministic.  scratch: device bytes ≥
+ * gpt_embedding_bwd_scratch_bytes(M, d, V). */
+size_t gpt_embedding_bwd_scratch_bytes(int M, int d, int V);
 gpt_status gpt_embedding_bwd(const int32_t* tokens, const float* gx, float* dwte, int M, int d,
                              int V, void* scratch, void* stream);
 

@@ -1,0 +1,159 @@
+"""The C ABI on the host (no GPU): the library loads and exports every symbol the header
+declares, the parameter packing agrees with the configs and the oracle, and argument errors come
+back as status codes before anything touches a device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from gpt_decoder_pretraining_b200 import build as B
+from gpt_decoder_pretraining_b200 import config as C
+from gpt_decoder_pretraining_b200 import step as S
+from oracle import gpt_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gptstep.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(S._LIB_PATH):
+        B.build()
+    return S.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gpt_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 20
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(S.EXPORTED)
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
+        assert lib.gpt_strerror(code) and lib.gpt_strerror(code) != b"unknown status"
+    assert lib.gpt_strerror(123) == b"unknown status"
+
+
+@pytest.mark.parametrize("name", C.PRESETS)
+def test_param_layout_matches_configs_and_oracle(lib, name):
+    cfg = C.preset(name)
+    offs, total = S.param_layout(cfg)
+    assert total == cfg.n_params == O.n_params(O.oracle_config(cfg))
+    pos, expect = 0, []
+    for _, (a, b) in cfg.tensor_shapes():
+        expect.append(pos)
+        pos += a * b
+    assert offs == expect
+    assert all(o % 64 == 0 for o in offs)
+    # the oracle unpacks the same flat buffer into the same tensors
+    if name == "smoke":
+        flat = np.arange(total, dtype=np.float64)
+        P = O.unpack(O.oracle_config(cfg), flat)
+        assert P["wte"][0, 0] == offs[0] and P["qkv0"][0, 0] == offs[1] and P["lm"][0, 0] == offs[-1]
+
+
+def _create(lib, cfg):
+    c, keep = S._cconfig(cfg)
+    h = ctypes.c_void_p()
+    return lib.gpt_step_create(ctypes.byref(c), ctypes.byref(h)), h, keep
+
+
+def test_config_validation(lib):
+    good = C.custom(2, 128, 64, 256, 32, 2)
+    st, h, _ = _create(lib, good)
+    assert st == 0
+    lib.gpt_step_destroy(h)
+    bad = [
+        (C.custom(2, 96, 32, 256, 32, 2), -2),                 # d_model not a multiple of 64
+        (C.custom(2, 128, 16, 256, 32, 2), -2),                # head_dim 16 unsupported
+        (C.custom(2, 128, 64, 70000 // 64 * 64, 32, 2), -2),   # vocab above 65536
+    ]
+    for cfg, code in bad:
+        assert _create(lib, cfg)[0] == code
+    cfg = C.custom(2, 128, 64, 256, 32, 2)
+    cfg.param_dtype = 7
+    assert _create(lib, cfg)[0] == -1
+    cfg = C.custom(2, 128, 64, 256, 32, 2)
+    cfg.n_heads = 3  # n_heads·head_dim ≠ d_model
+    assert _create(lib, cfg)[0] == -1
+
+
+def test_workspace_sizes_grow_with_the_model(lib):
+    sizes = []
+    for name in C.PRESETS:
+        st, h, _ = _create(lib, C.preset(name))
+        assert st == 0
+        n = ctypes.c_size_t()
+        assert lib.gpt_step_workspace_bytes(h, ctypes.byref(n)) == 0
+        sizes.append(n.value)
+        lib.gpt_step_destroy(h)
+    assert sizes[0] < sizes[1] < sizes[2] and sizes[3] > sizes[1]
+    assert sizes[3] < 60e9  # d24 fits a 180 GB B200 with room to spare
+
+
+def test_step_argument_errors_need_no_device(lib):
+    st, h, _ = _create(lib, C.custom(1, 64, 32, 256, 16, 1))
+    assert st == 0
+    n = ctypes.c_size_t()
+    lib.gpt_step_workspace_bytes(h, ctypes.byref(n))
+    fake = 1 << 20  # never dereferenced: validation fails first
+    call = lib.gpt_step_fwd_bwd
+    assert call(h, None, fake, fake, fake, fake, fake, n.value, 0, None) == -1           # null params
+    assert call(h, fake, fake, fake, fake, fake, fake, n.value, 1, None) == -1           # accumulate
+    assert call(h, fake, fake, fake, fake, fake, fake, n.value - 1, 0, None) == -3       # too small
+    assert call(h, fake + 8, fake, fake, fake, fake, fake, n.value, 0, None) == -2       # misaligned
+    assert lib.gpt_step_status(None, fake, None) == -1
+    lib.gpt_step_destroy(h)
+
+
+def test_kernel_entry_points_reject_bad_arguments(lib):
+    f = 1 << 20
+    assert lib.gpt_gemm(0, 0, 0, 64, 64, f, 64, f, 64, f, 64, None, None, 0, None, None) == -1
+    assert lib.gpt_gemm(5, 0, 64, 64, 64, f, 64, f, 64, f, 64, None, None, 0, None, None) == -1
+    assert lib.gpt_gemm(0, 0, 64, 64, 64, f, 60, f, 64, f, 64, None, None, 0, None, None) == -1
+    assert lib.gpt_gemm(0, 0, 64, 64, 64, f + 2, 64, f, 64, f, 64, None, None, 0, None, None) == -2
+    assert lib.gpt_attention_fwd(f, f, f, f, f, None, 1, 1, 16, 48, 0, 48, 48, 48, 48, 48, 48, None, None) == -2
+    assert lib.gpt_rmsnorm_fwd(None, f, f, 4, 64, None) == -1
+    assert lib.gpt_embedding_bwd(f, f, f, 16, 64, 70000, f, None) == -2
+
+
+def test_multi_rank_timing_uses_the_slowest_rank():
+    """bench.py with N>1 ranks: replicas, the job time is the max over ranks (gloo, 2 processes)."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + (os.getpid() % 1000)
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r, (ms, rate) in out:
+        assert ms == [20.0, 7.0]  # max over ranks of [10+10r, 7-r]
+        assert rate == pytest.approx(32768 * 2 / 0.020)
+
+
+def _rank_main(rank, world, port, q):
+    import sys
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch.distributed as dist
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    ms = bench.max_over_ranks([10.0 + 10.0 * rank, 7.0 - rank], world)
+    rate = bench.whole_job_rate(32768, world, ms[0])
+    dist.destroy_process_group()
+    q.put((rank, (ms, rate)))

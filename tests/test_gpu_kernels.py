@@ -228,7 +228,7 @@ def test_attention_fwd_bwd(B, H, T, Dh, window):
     S.attention_fwd(tq, tk, tv, to_n, lse_n, window, strides, strides, B, H, T, Dh, status=st,
                     qk_normalized=True)
     dq, dk, dv = (torch.zeros_like(tq) for _ in range(3))
-    delta = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
+    delta = S.attention_bwd_scratch(B, H, T)
     S.attention_bwd(tq, tk, tv, to, tdo, lse, delta, dq, dk, dv, window, strides, strides, B, H, T, Dh,
                     status=st)
     torch.cuda.synchronize()
@@ -267,9 +267,10 @@ def test_attention_token_major_strides():
 # --------------------------------------------------------------------------------------------------
 # embedding
 # --------------------------------------------------------------------------------------------------
-def test_embedding_fwd_bwd_deterministic():
+@pytest.mark.parametrize("V,d,M", [(512, 128, 3000), (64, 64, 40000), (2048, 1536, 700)])
+def test_embedding_fwd_bwd_deterministic(V, d, M):
+    """Zipf ids (long runs of the hot ids, runs crossing 64-token pieces, several sort segments)."""
     rng = np.random.default_rng(3)
-    V, d, M = 512, 128, 3000
     from gpt_decoder_pretraining_b200.inputs import _zipf_ids
     tok = _zipf_ids(rng, M, V)
     wte = randn(rng, V, d)
@@ -277,7 +278,7 @@ def test_embedding_fwd_bwd_deterministic():
     ttok = torch.from_numpy(tok).cuda()
     x = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
     S.embedding_fwd(ttok, bf16_tensor(wte), x)
-    scratch = torch.empty(S.embedding_bwd_scratch_bytes(M, V), dtype=torch.uint8, device="cuda")
+    scratch = torch.empty(S.embedding_bwd_scratch_bytes(M, d, V), dtype=torch.uint8, device="cuda")
     dw1 = torch.full((V, d), 7.0, dtype=torch.float32, device="cuda")
     dw2 = torch.empty((V, d), dtype=torch.float32, device="cuda")
     tg = torch.from_numpy(gx).cuda()
