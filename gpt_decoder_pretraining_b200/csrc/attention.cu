@@ -392,27 +392,27 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
       constexpr uint32_t id_o = idesc_bf16(128, DH, false, true);
-      const uint32_t qa = smem_u32(smem + S::OFF_Q);
-      const uint32_t kb0 = smem_u32(smem + S::OFF_K);
-      const uint32_t vb0 = smem_u32(smem + S::OFF_V);
+      // descriptors of stage 0 / tile 0, advanced by constant offsets in the loops
+      const uint64_t qd = sdesc_sw128(smem_u32(smem + S::OFF_Q), 16, 1024);
+      const uint64_t kd = sdesc_sw128(smem_u32(smem + S::OFF_K), 16, 1024);
+      const uint64_t vd = sdesc_sw128(smem_u32(smem + S::OFF_V), 128 * 128, 1024);
       auto issue_s = [&](int x, int j) {
-        const uint32_t q_base = qa + x * S::Q_TILE;
-        const uint32_t k_base = kb0 + (j & 1) * S::KV_TILE;
+        const uint64_t q_desc = sdesc_add(qd, x * S::Q_TILE);
+        const uint64_t k_desc = sdesc_add(kd, (j & 1) * S::KV_TILE);
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_bf16_ss(tmem + S::TM_S + x * 128, sdesc_sw128(q_base + off, 16, 1024),
-                      sdesc_sw128(k_base + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+          mma_bf16_ss(tmem + S::TM_S + x * 128, sdesc_add(q_desc, off), sdesc_add(k_desc, off), id_s,
+                      kk > 0 ? 1u : 0u);
         }
         tc_commit(&s_full[x]);
       };
       auto issue_pv = [&](int x, int j) {
-        const uint32_t v_base = vb0 + (j & 1) * S::KV_TILE;
+        const uint64_t v_desc = sdesc_add(vd, (j & 1) * S::KV_TILE);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16_ts(tmem + S::TM_O + x * DH, tmem + S::TM_S + x * 128 + kk * 8,
-                      sdesc_sw128(v_base + kk * 2048, 128 * 128, 1024), id_o,
-                      (j > 0 || kk > 0) ? 1u : 0u);
+                      sdesc_add(v_desc, kk * 2048), id_o, (j > 0 || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(bar_q, 0, abort_flag, a.status);
       if (ok) ok = mbar_wait(&kv_full[0], 0, abort_flag, a.status);
@@ -459,7 +459,8 @@ __global__ void __launch_bounds__(320, 1)
     const float c2 = c_nat * LOG2E;
     // l: exact sum of the weights (gives the LSE the backward pass needs); lb: sum of the bf16
     // weights that P·V actually uses, so that O = Σ P·v / lb is a convex combination of the v rows
-    float l = 0.f, lb = 0.f;
+    // (exact for a single visible key).  Both as packed pairs of partial sums.
+    float l0 = 0.f, l1 = 0.f, lb0 = 0.f, lb1 = 0.f;
     for (int j = 0; j < n_kv && ok; ++j) {
       if (!mbar_wait(&s_full[x], j & 1, abort_flag, a.status)) { ok = false; break; }
       tc_fence_after();
@@ -476,16 +477,18 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * e]), a.scale_log2, -c2));
-          float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * e + 1]), a.scale_log2, -c2));
+          float x0, x1;
+          fma2_bc(x0, x1, __uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]), a.scale_log2, -c2);
+          float p0 = ex2_approx(x0);
+          float p1 = ex2_approx(x1);
           if (need_mask) {
             const int key = kv0 + 32 * c + 2 * e;
             if (!(key <= t && key > t - W)) p0 = 0.f;
             if (!(key + 1 <= t && key + 1 > t - W)) p1 = 0.f;
           }
-          l += p0 + p1;
+          add2_acc(l0, l1, p0, p1);
           pk[e] = pack_bf2(p0, p1);
-          lb += bf_lo(pk[e]) + bf_hi(pk[e]);
+          add2_acc(lb0, lb1, bf_lo(pk[e]), bf_hi(pk[e]));
         }
         // P of chunk c overwrites S columns 16c..16c+15, all of which have been read already
         tmem_st16(s_addr + 16 * c, pk);
@@ -499,7 +502,8 @@ __global__ void __launch_bounds__(320, 1)
     if (ok) ok = mbar_wait(o_full, 0, abort_flag, a.status);
     if (ok) {
       tc_fence_after();
-      const float inv = 1.f / lb;
+      const float l = l0 + l1;
+      const float inv = 1.f / (lb0 + lb1);
       uint16_t* orow = a.o + b * a.sb_o + h * a.sh_o + (long long)t * a.st_o;
 #pragma unroll 1
       for (int c = 0; c < DH / 32; ++c) {
@@ -565,27 +569,28 @@ struct TcBwdShape {
 };
 
 // Issue one [128 × 64] product A·Bᵀ (A: 128 rows, B: 64 rows, both K-major [DH/64][rows][64]).
+// a_desc / b_desc: K-major SW128 descriptors of the two tiles' first rows.
 template <int DH>
-__device__ __forceinline__ void mma_rows_128x64(uint32_t d_tmem, uint32_t a_base, uint32_t b_base,
+__device__ __forceinline__ void mma_rows_128x64(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                                 uint32_t idesc) {
 #pragma unroll
   for (int kk = 0; kk < DH / 16; ++kk) {
-    mma_bf16_ss(d_tmem, sdesc_sw128(a_base + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024),
-                sdesc_sw128(b_base + (kk >> 2) * (64 * 128) + (kk & 3) * 32, 16, 1024), idesc,
-                kk > 0 ? 1u : 0u);
+    mma_bf16_ss(d_tmem, sdesc_add(a_desc, (kk >> 2) * (128 * 128) + (kk & 3) * 32),
+                sdesc_add(b_desc, (kk >> 2) * (64 * 128) + (kk & 3) * 32), idesc, kk > 0 ? 1u : 0u);
   }
 }
 
 // D[128 × DH] (+)= A[128 × 64] (tensor memory, packed bf16) · B[64 × DH] (shared, MN-major).
 // A's 64 columns are packed as two halves of 32: half h occupies tensor-memory columns
 // 32h .. 32h+15 of the 64-column buffer (each softmax warp-half writes inside the columns it read).
+// b_desc: MN-major SW128 descriptor of B's first row (64-element chunks 64·128 bytes apart).
 template <int DH>
-__device__ __forceinline__ void mma_acc_from_tmem(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base,
+__device__ __forceinline__ void mma_acc_from_tmem(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                                   uint32_t idesc, bool first) {
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk)
-    mma_bf16_ts(d_tmem, a_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
-                sdesc_sw128(b_base + kk * 2048, 64 * 128, 1024), idesc, (!first || kk > 0) ? 1u : 0u);
+    mma_bf16_ts(d_tmem, a_tmem + 32 * (kk >> 1) + 8 * (kk & 1), sdesc_add(b_desc, kk * 2048), idesc,
+                (!first || kk > 0) ? 1u : 0u);
 }
 
 
@@ -737,23 +742,28 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_acc = idesc_bf16(128, DH, false, true);
-      const uint32_t kb = smem_u32(smem + S::OFF_A), vb = smem_u32(smem + S::OFF_B);
+      const uint64_t kd = sdesc_sw128(smem_u32(smem + S::OFF_A), 16, 1024);
+      const uint64_t vd = sdesc_sw128(smem_u32(smem + S::OFF_B), 16, 1024);
       const uint32_t stage0 = smem_u32(smem + S::OFF_STAGE);
+      const uint64_t q_k = sdesc_sw128(stage0, 16, 1024);                          // Q, K-major
+      const uint64_t do_k = sdesc_sw128(stage0 + S::SMALL_TILE, 16, 1024);         // dO, K-major
+      const uint64_t q_mn = sdesc_sw128(stage0, 64 * 128, 1024);                   // Q, MN-major
+      const uint64_t do_mn = sdesc_sw128(stage0 + S::SMALL_TILE, 64 * 128, 1024);  // dO, MN-major
       bool ok = mbar_wait(kv_bar, 0, abort_flag, a.status);
       auto issue_acc = [&](int i) {  // dV += Pᵀ·dOᵢ, dK += dSᵀ·Qᵢ
         const int bf = i & 1;
-        const uint32_t qs = stage0 + (i % S::STAGES) * S::STAGE_BYTES;
-        mma_acc_from_tmem<DH>(tmem + S::TM_ACC, tmem + S::TM_S + bf * 64, qs + S::SMALL_TILE, id_acc, i == 0);
-        mma_acc_from_tmem<DH>(tmem + S::TM_ACC + DH, tmem + S::TM_P + bf * 64, qs, id_acc, i == 0);
+        const uint32_t so = (i % S::STAGES) * S::STAGE_BYTES;
+        mma_acc_from_tmem<DH>(tmem + S::TM_ACC, tmem + S::TM_S + bf * 64, sdesc_add(do_mn, so), id_acc, i == 0);
+        mma_acc_from_tmem<DH>(tmem + S::TM_ACC + DH, tmem + S::TM_P + bf * 64, sdesc_add(q_mn, so), id_acc, i == 0);
         tc_commit(&q_empty[i % S::STAGES]);
       };
       for (int i = 0; i < n_q && ok; ++i) {
         const int st = i % S::STAGES, bf = i & 1;
         if (!mbar_wait(&q_full[st], (i / S::STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t qs = stage0 + st * S::STAGE_BYTES;
-        mma_rows_128x64<DH>(tmem + S::TM_S + bf * 64, kb, qs, id_s);                  // Sᵀ
-        mma_rows_128x64<DH>(tmem + S::TM_P + bf * 64, vb, qs + S::SMALL_TILE, id_s);  // dPᵀ
+        const uint32_t so = st * S::STAGE_BYTES;
+        mma_rows_128x64<DH>(tmem + S::TM_S + bf * 64, kd, sdesc_add(q_k, so), id_s);    // Sᵀ
+        mma_rows_128x64<DH>(tmem + S::TM_P + bf * 64, vd, sdesc_add(do_k, so), id_s);   // dPᵀ
         tc_commit(&s_full[bf]);
         if (i >= 1) {
           if (!mbar_wait(&p_full[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
@@ -776,7 +786,6 @@ __global__ void __launch_bounds__(320, 1)
     const int key = kv0 + kr;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     bool ok = true;
-    // the next tile's Sᵀ / dPᵀ columns are loaded before this tile is released to the MMA warp
     uint32_t rs[32], rp[32];
     if (n_q > 0) {
       ok = mbar_wait(&s_full[0], 0, abort_flag, a.status);
@@ -805,15 +814,19 @@ __global__ void __launch_bounds__(320, 1)
         const float lv[4] = {L.x, L.y, L.z, L.w}, dv4[4] = {D.x, D.y, D.z, D.w};
         float pv[4], sv[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 4; u += 2) {
           const int j = 4 * g4 + u;
-          float p = ex2_approx(fmaf(__uint_as_float(rs[j]), a.scale_log2, -lv[u]));
+          float x0, x1;
+          fma2_b(x0, x1, __uint_as_float(rs[j]), __uint_as_float(rs[j + 1]), a.scale_log2, -lv[u], -lv[u + 1]);
+          pv[u] = ex2_approx(x0);
+          pv[u + 1] = ex2_approx(x1);
           if (!full) {
             const int qq = qc + j;
-            if (!((qq < T) && (key <= qq) && (key > qq - W))) p = 0.f;
+            if (!((qq < T) && (key <= qq) && (key > qq - W))) pv[u] = 0.f;
+            if (!((qq + 1 < T) && (key <= qq + 1) && (key > qq + 1 - W))) pv[u + 1] = 0.f;
           }
-          pv[u] = p;
-          sv[u] = p * (__uint_as_float(rp[j]) - dv4[u]);
+          sub2(sv[u], sv[u + 1], __uint_as_float(rp[j]), __uint_as_float(rp[j + 1]), dv4[u], dv4[u + 1]);
+          mul2(sv[u], sv[u + 1], pv[u], pv[u + 1], sv[u], sv[u + 1]);
         }
         pk[2 * g4] = pack_bf2(pv[0], pv[1]);
         pk[2 * g4 + 1] = pack_bf2(pv[2], pv[3]);
@@ -823,20 +836,18 @@ __global__ void __launch_bounds__(320, 1)
       // packed halves stay inside the columns this warp just read (see mma_acc_from_tmem)
       tmem_st16(tmem + lane_off + S::TM_S + bf * 64 + 32 * half, pk);
       tmem_st16(tmem + lane_off + S::TM_P + bf * 64 + 32 * half, dk);
-      const bool more = (i + 1 < n_q);
-      if (more) {
-        const int nb = (i + 1) & 1;
-        if (!mbar_wait(&s_full[nb], ((i + 1) >> 1) & 1, abort_flag, a.status)) { ok = false; }
-        if (ok) {
-          tc_fence_after();
-          tmem_ld32(tmem + lane_off + S::TM_S + nb * 64 + 32 * half, rs);
-          tmem_ld32(tmem + lane_off + S::TM_P + nb * 64 + 32 * half, rp);
-        }
-      }
+      // release this tile to the MMA warp first, then fetch the next one's columns
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[bf]);
-      if (more && ok) tmem_ld_wait();
+      if (i + 1 < n_q) {
+        const int nb = (i + 1) & 1;
+        if (!mbar_wait(&s_full[nb], ((i + 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        tmem_ld32(tmem + lane_off + S::TM_S + nb * 64 + 32 * half, rs);
+        tmem_ld32(tmem + lane_off + S::TM_P + nb * 64 + 32 * half, rp);
+        tmem_ld_wait();
+      }
     }
     // epilogue: half 0 writes the dV row, half 1 the dK row of each key
     if (ok) ok = mbar_wait(done, 0, abort_flag, a.status);
@@ -954,21 +965,25 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_acc = idesc_bf16(128, DH, false, true);
-      const uint32_t qb = smem_u32(smem + S::OFF_A), dob = smem_u32(smem + S::OFF_B);
+      const uint64_t qd = sdesc_sw128(smem_u32(smem + S::OFF_A), 16, 1024);
+      const uint64_t dod = sdesc_sw128(smem_u32(smem + S::OFF_B), 16, 1024);
       const uint32_t stage0 = smem_u32(smem + S::OFF_STAGE);
+      const uint64_t k_k = sdesc_sw128(stage0, 16, 1024);                   // K, K-major
+      const uint64_t v_k = sdesc_sw128(stage0 + S::SMALL_TILE, 16, 1024);   // V, K-major
+      const uint64_t k_mn = sdesc_sw128(stage0, 64 * 128, 1024);            // K, MN-major
       bool ok = mbar_wait(q_bar, 0, abort_flag, a.status);
       auto issue_acc = [&](int j) {  // dQ += dS·Kⱼ
-        const uint32_t ks = stage0 + (j % S::STAGES) * S::STAGE_BYTES;
-        mma_acc_from_tmem<DH>(tmem + S::TM_ACC, tmem + S::TM_S + (j & 1) * 64, ks, id_acc, j == 0);
+        const uint32_t so = (j % S::STAGES) * S::STAGE_BYTES;
+        mma_acc_from_tmem<DH>(tmem + S::TM_ACC, tmem + S::TM_S + (j & 1) * 64, sdesc_add(k_mn, so), id_acc, j == 0);
         tc_commit(&kv_empty[j % S::STAGES]);
       };
       for (int j = 0; j < n_kv && ok; ++j) {
         const int st = j % S::STAGES, bf = j & 1;
         if (!mbar_wait(&kv_full[st], (j / S::STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t ks = stage0 + st * S::STAGE_BYTES;
-        mma_rows_128x64<DH>(tmem + S::TM_S + bf * 64, qb, ks, id_s);                  // S
-        mma_rows_128x64<DH>(tmem + S::TM_P + bf * 64, dob, ks + S::SMALL_TILE, id_s);  // dP
+        const uint32_t so = st * S::STAGE_BYTES;
+        mma_rows_128x64<DH>(tmem + S::TM_S + bf * 64, qd, sdesc_add(k_k, so), id_s);    // S
+        mma_rows_128x64<DH>(tmem + S::TM_P + bf * 64, dod, sdesc_add(v_k, so), id_s);   // dP
         tc_commit(&s_full[bf]);
         if (j >= 1) {
           if (!mbar_wait(&p_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
@@ -993,7 +1008,6 @@ __global__ void __launch_bounds__(320, 1)
     const float l2 = (t < T) ? a.delta[bh * a.Tpad + t] : 0.f;
     const float dl = (t < T) ? a.delta[((long long)a.B * a.H + bh) * a.Tpad + t] : 0.f;
     bool ok = true;
-    // the next tile's S / dP columns are loaded before this tile is released to the MMA warp
     uint32_t rs[32], rp[32];
     if (n_kv > 0) {
       ok = mbar_wait(&s_full[0], 0, abort_flag, a.status);
@@ -1012,32 +1026,32 @@ __global__ void __launch_bounds__(320, 1)
       uint32_t dk[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        float dv[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int kk = k0 + 2 * e + u;
-          float p = ex2_approx(fmaf(__uint_as_float(rs[2 * e + u]), a.scale_log2, -l2));
-          if (need_mask && !((t < T) && (kk <= t) && (kk > t - W))) p = 0.f;
-          dv[u] = p * (__uint_as_float(rp[2 * e + u]) - dl);
+        float x0, x1, d0, d1;
+        fma2_bc(x0, x1, __uint_as_float(rs[2 * e]), __uint_as_float(rs[2 * e + 1]), a.scale_log2, -l2);
+        float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+        if (need_mask) {
+          const int kk = k0 + 2 * e;
+          if (!((t < T) && (kk <= t) && (kk > t - W))) p0 = 0.f;
+          if (!((t < T) && (kk + 1 <= t) && (kk + 1 > t - W))) p1 = 0.f;
         }
-        dk[e] = pack_bf2(dv[0], dv[1]);
+        add2_bc(d0, d1, __uint_as_float(rp[2 * e]), __uint_as_float(rp[2 * e + 1]), -dl);
+        mul2(d0, d1, p0, p1, d0, d1);
+        dk[e] = pack_bf2(d0, d1);
       }
       // the packed half stays inside the columns this warp just read (see mma_acc_from_tmem)
       tmem_st16(tmem + lane_off + S::TM_S + bf * 64 + 32 * half, dk);
-      const bool more = (j + 1 < n_kv);
-      if (more) {
-        const int nb = (j + 1) & 1;
-        if (!mbar_wait(&s_full[nb], ((j + 1) >> 1) & 1, abort_flag, a.status)) { ok = false; }
-        if (ok) {
-          tc_fence_after();
-          tmem_ld32(tmem + lane_off + S::TM_S + nb * 64 + 32 * half, rs);
-          tmem_ld32(tmem + lane_off + S::TM_P + nb * 64 + 32 * half, rp);
-        }
-      }
+      // release this tile to the MMA warp first, then fetch the next one's columns
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[bf]);
-      if (more && ok) tmem_ld_wait();
+      if (j + 1 < n_kv) {
+        const int nb = (j + 1) & 1;
+        if (!mbar_wait(&s_full[nb], ((j + 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        tmem_ld32(tmem + lane_off + S::TM_S + nb * 64 + 32 * half, rs);
+        tmem_ld32(tmem + lane_off + S::TM_P + nb * 64 + 32 * half, rp);
+        tmem_ld_wait();
+      }
     }
     if (ok) ok = mbar_wait(done, 0, abort_flag, a.status);
     if (ok) {

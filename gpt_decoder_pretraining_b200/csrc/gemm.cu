@@ -263,6 +263,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     // ---------------- MMA issuer (leader CTA) ----------------
     if (leader && lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(2 * BM, BN, A_MN, B_MN);
+      // stage-0 descriptors; stage s and slice kk are constant byte offsets from them
+      const uint32_t s0 = smem_u32(smem);
+      const uint64_t a_desc0 = A_MN ? sdesc_sw128(s0, 8192, 1024) : sdesc_sw128(s0, 16, 1024);
+      const uint64_t b_desc0 = B_MN ? sdesc_sw128(s0 + S::A_BYTES, 8192, 1024)
+                                    : sdesc_sw128(s0 + S::A_BYTES, 16, 1024);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -277,15 +282,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         for (int kt = kt0; kt < kt1; ++kt) {
           if (!mbar_wait(&full[stage], phase, abort_flag, args.status)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * S::STAGE_BYTES);
-          const uint32_t sb = sa + S::A_BYTES;
+          const uint64_t ad = sdesc_add(a_desc0, stage * S::STAGE_BYTES);
+          const uint64_t bd = sdesc_add(b_desc0, stage * S::STAGE_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = A_MN ? sdesc_sw128(sa + kk * 2048, 8192, 1024)
-                                     : sdesc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t bd = B_MN ? sdesc_sw128(sb + kk * 2048, 8192, 1024)
-                                     : sdesc_sw128(sb + kk * 32, 16, 1024);
-            mma_bf16_pair(d_tmem, ad, bd, idesc, (kt > kt0 || kk > 0) ? 1u : 0u);
+            mma_bf16_pair(d_tmem, sdesc_add(ad, A_MN ? kk * 2048 : kk * 32),
+                          sdesc_add(bd, B_MN ? kk * 2048 : kk * 32), idesc,
+                          (kt > kt0 || kk > 0) ? 1u : 0u);
           }
           tc_commit_pair(&empty[stage], 0x3);
           if (++stage == S::STAGES) { stage = 0; phase ^= 1; }

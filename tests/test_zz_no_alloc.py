@@ -65,7 +65,7 @@ def test_noalloc_attention_bwd_rejects_more_rows_than_the_array_holds():
     from gpt_decoder_pretraining_b200 import step as S
     t = torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda")
     lse = torch.zeros(64, dtype=torch.float32, device="cuda")
-    B, H, T, Dh = 1, 16, 65536, 64  # 2·1·16·65536 scratch values > 2^21
+    B, H, T, Dh = 1, 16, 65537, 64  # 2·1·16·65600 scratch values > 2^21
     with pytest.raises(S.GptError) as e:
         S.attention_bwd_noalloc(t, t, t, t, t, lse, t, t, t, 0, (H * T * Dh, T * Dh, Dh),
                                 (H * T * Dh, T * Dh, Dh), B, H, T, Dh)
