@@ -12,10 +12,12 @@ nanochat convention 6·(N − V·d) + 12·H·Dh·Σ_l min(w_l, T).
 * `e2e`: the same metric through the public API (GptStep) with the step's tokens/targets copied
   from pinned host memory and the loss copied back every step, inside the timed region.
 * `roofline`: the GEMM class (the dominant kernel family) — algorithmic FLOPs ÷ its CUDA-event
-  time measured inside the timed region — against the measured sustained bf16 peak.
+  time, from separate profiled steps that record an event around every launch on the step's
+  stream (kept out of the timed region) — against the measured sustained bf16 peak.
 * `cpu_baseline`: the CPU oracle timed on this host on a bounded sample (rank 0, N = 1).
-* N > 1 (torchrun): each rank runs an independent replica on its own batch (weak scaling); the
-  only collectives are the barrier and the max-reduction of the timings.
+* N > 1 (torchrun): data parallel with weak scaling — each rank runs the step on its own batch,
+  then the fp32 gradients are averaged across ranks by one NCCL all-reduce per step (inside the
+  timed region); the barrier and the max-reduction of the timings bracket the measurement.
 """
 from __future__ import annotations
 
@@ -36,6 +38,7 @@ import numpy as np  # noqa: E402
 from gpt_decoder_pretraining_b200.config import B200_DENSE_BF16_PEAK, preset  # noqa: E402
 from gpt_decoder_pretraining_b200.inputs import make_params, make_tokens  # noqa: E402
 
+METRIC = "training tokens/sec and MFU (% of B200 dense BF16) per fwd+bwd step, 1 GPU"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -164,7 +167,7 @@ def run_reference(args, cfg):
     sample = (f"one row of {scfg.seq_len} tokens of the {cfg.name} model (B=1), fp32 NumPy oracle "
               f"fwd+bwd, median of {args.steps} after {args.warmup} warm-up")
     line = {
-        "impl": "reference", "metric": "training tokens/sec per fwd+bwd step, 1 GPU", "value": value,
+        "impl": "reference", "metric": METRIC, "value": value,
         "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic", "mfu": mfu,
@@ -189,6 +192,21 @@ def max_over_ranks(values, world, device="cpu"):
     t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return [float(v) for v in t.cpu()]
+
+
+def average_gradients(grads, world):
+    """Data-parallel exchange: grads ← mean over ranks.  Every rank holds the same number of valid
+    targets, so this is the gradient of the mean loss over the global batch.  NCCL averages in the
+    collective itself; other backends (the CPU tests) sum and divide."""
+    if world <= 1:
+        return grads
+    import torch.distributed as dist
+    if dist.get_backend() == "nccl":
+        dist.all_reduce(grads, op=dist.ReduceOp.AVG)
+    else:
+        dist.all_reduce(grads)
+        grads /= world
+    return grads
 
 
 def whole_job_rate(units_per_rank_step, world, ms_per_step):
@@ -217,6 +235,9 @@ def run_ours(args, cfg):
         if world > 1:
             dist.barrier()
 
+    def exchange(grads):
+        average_gradients(grads, world)
+
     step = GptStep(cfg, device=dev)
     params_np = make_params(cfg.n_params, keep_fp32=(cfg.param_dtype == 1))
     params = torch.from_numpy(params_np).to(dev)
@@ -229,7 +250,8 @@ def run_ours(args, cfg):
 
     # warm-up
     for _ in range(args.warmup):
-        step(params, tokens, targets)
+        _, grads = step(params, tokens, targets)
+        exchange(grads)
     torch.cuda.synchronize(dev)
     st = step.status()
     if st != 0:
@@ -241,20 +263,27 @@ def run_ours(args, cfg):
     clocks = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
     clocks.start()
     time.sleep(0.3)
-    step.set_profiling(True)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
     launches = 0
     e0.record(stream)
     for _ in range(args.steps):
-        step(params, tokens, targets)
+        _, grads = step(params, tokens, targets)
+        exchange(grads)
         launches += step.last_launch_count()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     ms = e0.elapsed_time(e1) / args.steps
     clk = clocks.stop()
+
+    # ---------------- per-kernel breakdown: separate steps with an event around every launch ----------------
+    prof_steps = max(1, min(args.steps, 3))
+    step.set_profiling(True)
+    for _ in range(prof_steps):
+        step(params, tokens, targets)
+    torch.cuda.synchronize(dev)
     step.set_profiling(False)
     prof = step.profile()
 
@@ -270,7 +299,8 @@ def run_ours(args, cfg):
     for _ in range(args.steps):
         tok_d.copy_(tok_h, non_blocking=True)
         tgt_d.copy_(tgt_h, non_blocking=True)
-        loss, _ = step(params, tok_d, tgt_d)
+        loss, grads = step(params, tok_d, tgt_d)
+        exchange(grads)
         loss_h.copy_(loss, non_blocking=True)
     f1.record(stream)
     torch.cuda.synchronize(dev)
@@ -292,8 +322,8 @@ def run_ours(args, cfg):
     for name, (kms, calls, fl, by) in prof.items():
         if calls == 0:
             continue
-        ent = {"ms_per_step": kms / args.steps, "calls_per_step": calls // args.steps,
-               "share": kms / (ms * args.steps)}
+        ent = {"ms_per_step": kms / prof_steps, "calls_per_step": calls // prof_steps,
+               "share": kms / (ms * prof_steps)}
         if fl:
             ent["tflops"] = fl / (kms / 1e3) / 1e12
         if by:
@@ -301,7 +331,7 @@ def run_ours(args, cfg):
         kernels[name] = ent
     workload = f"{cfg.name} GPT fwd+bwd step"
     line = {
-        "metric": "training tokens/sec per fwd+bwd step, 1 GPU (MFU in 'mfu')",
+        "metric": METRIC,
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded N(0,0.02) params, "
@@ -309,7 +339,7 @@ def run_ours(args, cfg):
         "mfu": mfu, "mfu_of_measured_sustained": fpt * value / (world * peak_sus * 1e12),
         "flops_per_token": fpt,
         "config": {"workload": workload, "model": cfg.name, "global_batch": cfg.batch * world,
-                   "seq_len": cfg.seq_len, "parallelism": f"replicas{world}" if world > 1 else "none",
+                   "seq_len": cfg.seq_len, "parallelism": f"dp{world}" if world > 1 else "none",
                    "depth": cfg.depth, "d_model": cfg.d_model, "vocab": cfg.vocab,
                    "windows": "SSSL w=1024" if any(cfg.windows) else "full causal",
                    "l2": "inputs larger than L2 (activations ~tens of GB), no flush"},

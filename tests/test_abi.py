@@ -128,7 +128,7 @@ def test_kernel_entry_points_reject_bad_arguments(lib):
 
 
 def test_multi_rank_timing_uses_the_slowest_rank():
-    """bench.py with N>1 ranks: replicas, the job time is the max over ranks (gloo, 2 processes)."""
+    """bench.py with N>1 ranks: the job time is the max over ranks (gloo, 2 processes)."""
     import torch.multiprocessing as mp
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
@@ -157,3 +157,49 @@ def _rank_main(rank, world, port, q):
     rate = bench.whole_job_rate(32768, world, ms[0])
     dist.destroy_process_group()
     q.put((rank, (ms, rate)))
+
+
+def test_data_parallel_average_equals_the_full_batch_step():
+    """Two gloo ranks each take the oracle step on one row; bench.average_gradients over the ranks
+    gives the oracle gradient of the two-row batch (equal valid counts per rank)."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 30500 + (os.getpid() % 1000)
+    procs = [ctx.Process(target=_dp_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = dict(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    from oracle import gpt_oracle as O
+    from gpt_decoder_pretraining_b200.config import custom
+    from gpt_decoder_pretraining_b200.inputs import make_params, make_tokens
+    cfg = custom(2, 32, 16, 64, 12, 2, param_dtype=1)
+    params = make_params(cfg.n_params, keep_fp32=True, std=0.3).astype(np.float64)
+    tok, tgt = make_tokens(2, 12, 64, seed=1)
+    full = O.step(cfg, params, tok, tgt)
+    for r in range(2):
+        np.testing.assert_allclose(out[r], full["grads"], rtol=0, atol=1e-12)
+
+
+def _dp_rank_main(rank, world, port, q):
+    import sys
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch
+    import torch.distributed as dist
+    import bench
+    from oracle import gpt_oracle as O
+    from gpt_decoder_pretraining_b200.config import custom
+    from gpt_decoder_pretraining_b200.inputs import make_params, make_tokens
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    cfg1 = custom(2, 32, 16, 64, 12, 1, param_dtype=1)
+    params = make_params(cfg1.n_params, keep_fp32=True, std=0.3).astype(np.float64)
+    tok, tgt = make_tokens(2, 12, 64, seed=1)
+    g = torch.from_numpy(O.step(cfg1, params, tok[rank:rank + 1], tgt[rank:rank + 1])["grads"])
+    bench.average_gradients(g, world)
+    dist.destroy_process_group()
+    q.put((rank, g.numpy()))
