@@ -40,6 +40,7 @@ struct AttnArgs {
   float* lse;
   float* delta;  // backward: [2][B·H][Tpad] fp32 — LSE·log2(e), then rowsum(dO∘O); zero-padded
   int Tpad;      // T rounded up to a multiple of 64
+  uint16_t* ext; // backward: [2][B·H][Tpad][8] bf16 rows [hi, mid, lo, 0…] of −LSE·√Dh, −delta
   int* status;
   // optional QK-norm + RoPE backward fused into the dq / dk epilogues (rho_q == nullptr: off):
   // q̃ = RMS_Dh(RoPE(q)), so dq = Rᵀ·rho·(dq̃ − q̃·mean(q̃·dq̃)), likewise for k
@@ -388,8 +389,8 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
   } else if (warp == 9) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
+    // ---------------- MMA issuer: the warp runs the loop, one elected lane issues ----------------
+    {
       constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
       constexpr uint32_t id_o = idesc_bf16(128, DH, false, true);
       // descriptors of stage 0 / tile 0, advanced by constant offsets in the loops
@@ -399,23 +400,30 @@ __global__ void __launch_bounds__(320, 1)
       auto issue_s = [&](int x, int j) {
         const uint64_t q_desc = sdesc_add(qd, x * S::Q_TILE);
         const uint64_t k_desc = sdesc_add(kd, (j & 1) * S::KV_TILE);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_bf16_ss(tmem + S::TM_S + x * 128, sdesc_add(q_desc, off), sdesc_add(k_desc, off), id_s,
-                      kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < DH / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            mma_bf16_ss(tmem + S::TM_S + x * 128, sdesc_add(q_desc, off), sdesc_add(k_desc, off), id_s,
+                        kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&s_full[x]);
         }
-        tc_commit(&s_full[x]);
+        __syncwarp();
       };
-      auto issue_pv = [&](int x, int j) {
+      auto issue_pv = [&](int x, int j, bool release_kv) {
         const uint64_t v_desc = sdesc_add(vd, (j & 1) * S::KV_TILE);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + S::TM_O + x * DH, tmem + S::TM_S + x * 128 + kk * 8,
-                      sdesc_add(v_desc, kk * 2048), id_o, (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(tmem + S::TM_O + x * DH, tmem + S::TM_S + x * 128 + kk * 8,
+                        sdesc_add(v_desc, kk * 2048), id_o, (j > 0 || kk > 0) ? 1u : 0u);
+          if (release_kv) tc_commit(&kv_empty[j & 1]);
+        }
+        __syncwarp();
       };
-      bool ok = mbar_wait(bar_q, 0, abort_flag, a.status);
-      if (ok) ok = mbar_wait(&kv_full[0], 0, abort_flag, a.status);
+      bool ok = mbar_wait_warp(bar_q, 0, abort_flag, a.status);
+      if (ok) ok = mbar_wait_warp(&kv_full[0], 0, abort_flag, a.status);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
@@ -423,13 +431,12 @@ __global__ void __launch_bounds__(320, 1)
       }
       for (int j = 0; j < n_kv && ok; ++j) {
         for (int x = 0; x < 2 && ok; ++x) {
-          if (!mbar_wait(&p_full[x], j & 1, abort_flag, a.status)) { ok = false; break; }
+          if (!mbar_wait_warp(&p_full[x], j & 1, abort_flag, a.status)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(x, j);
-          if (x == 1) tc_commit(&kv_empty[j & 1]);
+          issue_pv(x, j, x == 1);
           if (j + 1 < n_kv) {
             if (x == 0) {
-              if (!mbar_wait(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag, a.status)) {
+              if (!mbar_wait_warp(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag, a.status)) {
                 ok = false;
                 break;
               }
@@ -439,7 +446,8 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
       }
-      tc_commit(o_full);
+      if (elect_one()) tc_commit(o_full);
+      __syncwarp();
     }
   } else {
     // ---------------- softmax warpgroups ----------------
@@ -561,8 +569,15 @@ struct TcBwdShape {
   static constexpr int OFF_B = BIG_TILE;               // V (dkdv) or dO (dq)
   static constexpr int OFF_STAGE = 2 * BIG_TILE;       // stages of (Q, dO) or (K, V)
   static constexpr int STAGE_BYTES = 2 * SMALL_TILE;
-  static constexpr int OFF_RED = OFF_STAGE + STAGES * STAGE_BYTES;  // [stage][lse2 | delta][64] fp32
-  static constexpr int OFF_BAR = OFF_RED + STAGES * 128 * 4;
+  // dK/dV kernel only: the K = 16 extension operands that fold −LSE and −delta into the Sᵀ / dPᵀ
+  // accumulators (unswizzled core-matrix layout, 16-byte rows).  A_EXT: 128 key rows of
+  // [1, 1, 1, 0, …]; per stage the query tile's [hi, mid, lo, 0, …] rows of −LSE·√Dh and −delta;
+  // ZERO: the second K core column of every extension operand.
+  static constexpr int EXT_ROWS_BYTES = 64 * 16;                     // one 64-row extension tile
+  static constexpr int OFF_A_EXT = OFF_STAGE + STAGES * STAGE_BYTES;  // 128 rows × 16 B
+  static constexpr int OFF_EXT = OFF_A_EXT + 128 * 16;                 // [stage][lse | delta] tiles
+  static constexpr int OFF_ZERO = OFF_EXT + STAGES * 2 * EXT_ROWS_BYTES;
+  static constexpr int OFF_BAR = OFF_ZERO + 128 * 16;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr int THREADS = 320;  // 8 softmax warps (two per TMEM lane quarter), TMA, MMA
   static constexpr int TM_S = 0, TM_P = 128, TM_ACC = 256;  // S[b] at b·64, dP[b] at 128 + b·64
@@ -671,11 +686,10 @@ template <int DH>
 __global__ void __launch_bounds__(320, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                             const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
-                            const __grid_constant__ CUtensorMap mpad, const AttnArgs a) {
+                            const __grid_constant__ CUtensorMap mext, const AttnArgs a) {
   using S = TcBwdShape<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  float* red = reinterpret_cast<float*>(smem + S::OFF_RED);  // [buf][0 = lse2, 1 = delta][64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
   uint64_t* kv_bar = bars;
   uint64_t* q_full = bars + 1;                // [STAGES]
@@ -709,6 +723,12 @@ __global__ void __launch_bounds__(320, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  // constant extension operands: A_EXT rows [1, 1, 1, 0, 0, 0, 0, 0] (bf16), ZERO all zeros
+  for (int r = threadIdx.x; r < 128; r += blockDim.x) {
+    *reinterpret_cast<uint4*>(smem + S::OFF_A_EXT + 16 * r) = make_uint4(0x3F803F80u, 0x3F80u, 0u, 0u);
+    *reinterpret_cast<uint4*>(smem + S::OFF_ZERO + 16 * r) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  fence_proxy_async_smem();
   if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -724,22 +744,24 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive_expect_tx(kv_bar, 2 * S::BIG_TILE);
       load_tile<DH, 128>(smem + S::OFF_A, &mk, kv_bar, kv0, h, b);
       load_tile<DH, 128>(smem + S::OFF_B, &mv, kv_bar, kv0, h, b);
-      const int bhrows = a.B * a.H;
+      const int rows = a.B * a.H * a.Tpad;
       for (int i = 0; i < n_q; ++i) {
         const int st = i % S::STAGES;
         if (!mbar_wait(&q_empty[st], ((i / S::STAGES) & 1) ^ 1, abort_flag, a.status)) break;
         const int t0 = (q_first + i) * 64;
-        mbar_arrive_expect_tx(&q_full[st], S::STAGE_BYTES + 2 * 64 * 4);
+        mbar_arrive_expect_tx(&q_full[st], S::STAGE_BYTES + 2 * S::EXT_ROWS_BYTES);
         uint8_t* dst = smem + S::OFF_STAGE + st * S::STAGE_BYTES;
         load_tile<DH, 64>(dst, &mq, &q_full[st], t0, h, b);
         load_tile<DH, 64>(dst + S::SMALL_TILE, &mdo, &q_full[st], t0, h, b);
-        tma_load_2d(red + st * 128, &mpad, &q_full[st], t0, (int)bh);
-        tma_load_2d(red + st * 128 + 64, &mpad, &q_full[st], t0, bhrows + (int)bh);
+        uint8_t* ext = smem + S::OFF_EXT + st * 2 * S::EXT_ROWS_BYTES;
+        const int row = (int)bh * a.Tpad + t0;
+        tma_load_2d(ext, &mext, &q_full[st], 0, row);                              // −LSE·√Dh
+        tma_load_2d(ext + S::EXT_ROWS_BYTES, &mext, &q_full[st], 0, rows + row);  // −delta
       }
     }
   } else if (warp == 9) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
+    // ---------------- MMA issuer: the warp runs the loop, one elected lane issues ----------------
+    {
       constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_acc = idesc_bf16(128, DH, false, true);
       const uint64_t kd = sdesc_sw128(smem_u32(smem + S::OFF_A), 16, 1024);
@@ -749,35 +771,57 @@ __global__ void __launch_bounds__(320, 1)
       const uint64_t do_k = sdesc_sw128(stage0 + S::SMALL_TILE, 16, 1024);         // dO, K-major
       const uint64_t q_mn = sdesc_sw128(stage0, 64 * 128, 1024);                   // Q, MN-major
       const uint64_t do_mn = sdesc_sw128(stage0 + S::SMALL_TILE, 64 * 128, 1024);  // dO, MN-major
-      bool ok = mbar_wait(kv_bar, 0, abort_flag, a.status);
+      // extension operands (K = 16, unswizzled): core matrices 128 B apart along M/N, the second
+      // K core column read from the zero block
+      const uint32_t a_ext = smem_u32(smem + S::OFF_A_EXT);
+      const uint64_t a_ext_d = sdesc_plain(a_ext, S::OFF_ZERO - S::OFF_A_EXT, 128);
+      const uint32_t ext0 = smem_u32(smem + S::OFF_EXT);
+      const uint64_t el_d = sdesc_plain(ext0, S::OFF_ZERO - S::OFF_EXT, 128);
+      const uint64_t ed_d = sdesc_plain(ext0 + S::EXT_ROWS_BYTES, S::OFF_ZERO - S::OFF_EXT - S::EXT_ROWS_BYTES, 128);
+      bool ok = mbar_wait_warp(kv_bar, 0, abort_flag, a.status);
       auto issue_acc = [&](int i) {  // dV += Pᵀ·dOᵢ, dK += dSᵀ·Qᵢ
         const int bf = i & 1;
         const uint32_t so = (i % S::STAGES) * S::STAGE_BYTES;
-        mma_acc_from_tmem<DH>(tmem + S::TM_ACC, tmem + S::TM_S + bf * 64, sdesc_add(do_mn, so), id_acc, i == 0);
-        mma_acc_from_tmem<DH>(tmem + S::TM_ACC + DH, tmem + S::TM_P + bf * 64, sdesc_add(q_mn, so), id_acc, i == 0);
-        tc_commit(&q_empty[i % S::STAGES]);
+        if (elect_one()) {
+          mma_acc_from_tmem<DH>(tmem + S::TM_ACC, tmem + S::TM_S + bf * 64, sdesc_add(do_mn, so), id_acc, i == 0);
+          mma_acc_from_tmem<DH>(tmem + S::TM_ACC + DH, tmem + S::TM_P + bf * 64, sdesc_add(q_mn, so), id_acc, i == 0);
+          tc_commit(&q_empty[i % S::STAGES]);
+        }
+        __syncwarp();
       };
       for (int i = 0; i < n_q && ok; ++i) {
         const int st = i % S::STAGES, bf = i & 1;
-        if (!mbar_wait(&q_full[st], (i / S::STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&q_full[st], (i / S::STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t so = st * S::STAGE_BYTES;
-        mma_rows_128x64<DH>(tmem + S::TM_S + bf * 64, kd, sdesc_add(q_k, so), id_s);    // Sᵀ
-        mma_rows_128x64<DH>(tmem + S::TM_P + bf * 64, vd, sdesc_add(do_k, so), id_s);   // dPᵀ
-        tc_commit(&s_full[bf]);
+        // the extension tiles of stage st sit st·2 tiles further from the zero block: their K
+        // core stride shrinks by the same amount (descriptor bits 16..29 hold it in 16-byte units)
+        const uint64_t lbo_fix = (uint64_t)((st * 2 * S::EXT_ROWS_BYTES) >> 4) << 16;
+        const uint32_t eo = st * 2 * S::EXT_ROWS_BYTES;
+        const uint64_t el_st = sdesc_add(el_d, eo) - lbo_fix, ed_st = sdesc_add(ed_d, eo) - lbo_fix;
+        const uint64_t q_st = sdesc_add(q_k, so), do_st = sdesc_add(do_k, so);
+        if (elect_one()) {
+          mma_rows_128x64<DH>(tmem + S::TM_S + bf * 64, kd, q_st, id_s);    // Sᵀ
+          mma_bf16_ss(tmem + S::TM_S + bf * 64, a_ext_d, el_st, id_s, 1u);
+          mma_rows_128x64<DH>(tmem + S::TM_P + bf * 64, vd, do_st, id_s);   // dPᵀ
+          mma_bf16_ss(tmem + S::TM_P + bf * 64, a_ext_d, ed_st, id_s, 1u);
+          tc_commit(&s_full[bf]);
+        }
+        __syncwarp();
         if (i >= 1) {
-          if (!mbar_wait(&p_full[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+          if (!mbar_wait_warp(&p_full[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
           tc_fence_after();
           issue_acc(i - 1);
         }
       }
       if (ok && n_q >= 1) {
-        if (mbar_wait(&p_full[(n_q - 1) & 1], ((n_q - 1) >> 1) & 1, abort_flag, a.status)) {
+        if (mbar_wait_warp(&p_full[(n_q - 1) & 1], ((n_q - 1) >> 1) & 1, abort_flag, a.status)) {
           tc_fence_after();
           issue_acc(n_q - 1);
         }
       }
-      tc_commit(done);
+      if (elect_one()) tc_commit(done);
+      __syncwarp();
     }
   } else {
     // ---------------- softmax-backward warps: thread = key row, warp half = 32 of the 64 queries
@@ -799,39 +843,25 @@ __global__ void __launch_bounds__(320, 1)
     for (int i = 0; i < n_q && ok; ++i) {
       const int bf = i & 1;
       const int qc = (q_first + i) * 64 + 32 * half;  // first query of this warp's 32 columns
-      const int st = i % S::STAGES;
-      // already complete (the MMA warp waited on it); makes the TMA-written rows visible here
-      if (!mbar_wait(&q_full[st], (i / S::STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
-      const float4* l2v = reinterpret_cast<const float4*>(red + st * 128 + 32 * half);
-      const float4* dlv = reinterpret_cast<const float4*>(red + st * 128 + 64 + 32 * half);
       // every (key, query) of the warp visible: no per-element mask
       const int kmin = kv0 + 32 * quarter, kmax_ = kmin + 31;
       const bool full = (kmax_ <= qc) && (kmin > qc + 31 - W) && (qc + 31 < T);
+      // the accumulators already hold Sᵀ − LSE/scale and dPᵀ − delta (extension MMAs)
       uint32_t pk[16], dk[16];
 #pragma unroll
-      for (int g4 = 0; g4 < 8; ++g4) {
-        const float4 L = l2v[g4], D = dlv[g4];
-        const float lv[4] = {L.x, L.y, L.z, L.w}, dv4[4] = {D.x, D.y, D.z, D.w};
-        float pv[4], sv[4];
-#pragma unroll
-        for (int u = 0; u < 4; u += 2) {
-          const int j = 4 * g4 + u;
-          float x0, x1;
-          fma2_b(x0, x1, __uint_as_float(rs[j]), __uint_as_float(rs[j + 1]), a.scale_log2, -lv[u], -lv[u + 1]);
-          pv[u] = ex2_approx(x0);
-          pv[u + 1] = ex2_approx(x1);
-          if (!full) {
-            const int qq = qc + j;
-            if (!((qq < T) && (key <= qq) && (key > qq - W))) pv[u] = 0.f;
-            if (!((qq + 1 < T) && (key <= qq + 1) && (key > qq + 1 - W))) pv[u + 1] = 0.f;
-          }
-          sub2(sv[u], sv[u + 1], __uint_as_float(rp[j]), __uint_as_float(rp[j + 1]), dv4[u], dv4[u + 1]);
-          mul2(sv[u], sv[u + 1], pv[u], pv[u + 1], sv[u], sv[u + 1]);
+      for (int e = 0; e < 16; ++e) {
+        const int j = 2 * e;
+        float x0, x1, s0, s1;
+        mul2_b(x0, x1, __uint_as_float(rs[j]), __uint_as_float(rs[j + 1]), a.scale_log2);
+        float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+        if (!full) {
+          const int qq = qc + j;
+          if (!((qq < T) && (key <= qq) && (key > qq - W))) p0 = 0.f;
+          if (!((qq + 1 < T) && (key <= qq + 1) && (key > qq + 1 - W))) p1 = 0.f;
         }
-        pk[2 * g4] = pack_bf2(pv[0], pv[1]);
-        pk[2 * g4 + 1] = pack_bf2(pv[2], pv[3]);
-        dk[2 * g4] = pack_bf2(sv[0], sv[1]);
-        dk[2 * g4 + 1] = pack_bf2(sv[2], sv[3]);
+        mul2(s0, s1, p0, p1, __uint_as_float(rp[j]), __uint_as_float(rp[j + 1]));
+        pk[e] = pack_bf2(p0, p1);
+        dk[e] = pack_bf2(s0, s1);
       }
       // packed halves stay inside the columns this warp just read (see mma_acc_from_tmem)
       tmem_st16(tmem + lane_off + S::TM_S + bf * 64 + 32 * half, pk);
@@ -962,7 +992,7 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
   } else if (warp == 9) {
-    if (lane == 0) {
+    {  // the warp runs the loop, one elected lane issues
       constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_acc = idesc_bf16(128, DH, false, true);
       const uint64_t qd = sdesc_sw128(smem_u32(smem + S::OFF_A), 16, 1024);
@@ -971,33 +1001,41 @@ __global__ void __launch_bounds__(320, 1)
       const uint64_t k_k = sdesc_sw128(stage0, 16, 1024);                   // K, K-major
       const uint64_t v_k = sdesc_sw128(stage0 + S::SMALL_TILE, 16, 1024);   // V, K-major
       const uint64_t k_mn = sdesc_sw128(stage0, 64 * 128, 1024);            // K, MN-major
-      bool ok = mbar_wait(q_bar, 0, abort_flag, a.status);
+      bool ok = mbar_wait_warp(q_bar, 0, abort_flag, a.status);
       auto issue_acc = [&](int j) {  // dQ += dS·Kⱼ
         const uint32_t so = (j % S::STAGES) * S::STAGE_BYTES;
-        mma_acc_from_tmem<DH>(tmem + S::TM_ACC, tmem + S::TM_S + (j & 1) * 64, sdesc_add(k_mn, so), id_acc, j == 0);
-        tc_commit(&kv_empty[j % S::STAGES]);
+        if (elect_one()) {
+          mma_acc_from_tmem<DH>(tmem + S::TM_ACC, tmem + S::TM_S + (j & 1) * 64, sdesc_add(k_mn, so), id_acc, j == 0);
+          tc_commit(&kv_empty[j % S::STAGES]);
+        }
+        __syncwarp();
       };
       for (int j = 0; j < n_kv && ok; ++j) {
         const int st = j % S::STAGES, bf = j & 1;
-        if (!mbar_wait(&kv_full[st], (j / S::STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&kv_full[st], (j / S::STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t so = st * S::STAGE_BYTES;
-        mma_rows_128x64<DH>(tmem + S::TM_S + bf * 64, qd, sdesc_add(k_k, so), id_s);    // S
-        mma_rows_128x64<DH>(tmem + S::TM_P + bf * 64, dod, sdesc_add(v_k, so), id_s);   // dP
-        tc_commit(&s_full[bf]);
+        const uint64_t k_st = sdesc_add(k_k, so), v_st = sdesc_add(v_k, so);
+        if (elect_one()) {
+          mma_rows_128x64<DH>(tmem + S::TM_S + bf * 64, qd, k_st, id_s);    // S
+          mma_rows_128x64<DH>(tmem + S::TM_P + bf * 64, dod, v_st, id_s);   // dP
+          tc_commit(&s_full[bf]);
+        }
+        __syncwarp();
         if (j >= 1) {
-          if (!mbar_wait(&p_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+          if (!mbar_wait_warp(&p_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
           tc_fence_after();
           issue_acc(j - 1);
         }
       }
       if (ok && n_kv >= 1) {
-        if (mbar_wait(&p_full[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort_flag, a.status)) {
+        if (mbar_wait_warp(&p_full[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort_flag, a.status)) {
           tc_fence_after();
           issue_acc(n_kv - 1);
         }
       }
-      tc_commit(done);
+      if (elect_one()) tc_commit(done);
+      __syncwarp();
     }
   } else {
     // ---------------- softmax-backward warps: thread = query row, warp half = 32 of the 64 keys
@@ -1129,10 +1167,20 @@ __global__ void attn_kmax_kernel(const uint16_t* __restrict__ k, float* __restri
 // ================================================================================================
 // backward (1): delta = rowsum(dO ∘ O), one warp per row
 // ================================================================================================
+// v as hi + mid + lo in bf16 (each a round-to-nearest-even of the remainder): ~24 significant bits
+__device__ __forceinline__ uint2 split3_bf16(float v) {
+  const uint16_t hi = f2bf(v);
+  const float r1 = v - bf2f(hi);
+  const uint16_t mid = f2bf(r1);
+  const uint16_t lo = f2bf(r1 - bf2f(mid));
+  return make_uint2((uint32_t)hi | ((uint32_t)mid << 16), (uint32_t)lo);
+}
+
 __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
-                                  const float* __restrict__ lse, float* __restrict__ pad, int B,
-                                  int H, int T, int Tpad, int Dh, long long sb, long long sh,
-                                  long long st, long long sbd, long long shd, long long std_) {
+                                  const float* __restrict__ lse, float* __restrict__ pad,
+                                  uint16_t* __restrict__ ext, float ext_scale, int B, int H, int T,
+                                  int Tpad, int Dh, long long sb, long long sh, long long st,
+                                  long long sbd, long long shd, long long std_) {
   // one warp per padded row (b, h, t < Tpad): pad[0][bh][t] = lse·log2(e), pad[1][bh][t] =
   // rowsum(dO∘O); rows t ≥ T are zero
   const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -1155,8 +1203,16 @@ __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t
 #pragma unroll
   for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
   if (lane == 0) {
-    pad[warp] = (t < T) ? lse[bh * T + t] * LOG2E : 0.f;
+    const float l = (t < T) ? lse[bh * T + t] : 0.f;
+    pad[warp] = l * LOG2E;
     pad[rows + warp] = acc;
+    if (ext != nullptr) {
+      // (Sᵀ + ext)·scale·log2 e = s·scale·log2 e − LSE·log2 e  and  dPᵀ + ext = dP − delta
+      const uint2 el = (t < T) ? split3_bf16(-l * ext_scale) : make_uint2(0, 0);
+      const uint2 ed = split3_bf16(-acc);
+      *reinterpret_cast<uint4*>(ext + warp * 8) = make_uint4(el.x, el.y, 0, 0);
+      *reinterpret_cast<uint4*>(ext + (rows + warp) * 8) = make_uint4(ed.x, ed.y, 0, 0);
+    }
   }
 }
 
@@ -1549,10 +1605,10 @@ gpt_status launch_bwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, c
 }
 
 // tcgen05 backward: maps with 128-row boxes (outer tiles) and 64-row boxes (inner tiles), and the
-// padded [2·B·H][Tpad] fp32 LSE / delta array in 64-float boxes.
+// [2·B·H·Tpad][8] bf16 extension rows in 64-row boxes.
 template <int DH>
 gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[4],
-                         const CUtensorMap& mpad, AttnArgs a, void* dq, cudaStream_t stream) {
+                         const CUtensorMap& mext, AttnArgs a, void* dq, cudaStream_t stream) {
   using S = TcBwdShape<DH>;
   static bool once = false;
   if (!once) {
@@ -1563,7 +1619,7 @@ gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[
   // dK/dV: outer 128-key tiles (K, V with 128-row boxes), inner 64-query tiles (Q, dO 64-row boxes)
   dim3 g1((a.T + 127) / 128, a.H, a.B);
   attn_bwd_dkdv_tc_kernel<DH><<<g1, S::THREADS, S::SMEM, stream>>>(m64[0], m128[1], m128[2], m64[3],
-                                                                   mpad, a);
+                                                                   mext, a);
   count_launch();
   GPT_CUDA_TRY(cudaGetLastError());
   // dQ: outer 128-query tiles (Q, dO 128-row boxes), inner 64-key tiles (K, V 64-row boxes)
@@ -1622,6 +1678,13 @@ gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, f
   return launch_fwd_tc<64>(mq2, mk2, mv2, a, kmax_scratch, kconst, stream);
 }
 
+// Backward scratch per padded row (b, h, t < ⌈T/64⌉·64): LSE·log2 e and delta (fp32), and the two
+// 16-byte extension rows of the dK/dV kernel.
+size_t attention_bwd_scratch_bytes(int B, int H, int T) {
+  if (B <= 0 || H <= 0 || T <= 0) return 0;
+  return (size_t)B * H * ((T + 63) / 64 * 64) * (2 * sizeof(float) + 2 * 16);
+}
+
 // Strides: (sbq, shq, stq) for q, k, v; (sbg, shg, stg) for dq, dk, dv; (sbo, sho, sto) for o;
 // (sbd, shd, std_) for dO.
 gpt_status attention_bwd(const void* q, const void* k, const void* v, const void* o,
@@ -1647,23 +1710,25 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
       !make_head_map(&mdo, dout, B, H, T, Dh, sbd, shd, std_, 64))
     return GPT_ERR_UNSUPPORTED_SHAPE;
   const int Tpad = (T + 63) / 64 * 64;
-  // the tensor-core kernels fetch the padded LSE / delta rows with TMA (64-float boxes)
-  CUtensorMap mpad;
+  // scratch: [2][B·H][Tpad] fp32 (LSE·log2 e, delta), then the dK/dV kernel's extension rows
+  // [2][B·H][Tpad][8] bf16, fetched with TMA in 64-row boxes
+  const long long rows = (long long)B * H * Tpad;
+  uint16_t* ext = (Dh != 32) ? reinterpret_cast<uint16_t*>(delta + 2 * rows) : nullptr;
+  CUtensorMap mext;
   if (Dh != 32) {
-    const uint64_t dims[2] = {(uint64_t)Tpad, (uint64_t)2 * B * H};
-    const uint64_t strides[1] = {(uint64_t)Tpad * 4};
-    const uint32_t box[2] = {64, 1};
-    if ((reinterpret_cast<uintptr_t>(delta) & 15) != 0 ||
-        !encode_map_f32(&mpad, delta, 2, dims, strides, box))
+    const uint64_t dims[2] = {8, (uint64_t)(2 * rows)};
+    const uint64_t strides[1] = {16};
+    const uint32_t box[2] = {8, 64};
+    if ((reinterpret_cast<uintptr_t>(delta) & 15) != 0 || 2 * rows >= (1ll << 31) ||
+        !encode_map_bf16(&mext, ext, 2, dims, strides, box, false))
       return GPT_ERR_UNSUPPORTED_SHAPE;
   }
   {
-    const long long rows = (long long)B * H * Tpad;
     const int threads = 256;
     const long long blocks = (rows * 32 + threads - 1) / threads;
     attn_delta_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
-        reinterpret_cast<const uint16_t*>(o), reinterpret_cast<const uint16_t*>(dout), lse, delta, B,
-        H, T, Tpad, Dh, sbo, sho, sto, sbd, shd, std_);
+        reinterpret_cast<const uint16_t*>(o), reinterpret_cast<const uint16_t*>(dout), lse, delta,
+        ext, sqrtf((float)Dh), B, H, T, Tpad, Dh, sbo, sho, sto, sbd, shd, std_);
     count_launch();
     GPT_CUDA_TRY(cudaGetLastError());
   }
@@ -1675,6 +1740,7 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   a.lse = const_cast<float*>(lse);
   a.delta = delta;
   a.Tpad = Tpad;
+  a.ext = ext;
   a.status = status;
   a.sb_o = sbg; a.sh_o = shg; a.st_o = stg;  // strides of the dq/dk/dv outputs
   a.rho_q = rho_q;
@@ -1695,8 +1761,8 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
                        is_do ? std_ : stq, 64))
       return GPT_ERR_UNSUPPORTED_SHAPE;
   }
-  if (Dh == 128) GPT_TRY(launch_bwd_tc<128>(m128, m64, mpad, a, dq, stream));
-  else GPT_TRY(launch_bwd_tc<64>(m128, m64, mpad, a, dq, stream));
+  if (Dh == 128) GPT_TRY(launch_bwd_tc<128>(m128, m64, mext, a, dq, stream));
+  else GPT_TRY(launch_bwd_tc<64>(m128, m64, mext, a, dq, stream));
   return GPT_OK;
 }
 
@@ -1732,7 +1798,8 @@ gpt_status attention_bwd_noalloc(const void* q, const void* k, const void* v, co
                                  long long shq, long long stq, long long sbo, long long sho,
                                  long long sto, int* status, cudaStream_t stream) {
   if (B <= 0 || H <= 0 || T <= 0) return GPT_ERR_INVALID_ARG;
-  if (2ll * B * H * ((T + 63) / 64 * 64) > NOALLOC_DELTA_ROWS) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)attention_bwd_scratch_bytes(B, H, T) > NOALLOC_DELTA_ROWS * 4)
+    return GPT_ERR_UNSUPPORTED_SHAPE;
   float* delta = nullptr;
   GPT_TRY(noalloc_delta_ptr(&delta));
   return attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, T, Dh, window, sbq, shq, stq,
@@ -1763,8 +1830,7 @@ extern "C" gpt_status gpt_attention_bwd(const void* q, const void* k, const void
 }
 
 extern "C" size_t gpt_attention_bwd_scratch_bytes(int B, int H, int T) {
-  if (B <= 0 || H <= 0 || T <= 0) return 0;
-  return (size_t)2 * B * H * ((T + 63) / 64 * 64) * sizeof(float);
+  return gpt::attention_bwd_scratch_bytes(B, H, T);
 }
 
 extern "C" gpt_status gpt_attention_bwd_noalloc(const void* q, const void* k, const void* v,

@@ -218,6 +218,18 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return d;
 }
 
+// Shared-memory descriptor for an unswizzled K-major tile of 8-row × 16-byte core matrices:
+// lbo_bytes = distance between core matrices adjacent along K, sbo_bytes = along M/N.
+__device__ __forceinline__ uint64_t sdesc_plain(uint32_t saddr, uint32_t lbo_bytes,
+                                                uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for tcgen05; layout type 0 = no swizzle
+  return d;
+}
+
 // A descriptor advanced by `bytes` (a multiple of 16 that keeps the address inside shared memory):
 // the start address sits in the low 14 bits as address >> 4, so this is one integer add.  Issue
 // loops form their descriptors this way from bases computed once, keeping the MMA thread's
@@ -338,6 +350,16 @@ __device__ __forceinline__ void add2_bc(float& d0, float& d1, float a0, float a1
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(c));
 }
+// (d0, d1) = (a0·b, a1·b)
+__device__ __forceinline__ void mul2_b(float& d0, float& d1, float a0, float a1, float b) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %4};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b));
+}
 // (d0, d1) = (a0·b0, a1·b1)
 __device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
   asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
@@ -369,6 +391,24 @@ __device__ __forceinline__ void sub2(float& d0, float& d1, float a0, float a1, f
       "mov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// One lane of the (converged) warp: the tcgen05 issue loops run warp-wide, so their loop state
+// and descriptors are warp-uniform, and only the elected lane issues the MMAs and commits.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+// mbar_wait by every lane of a warp; the verdict is made warp-uniform.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                               int* status) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, status);
+  return __all_sync(0xffffffffu, ok) != 0;
 }
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }

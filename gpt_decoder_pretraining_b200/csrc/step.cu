@@ -32,6 +32,7 @@ gpt_status rope_qknorm_bwd_heads(void* dqkv, const void* y_heads, const float* r
 gpt_status embedding_fwd(const int32_t* tok, const void* wte, void* x, int M, int d, int V,
                          int* status, cudaStream_t s);
 size_t embedding_bwd_scratch_bytes(int M, int d, int V);
+size_t attention_bwd_scratch_bytes(int B, int H, int T);
 gpt_status embedding_bwd(const int32_t* tok, const float* gx, float* dwte, int M, int d, int V,
                          void* scratch, cudaStream_t s);
 gpt_status ce_rows(const float2* stats, int ntiles, const float* zt, const int32_t* targets, int M,
@@ -196,7 +197,7 @@ static Plan make_plan(const gpt_config& c, size_t n_params) {
   p.dr = take(M * d * 2);
   p.dO = take(M * d * 2);
   p.dqkv = take(M * 3 * d * 2);
-  p.delta = take(2 * (size_t)c.batch * H * ((c.seq_len + 63) / 64 * 64) * 4);
+  p.delta = take(attention_bwd_scratch_bytes(c.batch, H, c.seq_len));
   p.emb = take(embedding_bwd_scratch_bytes((int)M, (int)d, (int)V));
   p.total = pos;
   return p;
