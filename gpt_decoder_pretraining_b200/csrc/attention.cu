@@ -1181,37 +1181,37 @@ __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t
                                   uint16_t* __restrict__ ext, float ext_scale, int B, int H, int T,
                                   int Tpad, int Dh, long long sb, long long sh, long long st,
                                   long long sbd, long long shd, long long std_) {
-  // one warp per padded row (b, h, t < Tpad): pad[0][bh][t] = lse·log2(e), pad[1][bh][t] =
-  // rowsum(dO∘O); rows t ≥ T are zero
-  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
+  // G = Dh/8 lanes per padded row (b, h, t < Tpad), 16-byte loads: pad[0][bh][t] = lse·log2(e),
+  // pad[1][bh][t] = rowsum(dO∘O); rows t ≥ T are zero
+  const int G = Dh >> 3;
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long r = gid / G;
+  const int part = (int)(gid % G);
   const long long rows = (long long)B * H * Tpad;
-  if (warp >= rows) return;
-  const int t = (int)(warp % Tpad);
-  const long long bh = warp / Tpad;
+  const bool in = r < rows;
+  const int t = in ? (int)(r % Tpad) : 0;
+  const long long bh = in ? r / Tpad : 0;
   const int h = (int)(bh % H), b = (int)(bh / H);
   float acc = 0.f;
-  if (t < T) {
-    const long long off = b * sb + h * sh + (long long)t * st;
-    const long long offd = b * sbd + h * shd + (long long)t * std_;
-    for (int j = 2 * lane; j < Dh; j += 64) {
-      const uint32_t x = *reinterpret_cast<const uint32_t*>(o + off + j);
-      const uint32_t y = *reinterpret_cast<const uint32_t*>(dout + offd + j);
-      acc += bf_lo(x) * bf_lo(y) + bf_hi(x) * bf_hi(y);
-    }
+  if (in && t < T) {
+    const uint4 x = *reinterpret_cast<const uint4*>(o + b * sb + h * sh + (long long)t * st + 8 * part);
+    const uint4 y = *reinterpret_cast<const uint4*>(dout + b * sbd + h * shd + (long long)t * std_ + 8 * part);
+    acc = bf_lo(x.x) * bf_lo(y.x) + bf_hi(x.x) * bf_hi(y.x) + bf_lo(x.y) * bf_lo(y.y) +
+          bf_hi(x.y) * bf_hi(y.y) + bf_lo(x.z) * bf_lo(y.z) + bf_hi(x.z) * bf_hi(y.z) +
+          bf_lo(x.w) * bf_lo(y.w) + bf_hi(x.w) * bf_hi(y.w);
   }
-#pragma unroll
-  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  if (lane == 0) {
+  // the G lanes of a row are consecutive and G divides 32
+  for (int s = G >> 1; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (in && part == 0) {
     const float l = (t < T) ? lse[bh * T + t] : 0.f;
-    pad[warp] = l * LOG2E;
-    pad[rows + warp] = acc;
+    pad[r] = l * LOG2E;
+    pad[rows + r] = acc;
     if (ext != nullptr) {
       // (Sᵀ + ext)·scale·log2 e = s·scale·log2 e − LSE·log2 e  and  dPᵀ + ext = dP − delta
       const uint2 el = (t < T) ? split3_bf16(-l * ext_scale) : make_uint2(0, 0);
       const uint2 ed = split3_bf16(-acc);
-      *reinterpret_cast<uint4*>(ext + warp * 8) = make_uint4(el.x, el.y, 0, 0);
-      *reinterpret_cast<uint4*>(ext + (rows + warp) * 8) = make_uint4(ed.x, ed.y, 0, 0);
+      *reinterpret_cast<uint4*>(ext + r * 8) = make_uint4(el.x, el.y, 0, 0);
+      *reinterpret_cast<uint4*>(ext + (rows + r) * 8) = make_uint4(ed.x, ed.y, 0, 0);
     }
   }
 }
@@ -1725,7 +1725,7 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   }
   {
     const int threads = 256;
-    const long long blocks = (rows * 32 + threads - 1) / threads;
+    const long long blocks = (rows * (Dh / 8) + threads - 1) / threads;
     attn_delta_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
         reinterpret_cast<const uint16_t*>(o), reinterpret_cast<const uint16_t*>(dout), lse, delta,
         ext, sqrtf((float)Dh), B, H, T, Tpad, Dh, sbo, sho, sto, sbd, shd, std_);

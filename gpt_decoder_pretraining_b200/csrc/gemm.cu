@@ -260,8 +260,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer (leader CTA) ----------------
-    if (leader && lane == 0) {
+    // ---------------- MMA issuer (leader CTA): the warp runs the loop, one elected lane issues ----------------
+    if (leader) {
       constexpr uint32_t idesc = idesc_bf16(2 * BM, BN, A_MN, B_MN);
       // stage-0 descriptors; stage s and slice kk are constant byte offsets from them
       const uint32_t s0 = smem_u32(smem);
@@ -275,26 +275,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       for (int u = pair; u < num_units; u += num_pairs) {
         int tm, tn, kt0, kt1;
         unit_coords(u, tm, tn, kt0, kt1);
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, args.status)) break;
+        if (!mbar_wait_warp(&tempty[acc], acc_phase ^ 1, abort_flag, args.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         bool ok = true;
         for (int kt = kt0; kt < kt1; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, args.status)) { ok = false; break; }
+          if (!mbar_wait_warp(&full[stage], phase, abort_flag, args.status)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ad = sdesc_add(a_desc0, stage * S::STAGE_BYTES);
           const uint64_t bd = sdesc_add(b_desc0, stage * S::STAGE_BYTES);
+          if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            mma_bf16_pair(d_tmem, sdesc_add(ad, A_MN ? kk * 2048 : kk * 32),
-                          sdesc_add(bd, B_MN ? kk * 2048 : kk * 32), idesc,
-                          (kt > kt0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              mma_bf16_pair(d_tmem, sdesc_add(ad, A_MN ? kk * 2048 : kk * 32),
+                            sdesc_add(bd, B_MN ? kk * 2048 : kk * 32), idesc,
+                            (kt > kt0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit_pair(&empty[stage], 0x3);
           }
-          tc_commit_pair(&empty[stage], 0x3);
+          __syncwarp();
           if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        tc_commit_pair(&tfull[acc], 0x3);
+        if (elect_one()) tc_commit_pair(&tfull[acc], 0x3);
+        __syncwarp();
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1;
       }
