@@ -310,6 +310,13 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// √x with the hardware approximation (x ≥ 0; relative error ~2^-22).
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float y;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // 2^x with the hardware approximation (relative error ~2^-22, subnormal results flushed to 0).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

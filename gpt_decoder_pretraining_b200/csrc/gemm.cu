@@ -30,7 +30,6 @@ namespace gpt {
 constexpr int BM = 128;   // rows per CTA (the pair covers 256)
 constexpr int BN = 256;   // columns per tile (each CTA stages 128 rows of B)
 constexpr int BK = 64;
-constexpr int GEMM_THREADS = 192;
 
 enum : int {
   EPI_CE_STATS = 100,
@@ -39,6 +38,14 @@ enum : int {
   EPI_BF16_HEADS = 103,   // bf16 store with row m = b·T + t, column n = h·Dh + j sent to [B, H, T, Dh]
   EPI_QKV_ROPE = 200      // + Dh: RoPE + QK-norm of the q and k heads, all three to [3][B][H][T][Dh]
 };
+
+// TMA warp, MMA warp, then 4 epilogue warps per column group (one per TMEM lane quarter).  Two
+// column groups halve the epilogue time of a tile; the QKV + RoPE epilogue keeps one group, since it
+// holds a whole head per thread and more threads would leave it too few registers.
+template <int EPI>
+constexpr int gemm_col_groups() { return EPI > EPI_QKV_ROPE ? 1 : 2; }
+template <int EPI>
+constexpr int gemm_threads() { return 64 + 128 * gemm_col_groups<EPI>(); }
 
 struct GemmArgs {
   int M, N, K;
@@ -119,7 +126,7 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, int m, int n0,
           for (int e = 0; e < 4; ++e) {
             const float lo = bf_lo(pw[e]), hi = bf_hi(pw[e]);
             if (EPI == GPT_EPI_RESID) { w[2 * e] += lo; w[2 * e + 1] += hi; }
-            else { w[2 * e] *= 2.f * lo; w[2 * e + 1] *= 2.f * hi; }
+            else { w[2 * e] *= 2.f * sqrt_approx(lo); w[2 * e + 1] *= 2.f * sqrt_approx(hi); }
           }
         }
         uint4 o;
@@ -133,35 +140,32 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, int m, int n0,
         if (n0 + j >= a.N) continue;
         float w = v[j];
         if (EPI == GPT_EPI_RESID) w += bf2f(x[j]);
-        if (EPI == GPT_EPI_DRELU2) w *= 2.f * bf2f(x[j]);
+        if (EPI == GPT_EPI_DRELU2) w *= 2.f * sqrt_approx(bf2f(x[j]));
         c[j] = f2bf(w);
       }
     }
     return;
   }
   if (EPI == GPT_EPI_RELU2) {
-    uint16_t* c2 = reinterpret_cast<uint16_t*>(a.C2) + (size_t)m * a.ldc + n0;
+    // only h = max(u,0)² is stored: the next GEMM's operand, and (as √h = max(u,0)) all the
+    // backward needs
     if (full) {
 #pragma unroll
       for (int j = 0; j < 32; j += 8) {
         float r[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) r[e] = fmaxf(v[j + e], 0.f);
-        uint4 o, o2;
-        o.x = pack_bf2(r[0], r[1]); o.y = pack_bf2(r[2], r[3]);
-        o.z = pack_bf2(r[4], r[5]); o.w = pack_bf2(r[6], r[7]);
-        o2.x = pack_bf2(r[0] * r[0], r[1] * r[1]); o2.y = pack_bf2(r[2] * r[2], r[3] * r[3]);
-        o2.z = pack_bf2(r[4] * r[4], r[5] * r[5]); o2.w = pack_bf2(r[6] * r[6], r[7] * r[7]);
+        uint4 o;
+        o.x = pack_bf2(r[0] * r[0], r[1] * r[1]); o.y = pack_bf2(r[2] * r[2], r[3] * r[3]);
+        o.z = pack_bf2(r[4] * r[4], r[5] * r[5]); o.w = pack_bf2(r[6] * r[6], r[7] * r[7]);
         *reinterpret_cast<uint4*>(c + j) = o;
-        *reinterpret_cast<uint4*>(c2 + j) = o2;
       }
     } else {
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         if (n0 + j >= a.N) continue;
         const float r = fmaxf(v[j], 0.f);
-        c[j] = f2bf(r);
-        c2[j] = f2bf(r * r);
+        c[j] = f2bf(r * r);
       }
     }
   }
@@ -171,7 +175,7 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, int m, int n0,
 // the kernel
 // ------------------------------------------------------------------------------------------------
 template <bool A_MN, bool B_MN, int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(), 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmArgs args) {
   using S = GemmShape;
@@ -195,7 +199,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 2 * 128);  // epilogue threads of both CTAs
+      mbar_init(&tempty[b], 2 * 128 * gemm_col_groups<EPI>());  // epilogue threads of both CTAs
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -304,8 +308,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       }
     }
   } else {
-    // ---------------- epilogue warps (both CTAs) ----------------
+    // ---------------- epilogue warps (both CTAs): lane quarter q, column half `half` ----------------
     const int q = warp & 3;
+    constexpr int G = gemm_col_groups<EPI>();
+    const int half = (warp - 2) >> 2;  // column group
     const int row_in_tile = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -333,7 +339,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         const long long bhtd = (long long)(args.M / args.T) * args.H * args.T * DH;
         const int b = m / args.T, t = m % args.T;
 #pragma unroll 1
-        for (int hh = 0; hh < BN / DH; ++hh) {
+        for (int hh = half * (BN / DH / G); hh < (half + 1) * (BN / DH / G); ++hh) {
           const int n_head = tn * BN + hh * DH;
           float xh[DH];
 #pragma unroll
@@ -380,7 +386,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         }
       } else {
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = half * (BN / 32 / G); c < (half + 1) * (BN / 32 / G); ++c) {
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + c * 32, r);
         tmem_ld_wait();
@@ -436,8 +442,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         }
       }
       }
-      if (EPI == EPI_CE_STATS && m < args.M) {
-        args.ce.stats[(size_t)m * args.ce.stats_ld + args.ce.stats_col0 + tn] =
+      if (EPI == EPI_CE_STATS && m < args.M && tn * BN + half * (BN / G) < args.N) {
+        args.ce.stats[(size_t)m * args.ce.stats_ld + args.ce.stats_col0 + G * tn + half] =
             make_float2(run_max, run_sum);
       }
       tc_fence_before();
@@ -477,7 +483,7 @@ static gpt_status launch_inst(const CUtensorMap& ma, const CUtensorMap& mb, cons
   GPT_TRY(device_info(&sms));
   const int units = a.tiles_m * a.tiles_n * a.splits;
   const int pairs = std::max(1, std::min(units, sms / 2));
-  kern<<<2 * pairs, GEMM_THREADS, S::SMEM_BYTES, stream>>>(ma, mb, a);
+  kern<<<2 * pairs, gemm_threads<EPI>(), S::SMEM_BYTES, stream>>>(ma, mb, a);
   count_launch();
   GPT_CUDA_TRY(cudaGetLastError());
   return GPT_OK;
@@ -543,7 +549,6 @@ gpt_status gemm_launch(int op, int epi, int M, int N, int K, const void* A, int 
                        cudaStream_t stream) {
   GPT_TRY(check_gemm_args(op, M, N, K, A, lda, B, ldb, C, ldc));
   if (epi < GPT_EPI_BF16 || epi > GPT_EPI_F32_ADD) return GPT_ERR_INVALID_ARG;
-  if (epi == GPT_EPI_RELU2 && !C2) return GPT_ERR_INVALID_ARG;
   if (epi == GPT_EPI_DRELU2 && (!aux || ldaux < N || (ldaux % 8))) return GPT_ERR_INVALID_ARG;
   const bool a_mn = (op == GPT_GEMM_TN);
   const bool b_mn = (op != GPT_GEMM_NT);
@@ -617,7 +622,7 @@ gpt_status gemm_qkv_rope_launch(int M, int d, const void* A, const void* Wqkv, v
   return launch_inst<false, false, EPI_QKV_ROPE + 32>(ma, mb, a, stream);
 }
 
-int gemm_ce_tile_n() { return BN; }
+int gemm_ce_tile_n() { return BN / gemm_col_groups<EPI_CE_STATS>(); }
 
 gpt_status gemm_ce_launch(bool grad, int M, int N, int K, const void* A, int lda, const void* B,
                           int ldb, void* C, int ldc, const CeArgs& ce, int* status,

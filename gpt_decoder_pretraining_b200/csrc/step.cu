@@ -100,7 +100,7 @@ struct Plan {
   size_t status, rope, pshadow;
   size_t x, xf, rhof;
   // per layer (base + l·stride)
-  size_t r1, rho1, qkv, rq, rk, lse, o, r2, rho2, act, hsq, layer_stride;
+  size_t r1, rho1, qkv, rq, rk, lse, o, r2, rho2, hsq, layer_stride;
   // CE
   size_t stats, zt, lse_ce, ell, inv_n, dz, dxf;
   // backward transients
@@ -171,15 +171,14 @@ static Plan make_plan(const gpt_config& c, size_t n_params) {
   p.o = take(M * d * 2) - layer0;
   p.r2 = take(M * d * 2) - layer0;
   p.rho2 = take(M * 4) - layer0;
-  p.act = take(M * F * 2) - layer0;
   p.hsq = take(M * F * 2) - layer0;
   p.layer_stride = pos - layer0;
   pos = layer0 + p.layer_stride * (size_t)c.depth;
   // make the per-layer offsets absolute for layer 0
   p.r1 += layer0; p.rho1 += layer0; p.qkv += layer0; p.rq += layer0; p.rk += layer0;
-  p.lse += layer0; p.o += layer0; p.r2 += layer0; p.rho2 += layer0; p.act += layer0; p.hsq += layer0;
+  p.lse += layer0; p.o += layer0; p.r2 += layer0; p.rho2 += layer0; p.hsq += layer0;
   // cross-entropy
-  const int tiles = (int)((V + 255) / 256);
+  const int tiles = (int)((V + gemm_ce_tile_n() - 1) / gemm_ce_tile_n());
   p.stats = take(M * tiles * sizeof(float2));
   p.zt = take(M * 4);
   p.lse_ce = take(M * 4);
@@ -281,7 +280,6 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
     uint16_t* o = reinterpret_cast<uint16_t*>(at(p.o, l));
     uint16_t* r2 = reinterpret_cast<uint16_t*>(at(p.r2, l));
     float* rho2 = reinterpret_cast<float*>(at(p.rho2, l));
-    uint16_t* act = reinterpret_cast<uint16_t*>(at(p.act, l));
     uint16_t* hsq = reinterpret_cast<uint16_t*>(at(p.hsq, l));
     PROF(PROF_NORM, 0, 4.0 * (double)M * d + 4.0 * M, rmsnorm_fwd(x, r1, rho1, M, d, s));
     // q̃, k̃, v head-major [3][B][H][T][Dh]; RoPE + QK-norm fused into the projection epilogue
@@ -293,7 +291,7 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
     PROF(PROF_GEMM, gemm_flops(M, d, d), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_RESID, M, d, d, o, d, W(wq + 1), d, x, d, nullptr,
                         nullptr, 0, status, s));
     PROF(PROF_NORM, 0, 4.0 * (double)M * d + 4.0 * M, rmsnorm_fwd(x, r2, rho2, M, d, s));
-    PROF(PROF_GEMM, gemm_flops(M, F, d), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_RELU2, M, F, d, r2, d, W(wq + 2), d, act, F, hsq,
+    PROF(PROF_GEMM, gemm_flops(M, F, d), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_RELU2, M, F, d, r2, d, W(wq + 2), d, hsq, F, nullptr,
                         nullptr, 0, status, s));
     PROF(PROF_GEMM, gemm_flops(M, d, F), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_RESID, M, d, F, hsq, F, W(wq + 3), F, x, d, nullptr,
                         nullptr, 0, status, s));
@@ -302,7 +300,7 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
 
   // ---------------- lm-head + cross-entropy ----------------
   const int wlm = 1 + 4 * c.depth;
-  const int tiles = (V + 255) / 256;
+  const int tiles = (V + gemm_ce_tile_n() - 1) / gemm_ce_tile_n();
   CeArgs ce{};
   ce.targets = targets;
   ce.lse = reinterpret_cast<float*>(ws + p.lse_ce);
@@ -349,11 +347,10 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
     uint16_t* o = reinterpret_cast<uint16_t*>(at(p.o, l));
     uint16_t* r2 = reinterpret_cast<uint16_t*>(at(p.r2, l));
     float* rho2 = reinterpret_cast<float*>(at(p.rho2, l));
-    uint16_t* act = reinterpret_cast<uint16_t*>(at(p.act, l));
     uint16_t* hsq = reinterpret_cast<uint16_t*>(at(p.hsq, l));
     // MLP
     PROF(PROF_GEMM, gemm_flops(M, F, d), 0, gemm_launch(GPT_GEMM_NN, GPT_EPI_DRELU2, M, F, d, gxb, d, W(wq + 3), F, du, F, nullptr,
-                        act, F, status, s));
+                        hsq, F, status, s));
     PROF(PROF_GEMM, gemm_flops(d, F, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, d, F, M, gxb, d, hsq, F, G(wq + 3), F, nullptr,
                         nullptr, 0, status, s));
     PROF(PROF_GEMM, gemm_flops(F, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, F, d, M, du, F, r2, d, G(wq + 2), d, nullptr,
@@ -503,7 +500,7 @@ gpt_status gpt_step_status(const gpt_step* step, const void* workspace, void* st
 
 size_t gpt_lmhead_ce_scratch_bytes(int M, int d, int V) {
   (void)d;
-  const size_t tiles = (size_t)(V + 255) / 256;
+  const size_t tiles = (size_t)(V + gpt::gemm_ce_tile_n() - 1) / gpt::gemm_ce_tile_n();
   return gpt::al256((size_t)M * tiles * 8) + 4 * gpt::al256((size_t)M * 4) + 256 +
          gpt::al256((size_t)M * V * 2);
 }
@@ -516,7 +513,7 @@ gpt_status gpt_lmhead_ce_fwd_bwd(const void* xf, const void* wlm, const int32_t*
   if ((d % 64) || (V % 64)) return GPT_ERR_UNSUPPORTED_SHAPE;
   cudaStream_t s = gpt::as_stream(stream);
   uint8_t* p = reinterpret_cast<uint8_t*>(scratch);
-  const int tiles = (V + 255) / 256;
+  const int tiles = (V + gpt::gemm_ce_tile_n() - 1) / gpt::gemm_ce_tile_n();
   gpt::CeArgs ce{};
   ce.targets = targets;
   ce.stats = reinterpret_cast<float2*>(p);

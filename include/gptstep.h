@@ -128,8 +128,9 @@ gpt_status gpt_step_profile(gpt_step* step, double* ms, int64_t* calls, double* 
  * epilogue (what is written for each accumulator value acc at (m, n)):
  *   GPT_EPI_BF16    C = bf16(acc)
  *   GPT_EPI_RESID   C = bf16(C + acc)                 (C bf16, residual add in place)
- *   GPT_EPI_RELU2   C = bf16(max(acc,0)), C2 = bf16(max(acc,0)²)   (C2 uses ldc)
- *   GPT_EPI_DRELU2  C = bf16(acc · 2 · aux)           (aux bf16 = max(u,0) saved by RELU2)
+ *   GPT_EPI_RELU2   C = bf16(max(acc,0)²)             (C2 unused)
+ *   GPT_EPI_DRELU2  C = bf16(acc · 2 · √aux)          (aux bf16 = max(u,0)² saved by RELU2, so
+ *                                                       √aux = max(u,0): the ReLU² derivative)
  *   GPT_EPI_F32     C = acc                           (C fp32)
  *   GPT_EPI_F32_ADD C = C + acc                       (C fp32)
  * Sizes: M, N ≥ 1; K ≥ 1 (tails are zero-filled).  Pointers 16-byte aligned. */

@@ -66,14 +66,14 @@ def test_gemm_epilogues(M, N, K):
     X = randn(rng, M, N, scale=3.0)
     tX = bf16_tensor(X)
     S.gemm(0, S.EPI_RESID, tA, tB, tX, M, N, K)
-    # ReLU² (relu and its square)
-    Ca = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+    # ReLU²: h = max(acc, 0)²
     Ch = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
-    S.gemm(0, S.EPI_RELU2, tA, tB, Ca, M, N, K, C2=Ch)
-    # dReLU²: acc·2·aux
-    aux = np.maximum(randn(rng, M, N), 0)
+    S.gemm(0, S.EPI_RELU2, tA, tB, Ch, M, N, K)
+    # dReLU² from the saved h: acc·2·√h
+    taux = bf16_tensor(np.maximum(randn(rng, M, N), 0) ** 2)
+    aux = to_np(taux).astype(np.float64)
     Cd = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
-    S.gemm(0, S.EPI_DRELU2, tA, tB, Cd, M, N, K, aux=bf16_tensor(aux))
+    S.gemm(0, S.EPI_DRELU2, tA, tB, Cd, M, N, K, aux=taux)
     # fp32 accumulate
     base = rng.standard_normal((M, N)).astype(np.float32)
     Cf = torch.from_numpy(base).cuda()
@@ -81,9 +81,8 @@ def test_gemm_epilogues(M, N, K):
     torch.cuda.synchronize()
     assert_close_rel(to_np(tX), X + acc, rel=8e-3, what="resid")
     r = np.maximum(acc, 0)
-    assert_close_rel(to_np(Ca), r, rel=8e-3, what="relu")
     assert_close_rel(to_np(Ch), r * r, rel=8e-3, what="relu2")
-    assert_close_rel(to_np(Cd), acc * 2 * aux, rel=8e-3, what="drelu2")
+    assert_close_rel(to_np(Cd), acc * 2 * np.sqrt(aux), rel=8e-3, what="drelu2")
     assert_close_rel(to_np(Cf), base + acc, rel=1e-5, cos=0.9999999, what="f32 add")
 
 
