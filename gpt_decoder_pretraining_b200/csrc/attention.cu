@@ -292,6 +292,11 @@ __global__ void __launch_bounds__(256)
 // is the exact softmax; p ∈ [e^{−2c_t}, 1] cannot overflow and, for c_t ≤ 40, cannot underflow.
 // With a fixed shift O never needs rescaling inside tensor memory.
 // ================================================================================================
+// bar.sync on a named barrier (ids 1..15) for `count` threads.
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 template <int DH>
 struct TcFwdShape {
   static constexpr int BQ = 128, BK = 128;
@@ -301,8 +306,12 @@ struct TcFwdShape {
   static constexpr int OFF_K = 2 * Q_TILE;
   static constexpr int OFF_V = OFF_K + 2 * KV_TILE;
   static constexpr int OFF_BAR = OFF_V + 2 * KV_TILE;
-  static constexpr int SMEM = OFF_BAR + 256 + 1024;
-  static constexpr int THREADS = 320;
+  static constexpr int OFF_RED = OFF_BAR + 256;  // [x][half][row] (l, lb) partial row sums
+  static constexpr int SMEM = OFF_RED + 2 * 2 * 128 * 8 + 1024;
+  // 16 softmax warps (query tile x = warp / 8, key half = warp / 4 % 2, lane quarter = warp % 4),
+  // then the TMA warp and the MMA warp
+  static constexpr int THREADS = 576;
+  static constexpr int TMA_WARP = 16, MMA_WARP = 17;
   static constexpr int TM_S = 0;    // S_x at x·128
   static constexpr int TM_O = 256;  // O_x at 256 + x·DH
 };
@@ -325,7 +334,7 @@ __device__ __forceinline__ float q_row_sumsq(const uint8_t* tile, int r) {
 }
 
 template <int DH>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(576, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                        const __grid_constant__ CUtensorMap mv, const AttnArgs a, const float* kmax,
                        float kmax_const) {
@@ -358,13 +367,13 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], 256);
     }
     mbar_init(o_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == S::MMA_WARP) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -373,7 +382,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == S::TMA_WARP) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       mbar_arrive_expect_tx(bar_q, 2 * S::Q_TILE);
@@ -388,7 +397,7 @@ __global__ void __launch_bounds__(320, 1)
         load_tile<DH, 128>(smem + S::OFF_V + st * S::KV_TILE, &mv, &kv_full[st], k0, h, b);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == S::MMA_WARP) {
     // ---------------- MMA issuer: the warp runs the loop, one elected lane issues ----------------
     {
       constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
@@ -415,8 +424,8 @@ __global__ void __launch_bounds__(320, 1)
         const uint64_t v_desc = sdesc_add(vd, (j & 1) * S::KV_TILE);
         if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ts(tmem + S::TM_O + x * DH, tmem + S::TM_S + x * 128 + kk * 8,
+          for (int kk = 0; kk < 8; ++kk)  // key half kk/4 packed in S columns 64·(kk/4) + 8·(kk%4)
+            mma_bf16_ts(tmem + S::TM_O + x * DH, tmem + S::TM_S + x * 128 + 64 * (kk >> 2) + 8 * (kk & 3),
                         sdesc_add(v_desc, kk * 2048), id_o, (j > 0 || kk > 0) ? 1u : 0u);
           if (release_kv) tc_commit(&kv_empty[j & 1]);
         }
@@ -450,47 +459,48 @@ __global__ void __launch_bounds__(320, 1)
       __syncwarp();
     }
   } else {
-    // ---------------- softmax warpgroups ----------------
-    const int x = warp >> 2;
+    // ---------------- softmax warps: thread = one query row × one half (64 keys) of each KV tile
+    const int x = warp >> 3;
+    const int half = (warp >> 2) & 1;
     const int quarter = warp & 3;
     const int row = 32 * quarter + lane;
     const int t = q0 + 128 * x + row;
     const int tile0 = q0 + 128 * x;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
-    const uint32_t s_addr = tmem + lane_off + S::TM_S + x * 128;
+    const uint32_t s_addr = tmem + lane_off + S::TM_S + x * 128 + 64 * half;
     bool ok = mbar_wait(bar_q, 0, abort_flag, a.status);
     // fixed shift c_t (log2 units)
     const float qn = sqrtf(q_row_sumsq<DH>(smem + S::OFF_Q + x * S::Q_TILE, row));
     const float km = kmax ? kmax[(long long)b * a.H + h] : kmax_const;
     const float c_nat = qn * km * a.scale * 1.001f + 1e-3f;
-    if (c_nat > 40.f && t < T) set_status(a.status, GPT_ERR_NUMERIC_RANGE);
+    if (c_nat > 40.f && t < T && half == 0) set_status(a.status, GPT_ERR_NUMERIC_RANGE);
     const float c2 = c_nat * LOG2E;
     // l: exact sum of the weights (gives the LSE the backward pass needs); lb: sum of the bf16
     // weights that P·V actually uses, so that O = Σ P·v / lb is a convex combination of the v rows
-    // (exact for a single visible key).  Both as packed pairs of partial sums.
+    // (exact for a single visible key).  Both as packed pairs of partial sums over this half.
     float l0 = 0.f, l1 = 0.f, lb0 = 0.f, lb1 = 0.f;
     for (int j = 0; j < n_kv && ok; ++j) {
       if (!mbar_wait(&s_full[x], j & 1, abort_flag, a.status)) { ok = false; break; }
       tc_fence_after();
-      const int kv0 = (kv_first + j) * 128;
-      const bool need_mask = (kv0 + 127 > tile0) || (kv0 <= tile0 + 127 - W);
-      // chunk c+1 is loaded from tensor memory while chunk c is exponentiated
-      uint32_t rbuf[2][32];
-      tmem_ld32(s_addr, rbuf[0]);
+      const int kv0 = (kv_first + j) * 128 + 64 * half;  // first key of this thread's half
+      const bool need_mask = (kv0 + 63 > tile0) || (kv0 <= tile0 + 127 - W);
+      // chunk c+1 (16 keys) is loaded from tensor memory while chunk c is exponentiated
+      uint32_t rbuf[2][16];
+      tmem_ld16(s_addr, rbuf[0]);
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t (&r)[32] = rbuf[c & 1];
-        if (c < 3) tmem_ld32(s_addr + 32 * (c + 1), rbuf[(c + 1) & 1]);
-        uint32_t pk[16];
+        uint32_t (&r)[16] = rbuf[c & 1];
+        if (c < 3) tmem_ld16(s_addr + 16 * (c + 1), rbuf[(c + 1) & 1]);
+        uint32_t pk[8];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
+        for (int e = 0; e < 8; ++e) {
           float x0, x1;
           fma2_bc(x0, x1, __uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]), a.scale_log2, -c2);
           float p0 = ex2_approx(x0);
           float p1 = ex2_approx(x1);
           if (need_mask) {
-            const int key = kv0 + 32 * c + 2 * e;
+            const int key = kv0 + 16 * c + 2 * e;
             if (!(key <= t && key > t - W)) p0 = 0.f;
             if (!(key + 1 <= t && key + 1 > t - W)) p1 = 0.f;
           }
@@ -498,23 +508,28 @@ __global__ void __launch_bounds__(320, 1)
           pk[e] = pack_bf2(p0, p1);
           add2_acc(lb0, lb1, bf_lo(pk[e]), bf_hi(pk[e]));
         }
-        // P of chunk c overwrites S columns 16c..16c+15, all of which have been read already
-        tmem_st16(s_addr + 16 * c, pk);
+        // P of chunk c overwrites this half's S columns 8c..8c+7, all of which have been read
+        tmem_st8(s_addr + 8 * c, pk);
         if (c < 3) tmem_ld_wait();
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[x]);
     }
-    // epilogue: O / l
+    // the row's two halves combine their sums (both halves of group x reach this barrier)
+    float2* red = reinterpret_cast<float2*>(smem + S::OFF_RED);
+    red[(x * 2 + half) * 128 + row] = make_float2(l0 + l1, lb0 + lb1);
+    named_barrier_sync(1 + x, 256);
+    const float2 s0 = red[(x * 2 + 0) * 128 + row], s1 = red[(x * 2 + 1) * 128 + row];
+    const float l = s0.x + s1.x;
+    const float inv = 1.f / (s0.y + s1.y);
+    // epilogue: O / lb, this half's DH/2 columns
     if (ok) ok = mbar_wait(o_full, 0, abort_flag, a.status);
     if (ok) {
       tc_fence_after();
-      const float l = l0 + l1;
-      const float inv = 1.f / (lb0 + lb1);
       uint16_t* orow = a.o + b * a.sb_o + h * a.sh_o + (long long)t * a.st_o;
 #pragma unroll 1
-      for (int c = 0; c < DH / 32; ++c) {
+      for (int c = half * (DH / 64); c < (half + 1) * (DH / 64); ++c) {
         uint32_t r[32];
         tmem_ld32(tmem + lane_off + S::TM_O + x * DH + 32 * c, r);
         tmem_ld_wait();
@@ -530,7 +545,7 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
       }
-      if (t < T) a.lse[((long long)b * a.H + h) * T + t] = (c2 + log2f(l)) * LN2;
+      if (t < T && half == 0) a.lse[((long long)b * a.H + h) * T + t] = (c2 + log2f(l)) * LN2;
     }
   }
 
@@ -541,7 +556,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 9) tmem_dealloc(tmem, 512);
+  if (warp == S::MMA_WARP) tmem_dealloc(tmem, 512);
 }
 
 // ================================================================================================
