@@ -41,6 +41,7 @@ struct AttnArgs {
   float* delta;  // backward: [2][B·H][Tpad] fp32 — LSE·log2(e), then rowsum(dO∘O); zero-padded
   int Tpad;      // T rounded up to a multiple of 64
   uint16_t* ext; // backward: [2][B·H][Tpad][8] bf16 rows [hi, mid, lo, 0…] of −LSE·√Dh, −delta
+  uint16_t* ds_t; // backward (optional): dSᵀ [B·H][T][Tpad] bf16, written by the dK/dV kernel
   int* status;
   // optional QK-norm + RoPE backward fused into the dq / dk epilogues (rho_q == nullptr: off):
   // q̃ = RMS_Dh(RoPE(q)), so dq = Rᵀ·rho·(dq̃ − q̃·mean(q̃·dq̃)), likewise for k
@@ -720,7 +721,10 @@ __global__ void __launch_bounds__(320, 1)
   const int T = a.T, W = a.window;
   const int kv0 = blockIdx.x * 128;
   const int q_first = kv0 / 64;
-  const int q_last = min(T - 1, kv0 + 127 + W - 1) / 64;
+  // with dSᵀ stored, cover every 128-query tile that reads one of these keys (tiles beyond the
+  // window are fully masked and store zeros)
+  const int q_reach = a.ds_t ? ((kv0 + 126 + W) / 128) * 128 + 127 : kv0 + 127 + W - 1;
+  const int q_last = min(T - 1, q_reach) / 64;
   const int n_q = q_last - q_first + 1;
   const long long bh = (long long)b * a.H + h;
 
@@ -877,6 +881,11 @@ __global__ void __launch_bounds__(320, 1)
         mul2(s0, s1, p0, p1, __uint_as_float(rp[j]), __uint_as_float(rp[j + 1]));
         pk[e] = pack_bf2(p0, p1);
         dk[e] = pack_bf2(s0, s1);
+      }
+      if (a.ds_t != nullptr && key < T) {
+        uint4* dst = reinterpret_cast<uint4*>(a.ds_t + ((size_t)bh * T + key) * a.Tpad + qc);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) dst[u] = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
       }
       // packed halves stay inside the columns this warp just read (see mma_acc_from_tmem)
       tmem_st16(tmem + lane_off + S::TM_S + bf * 64 + 32 * half, pk);
@@ -1148,6 +1157,158 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+// ================================================================================================
+// backward (3'): dQ from the dSᵀ tiles the dK/dV kernel stored — one CTA per 128-query tile, loop
+// over its 64-key tiles: dQ += dS·Kⱼ with A = dS read MN-major from the [64 keys][128 queries] dSᵀ
+// tile and B = Kⱼ (MN-major).  No scores are recomputed; the epilogue is the dQ kernel's.
+// ================================================================================================
+template <int DH>
+struct DqDsShape {
+  static constexpr int STAGES = 4;
+  static constexpr int Q_TILE = 128 * DH * 2;   // q̃ tile (the QK-norm + RoPE backward reads it)
+  static constexpr int DS_TILE = 64 * 128 * 2;  // [2 query chunks][64 keys][64 queries]
+  static constexpr int K_TILE = 64 * DH * 2;
+  static constexpr int STAGE_BYTES = DS_TILE + K_TILE;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_STAGE = Q_TILE;
+  static constexpr int OFF_BAR = OFF_STAGE + STAGES * STAGE_BYTES;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int THREADS = 192;  // 4 epilogue warps, TMA warp, MMA warp
+  static constexpr int TMEM_COLS = DH < 32 ? 32 : DH;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                          const __grid_constant__ CUtensorMap mds, const AttnArgs a) {
+  using S = DqDsShape<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
+  uint64_t* q_bar = bars;
+  uint64_t* full = bars + 1;               // [STAGES]
+  uint64_t* empty = full + S::STAGES;      // [STAGES]
+  uint64_t* done = empty + S::STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int qt = gridDim.x - 1 - blockIdx.x;  // longest rows first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int T = a.T, W = a.window;
+  const int q0 = qt * 128;
+  const int key_lo = max(0, q0 - W + 1);
+  const int key_hi = min(T, q0 + 128);
+  const int kv_first = key_lo / 64;
+  const int n_kv = (key_hi - 1) / 64 - kv_first + 1;
+  const int bh = b * a.H + h;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_bar, 1);
+    for (int i = 0; i < S::STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, S::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_bar, S::Q_TILE);
+      load_tile<DH, 128>(smem + S::OFF_Q, &mq, q_bar, q0, h, b);
+      for (int j = 0; j < n_kv; ++j) {
+        const int st = j % S::STAGES;
+        if (!mbar_wait(&empty[st], ((j / S::STAGES) & 1) ^ 1, abort_flag, a.status)) break;
+        mbar_arrive_expect_tx(&full[st], S::STAGE_BYTES);
+        uint8_t* dst = smem + S::OFF_STAGE + st * S::STAGE_BYTES;
+        const int k0 = (kv_first + j) * 64;
+        tma_load_3d(dst, &mds, &full[st], q0, k0, bh);                  // queries q0 .. q0+63
+        tma_load_3d(dst + S::DS_TILE / 2, &mds, &full[st], q0 + 64, k0, bh);  // q0+64 .. q0+127
+        load_tile<DH, 64>(dst + S::DS_TILE, &mk, &full[st], k0, h, b);
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------- MMA issuer: the warp runs the loop, one elected lane issues ----------------
+    constexpr uint32_t id_acc = idesc_bf16(128, DH, true, true);
+    const uint32_t stage0 = smem_u32(smem + S::OFF_STAGE);
+    const uint64_t ds_d = sdesc_sw128(stage0, S::DS_TILE / 2, 1024);       // dS, MN-major (queries)
+    const uint64_t k_d = sdesc_sw128(stage0 + S::DS_TILE, 64 * 128, 1024);  // K, MN-major (Dh)
+    bool ok = true;
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int st = j % S::STAGES;
+      if (!mbar_wait_warp(&full[st], (j / S::STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t so = st * S::STAGE_BYTES;
+      const uint64_t a_st = sdesc_add(ds_d, so), b_st = sdesc_add(k_d, so);
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ss(tmem, sdesc_add(a_st, kk * 2048), sdesc_add(b_st, kk * 2048), id_acc,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&empty[st]);
+      }
+      __syncwarp();
+    }
+    if (elect_one()) tc_commit(done);
+    __syncwarp();
+  } else {
+    // ---------------- epilogue warps: thread = query row ----------------
+    const int row = 32 * warp + lane;
+    const int t = q0 + row;
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    bool ok = mbar_wait(q_bar, 0, abort_flag, a.status);
+    if (ok) ok = mbar_wait(done, 0, abort_flag, a.status);
+    if (ok) {
+      tc_fence_after();
+      uint16_t* dst = a.o + b * a.sb_o + h * a.sh_o + (long long)t * a.st_o;
+      if (a.rho_q != nullptr) {
+        const bool valid = t < T;
+        const float rho = valid ? a.rho_q[((long long)b * T + t) * a.H + h] : 0.f;
+        qknorm_rope_bwd_tmem<DH, 128>(tmem + lane_off, a.scale, smem + S::OFF_Q, row, rho,
+                                      a.cos_sin + (size_t)(valid ? t : 0) * DH, dst, valid);
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < DH / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_off + 32 * c, r);
+          tmem_ld_wait();
+          if (t < T) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              uint4 w;
+              w.x = pack_bf2(__uint_as_float(r[8 * u + 0]) * a.scale, __uint_as_float(r[8 * u + 1]) * a.scale);
+              w.y = pack_bf2(__uint_as_float(r[8 * u + 2]) * a.scale, __uint_as_float(r[8 * u + 3]) * a.scale);
+              w.z = pack_bf2(__uint_as_float(r[8 * u + 4]) * a.scale, __uint_as_float(r[8 * u + 5]) * a.scale);
+              w.w = pack_bf2(__uint_as_float(r[8 * u + 6]) * a.scale, __uint_as_float(r[8 * u + 7]) * a.scale);
+              *reinterpret_cast<uint4*>(dst + 32 * c + 8 * u) = w;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  if (*abort_flag && threadIdx.x == 0) {
+    for (int i = 0; i < 2000; ++i) __nanosleep(1000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem, S::TMEM_COLS);
 }
 
 // max_t ‖k_t‖ for each (batch, head): one CTA per (h, b).
@@ -1623,12 +1784,15 @@ gpt_status launch_bwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, c
 // [2·B·H·Tpad][8] bf16 extension rows in 64-row boxes.
 template <int DH>
 gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[4],
-                         const CUtensorMap& mext, AttnArgs a, void* dq, cudaStream_t stream) {
+                         const CUtensorMap& mext, const CUtensorMap* mds, AttnArgs a, void* dq,
+                         cudaStream_t stream) {
   using S = TcBwdShape<DH>;
+  using SD = DqDsShape<DH>;
   static bool once = false;
   if (!once) {
     GPT_TRY(set_smem(attn_bwd_dkdv_tc_kernel<DH>, S::SMEM));
     GPT_TRY(set_smem(attn_bwd_dq_tc_kernel<DH>, S::SMEM));
+    GPT_TRY(set_smem(attn_bwd_dq_ds_kernel<DH>, SD::SMEM));
     once = true;
   }
   // dK/dV: outer 128-key tiles (K, V with 128-row boxes), inner 64-query tiles (Q, dO 64-row boxes)
@@ -1637,10 +1801,15 @@ gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[
                                                                    mext, a);
   count_launch();
   GPT_CUDA_TRY(cudaGetLastError());
-  // dQ: outer 128-query tiles (Q, dO 128-row boxes), inner 64-key tiles (K, V 64-row boxes)
   a.o = reinterpret_cast<uint16_t*>(dq);
   dim3 g2((a.T + 127) / 128, a.H, a.B);
-  attn_bwd_dq_tc_kernel<DH><<<g2, S::THREADS, S::SMEM, stream>>>(m128[0], m64[1], m64[2], m128[3], a);
+  if (mds != nullptr) {
+    // dQ = dS·K from the stored dSᵀ tiles: outer 128-query tiles, inner 64-key tiles
+    attn_bwd_dq_ds_kernel<DH><<<g2, SD::THREADS, SD::SMEM, stream>>>(m128[0], m64[1], *mds, a);
+  } else {
+    // dQ with S and dP recomputed: outer 128-query tiles (Q, dO 128-row boxes), inner 64-key tiles
+    attn_bwd_dq_tc_kernel<DH><<<g2, S::THREADS, S::SMEM, stream>>>(m128[0], m64[1], m64[2], m128[3], a);
+  }
   count_launch();
   GPT_CUDA_TRY(cudaGetLastError());
   return GPT_OK;
@@ -1695,9 +1864,10 @@ gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, f
 
 // Backward scratch per padded row (b, h, t < ⌈T/64⌉·64): LSE·log2 e and delta (fp32), and the two
 // 16-byte extension rows of the dK/dV kernel.
-size_t attention_bwd_scratch_bytes(int B, int H, int T) {
+size_t attention_bwd_scratch_bytes(int B, int H, int T, bool store_ds) {
   if (B <= 0 || H <= 0 || T <= 0) return 0;
-  return (size_t)B * H * ((T + 63) / 64 * 64) * (2 * sizeof(float) + 2 * 16);
+  const size_t rows = (size_t)B * H * ((T + 63) / 64 * 64);
+  return rows * (2 * sizeof(float) + 2 * 16) + (store_ds ? rows * (size_t)T * 2 : 0);
 }
 
 // Strides: (sbq, shq, stq) for q, k, v; (sbg, shg, stg) for dq, dk, dv; (sbo, sho, sto) for o;
@@ -1708,7 +1878,7 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
                          long long shq, long long stq, long long sbg, long long shg, long long stg,
                          long long sbo, long long sho, long long sto, long long sbd, long long shd,
                          long long std_, int* status, cudaStream_t stream, const float* rho_q,
-                         const float* rho_k, const float* cos_sin) {
+                         const float* rho_k, const float* cos_sin, bool store_ds) {
   GPT_TRY(check_attn(q, B, H, T, Dh, sbq, shq, stq));
   GPT_TRY(check_attn(k, B, H, T, Dh, sbq, shq, stq));
   GPT_TRY(check_attn(v, B, H, T, Dh, sbq, shq, stq));
@@ -1729,6 +1899,15 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   // [2][B·H][Tpad][8] bf16, fetched with TMA in 64-row boxes
   const long long rows = (long long)B * H * Tpad;
   uint16_t* ext = (Dh != 32) ? reinterpret_cast<uint16_t*>(delta + 2 * rows) : nullptr;
+  // dSᵀ [B·H][T][Tpad] bf16 after the extension rows, when the scratch holds it
+  uint16_t* ds_t = (Dh != 32 && store_ds) ? ext + 2 * rows * 8 : nullptr;
+  CUtensorMap mds;
+  if (ds_t != nullptr) {
+    const uint64_t dims[3] = {(uint64_t)Tpad, (uint64_t)T, (uint64_t)B * H};
+    const uint64_t strides[2] = {(uint64_t)Tpad * 2, (uint64_t)T * Tpad * 2};
+    const uint32_t box[3] = {64, 64, 1};
+    if (!encode_map_bf16(&mds, ds_t, 3, dims, strides, box, true)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  }
   CUtensorMap mext;
   if (Dh != 32) {
     const uint64_t dims[2] = {8, (uint64_t)(2 * rows)};
@@ -1756,6 +1935,7 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   a.delta = delta;
   a.Tpad = Tpad;
   a.ext = ext;
+  a.ds_t = ds_t;
   a.status = status;
   a.sb_o = sbg; a.sh_o = shg; a.st_o = stg;  // strides of the dq/dk/dv outputs
   a.rho_q = rho_q;
@@ -1776,8 +1956,8 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
                        is_do ? std_ : stq, 64))
       return GPT_ERR_UNSUPPORTED_SHAPE;
   }
-  if (Dh == 128) GPT_TRY(launch_bwd_tc<128>(m128, m64, mext, a, dq, stream));
-  else GPT_TRY(launch_bwd_tc<64>(m128, m64, mext, a, dq, stream));
+  if (Dh == 128) GPT_TRY(launch_bwd_tc<128>(m128, m64, mext, ds_t ? &mds : nullptr, a, dq, stream));
+  else GPT_TRY(launch_bwd_tc<64>(m128, m64, mext, ds_t ? &mds : nullptr, a, dq, stream));
   return GPT_OK;
 }
 
@@ -1813,13 +1993,15 @@ gpt_status attention_bwd_noalloc(const void* q, const void* k, const void* v, co
                                  long long shq, long long stq, long long sbo, long long sho,
                                  long long sto, int* status, cudaStream_t stream) {
   if (B <= 0 || H <= 0 || T <= 0) return GPT_ERR_INVALID_ARG;
-  if ((long long)attention_bwd_scratch_bytes(B, H, T) > NOALLOC_DELTA_ROWS * 4)
+  // the fixed array holds the per-row scratch only: dQ recomputes the scores instead of reading
+  // a stored dSᵀ
+  if ((long long)attention_bwd_scratch_bytes(B, H, T, false) > NOALLOC_DELTA_ROWS * 4)
     return GPT_ERR_UNSUPPORTED_SHAPE;
   float* delta = nullptr;
   GPT_TRY(noalloc_delta_ptr(&delta));
   return attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, T, Dh, window, sbq, shq, stq,
                        sbq, shq, stq, sbo, sho, sto, sbo, sho, sto, status, stream, nullptr,
-                       nullptr, nullptr);
+                       nullptr, nullptr, false);
 }
 
 }  // namespace gpt
@@ -1841,11 +2023,11 @@ extern "C" gpt_status gpt_attention_bwd(const void* q, const void* k, const void
                                         long long st_o, int* status, void* stream) {
   return gpt::attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, T, Dh, window, sb_qkv,
                             sh_qkv, st_qkv, sb_qkv, sh_qkv, st_qkv, sb_o, sh_o, st_o, sb_o, sh_o,
-                            st_o, status, gpt::as_stream(stream), nullptr, nullptr, nullptr);
+                            st_o, status, gpt::as_stream(stream), nullptr, nullptr, nullptr, true);
 }
 
 extern "C" size_t gpt_attention_bwd_scratch_bytes(int B, int H, int T) {
-  return gpt::attention_bwd_scratch_bytes(B, H, T);
+  return gpt::attention_bwd_scratch_bytes(B, H, T, true);
 }
 
 extern "C" gpt_status gpt_attention_bwd_noalloc(const void* q, const void* k, const void* v,

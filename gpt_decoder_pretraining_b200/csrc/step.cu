@@ -32,7 +32,7 @@ gpt_status rope_qknorm_bwd_heads(void* dqkv, const void* y_heads, const float* r
 gpt_status embedding_fwd(const int32_t* tok, const void* wte, void* x, int M, int d, int V,
                          int* status, cudaStream_t s);
 size_t embedding_bwd_scratch_bytes(int M, int d, int V);
-size_t attention_bwd_scratch_bytes(int B, int H, int T);
+size_t attention_bwd_scratch_bytes(int B, int H, int T, bool store_ds);
 gpt_status embedding_bwd(const int32_t* tok, const float* gx, float* dwte, int M, int d, int V,
                          void* scratch, cudaStream_t s);
 gpt_status ce_rows(const float2* stats, int ntiles, const float* zt, const int32_t* targets, int M,
@@ -50,7 +50,7 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
                          long long shq, long long stq, long long sbg, long long shg, long long stg,
                          long long sbo, long long sho, long long sto, long long sbd, long long shd,
                          long long std_, int* status, cudaStream_t stream, const float* rho_q,
-                         const float* rho_k, const float* cos_sin);
+                         const float* rho_k, const float* cos_sin, bool store_ds);
 
 static inline size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
 
@@ -196,7 +196,7 @@ static Plan make_plan(const gpt_config& c, size_t n_params) {
   p.dr = take(M * d * 2);
   p.dO = take(M * d * 2);
   p.dqkv = take(M * 3 * d * 2);
-  p.delta = take(attention_bwd_scratch_bytes(c.batch, H, c.seq_len));
+  p.delta = take(attention_bwd_scratch_bytes(c.batch, H, c.seq_len, true));
   p.emb = take(embedding_bwd_scratch_bytes((int)M, (int)d, (int)V));
   p.total = pos;
   return p;
@@ -367,7 +367,7 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
          attention_bwd(qkv, qkv + bhtd, qkv + 2 * bhtd, o, dO, lse, delta, dqkv, dqkv + d,
                        dqkv + 2 * d, B, H, T, Dh, st->window[l], hs_b, hs_h, hs_t, qs_b, qs_h,
                        qs_t, os_b, os_h, os_t, hs_b, hs_h, hs_t, status, s,
-                       Dh == 32 ? nullptr : rq, rk, rope));
+                       Dh == 32 ? nullptr : rq, rk, rope, true));
     if (Dh == 32) {  // the mma.sync path for head_dim 32 has no fused QK-norm/RoPE backward
       PROF(PROF_ROPE, 0, 12.0 * (double)M * d,
            rope_qknorm_bwd_heads(dqkv, qkv, rq, rk, rope, B, T, H, Dh, s));
