@@ -181,7 +181,9 @@ gpt_status gpt_rope_table(float* cos_sin, int T, int Dh, void* stream);
  * gpt_attention_bwd_scratch_bytes(B, H, T) bytes, 16-byte aligned; per row (zero-padded to a
  * multiple of 64 rows per (b, h)) the backward stores LSE·log2(e) and rowsum(dO∘O) in fp32 and,
  * for Dh ≥ 64, both again as bf16 hi/mid/lo triples that its dK/dV kernel adds into the score
- * accumulators with one extra K = 16 tensor-core step.
+ * accumulators with one extra K = 16 tensor-core step; after these rows, for Dh ≥ 64, the dK/dV
+ * kernel stores dSᵀ (bf16 [B·H][T][⌈T/64⌉·64], causal band / window only) and the dQ kernel
+ * contracts it with K.
  * The forward shifts each row's exponentials by the Cauchy–Schwarz bound c_t = ‖q_t‖·max_j‖k_j‖/√Dh
  * instead of a running maximum (softmax is invariant to the shift, so the result is exact); this
  * needs c_t ≤ 40 so that no row underflows, which always holds after QK-norm (c_t ≈ √Dh) — rows
@@ -193,7 +195,7 @@ gpt_status gpt_attention_fwd(const void* q, const void* k, const void* v, void* 
                              long long sh_qkv, long long st_qkv, long long sb_o, long long sh_o,
                              long long st_o, int* status, void* stream);
 /* Bytes of the `delta` scratch that gpt_attention_bwd needs for (B, H, T): 40 bytes per row of
- * B·H·⌈T/64⌉·64.  Returns 0 for a non-positive size. */
+ * R = B·H·⌈T/64⌉·64, plus 2·T·R bytes of dSᵀ.  Returns 0 for a non-positive size. */
 size_t gpt_attention_bwd_scratch_bytes(int B, int H, int T);
 gpt_status gpt_attention_bwd(const void* q, const void* k, const void* v, const void* o,
                              const void* dout, const float* lse, float* delta, void* dq, void* dk,
@@ -203,15 +205,16 @@ gpt_status gpt_attention_bwd(const void* q, const void* k, const void* v, const 
 
 /* Attention backward that allocates nothing.  The pages have no counterpart: this is a calling
  * convenience, not part of the method.  Arguments and results are those of gpt_attention_bwd
- * without `delta`; the per-row scratch that the backward needs (gpt_attention_bwd_scratch_bytes)
- * is kept in a static device array inside this library (GPT_ATTN_BWD_NOALLOC_MAX_ROWS fp32 values =
- * 8 MiB), which every GPU that loads the library holds until the process exits.
+ * without `delta`; the per-row scratch that the backward needs (40 bytes per row of
+ * B·H·⌈T/64⌉·64) is kept in a static device array inside this library
+ * (GPT_ATTN_BWD_NOALLOC_MAX_ROWS fp32 values = 8 MiB), which every GPU that loads the library holds
+ * until the process exits.  dSᵀ is not stored: the dQ kernel recomputes the scores instead.
  * It serves callers that cannot obtain device memory where they call the backward — for example
  * code running under a device-memory budget fixed at start-up, or inside a host framework whose own
  * allocator owns all device memory and allows no side allocations — and therefore cannot hand
  * gpt_attention_bwd its scratch buffer.  It calls no cudaMalloc, cudaFree or allocating routine.
- *   - gpt_attention_bwd_scratch_bytes(B, H, T) > 4·GPT_ATTN_BWD_NOALLOC_MAX_ROWS returns
- *     GPT_ERR_UNSUPPORTED_SHAPE; nothing is enqueued.
+ *   - 40·B·H·⌈T/64⌉·64 > 4·GPT_ATTN_BWD_NOALLOC_MAX_ROWS returns GPT_ERR_UNSUPPORTED_SHAPE;
+ *     nothing is enqueued.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
  *     that device current); make that first call before any stream capture.
  *   - All calls share the one array.  Each call writes the rows it uses before reading them, so
