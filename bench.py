@@ -155,6 +155,16 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
+def workload_config(cfg, world):
+    """The `config` object both arms print: the workload, not the implementation."""
+    return {"workload": f"{cfg.name} GPT fwd+bwd step", "model": cfg.name,
+            "global_batch": cfg.batch * world, "seq_len": cfg.seq_len,
+            "parallelism": f"dp{world}" if world > 1 else "none",
+            "depth": cfg.depth, "d_model": cfg.d_model, "vocab": cfg.vocab,
+            "windows": "SSSL w=1024" if any(cfg.windows) else "full causal",
+            "l2": "inputs larger than L2 (activations ~tens of GB), no flush"}
+
+
 def run_reference(args, cfg):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -171,8 +181,7 @@ def run_reference(args, cfg):
         "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic", "mfu": mfu,
-        "config": {"workload": f"{cfg.name} GPT fwd+bwd step (CPU oracle sample)", "model": cfg.name,
-                   "global_batch": 1, "seq_len": scfg.seq_len, "parallelism": "none"},
+        "config": workload_config(cfg, max(1, args.gpus)),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -181,7 +190,7 @@ def run_reference(args, cfg):
 
 
 # ------------------------------------------------------------------------------------------------
-# multi-rank bookkeeping (replicas: no collective on the data path)
+# multi-rank bookkeeping and the data-parallel exchange
 # ------------------------------------------------------------------------------------------------
 def max_over_ranks(values, world, device="cpu"):
     """Element-wise maximum of per-rank timings (the slowest rank sets the job's time)."""
@@ -338,11 +347,7 @@ def run_ours(args, cfg):
                                    f"{cfg.token_dist} token ids)",
         "mfu": mfu, "mfu_of_measured_sustained": fpt * value / (world * peak_sus * 1e12),
         "flops_per_token": fpt,
-        "config": {"workload": workload, "model": cfg.name, "global_batch": cfg.batch * world,
-                   "seq_len": cfg.seq_len, "parallelism": f"dp{world}" if world > 1 else "none",
-                   "depth": cfg.depth, "d_model": cfg.d_model, "vocab": cfg.vocab,
-                   "windows": "SSSL w=1024" if any(cfg.windows) else "full causal",
-                   "l2": "inputs larger than L2 (activations ~tens of GB), no flush"},
+        "config": workload_config(cfg, world),
         "loss_first_step": loss0,
         "e2e": {"value": value_e2e, "unit": "tokens/s",
                 "h2d_bytes_per_step": int(tok_np.nbytes + tgt_np.nbytes), "d2h_bytes_per_step": 4},
