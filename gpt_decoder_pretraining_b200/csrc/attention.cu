@@ -496,10 +496,14 @@ __global__ void __launch_bounds__(576, 1)
         uint32_t pk[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          float x0, x1;
+          float x0, x1, p0, p1;
           fma2_bc(x0, x1, __uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]), a.scale_log2, -c2);
-          float p0 = ex2_approx(x0);
-          float p1 = ex2_approx(x1);
+          if ((e & 3) == 3) {  // one pair in four on the FMA pipe
+            exp2_poly2(p0, p1, x0, x1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
           if (need_mask) {
             const int key = kv0 + 16 * c + 2 * e;
             if (!(key <= t && key > t - W)) p0 = 0.f;

@@ -443,6 +443,38 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, v
   return __all_sync(0xffffffffu, ok) != 0;
 }
 
+// (d0, d1) = (a0·b0 + c, a1·b1 + c)
+__device__ __forceinline__ void fma2_c(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                       float c) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %6};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c));
+}
+
+// 2^x for a pair, x ≥ −126, on the FMA pipe instead of the exponential unit: x = n + f with
+// n = round(x) (the 1.5·2^23 rounding constant), |f| ≤ 1/2; 2^f by a cubic fitted to 2^f on
+// [−1/2, 1/2] by reweighted least squares (max relative error 7.5e-5, far below the bf16 rounding
+// that P gets next); n is added to the exponent field.  Used for a quarter of the softmax weights so
+// that the exponential unit and the FMA pipe share the work.
+__device__ __forceinline__ void exp2_poly2(float& p0, float& p1, float x0, float x1) {
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  float t0, t1, r0, r1, f0, f1, q0, q1;
+  add2_bc(t0, t1, x0, x1, 12582912.f);
+  add2_bc(r0, r1, t0, t1, -12582912.f);
+  sub2(f0, f1, x0, x1, r0, r1);
+  fma2_bc(q0, q1, f0, f1, 0.0551716052f, 0.242611110f);
+  fma2_c(q0, q1, q0, q1, f0, f1, 0.693260968f);
+  fma2_c(q0, q1, q0, q1, f0, f1, 0.999928057f);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
