@@ -1,17 +1,23 @@
 // Causal / sliding-window flash attention, forward and backward, for head_dim 32, 64 or 128.
 //
 // The causal softmax attention of the nanochat decoder ("nanochat User Guide" §10: sliding-window
-// attention pattern; queries see keys t−w < j ≤ t).  Q/K/V/dO tiles are staged into shared memory
-// by 4-D TMA loads (128-byte swizzle, double-buffered, mbarrier completion); the products run on
-// the tensor cores as m16n8k16 bf16 MMAs with fp32 accumulation; the online softmax lives in
-// registers, with row statistics reduced over each quad by warp shuffles.  KV tiles entirely
-// outside the causal band or the window are never loaded.
+// attention pattern; queries see keys t−w < j ≤ t).  KV tiles entirely outside the causal band or the
+// window are never loaded.
 //
-//   forward     grid (q tiles of 128, H, B), 8 warps × 16 query rows; O and LSE (natural log).
-//   backward    (1) delta = rowsum(dO∘O);  (2) dK, dV: grid over 64-key tiles, loop over the query
-//               tiles that see them;  (3) dQ: grid over 64-query tiles, loop over their key tiles.
-//               No atomics: every output element is written by exactly one thread, so results are
-//               bitwise reproducible.
+// head_dim 64 / 128 (the model's heads): tcgen05 kernels.  Q/K/V/dO tiles arrive by 4-D TMA loads
+// (128-byte swizzle, mbarrier rings); scores and accumulators live in tensor memory; one warp issues
+// the MMAs (warp-wide loop, one elected lane), softmax warps read scores with tcgen05.ld and write
+// bf16 weights back for the next MMA.
+//   forward     grid (256-query blocks, H, B): 2 query tiles of 128, 16 softmax warps.  Each row's
+//               exponentials are shifted by the Cauchy–Schwarz bound ‖q‖·max‖k‖/√Dh rather than a
+//               running maximum (softmax is shift-invariant), so O needs no rescaling.
+//   backward    (1) delta pre-pass: rowsum(dO∘O), LSE, and their bf16 "extension rows";
+//               (2) dK, dV: grid over 128-key tiles, loop over 64-query tiles; −LSE and −delta enter
+//                   the score accumulators through one extra K = 16 MMA each; dSᵀ is stored;
+//               (3) dQ = dS·K from the stored dSᵀ (or, for the allocation-free entry, with the scores
+//                   recomputed).
+// head_dim 32 (small test configurations): m16n8k16 mma.sync kernels with an online softmax.
+// No atomics anywhere: every output element has one writer, so results are bitwise reproducible.
 
 #include <algorithm>
 #include <mutex>
@@ -101,7 +107,7 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 
 // ================================================================================================
-// forward
+// forward, mma.sync (head_dim 32)
 // ================================================================================================
 template <int DH>
 struct FwdShape {
@@ -565,16 +571,18 @@ __global__ void __launch_bounds__(576, 1)
 }
 
 // ================================================================================================
-// backward on the tcgen05 tensor cores (head_dim 64 or 128), two deterministic kernels
+// backward on the tcgen05 tensor cores (head_dim 64 or 128), deterministic kernels
 //
 // dK/dV kernel: one CTA per 128-key tile; loops over the 64-query tiles that see it.
 //   Sᵀ = K·Qᵢᵀ and dPᵀ = V·dOᵢᵀ (128 keys × 64 queries, A and B from shared memory) go to tensor
-//   memory; the softmax warps (one key row per thread) form Pᵀ = exp(Sᵀ/√Dh − LSE) and
-//   dSᵀ = Pᵀ∘(dPᵀ − delta), write both back over Sᵀ / dPᵀ as packed bf16, and the MMA warp
-//   accumulates dV += Pᵀ·dOᵢ and dK += dSᵀ·Qᵢ with A read from tensor memory.
-// dQ kernel: one CTA per 128-query tile; loops over its 64-key tiles.
-//   S = Q·Kⱼᵀ, dP = dO·Vⱼᵀ; the softmax warps (one query row per thread) write dS over S and the
-//   MMA warp accumulates dQ += dS·Kⱼ.
+//   memory, each followed by a K = 16 extension MMA that adds −LSE·√Dh resp. −delta per query
+//   column; the softmax warps (one key row per thread) form Pᵀ = 2^(Sᵀ·log2 e/√Dh) and
+//   dSᵀ = Pᵀ∘dPᵀ, write both back over Sᵀ / dPᵀ as packed bf16 (and dSᵀ to global memory when the
+//   caller's scratch holds it), and the MMA warp accumulates dV += Pᵀ·dOᵢ and dK += dSᵀ·Qᵢ with A
+//   read from tensor memory.
+// dQ: from the stored dSᵀ (attn_bwd_dq_ds_kernel, below), or with the scores recomputed: one CTA
+//   per 128-query tile looping over its 64-key tiles, S = Q·Kⱼᵀ, dP = dO·Vⱼᵀ, the softmax warps
+//   (one query row per thread) write dS over S and the MMA warp accumulates dQ += dS·Kⱼ.
 // S/dP buffers are double-buffered in tensor memory, so tile i+1's products run while the softmax
 // warps work on tile i.  Each output element has exactly one writer: results are reproducible.
 // ================================================================================================
@@ -1345,7 +1353,7 @@ __global__ void attn_kmax_kernel(const uint16_t* __restrict__ k, float* __restri
 }
 
 // ================================================================================================
-// backward (1): delta = rowsum(dO ∘ O), one warp per row
+// backward (1): delta = rowsum(dO ∘ O), LSE·log2 e and the extension rows, Dh/8 lanes per row
 // ================================================================================================
 // v as hi + mid + lo in bf16 (each a round-to-nearest-even of the remainder): ~24 significant bits
 __device__ __forceinline__ uint2 split3_bf16(float v) {
@@ -1397,7 +1405,8 @@ __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t
 }
 
 // ================================================================================================
-// backward (2): dK, dV for a 64-key tile; 4 warps × 16 keys; loop over 64-query tiles
+// backward (2), mma.sync (head_dim 32): dK, dV for a 64-key tile; 4 warps × 16 keys; loop over
+// 64-query tiles
 // ================================================================================================
 template <int DH>
 struct BwdShape {
@@ -1565,7 +1574,8 @@ __global__ void __launch_bounds__(128)
 }
 
 // ================================================================================================
-// backward (3): dQ for a 64-query tile; 4 warps × 16 rows; loop over key tiles
+// backward (3), mma.sync (head_dim 32): dQ for a 64-query tile; 4 warps × 16 rows; loop over key
+// tiles
 // ================================================================================================
 template <int DH>
 __global__ void __launch_bounds__(128)
