@@ -7,10 +7,13 @@
 //
 //   warp 0      TMA producer (both CTAs): 128×64 A and 128×64 B tiles (128-byte swizzle) into the
 //               ring; every load counts its bytes on the leader CTA's "full" barrier.
-//   warp 1      MMA issuer (leader CTA only): tcgen05.mma 256×256×16 into a double-buffered
-//               accumulator; commits free the ring stage and publish the tile in both CTAs.
-//   warps 2..5  epilogue (both CTAs): tcgen05.ld one accumulator row per thread, fused epilogue
-//               (bf16 cast, residual add, ReLU², dReLU², fp32 store / add, split-K reduction, or the
+//   warp 1      MMA issuer (leader CTA only; the warp runs the loop, one elected lane issues):
+//               tcgen05.mma 256×256×16 into a double-buffered accumulator; commits free the ring
+//               stage and publish the tile in both CTAs.
+//   warps 2..   epilogue (both CTAs): 4 warps per column group (one per tensor-memory lane
+//               quarter; two groups split the 256 columns, one for the QKV + RoPE epilogue);
+//               tcgen05.ld one accumulator row per thread, fused epilogue (bf16 cast, residual add,
+//               ReLU², dReLU², fp32 store / add, split-K reduction, QKV + RoPE + QK-norm, or the
 //               cross-entropy statistics / gradient of the fused lm-head), global store; then
 //               release the accumulator buffer to the leader.
 // Tiles (and K halves, for split-K) are distributed persistently over the CTA pairs.
