@@ -1744,17 +1744,11 @@ gpt_status check_attn(const void* p, int B, int H, int T, int Dh, long long sb, 
   return GPT_OK;
 }
 
-template <typename K>
-gpt_status set_smem(K kern, int bytes) {
-  GPT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
-  return GPT_OK;
-}
 
 template <int DH>
 gpt_status launch_fwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const AttnArgs& a, cudaStream_t stream) {
-  static bool once = false;
-  if (!once) { GPT_TRY(set_smem(attn_fwd_kernel<DH>, FwdShape<DH>::SMEM)); once = true; }
+  GPT_TRY(ensure_smem(attn_fwd_kernel<DH>, FwdShape<DH>::SMEM));
   attn_fwd_kernel<DH><<<grid, 256, FwdShape<DH>::SMEM, stream>>>(mq, mk, mv, a);
   count_launch();
   GPT_CUDA_TRY(cudaGetLastError());
@@ -1765,8 +1759,7 @@ template <int DH>
 gpt_status launch_fwd_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const AttnArgs& a, const float* kmax, float kmax_const, cudaStream_t stream) {
   using S = TcFwdShape<DH>;
-  static bool once = false;
-  if (!once) { GPT_TRY(set_smem(attn_fwd_tc_kernel<DH>, S::SMEM)); once = true; }
+  GPT_TRY(ensure_smem(attn_fwd_tc_kernel<DH>, S::SMEM));
   dim3 grid((a.T + 255) / 256, a.H, a.B);
   attn_fwd_tc_kernel<DH><<<grid, S::THREADS, S::SMEM, stream>>>(mq, mk, mv, a, kmax, kmax_const);
   count_launch();
@@ -1778,12 +1771,8 @@ template <int DH>
 gpt_status launch_bwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const CUtensorMap& mdo, AttnArgs a, void* dq, cudaStream_t stream) {
   constexpr int smem = BwdShape<DH>::SMEM;
-  static bool once = false;
-  if (!once) {
-    GPT_TRY(set_smem(attn_bwd_dkdv_kernel<DH>, smem));
-    GPT_TRY(set_smem(attn_bwd_dq_kernel<DH>, smem));
-    once = true;
-  }
+  GPT_TRY(ensure_smem(attn_bwd_dkdv_kernel<DH>, smem));
+  GPT_TRY(ensure_smem(attn_bwd_dq_kernel<DH>, smem));
   attn_bwd_dkdv_kernel<DH><<<grid, 128, smem, stream>>>(mq, mk, mv, mdo, a);
   count_launch();
   GPT_CUDA_TRY(cudaGetLastError());
@@ -1802,13 +1791,9 @@ gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[
                          cudaStream_t stream) {
   using S = TcBwdShape<DH>;
   using SD = DqDsShape<DH>;
-  static bool once = false;
-  if (!once) {
-    GPT_TRY(set_smem(attn_bwd_dkdv_tc_kernel<DH>, S::SMEM));
-    GPT_TRY(set_smem(attn_bwd_dq_tc_kernel<DH>, S::SMEM));
-    GPT_TRY(set_smem(attn_bwd_dq_ds_kernel<DH>, SD::SMEM));
-    once = true;
-  }
+  GPT_TRY(ensure_smem(attn_bwd_dkdv_tc_kernel<DH>, S::SMEM));
+  GPT_TRY(ensure_smem(attn_bwd_dq_tc_kernel<DH>, S::SMEM));
+  GPT_TRY(ensure_smem(attn_bwd_dq_ds_kernel<DH>, SD::SMEM));
   // dK/dV: outer 128-key tiles (K, V with 128-row boxes), inner 64-query tiles (Q, dO 64-row boxes)
   dim3 g1((a.T + 127) / 128, a.H, a.B);
   attn_bwd_dkdv_tc_kernel<DH><<<g1, S::THREADS, S::SMEM, stream>>>(m64[0], m128[1], m128[2], m64[3],

@@ -476,12 +476,7 @@ static gpt_status launch_inst(const CUtensorMap& ma, const CUtensorMap& mb, cons
                               cudaStream_t stream) {
   using S = GemmShape;
   auto kern = gemm_kernel<A_MN, B_MN, EPI>;
-  static bool attr_done = false;  // per instantiation
-  if (!attr_done) {
-    GPT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      S::SMEM_BYTES));
-    attr_done = true;
-  }
+  GPT_TRY(ensure_smem(kern, S::SMEM_BYTES));
   int sms = 0;
   GPT_TRY(device_info(&sms));
   const int units = a.tiles_m * a.tiles_n * a.splits;

@@ -2,6 +2,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <unordered_map>
 
 #include "host.h"
 
@@ -10,10 +11,12 @@ namespace gpt {
 thread_local int64_t g_launch_count = 0;
 
 gpt_status device_info(int* num_sms) {
+  static std::mutex mu;
   static int cached_sms[64] = {0};
   int dev = 0;
   GPT_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return GPT_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
   if (cached_sms[dev] == 0) {
     int major = 0, sms = 0;
     GPT_CUDA_TRY(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
@@ -22,6 +25,21 @@ gpt_status device_info(int* num_sms) {
     cached_sms[dev] = sms;
   }
   *num_sms = cached_sms[dev];
+  return GPT_OK;
+}
+
+gpt_status ensure_smem_limit(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::unordered_map<const void*, uint64_t> done;  // kernel -> bit per device
+  int dev = 0;
+  GPT_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return GPT_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
+  uint64_t& mask = done[kernel];
+  if (!((mask >> dev) & 1)) {
+    GPT_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+    mask |= 1ull << dev;
+  }
   return GPT_OK;
 }
 

@@ -36,6 +36,14 @@ bool encode_map_f32(CUtensorMap* map, const void* base, int rank, const uint64_t
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current device, once per
+// (kernel, device); safe to call from several host threads.
+gpt_status ensure_smem_limit(const void* kernel, int bytes);
+template <typename K>
+inline gpt_status ensure_smem(K kernel, int bytes) {
+  return ensure_smem_limit(reinterpret_cast<const void*>(kernel), bytes);
+}
+
 // Kernel-launch counter for reporting how many of this library's kernels a step enqueued.
 extern thread_local int64_t g_launch_count;
 inline void count_launch(int n = 1) { g_launch_count += n; }

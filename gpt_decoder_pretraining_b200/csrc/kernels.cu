@@ -626,12 +626,7 @@ gpt_status embedding_bwd(const int32_t* tok, const float* gx, float* dwte, int M
   int* nruns = reinterpret_cast<int*>(p + al((size_t)seg * 4) + al((size_t)(seg + 1) * 4));
   float* partial = reinterpret_cast<float*>(p + al((size_t)seg * 4) + al((size_t)(seg + 1) * 4) + al(4));
   GPT_CUDA_TRY(cudaMemsetAsync(dwte, 0, (size_t)V * d * sizeof(float), s));
-  static bool attr = false;
-  if (!attr) {
-    GPT_CUDA_TRY(cudaFuncSetAttribute(embedding_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      EMB_SEG * 4));
-    attr = true;
-  }
+  GPT_TRY(ensure_smem(embedding_sort_kernel, EMB_SEG * 4));
   const int threads = std::min(512, std::max(32, ((d / 4) + 31) / 32 * 32));
   for (int s0 = 0; s0 < M; s0 += EMB_SEG) {
     const int n = std::min(EMB_SEG, M - s0);
