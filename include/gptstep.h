@@ -38,7 +38,7 @@ extern "C" {
 typedef enum gpt_status {
   GPT_OK = 0,
   GPT_ERR_INVALID_ARG = -1,        /* null pointer, non-positive size, bad enum */
-  GPT_ERR_UNSUPPORTED_SHAPE = -2,  /* a size this build cannot tile (see each call) */
+  GPT_ERR_UNSUPPORTED_SHAPE = -2,  /* a size the library cannot tile (see each call) */
   GPT_ERR_WORKSPACE_TOO_SMALL = -3,
   GPT_ERR_CUDA = -4,               /* a CUDA runtime call or kernel launch failed */
   GPT_ERR_DEVICE_TIMEOUT = -5,     /* a bounded device-side wait expired; results are invalid */
