@@ -495,6 +495,19 @@ __global__ void cast_f32_bf16_kernel(const float* __restrict__ src, uint16_t* __
   }
 }
 
+// dst[i] += src[i] (gradient accumulation across micro-batches), four floats per thread
+__global__ void add_f32_kernel(float* __restrict__ dst, const float* __restrict__ src, size_t n) {
+  const size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (i + 4 <= n) {
+    float4 a = *reinterpret_cast<const float4*>(dst + i);
+    const float4 b = *reinterpret_cast<const float4*>(src + i);
+    a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+    *reinterpret_cast<float4*>(dst + i) = a;
+  } else {
+    for (size_t j = i; j < n; ++j) dst[j] += src[j];
+  }
+}
+
 // ------------------------------------------------------------------------------------------------
 // launchers
 // ------------------------------------------------------------------------------------------------
@@ -659,6 +672,15 @@ gpt_status ce_rows(const float2* stats, int ntiles, const float* zt, const int32
 gpt_status ce_finalize(const float* ell, const int32_t* targets, int M, int V, float* loss,
                        float* inv_n, cudaStream_t s) {
   ce_finalize_kernel<<<1, 1024, 0, s>>>(ell, targets, M, V, loss, inv_n);
+  count_launch();
+  GPT_CUDA_TRY(cudaGetLastError());
+  return GPT_OK;
+}
+
+gpt_status add_f32(float* dst, const float* src, size_t n, cudaStream_t s) {
+  const size_t threads = 256, per = 4;
+  const size_t blocks = (n + threads * per - 1) / (threads * per);
+  add_f32_kernel<<<(unsigned)blocks, (unsigned)threads, 0, s>>>(dst, src, n);
   count_launch();
   GPT_CUDA_TRY(cudaGetLastError());
   return GPT_OK;

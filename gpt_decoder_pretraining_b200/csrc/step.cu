@@ -40,6 +40,7 @@ gpt_status ce_rows(const float2* stats, int ntiles, const float* zt, const int32
 gpt_status ce_finalize(const float* ell, const int32_t* targets, int M, int V, float* loss,
                        float* inv_n, cudaStream_t s);
 gpt_status cast_f32_bf16(const float* src, void* dst, size_t n, cudaStream_t s);
+gpt_status add_f32(float* dst, const float* src, size_t n, cudaStream_t s);
 gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                          int H, int T, int Dh, int window, long long sbq, long long shq,
                          long long stq, long long sbo, long long sho, long long sto, int* status,
@@ -105,6 +106,7 @@ struct Plan {
   size_t stats, zt, lse_ce, ell, inv_n, dz, dxf;
   // backward transients
   size_t gx, gxb, du, dr, dO, dqkv, delta, emb;
+  size_t gacc;  // this micro-batch's gradients when the call accumulates into the caller's
   size_t total;
   int vc;  // vocabulary chunk of the backward lm-head
 };
@@ -198,6 +200,7 @@ static Plan make_plan(const gpt_config& c, size_t n_params) {
   p.dqkv = take(M * 3 * d * 2);
   p.delta = take(attention_bwd_scratch_bytes(c.batch, H, c.seq_len, true));
   p.emb = take(embedding_bwd_scratch_bytes((int)M, (int)d, (int)V));
+  p.gacc = take(n_params * 4);
   p.total = pos;
   return p;
 }
@@ -468,7 +471,7 @@ gpt_status gpt_step_fwd_bwd(gpt_step* step, const void* params, const int32_t* t
                             size_t workspace_bytes, int accumulate, void* stream) {
   if (!step || !params || !tokens || !targets || !loss || !grads || !workspace)
     return GPT_ERR_INVALID_ARG;
-  if (accumulate != 0) return GPT_ERR_INVALID_ARG;
+  if (accumulate != 0 && accumulate != 1) return GPT_ERR_INVALID_ARG;
   if (workspace_bytes < step->plan.total) return GPT_ERR_WORKSPACE_TOO_SMALL;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255) || (reinterpret_cast<uintptr_t>(params) & 15) ||
       (reinterpret_cast<uintptr_t>(grads) & 15))
@@ -477,8 +480,13 @@ gpt_status gpt_step_fwd_bwd(gpt_step* step, const void* params, const int32_t* t
   gpt_status dv = gpt::device_info(&sms);
   if (dv != GPT_OK) return dv;
   const int64_t before = gpt::g_launch_count;
-  gpt_status r = gpt::run_step(step, params, tokens, targets, loss, grads,
-                               reinterpret_cast<uint8_t*>(workspace), gpt::as_stream(stream));
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  // accumulate = 1: the step's gradients go to workspace scratch and are then added to `grads`
+  // element by element (one fp32 add per element, so the result does not depend on scheduling)
+  float* g = accumulate ? reinterpret_cast<float*>(ws + step->plan.gacc) : grads;
+  gpt_status r = gpt::run_step(step, params, tokens, targets, loss, g, ws, gpt::as_stream(stream));
+  if (r == GPT_OK && accumulate)
+    r = gpt::add_f32(grads, g, step->layout.total, gpt::as_stream(stream));
   step->last_launches = gpt::g_launch_count - before;
   return r;
 }

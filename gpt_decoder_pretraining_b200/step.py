@@ -159,8 +159,9 @@ class GptStep:
         except Exception:
             pass
 
-    def __call__(self, params, tokens, targets, grads=None, loss=None):
-        """Enqueue one step on the current stream; returns (loss tensor [1], grads tensor)."""
+    def __call__(self, params, tokens, targets, grads=None, loss=None, accumulate=False):
+        """Enqueue one step on the current stream; returns (loss tensor [1], grads tensor).
+        With ``accumulate`` the step's gradients are added to ``grads`` instead of replacing them."""
         grads = self.grads if grads is None else grads
         loss = self.loss if loss is None else loss
         want = "torch.float32" if self.cfg.param_dtype == DTYPE_F32 else "torch.bfloat16"
@@ -170,7 +171,7 @@ class GptStep:
             raise ValueError("tokens/targets must be int32")
         st = lib().gpt_step_fwd_bwd(self._h, params.data_ptr(), tokens.data_ptr(), targets.data_ptr(),
                                     loss.data_ptr(), grads.data_ptr(), self.workspace.data_ptr(),
-                                    self.workspace_bytes, 0, _stream())
+                                    self.workspace_bytes, 1 if accumulate else 0, _stream())
         _check(st, "gpt_step_fwd_bwd")
         return loss, grads
 

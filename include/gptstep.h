@@ -86,7 +86,9 @@ gpt_status gpt_step_workspace_bytes(const gpt_step* step, size_t* bytes);
  *   tokens    [batch, seq_len] int32 in [0, V)
  *   targets   [batch, seq_len] int32 in [0, V) or −1 (ignored)
  *   loss      1 float: Σ_valid ℓ / n_valid, or 0 when no target is valid (grads are then 0 too)
- *   grads     [n_params] fp32, overwritten (accumulate must be 0 in this version)
+ *   grads     [n_params] fp32: overwritten (accumulate = 0) or added to (accumulate = 1: the
+ *             step's own gradients go to workspace scratch first and are then added element by
+ *             element, so micro-batches accumulate deterministically; loss is this call's alone)
  *   workspace ≥ gpt_step_workspace_bytes, 256-byte aligned
  * Out-of-range ids are clamped for memory safety and flagged in the device status word. */
 gpt_status gpt_step_fwd_bwd(gpt_step* step, const void* params, const int32_t* tokens,

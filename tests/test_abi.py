@@ -109,7 +109,7 @@ def test_step_argument_errors_need_no_device(lib):
     fake = 1 << 20  # never dereferenced: validation fails first
     call = lib.gpt_step_fwd_bwd
     assert call(h, None, fake, fake, fake, fake, fake, n.value, 0, None) == -1           # null params
-    assert call(h, fake, fake, fake, fake, fake, fake, n.value, 1, None) == -1           # accumulate
+    assert call(h, fake, fake, fake, fake, fake, fake, n.value, 2, None) == -1           # accumulate ∉ {0, 1}
     assert call(h, fake, fake, fake, fake, fake, fake, n.value - 1, 0, None) == -3       # too small
     assert call(h, fake + 8, fake, fake, fake, fake, fake, n.value, 0, None) == -2       # misaligned
     assert lib.gpt_step_status(None, fake, None) == -1

@@ -103,3 +103,25 @@ def test_step_token_out_of_range_sets_status():
     st(p, torch.from_numpy(tokens).cuda(), torch.from_numpy(targets).cuda())
     assert st.status() == -6
     assert st.status() == 0  # reading clears the word
+
+
+def test_step_accumulates_gradients_across_micro_batches():
+    """accumulate = 1 adds this micro-batch's gradients to the buffer: two steps give exactly the
+    fp32 sum of the two single-step gradients (each element is one fp32 addition)."""
+    from gpt_decoder_pretraining_b200.step import GptStep
+    cfg = custom(2, 128, 64, 512, 96, 2, windows=[40, 0])
+    params, tokens, targets = make_config_inputs(cfg)
+    tokens_b, targets_b = np.roll(tokens, 5, axis=1), np.roll(targets, 5, axis=1)
+    st = GptStep(cfg)
+    p = torch.from_numpy(params.astype(np.float32)).cuda().to(torch.bfloat16)
+    as_t = lambda a: torch.from_numpy(np.ascontiguousarray(a).astype(np.int32)).cuda()  # noqa: E731
+    _, g = st(p, as_t(tokens), as_t(targets))
+    g_a = g.cpu().numpy().copy()
+    _, g = st(p, as_t(tokens_b), as_t(targets_b))
+    g_b = g.cpu().numpy().copy()
+    acc = torch.zeros_like(g)
+    st(p, as_t(tokens), as_t(targets), grads=acc)
+    st(p, as_t(tokens_b), as_t(targets_b), grads=acc, accumulate=True)
+    torch.cuda.synchronize()
+    assert st.status() == 0
+    assert np.array_equal(acc.cpu().numpy(), (g_a + g_b).astype(np.float32))
