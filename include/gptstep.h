@@ -198,7 +198,7 @@ gpt_status gpt_attention_fwd(const void* q, const void* k, const void* v, void* 
                              long long st_o, int* status, void* stream);
 /* Bytes of the `delta` scratch that gpt_attention_bwd needs for (B, H, T): 40 bytes per row of
  * R = B·H·⌈T/64⌉·64, plus 2·T·R bytes of dSᵀ — quadratic in T (1.6 GB for B·H = 192 at T = 2048,
- * 34 GB for B·H·T = 2^21 at T = 8192).  Callers short of memory can use
+ * 34 GB for B·H·T = 2^21 at T = 8192).  Callers short of memory can use, within its row limit,
  * gpt_attention_bwd_noalloc, which recomputes the scores instead.  Returns 0 for a non-positive
  * size. */
 size_t gpt_attention_bwd_scratch_bytes(int B, int H, int T);
