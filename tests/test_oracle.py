@@ -8,6 +8,8 @@
   per-position loss gradients, batch linearity and row-permutation invariance;
 * special cases that reduce to library routines: torch's rms_norm, linear (y = x·Wᵀ),
   scaled_dot_product_attention and cross_entropy, differentiated by autograd;
+* the whole step rebuilt from those torch library ops (RoPE from its definition), every gradient
+  from autograd, equal to the oracle to rounding;
 * the figures the pages print (tests/golden/page_figures.txt) and the ≈ ln V initial loss.
 """
 import math
@@ -377,3 +379,55 @@ def test_planted_mistakes_are_caught(monkeypatch, mistake):
             return keep
         monkeypatch.setattr(O, "attention_mask", bad_mask)
     assert not _run_pins(None)
+
+
+def _torch_model_loss(cfg, flat, tokens, targets):
+    """The architecture written with torch library ops only (embedding, rms_norm, linear, sdpa with a
+    boolean mask, cross_entropy with ignore_index); autograd supplies every gradient."""
+    d, H, Dh, T = cfg.d_model, cfg.n_heads, cfg.head_dim, cfg.seq_len
+    ws, off = {}, 0
+    for name, (a, b) in cfg.tensor_shapes():
+        ws[name] = flat[off:off + a * b].view(a, b)
+        off += a * b
+    pos = torch.arange(T, dtype=torch.float64)
+    inv = 10000.0 ** (-2.0 * torch.arange(Dh // 2, dtype=torch.float64) / Dh)
+    ang = pos[:, None] * inv[None, :]
+    cos, sin = torch.cos(ang), torch.sin(ang)
+
+    def rotate(x):  # pairs (i, i + Dh/2), positions along dim −2
+        a, b = x[..., :Dh // 2], x[..., Dh // 2:]
+        return torch.cat([a * cos - b * sin, a * sin + b * cos], dim=-1)
+
+    x = F.embedding(tokens, ws["wte"])
+    B = tokens.shape[0]
+    for l in range(cfg.depth):
+        w = cfg.effective_window(l)
+        i = torch.arange(T)
+        keep = (i[None, :] <= i[:, None]) & (i[None, :] > i[:, None] - w)
+        r = F.rms_norm(x, (d,), eps=1e-6)
+        qkv = F.linear(r, ws[f"h{l}.w_qkv"])
+        q, k, v = (t.view(B, T, H, Dh).transpose(1, 2) for t in qkv.split(d, dim=-1))
+        q = F.rms_norm(rotate(q), (Dh,), eps=1e-6)
+        k = F.rms_norm(rotate(k), (Dh,), eps=1e-6)
+        o = F.scaled_dot_product_attention(q, k, v, attn_mask=keep)
+        x = x + F.linear(o.transpose(1, 2).reshape(B, T, d), ws[f"h{l}.w_o"])
+        u = F.linear(F.rms_norm(x, (d,), eps=1e-6), ws[f"h{l}.w_fc"])
+        x = x + F.linear(torch.relu(u) ** 2, ws[f"h{l}.w_proj"])
+    z = F.linear(F.rms_norm(x, (d,), eps=1e-6), ws["w_lm"])
+    return F.cross_entropy(z.view(-1, cfg.vocab), targets.view(-1), ignore_index=-1, reduction="mean")
+
+
+@pytest.mark.parametrize("windows", [None, [3, 0]])
+def test_whole_step_vs_torch_autograd(windows):
+    """Every gradient of the oracle's step equals torch autograd through library ops, to rounding."""
+    cfg = tiny(depth=2, d=32, hd=16, V=64, T=12, B=2, windows=windows)
+    p, t, y = inputs_for(cfg, seed=5)
+    y = y.copy()
+    y[1, :3] = -1
+    r = O.step(cfg, p, t, y, dtype=np.float64)
+    flat = torch.tensor(p, requires_grad=True)
+    loss = _torch_model_loss(cfg, flat, torch.tensor(t, dtype=torch.long), torch.tensor(y, dtype=torch.long))
+    loss.backward()
+    assert abs(r["loss"] - loss.item()) < 1e-12
+    g = flat.grad.numpy()
+    np.testing.assert_allclose(r["grads"], g, rtol=0, atol=1e-12 * max(1.0, np.abs(g).max()))
