@@ -203,3 +203,14 @@ def _dp_rank_main(rank, world, port, q):
     bench.average_gradients(g, world)
     dist.destroy_process_group()
     q.put((rank, g.numpy()))
+
+
+def test_attention_backward_scratch_size(lib):
+    """Per padded row 40 bytes (LSE·log2 e and delta in fp32, two 16-byte extension rows), then
+    dSᵀ: 2·T bytes per padded row."""
+    f = lib.gpt_attention_bwd_scratch_bytes
+    f.restype = ctypes.c_size_t
+    for B, H, T in [(1, 1, 1), (2, 3, 200), (16, 12, 2048), (4, 8, 130)]:
+        rows = B * H * ((T + 63) // 64 * 64)
+        assert f(B, H, T) == rows * 40 + rows * T * 2
+    assert f(0, 1, 1) == 0 and f(1, 1, 0) == 0
