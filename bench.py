@@ -14,7 +14,14 @@ nanochat convention 6·(N − V·d) + 12·H·Dh·Σ_l min(w_l, T).
 * `roofline`: the GEMM class (the dominant kernel family) — algorithmic FLOPs ÷ its CUDA-event
   time, from separate profiled steps that record an event around every launch on the step's
   stream (kept out of the timed region) — against the measured sustained bf16 peak.
-* `cpu_baseline`: the CPU oracle timed on this host on a bounded sample (rank 0, N = 1).
+* `roofline`: `achieved` counts the method's GEMM FLOPs, 6·(N − V·d) per token; the lm-head logit
+  recompute of the backward pass is reported separately as executed work (`executed_tflops`).
+* `cpu_baseline`: the CPU oracle timed on this host on one row of the workload's sequence length
+  (median of 3 runs; rank 0, N = 1).
+* `also`: the second configuration the MFU target names (d20 by default), measured in the same run
+  on the same GPU (N = 1 only).
+* `--impl reference`: the oracle as it stands, one row of 512 tokens per step (a bounded sample
+  that keeps K + W steps within minutes); its `config` states that sample.
 * N > 1 (torchrun): data parallel with weak scaling — each rank runs the step on its own batch,
   then the fp32 gradients are averaged across ranks by one NCCL all-reduce per step (inside the
   timed region); the barrier and the max-reduction of the timings bracket the measurement.
@@ -170,18 +177,23 @@ def run_reference(args, cfg):
     if rank != 0:
         return 0
     cores = cpu_cores()
-    scfg, times = time_oracle(cfg, args.cpu_sample_tokens, repeats=args.steps, warmup=args.warmup)
+    scfg, times = time_oracle(cfg, args.ref_sample_tokens, repeats=args.steps, warmup=args.warmup)
     per_step = statistics.median(times)
     value = scfg.seq_len / per_step
     mfu = cfg.flops_per_token() * value / B200_DENSE_BF16_PEAK
     sample = (f"one row of {scfg.seq_len} tokens of the {cfg.name} model (B=1), fp32 NumPy oracle "
               f"fwd+bwd, median of {args.steps} after {args.warmup} warm-up")
+    # the model of the workload, timed on what one step of this arm processes: one row
+    config = workload_config(scfg, 1)
+    config.update(workload=f"{cfg.name} GPT fwd+bwd step", model=cfg.name,
+                  timed_sample=f"B 1 x T {scfg.seq_len} per step (a bounded CPU sample of the "
+                               f"B {cfg.batch * max(1, args.gpus)} x T {cfg.seq_len} workload)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value,
         "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic", "mfu": mfu,
-        "config": workload_config(cfg, max(1, args.gpus)),
+        "config": config,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -226,26 +238,19 @@ def whole_job_rate(units_per_rank_step, world, ms_per_step):
 # ------------------------------------------------------------------------------------------------
 # GPU arm
 # ------------------------------------------------------------------------------------------------
-def run_ours(args, cfg):
+def gemm_method_flops(cfg):
+    """FLOPs of the step's dense contractions as the method defines them: 6·(N − V·d) per token
+    (forward, data gradient and weight gradient of every projection, MLP and lm-head matrix).
+    The lm-head logit recompute of the backward pass is executed work on top of this."""
+    return 6.0 * (cfg.n_params - cfg.vocab * cfg.d_model) * cfg.tokens
+
+
+def measure_step(args, cfg, dev, world, rank, barrier, exchange, with_e2e=True):
+    """Warm up, time `args.steps` steps on device-resident inputs (CUDA events on the step's stream,
+    barrier + synchronize on both sides), then per-kernel-class profile steps and, optionally, the
+    same steps end to end through the public API with host buffers.  Returns a dict."""
     import torch
-    import torch.distributed as dist
     from gpt_decoder_pretraining_b200.step import GptStep
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def exchange(grads):
-        average_gradients(grads, world)
 
     step = GptStep(cfg, device=dev)
     params_np = make_params(cfg.n_params, keep_fp32=(cfg.param_dtype == 1))
@@ -257,14 +262,13 @@ def run_ours(args, cfg):
     targets = torch.from_numpy(tgt_np).to(dev)
     stream = torch.cuda.current_stream(dev)
 
-    # warm-up
     for _ in range(args.warmup):
         _, grads = step(params, tokens, targets)
         exchange(grads)
     torch.cuda.synchronize(dev)
     st = step.status()
     if st != 0:
-        raise RuntimeError(f"device status {st} after warm-up")
+        raise RuntimeError(f"device status {st} after warm-up ({cfg.name})")
     loss0 = float(step.loss.item())
 
     # ---------------- timed region (device-resident inputs) ----------------
@@ -296,37 +300,28 @@ def run_ours(args, cfg):
     step.set_profiling(False)
     prof = step.profile()
 
-    # ---------------- end to end through the public API, host buffers ----------------
-    tok_h = torch.from_numpy(tok_np).pin_memory()
-    tgt_h = torch.from_numpy(tgt_np).pin_memory()
-    loss_h = torch.zeros(1, dtype=torch.float32).pin_memory()
-    tok_d, tgt_d = torch.empty_like(tokens), torch.empty_like(targets)
-    barrier()
-    torch.cuda.synchronize(dev)
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(args.steps):
-        tok_d.copy_(tok_h, non_blocking=True)
-        tgt_d.copy_(tgt_h, non_blocking=True)
-        loss, grads = step(params, tok_d, tgt_d)
-        exchange(grads)
-        loss_h.copy_(loss, non_blocking=True)
-    f1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    ms_e2e = f0.elapsed_time(f1) / args.steps
-
-    ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, dev)
-    tokens_step = cfg.batch * cfg.seq_len
-    value = whole_job_rate(tokens_step, world, ms)
-    value_e2e = whole_job_rate(tokens_step, world, ms_e2e)
-    fpt = cfg.flops_per_token()
-    mfu = fpt * value / (world * B200_DENSE_BF16_PEAK)
-
-    peaks, peak_src = load_peaks()
-    g_ms, g_calls, g_fl, _ = prof["gemm"]
-    achieved = (g_fl / (g_ms / 1e3)) / 1e12 if g_ms > 0 else None
-    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    ms_e2e = None
+    if with_e2e:
+        # ---------------- end to end through the public API, host buffers ----------------
+        tok_h = torch.from_numpy(tok_np).pin_memory()
+        tgt_h = torch.from_numpy(tgt_np).pin_memory()
+        loss_h = torch.zeros(1, dtype=torch.float32).pin_memory()
+        tok_d, tgt_d = torch.empty_like(tokens), torch.empty_like(targets)
+        barrier()
+        torch.cuda.synchronize(dev)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            tok_d.copy_(tok_h, non_blocking=True)
+            tgt_d.copy_(tgt_h, non_blocking=True)
+            loss, grads = step(params, tok_d, tgt_d)
+            exchange(grads)
+            loss_h.copy_(loss, non_blocking=True)
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ms_e2e = f0.elapsed_time(f1) / args.steps
+    ms, ms_e2e_m = max_over_ranks([ms, ms_e2e if ms_e2e is not None else 0.0], world, dev)
     kernels = {}
     for name, (kms, calls, fl, by) in prof.items():
         if calls == 0:
@@ -338,6 +333,50 @@ def run_ours(args, cfg):
         if by:
             ent["gbs"] = by / (kms / 1e3) / 1e9
         kernels[name] = ent
+    out = {"ms": ms, "ms_e2e": ms_e2e_m if ms_e2e is not None else None, "clocks": clk,
+           "launches": launches, "loss0": loss0, "prof": prof, "prof_steps": prof_steps,
+           "kernels": kernels, "params_np": params_np,
+           "h2d": int(tok_np.nbytes + tgt_np.nbytes)}
+    del step, params, tokens, targets, grads
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def exchange(grads):
+        average_gradients(grads, world)
+
+    r = measure_step(args, cfg, dev, world, rank, barrier, exchange)
+    ms, ms_e2e = r["ms"], r["ms_e2e"]
+    tokens_step = cfg.batch * cfg.seq_len
+    value = whole_job_rate(tokens_step, world, ms)
+    value_e2e = whole_job_rate(tokens_step, world, ms_e2e)
+    fpt = cfg.flops_per_token()
+    mfu = fpt * value / (world * B200_DENSE_BF16_PEAK)
+
+    peaks, peak_src = load_peaks()
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    g_ms, g_calls, g_fl, _ = r["prof"]["gemm"]
+    g_ms_step = g_ms / r["prof_steps"]
+    method = gemm_method_flops(cfg)
+    achieved = (method / (g_ms_step / 1e3)) / 1e12 if g_ms > 0 else None
+    executed = (g_fl / (g_ms / 1e3)) / 1e12 if g_ms > 0 else None
     workload = f"{cfg.name} GPT fwd+bwd step"
     line = {
         "metric": METRIC,
@@ -348,26 +387,52 @@ def run_ours(args, cfg):
         "mfu": mfu, "mfu_of_measured_sustained": fpt * value / (world * peak_sus * 1e12),
         "flops_per_token": fpt,
         "config": workload_config(cfg, world),
-        "loss_first_step": loss0,
+        "loss_first_step": r["loss0"],
         "e2e": {"value": value_e2e, "unit": "tokens/s",
-                "h2d_bytes_per_step": int(tok_np.nbytes + tgt_np.nbytes), "d2h_bytes_per_step": 4},
-        "gpu_launches": int(launches),
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": 4},
+        "gpu_launches": int(r["launches"]),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
                      "frac": (achieved / peak_sus) if achieved else None,
                      "peak_source": f"bf16_tflops_sustained of {peak_src}",
                      "kernel": "tcgen05 GEMM family (all projection, MLP and lm-head GEMMs)",
+                     "achieved_basis": "6·(N − V·d)·B·T FLOP per step (the method's GEMM work) ÷ the "
+                                       "family's summed CUDA-event time per step",
+                     "gemm_method_flops_per_step": method,
+                     "gemm_ms_per_step": g_ms_step,
+                     "executed_tflops": executed,
+                     "executed_basis": "all launched GEMM FLOPs, including the lm-head logit recompute "
+                                       "of the backward pass (2·B·T·d·V per step)",
                      "traffic": load_traffic(workload)},
-        "kernels": kernels,
-        "clocks": clk,
+        "kernels": r["kernels"],
+        "clocks": r["clocks"],
     }
+    # the other configuration the ≥ 45% MFU target names, measured in the same run
+    if world == 1 and not args.no_also and cfg.name != args.also:
+        import dataclasses
+        acfg = preset(args.also)
+        a_args = dataclasses.replace(args) if dataclasses.is_dataclass(args) else argparse.Namespace(**vars(args))
+        a_args.steps = min(args.steps, 10)
+        ra = measure_step(a_args, acfg, dev, world, rank, barrier, exchange, with_e2e=False)
+        av = whole_job_rate(acfg.batch * acfg.seq_len, world, ra["ms"])
+        ag_ms, _, ag_fl, _ = ra["prof"]["gemm"]
+        ag_step = ag_ms / ra["prof_steps"]
+        line["also"] = {acfg.name: {
+            "workload": f"{acfg.name} GPT fwd+bwd step", "config": workload_config(acfg, world),
+            "steps": a_args.steps, "warmup": args.warmup, "ms_per_step": ra["ms"], "tokens_per_s": av,
+            "mfu": acfg.flops_per_token() * av / B200_DENSE_BF16_PEAK,
+            "gemm_tflops_method": gemm_method_flops(acfg) / (ag_step / 1e3) / 1e12 if ag_ms > 0 else None,
+            "kernels": ra["kernels"], "clocks": ra["clocks"], "loss_first_step": ra["loss0"]}}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         cores = cpu_cores()
-        scfg, times = time_oracle(cfg, args.cpu_sample_tokens, repeats=1, warmup=0, params=params_np)
-        cv = scfg.seq_len / times[0]
+        scfg, times = time_oracle(cfg, args.cpu_sample_tokens, repeats=args.cpu_repeats, warmup=0,
+                                  params=r["params_np"])
+        med = statistics.median(times)
+        cv = scfg.seq_len / med
         line["cpu_baseline"] = {
             "value": cv, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"one row of {scfg.seq_len} tokens of the {cfg.name} model (B=1), fp32 NumPy "
-                      f"oracle fwd+bwd, one timed run ({times[0]:.1f} s)"}
+                      f"oracle fwd+bwd, median of {len(times)} runs "
+                      f"({', '.join(f'{t:.1f}' for t in times)} s)"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -446,8 +511,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="d24")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-sample-tokens", type=int, default=512)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=2048,
+                    help="tokens of the one-row CPU oracle sample timed for cpu_baseline")
+    ap.add_argument("--cpu-repeats", type=int, default=3, help="timed oracle runs (median reported)")
+    ap.add_argument("--ref-sample-tokens", type=int, default=512,
+                    help="tokens of the one-row oracle sample of each --impl reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--also", default="d20", help="second configuration measured in the same run")
+    ap.add_argument("--no-also", action="store_true")
     ap.add_argument("--kernel", choices=["gemm", "attention"], default=None,
                     help="time one kernel-level workload instead of the step")
     ap.add_argument("--gemm-shape", default="32768,6144,1536")

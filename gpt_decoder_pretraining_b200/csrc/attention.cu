@@ -27,6 +27,8 @@
 
 namespace gpt {
 
+gpt_status wait_limit_set_attention(long long cycles) { return set_wait_limit_here(cycles); }
+
 namespace {
 
 constexpr float LOG2E = 1.4426950408889634f;
@@ -475,7 +477,7 @@ __global__ void __launch_bounds__(576, 1)
     const int tile0 = q0 + 128 * x;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const uint32_t s_addr = tmem + lane_off + S::TM_S + x * 128 + 64 * half;
-    bool ok = mbar_wait(bar_q, 0, abort_flag, a.status);
+    bool ok = mbar_wait_warp(bar_q, 0, abort_flag, a.status);
     // fixed shift c_t (log2 units)
     const float qn = sqrtf(q_row_sumsq<DH>(smem + S::OFF_Q + x * S::Q_TILE, row));
     const float km = kmax ? kmax[(long long)b * a.H + h] : kmax_const;
@@ -487,7 +489,7 @@ __global__ void __launch_bounds__(576, 1)
     // (exact for a single visible key).  Both as packed pairs of partial sums over this half.
     float l0 = 0.f, l1 = 0.f, lb0 = 0.f, lb1 = 0.f;
     for (int j = 0; j < n_kv && ok; ++j) {
-      if (!mbar_wait(&s_full[x], j & 1, abort_flag, a.status)) { ok = false; break; }
+      if (!mbar_wait_warp(&s_full[x], j & 1, abort_flag, a.status)) { ok = false; break; }
       tc_fence_after();
       const int kv0 = (kv_first + j) * 128 + 64 * half;  // first key of this thread's half
       const bool need_mask = (kv0 + 63 > tile0) || (kv0 <= tile0 + 127 - W);
@@ -535,7 +537,7 @@ __global__ void __launch_bounds__(576, 1)
     const float l = s0.x + s1.x;
     const float inv = 1.f / (s0.y + s1.y);
     // epilogue: O / lb, this half's DH/2 columns
-    if (ok) ok = mbar_wait(o_full, 0, abort_flag, a.status);
+    if (ok) ok = mbar_wait_warp(o_full, 0, abort_flag, a.status);
     if (ok) {
       tc_fence_after();
       uint16_t* orow = a.o + b * a.sb_o + h * a.sh_o + (long long)t * a.st_o;
@@ -863,7 +865,7 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = true;
     uint32_t rs[32], rp[32];
     if (n_q > 0) {
-      ok = mbar_wait(&s_full[0], 0, abort_flag, a.status);
+      ok = mbar_wait_warp(&s_full[0], 0, abort_flag, a.status);
       if (ok) {
         tc_fence_after();
         tmem_ld32(tmem + lane_off + S::TM_S + 32 * half, rs);
@@ -908,7 +910,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(&p_full[bf]);
       if (i + 1 < n_q) {
         const int nb = (i + 1) & 1;
-        if (!mbar_wait(&s_full[nb], ((i + 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&s_full[nb], ((i + 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
         tmem_ld32(tmem + lane_off + S::TM_S + nb * 64 + 32 * half, rs);
         tmem_ld32(tmem + lane_off + S::TM_P + nb * 64 + 32 * half, rp);
@@ -916,7 +918,7 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     // epilogue: half 0 writes the dV row, half 1 the dK row of each key
-    if (ok) ok = mbar_wait(done, 0, abort_flag, a.status);
+    if (ok) ok = mbar_wait_warp(done, 0, abort_flag, a.status);
     if (ok) {
       tc_fence_after();
       const long long off = b * a.sb_o + h * a.sh_o + (long long)key * a.st_o;
@@ -1084,7 +1086,7 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = true;
     uint32_t rs[32], rp[32];
     if (n_kv > 0) {
-      ok = mbar_wait(&s_full[0], 0, abort_flag, a.status);
+      ok = mbar_wait_warp(&s_full[0], 0, abort_flag, a.status);
       if (ok) {
         tc_fence_after();
         tmem_ld32(tmem + lane_off + S::TM_S + 32 * half, rs);
@@ -1120,14 +1122,14 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(&p_full[bf]);
       if (j + 1 < n_kv) {
         const int nb = (j + 1) & 1;
-        if (!mbar_wait(&s_full[nb], ((j + 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&s_full[nb], ((j + 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
         tmem_ld32(tmem + lane_off + S::TM_S + nb * 64 + 32 * half, rs);
         tmem_ld32(tmem + lane_off + S::TM_P + nb * 64 + 32 * half, rp);
         tmem_ld_wait();
       }
     }
-    if (ok) ok = mbar_wait(done, 0, abort_flag, a.status);
+    if (ok) ok = mbar_wait_warp(done, 0, abort_flag, a.status);
     if (ok) {
       tc_fence_after();
       uint16_t* dst = a.o + b * a.sb_o + h * a.sh_o + (long long)t * a.st_o;
@@ -1281,8 +1283,8 @@ __global__ void __launch_bounds__(192, 1)
     const int row = 32 * warp + lane;
     const int t = q0 + row;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
-    bool ok = mbar_wait(q_bar, 0, abort_flag, a.status);
-    if (ok) ok = mbar_wait(done, 0, abort_flag, a.status);
+    bool ok = mbar_wait_warp(q_bar, 0, abort_flag, a.status);
+    if (ok) ok = mbar_wait_warp(done, 0, abort_flag, a.status);
     if (ok) {
       tc_fence_after();
       uint16_t* dst = a.o + b * a.sb_o + h * a.sh_o + (long long)t * a.st_o;
@@ -1962,11 +1964,12 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
 
 // ------------------------------------------------------------------------------------------------
 // Allocation-free attention backward: the backward's per-row scratch (LSE·log2 e and
-// delta = rowsum(dO∘O), 2·B·H·⌈T/64⌉·64 floats) lives in this fixed array instead of a
-// caller-supplied buffer.  Every GPU that loads the library holds it until exit.
+// delta = rowsum(dO∘O) in fp32, then the two 16-byte bf16 extension rows: 40 bytes = 10 floats per
+// row of B·H·⌈T/64⌉·64) lives in this fixed array instead of a caller-supplied buffer.  Every GPU
+// that loads the library holds it until exit.
 // ------------------------------------------------------------------------------------------------
-constexpr long long NOALLOC_DELTA_ROWS = GPT_ATTN_BWD_NOALLOC_MAX_ROWS;
-static __device__ __align__(256) float g_noalloc_delta[NOALLOC_DELTA_ROWS];
+constexpr long long NOALLOC_FLOATS = GPT_ATTN_BWD_NOALLOC_FLOATS;
+static __device__ __align__(256) float g_noalloc_delta[NOALLOC_FLOATS];
 
 // Device address of g_noalloc_delta on the current device, looked up once per device with that
 // device current.  In host code the symbol itself is only a host-side stand-in for the array.
@@ -1994,7 +1997,7 @@ gpt_status attention_bwd_noalloc(const void* q, const void* k, const void* v, co
   if (B <= 0 || H <= 0 || T <= 0) return GPT_ERR_INVALID_ARG;
   // the fixed array holds the per-row scratch only: dQ recomputes the scores instead of reading
   // a stored dSᵀ
-  if ((long long)attention_bwd_scratch_bytes(B, H, T, false) > NOALLOC_DELTA_ROWS * 4)
+  if ((long long)attention_bwd_scratch_bytes(B, H, T, false) > NOALLOC_FLOATS * 4)
     return GPT_ERR_UNSUPPORTED_SHAPE;
   float* delta = nullptr;
   GPT_TRY(noalloc_delta_ptr(&delta));

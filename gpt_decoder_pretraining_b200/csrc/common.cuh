@@ -78,6 +78,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
 #define GPT_WAIT_LIMIT_CYCLES 4000000000ll
 #endif
 
+// The limit in force, one copy per translation unit (each .cu file sets its own copy through
+// set_wait_limit_here, called by gpt_set_wait_limit for every file that has waiting kernels).
+// Read only on the slow path of a wait, after the first poll failed.
+static __device__ long long g_wait_limit_cycles = GPT_WAIT_LIMIT_CYCLES;
+
+// Host side: set this translation unit's copy on the current device (cycles <= 0: the default).
+static inline gpt_status set_wait_limit_here(long long cycles) {
+  const long long v = cycles > 0 ? cycles : GPT_WAIT_LIMIT_CYCLES;
+  return cudaMemcpyToSymbol(g_wait_limit_cycles, &v, sizeof(v)) == cudaSuccess ? GPT_OK
+                                                                               : GPT_ERR_CUDA;
+}
+
 // Wait until the barrier's phase with the given parity has completed.  Returns false (after
 // recording a timeout) if the limit expired or another role of the CTA already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -85,10 +97,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
   const long long t0 = clock64();
+  const long long limit = *(volatile long long*)&g_wait_limit_cycles;
   while (true) {
     if (mbar_try_wait(addr, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > GPT_WAIT_LIMIT_CYCLES) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       set_status(status, GPT_ERR_DEVICE_TIMEOUT);
       return false;

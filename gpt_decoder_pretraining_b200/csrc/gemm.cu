@@ -30,6 +30,8 @@
 
 namespace gpt {
 
+gpt_status wait_limit_set_gemm(long long cycles) { return set_wait_limit_here(cycles); }
+
 constexpr int BM = 128;   // rows per CTA (the pair covers 256)
 constexpr int BN = 256;   // columns per tile (each CTA stages 128 rows of B)
 constexpr int BK = 64;
@@ -322,7 +324,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
       int tm, tn, kt0, kt1;
       unit_coords(u, tm, tn, kt0, kt1);
       const int m = tm * 2 * BM + rank * BM + row_in_tile;
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, args.status)) break;
+      if (!mbar_wait_warp(&tfull[acc], acc_phase, abort_flag, args.status)) break;
       tc_fence_after();
       float run_max = -INFINITY, run_sum = 0.f;
       int tgt = -1;

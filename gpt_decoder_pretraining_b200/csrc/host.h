@@ -48,6 +48,11 @@ inline gpt_status ensure_smem(K kernel, int bytes) {
 extern thread_local int64_t g_launch_count;
 inline void count_launch(int n = 1) { g_launch_count += n; }
 
+// Set the bounded-wait limit of the kernels of one translation unit on the current device.
+gpt_status wait_limit_set_gemm(long long cycles);
+gpt_status wait_limit_set_attention(long long cycles);
+gpt_status wait_limit_set_diag(long long cycles);
+
 // Kernel-level launchers used by the step orchestrator (same semantics as the C entry points).
 gpt_status gemm_launch(int op, int epi, int M, int N, int K, const void* A, int lda, const void* B,
                        int ldb, void* C, int ldc, void* C2, const void* aux, int ldaux, int* status,

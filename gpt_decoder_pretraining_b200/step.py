@@ -35,7 +35,7 @@ EXPORTED = [
     "gpt_rope_table", "gpt_attention_fwd", "gpt_attention_bwd", "gpt_attention_bwd_noalloc",
     "gpt_embedding_fwd",
     "gpt_attention_bwd_scratch_bytes", "gpt_embedding_bwd_scratch_bytes", "gpt_embedding_bwd", "gpt_lmhead_ce_scratch_bytes",
-    "gpt_lmhead_ce_fwd_bwd",
+    "gpt_lmhead_ce_fwd_bwd", "gpt_set_wait_limit", "gpt_debug_wait_probe", "gpt_debug_exp2_poly2",
 ]
 
 
@@ -97,6 +97,9 @@ def lib():
         L.gpt_lmhead_ce_scratch_bytes.argtypes = [i32, i32, i32]
         L.gpt_lmhead_ce_scratch_bytes.restype = sz
         L.gpt_lmhead_ce_fwd_bwd.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+        L.gpt_set_wait_limit.argtypes = [ll]
+        L.gpt_debug_wait_probe.argtypes = [vp, vp]
+        L.gpt_debug_exp2_poly2.argtypes = [vp, vp, i32, vp]
         _lib = L
     return _lib
 
@@ -309,6 +312,21 @@ def lmhead_ce_fwd_bwd(xf, wlm, targets, loss, lse, dx, dW, scratch, status=None)
     _check(lib().gpt_lmhead_ce_fwd_bwd(xf.data_ptr(), wlm.data_ptr(), targets.data_ptr(), M, d, V,
                                        loss.data_ptr(), lse.data_ptr(), dx.data_ptr(), dW.data_ptr(),
                                        scratch.data_ptr(), _ptr(status), _stream()), "lmhead_ce_fwd_bwd")
+
+
+def set_wait_limit(cycles: int):
+    """gpt_set_wait_limit: bound of every device-side wait on the current device (≤ 0: default)."""
+    _check(lib().gpt_set_wait_limit(int(cycles)), "set_wait_limit")
+
+
+def debug_wait_probe(status):
+    """gpt_debug_wait_probe: a wait that nothing completes; *status receives the timeout code."""
+    _check(lib().gpt_debug_wait_probe(status.data_ptr(), _stream()), "debug_wait_probe")
+
+
+def debug_exp2_poly2(x, y):
+    """gpt_debug_exp2_poly2: the attention forward's FMA-pipe 2^x on the fp32 array x."""
+    _check(lib().gpt_debug_exp2_poly2(x.data_ptr(), y.data_ptr(), x.numel(), _stream()), "debug_exp2_poly2")
 
 
 def flat_to_bf16_tensor(params_f32: np.ndarray, device="cuda"):

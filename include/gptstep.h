@@ -212,20 +212,23 @@ gpt_status gpt_attention_bwd(const void* q, const void* k, const void* v, const 
  * convenience, not part of the method.  Arguments and results are those of gpt_attention_bwd
  * without `delta`; the per-row scratch that the backward needs (40 bytes per row of
  * B·H·⌈T/64⌉·64) is kept in a static device array inside this library
- * (GPT_ATTN_BWD_NOALLOC_MAX_ROWS fp32 values = 8 MiB), which every GPU that loads the library holds
+ * (GPT_ATTN_BWD_NOALLOC_FLOATS fp32 values = 8 MiB), which every GPU that loads the library holds
  * until the process exits.  dSᵀ is not stored: the dQ kernel recomputes the scores instead.
  * It serves callers that cannot obtain device memory where they call the backward — for example
  * code running under a device-memory budget fixed at start-up, or inside a host framework whose own
  * allocator owns all device memory and allows no side allocations — and therefore cannot hand
  * gpt_attention_bwd its scratch buffer.  It calls no cudaMalloc, cudaFree or allocating routine.
- *   - 40·B·H·⌈T/64⌉·64 > 4·GPT_ATTN_BWD_NOALLOC_MAX_ROWS returns GPT_ERR_UNSUPPORTED_SHAPE;
- *     nothing is enqueued.
+ *   - The array holds GPT_ATTN_BWD_NOALLOC_FLOATS fp32 values; at 40 bytes (10 floats) per padded
+ *     row it serves B·H·⌈T/64⌉·64 ≤ GPT_ATTN_BWD_NOALLOC_MAX_ROWS rows (209,715; the largest
+ *     multiple of 64 below it, 209,664, is the largest accepted).  Larger shapes return
+ *     GPT_ERR_UNSUPPORTED_SHAPE before anything is enqueued or any CUDA call is made.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
  *     that device current); make that first call before any stream capture.
  *   - All calls share the one array.  Each call writes the rows it uses before reading them, so
  *     nothing needs clearing, but calls that overlap on the GPU (unordered streams, several host
  *     threads) race on it and give wrong results: order them on one stream. */
-#define GPT_ATTN_BWD_NOALLOC_MAX_ROWS (1ll << 21)
+#define GPT_ATTN_BWD_NOALLOC_FLOATS (1ll << 21)
+#define GPT_ATTN_BWD_NOALLOC_MAX_ROWS (GPT_ATTN_BWD_NOALLOC_FLOATS / 10)
 gpt_status gpt_attention_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                                      const void* dout, const float* lse, void* dq, void* dk,
                                      void* dv, int B, int H, int T, int Dh, int window,
@@ -254,6 +257,30 @@ size_t gpt_lmhead_ce_scratch_bytes(int M, int d, int V);
 gpt_status gpt_lmhead_ce_fwd_bwd(const void* xf, const void* wlm, const int32_t* targets, int M,
                                  int d, int V, float* loss, float* lse, float* dx, float* dW,
                                  void* scratch, int* status, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Diagnostics.  Not part of the method: they exist so that the failure handling of the kernels and
+ * the accuracy of one of their approximations can be tested on a GPU without faulting it.
+ * --------------------------------------------------------------------------------------------- */
+
+/* Every mbarrier wait inside the GEMM and attention kernels gives up after a limit (SM clock
+ * cycles, default 4e9 ≈ 2 s): it then records GPT_ERR_DEVICE_TIMEOUT in the call's status word,
+ * makes the CTA's other roles stop waiting, lets copies already in flight land, frees its tensor
+ * memory and returns; nothing traps.  This sets the limit for kernels launched afterwards on the
+ * CURRENT device (cycles ≤ 0 restores the default).  It is a blocking copy to device memory: call it
+ * between launches, not while kernels of this library run.  A small limit makes ordinary waits
+ * (a TMA load in flight) run out, which is how the tests exercise the timeout path. */
+gpt_status gpt_set_wait_limit(long long cycles);
+
+/* Launch one CTA that waits, with the bounded wait of the kernels above, on an mbarrier that
+ * nothing ever completes.  The wait runs out after the current limit and *status (device int)
+ * receives GPT_ERR_DEVICE_TIMEOUT; the kernel then returns and the context stays usable. */
+gpt_status gpt_debug_wait_probe(int* status, void* stream);
+
+/* y[i] = 2^x[i] computed as the attention forward computes a quarter of its softmax weights on the
+ * FMA pipe: x clamped to ≥ −126, x = n + f with n = round(x), 2^f by a fitted cubic on [−1/2, 1/2]
+ * (relative error ≤ 7.5e-5), n added to the exponent field.  x, y: device fp32 arrays of n. */
+gpt_status gpt_debug_exp2_poly2(const float* x, float* y, int n, void* stream);
 
 #ifdef __cplusplus
 }
