@@ -461,8 +461,15 @@ def run_kernel(args):
         A = torch.randn(a_shape, device=dev, generator=g).to(torch.bfloat16)
         B = torch.randn(b_shape, device=dev, generator=g).to(torch.bfloat16)
         C = torch.empty(M, N, device=dev, dtype=torch.float32 if op == 2 else torch.bfloat16)
-        epi = S.EPI_F32 if op == 2 else S.EPI_BF16
-        run = lambda: S.gemm(op, epi, A, B, C, M, N, K)  # noqa: E731
+        epi = {"auto": S.EPI_F32 if op == 2 else S.EPI_BF16, "bf16": S.EPI_BF16, "resid": S.EPI_RESID,
+               "relu2": S.EPI_RELU2, "drelu2": S.EPI_DRELU2, "f32": S.EPI_F32}[args.gemm_epi]
+        if epi in (S.EPI_F32,) and C.dtype != torch.float32:
+            C = torch.empty(M, N, device=dev, dtype=torch.float32)
+        if epi not in (S.EPI_F32,) and C.dtype != torch.bfloat16:
+            C = torch.zeros(M, N, device=dev, dtype=torch.bfloat16)
+        aux = torch.rand(M, N, device=dev, generator=g).to(torch.bfloat16) if epi == S.EPI_DRELU2 else None
+        scratch = None if args.no_stream_k else "auto"
+        run = lambda: S.gemm(op, epi, A, B, C, M, N, K, aux=aux, scratch=scratch)  # noqa: E731
         flops = 2.0 * M * N * K
         unit_desc = f"GEMM {args.gemm_op} M={M} N={N} K={K}"
     else:
@@ -523,6 +530,8 @@ def main():
                     help="time one kernel-level workload instead of the step")
     ap.add_argument("--gemm-shape", default="32768,6144,1536")
     ap.add_argument("--gemm-op", default="nt", choices=["nt", "nn", "tn"])
+    ap.add_argument("--gemm-epi", default="auto", choices=["auto", "bf16", "resid", "relu2", "drelu2", "f32"])
+    ap.add_argument("--no-stream-k", action="store_true", help="GEMM workload: every tile whole")
     ap.add_argument("--attn", default="2048,128,0", help="T,Dh,window (window 0 = full causal)")
     ap.add_argument("--attn-pass", default="fwd", choices=["fwd", "bwd"])
     ap.add_argument("--attn-rows", type=int, default=1 << 21, help="batch·heads·seq of the attention workload")

@@ -348,6 +348,16 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// Same, for a 3-d tensor map (the third coordinate selects the matrix of a batch).
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar) & PAIR_LEADER_MASK), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 // √x with the hardware approximation (x ≥ 0; relative error ~2^-22).
 __device__ __forceinline__ float sqrt_approx(float x) {
   float y;

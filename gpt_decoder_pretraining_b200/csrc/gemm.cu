@@ -16,7 +16,11 @@
 //               ReLU², dReLU², fp32 store / add, split-K reduction, QKV + RoPE + QK-norm, or the
 //               cross-entropy statistics / gradient of the fused lm-head), global store; then
 //               release the accumulator buffer to the leader.
-// Tiles (and K halves, for split-K) are distributed persistently over the CTA pairs.
+// Tiles are distributed persistently over the CTA pairs.  When the tile count leaves the last wave
+// partly empty, the tail tiles are split along K into equal ranges per pair ("stream-K"): every pair
+// then finishes at the same time, and a tile whose K range is split is summed from its pieces,
+// in ascending K order, by the piece that finishes last (no waiting, no atomics on the output,
+// bitwise reproducible).
 //
 // Operand majors: A and B may each be K-contiguous ("K-major") or M/N-contiguous ("MN-major"),
 // which covers y = x·Wᵀ (forward), dx = dy·W (activation gradient) and dW = dyᵀ·x (weight
@@ -39,7 +43,6 @@ constexpr int BK = 64;
 enum : int {
   EPI_CE_STATS = 100,
   EPI_CE_GRAD = 101,
-  EPI_F32_RED = 102,
   EPI_BF16_HEADS = 103,   // bf16 store with row m = b·T + t, column n = h·Dh + j sent to [B, H, T, Dh]
   EPI_QKV_ROPE = 200      // + Dh: RoPE + QK-norm of the q and k heads, all three to [3][B][H][T][Dh]
 };
@@ -52,10 +55,79 @@ constexpr int gemm_col_groups() { return EPI > EPI_QKV_ROPE ? 1 : 2; }
 template <int EPI>
 constexpr int gemm_threads() { return 64 + 128 * gemm_col_groups<EPI>(); }
 
+// Persistent schedule over the CTA pairs.  Output tiles 0 .. dp_tiles−1 are dealt round-robin and
+// computed whole; the sk_tiles after them are computed "stream-K": their sk_tiles·k_tiles K-steps,
+// in tile-major order, are cut into num_pairs contiguous ranges (sk_base steps each, one more for
+// the first sk_rem pairs), one per pair.  sk_smax is the most pieces any such tile is cut into.
+struct Sched {
+  int num_pairs, k_tiles;
+  int dp_tiles, sk_tiles;
+  long long sk_base;
+  int sk_rem;
+  int sk_smax;
+};
+
+__host__ __device__ inline long long sk_begin(const Sched& s, int p) {
+  return (long long)p * s.sk_base + (p < s.sk_rem ? p : s.sk_rem);
+}
+// The pair whose range holds stream-K step i.
+__host__ __device__ inline int sk_pair_of(const Sched& s, long long i) {
+  const long long cut = (long long)s.sk_rem * (s.sk_base + 1);
+  if (i < cut) return (int)(i / (s.sk_base + 1));
+  return s.sk_rem + (int)((i - cut) / s.sk_base);
+}
+
+// One unit of a pair's work: k-tiles [k0, k1) of output tile `tile`.
+struct Work {
+  int tile, k0, k1;
+};
+struct WorkIter {
+  int dp_next;
+  long long sk_i, sk_end;
+  __device__ WorkIter(const Sched& s, int p)
+      : dp_next(p), sk_i(sk_begin(s, p)), sk_end(sk_begin(s, p + 1)) {}
+  __device__ bool next(const Sched& s, Work& w) {
+    if (dp_next < s.dp_tiles) {
+      w.tile = dp_next;
+      w.k0 = 0;
+      w.k1 = s.k_tiles;
+      dp_next += s.num_pairs;
+      return true;
+    }
+    if (sk_i < sk_end) {
+      const long long t = sk_i / s.k_tiles;
+      const int k0 = (int)(sk_i - t * s.k_tiles);
+      const long long lim = k0 + (sk_end - sk_i);
+      const int k1 = lim < s.k_tiles ? (int)lim : s.k_tiles;
+      w.tile = s.dp_tiles + (int)t;
+      w.k0 = k0;
+      w.k1 = k1;
+      sk_i += k1 - k0;
+      return true;
+    }
+    return false;
+  }
+};
+
+// Stream-K piece exchange: each piece of a split tile writes its fp32 partial tile to its own slot
+// (256 × 256 floats, slot = tile·sk_smax + piece), then counts itself in one counter per epilogue
+// warp (32 rows × 128 columns: 16 per tile).
+constexpr int SK_WARPS_PER_TILE = 16;
+constexpr int SK_MAX_TILES = 320;
+constexpr int SK_MAX_SLOTS = 320;
+constexpr size_t SK_SLOT_FLOATS = 256 * 256;
+static_assert(GEMM_SK_COUNTER_BYTES == (size_t)SK_MAX_TILES * SK_WARPS_PER_TILE * sizeof(int),
+              "counter region size");
+
 struct GemmArgs {
   int M, N, K;
   int tiles_m, tiles_n, k_tiles;  // tiles_m counts 256-row pair tiles
-  int splits;                      // split-K factor (1 or 2)
+  Sched sched;
+  float* sk_part;                  // [sk_tiles·sk_smax][256][256] partial tiles
+  int* sk_cnt;                     // [sk_tiles·16] arrival counters, zero between launches
+  int batch;                       // independent matrices; tile t belongs to matrix t / (tiles_m·tiles_n)
+  long long c_bstride, aux_bstride;  // elements between consecutive matrices of C and aux
+  float alpha, beta;               // GPT_EPI_AXPBY
   void* C;
   int ldc;
   void* C2;
@@ -82,20 +154,50 @@ struct GemmShape {
 // ------------------------------------------------------------------------------------------------
 // epilogue: one thread owns row m, columns n0 .. n0+31 of the tile (32 fp32 values in v)
 // ------------------------------------------------------------------------------------------------
+// With use_pre, `pre` holds the 32 bf16 values of the residual (RESID) or of the saved activation
+// (DRELU2) at (m, n0 ..), loaded ahead of the accumulator; otherwise they are loaded here.
 template <int EPI>
-__device__ __forceinline__ void epilogue_store(const GemmArgs& a, int m, int n0, const float* v) {
+__device__ __forceinline__ void epilogue_store(const GemmArgs& a, int b, int m, int n0, const float* v,
+                                               bool use_pre, const uint4 (&pre)[4]) {
   const bool full = (n0 + 32 <= a.N);
-  if (EPI == EPI_F32_RED) {
-    // split-K: exactly two partial sums land on a zeroed output; fp32 addition is commutative,
-    // so 0 + a + b is the same whichever half arrives first
-    float* c = reinterpret_cast<float*>(a.C) + (size_t)m * a.ldc + n0;
+  if (EPI == GPT_EPI_AXPBY) {
+    // C = alpha·acc + beta·aux (bf16); aux is not read when beta = 0
+    uint16_t* c = reinterpret_cast<uint16_t*>(a.C) + b * a.c_bstride + (size_t)m * a.ldc + n0;
+    const uint16_t* x = a.aux + b * a.aux_bstride + (size_t)m * a.ldaux + n0;
+    const bool rd = a.beta != 0.f;
+    if (full) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (n0 + j < a.N) atomicAdd(c + j, v[j]);
+      for (int j = 0; j < 32; j += 8) {
+        float w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = a.alpha * v[j + e];
+        if (rd) {
+          const uint4 p = *reinterpret_cast<const uint4*>(x + j);
+          const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            w[2 * e] = fmaf(a.beta, bf_lo(pw[e]), w[2 * e]);
+            w[2 * e + 1] = fmaf(a.beta, bf_hi(pw[e]), w[2 * e + 1]);
+          }
+        }
+        uint4 o;
+        o.x = pack_bf2(w[0], w[1]); o.y = pack_bf2(w[2], w[3]);
+        o.z = pack_bf2(w[4], w[5]); o.w = pack_bf2(w[6], w[7]);
+        *reinterpret_cast<uint4*>(c + j) = o;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (n0 + j >= a.N) continue;
+        float w = a.alpha * v[j];
+        if (rd) w = fmaf(a.beta, bf2f(x[j]), w);
+        c[j] = f2bf(w);
+      }
+    }
     return;
   }
   if (EPI == GPT_EPI_F32 || EPI == GPT_EPI_F32_ADD) {
-    float* c = reinterpret_cast<float*>(a.C) + (size_t)m * a.ldc + n0;
+    float* c = reinterpret_cast<float*>(a.C) + b * a.c_bstride + (size_t)m * a.ldc + n0;
     if (full) {
 #pragma unroll
       for (int j = 0; j < 32; j += 4) {
@@ -113,11 +215,11 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, int m, int n0,
     }
     return;
   }
-  uint16_t* c = reinterpret_cast<uint16_t*>(a.C) + (size_t)m * a.ldc + n0;
+  uint16_t* c = reinterpret_cast<uint16_t*>(a.C) + b * a.c_bstride + (size_t)m * a.ldc + n0;
   if (EPI == GPT_EPI_BF16 || EPI == GPT_EPI_RESID || EPI == GPT_EPI_DRELU2) {
     const uint16_t* x = nullptr;
     if (EPI == GPT_EPI_RESID) x = c;
-    if (EPI == GPT_EPI_DRELU2) x = a.aux + (size_t)m * a.ldaux + n0;
+    if (EPI == GPT_EPI_DRELU2) x = a.aux + b * a.aux_bstride + (size_t)m * a.ldaux + n0;
     if (full) {
 #pragma unroll
       for (int j = 0; j < 32; j += 8) {
@@ -125,7 +227,7 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, int m, int n0,
 #pragma unroll
         for (int e = 0; e < 8; ++e) w[e] = v[j + e];
         if (EPI != GPT_EPI_BF16) {
-          uint4 p = *reinterpret_cast<const uint4*>(x + j);
+          const uint4 p = use_pre ? pre[j / 8] : *reinterpret_cast<const uint4*>(x + j);
           const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -176,6 +278,130 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, int m, int n0,
   }
 }
 
+template <int EPI>
+__device__ __forceinline__ void epilogue_store(const GemmArgs& a, int b, int m, int n0, const float* v) {
+  const uint4 none[4] = {};
+  epilogue_store<EPI>(a, b, m, n0, v, false, none);
+}
+
+// Epilogues that write each accumulator element on its own (bf16 cast, residual add, ReLU²,
+// dReLU², fp32 store / add): these are the ones whose tiles may be split stream-K.
+template <int EPI>
+constexpr bool epi_plain() {
+  return EPI == GPT_EPI_BF16 || EPI == GPT_EPI_RESID || EPI == GPT_EPI_RELU2 ||
+         EPI == GPT_EPI_DRELU2 || EPI == GPT_EPI_F32 || EPI == GPT_EPI_F32_ADD || EPI == GPT_EPI_AXPBY;
+}
+
+// One epilogue warp's share of a work unit: rows 32q .. 32q+31 of this CTA's 128, columns
+// 128·half .. +127 of the tile.  Waits for the accumulator (`tfull`), then either stores the tile
+// (a whole-K unit) or, for a stream-K piece, publishes its partial sums and — if it is the last
+// piece of the tile to arrive — adds all pieces in ascending K order and stores the sum.
+// Returns false if the wait gave up.
+template <int EPI>
+__device__ __forceinline__ bool plain_epilogue(const GemmArgs& a, const Work& w, int bb, int m, int tn,
+                                               uint32_t tm_addr, uint32_t rank, int q, int half,
+                                               int lane, uint64_t* tfull, uint32_t parity,
+                                               volatile int* abort_flag) {
+  constexpr int NC = BN / 32 / 2;  // 32-column chunks per thread
+  const Sched& sch = a.sched;
+  const bool piece = w.tile >= sch.dp_tiles && !(w.k0 == 0 && w.k1 == sch.k_tiles);
+  const int nbase = tn * BN + half * (BN / 2);
+  constexpr bool kPre = (EPI == GPT_EPI_RESID || EPI == GPT_EPI_DRELU2);
+  // The residual / saved activation does not depend on the accumulator: chunk 0 is fetched before
+  // the wait for the tile, and chunk c+1 before chunk c is read from tensor memory, so that one
+  // 64-byte row segment per thread is always in flight (within the epilogue warps' registers).
+  const bool pre_ok = kPre && !piece && m < a.M;
+  uint4 cur[4], nxt[4];
+  auto fetch = [&](int c, uint4 (&dst)[4]) {
+    const int n0 = nbase + 32 * c;
+    if (pre_ok && n0 + 32 <= a.N) {
+      const uint16_t* src = (EPI == GPT_EPI_RESID)
+                                ? reinterpret_cast<const uint16_t*>(a.C) + bb * a.c_bstride + (size_t)m * a.ldc + n0
+                                : a.aux + bb * a.aux_bstride + (size_t)m * a.ldaux + n0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) dst[e] = *reinterpret_cast<const uint4*>(src + 8 * e);
+    }
+  };
+  if (kPre) fetch(0, cur);
+  if (!mbar_wait_warp(tfull, parity, abort_flag, a.status)) return false;
+  tc_fence_after();
+  const uint32_t t0 = tm_addr + half * (BN / 2);
+  if (!piece) {
+#pragma unroll 1
+    for (int c = 0; c < NC; ++c) {
+      if (kPre && c + 1 < NC) fetch(c + 1, nxt);
+      uint32_t r[32];
+      tmem_ld32(t0 + 32 * c, r);
+      tmem_ld_wait();
+      const int n0 = nbase + 32 * c;
+      const bool use_pre = pre_ok && n0 + 32 <= a.N;
+      if (m < a.M && n0 < a.N)
+        epilogue_store<EPI>(a, bb, m, n0, reinterpret_cast<const float*>(r), use_pre, cur);
+      if (kPre) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cur[e] = nxt[e];
+      }
+    }
+    return true;
+  }
+  // ---- stream-K piece ----
+  const int st = w.tile - sch.dp_tiles;
+  const long long s0 = (long long)st * sch.k_tiles;
+  const int first = sk_pair_of(sch, s0);
+  const int nseg = sk_pair_of(sch, s0 + sch.k_tiles - 1) - first + 1;
+  const int seg = sk_pair_of(sch, s0 + w.k0) - first;
+  const size_t row_off = (size_t)(rank * BM + q * 32 + lane) * BN + half * (BN / 2);
+  float* mine = a.sk_part + (size_t)(st * sch.sk_smax + seg) * SK_SLOT_FLOATS + row_off;
+#pragma unroll 1
+  for (int c = 0; c < NC; ++c) {
+    uint32_t r[32];
+    tmem_ld32(t0 + 32 * c, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 32; j += 4)
+      *reinterpret_cast<uint4*>(mine + 32 * c + j) = make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+  }
+  __threadfence();
+  __syncwarp();
+  int* cnt = a.sk_cnt + st * SK_WARPS_PER_TILE + (int)rank * 8 + half * 4 + q;
+  int old = 0;
+  if (lane == 0) old = atomicAdd(cnt, 1);
+  old = __shfl_sync(0xffffffffu, old, 0);
+  if (old != nseg - 1) return true;
+  // last piece: every other piece's partial is visible; sum in ascending K (= slot) order
+  __threadfence();
+  const float* slot0 = a.sk_part + (size_t)st * sch.sk_smax * SK_SLOT_FLOATS + row_off;
+#pragma unroll 1
+  for (int c = 0; c < NC; ++c) {
+    uint32_t r[32];
+    tmem_ld32(t0 + 32 * c, r);
+    tmem_ld_wait();
+    float v[32];
+#pragma unroll 1
+    for (int sgi = 0; sgi < nseg; ++sgi) {
+      if (sgi == seg) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = (sgi == 0) ? __uint_as_float(r[j]) : v[j] + __uint_as_float(r[j]);
+      } else {
+        const float4* src = reinterpret_cast<const float4*>(slot0 + (size_t)sgi * SK_SLOT_FLOATS + 32 * c);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 p = __ldcg(src + j);
+          if (sgi == 0) {
+            v[4 * j] = p.x; v[4 * j + 1] = p.y; v[4 * j + 2] = p.z; v[4 * j + 3] = p.w;
+          } else {
+            v[4 * j] += p.x; v[4 * j + 1] += p.y; v[4 * j + 2] += p.z; v[4 * j + 3] += p.w;
+          }
+        }
+      }
+    }
+    const int n0 = nbase + 32 * c;
+    if (m < a.M && n0 < a.N) epilogue_store<EPI>(a, bb, m, n0, v);
+  }
+  if (lane == 0) atomicExch(cnt, 0);  // ready for the next launch
+  return true;
+}
+
 // ------------------------------------------------------------------------------------------------
 // the kernel
 // ------------------------------------------------------------------------------------------------
@@ -220,26 +446,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
-  const int mn_tiles = args.tiles_m * args.tiles_n;
-  const int num_units = mn_tiles * args.splits;
-  const int kt_per_split = (args.k_tiles + args.splits - 1) / args.splits;
-  auto unit_coords = [&](int u, int& tm, int& tn, int& kt0, int& kt1) {
-    const int ks = u / mn_tiles, r = u % mn_tiles;
-    tm = r / args.tiles_n;
-    tn = r % args.tiles_n;
-    kt0 = ks * kt_per_split;
-    kt1 = min(args.k_tiles, kt0 + kt_per_split);
-  };
+  const int pair = blockIdx.x >> 1;
+  const Sched& sch = args.sched;
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int u = pair; u < num_units; u += num_pairs) {
-        int tm, tn, kt0, kt1;
-        unit_coords(u, tm, tn, kt0, kt1);
+      WorkIter it(sch, pair);
+      Work w;
+      const int per_mat = args.tiles_m * args.tiles_n;
+      while (it.next(sch, w)) {
+        const int bb = w.tile / per_mat, tr = w.tile % per_mat;
+        const int tm = tr / args.tiles_n, tn = tr % args.tiles_n;
+        const int kt0 = w.k0, kt1 = w.k1;
         const int arow = tm * 2 * BM + rank * BM;        // this CTA's 128 rows of A
         const int brow = tn * BN + rank * (BN / 2);      // this CTA's 128 rows of B
         bool ok = true;
@@ -250,18 +471,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * S::STAGE_BYTES);
           const int k0 = kt * BK;
           if (!A_MN) {
-            tma_load_2d_pair(sa, &tmA, &full[stage], k0, arow);
+            tma_load_3d_pair(sa, &tmA, &full[stage], k0, arow, bb);
           } else {
 #pragma unroll
             for (int c = 0; c < BM / 64; ++c)
-              tma_load_2d_pair(sa + c * 8192, &tmA, &full[stage], arow + c * 64, k0);
+              tma_load_3d_pair(sa + c * 8192, &tmA, &full[stage], arow + c * 64, k0, bb);
           }
           if (!B_MN) {
-            tma_load_2d_pair(sb, &tmB, &full[stage], k0, brow);
+            tma_load_3d_pair(sb, &tmB, &full[stage], k0, brow, bb);
           } else {
 #pragma unroll
             for (int c = 0; c < (BN / 2) / 64; ++c)
-              tma_load_2d_pair(sb + c * 8192, &tmB, &full[stage], brow + c * 64, k0);
+              tma_load_3d_pair(sb + c * 8192, &tmB, &full[stage], brow + c * 64, k0, bb);
           }
           if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
         }
@@ -281,9 +502,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int u = pair; u < num_units; u += num_pairs) {
-        int tm, tn, kt0, kt1;
-        unit_coords(u, tm, tn, kt0, kt1);
+      WorkIter it(sch, pair);
+      Work w;
+      while (it.next(sch, w)) {
+        const int kt0 = w.k0, kt1 = w.k1;
         if (!mbar_wait_warp(&tempty[acc], acc_phase ^ 1, abort_flag, args.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
@@ -320,10 +542,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
     const int row_in_tile = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = pair; u < num_units; u += num_pairs) {
-      int tm, tn, kt0, kt1;
-      unit_coords(u, tm, tn, kt0, kt1);
+    WorkIter it(sch, pair);
+    Work w;
+    const int per_mat = args.tiles_m * args.tiles_n;
+    while (it.next(sch, w)) {
+      const int bb = w.tile / per_mat, tr = w.tile % per_mat;
+      const int tm = tr / args.tiles_n, tn = tr % args.tiles_n;
       const int m = tm * 2 * BM + rank * BM + row_in_tile;
+      if constexpr (epi_plain<EPI>()) {
+        if (!plain_epilogue<EPI>(args, w, bb, m, tn, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN,
+                                 rank, q, half, lane, &tfull[acc], acc_phase, abort_flag))
+          break;
+        tc_fence_before();
+        mbar_arrive_leader(&tempty[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+        continue;
+      }
       if (!mbar_wait_warp(&tfull[acc], acc_phase, abort_flag, args.status)) break;
       tc_fence_after();
       float run_max = -INFINITY, run_sum = 0.f;
@@ -425,7 +660,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
               const float p = __expf(v[j] - lse_m);
               v[j] = (p - ((n0 + j == tgt) ? 1.f : 0.f)) * scale;
             }
-            epilogue_store<GPT_EPI_BF16>(args, m, n0, v);
+            epilogue_store<GPT_EPI_BF16>(args, 0, m, n0, v);
           }
         } else if (EPI == EPI_BF16_HEADS) {
           if (m < args.M && n0 < args.N) {
@@ -443,7 +678,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
             }
           }
         } else {
-          if (m < args.M && n0 < args.N) epilogue_store<EPI>(args, m, n0, v);
+          if (m < args.M && n0 < args.N) epilogue_store<EPI>(args, 0, m, n0, v);
         }
       }
       }
@@ -479,11 +714,7 @@ static gpt_status launch_inst(const CUtensorMap& ma, const CUtensorMap& mb, cons
   using S = GemmShape;
   auto kern = gemm_kernel<A_MN, B_MN, EPI>;
   GPT_TRY(ensure_smem(kern, S::SMEM_BYTES));
-  int sms = 0;
-  GPT_TRY(device_info(&sms));
-  const int units = a.tiles_m * a.tiles_n * a.splits;
-  const int pairs = std::max(1, std::min(units, sms / 2));
-  kern<<<2 * pairs, gemm_threads<EPI>(), S::SMEM_BYTES, stream>>>(ma, mb, a);
+  kern<<<2 * a.sched.num_pairs, gemm_threads<EPI>(), S::SMEM_BYTES, stream>>>(ma, mb, a);
   count_launch();
   GPT_CUDA_TRY(cudaGetLastError());
   return GPT_OK;
@@ -499,18 +730,22 @@ static gpt_status dispatch_epi(int epi, const CUtensorMap& ma, const CUtensorMap
     case GPT_EPI_DRELU2: return launch_inst<A_MN, B_MN, GPT_EPI_DRELU2>(ma, mb, a, s);
     case GPT_EPI_F32: return launch_inst<A_MN, B_MN, GPT_EPI_F32>(ma, mb, a, s);
     case GPT_EPI_F32_ADD: return launch_inst<A_MN, B_MN, GPT_EPI_F32_ADD>(ma, mb, a, s);
-    case EPI_F32_RED: return launch_inst<A_MN, B_MN, EPI_F32_RED>(ma, mb, a, s);
+    case GPT_EPI_AXPBY: return launch_inst<A_MN, B_MN, GPT_EPI_AXPBY>(ma, mb, a, s);
     default: return GPT_ERR_INVALID_ARG;
   }
 }
 
-// Operand map for one CTA's half of a pair tile: K-major [rows, K] with box {64, 128};
-// MN-major [K rows, MN cols] with box {64, 64}.
+// Operand map for one CTA's half of a pair tile, over `batch` matrices `bstride` elements apart
+// (third map dimension): K-major [rows, K] with box {64, 128, 1}; MN-major [K rows, MN cols] with
+// box {64, 64, 1}.
 static bool make_operand_map(CUtensorMap* map, const void* base, bool mn_major, int mn, int K,
-                             int ld) {
-  uint64_t dims[2], strides[1];
-  uint32_t box[2];
+                             int ld, int batch = 1, long long bstride = 0) {
+  uint64_t dims[3], strides[2];
+  uint32_t box[3];
   strides[0] = (uint64_t)ld * 2;
+  const uint64_t outer = mn_major ? (uint64_t)K : (uint64_t)mn;
+  // a single matrix still gets a valid (unused) stride for the third dimension
+  strides[1] = batch > 1 ? (uint64_t)bstride * 2 : ((strides[0] * outer + 15) & ~(uint64_t)15);
   if (!mn_major) {
     dims[0] = (uint64_t)K; dims[1] = (uint64_t)mn;
     box[0] = 64; box[1] = 128;
@@ -518,7 +753,9 @@ static bool make_operand_map(CUtensorMap* map, const void* base, bool mn_major, 
     dims[0] = (uint64_t)mn; dims[1] = (uint64_t)K;
     box[0] = 64; box[1] = 64;
   }
-  return encode_map_bf16(map, base, 2, dims, strides, box, true);
+  dims[2] = (uint64_t)batch;
+  box[2] = 1;
+  return encode_map_bf16(map, base, 3, dims, strides, box, true);
 }
 
 static gpt_status check_gemm_args(int op, int M, int N, int K, const void* A, int lda, const void* B,
@@ -536,53 +773,124 @@ static gpt_status check_gemm_args(int op, int M, int N, int K, const void* A, in
   return GPT_OK;
 }
 
-static void fill_args(GemmArgs& a, int M, int N, int K, int splits) {
+// Tiles and the plain round-robin schedule (every tile whole, one CTA pair per tile up to the SM
+// count).
+static gpt_status fill_args(GemmArgs& a, int M, int N, int K, int batch = 1) {
+  int sms = 0;
+  GPT_TRY(device_info(&sms));
   a.M = M; a.N = N; a.K = K;
   a.tiles_m = (M + 2 * BM - 1) / (2 * BM);
   a.tiles_n = (N + BN - 1) / BN;
   a.k_tiles = (K + BK - 1) / BK;
-  a.splits = splits;
+  a.batch = batch;
+  a.alpha = 1.f;
+  a.beta = 0.f;
+  const long long tiles_ll = (long long)a.tiles_m * a.tiles_n * batch;
+  if (tiles_ll > (1ll << 30)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  const int tiles = (int)tiles_ll;
+  Sched& s = a.sched;
+  s = Sched{};
+  s.num_pairs = std::max(1, std::min(tiles, sms / 2));
+  s.k_tiles = a.k_tiles;
+  s.dp_tiles = tiles;
+  return GPT_OK;
 }
 
-gpt_status gemm_launch(int op, int epi, int M, int N, int K, const void* A, int lda, const void* B,
-                       int ldb, void* C, int ldc, void* C2, const void* aux, int ldaux, int* status,
-                       cudaStream_t stream) {
-  GPT_TRY(check_gemm_args(op, M, N, K, A, lda, B, ldb, C, ldc));
-  if (epi < GPT_EPI_BF16 || epi > GPT_EPI_F32_ADD) return GPT_ERR_INVALID_ARG;
-  if (epi == GPT_EPI_DRELU2 && (!aux || ldaux < N || (ldaux % 8))) return GPT_ERR_INVALID_ARG;
+// Stream-K plan for the tail of the tile list, or false when the round-robin schedule is as good.
+// Cost model, in k-step times of one CTA pair: round robin takes ⌈tiles/P⌉·k_tiles; stream-K takes
+// (dp waves)·k_tiles + ⌈sk steps/P⌉ plus the piece exchange, ≈ 8 k-steps per extra piece that the
+// last piece reads back (a 128 KB partial per CTA at its share of HBM bandwidth) + 4 for writing.
+bool plan_stream_k(int tiles, int k_tiles, int pairs, Sched* out) {
+  if (pairs < 2 || tiles <= 0 || k_tiles <= 0 || tiles % pairs == 0) return false;
+  const long long rr_cost = (long long)((tiles + pairs - 1) / pairs) * k_tiles;
+  const int sk_tiles = tiles < pairs ? tiles : tiles % pairs + pairs;
+  const int dp_tiles = tiles - sk_tiles;
+  Sched s{};
+  s.num_pairs = pairs;
+  s.k_tiles = k_tiles;
+  s.dp_tiles = dp_tiles;
+  s.sk_tiles = sk_tiles;
+  const long long total = (long long)sk_tiles * k_tiles;
+  s.sk_base = total / pairs;
+  s.sk_rem = (int)(total % pairs);
+  if (s.sk_base < 1) return false;
+  int smax = 1;
+  for (int t = 0; t < sk_tiles; ++t) {
+    const long long s0 = (long long)t * k_tiles;
+    smax = std::max(smax, sk_pair_of(s, s0 + k_tiles - 1) - sk_pair_of(s, s0) + 1);
+  }
+  s.sk_smax = smax;
+  if (sk_tiles > SK_MAX_TILES || (long long)sk_tiles * smax > SK_MAX_SLOTS) return false;
+  const long long sk_cost = (long long)(dp_tiles / pairs) * k_tiles + (total + pairs - 1) / pairs +
+                            8 * (smax - 1) + 4;
+  if (100 * sk_cost > 97 * rr_cost) return false;
+  *out = s;
+  return true;
+}
+
+size_t gemm_sk_scratch_bytes() {
+  return ((GEMM_SK_COUNTER_BYTES + 255) & ~(size_t)255) +
+         (size_t)SK_MAX_SLOTS * SK_SLOT_FLOATS * sizeof(float);
+}
+
+gpt_status gemm_launch_batched(const GemmBatch& g, cudaStream_t stream, void* sk_scratch) {
+  const int op = g.op, M = g.M, N = g.N, K = g.K;
+  int epi = g.epi;
+  GPT_TRY(check_gemm_args(op, M, N, K, g.A, g.lda, g.B, g.ldb, g.C, g.ldc));
+  if (epi < GPT_EPI_BF16 || epi > GPT_EPI_AXPBY) return GPT_ERR_INVALID_ARG;
+  if (epi == GPT_EPI_DRELU2 && (!g.aux || g.ldaux < N || (g.ldaux % 8))) return GPT_ERR_INVALID_ARG;
+  if (epi == GPT_EPI_AXPBY && g.beta != 0.f && (!g.aux || g.ldaux < N || (g.ldaux % 8) ||
+                                                (reinterpret_cast<uintptr_t>(g.aux) & 15)))
+    return GPT_ERR_INVALID_ARG;
+  if (g.batch < 1) return GPT_ERR_INVALID_ARG;
+  if (g.batch > 1) {
+    // matrices must not overlap and their starts must keep 16-byte alignment (TMA)
+    const long long a_rows = (op == GPT_GEMM_TN) ? K : M, b_rows = (op == GPT_GEMM_NT) ? N : K;
+    if (g.a_bstride < a_rows * g.lda || g.b_bstride < b_rows * g.ldb || g.c_bstride < (long long)M * g.ldc)
+      return GPT_ERR_INVALID_ARG;
+    if ((g.a_bstride % 8) || (g.b_bstride % 8) || (g.c_bstride % 8)) return GPT_ERR_UNSUPPORTED_SHAPE;
+    if (g.aux && ((g.aux_bstride % 8) || g.aux_bstride < (long long)M * g.ldaux)) return GPT_ERR_INVALID_ARG;
+  }
+  if (reinterpret_cast<uintptr_t>(sk_scratch) & 255) return GPT_ERR_UNSUPPORTED_SHAPE;
   const bool a_mn = (op == GPT_GEMM_TN);
   const bool b_mn = (op != GPT_GEMM_NT);
   CUtensorMap ma, mb;
-  if (!make_operand_map(&ma, A, a_mn, M, K, lda)) return GPT_ERR_UNSUPPORTED_SHAPE;
-  if (!make_operand_map(&mb, B, b_mn, N, K, ldb)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if (!make_operand_map(&ma, g.A, a_mn, M, K, g.lda, g.batch, g.a_bstride)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if (!make_operand_map(&mb, g.B, b_mn, N, K, g.ldb, g.batch, g.b_bstride)) return GPT_ERR_UNSUPPORTED_SHAPE;
   GemmArgs a{};
-  fill_args(a, M, N, K, 1);
-  a.C = C; a.ldc = ldc; a.C2 = C2;
-  a.aux = reinterpret_cast<const uint16_t*>(aux); a.ldaux = ldaux;
-  a.status = status;
-  // A plain fp32 store (weight gradients: few tiles, long K) is split into two K halves when that
-  // shortens the schedule (waves of CTA pairs × k-tiles per unit); the halves add onto a zeroed
-  // output.
-  int sms = 0;
-  GPT_TRY(device_info(&sms));
-  if (epi == GPT_EPI_F32 && a.k_tiles >= 8) {
-    const long long pairs = std::max(1, sms / 2), units = (long long)a.tiles_m * a.tiles_n;
-    const long long t1 = ((units + pairs - 1) / pairs) * a.k_tiles;
-    const long long t2 = ((2 * units + pairs - 1) / pairs) * ((a.k_tiles + 1) / 2);
-    if (t2 < t1) {
-      if (ldc == N) {
-        GPT_CUDA_TRY(cudaMemsetAsync(C, 0, (size_t)M * N * sizeof(float), stream));
-      } else {
-        GPT_CUDA_TRY(cudaMemset2DAsync(C, (size_t)ldc * sizeof(float), 0, (size_t)N * sizeof(float),
-                                       M, stream));
-      }
-      a.splits = 2;
-      epi = EPI_F32_RED;
+  GPT_TRY(fill_args(a, M, N, K, g.batch));
+  a.C = g.C; a.ldc = g.ldc; a.C2 = nullptr;
+  a.aux = reinterpret_cast<const uint16_t*>(g.aux); a.ldaux = g.ldaux;
+  a.c_bstride = g.batch > 1 ? g.c_bstride : 0;
+  a.aux_bstride = g.batch > 1 ? g.aux_bstride : 0;
+  a.alpha = g.alpha;
+  a.beta = g.beta;
+  a.status = g.status;
+  if (sk_scratch) {
+    int sms = 0;
+    GPT_TRY(device_info(&sms));
+    Sched sk;
+    if (plan_stream_k(a.tiles_m * a.tiles_n * g.batch, a.k_tiles, std::max(1, sms / 2), &sk)) {
+      a.sched = sk;
+      a.sk_cnt = reinterpret_cast<int*>(sk_scratch);
+      a.sk_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sk_scratch) +
+                                           ((GEMM_SK_COUNTER_BYTES + 255) & ~(size_t)255));
     }
   }
   if (op == GPT_GEMM_NT) return dispatch_epi<false, false>(epi, ma, mb, a, stream);
   if (op == GPT_GEMM_NN) return dispatch_epi<false, true>(epi, ma, mb, a, stream);
   return dispatch_epi<true, true>(epi, ma, mb, a, stream);
+}
+
+gpt_status gemm_launch(int op, int epi, int M, int N, int K, const void* A, int lda, const void* B,
+                       int ldb, void* C, int ldc, void* C2, const void* aux, int ldaux, int* status,
+                       cudaStream_t stream, void* sk_scratch) {
+  (void)C2;
+  GemmBatch g{};
+  g.op = op; g.epi = epi; g.M = M; g.N = N; g.K = K; g.batch = 1;
+  g.A = A; g.lda = lda; g.B = B; g.ldb = ldb; g.C = C; g.ldc = ldc;
+  g.aux = aux; g.ldaux = ldaux; g.alpha = 1.f; g.beta = 0.f; g.status = status;
+  return gemm_launch_batched(g, stream, sk_scratch);
 }
 
 gpt_status gemm_heads_launch(int op, int M, int N, int K, const void* A, int lda, const void* B,
@@ -595,7 +903,7 @@ gpt_status gemm_heads_launch(int op, int M, int N, int K, const void* A, int lda
   if (!make_operand_map(&ma, A, a_mn, M, K, lda)) return GPT_ERR_UNSUPPORTED_SHAPE;
   if (!make_operand_map(&mb, B, b_mn, N, K, ldb)) return GPT_ERR_UNSUPPORTED_SHAPE;
   GemmArgs a{};
-  fill_args(a, M, N, K, 1);
+  GPT_TRY(fill_args(a, M, N, K));
   a.C = heads; a.ldc = N; a.status = status;
   a.T = T; a.H = H; a.Dh = Dh;
   if (op == GPT_GEMM_NT) return launch_inst<false, false, EPI_BF16_HEADS>(ma, mb, a, stream);
@@ -614,7 +922,7 @@ gpt_status gemm_qkv_rope_launch(int M, int d, const void* A, const void* Wqkv, v
   if (!make_operand_map(&ma, A, false, M, K, K)) return GPT_ERR_UNSUPPORTED_SHAPE;
   if (!make_operand_map(&mb, Wqkv, false, N, K, K)) return GPT_ERR_UNSUPPORTED_SHAPE;
   GemmArgs a{};
-  fill_args(a, M, N, K, 1);
+  GPT_TRY(fill_args(a, M, N, K));
   a.C = heads; a.ldc = N; a.status = status;
   a.T = T; a.H = H; a.Dh = Dh; a.d = d; a.cs = cs; a.rho_q = rho_q; a.rho_k = rho_k;
   if (Dh == 128) return launch_inst<false, false, EPI_QKV_ROPE + 128>(ma, mb, a, stream);
@@ -632,7 +940,7 @@ gpt_status gemm_ce_launch(bool grad, int M, int N, int K, const void* A, int lda
   if (!make_operand_map(&ma, A, false, M, K, lda)) return GPT_ERR_UNSUPPORTED_SHAPE;
   if (!make_operand_map(&mb, B, false, N, K, ldb)) return GPT_ERR_UNSUPPORTED_SHAPE;
   GemmArgs a{};
-  fill_args(a, M, N, K, 1);
+  GPT_TRY(fill_args(a, M, N, K));
   a.C = C; a.ldc = ldc;
   a.status = status;
   a.ce = ce;
@@ -650,9 +958,35 @@ extern "C" gpt_status gpt_qkv_proj_rope(const void* r, const void* w_qkv, void* 
                                    status, gpt::as_stream(stream));
 }
 
+extern "C" size_t gpt_gemm_scratch_bytes(void) { return gpt::gemm_sk_scratch_bytes(); }
+
+extern "C" gpt_status gpt_gemm_batched(int op, int epilogue, int batch, int M, int N, int K,
+                                       const void* A, int lda, long long a_bstride, const void* B,
+                                       int ldb, long long b_bstride, void* C, int ldc,
+                                       long long c_bstride, const void* aux, int ldaux,
+                                       long long aux_bstride, float alpha, float beta,
+                                       int* status, void* stream) {
+  gpt::GemmBatch g{};
+  g.op = op; g.epi = epilogue; g.M = M; g.N = N; g.K = K; g.batch = batch;
+  g.A = A; g.lda = lda; g.a_bstride = a_bstride;
+  g.B = B; g.ldb = ldb; g.b_bstride = b_bstride;
+  g.C = C; g.ldc = ldc; g.c_bstride = c_bstride;
+  g.aux = aux; g.ldaux = ldaux; g.aux_bstride = aux_bstride;
+  g.alpha = alpha; g.beta = beta; g.status = status;
+  if (epilogue != GPT_EPI_AXPBY) { g.alpha = 1.f; g.beta = 0.f; }
+  return gpt::gemm_launch_batched(g, gpt::as_stream(stream), nullptr);
+}
+
 extern "C" gpt_status gpt_gemm(int op, int epilogue, int M, int N, int K, const void* A, int lda,
                                const void* B, int ldb, void* C, int ldc, void* C2,
-                               const void* aux, int ldaux, int* status, void* stream) {
-  return gpt::gemm_launch(op, epilogue, M, N, K, A, lda, B, ldb, C, ldc, C2, aux, ldaux, status,
-                          gpt::as_stream(stream));
+                               const void* aux, int ldaux, void* scratch, int* status,
+                               void* stream) {
+  cudaStream_t s = gpt::as_stream(stream);
+  if (scratch) {
+    // the arrival counters start at zero; every launch leaves them at zero again
+    if (reinterpret_cast<uintptr_t>(scratch) & 255) return GPT_ERR_UNSUPPORTED_SHAPE;
+    GPT_CUDA_TRY(cudaMemsetAsync(scratch, 0, gpt::GEMM_SK_COUNTER_BYTES, s));
+  }
+  return gpt::gemm_launch(op, epilogue, M, N, K, A, lda, B, ldb, C, ldc, C2, aux, ldaux, status, s,
+                          scratch);
 }

@@ -54,9 +54,26 @@ gpt_status wait_limit_set_attention(long long cycles);
 gpt_status wait_limit_set_diag(long long cycles);
 
 // Kernel-level launchers used by the step orchestrator (same semantics as the C entry points).
+// sk_scratch (may be null): gemm_sk_scratch_bytes() bytes, 256-byte aligned, whose leading
+// arrival counters are zero; with it, tiles of a partly empty last wave may be split along K.
 gpt_status gemm_launch(int op, int epi, int M, int N, int K, const void* A, int lda, const void* B,
                        int ldb, void* C, int ldc, void* C2, const void* aux, int ldaux, int* status,
-                       cudaStream_t stream);
+                       cudaStream_t stream, void* sk_scratch = nullptr);
+size_t gemm_sk_scratch_bytes();
+// A batch of independent GEMMs of one shape: matrix i of each operand starts `*_bstride` elements
+// after matrix i−1 (ignored for batch = 1).  GPT_EPI_AXPBY writes bf16(alpha·acc + beta·aux).
+struct GemmBatch {
+  int op, epi, M, N, K, batch;
+  const void* A; int lda; long long a_bstride;
+  const void* B; int ldb; long long b_bstride;
+  void* C; int ldc; long long c_bstride;
+  const void* aux; int ldaux; long long aux_bstride;
+  float alpha, beta;
+  int* status;
+};
+gpt_status gemm_launch_batched(const GemmBatch& g, cudaStream_t stream, void* sk_scratch);
+// Bytes at the start of the stream-K scratch holding the arrival counters (zeroed per step).
+constexpr size_t GEMM_SK_COUNTER_BYTES = 320 * 16 * sizeof(int);
 
 struct CeArgs {
   const int32_t* targets;

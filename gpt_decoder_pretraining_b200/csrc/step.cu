@@ -105,7 +105,7 @@ struct Plan {
   // CE
   size_t stats, zt, lse_ce, ell, inv_n, dz, dxf;
   // backward transients
-  size_t gx, gxb, du, dr, dO, dqkv, delta, emb;
+  size_t gx, gxb, du, dr, dO, dqkv, delta, emb, sk;
   size_t gacc;  // this micro-batch's gradients when the call accumulates into the caller's
   size_t total;
   int vc;  // vocabulary chunk of the backward lm-head
@@ -146,6 +146,12 @@ struct gpt_step {
   gpt::Plan plan;
   int64_t last_launches = 0;
   gpt::Profiler prof;
+  // gradient buckets (W_lm, layers depth−1 .. 0, wte) and the events recorded when each is final
+  std::vector<cudaEvent_t> grad_events;
+  bool record_in_step = true;  // false while a call accumulates: events follow the final add
+  ~gpt_step() {
+    for (cudaEvent_t e : grad_events) cudaEventDestroy(e);
+  }
 };
 
 namespace gpt {
@@ -200,6 +206,7 @@ static Plan make_plan(const gpt_config& c, size_t n_params) {
   p.dqkv = take(M * 3 * d * 2);
   p.delta = take(attention_bwd_scratch_bytes(c.batch, H, c.seq_len, true));
   p.emb = take(embedding_bwd_scratch_bytes((int)M, (int)d, (int)V));
+  p.sk = take(gemm_sk_scratch_bytes());
   p.gacc = take(n_params * 4);
   p.total = pos;
   return p;
@@ -252,6 +259,9 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
   int* status = reinterpret_cast<int*>(ws + p.status);
   float* rope = reinterpret_cast<float*>(ws + p.rope);
   GPT_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
+  // stream-K arrival counters of the GEMMs: zero here, and every GEMM leaves them at zero
+  void* sk = ws + p.sk;
+  GPT_CUDA_TRY(cudaMemsetAsync(sk, 0, GEMM_SK_COUNTER_BYTES, s));
   const uint16_t* P = reinterpret_cast<const uint16_t*>(params);
   if (c.param_dtype == GPT_DTYPE_F32) {
     PROF(PROF_CE, 0, 6.0 * L.total, cast_f32_bf16(reinterpret_cast<const float*>(params), ws + p.pshadow, L.total, s));
@@ -268,6 +278,12 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
   const long long hs_b = (long long)H * T * Dh, hs_h = (long long)T * Dh, hs_t = Dh;  // head-major
   const long long bhtd = (long long)B * H * T * Dh;
 
+  // bucket b of the gradient is final: b = 0 W_lm, 1 + (depth − 1 − l) layer l, depth + 1 wte
+  auto bucket_done = [&](int b) -> gpt_status {
+    if (!st->grad_events.empty() && st->record_in_step)
+      GPT_CUDA_TRY(cudaEventRecord(st->grad_events[b], s));
+    return GPT_OK;
+  };
   PROF(PROF_ROPE, 0, (double)T * Dh * 4, rope_table(rope, T, Dh, s));
   PROF(PROF_EMBED, 0, 4.0 * (double)M * d, embedding_fwd(tokens, W(0), x, M, d, V, status, s));
 
@@ -292,12 +308,12 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
          attention_fwd(qkv, qkv + bhtd, qkv + 2 * bhtd, o, lse, B, H, T, Dh, st->window[l], hs_b,
                        hs_h, hs_t, os_b, os_h, os_t, status, s, nullptr));
     PROF(PROF_GEMM, gemm_flops(M, d, d), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_RESID, M, d, d, o, d, W(wq + 1), d, x, d, nullptr,
-                        nullptr, 0, status, s));
+                        nullptr, 0, status, s, sk));
     PROF(PROF_NORM, 0, 4.0 * (double)M * d + 4.0 * M, rmsnorm_fwd(x, r2, rho2, M, d, s));
     PROF(PROF_GEMM, gemm_flops(M, F, d), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_RELU2, M, F, d, r2, d, W(wq + 2), d, hsq, F, nullptr,
-                        nullptr, 0, status, s));
+                        nullptr, 0, status, s, sk));
     PROF(PROF_GEMM, gemm_flops(M, d, F), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_RESID, M, d, F, hsq, F, W(wq + 3), F, x, d, nullptr,
-                        nullptr, 0, status, s));
+                        nullptr, 0, status, s, sk));
   }
   PROF(PROF_NORM, 0, 4.0 * (double)M * d + 4.0 * M, rmsnorm_fwd(x, xf, rhof, M, d, s));
 
@@ -325,12 +341,13 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
     ce.n_offset = c0;
     PROF(PROF_GEMM, gemm_flops(M, n, d), 0, gemm_ce_launch(true, M, n, d, xf, d, W(wlm) + (size_t)c0 * d, d, dz, n, ce, status, s));
     PROF(PROF_GEMM, gemm_flops(n, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, n, d, M, dz, n, xf, d, G(wlm) + (size_t)c0 * d, d,
-                        nullptr, nullptr, 0, status, s));
+                        nullptr, nullptr, 0, status, s, sk));
     PROF(PROF_GEMM, gemm_flops(M, d, n), 0, gemm_launch(GPT_GEMM_NN, c0 == 0 ? GPT_EPI_F32 : GPT_EPI_F32_ADD, M, d, n, dz, n,
-                        W(wlm) + (size_t)c0 * d, d, dxf, d, nullptr, nullptr, 0, status, s));
+                        W(wlm) + (size_t)c0 * d, d, dxf, d, nullptr, nullptr, 0, status, s, sk));
   }
   float* gx = reinterpret_cast<float*>(ws + p.gx);
   uint16_t* gxb = reinterpret_cast<uint16_t*>(ws + p.gxb);
+  GPT_TRY(bucket_done(0));
   PROF(PROF_NORM, 0, 12.0 * (double)M * d, rmsnorm_bwd(dxf, 1, xf, rhof, gx, gxb, 0, M, d, s));
 
   // ---------------- backward ----------------
@@ -353,19 +370,19 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
     uint16_t* hsq = reinterpret_cast<uint16_t*>(at(p.hsq, l));
     // MLP
     PROF(PROF_GEMM, gemm_flops(M, F, d), 0, gemm_launch(GPT_GEMM_NN, GPT_EPI_DRELU2, M, F, d, gxb, d, W(wq + 3), F, du, F, nullptr,
-                        hsq, F, status, s));
+                        hsq, F, status, s, sk));
     PROF(PROF_GEMM, gemm_flops(d, F, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, d, F, M, gxb, d, hsq, F, G(wq + 3), F, nullptr,
-                        nullptr, 0, status, s));
+                        nullptr, 0, status, s, sk));
     PROF(PROF_GEMM, gemm_flops(F, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, F, d, M, du, F, r2, d, G(wq + 2), d, nullptr,
-                        nullptr, 0, status, s));
+                        nullptr, 0, status, s, sk));
     PROF(PROF_GEMM, gemm_flops(M, d, F), 0, gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, F, du, F, W(wq + 2), d, dr, d, nullptr,
-                        nullptr, 0, status, s));
+                        nullptr, 0, status, s, sk));
     PROF(PROF_NORM, 0, 14.0 * (double)M * d, rmsnorm_bwd(dr, 0, r2, rho2, gx, gxb, 1, M, d, s));
     // attention
     PROF(PROF_GEMM, gemm_flops(M, d, d), 0,
          gemm_heads_launch(GPT_GEMM_NN, M, d, d, gxb, d, W(wq + 1), d, dO, T, H, Dh, status, s));
     PROF(PROF_GEMM, gemm_flops(d, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, d, d, M, gxb, d, o, d, G(wq + 1), d, nullptr,
-                        nullptr, 0, status, s));
+                        nullptr, 0, status, s, sk));
     PROF(PROF_ATTN_BWD, 8.0 * Dh * H * B * attn_pairs(T, st->window[l]), 0,
          attention_bwd(qkv, qkv + bhtd, qkv + 2 * bhtd, o, dO, lse, delta, dqkv, dqkv + d,
                        dqkv + 2 * d, B, H, T, Dh, st->window[l], hs_b, hs_h, hs_t, qs_b, qs_h,
@@ -376,12 +393,14 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
            rope_qknorm_bwd_heads(dqkv, qkv, rq, rk, rope, B, T, H, Dh, s));
     }
     PROF(PROF_GEMM, gemm_flops(3.0 * d, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, 3 * d, d, M, dqkv, 3 * d, r1, d, G(wq), d,
-                        nullptr, nullptr, 0, status, s));
+                        nullptr, nullptr, 0, status, s, sk));
+    GPT_TRY(bucket_done(1 + (c.depth - 1 - l)));
     PROF(PROF_GEMM, gemm_flops(M, d, 3.0 * d), 0, gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, 3 * d, dqkv, 3 * d, W(wq), d, dr, d,
-                        nullptr, nullptr, 0, status, s));
+                        nullptr, nullptr, 0, status, s, sk));
     PROF(PROF_NORM, 0, 14.0 * (double)M * d, rmsnorm_bwd(dr, 0, r1, rho1, gx, gxb, 1, M, d, s));
   }
   PROF(PROF_EMBED, 0, 4.0 * (double)M * d + 8.0 * V * d, embedding_bwd(tokens, gx, G(0), M, d, V, ws + p.emb, s));
+  GPT_TRY(bucket_done(c.depth + 1));
   return GPT_OK;
 }
 
@@ -422,6 +441,53 @@ gpt_status gpt_step_create(const gpt_config* cfg, gpt_step** out) {
 }
 
 void gpt_step_destroy(gpt_step* step) { delete step; }
+
+int gpt_step_grad_buckets(const gpt_step* step) { return step ? step->cfg.depth + 2 : -1; }
+
+gpt_status gpt_step_grad_bucket(const gpt_step* step, int i, size_t* begin, size_t* end) {
+  if (!step || !begin || !end) return GPT_ERR_INVALID_ARG;
+  const int L = step->cfg.depth;
+  if (i < 0 || i > L + 1) return GPT_ERR_INVALID_ARG;
+  const auto& off = step->layout.off;
+  const size_t vd = (size_t)step->cfg.vocab * step->cfg.d_model;
+  if (i == 0) {
+    *begin = off[1 + 4 * (size_t)L];
+    *end = *begin + vd;
+  } else if (i == L + 1) {
+    *begin = 0;
+    *end = vd;
+  } else {
+    const int l = L - i;  // bucket 1 is the last layer
+    *begin = off[1 + 4 * (size_t)l];
+    *end = off[1 + 4 * (size_t)l + 4];
+  }
+  return GPT_OK;
+}
+
+gpt_status gpt_step_enable_grad_events(gpt_step* step, int enable) {
+  if (!step) return GPT_ERR_INVALID_ARG;
+  for (cudaEvent_t e : step->grad_events) cudaEventDestroy(e);
+  step->grad_events.clear();
+  if (!enable) return GPT_OK;
+  int sms = 0;
+  GPT_TRY(gpt::device_info(&sms));
+  for (int i = 0; i < step->cfg.depth + 2; ++i) {
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      for (cudaEvent_t x : step->grad_events) cudaEventDestroy(x);
+      step->grad_events.clear();
+      return GPT_ERR_CUDA;
+    }
+    step->grad_events.push_back(e);
+  }
+  return GPT_OK;
+}
+
+gpt_status gpt_step_wait_grad_bucket(const gpt_step* step, int i, void* stream) {
+  if (!step || i < 0 || i >= (int)step->grad_events.size()) return GPT_ERR_INVALID_ARG;
+  GPT_CUDA_TRY(cudaStreamWaitEvent(gpt::as_stream(stream), step->grad_events[i], 0));
+  return GPT_OK;
+}
 
 gpt_status gpt_step_workspace_bytes(const gpt_step* step, size_t* bytes) {
   if (!step || !bytes) return GPT_ERR_INVALID_ARG;
@@ -484,9 +550,15 @@ gpt_status gpt_step_fwd_bwd(gpt_step* step, const void* params, const int32_t* t
   // accumulate = 1: the step's gradients go to workspace scratch and are then added to `grads`
   // element by element (one fp32 add per element, so the result does not depend on scheduling)
   float* g = accumulate ? reinterpret_cast<float*>(ws + step->plan.gacc) : grads;
+  step->record_in_step = !accumulate;
   gpt_status r = gpt::run_step(step, params, tokens, targets, loss, g, ws, gpt::as_stream(stream));
   if (r == GPT_OK && accumulate)
     r = gpt::add_f32(grads, g, step->layout.total, gpt::as_stream(stream));
+  if (r == GPT_OK && accumulate) {
+    for (cudaEvent_t e : step->grad_events)
+      if (cudaEventRecord(e, gpt::as_stream(stream)) != cudaSuccess) r = GPT_ERR_CUDA;
+  }
+  step->record_in_step = true;
   step->last_launches = gpt::g_launch_count - before;
   return r;
 }

@@ -30,13 +30,26 @@ EPI_BF16, EPI_RESID, EPI_RELU2, EPI_DRELU2, EPI_F32, EPI_F32_ADD = 0, 1, 2, 3, 4
 EXPORTED = [
     "gpt_param_layout", "gpt_step_create", "gpt_step_destroy", "gpt_step_workspace_bytes",
     "gpt_step_fwd_bwd", "gpt_step_status", "gpt_strerror", "gpt_step_last_launch_count",
-    "gpt_step_set_profiling", "gpt_step_profile",
-    "gpt_gemm", "gpt_qkv_proj_rope", "gpt_rmsnorm_fwd", "gpt_rmsnorm_bwd", "gpt_rope_qknorm_fwd", "gpt_rope_qknorm_bwd",
+    "gpt_step_set_profiling", "gpt_step_profile", "gpt_step_grad_buckets", "gpt_step_grad_bucket",
+    "gpt_step_enable_grad_events", "gpt_step_wait_grad_bucket",
+    "gpt_gemm", "gpt_gemm_scratch_bytes", "gpt_qkv_proj_rope", "gpt_rmsnorm_fwd", "gpt_rmsnorm_bwd", "gpt_rope_qknorm_fwd", "gpt_rope_qknorm_bwd",
     "gpt_rope_table", "gpt_attention_fwd", "gpt_attention_bwd", "gpt_attention_bwd_noalloc",
     "gpt_embedding_fwd",
     "gpt_attention_bwd_scratch_bytes", "gpt_embedding_bwd_scratch_bytes", "gpt_embedding_bwd", "gpt_lmhead_ce_scratch_bytes",
     "gpt_lmhead_ce_fwd_bwd", "gpt_set_wait_limit", "gpt_debug_wait_probe", "gpt_debug_exp2_poly2",
+    "gpt_gemm_batched", "gpt_adamw_step", "gpt_muon_scratch_bytes", "gpt_muon_step",
+    "gpt_optim_scratch_bytes", "gpt_optim_step",
 ]
+
+
+class OptimHparams(ctypes.Structure):
+    """gpt_optim_hparams: Muon and AdamW hyperparameters (every value is the caller's)."""
+    _fields_ = [("muon_lr", ctypes.c_float), ("muon_momentum", ctypes.c_float),
+                ("muon_nesterov", ctypes.c_int32), ("ns_steps", ctypes.c_int32),
+                ("ns_a", ctypes.c_float), ("ns_b", ctypes.c_float), ("ns_c", ctypes.c_float),
+                ("adam_lr_wte", ctypes.c_float), ("adam_lr_lm", ctypes.c_float),
+                ("beta1", ctypes.c_float), ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
+                ("weight_decay", ctypes.c_float)]
 
 
 class GptError(RuntimeError):
@@ -76,7 +89,13 @@ def lib():
         L.gpt_step_set_profiling.argtypes = [vp, i32]
         L.gpt_step_profile.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64),
                                        ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double), i32]
-        L.gpt_gemm.argtypes = [i32, i32, i32, i32, i32, vp, i32, vp, i32, vp, i32, vp, vp, i32, vp, vp]
+        L.gpt_step_grad_buckets.argtypes = [vp]
+        L.gpt_step_grad_bucket.argtypes = [vp, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+        L.gpt_step_enable_grad_events.argtypes = [vp, i32]
+        L.gpt_step_wait_grad_bucket.argtypes = [vp, i32, vp]
+        L.gpt_gemm.argtypes = [i32, i32, i32, i32, i32, vp, i32, vp, i32, vp, i32, vp, vp, i32, vp, vp, vp]
+        L.gpt_gemm_scratch_bytes.argtypes = []
+        L.gpt_gemm_scratch_bytes.restype = sz
         L.gpt_qkv_proj_rope.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp]
         L.gpt_rmsnorm_fwd.argtypes = [vp, vp, vp, i32, i32, vp]
         L.gpt_rmsnorm_bwd.argtypes = [vp, i32, vp, vp, vp, vp, i32, i32, i32, vp]
@@ -97,6 +116,18 @@ def lib():
         L.gpt_lmhead_ce_scratch_bytes.argtypes = [i32, i32, i32]
         L.gpt_lmhead_ce_scratch_bytes.restype = sz
         L.gpt_lmhead_ce_fwd_bwd.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+        f32 = ctypes.c_float
+        L.gpt_gemm_batched.argtypes = [i32, i32, i32, i32, i32, i32, vp, i32, ll, vp, i32, ll, vp, i32, ll,
+                                       vp, i32, ll, f32, f32, vp, vp]
+        L.gpt_adamw_step.argtypes = [vp, vp, i32, vp, vp, vp, ll, i32, f32, f32, f32, f32, f32, vp]
+        L.gpt_muon_scratch_bytes.argtypes = [i32, i32, i32]
+        L.gpt_muon_scratch_bytes.restype = sz
+        L.gpt_muon_step.argtypes = [vp, vp, i32, vp, vp, i32, i32, ll, i32, i32, f32, f32, i32, i32,
+                                    f32, f32, f32, vp, sz, vp, vp]
+        L.gpt_optim_scratch_bytes.argtypes = [ctypes.POINTER(_Config)]
+        L.gpt_optim_scratch_bytes.restype = sz
+        L.gpt_optim_step.argtypes = [ctypes.POINTER(_Config), vp, vp, vp, vp, vp, i32,
+                                     ctypes.POINTER(OptimHparams), vp, sz, vp, vp]
         L.gpt_set_wait_limit.argtypes = [ll]
         L.gpt_debug_wait_probe.argtypes = [vp, vp]
         L.gpt_debug_exp2_poly2.argtypes = [vp, vp, i32, vp]
@@ -178,6 +209,25 @@ class GptStep:
         _check(st, "gpt_step_fwd_bwd")
         return loss, grads
 
+    def grad_buckets(self):
+        """[(begin, end)] element ranges of the gradient buckets, in the order the backward pass
+        finishes them (W_lm, the layers from the last to the first, wte)."""
+        out = []
+        for i in range(int(lib().gpt_step_grad_buckets(self._h))):
+            b, e = ctypes.c_size_t(), ctypes.c_size_t()
+            _check(lib().gpt_step_grad_bucket(self._h, i, ctypes.byref(b), ctypes.byref(e)), "grad_bucket")
+            out.append((int(b.value), int(e.value)))
+        return out
+
+    def enable_grad_events(self, on: bool = True):
+        _check(lib().gpt_step_enable_grad_events(self._h, int(bool(on))), "enable_grad_events")
+
+    def wait_grad_bucket(self, i: int, stream=None):
+        """Make `stream` (default: the current stream) wait until bucket i of the last step is final."""
+        import torch
+        st = (stream or torch.cuda.current_stream()).cuda_stream
+        _check(lib().gpt_step_wait_grad_bucket(self._h, i, st), "wait_grad_bucket")
+
     def status(self) -> int:
         return int(lib().gpt_step_status(self._h, self.workspace.data_ptr(), _stream()))
 
@@ -201,15 +251,31 @@ class GptStep:
 # ------------------------------------------------------------------------------------------------
 # kernel-level calls (tensors in, tensors out); used by the unit parity tests and the benchmark
 # ------------------------------------------------------------------------------------------------
+_gemm_scratch = {}
+
+
+def gemm_scratch(device):
+    """A device buffer for gpt_gemm's stream-K scratch, one per device, kept for reuse."""
+    import torch
+    dev = torch.device(device)
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    if key not in _gemm_scratch:
+        _gemm_scratch[key] = torch.empty(int(lib().gpt_gemm_scratch_bytes()), dtype=torch.uint8, device=dev)
+    return _gemm_scratch[key]
+
+
 def gemm(op: int, epi: int, A, B, C, M: int, N: int, K: int, C2=None, aux=None, status=None,
-         lda=None, ldb=None, ldc=None):
-    """C (op) A·B as defined for gpt_gemm; row strides default to the tensors' last dimension."""
+         lda=None, ldb=None, ldc=None, scratch="auto"):
+    """C (op) A·B as defined for gpt_gemm; row strides default to the tensors' last dimension.
+    scratch: "auto" (a cached per-device buffer, so that stream-K may be used), None, or a tensor."""
     lda = lda or A.shape[-1]
     ldb = ldb or B.shape[-1]
     ldc = ldc or C.shape[-1]
     ldaux = aux.shape[-1] if aux is not None else 0
+    if isinstance(scratch, str):
+        scratch = gemm_scratch(C.device)
     _check(lib().gpt_gemm(op, epi, M, N, K, A.data_ptr(), lda, B.data_ptr(), ldb, C.data_ptr(), ldc,
-                          _ptr(C2), _ptr(aux), ldaux, _ptr(status), _stream()), "gpt_gemm")
+                          _ptr(C2), _ptr(aux), ldaux, _ptr(scratch), _ptr(status), _stream()), "gpt_gemm")
 
 
 def qkv_proj_rope(r, w_qkv, heads, rho_q, rho_k, cs, B, T, H, Dh, status=None):
@@ -312,6 +378,62 @@ def lmhead_ce_fwd_bwd(xf, wlm, targets, loss, lse, dx, dW, scratch, status=None)
     _check(lib().gpt_lmhead_ce_fwd_bwd(xf.data_ptr(), wlm.data_ptr(), targets.data_ptr(), M, d, V,
                                        loss.data_ptr(), lse.data_ptr(), dx.data_ptr(), dW.data_ptr(),
                                        scratch.data_ptr(), _ptr(status), _stream()), "lmhead_ce_fwd_bwd")
+
+
+def gemm_batched(op: int, epi: int, batch: int, M: int, N: int, K: int, A, lda, a_bstride, B, ldb, b_bstride,
+                 C, ldc, c_bstride, aux=None, ldaux=0, aux_bstride=0, alpha=1.0, beta=0.0, status=None):
+    """gpt_gemm_batched (strides in elements)."""
+    _check(lib().gpt_gemm_batched(op, epi, batch, M, N, K, A.data_ptr(), lda, a_bstride, B.data_ptr(), ldb,
+                                  b_bstride, C.data_ptr(), ldc, c_bstride, _ptr(aux), ldaux, aux_bstride,
+                                  float(alpha), float(beta), _ptr(status), _stream()), "gpt_gemm_batched")
+
+
+def adamw_step(master, params, grads, m, v, t: int, lr, beta1, beta2, eps, weight_decay, param_dtype=None):
+    """gpt_adamw_step over all elements of `master` (params may be None)."""
+    pdt = param_dtype if param_dtype is not None else (
+        DTYPE_F32 if params is None or str(params.dtype) == "torch.float32" else 0)
+    _check(lib().gpt_adamw_step(master.data_ptr(), _ptr(params), pdt, grads.data_ptr(), m.data_ptr(),
+                                v.data_ptr(), master.numel(), t, lr, beta1, beta2, eps, weight_decay,
+                                _stream()), "gpt_adamw_step")
+
+
+def muon_scratch_bytes(n: int, rows: int, cols: int) -> int:
+    return int(lib().gpt_muon_scratch_bytes(n, rows, cols))
+
+
+def muon_step(master, params, grads, buf, groups, per_group, group_stride, rows, cols, lr, momentum,
+              nesterov=True, ns_steps=5, ns=(3.4445, -4.7750, 2.0315), scratch=None, status=None):
+    """gpt_muon_step on a group of matrices laid out as in the flat parameter packing."""
+    import torch
+    pdt = DTYPE_F32 if params is None or str(params.dtype) == "torch.float32" else 0
+    need = muon_scratch_bytes(groups * per_group, rows, cols)
+    if scratch is None:
+        scratch = torch.empty(need, dtype=torch.uint8, device=master.device)
+    _check(lib().gpt_muon_step(master.data_ptr(), _ptr(params), pdt, grads.data_ptr(), buf.data_ptr(), groups,
+                               per_group, group_stride, rows, cols, lr, momentum, int(bool(nesterov)),
+                               ns_steps, ns[0], ns[1], ns[2], scratch.data_ptr(), scratch.numel(),
+                               _ptr(status), _stream()), "gpt_muon_step")
+
+
+def optim_scratch_bytes(cfg: GptConfig) -> int:
+    c, _keep = _cconfig(cfg)
+    return int(lib().gpt_optim_scratch_bytes(ctypes.byref(c)))
+
+
+def optim_step(cfg: GptConfig, master, params, grads, state_m, state_v, t: int, hp: dict, scratch=None,
+               status=None):
+    """gpt_optim_step: Muon + AdamW over the whole flat packing (hp keys as gpt_optim_hparams)."""
+    import torch
+    c, _keep = _cconfig(cfg)
+    h = OptimHparams(hp["muon_lr"], hp["muon_momentum"], int(hp.get("muon_nesterov", 1)), hp["ns_steps"],
+                     hp["ns_coeffs"][0], hp["ns_coeffs"][1], hp["ns_coeffs"][2], hp["adam_lr_wte"],
+                     hp["adam_lr_lm"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
+    need = optim_scratch_bytes(cfg)
+    if scratch is None:
+        scratch = torch.empty(max(need, 256), dtype=torch.uint8, device=master.device)
+    _check(lib().gpt_optim_step(ctypes.byref(c), master.data_ptr(), _ptr(params), grads.data_ptr(),
+                                state_m.data_ptr(), state_v.data_ptr(), t, ctypes.byref(h),
+                                scratch.data_ptr(), scratch.numel(), _ptr(status), _stream()), "gpt_optim_step")
 
 
 def set_wait_limit(cycles: int):

@@ -104,6 +104,21 @@ const char* gpt_strerror(int status);
 /* Number of kernel launches the last gpt_step_fwd_bwd enqueued (host counter, for reporting). */
 int64_t gpt_step_last_launch_count(const gpt_step* step);
 
+/* Gradient buckets, for a data-parallel exchange that overlaps the backward pass.  The gradient
+ * buffer splits into depth + 2 buckets in the order the backward pass finishes them: bucket 0 is
+ * W_lm, bucket 1 + (depth − 1 − l) is layer l's W_qkv, W_o, W_fc, W_proj (contiguous in the
+ * packing), bucket depth + 1 is wte.  gpt_step_grad_bucket gives bucket i's element range
+ * [*begin, *end) (host-only).  With events enabled (created on the current device, owned by the
+ * step), every gpt_step_fwd_bwd records one event per bucket on its stream as soon as that bucket
+ * is final (with accumulate = 1, after the final addition); gpt_step_wait_grad_bucket makes
+ * `stream` wait for bucket i of the last enqueued step, so that a collective on another stream
+ * can start on it while the rest of the backward pass runs (Introducing nanochat: the 8-GPU run;
+ * alpha-nanochat-d24, The run: the sharded optimizer exchanges gradients across ranks). */
+int gpt_step_grad_buckets(const gpt_step* step);
+gpt_status gpt_step_grad_bucket(const gpt_step* step, int i, size_t* begin, size_t* end);
+gpt_status gpt_step_enable_grad_events(gpt_step* step, int enable);
+gpt_status gpt_step_wait_grad_bucket(const gpt_step* step, int i, void* stream);
+
 /* Per-kernel-class timing.  While enabled, every launcher call of gpt_step_fwd_bwd is bracketed
  * by two CUDA events recorded on the step's stream.  gpt_step_profile waits for those events and
  * returns, for each class c < n_classes, the summed milliseconds, number of calls, algorithmic
@@ -135,15 +150,36 @@ gpt_status gpt_step_profile(gpt_step* step, double* ms, int64_t* calls, double* 
  *                                                       √aux = max(u,0): the ReLU² derivative)
  *   GPT_EPI_F32     C = acc                           (C fp32)
  *   GPT_EPI_F32_ADD C = C + acc                       (C fp32)
- * Sizes: M, N ≥ 1; K ≥ 1 (tails are zero-filled).  Pointers 16-byte aligned. */
+ *   GPT_EPI_AXPBY   C = bf16(alpha·acc + beta·aux)    (aux bf16, not read when beta = 0; only
+ *                                                       through gpt_gemm_batched)
+ * Sizes: M, N ≥ 1; K ≥ 1 (tails are zero-filled).  Pointers 16-byte aligned.
+ * scratch: NULL, or gpt_gemm_scratch_bytes() bytes of device memory (256-byte aligned) that the
+ * call may use to split the tiles of a partly empty last wave along K across all CTA pairs
+ * ("stream-K": each pair gets an equal share of the K-steps; the pieces of a split tile are summed
+ * in ascending K order by the piece that finishes last, so results are bitwise reproducible and no
+ * output is zeroed or updated atomically).  The call zeroes the scratch's counters on `stream`
+ * first; concurrent calls need separate scratch buffers.  With NULL every tile is computed whole. */
 enum { GPT_GEMM_NT = 0, GPT_GEMM_NN = 1, GPT_GEMM_TN = 2 };
 enum {
   GPT_EPI_BF16 = 0, GPT_EPI_RESID = 1, GPT_EPI_RELU2 = 2, GPT_EPI_DRELU2 = 3,
-  GPT_EPI_F32 = 4, GPT_EPI_F32_ADD = 5
+  GPT_EPI_F32 = 4, GPT_EPI_F32_ADD = 5, GPT_EPI_AXPBY = 6
 };
+size_t gpt_gemm_scratch_bytes(void);
 gpt_status gpt_gemm(int op, int epilogue, int M, int N, int K, const void* A, int lda,
                     const void* B, int ldb, void* C, int ldc, void* C2, const void* aux,
-                    int ldaux, int* status, void* stream);
+                    int ldaux, void* scratch, int* status, void* stream);
+
+/* `batch` independent GEMMs of one shape and op (as gpt_gemm): matrix i of A, B, C and aux starts
+ * i·*_bstride elements after matrix 0 (multiples of 8; the matrices must not overlap).  Any
+ * epilogue of gpt_gemm, plus GPT_EPI_AXPBY (alpha, beta are ignored by the others).  One launch
+ * covers the whole batch: output tiles of all matrices are dealt to the CTA pairs together.  Used
+ * by the Newton–Schulz iterations of Muon (gpt_muon_step), whose matrices come in groups of one
+ * shape. */
+gpt_status gpt_gemm_batched(int op, int epilogue, int batch, int M, int N, int K, const void* A,
+                            int lda, long long a_bstride, const void* B, int ldb,
+                            long long b_bstride, void* C, int ldc, long long c_bstride,
+                            const void* aux, int ldaux, long long aux_bstride, float alpha,
+                            float beta, int* status, void* stream);
 
 /* Fused QKV projection with RoPE + QK-norm, the step's forward entry into attention:
  * [q | k | v] = r·W_qkvᵀ (r bf16 [B·T, d], W_qkv bf16 [3d, d], d = H·Dh); each q and k head becomes
@@ -257,6 +293,60 @@ size_t gpt_lmhead_ce_scratch_bytes(int M, int d, int V);
 gpt_status gpt_lmhead_ce_fwd_bwd(const void* xf, const void* wlm, const int32_t* targets, int M,
                                  int d, int V, float* loss, float* lse, float* dx, float* dW,
                                  void* scratch, int* status, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * The optimizer step after the training step (Introducing nanochat, Pretraining log: the block
+ * matrices go to Muon, grouped by shape — q, k, v, the output projection, W_fc, W_proj — and the
+ * embedding and lm-head to AdamW, whose learning rates are scaled by 1/√(d/768)).  The pages print
+ * no hyperparameter values and no Muon internals: the published method is restated below and
+ * every value is an argument.  Weights are updated in an fp32 master copy; `params` (may be NULL
+ * or equal to the master) receives the new values in the step's parameter dtype (bf16 rounded to
+ * nearest even, or fp32).  Optimizer state buffers are fp32, caller-owned, zero before step 1.
+ * --------------------------------------------------------------------------------------------- */
+
+/* AdamW with decoupled weight decay over n elements (t ≥ 1 counts steps from 1):
+ *   m ← β1·m + (1−β1)·g;  v ← β2·v + (1−β2)·g²;  m̂ = m/(1−β1^t);  v̂ = v/(1−β2^t)
+ *   W ← W·(1 − lr·weight_decay) − lr·m̂/(√v̂ + eps)
+ * master, grads, m, v (and params) 16-byte aligned.  One fused elementwise kernel. */
+gpt_status gpt_adamw_step(float* master, void* params, int param_dtype, const float* grads,
+                          float* m, float* v, long long n, int t, float lr, float beta1,
+                          float beta2, float eps, float weight_decay, void* stream);
+
+/* Muon on a group of n = groups·per_group matrices of shape rows × cols: matrix i starts at
+ * element (i / per_group)·group_stride + (i % per_group)·rows·cols of master, grads and
+ * momentum_buf (the packing of the flat parameter buffer: per layer q, k, v, o are four contiguous
+ * d×d matrices, layers one stride apart).  Per matrix:
+ *   buf ← momentum·buf + g;  u = g + momentum·buf (nesterov ≠ 0) or buf;  X = u/(‖u‖_F + 1e-7)
+ *   ns_steps times: A = X·Xᵀ;  X ← ns_a·X + (ns_b·A + ns_c·A·A)·X  (tall matrices iterated as their
+ *   transpose; the published quintic is (3.4445, −4.7750, 2.0315) for 5 steps)
+ *   W ← W − lr·√max(1, rows/cols)·X
+ * The Newton–Schulz products are batched tcgen05 GEMMs over the group in bf16 with fp32
+ * accumulation (the precision the method is published with); ‖u‖ is summed in a fixed order.
+ * rows, cols multiples of 8.  scratch ≥ gpt_muon_scratch_bytes(n, rows, cols), 256-byte aligned. */
+size_t gpt_muon_scratch_bytes(int n_matrices, int rows, int cols);
+gpt_status gpt_muon_step(float* master, void* params, int param_dtype, const float* grads,
+                         float* momentum_buf, int groups, int per_group, long long group_stride,
+                         int rows, int cols, float lr, float momentum, int nesterov, int ns_steps,
+                         float ns_a, float ns_b, float ns_c, void* scratch, size_t scratch_bytes,
+                         int* status, void* stream);
+
+typedef struct gpt_optim_hparams {
+  float muon_lr, muon_momentum;
+  int32_t muon_nesterov, ns_steps;
+  float ns_a, ns_b, ns_c;
+  float adam_lr_wte, adam_lr_lm;  /* before the 1/√(d_model/768) scale */
+  float beta1, beta2, eps, weight_decay;
+} gpt_optim_hparams;
+
+/* The whole optimizer step over the flat packing of cfg: Muon on every layer's q, k, v, o (one
+ * group), W_fc (one group), W_proj (one group); AdamW on wte and W_lm with learning rates
+ * adam_lr_* · 1/√(d_model/768).  state_m holds Muon's momentum buffers and AdamW's first moments,
+ * state_v AdamW's second moments, both fp32 [n_params] in the same packing.  scratch ≥
+ * gpt_optim_scratch_bytes(cfg). */
+size_t gpt_optim_scratch_bytes(const gpt_config* cfg);
+gpt_status gpt_optim_step(const gpt_config* cfg, float* master, void* params, const float* grads,
+                          float* state_m, float* state_v, int t, const gpt_optim_hparams* hp,
+                          void* scratch, size_t scratch_bytes, int* status, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
  * Diagnostics.  Not part of the method: they exist so that the failure handling of the kernels and

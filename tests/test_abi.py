@@ -118,10 +118,10 @@ def test_step_argument_errors_need_no_device(lib):
 
 def test_kernel_entry_points_reject_bad_arguments(lib):
     f = 1 << 20
-    assert lib.gpt_gemm(0, 0, 0, 64, 64, f, 64, f, 64, f, 64, None, None, 0, None, None) == -1
-    assert lib.gpt_gemm(5, 0, 64, 64, 64, f, 64, f, 64, f, 64, None, None, 0, None, None) == -1
-    assert lib.gpt_gemm(0, 0, 64, 64, 64, f, 60, f, 64, f, 64, None, None, 0, None, None) == -1
-    assert lib.gpt_gemm(0, 0, 64, 64, 64, f + 2, 64, f, 64, f, 64, None, None, 0, None, None) == -2
+    assert lib.gpt_gemm(0, 0, 0, 64, 64, f, 64, f, 64, f, 64, None, None, 0, None, None, None) == -1
+    assert lib.gpt_gemm(5, 0, 64, 64, 64, f, 64, f, 64, f, 64, None, None, 0, None, None, None) == -1
+    assert lib.gpt_gemm(0, 0, 64, 64, 64, f, 60, f, 64, f, 64, None, None, 0, None, None, None) == -1
+    assert lib.gpt_gemm(0, 0, 64, 64, 64, f + 2, 64, f, 64, f, 64, None, None, 0, None, None, None) == -2
     assert lib.gpt_attention_fwd(f, f, f, f, f, None, 1, 1, 16, 48, 0, 48, 48, 48, 48, 48, 48, None, None) == -2
     assert lib.gpt_rmsnorm_fwd(None, f, f, 4, 64, None) == -1
     assert lib.gpt_embedding_bwd(f, f, f, 16, 64, 70000, f, None) == -2
@@ -159,14 +159,14 @@ def _rank_main(rank, world, port, q):
     q.put((rank, (ms, rate)))
 
 
-def test_data_parallel_average_equals_the_full_batch_step():
+def test_data_parallel_average_equals_the_full_batch_step(bucketed=False):
     """Two gloo ranks each take the oracle step on one row; bench.average_gradients over the ranks
     gives the oracle gradient of the two-row batch (equal valid counts per rank)."""
     import torch.multiprocessing as mp
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = 30500 + (os.getpid() % 1000)
-    procs = [ctx.Process(target=_dp_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    port = 30500 + (os.getpid() % 1000) + (500 if bucketed else 0)
+    procs = [ctx.Process(target=_dp_rank_main, args=(r, 2, port, q, bucketed)) for r in range(2)]
     for p in procs:
         p.start()
     out = dict(q.get(timeout=180) for _ in procs)
@@ -184,7 +184,7 @@ def test_data_parallel_average_equals_the_full_batch_step():
         np.testing.assert_allclose(out[r], full["grads"], rtol=0, atol=1e-12)
 
 
-def _dp_rank_main(rank, world, port, q):
+def _dp_rank_main(rank, world, port, q, bucketed=False):
     import sys
     sys.path.insert(0, ROOT)
     import datetime
@@ -200,9 +200,52 @@ def _dp_rank_main(rank, world, port, q):
     params = make_params(cfg1.n_params, keep_fp32=True, std=0.3).astype(np.float64)
     tok, tgt = make_tokens(2, 12, 64, seed=1)
     g = torch.from_numpy(O.step(cfg1, params, tok[rank:rank + 1], tgt[rank:rank + 1])["grads"])
-    bench.average_gradients(g, world)
+    if bucketed:
+        from gpt_decoder_pretraining_b200 import dp
+        buckets = dp.grad_buckets(cfg1)
+        order = []
+        dp.average_in_buckets(g, buckets, world, wait=order.append)
+        assert order == list(range(len(buckets)))
+    else:
+        bench.average_gradients(g, world)
     dist.destroy_process_group()
     q.put((rank, g.numpy()))
+
+
+def _host_buckets(cfg):
+    """Gradient buckets as the library defines them (host-only calls, no device)."""
+    lib = S.lib()
+    st, h, _keep = _create(lib, cfg)
+    assert st == 0
+    n = lib.gpt_step_grad_buckets(h)
+    out = []
+    for i in range(n):
+        b, e = ctypes.c_size_t(), ctypes.c_size_t()
+        assert lib.gpt_step_grad_bucket(h, i, ctypes.byref(b), ctypes.byref(e)) == 0
+        out.append((b.value, e.value))
+    lib.gpt_step_destroy(h)
+    return out
+
+
+@pytest.mark.parametrize("name", ["smoke", "d20"])
+def test_gradient_buckets_tile_the_packing_in_backward_order(lib, name):
+    from gpt_decoder_pretraining_b200 import dp
+    cfg = C.preset(name)
+    b = _host_buckets(cfg)
+    assert b == dp.grad_buckets(cfg)
+    offs, total = S.param_layout(cfg)
+    assert len(b) == cfg.depth + 2
+    assert b[0] == (offs[-1], total)                       # W_lm first
+    assert b[-1] == (0, cfg.vocab * cfg.d_model)           # wte last
+    for i in range(1, cfg.depth + 1):                      # layers from the last to the first
+        l = cfg.depth - i
+        assert b[i] == (offs[1 + 4 * l], offs[1 + 4 * l + 4] if l + 1 < cfg.depth else offs[-1])
+    assert sum(e - s for s, e in b) == total and len({s for s, _ in b}) == len(b)
+
+
+def test_bucketed_data_parallel_average_equals_the_full_batch_step():
+    """The per-bucket exchange (the order and ranges the library reports) gives the same average."""
+    test_data_parallel_average_equals_the_full_batch_step(bucketed=True)
 
 
 def test_attention_backward_scratch_size(lib):

@@ -86,6 +86,56 @@ def test_gemm_epilogues(M, N, K):
     assert_close_rel(to_np(Cf), base + acc, rel=1e-5, cos=0.9999999, what="f32 add")
 
 
+# Shapes whose tile count leaves the last wave of CTA pairs partly empty, so that the GEMM splits
+# the tail tiles along K (stream-K): fewer tiles than CTA pairs (every tile in pieces, up to four
+# per tile), a weight-gradient shape of 100 tiles, and 84 ragged tiles.
+SK_SHAPES = [(1536, 1536, 16384, 2), (1280, 5120, 8192, 2), (3000, 1700, 2560, 0), (3000, 1700, 2560, 1)]
+
+
+@pytest.mark.parametrize("M,N,K,op", SK_SHAPES)
+def test_gemm_stream_k_tail_matches_fp64_and_is_reproducible(M, N, K, op):
+    rng = np.random.default_rng(M + N + K + op)
+    A = randn(rng, *((K, M) if op == 2 else (M, K)))
+    B = randn(rng, *((N, K) if op == 0 else (K, N)))
+    ref = (A.T if op == 2 else A) @ (B.T if op == 0 else B)
+    tA, tB = bf16_tensor(A), bf16_tensor(B)
+    st = _status()
+    C1 = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    C2 = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    S.gemm(op, S.EPI_F32, tA, tB, C1, M, N, K, status=st)
+    S.gemm(op, S.EPI_F32, tA, tB, C2, M, N, K, status=st)
+    Cn = torch.zeros(M, N, dtype=torch.float32, device="cuda")
+    S.gemm(op, S.EPI_F32, tA, tB, Cn, M, N, K, status=st, scratch=None)  # every tile whole
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert_close_rel(to_np(C1), ref, rel=1e-5, cos=0.9999999, what="f32 stream-K")
+    assert torch.equal(C1, C2)  # bitwise reproducible
+    assert_close_rel(to_np(C1), to_np(Cn), rel=1e-5, cos=0.9999999, what="stream-K vs whole tiles")
+    if op == 2:
+        return
+    # the element-wise epilogues on the same split schedule
+    acc = ref
+    X = randn(rng, M, N, scale=3.0)
+    tX = bf16_tensor(X)
+    S.gemm(op, S.EPI_RESID, tA, tB, tX, M, N, K, status=st)
+    taux = bf16_tensor(np.maximum(randn(rng, M, N), 0) ** 2)
+    aux = to_np(taux)
+    Cd = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+    S.gemm(op, S.EPI_DRELU2, tA, tB, Cd, M, N, K, aux=taux, status=st)
+    Ch = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+    S.gemm(op, S.EPI_RELU2, tA, tB, Ch, M, N, K, status=st)
+    base = rng.standard_normal((M, N)).astype(np.float32)
+    Cf = torch.from_numpy(base).cuda()
+    S.gemm(op, S.EPI_F32_ADD, tA, tB, Cf, M, N, K, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert_close_rel(to_np(tX), X + acc, rel=8e-3, what="resid")
+    assert_close_rel(to_np(Cd), acc * 2 * np.sqrt(aux), rel=8e-3, what="drelu2")
+    r = np.maximum(acc, 0)
+    assert_close_rel(to_np(Ch), r * r, rel=8e-3, what="relu2")
+    assert_close_rel(to_np(Cf), base + acc, rel=1e-5, cos=0.9999999, what="f32 add")
+
+
 def test_gemm_rejects_bad_arguments():
     t = torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(S.GptError):
