@@ -342,6 +342,58 @@ def measure_step(args, cfg, dev, world, rank, barrier, exchange, with_e2e=True):
     return out
 
 
+def muon_ns_flops(cfg, steps=5):
+    """Newton–Schulz FLOPs of one Muon step over the model: per matrix (r ≤ c after transposing)
+    and iteration X·Xᵀ (2r²c), A·A (2r³) and B·X (2r²c)."""
+    def one(rows, cols):
+        r, c = min(rows, cols), max(rows, cols)
+        return steps * (4.0 * r * r * c + 2.0 * r ** 3)
+    d, F = cfg.d_model, cfg.d_mlp
+    return cfg.depth * (4 * one(d, d) + one(F, d) + one(d, F))
+
+
+OPTIM_HP = {"muon_lr": 0.02, "muon_momentum": 0.95, "muon_nesterov": 1, "ns_steps": 5,
+            "ns_coeffs": (3.4445, -4.7750, 2.0315), "adam_lr_wte": 0.2, "adam_lr_lm": 0.004,
+            "beta1": 0.8, "beta2": 0.95, "eps": 1e-10, "weight_decay": 0.0}
+
+
+def measure_optimizer(args, cfg, dev, params_np):
+    """Time gpt_optim_step (Muon on the block matrices, AdamW on wte / W_lm) over the whole model,
+    on fp32 master weights, fp32 gradients and optimizer state resident in HBM."""
+    import torch
+    from gpt_decoder_pretraining_b200 import step as S
+    n = cfg.n_params
+    master = torch.from_numpy(params_np.astype(np.float32)).to(dev)
+    params = master.to(torch.bfloat16)
+    g = torch.Generator(device=dev)
+    g.manual_seed(3)
+    grads = torch.randn(n, device=dev, generator=g) * 1e-3
+    sm, sv = torch.zeros(n, device=dev), torch.zeros(n, device=dev)
+    scratch = torch.empty(max(256, S.optim_scratch_bytes(cfg)), dtype=torch.uint8, device=dev)
+    t = 1
+    for _ in range(2):
+        S.optim_step(cfg, master, params, grads, sm, sv, t, OPTIM_HP, scratch=scratch)
+        t += 1
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    k = max(1, min(args.steps, 5))
+    e0.record()
+    for _ in range(k):
+        S.optim_step(cfg, master, params, grads, sm, sv, t, OPTIM_HP, scratch=scratch)
+        t += 1
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / k
+    adam_elems = 2 * cfg.vocab * cfg.d_model
+    out = {"ms_per_step": ms, "steps": k,
+           "what": "Muon (momentum, 5 Newton-Schulz steps in batched bf16 tcgen05 GEMMs, update) on every "
+                   "block matrix + fused AdamW on wte and W_lm, fp32 master weights and state",
+           "muon_ns_flops": muon_ns_flops(cfg), "adamw_bytes": 30.0 * adam_elems}
+    del master, params, grads, sm, sv, scratch
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, cfg):
     import torch
     import torch.distributed as dist
@@ -406,6 +458,8 @@ def run_ours(args, cfg):
         "kernels": r["kernels"],
         "clocks": r["clocks"],
     }
+    if world == 1 and not args.no_optim:
+        line["optimizer"] = measure_optimizer(args, cfg, torch.device("cuda", local), r["params_np"])
     # the other configuration the ≥ 45% MFU target names, measured in the same run
     if world == 1 and not args.no_also and cfg.name != args.also:
         import dataclasses
@@ -472,6 +526,37 @@ def run_kernel(args):
         run = lambda: S.gemm(op, epi, A, B, C, M, N, K, aux=aux, scratch=scratch)  # noqa: E731
         flops = 2.0 * M * N * K
         unit_desc = f"GEMM {args.gemm_op} M={M} N={N} K={K}"
+    elif args.kernel == "rmsnorm":
+        # RMSNorm forward and backward (bf16 dy, fp32 accumulate + bf16 copy) on [rows, d]
+        rows, d = (int(x) for x in args.rows_d.split(","))
+        x = torch.randn(rows, d, device=dev, generator=g).to(torch.bfloat16)
+        y = torch.empty_like(x)
+        rho = torch.empty(rows, device=dev)
+        dy = torch.randn(rows, d, device=dev, generator=g).to(torch.bfloat16)
+        gx = torch.zeros(rows, d, device=dev)
+        gxb = torch.empty_like(x)
+        if args.norm_pass == "fwd":
+            run = lambda: S.rmsnorm_fwd(x, y, rho)  # noqa: E731
+            nbytes = 4.0 * rows * d + 4.0 * rows
+        else:
+            S.rmsnorm_fwd(x, y, rho)
+            run = lambda: S.rmsnorm_bwd(dy, y, rho, gx, gxb, accumulate=True)  # noqa: E731
+            nbytes = 14.0 * rows * d + 4.0 * rows
+        flops = None
+        unit_desc = f"RMSNorm {args.norm_pass} rows={rows} d={d}"
+    elif args.kernel == "embedding":
+        # embedding backward (sort, fixed-order pieces, fix-up) on Zipf(1.1) ids
+        from gpt_decoder_pretraining_b200.inputs import make_tokens as mk
+        M, d, V = (int(x) for x in args.emb.split(","))
+        tok_np, _ = mk(1, M, V, "zipf1.1")
+        tok = torch.from_numpy(tok_np.reshape(-1)).to(dev)
+        gx = torch.randn(M, d, device=dev, generator=g)
+        dw = torch.empty(V, d, device=dev)
+        scr = torch.empty(S.embedding_bwd_scratch_bytes(M, d, V), dtype=torch.uint8, device=dev)
+        run = lambda: S.embedding_bwd(tok, gx, dw, scr)  # noqa: E731
+        nbytes = 4.0 * M * d + 4.0 * V * d
+        flops = None
+        unit_desc = f"embedding bwd M={M} d={d} V={V} (Zipf ids)"
     else:
         T, Dh, W = (int(x) for x in args.attn.split(","))
         H = args.attn_heads
@@ -504,6 +589,13 @@ def run_kernel(args):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
+    if flops is None:
+        gbs = nbytes / (ms / 1e3) / 1e9
+        peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        print(json.dumps({"kernel": unit_desc, "ms": ms, "gbs": gbs, "algorithmic_bytes": nbytes,
+                          "peak_hbm_gbs": peak, "frac_of_hbm": gbs / peak, "peak_source": src,
+                          "steps": args.steps}), flush=True)
+        return 0
     tf = flops / (ms / 1e3) / 1e12
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     print(json.dumps({"kernel": unit_desc, "ms": ms, "tflops": tf, "peak_burst_tflops": peak,
@@ -526,7 +618,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--also", default="d20", help="second configuration measured in the same run")
     ap.add_argument("--no-also", action="store_true")
-    ap.add_argument("--kernel", choices=["gemm", "attention"], default=None,
+    ap.add_argument("--no-optim", action="store_true", help="skip the optimizer-step measurement")
+    ap.add_argument("--rows-d", default="65536,1536", help="rmsnorm workload: rows,d")
+    ap.add_argument("--norm-pass", default="fwd", choices=["fwd", "bwd"])
+    ap.add_argument("--emb", default="32768,1536,32768", help="embedding workload: M,d,V")
+    ap.add_argument("--kernel", choices=["gemm", "attention", "rmsnorm", "embedding"], default=None,
                     help="time one kernel-level workload instead of the step")
     ap.add_argument("--gemm-shape", default="32768,6144,1536")
     ap.add_argument("--gemm-op", default="nt", choices=["nt", "nn", "tn"])

@@ -58,6 +58,7 @@ class GptConfig:
     windows: List[int] = field(default_factory=list)  # per layer; 0 or >= seq_len = full causal
     param_dtype: int = DTYPE_BF16
     token_dist: str = "uniform"  # "uniform" or "zipf1.1"
+    n_kv_heads: int = 0  # key/value heads of grouped-query attention; 0 = n_heads
 
     def __post_init__(self):
         if not self.windows:
@@ -66,6 +67,12 @@ class GptConfig:
             raise ValueError("windows must have one entry per layer")
         if self.n_heads * self.head_dim != self.d_model:
             raise ValueError("n_heads * head_dim must equal d_model")
+        if self.n_kv_heads and (self.n_kv_heads < 0 or self.n_heads % self.n_kv_heads):
+            raise ValueError("n_heads must be a multiple of n_kv_heads")
+
+    @property
+    def kv_heads(self) -> int:
+        return self.n_kv_heads if self.n_kv_heads > 0 else self.n_heads
 
     # ---- shapes ---------------------------------------------------------------------------
     @property
@@ -80,9 +87,10 @@ class GptConfig:
         """(name, shape) in packing order: wte, per layer qkv/o/fc/proj, lm_head."""
         d, F, V = self.d_model, self.d_mlp, self.vocab
         shapes = [("wte", (V, d))]
+        qkv = d + 2 * self.kv_heads * self.head_dim
         for l in range(self.depth):
             shapes += [
-                (f"h{l}.w_qkv", (3 * d, d)),
+                (f"h{l}.w_qkv", (qkv, d)),
                 (f"h{l}.w_o", (d, d)),
                 (f"h{l}.w_fc", (F, d)),
                 (f"h{l}.w_proj", (d, F)),
@@ -147,8 +155,9 @@ PRESETS = ("smoke", "d12", "d20", "d24")
 
 def custom(depth: int, d_model: int, head_dim: int, vocab: int, seq_len: int, batch: int,
            windows: Optional[Sequence[int]] = None, d_mlp: Optional[int] = None,
-           param_dtype: int = DTYPE_BF16, token_dist: str = "uniform", name: str = "custom") -> GptConfig:
+           param_dtype: int = DTYPE_BF16, token_dist: str = "uniform", name: str = "custom",
+           n_kv_heads: int = 0) -> GptConfig:
     """A config with nanochat's proportions (F = 4d) unless d_mlp is given."""
     return GptConfig(name, depth, d_model, d_model // head_dim, head_dim, d_mlp or 4 * d_model, vocab,
                      seq_len, batch, list(windows) if windows is not None else [0] * depth,
-                     param_dtype, token_dist)
+                     param_dtype, token_dist, n_kv_heads)

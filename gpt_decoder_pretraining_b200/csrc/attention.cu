@@ -122,6 +122,8 @@ template <int DH>
 __global__ void __launch_bounds__(256)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                     const __grid_constant__ CUtensorMap mv, const AttnArgs a) {
+  pdl_wait();
+  pdl_trigger();
   using S = FwdShape<DH>;
   constexpr int BMQ = S::BMQ, BNK = S::BNK;
   extern __shared__ uint8_t smem_raw[];
@@ -390,6 +392,8 @@ __global__ void __launch_bounds__(576, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == S::TMA_WARP) {
     // ---------------- TMA producer ----------------
@@ -770,6 +774,8 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 8) {
     // ---------------- TMA producer: K, V once; per query tile Q, dO and the LSE / delta rows ----------------
@@ -1013,6 +1019,8 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 8) {
     if (lane == 0) {
@@ -1178,9 +1186,12 @@ __global__ void __launch_bounds__(320, 1)
 // over its 64-key tiles: dQ += dS·Kⱼ with A = dS read MN-major from the [64 keys][128 queries] dSᵀ
 // tile and B = Kⱼ (MN-major).  No scores are recomputed; the epilogue is the dQ kernel's.
 // ================================================================================================
+// Two CTAs share an SM (two stages each, ≈97 KB of shared memory and DH tensor-memory columns per
+// CTA), so that one CTA's prologue (Q tile, first dSᵀ tiles) and epilogue (QK-norm + RoPE backward)
+// overlap the other's stream of dSᵀ tiles: the kernel is bound by reading dSᵀ from HBM.
 template <int DH>
 struct DqDsShape {
-  static constexpr int STAGES = 4;
+  static constexpr int STAGES = 2;
   static constexpr int Q_TILE = 128 * DH * 2;   // q̃ tile (the QK-norm + RoPE backward reads it)
   static constexpr int DS_TILE = 64 * 128 * 2;  // [2 query chunks][64 keys][64 queries]
   static constexpr int K_TILE = 64 * DH * 2;
@@ -1194,7 +1205,7 @@ struct DqDsShape {
 };
 
 template <int DH>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, 2)
     attn_bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                           const __grid_constant__ CUtensorMap mds, const AttnArgs a) {
   using S = DqDsShape<DH>;
@@ -1237,6 +1248,8 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 4) {
     // ---------------- TMA producer ----------------
@@ -1328,6 +1341,8 @@ __global__ void __launch_bounds__(192, 1)
 // max_t ‖k_t‖ for each (batch, head): one CTA per (h, b).
 __global__ void attn_kmax_kernel(const uint16_t* __restrict__ k, float* __restrict__ kmax, int H,
                                  int T, int Dh, long long sb, long long sh, long long st) {
+  pdl_wait();
+  pdl_trigger();
   const int h = blockIdx.x, b = blockIdx.y;
   const uint16_t* base = k + b * sb + h * sh;
   float m = 0.f;
@@ -1371,6 +1386,8 @@ __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t
                                   uint16_t* __restrict__ ext, float ext_scale, int B, int H, int T,
                                   int Tpad, int Dh, long long sb, long long sh, long long st,
                                   long long sbd, long long shd, long long std_) {
+  pdl_wait();
+  pdl_trigger();
   // G = Dh/8 lanes per padded row (b, h, t < Tpad), 16-byte loads: pad[0][bh][t] = lse·log2(e),
   // pad[1][bh][t] = rowsum(dO∘O); rows t ≥ T are zero
   const int G = Dh >> 3;
@@ -1422,6 +1439,8 @@ __global__ void __launch_bounds__(128)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                          const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
                          const AttnArgs a) {
+  pdl_wait();
+  pdl_trigger();
   using S = BwdShape<DH>;
   constexpr int BNK = S::BNK, BMQ = S::BMQ;
   extern __shared__ uint8_t smem_raw[];
@@ -1584,6 +1603,8 @@ __global__ void __launch_bounds__(128)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                        const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
                        const AttnArgs a) {
+  pdl_wait();
+  pdl_trigger();
   using S = BwdShape<DH>;
   constexpr int BNK = S::BNK, BMQ = S::BMQ;
   extern __shared__ uint8_t smem_raw[];
@@ -1751,10 +1772,7 @@ template <int DH>
 gpt_status launch_fwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const AttnArgs& a, cudaStream_t stream) {
   GPT_TRY(ensure_smem(attn_fwd_kernel<DH>, FwdShape<DH>::SMEM));
-  attn_fwd_kernel<DH><<<grid, 256, FwdShape<DH>::SMEM, stream>>>(mq, mk, mv, a);
-  count_launch();
-  GPT_CUDA_TRY(cudaGetLastError());
-  return GPT_OK;
+  return launch_kernel(attn_fwd_kernel<DH>, grid, dim3(256), FwdShape<DH>::SMEM, stream, mq, mk, mv, a);
 }
 
 template <int DH>
@@ -1763,10 +1781,8 @@ gpt_status launch_fwd_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
   using S = TcFwdShape<DH>;
   GPT_TRY(ensure_smem(attn_fwd_tc_kernel<DH>, S::SMEM));
   dim3 grid((a.T + 255) / 256, a.H, a.B);
-  attn_fwd_tc_kernel<DH><<<grid, S::THREADS, S::SMEM, stream>>>(mq, mk, mv, a, kmax, kmax_const);
-  count_launch();
-  GPT_CUDA_TRY(cudaGetLastError());
-  return GPT_OK;
+  return launch_kernel(attn_fwd_tc_kernel<DH>, grid, dim3(S::THREADS), S::SMEM, stream, mq, mk, mv, a,
+                       kmax, kmax_const);
 }
 
 template <int DH>
@@ -1775,14 +1791,9 @@ gpt_status launch_bwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, c
   constexpr int smem = BwdShape<DH>::SMEM;
   GPT_TRY(ensure_smem(attn_bwd_dkdv_kernel<DH>, smem));
   GPT_TRY(ensure_smem(attn_bwd_dq_kernel<DH>, smem));
-  attn_bwd_dkdv_kernel<DH><<<grid, 128, smem, stream>>>(mq, mk, mv, mdo, a);
-  count_launch();
-  GPT_CUDA_TRY(cudaGetLastError());
+  GPT_TRY(launch_kernel(attn_bwd_dkdv_kernel<DH>, grid, dim3(128), smem, stream, mq, mk, mv, mdo, a));
   a.o = reinterpret_cast<uint16_t*>(dq);
-  attn_bwd_dq_kernel<DH><<<grid, 128, smem, stream>>>(mq, mk, mv, mdo, a);
-  count_launch();
-  GPT_CUDA_TRY(cudaGetLastError());
-  return GPT_OK;
+  return launch_kernel(attn_bwd_dq_kernel<DH>, grid, dim3(128), smem, stream, mq, mk, mv, mdo, a);
 }
 
 // tcgen05 backward: maps with 128-row boxes (outer tiles) and 64-row boxes (inner tiles), and the
@@ -1798,22 +1809,19 @@ gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[
   GPT_TRY(ensure_smem(attn_bwd_dq_ds_kernel<DH>, SD::SMEM));
   // dK/dV: outer 128-key tiles (K, V with 128-row boxes), inner 64-query tiles (Q, dO 64-row boxes)
   dim3 g1((a.T + 127) / 128, a.H, a.B);
-  attn_bwd_dkdv_tc_kernel<DH><<<g1, S::THREADS, S::SMEM, stream>>>(m64[0], m128[1], m128[2], m64[3],
-                                                                   mext, a);
-  count_launch();
-  GPT_CUDA_TRY(cudaGetLastError());
+  GPT_TRY(launch_kernel(attn_bwd_dkdv_tc_kernel<DH>, g1, dim3(S::THREADS), S::SMEM, stream, m64[0],
+                        m128[1], m128[2], m64[3], mext, a));
   a.o = reinterpret_cast<uint16_t*>(dq);
   dim3 g2((a.T + 127) / 128, a.H, a.B);
   if (mds != nullptr) {
     // dQ = dS·K from the stored dSᵀ tiles: outer 128-query tiles, inner 64-key tiles
-    attn_bwd_dq_ds_kernel<DH><<<g2, SD::THREADS, SD::SMEM, stream>>>(m128[0], m64[1], *mds, a);
+    return launch_kernel(attn_bwd_dq_ds_kernel<DH>, g2, dim3(SD::THREADS), SD::SMEM, stream, m128[0],
+                         m64[1], *mds, a);
   } else {
     // dQ with S and dP recomputed: outer 128-query tiles (Q, dO 128-row boxes), inner 64-key tiles
-    attn_bwd_dq_tc_kernel<DH><<<g2, S::THREADS, S::SMEM, stream>>>(m128[0], m64[1], m64[2], m128[3], a);
+    return launch_kernel(attn_bwd_dq_tc_kernel<DH>, g2, dim3(S::THREADS), S::SMEM, stream, m128[0],
+                         m64[1], m64[2], m128[3], a);
   }
-  count_launch();
-  GPT_CUDA_TRY(cudaGetLastError());
-  return GPT_OK;
 }
 
 }  // namespace
@@ -1854,10 +1862,8 @@ gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, f
     return GPT_ERR_UNSUPPORTED_SHAPE;
   const float kconst = sqrtf((float)Dh) * 1.002f;
   if (kmax_scratch) {
-    attn_kmax_kernel<<<dim3(H, B), 256, 0, stream>>>(reinterpret_cast<const uint16_t*>(k),
-                                                    kmax_scratch, H, T, Dh, sbq, shq, stq);
-    count_launch();
-    GPT_CUDA_TRY(cudaGetLastError());
+    GPT_TRY(launch_kernel(attn_kmax_kernel, dim3(H, B), dim3(256), 0, stream,
+                          reinterpret_cast<const uint16_t*>(k), kmax_scratch, H, T, Dh, sbq, shq, stq));
   }
   if (Dh == 128) return launch_fwd_tc<128>(mq2, mk2, mv2, a, kmax_scratch, kconst, stream);
   return launch_fwd_tc<64>(mq2, mk2, mv2, a, kmax_scratch, kconst, stream);
@@ -1921,11 +1927,10 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   {
     const int threads = 256;
     const long long blocks = (rows * (Dh / 8) + threads - 1) / threads;
-    attn_delta_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
-        reinterpret_cast<const uint16_t*>(o), reinterpret_cast<const uint16_t*>(dout), lse, delta,
-        ext, sqrtf((float)Dh), B, H, T, Tpad, Dh, sbo, sho, sto, sbd, shd, std_);
-    count_launch();
-    GPT_CUDA_TRY(cudaGetLastError());
+    GPT_TRY(launch_kernel(attn_delta_kernel, dim3((unsigned)blocks), dim3(threads), 0, stream,
+                          reinterpret_cast<const uint16_t*>(o), reinterpret_cast<const uint16_t*>(dout),
+                          lse, delta, ext, sqrtf((float)Dh), B, H, T, Tpad, Dh, sbo, sho, sto, sbd, shd,
+                          std_));
   }
   AttnArgs a{};
   a.B = B; a.H = H; a.T = T;

@@ -323,6 +323,22 @@ __device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, u
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Leader-issued MMA over the pair on 8-bit floats: D (256 × N, fp32) (+)= A (256 × 32) · B (N × 32),
+// A and B e4m3 (kind::f8f6f4; one instruction covers K = 32, i.e. 32 bytes of a 128-byte row).
+__device__ __forceinline__ void mma_e4m3_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Instruction descriptor, kind::f8f6f4: fp32 accumulator, e4m3 A and B (format code 0), K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // Arrive once on `bar` (same offset) in every CTA of `cta_mask` when the pair's MMAs issued so far
 // have completed.
 __device__ __forceinline__ void tc_commit_pair(uint64_t* bar, uint16_t cta_mask) {
@@ -496,6 +512,17 @@ __device__ __forceinline__ void exp2_poly2(float& p0, float& p1, float x0, float
   fma2_c(q0, q1, q0, q1, f0, f1, 0.999928057f);
   p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
   p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+// Programmatic dependent launch.  Kernels of the step are launched so that the next kernel's CTAs
+// may start while this one drains: every kernel runs its prologue (barriers, tensor-memory
+// allocation, descriptor prefetch — nothing in global memory), then pdl_wait(), which returns once
+// the preceding kernel has completed and its writes are visible, and then pdl_trigger(), which lets
+// the following kernel launch once every CTA of this one has started.  Both are no-ops in a kernel
+// launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }

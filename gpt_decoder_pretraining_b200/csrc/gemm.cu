@@ -128,6 +128,8 @@ struct GemmArgs {
   int batch;                       // independent matrices; tile t belongs to matrix t / (tiles_m·tiles_n)
   long long c_bstride, aux_bstride;  // elements between consecutive matrices of C and aux
   float alpha, beta;               // GPT_EPI_AXPBY
+  const float* dq_a;               // e4m3 operands: device dequantisation factors (else null)
+  const float* dq_b;
   void* C;
   int ldc;
   void* C2;
@@ -165,12 +167,14 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, int b, int m, 
     uint16_t* c = reinterpret_cast<uint16_t*>(a.C) + b * a.c_bstride + (size_t)m * a.ldc + n0;
     const uint16_t* x = a.aux + b * a.aux_bstride + (size_t)m * a.ldaux + n0;
     const bool rd = a.beta != 0.f;
+    // 8-bit operands: the accumulator is in units of (1/scale_a)·(1/scale_b)
+    const float al = a.dq_a ? a.alpha * (*a.dq_a) * (*a.dq_b) : a.alpha;
     if (full) {
 #pragma unroll
       for (int j = 0; j < 32; j += 8) {
         float w[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) w[e] = a.alpha * v[j + e];
+        for (int e = 0; e < 8; ++e) w[e] = al * v[j + e];
         if (rd) {
           const uint4 p = *reinterpret_cast<const uint4*>(x + j);
           const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
@@ -189,7 +193,7 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, int b, int m, 
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         if (n0 + j >= a.N) continue;
-        float w = a.alpha * v[j];
+        float w = al * v[j];
         if (rd) w = fmaf(a.beta, bf2f(x[j]), w);
         c[j] = f2bf(w);
       }
@@ -405,10 +409,13 @@ __device__ __forceinline__ bool plain_epilogue(const GemmArgs& a, const Work& w,
 // ------------------------------------------------------------------------------------------------
 // the kernel
 // ------------------------------------------------------------------------------------------------
-template <bool A_MN, bool B_MN, int EPI>
+// F8: A and B are e4m3 (one byte per element): a k-tile is 128 elements (the same 128-byte rows as
+// 64 bf16), one MMA instruction covers K = 32, and the accumulator is scaled in the epilogue.
+template <bool A_MN, bool B_MN, int EPI, bool F8 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(), 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmArgs args) {
+  constexpr int KE = F8 ? 2 * BK : BK;  // elements per k-tile
   using S = GemmShape;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -445,6 +452,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
   cluster_sync_all();  // barriers of both CTAs initialised before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // inputs written by the preceding kernel are visible from here on
+  pdl_trigger();
 
   const int pair = blockIdx.x >> 1;
   const Sched& sch = args.sched;
@@ -469,7 +478,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
           uint8_t* sa = smem + stage * S::STAGE_BYTES;
           uint8_t* sb = sa + S::A_BYTES;
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * S::STAGE_BYTES);
-          const int k0 = kt * BK;
+          const int k0 = kt * KE;
           if (!A_MN) {
             tma_load_3d_pair(sa, &tmA, &full[stage], k0, arow, bb);
           } else {
@@ -492,7 +501,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
   } else if (warp == 1) {
     // ---------------- MMA issuer (leader CTA): the warp runs the loop, one elected lane issues ----------------
     if (leader) {
-      constexpr uint32_t idesc = idesc_bf16(2 * BM, BN, A_MN, B_MN);
+      constexpr uint32_t idesc = F8 ? idesc_e4m3(2 * BM, BN) : idesc_bf16(2 * BM, BN, A_MN, B_MN);
       // stage-0 descriptors; stage s and slice kk are constant byte offsets from them
       const uint32_t s0 = smem_u32(smem);
       const uint64_t a_desc0 = A_MN ? sdesc_sw128(s0, 8192, 1024) : sdesc_sw128(s0, 16, 1024);
@@ -518,9 +527,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
           if (elect_one()) {
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
-              mma_bf16_pair(d_tmem, sdesc_add(ad, A_MN ? kk * 2048 : kk * 32),
-                            sdesc_add(bd, B_MN ? kk * 2048 : kk * 32), idesc,
-                            (kt > kt0 || kk > 0) ? 1u : 0u);
+              if constexpr (F8) {
+                mma_e4m3_pair(d_tmem, sdesc_add(ad, kk * 32), sdesc_add(bd, kk * 32), idesc,
+                              (kt > kt0 || kk > 0) ? 1u : 0u);
+              } else {
+                mma_bf16_pair(d_tmem, sdesc_add(ad, A_MN ? kk * 2048 : kk * 32),
+                              sdesc_add(bd, B_MN ? kk * 2048 : kk * 32), idesc,
+                              (kt > kt0 || kk > 0) ? 1u : 0u);
+              }
             }
             tc_commit_pair(&empty[stage], 0x3);
           }
@@ -708,16 +722,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
 // ------------------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------------------
-template <bool A_MN, bool B_MN, int EPI>
+template <bool A_MN, bool B_MN, int EPI, bool F8 = false>
 static gpt_status launch_inst(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& a,
                               cudaStream_t stream) {
   using S = GemmShape;
-  auto kern = gemm_kernel<A_MN, B_MN, EPI>;
+  auto kern = gemm_kernel<A_MN, B_MN, EPI, F8>;
   GPT_TRY(ensure_smem(kern, S::SMEM_BYTES));
-  kern<<<2 * a.sched.num_pairs, gemm_threads<EPI>(), S::SMEM_BYTES, stream>>>(ma, mb, a);
-  count_launch();
-  GPT_CUDA_TRY(cudaGetLastError());
-  return GPT_OK;
+  return launch_kernel(kern, dim3(2 * a.sched.num_pairs), dim3(gemm_threads<EPI>()), S::SMEM_BYTES,
+                       stream, ma, mb, a);
 }
 
 template <bool A_MN, bool B_MN>
@@ -775,13 +787,13 @@ static gpt_status check_gemm_args(int op, int M, int N, int K, const void* A, in
 
 // Tiles and the plain round-robin schedule (every tile whole, one CTA pair per tile up to the SM
 // count).
-static gpt_status fill_args(GemmArgs& a, int M, int N, int K, int batch = 1) {
+static gpt_status fill_args(GemmArgs& a, int M, int N, int K, int batch = 1, int k_per_tile = BK) {
   int sms = 0;
   GPT_TRY(device_info(&sms));
   a.M = M; a.N = N; a.K = K;
   a.tiles_m = (M + 2 * BM - 1) / (2 * BM);
   a.tiles_n = (N + BN - 1) / BN;
-  a.k_tiles = (K + BK - 1) / BK;
+  a.k_tiles = (K + k_per_tile - 1) / k_per_tile;
   a.batch = batch;
   a.alpha = 1.f;
   a.beta = 0.f;
@@ -893,6 +905,46 @@ gpt_status gemm_launch(int op, int epi, int M, int N, int K, const void* A, int 
   return gemm_launch_batched(g, stream, sk_scratch);
 }
 
+// C[M,N] (bf16) = alpha·dq_a·dq_b·(A·Bᵀ) with A [M,K] and B [N,K] e4m3, K-contiguous (NT).
+gpt_status gemm_e4m3_launch(int M, int N, int K, const void* A, int lda, const void* B, int ldb,
+                            void* C, int ldc, const float* dq_a, const float* dq_b, float alpha,
+                            int* status, cudaStream_t stream, void* sk_scratch) {
+  if (!A || !B || !C || !dq_a || !dq_b) return GPT_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0 || lda < K || ldb < K || ldc < N) return GPT_ERR_INVALID_ARG;
+  if ((lda % 16) || (ldb % 16) || (ldc % 8)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) |
+       reinterpret_cast<uintptr_t>(C)) & 15)
+    return GPT_ERR_UNSUPPORTED_SHAPE;
+  if (reinterpret_cast<uintptr_t>(sk_scratch) & 255) return GPT_ERR_UNSUPPORTED_SHAPE;
+  CUtensorMap ma, mb;
+  {
+    const uint64_t da[3] = {(uint64_t)K, (uint64_t)M, 1}, db[3] = {(uint64_t)K, (uint64_t)N, 1};
+    const uint64_t sa[2] = {(uint64_t)lda, ((uint64_t)lda * M + 15) & ~(uint64_t)15};
+    const uint64_t sb[2] = {(uint64_t)ldb, ((uint64_t)ldb * N + 15) & ~(uint64_t)15};
+    const uint32_t box[3] = {128, 128, 1};
+    if (!encode_map_u8(&ma, A, 3, da, sa, box) || !encode_map_u8(&mb, B, 3, db, sb, box))
+      return GPT_ERR_UNSUPPORTED_SHAPE;
+  }
+  GemmArgs a{};
+  GPT_TRY(fill_args(a, M, N, K, 1, 2 * BK));
+  a.C = C; a.ldc = ldc;
+  a.alpha = alpha; a.beta = 0.f;
+  a.dq_a = dq_a; a.dq_b = dq_b;
+  a.status = status;
+  if (sk_scratch) {
+    int sms = 0;
+    GPT_TRY(device_info(&sms));
+    Sched sk;
+    if (plan_stream_k(a.tiles_m * a.tiles_n, a.k_tiles, std::max(1, sms / 2), &sk)) {
+      a.sched = sk;
+      a.sk_cnt = reinterpret_cast<int*>(sk_scratch);
+      a.sk_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sk_scratch) +
+                                           ((GEMM_SK_COUNTER_BYTES + 255) & ~(size_t)255));
+    }
+  }
+  return launch_inst<false, false, GPT_EPI_AXPBY, true>(ma, mb, a, stream);
+}
+
 gpt_status gemm_heads_launch(int op, int M, int N, int K, const void* A, int lda, const void* B,
                              int ldb, void* heads, int T, int H, int Dh, int* status,
                              cudaStream_t stream) {
@@ -959,6 +1011,18 @@ extern "C" gpt_status gpt_qkv_proj_rope(const void* r, const void* w_qkv, void* 
 }
 
 extern "C" size_t gpt_gemm_scratch_bytes(void) { return gpt::gemm_sk_scratch_bytes(); }
+
+extern "C" gpt_status gpt_gemm_e4m3(int M, int N, int K, const void* A, int lda, const void* B,
+                                    int ldb, void* C, int ldc, const float* dq_a, const float* dq_b,
+                                    float alpha, void* scratch, int* status, void* stream) {
+  cudaStream_t s = gpt::as_stream(stream);
+  if (scratch) {
+    if (reinterpret_cast<uintptr_t>(scratch) & 255) return GPT_ERR_UNSUPPORTED_SHAPE;
+    GPT_CUDA_TRY(cudaMemsetAsync(scratch, 0, gpt::GEMM_SK_COUNTER_BYTES, s));
+  }
+  return gpt::gemm_e4m3_launch(M, N, K, A, lda, B, ldb, C, ldc, dq_a, dq_b, alpha, status, s,
+                               scratch);
+}
 
 extern "C" gpt_status gpt_gemm_batched(int op, int epilogue, int batch, int M, int N, int K,
                                        const void* A, int lda, long long a_bstride, const void* B,

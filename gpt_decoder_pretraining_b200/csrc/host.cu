@@ -1,6 +1,7 @@
 // Host utilities: device properties, TMA tensor-map encoding, status strings.
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 #include <unordered_map>
 
@@ -9,6 +10,14 @@
 namespace gpt {
 
 thread_local int64_t g_launch_count = 0;
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("GPTSTEP_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
 
 gpt_status device_info(int* num_sms) {
   static std::mutex mu;
@@ -81,6 +90,11 @@ bool encode_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_
                      const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128) {
   return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box,
                     swizzle128);
+}
+
+bool encode_map_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                   const uint64_t* strides_bytes, const uint32_t* box) {
+  return encode_map(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, rank, dims, strides_bytes, box, true);
 }
 
 bool encode_map_f32(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/gptstep.h"
 
 namespace gpt {
@@ -30,6 +32,9 @@ gpt_status device_info(int* num_sms);
 // Returns false if the driver rejects the map (alignment, box size).
 bool encode_map_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                      const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128);
+// Same for a tensor of bytes (e4m3), 128-byte swizzle.
+bool encode_map_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                   const uint64_t* strides_bytes, const uint32_t* box);
 // Same for an fp32 tensor, no swizzle.
 bool encode_map_f32(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                     const uint64_t* strides_bytes, const uint32_t* box);
@@ -47,6 +52,30 @@ inline gpt_status ensure_smem(K kernel, int bytes) {
 // Kernel-launch counter for reporting how many of this library's kernels a step enqueued.
 extern thread_local int64_t g_launch_count;
 inline void count_launch(int n = 1) { g_launch_count += n; }
+
+// Whether kernels are launched with programmatic stream serialization (default on; the environment
+// variable GPTSTEP_PDL=0 turns it off for comparison).
+bool pdl_enabled();
+
+// Launch `kern` on `s` with programmatic dependent launch allowed (see pdl_wait in common.cuh) and
+// count it.  Launch errors are reported as GPT_ERR_CUDA.
+template <typename... KArgs, typename... Args>
+inline gpt_status launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) return GPT_ERR_CUDA;
+  count_launch();
+  return GPT_OK;
+}
 
 // Set the bounded-wait limit of the kernels of one translation unit on the current device.
 gpt_status wait_limit_set_gemm(long long cycles);

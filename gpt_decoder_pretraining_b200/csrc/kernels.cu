@@ -27,6 +27,8 @@ __device__ __forceinline__ float warp_sum(float v) {
 // ------------------------------------------------------------------------------------------------
 __global__ void rmsnorm_fwd_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ y,
                                    float* __restrict__ rho, int rows, int d) {
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (row >= rows) return;
   const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * d);
@@ -70,6 +72,8 @@ template <bool DY_F32>
 __global__ void rmsnorm_bwd_kernel(const void* __restrict__ dy, const uint16_t* __restrict__ y,
                                    const float* __restrict__ rho, float* __restrict__ gx,
                                    uint16_t* __restrict__ gx_bf16, int accumulate, int rows, int d) {
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (row >= rows) return;
   const int nv = d >> 3;
@@ -112,6 +116,8 @@ __global__ void rmsnorm_bwd_kernel(const void* __restrict__ dy, const uint16_t* 
 // RoPE + QK-norm
 // ------------------------------------------------------------------------------------------------
 __global__ void rope_table_kernel(float* __restrict__ cs, int T, int half, int Dh) {
+  pdl_wait();
+  pdl_trigger();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= T * half) return;
   const int t = idx / half, i = idx % half;
@@ -131,6 +137,8 @@ template <int ROUNDS>
 __global__ void __launch_bounds__(256) rope_qknorm_fwd_kernel(uint16_t* __restrict__ qkv, float* __restrict__ rho_q,
                                                               float* __restrict__ rho_k, const float* __restrict__ cs,
                                                               int M, int T, int H, int Dh) {
+  pdl_wait();
+  pdl_trigger();
   const long long m = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (m >= M) return;
@@ -199,6 +207,8 @@ template <int ROUNDS, bool Y_HEADS>
 __global__ void __launch_bounds__(256) rope_qknorm_bwd_kernel(uint16_t* __restrict__ dqkv, const uint16_t* __restrict__ qkv,
                                                               const float* __restrict__ rho_q, const float* __restrict__ rho_k,
                                                               const float* __restrict__ cs, int M, int T, int H, int Dh) {
+  pdl_wait();
+  pdl_trigger();
   const long long m = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (m >= M) return;
@@ -274,6 +284,8 @@ __global__ void __launch_bounds__(256) rope_qknorm_bwd_kernel(uint16_t* __restri
 // ------------------------------------------------------------------------------------------------
 __global__ void embedding_fwd_kernel(const int32_t* __restrict__ tok, const uint16_t* __restrict__ wte,
                                      uint16_t* __restrict__ x, int M, int d, int V, int* status) {
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (row >= M) return;
   int id = tok[row];
@@ -294,6 +306,8 @@ __global__ void __launch_bounds__(1024) embedding_sort_kernel(const int32_t* __r
                                                               int V, uint32_t* __restrict__ keys_out,
                                                               int* __restrict__ run_start,
                                                               int* __restrict__ nruns) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint32_t sk[];  // [P] keys, then [P/1024 + 1] scan scratch
   int P = 1;
   while (P < n) P <<= 1;
@@ -365,6 +379,8 @@ constexpr int EMB_PIECE = 64;
 __global__ void embedding_piece_kernel(const uint32_t* __restrict__ keys, int n, const float* __restrict__ gx,
                                        float* __restrict__ dwte, float* __restrict__ partial, int seg0, int d,
                                        int accumulate) {
+  pdl_wait();
+  pdl_trigger();
   const int p = blockIdx.x;
   const int s = p * EMB_PIECE, e = min(n, s + EMB_PIECE);
   const int idx_before = (s > 0) ? (int)(keys[s - 1] >> 16) : -1;
@@ -402,6 +418,8 @@ __global__ void embedding_piece_kernel(const uint32_t* __restrict__ keys, int n,
 __global__ void embedding_fixup_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ run_start,
                                        const int* __restrict__ nruns, const float* __restrict__ partial,
                                        float* __restrict__ dwte, int d, int accumulate) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   if (r >= *nruns) return;
   const int s = run_start[r], e = run_start[r + 1];
@@ -433,6 +451,8 @@ __global__ void embedding_fixup_kernel(const uint32_t* __restrict__ keys, const 
 __global__ void ce_rows_kernel(const float2* __restrict__ stats, int ntiles, const float* __restrict__ zt,
                                const int32_t* __restrict__ targets, int M, int V, float* __restrict__ lse,
                                float* __restrict__ ell, int* status) {
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (row >= M) return;
   const float2* s = stats + (size_t)row * ntiles;
@@ -457,6 +477,8 @@ __global__ void __launch_bounds__(1024) ce_finalize_kernel(const float* __restri
                                                            const int32_t* __restrict__ targets, int M,
                                                            int V, float* __restrict__ loss,
                                                            float* __restrict__ inv_n) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ double ssum[1024];
   __shared__ int scnt[1024];
   double acc = 0.0;
@@ -483,6 +505,8 @@ __global__ void __launch_bounds__(1024) ce_finalize_kernel(const float* __restri
 }
 
 __global__ void cast_f32_bf16_kernel(const float* __restrict__ src, uint16_t* __restrict__ dst, size_t n) {
+  pdl_wait();
+  pdl_trigger();
   const size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (i + 4 <= n) {
     const float4 v = *reinterpret_cast<const float4*>(src + i);
@@ -497,6 +521,8 @@ __global__ void cast_f32_bf16_kernel(const float* __restrict__ src, uint16_t* __
 
 // dst[i] += src[i] (gradient accumulation across micro-batches), four floats per thread
 __global__ void add_f32_kernel(float* __restrict__ dst, const float* __restrict__ src, size_t n) {
+  pdl_wait();
+  pdl_trigger();
   const size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (i + 4 <= n) {
     float4 a = *reinterpret_cast<const float4*>(dst + i);
@@ -518,11 +544,8 @@ static inline unsigned blocks_for_warps(long long warps, int threads) {
 gpt_status rmsnorm_fwd(const void* x, void* y, float* rho, int rows, int d, cudaStream_t s) {
   if (!x || !y || !rho || rows <= 0 || d <= 0) return GPT_ERR_INVALID_ARG;
   if (d % 8) return GPT_ERR_UNSUPPORTED_SHAPE;
-  rmsnorm_fwd_kernel<<<blocks_for_warps(rows, 256), 256, 0, s>>>(
-      reinterpret_cast<const uint16_t*>(x), reinterpret_cast<uint16_t*>(y), rho, rows, d);
-  count_launch();
-  GPT_CUDA_TRY(cudaGetLastError());
-  return GPT_OK;
+  return launch_kernel(rmsnorm_fwd_kernel, dim3(blocks_for_warps(rows, 256)), dim3(256), 0, s,
+                       reinterpret_cast<const uint16_t*>(x), reinterpret_cast<uint16_t*>(y), rho, rows, d);
 }
 
 gpt_status rmsnorm_bwd(const void* dy, int dy_f32, const void* y, const float* rho, float* gx,
@@ -531,23 +554,18 @@ gpt_status rmsnorm_bwd(const void* dy, int dy_f32, const void* y, const float* r
   if (d % 8) return GPT_ERR_UNSUPPORTED_SHAPE;
   const unsigned nb = blocks_for_warps(rows, 256);
   if (dy_f32)
-    rmsnorm_bwd_kernel<true><<<nb, 256, 0, s>>>(dy, reinterpret_cast<const uint16_t*>(y), rho, gx,
-                                                reinterpret_cast<uint16_t*>(gx_bf16), accumulate, rows, d);
-  else
-    rmsnorm_bwd_kernel<false><<<nb, 256, 0, s>>>(dy, reinterpret_cast<const uint16_t*>(y), rho, gx,
-                                                 reinterpret_cast<uint16_t*>(gx_bf16), accumulate, rows, d);
-  count_launch();
-  GPT_CUDA_TRY(cudaGetLastError());
-  return GPT_OK;
+    return launch_kernel(rmsnorm_bwd_kernel<true>, dim3(nb), dim3(256), 0, s, dy,
+                         reinterpret_cast<const uint16_t*>(y), rho, gx,
+                         reinterpret_cast<uint16_t*>(gx_bf16), accumulate, rows, d);
+  return launch_kernel(rmsnorm_bwd_kernel<false>, dim3(nb), dim3(256), 0, s, dy,
+                       reinterpret_cast<const uint16_t*>(y), rho, gx,
+                       reinterpret_cast<uint16_t*>(gx_bf16), accumulate, rows, d);
 }
 
 gpt_status rope_table(float* cs, int T, int Dh, cudaStream_t s) {
   if (!cs || T <= 0 || Dh <= 0 || (Dh % 4)) return GPT_ERR_INVALID_ARG;
   const int n = T * (Dh / 2);
-  rope_table_kernel<<<(n + 255) / 256, 256, 0, s>>>(cs, T, Dh / 2, Dh);
-  count_launch();
-  GPT_CUDA_TRY(cudaGetLastError());
-  return GPT_OK;
+  return launch_kernel(rope_table_kernel, dim3((n + 255) / 256), dim3(256), 0, s, cs, T, Dh / 2, Dh);
 }
 
 static gpt_status check_rope(int B, int T, int H, int Dh) {
@@ -611,11 +629,9 @@ gpt_status embedding_fwd(const int32_t* tok, const void* wte, void* x, int M, in
                          int* status, cudaStream_t s) {
   if (!tok || !wte || !x || M <= 0 || d <= 0 || V <= 0) return GPT_ERR_INVALID_ARG;
   if (d % 8) return GPT_ERR_UNSUPPORTED_SHAPE;
-  embedding_fwd_kernel<<<blocks_for_warps(M, 256), 256, 0, s>>>(
-      tok, reinterpret_cast<const uint16_t*>(wte), reinterpret_cast<uint16_t*>(x), M, d, V, status);
-  count_launch();
-  GPT_CUDA_TRY(cudaGetLastError());
-  return GPT_OK;
+  return launch_kernel(embedding_fwd_kernel, dim3(blocks_for_warps(M, 256)), dim3(256), 0, s, tok,
+                       reinterpret_cast<const uint16_t*>(wte), reinterpret_cast<uint16_t*>(x), M, d, V,
+                       status);
 }
 
 size_t embedding_bwd_scratch_bytes(int M, int d, int V) {
@@ -663,36 +679,26 @@ gpt_status embedding_bwd(const int32_t* tok, const float* gx, float* dwte, int M
 
 gpt_status ce_rows(const float2* stats, int ntiles, const float* zt, const int32_t* targets, int M,
                    int V, float* lse, float* ell, int* status, cudaStream_t s) {
-  ce_rows_kernel<<<blocks_for_warps(M, 256), 256, 0, s>>>(stats, ntiles, zt, targets, M, V, lse, ell, status);
-  count_launch();
-  GPT_CUDA_TRY(cudaGetLastError());
-  return GPT_OK;
+  return launch_kernel(ce_rows_kernel, dim3(blocks_for_warps(M, 256)), dim3(256), 0, s, stats, ntiles, zt,
+                       targets, M, V, lse, ell, status);
 }
 
 gpt_status ce_finalize(const float* ell, const int32_t* targets, int M, int V, float* loss,
                        float* inv_n, cudaStream_t s) {
-  ce_finalize_kernel<<<1, 1024, 0, s>>>(ell, targets, M, V, loss, inv_n);
-  count_launch();
-  GPT_CUDA_TRY(cudaGetLastError());
-  return GPT_OK;
+  return launch_kernel(ce_finalize_kernel, dim3(1), dim3(1024), 0, s, ell, targets, M, V, loss, inv_n);
 }
 
 gpt_status add_f32(float* dst, const float* src, size_t n, cudaStream_t s) {
   const size_t threads = 256, per = 4;
   const size_t blocks = (n + threads * per - 1) / (threads * per);
-  add_f32_kernel<<<(unsigned)blocks, (unsigned)threads, 0, s>>>(dst, src, n);
-  count_launch();
-  GPT_CUDA_TRY(cudaGetLastError());
-  return GPT_OK;
+  return launch_kernel(add_f32_kernel, dim3((unsigned)blocks), dim3((unsigned)threads), 0, s, dst, src, n);
 }
 
 gpt_status cast_f32_bf16(const float* src, void* dst, size_t n, cudaStream_t s) {
   const size_t threads = 256, per = 4;
   const size_t blocks = (n + threads * per - 1) / (threads * per);
-  cast_f32_bf16_kernel<<<(unsigned)blocks, (unsigned)threads, 0, s>>>(src, reinterpret_cast<uint16_t*>(dst), n);
-  count_launch();
-  GPT_CUDA_TRY(cudaGetLastError());
-  return GPT_OK;
+  return launch_kernel(cast_f32_bf16_kernel, dim3((unsigned)blocks), dim3((unsigned)threads), 0, s, src,
+                       reinterpret_cast<uint16_t*>(dst), n);
 }
 
 }  // namespace gpt

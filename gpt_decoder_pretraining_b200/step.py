@@ -38,7 +38,7 @@ EXPORTED = [
     "gpt_attention_bwd_scratch_bytes", "gpt_embedding_bwd_scratch_bytes", "gpt_embedding_bwd", "gpt_lmhead_ce_scratch_bytes",
     "gpt_lmhead_ce_fwd_bwd", "gpt_set_wait_limit", "gpt_debug_wait_probe", "gpt_debug_exp2_poly2",
     "gpt_gemm_batched", "gpt_adamw_step", "gpt_muon_scratch_bytes", "gpt_muon_step",
-    "gpt_optim_scratch_bytes", "gpt_optim_step",
+    "gpt_optim_scratch_bytes", "gpt_optim_step", "gpt_gemm_e4m3", "gpt_quantize_e4m3",
 ]
 
 
@@ -128,6 +128,8 @@ def lib():
         L.gpt_optim_scratch_bytes.restype = sz
         L.gpt_optim_step.argtypes = [ctypes.POINTER(_Config), vp, vp, vp, vp, vp, i32,
                                      ctypes.POINTER(OptimHparams), vp, sz, vp, vp]
+        L.gpt_gemm_e4m3.argtypes = [i32, i32, i32, vp, i32, vp, i32, vp, i32, vp, vp, f32, vp, vp, vp]
+        L.gpt_quantize_e4m3.argtypes = [vp, ll, vp, vp, vp, vp]
         L.gpt_set_wait_limit.argtypes = [ll]
         L.gpt_debug_wait_probe.argtypes = [vp, vp]
         L.gpt_debug_exp2_poly2.argtypes = [vp, vp, i32, vp]
@@ -434,6 +436,24 @@ def optim_step(cfg: GptConfig, master, params, grads, state_m, state_v, t: int, 
     _check(lib().gpt_optim_step(ctypes.byref(c), master.data_ptr(), _ptr(params), grads.data_ptr(),
                                 state_m.data_ptr(), state_v.data_ptr(), t, ctypes.byref(h),
                                 scratch.data_ptr(), scratch.numel(), _ptr(status), _stream()), "gpt_optim_step")
+
+
+def quantize_e4m3(x, q, dq, amax_scratch=None):
+    """gpt_quantize_e4m3: x bf16 → q (uint8 codes), dq (device float [1]) with x ≈ q·dq."""
+    import torch
+    if amax_scratch is None:
+        amax_scratch = torch.empty(1, dtype=torch.int32, device=x.device)
+    _check(lib().gpt_quantize_e4m3(x.data_ptr(), x.numel(), q.data_ptr(), dq.data_ptr(),
+                                   amax_scratch.data_ptr(), _stream()), "gpt_quantize_e4m3")
+
+
+def gemm_e4m3(A, B, C, dq_a, dq_b, M: int, N: int, K: int, alpha=1.0, status=None, scratch="auto"):
+    """gpt_gemm_e4m3: C (bf16) = alpha·dq_a·dq_b·A·Bᵀ on e4m3 codes A [M,K], B [N,K] (uint8)."""
+    if isinstance(scratch, str):
+        scratch = gemm_scratch(C.device)
+    _check(lib().gpt_gemm_e4m3(M, N, K, A.data_ptr(), A.shape[-1], B.data_ptr(), B.shape[-1], C.data_ptr(),
+                               C.shape[-1], dq_a.data_ptr(), dq_b.data_ptr(), float(alpha), _ptr(scratch),
+                               _ptr(status), _stream()), "gpt_gemm_e4m3")
 
 
 def set_wait_limit(cycles: int):

@@ -181,6 +181,22 @@ gpt_status gpt_gemm_batched(int op, int epilogue, int batch, int M, int N, int K
                             const void* aux, int ldaux, long long aux_bstride, float alpha,
                             float beta, int* status, void* stream);
 
+/* 8-bit GEMM (the FP8 matrix products of the d24 speedrun, supa beginna nanochat, and of the
+ * alpha-nanochat-d24 run): tcgen05 kind::f8f6f4 on e4m3 operands with per-tensor scales.
+ *   C[M,N] (bf16) = bf16(alpha · dq_a · dq_b · Σ_k A[m,k]·B[n,k])      (NT: A, B K-contiguous)
+ * A, B: e4m3 bytes, lda/ldb multiples of 16; dq_a, dq_b: DEVICE floats (from gpt_quantize_e4m3);
+ * fp32 accumulation; scratch as for gpt_gemm (NULL: every tile whole). */
+gpt_status gpt_gemm_e4m3(int M, int N, int K, const void* A, int lda, const void* B, int ldb,
+                         void* C, int ldc, const float* dq_a, const float* dq_b, float alpha,
+                         void* scratch, int* status, void* stream);
+
+/* Per-tensor e4m3 quantisation of n bf16 values: amax = max|x|, scale = 448/amax (1 if amax = 0),
+ * q = e4m3(x·scale) (one fp32 multiply, round to nearest even, saturated to ±448), *dq = amax/448
+ * (1 if amax = 0) — so x ≈ q·dq.  q: n bytes (8-byte aligned); dq: device float; amax_scratch:
+ * one device unsigned int (zeroed by the call).  Deterministic. */
+gpt_status gpt_quantize_e4m3(const void* x, long long n, void* q, float* dq,
+                             unsigned int* amax_scratch, void* stream);
+
 /* Fused QKV projection with RoPE + QK-norm, the step's forward entry into attention:
  * [q | k | v] = r·W_qkvᵀ (r bf16 [B·T, d], W_qkv bf16 [3d, d], d = H·Dh); each q and k head becomes
  * RMS_Dh(RoPE(·, t)) as in gpt_rope_qknorm_fwd; all three are stored head-major in `heads`

@@ -48,18 +48,28 @@ class OracleConfig:
     seq_len: int
     batch: int
     windows: List[int]
+    n_kv_heads: int = 0  # key/value heads (grouped-query attention); 0 means n_heads
+
+    @property
+    def kv_heads(self) -> int:
+        return self.n_kv_heads if self.n_kv_heads > 0 else self.n_heads
 
 
 def oracle_config(cfg) -> OracleConfig:
     """Copy the fields the oracle needs from any object that has them."""
     return OracleConfig(cfg.depth, cfg.d_model, cfg.n_heads, cfg.head_dim, cfg.d_mlp, cfg.vocab,
-                        cfg.seq_len, cfg.batch, list(cfg.windows))
+                        cfg.seq_len, cfg.batch, list(cfg.windows), int(getattr(cfg, "n_kv_heads", 0) or 0))
 
 
 # ------------------------------------------------------------------------------------------------
-# parameter packing: wte [V,d]; per layer W_qkv [3d,d], W_o [d,d], W_fc [F,d], W_proj [d,F];
-# W_lm [V,d]; every matrix row-major [out, in] and applied as y = x·Wᵀ.
+# parameter packing: wte [V,d]; per layer W_qkv [d + 2·dkv, d] (rows q | k | v, dkv = kv_heads·Dh,
+# = 3d without grouping), W_o [d,d], W_fc [F,d], W_proj [d,F]; W_lm [V,d]; every matrix row-major
+# [out, in] and applied as y = x·Wᵀ.
 # ------------------------------------------------------------------------------------------------
+def qkv_rows(cfg: OracleConfig) -> int:
+    return cfg.d_model + 2 * cfg.kv_heads * cfg.head_dim
+
+
 def unpack(cfg: OracleConfig, flat: np.ndarray) -> Dict[str, np.ndarray]:
     d, F, V = cfg.d_model, cfg.d_mlp, cfg.vocab
     out = {}
@@ -72,7 +82,7 @@ def unpack(cfg: OracleConfig, flat: np.ndarray) -> Dict[str, np.ndarray]:
 
     take("wte", V, d)
     for l in range(cfg.depth):
-        take(f"qkv{l}", 3 * d, d)
+        take(f"qkv{l}", qkv_rows(cfg), d)
         take(f"o{l}", d, d)
         take(f"fc{l}", F, d)
         take(f"proj{l}", d, F)
@@ -84,7 +94,7 @@ def unpack(cfg: OracleConfig, flat: np.ndarray) -> Dict[str, np.ndarray]:
 
 def n_params(cfg: OracleConfig) -> int:
     d, F, V = cfg.d_model, cfg.d_mlp, cfg.vocab
-    return 2 * V * d + cfg.depth * (3 * d * d + d * d + 2 * F * d)
+    return 2 * V * d + cfg.depth * (qkv_rows(cfg) * d + d * d + 2 * F * d)
 
 
 # ------------------------------------------------------------------------------------------------
@@ -147,39 +157,47 @@ def logsumexp_rows(z: np.ndarray) -> np.ndarray:
 
 
 def attention_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, window: int):
-    """Causal (optionally windowed) softmax attention for one sequence, inputs [T, H, Dh].
+    """Causal (optionally windowed) softmax attention for one sequence: q [T, H, Dh], k and v
+    [T, Hkv, Dh] with H a multiple of Hkv.  Query head h reads key/value head h // (H/Hkv) (grouped
+    -query attention, consecutive query heads sharing one key/value head; Hkv = H is plain
+    multi-head attention).
 
     Returns o [T, H, Dh], the probabilities p [H, T, T] and lse [H, T] (natural log of the
     row sums of exp(scores)).
     """
     T, H, Dh = q.shape
+    group = H // k.shape[1]
     keep = attention_mask(T, window)
     scale = 1.0 / math.sqrt(Dh)
-    o = np.zeros_like(v)
+    o = np.zeros_like(q)
     p_all = np.zeros((H, T, T), dtype=q.dtype)
     lse = np.zeros((H, T), dtype=q.dtype)
     for h in range(H):
-        s = (q[:, h, :] @ k[:, h, :].T) * scale
+        g = h // group
+        s = (q[:, h, :] @ k[:, g, :].T) * scale
         s = np.where(keep, s, -np.inf)
         p = softmax_rows(s)
         lse[h] = logsumexp_rows(s)
         p_all[h] = p
-        o[:, h, :] = p @ v[:, h, :]
+        o[:, h, :] = p @ v[:, g, :]
     return o, p_all, lse
 
 
 def attention_backward(do: np.ndarray, q: np.ndarray, k: np.ndarray, v: np.ndarray, p: np.ndarray):
-    """Gradients of attention_forward given dO [T, H, Dh] and the saved probabilities."""
+    """Gradients of attention_forward given dO [T, H, Dh] and the saved probabilities; the
+    gradient of a shared key/value head sums over the query heads of its group."""
     T, H, Dh = q.shape
+    group = H // k.shape[1]
     scale = 1.0 / math.sqrt(Dh)
     dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     for h in range(H):
+        g = h // group
         ph = p[h]
-        dv[:, h, :] = ph.T @ do[:, h, :]
-        dp = do[:, h, :] @ v[:, h, :].T
+        dv[:, g, :] += ph.T @ do[:, h, :]
+        dp = do[:, h, :] @ v[:, g, :].T
         ds = ph * (dp - np.sum(dp * ph, axis=-1, keepdims=True))
-        dq[:, h, :] = (ds @ k[:, h, :]) * scale
-        dk[:, h, :] = (ds.T @ q[:, h, :]) * scale
+        dq[:, h, :] = (ds @ k[:, g, :]) * scale
+        dk[:, g, :] += (ds.T @ q[:, h, :]) * scale
     return dq, dk, dv
 
 
@@ -190,6 +208,8 @@ def forward_sequence(cfg: OracleConfig, P: Dict[str, np.ndarray], tok: np.ndarra
                      dtype=np.float64) -> dict:
     """Forward pass of one row; returns every intermediate the backward pass needs."""
     T, d, H, Dh = len(tok), cfg.d_model, cfg.n_heads, cfg.head_dim
+    Hkv = cfg.kv_heads
+    dkv = Hkv * Dh
     cos, sin = rope_angles(T, Dh, dtype)
     c = {"layers": []}
     x = P["wte"][tok].astype(dtype)
@@ -198,9 +218,9 @@ def forward_sequence(cfg: OracleConfig, P: Dict[str, np.ndarray], tok: np.ndarra
         L = {}
         r1, rho1 = rmsnorm(x)
         qkv = r1 @ P[f"qkv{l}"].T
-        q = qkv[:, 0 * d:1 * d].reshape(T, H, Dh)
-        k = qkv[:, 1 * d:2 * d].reshape(T, H, Dh)
-        v = qkv[:, 2 * d:3 * d].reshape(T, H, Dh)
+        q = qkv[:, :d].reshape(T, H, Dh)
+        k = qkv[:, d:d + dkv].reshape(T, Hkv, Dh)
+        v = qkv[:, d + dkv:d + 2 * dkv].reshape(T, Hkv, Dh)
         qn, rq = rmsnorm(rope(q, cos, sin))
         kn, rk = rmsnorm(rope(k, cos, sin))
         o, p, lse = attention_forward(qn, kn, v, cfg.windows[l])
@@ -248,7 +268,8 @@ def backward_sequence(cfg: OracleConfig, P: Dict[str, np.ndarray], tok: np.ndarr
         dqn, dkn, dv = attention_backward(do, L["qn"], L["kn"], L["v"], L["p"])
         dq = rope_inverse(rmsnorm_backward(dqn, L["qn"], L["rq"]), c["cos"], c["sin"])
         dk = rope_inverse(rmsnorm_backward(dkn, L["kn"], L["rk"]), c["cos"], c["sin"])
-        dqkv = np.concatenate([dq.reshape(T, d), dk.reshape(T, d), dv.reshape(T, d)], axis=1)
+        dkv = cfg.kv_heads * Dh
+        dqkv = np.concatenate([dq.reshape(T, d), dk.reshape(T, dkv), dv.reshape(T, dkv)], axis=1)
         G[f"qkv{l}"] += dqkv.T @ L["r1"]
         dx = dx + rmsnorm_backward(dqkv @ P[f"qkv{l}"], L["r1"], L["rho1"])
     np.add.at(G["wte"], tok, dx)
@@ -312,10 +333,10 @@ def forward_loss(cfg, params: np.ndarray, tokens: np.ndarray, targets: np.ndarra
 # per-kernel reference functions (same definitions, exposed on their own for unit parity tests)
 # ------------------------------------------------------------------------------------------------
 def attention_batch_forward(q, k, v, window, dtype=np.float64):
-    """q, k, v [B, H, T, Dh] → o [B, H, T, Dh], lse [B, H, T]."""
+    """q [B, H, T, Dh], k, v [B, Hkv, T, Dh] → o [B, H, T, Dh], lse [B, H, T]."""
     q, k, v = (np.asarray(a, dtype=dtype) for a in (q, k, v))
     B = q.shape[0]
-    o = np.zeros_like(v)
+    o = np.zeros_like(q)
     lse = np.zeros(q.shape[:3], dtype=dtype)
     for b in range(B):
         ob, _, lb = attention_forward(q[b].transpose(1, 0, 2), k[b].transpose(1, 0, 2),
@@ -326,7 +347,7 @@ def attention_batch_forward(q, k, v, window, dtype=np.float64):
 
 
 def attention_batch_backward(q, k, v, do, window, dtype=np.float64):
-    """Gradients dq, dk, dv [B, H, T, Dh] of Σ o·dO for attention_batch_forward."""
+    """Gradients dq [B, H, T, Dh], dk, dv [B, Hkv, T, Dh] of Σ o·dO for attention_batch_forward."""
     q, k, v, do = (np.asarray(a, dtype=dtype) for a in (q, k, v, do))
     dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     for b in range(q.shape[0]):

@@ -37,8 +37,8 @@ def golden():
     return vals
 
 
-def tiny(depth=2, d=32, hd=16, V=64, T=12, B=2, windows=None):
-    return custom(depth, d, hd, V, T, B, windows=windows, param_dtype=1)
+def tiny(depth=2, d=32, hd=16, V=64, T=12, B=2, windows=None, n_kv_heads=0):
+    return custom(depth, d, hd, V, T, B, windows=windows, param_dtype=1, n_kv_heads=n_kv_heads)
 
 
 def inputs_for(cfg, seed=0, std=0.3):
@@ -406,10 +406,13 @@ def _torch_model_loss(cfg, flat, tokens, targets):
         keep = (i[None, :] <= i[:, None]) & (i[None, :] > i[:, None] - w)
         r = F.rms_norm(x, (d,), eps=1e-6)
         qkv = F.linear(r, ws[f"h{l}.w_qkv"])
-        q, k, v = (t.view(B, T, H, Dh).transpose(1, 2) for t in qkv.split(d, dim=-1))
+        Hk = cfg.kv_heads
+        qq, kk, vv = qkv.split([d, Hk * Dh, Hk * Dh], dim=-1)
+        q = qq.view(B, T, H, Dh).transpose(1, 2)
+        k, v = (t.view(B, T, Hk, Dh).transpose(1, 2) for t in (kk, vv))
         q = F.rms_norm(rotate(q), (Dh,), eps=1e-6)
         k = F.rms_norm(rotate(k), (Dh,), eps=1e-6)
-        o = F.scaled_dot_product_attention(q, k, v, attn_mask=keep)
+        o = F.scaled_dot_product_attention(q, k, v, attn_mask=keep, enable_gqa=Hk != H)
         x = x + F.linear(o.transpose(1, 2).reshape(B, T, d), ws[f"h{l}.w_o"])
         u = F.linear(F.rms_norm(x, (d,), eps=1e-6), ws[f"h{l}.w_fc"])
         x = x + F.linear(torch.relu(u) ** 2, ws[f"h{l}.w_proj"])
@@ -417,10 +420,11 @@ def _torch_model_loss(cfg, flat, tokens, targets):
     return F.cross_entropy(z.view(-1, cfg.vocab), targets.view(-1), ignore_index=-1, reduction="mean")
 
 
-@pytest.mark.parametrize("windows", [None, [3, 0]])
-def test_whole_step_vs_torch_autograd(windows):
-    """Every gradient of the oracle's step equals torch autograd through library ops, to rounding."""
-    cfg = tiny(depth=2, d=32, hd=16, V=64, T=12, B=2, windows=windows)
+@pytest.mark.parametrize("windows,kv", [(None, 0), ([3, 0], 0), (None, 2), ([3, 0], 1)])
+def test_whole_step_vs_torch_autograd(windows, kv):
+    """Every gradient of the oracle's step equals torch autograd through library ops, to rounding;
+    kv > 0: grouped-query attention with kv key/value heads (torch: sdpa with enable_gqa)."""
+    cfg = tiny(depth=2, d=64, hd=16, V=64, T=12, B=2, windows=windows, n_kv_heads=kv)
     p, t, y = inputs_for(cfg, seed=5)
     y = y.copy()
     y[1, :3] = -1
@@ -431,3 +435,43 @@ def test_whole_step_vs_torch_autograd(windows):
     assert abs(r["loss"] - loss.item()) < 1e-12
     g = flat.grad.numpy()
     np.testing.assert_allclose(r["grads"], g, rtol=0, atol=1e-12 * max(1.0, np.abs(g).max()))
+
+
+@pytest.mark.parametrize("kv", [1, 2])
+def test_grouped_query_attention_equals_duplicated_heads(kv):
+    """Grouped-query attention is multi-head attention whose consecutive query heads see copies of
+    one key/value head: duplicating W_k and W_v row blocks gives the same loss, the same gradients
+    of every other tensor, and key/value gradients that are the group sums of the duplicated ones."""
+    g_cfg = tiny(depth=2, d=64, hd=16, V=64, T=10, B=2, windows=[4, 0], n_kv_heads=kv)
+    m_cfg = tiny(depth=2, d=64, hd=16, V=64, T=10, B=2, windows=[4, 0])
+    H, Dh, d = g_cfg.n_heads, g_cfg.head_dim, g_cfg.d_model
+    G = H // kv
+    p, t, y = inputs_for(g_cfg, seed=9)
+    gP = O.unpack(O.oracle_config(g_cfg), p)
+    mflat = np.zeros(m_cfg.n_params)
+    mP = O.unpack(O.oracle_config(m_cfg), mflat)
+    for name in gP:
+        if not name.startswith("qkv"):
+            mP[name][...] = gP[name]
+            continue
+        w = gP[name]
+        mP[name][:d] = w[:d]
+        for h in range(H):
+            src = h // G
+            mP[name][d + h * Dh:d + (h + 1) * Dh] = w[d + src * Dh:d + (src + 1) * Dh]
+            mP[name][2 * d + h * Dh:2 * d + (h + 1) * Dh] = w[d + kv * Dh + src * Dh:d + kv * Dh + (src + 1) * Dh]
+    rg = O.step(g_cfg, p, t, y)
+    rm = O.step(m_cfg, mflat, t, y)
+    assert abs(rg["loss"] - rm["loss"]) < 1e-12
+    gG = O.unpack(O.oracle_config(g_cfg), rg["grads"])
+    mG = O.unpack(O.oracle_config(m_cfg), rm["grads"])
+    for name in gG:
+        if not name.startswith("qkv"):
+            np.testing.assert_allclose(gG[name], mG[name], atol=1e-13)
+            continue
+        np.testing.assert_allclose(gG[name][:d], mG[name][:d], atol=1e-13)
+        for part in (1, 2):
+            for g in range(kv):
+                want = sum(mG[name][part * d + h * Dh:part * d + (h + 1) * Dh] for h in range(g * G, (g + 1) * G))
+                got = gG[name][d + (part - 1) * kv * Dh + g * Dh:d + (part - 1) * kv * Dh + (g + 1) * Dh]
+                np.testing.assert_allclose(got, want, atol=1e-13)
