@@ -36,12 +36,14 @@ constexpr float LN2 = 0.6931471805599453f;
 
 struct AttnArgs {
   int B, H, T, window;  // window: effective (T for full causal)
+  int Hkv, group;       // key/value heads and query heads per key/value head (H = Hkv·group)
   float scale_log2;     // log2(e)/sqrt(Dh)
   float scale;          // 1/sqrt(Dh)
   uint16_t* o;          // forward output / backward dq
   uint16_t* dk;
   uint16_t* dv;
-  long long sb_o, sh_o, st_o;        // strides of o (fwd) or of dq/dk/dv (bwd)
+  long long sb_o, sh_o, st_o;        // strides of o (fwd) or of dq (bwd)
+  long long sb_g, sh_g, st_g;        // bwd: strides of dk/dv (Hkv heads)
   const uint16_t* obuf;              // bwd: o
   const uint16_t* dobuf;             // bwd: dO
   long long sb_d, sh_d, st_d;        // strides of o/dO in the backward
@@ -156,8 +158,8 @@ __global__ void __launch_bounds__(256)
     load_tile<DH, BMQ>(sQ, &mq, &bar[0], q0, h, b);
     for (int i = 0; i < 2 && i < n_kv; ++i) {
       mbar_arrive_expect_tx(&bar[1 + i], 2 * S::KV_BYTES);
-      load_tile<DH, BNK>(sK0 + i * S::KV_BYTES, &mk, &bar[1 + i], (kv_first + i) * BNK, h, b);
-      load_tile<DH, BNK>(sV0 + i * S::KV_BYTES, &mv, &bar[1 + i], (kv_first + i) * BNK, h, b);
+      load_tile<DH, BNK>(sK0 + i * S::KV_BYTES, &mk, &bar[1 + i], (kv_first + i) * BNK, h / a.group, b);
+      load_tile<DH, BNK>(sV0 + i * S::KV_BYTES, &mv, &bar[1 + i], (kv_first + i) * BNK, h / a.group, b);
     }
   }
   bool ok = mbar_wait(&bar[0], 0, abort_flag, a.status);
@@ -257,8 +259,8 @@ __global__ void __launch_bounds__(256)
     __syncthreads();
     if (tid == 0 && i + 2 < n_kv) {
       mbar_arrive_expect_tx(&bar[1 + buf], 2 * S::KV_BYTES);
-      load_tile<DH, BNK>(sK0 + buf * S::KV_BYTES, &mk, &bar[1 + buf], (kv_first + i + 2) * BNK, h, b);
-      load_tile<DH, BNK>(sV0 + buf * S::KV_BYTES, &mv, &bar[1 + buf], (kv_first + i + 2) * BNK, h, b);
+      load_tile<DH, BNK>(sK0 + buf * S::KV_BYTES, &mk, &bar[1 + buf], (kv_first + i + 2) * BNK, h / a.group, b);
+      load_tile<DH, BNK>(sV0 + buf * S::KV_BYTES, &mv, &bar[1 + buf], (kv_first + i + 2) * BNK, h / a.group, b);
     }
   }
   // finalize
@@ -401,13 +403,14 @@ __global__ void __launch_bounds__(576, 1)
       mbar_arrive_expect_tx(bar_q, 2 * S::Q_TILE);
       load_tile<DH, 128>(smem + S::OFF_Q, &mq, bar_q, q0, h, b);
       load_tile<DH, 128>(smem + S::OFF_Q + S::Q_TILE, &mq, bar_q, q0 + 128, h, b);
+      const int hk = h / a.group;  // the key/value head this query head reads
       for (int j = 0; j < n_kv; ++j) {
         const int st = j & 1;
         if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1, abort_flag, a.status)) break;
         mbar_arrive_expect_tx(&kv_full[st], 2 * S::KV_TILE);
         const int k0 = (kv_first + j) * 128;
-        load_tile<DH, 128>(smem + S::OFF_K + st * S::KV_TILE, &mk, &kv_full[st], k0, h, b);
-        load_tile<DH, 128>(smem + S::OFF_V + st * S::KV_TILE, &mv, &kv_full[st], k0, h, b);
+        load_tile<DH, 128>(smem + S::OFF_K + st * S::KV_TILE, &mk, &kv_full[st], k0, hk, b);
+        load_tile<DH, 128>(smem + S::OFF_V + st * S::KV_TILE, &mv, &kv_full[st], k0, hk, b);
       }
     }
   } else if (warp == S::MMA_WARP) {
@@ -484,7 +487,7 @@ __global__ void __launch_bounds__(576, 1)
     bool ok = mbar_wait_warp(bar_q, 0, abort_flag, a.status);
     // fixed shift c_t (log2 units)
     const float qn = sqrtf(q_row_sumsq<DH>(smem + S::OFF_Q + x * S::Q_TILE, row));
-    const float km = kmax ? kmax[(long long)b * a.H + h] : kmax_const;
+    const float km = kmax ? kmax[(long long)b * a.Hkv + h / a.group] : kmax_const;
     const float c_nat = qn * km * a.scale * 1.001f + 1e-3f;
     if (c_nat > 40.f && t < T && half == 0) set_status(a.status, GPT_ERR_NUMERIC_RANGE);
     const float c2 = c_nat * LOG2E;
@@ -735,7 +738,7 @@ __global__ void __launch_bounds__(320, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = warp_id(), lane = lane_id();
-  const int h = blockIdx.y, b = blockIdx.z;
+  const int hk = blockIdx.y, b = blockIdx.z;  // one key/value head; its group's query heads in turn
   const int T = a.T, W = a.window;
   const int kv0 = blockIdx.x * 128;
   const int q_first = kv0 / 64;
@@ -743,8 +746,8 @@ __global__ void __launch_bounds__(320, 1)
   // window are fully masked and store zeros)
   const int q_reach = a.ds_t ? ((kv0 + 126 + W) / 128) * 128 + 127 : kv0 + 127 + W - 1;
   const int q_last = min(T - 1, q_reach) / 64;
-  const int n_q = q_last - q_first + 1;
-  const long long bh = (long long)b * a.H + h;
+  const int n_qt = q_last - q_first + 1;  // query tiles per query head
+  const int n_q = n_qt * a.group;         // iterations: query head hk·group + i / n_qt, tile i % n_qt
 
   if (threadIdx.x == 0) {
     mbar_init(kv_bar, 1);
@@ -781,13 +784,15 @@ __global__ void __launch_bounds__(320, 1)
     // ---------------- TMA producer: K, V once; per query tile Q, dO and the LSE / delta rows ----------------
     if (lane == 0) {
       mbar_arrive_expect_tx(kv_bar, 2 * S::BIG_TILE);
-      load_tile<DH, 128>(smem + S::OFF_A, &mk, kv_bar, kv0, h, b);
-      load_tile<DH, 128>(smem + S::OFF_B, &mv, kv_bar, kv0, h, b);
+      load_tile<DH, 128>(smem + S::OFF_A, &mk, kv_bar, kv0, hk, b);
+      load_tile<DH, 128>(smem + S::OFF_B, &mv, kv_bar, kv0, hk, b);
       const int rows = a.B * a.H * a.Tpad;
       for (int i = 0; i < n_q; ++i) {
         const int st = i % S::STAGES;
         if (!mbar_wait(&q_empty[st], ((i / S::STAGES) & 1) ^ 1, abort_flag, a.status)) break;
-        const int t0 = (q_first + i) * 64;
+        const int h = hk * a.group + i / n_qt;
+        const long long bh = (long long)b * a.H + h;
+        const int t0 = (q_first + i % n_qt) * 64;
         mbar_arrive_expect_tx(&q_full[st], S::STAGE_BYTES + 2 * S::EXT_ROWS_BYTES);
         uint8_t* dst = smem + S::OFF_STAGE + st * S::STAGE_BYTES;
         load_tile<DH, 64>(dst, &mq, &q_full[st], t0, h, b);
@@ -881,7 +886,8 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int i = 0; i < n_q && ok; ++i) {
       const int bf = i & 1;
-      const int qc = (q_first + i) * 64 + 32 * half;  // first query of this warp's 32 columns
+      const long long bh = (long long)b * a.H + hk * a.group + i / n_qt;  // the query head
+      const int qc = (q_first + i % n_qt) * 64 + 32 * half;  // first query of this warp's 32 columns
       // every (key, query) of the warp visible: no per-element mask
       const int kmin = kv0 + 32 * quarter, kmax_ = kmin + 31;
       const bool full = (kmax_ <= qc) && (kmin > qc + 31 - W) && (qc + 31 < T);
@@ -927,10 +933,10 @@ __global__ void __launch_bounds__(320, 1)
     if (ok) ok = mbar_wait_warp(done, 0, abort_flag, a.status);
     if (ok) {
       tc_fence_after();
-      const long long off = b * a.sb_o + h * a.sh_o + (long long)key * a.st_o;
+      const long long off = b * a.sb_g + hk * a.sh_g + (long long)key * a.st_g;
       if (half == 1 && a.rho_k != nullptr) {
         const bool valid = key < T;
-        const float rho = valid ? a.rho_k[((long long)b * T + key) * a.H + h] : 0.f;
+        const float rho = valid ? a.rho_k[((long long)b * T + key) * a.Hkv + hk] : 0.f;
         qknorm_rope_bwd_tmem<DH, 128>(tmem + lane_off + S::TM_ACC + DH, a.scale, smem + S::OFF_A, kr,
                                       rho, a.cos_sin + (size_t)(valid ? key : 0) * DH, a.dk + off, valid);
       } else {
@@ -1033,8 +1039,8 @@ __global__ void __launch_bounds__(320, 1)
         mbar_arrive_expect_tx(&kv_full[st], S::STAGE_BYTES);
         uint8_t* dst = smem + S::OFF_STAGE + st * S::STAGE_BYTES;
         const int k0 = (kv_first + j) * 64;
-        load_tile<DH, 64>(dst, &mk, &kv_full[st], k0, h, b);
-        load_tile<DH, 64>(dst + S::SMALL_TILE, &mv, &kv_full[st], k0, h, b);
+        load_tile<DH, 64>(dst, &mk, &kv_full[st], k0, h / a.group, b);
+        load_tile<DH, 64>(dst + S::SMALL_TILE, &mv, &kv_full[st], k0, h / a.group, b);
       }
     }
   } else if (warp == 9) {
@@ -1264,7 +1270,7 @@ __global__ void __launch_bounds__(192, 2)
         const int k0 = (kv_first + j) * 64;
         tma_load_3d(dst, &mds, &full[st], q0, k0, bh);                  // queries q0 .. q0+63
         tma_load_3d(dst + S::DS_TILE / 2, &mds, &full[st], q0 + 64, k0, bh);  // q0+64 .. q0+127
-        load_tile<DH, 64>(dst + S::DS_TILE, &mk, &full[st], k0, h, b);
+        load_tile<DH, 64>(dst + S::DS_TILE, &mk, &full[st], k0, h / a.group, b);
       }
     }
   } else if (warp == 5) {
@@ -1578,7 +1584,7 @@ __global__ void __launch_bounds__(128)
     for (int r = 0; r < 2; ++r) {
       const int key = key_r0 + 8 * r;
       if (key < T) {
-        const long long off = b * a.sb_o + h * a.sh_o + (long long)key * a.st_o;
+        const long long off = b * a.sb_g + h * a.sh_g + (long long)key * a.st_g;
 #pragma unroll
         for (int d = 0; d < DH / 8; ++d) {
           *reinterpret_cast<uint32_t*>(a.dk + off + 8 * d + 2 * t4) =
@@ -1808,7 +1814,7 @@ gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[
   GPT_TRY(ensure_smem(attn_bwd_dq_tc_kernel<DH>, S::SMEM));
   GPT_TRY(ensure_smem(attn_bwd_dq_ds_kernel<DH>, SD::SMEM));
   // dK/dV: outer 128-key tiles (K, V with 128-row boxes), inner 64-query tiles (Q, dO 64-row boxes)
-  dim3 g1((a.T + 127) / 128, a.H, a.B);
+  dim3 g1((a.T + 127) / 128, a.Hkv, a.B);  // one CTA per key tile of each key/value head
   GPT_TRY(launch_kernel(attn_bwd_dkdv_tc_kernel<DH>, g1, dim3(S::THREADS), S::SMEM, stream, m64[0],
                         m128[1], m128[2], m64[3], mext, a));
   a.o = reinterpret_cast<uint16_t*>(dq);
@@ -1826,44 +1832,47 @@ gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[
 
 }  // namespace
 
-// kmax_scratch: B·H floats for max_t ‖k_t‖, or nullptr when every k row is RMS-normalised over
-// Dh (QK-norm), in which case ‖k‖ ≤ √Dh·(1 + 2⁻⁹) after bf16 rounding bounds it.
+// kmax_scratch: B·Hkv floats for max_t ‖k_t‖, or nullptr when every k row is RMS-normalised over
+// Dh (QK-norm), in which case ‖k‖ ≤ √Dh·(1 + 2⁻⁹) after bf16 rounding bounds it.  Query head h
+// reads key/value head h / (H/Hkv).
 gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                         int H, int T, int Dh, int window, long long sbq, long long shq,
-                         long long stq, long long sbo, long long sho, long long sto, int* status,
-                         cudaStream_t stream, float* kmax_scratch) {
-  GPT_TRY(check_attn(q, B, H, T, Dh, sbq, shq, stq));
-  GPT_TRY(check_attn(k, B, H, T, Dh, sbq, shq, stq));
-  GPT_TRY(check_attn(v, B, H, T, Dh, sbq, shq, stq));
-  GPT_TRY(check_attn(o, B, H, T, Dh, sbo, sho, sto));
+                         int H, int Hkv, int T, int Dh, int window, HeadLayout lq, HeadLayout lkv,
+                         HeadLayout lo, int* status, cudaStream_t stream, float* kmax_scratch) {
+  if (Hkv <= 0 || H % Hkv) return GPT_ERR_INVALID_ARG;
+  GPT_TRY(check_attn(q, B, H, T, Dh, lq.sb, lq.sh, lq.st));
+  GPT_TRY(check_attn(k, B, Hkv, T, Dh, lkv.sb, lkv.sh, lkv.st));
+  GPT_TRY(check_attn(v, B, Hkv, T, Dh, lkv.sb, lkv.sh, lkv.st));
+  GPT_TRY(check_attn(o, B, H, T, Dh, lo.sb, lo.sh, lo.st));
   if (!lse) return GPT_ERR_INVALID_ARG;
-  CUtensorMap mq, mk, mv;
-  if (!make_head_map(&mq, q, B, H, T, Dh, sbq, shq, stq, 128) ||
-      !make_head_map(&mk, k, B, H, T, Dh, sbq, shq, stq, 64) ||
-      !make_head_map(&mv, v, B, H, T, Dh, sbq, shq, stq, 64))
-    return GPT_ERR_UNSUPPORTED_SHAPE;
   AttnArgs a{};
   a.B = B; a.H = H; a.T = T;
+  a.Hkv = Hkv; a.group = H / Hkv;
   a.window = (window > 0 && window < T) ? window : T;
   a.scale = 1.f / sqrtf((float)Dh);
   a.scale_log2 = a.scale * LOG2E;
   a.o = reinterpret_cast<uint16_t*>(o);
-  a.sb_o = sbo; a.sh_o = sho; a.st_o = sto;
+  a.sb_o = lo.sb; a.sh_o = lo.sh; a.st_o = lo.st;
   a.lse = lse;
   a.status = status;
   if (Dh == 32) {
+    CUtensorMap mq, mk, mv;
+    if (!make_head_map(&mq, q, B, H, T, Dh, lq.sb, lq.sh, lq.st, 128) ||
+        !make_head_map(&mk, k, B, Hkv, T, Dh, lkv.sb, lkv.sh, lkv.st, 64) ||
+        !make_head_map(&mv, v, B, Hkv, T, Dh, lkv.sb, lkv.sh, lkv.st, 64))
+      return GPT_ERR_UNSUPPORTED_SHAPE;
     dim3 grid((T + 127) / 128, H, B);
     return launch_fwd<32>(grid, mq, mk, mv, a, stream);
   }
   CUtensorMap mq2, mk2, mv2;
-  if (!make_head_map(&mq2, q, B, H, T, Dh, sbq, shq, stq, 128) ||
-      !make_head_map(&mk2, k, B, H, T, Dh, sbq, shq, stq, 128) ||
-      !make_head_map(&mv2, v, B, H, T, Dh, sbq, shq, stq, 128))
+  if (!make_head_map(&mq2, q, B, H, T, Dh, lq.sb, lq.sh, lq.st, 128) ||
+      !make_head_map(&mk2, k, B, Hkv, T, Dh, lkv.sb, lkv.sh, lkv.st, 128) ||
+      !make_head_map(&mv2, v, B, Hkv, T, Dh, lkv.sb, lkv.sh, lkv.st, 128))
     return GPT_ERR_UNSUPPORTED_SHAPE;
   const float kconst = sqrtf((float)Dh) * 1.002f;
   if (kmax_scratch) {
-    GPT_TRY(launch_kernel(attn_kmax_kernel, dim3(H, B), dim3(256), 0, stream,
-                          reinterpret_cast<const uint16_t*>(k), kmax_scratch, H, T, Dh, sbq, shq, stq));
+    GPT_TRY(launch_kernel(attn_kmax_kernel, dim3(Hkv, B), dim3(256), 0, stream,
+                          reinterpret_cast<const uint16_t*>(k), kmax_scratch, Hkv, T, Dh, lkv.sb,
+                          lkv.sh, lkv.st));
   }
   if (Dh == 128) return launch_fwd_tc<128>(mq2, mk2, mv2, a, kmax_scratch, kconst, stream);
   return launch_fwd_tc<64>(mq2, mk2, mv2, a, kmax_scratch, kconst, stream);
@@ -1877,30 +1886,25 @@ size_t attention_bwd_scratch_bytes(int B, int H, int T, bool store_ds) {
   return rows * (2 * sizeof(float) + 2 * 16) + (store_ds ? rows * (size_t)T * 2 : 0);
 }
 
-// Strides: (sbq, shq, stq) for q, k, v; (sbg, shg, stg) for dq, dk, dv; (sbo, sho, sto) for o;
-// (sbd, shd, std_) for dO.
+// Layouts: lq for q, lkv for k and v (Hkv heads), ldq for dq, ldkv for dk and dv, lo for o, ldo for
+// dO.  dK and dV of a key/value head sum over the query heads of its group.
 gpt_status attention_bwd(const void* q, const void* k, const void* v, const void* o,
                          const void* dout, const float* lse, float* delta, void* dq, void* dk,
-                         void* dv, int B, int H, int T, int Dh, int window, long long sbq,
-                         long long shq, long long stq, long long sbg, long long shg, long long stg,
-                         long long sbo, long long sho, long long sto, long long sbd, long long shd,
-                         long long std_, int* status, cudaStream_t stream, const float* rho_q,
+                         void* dv, int B, int H, int Hkv, int T, int Dh, int window, HeadLayout lq,
+                         HeadLayout lkv, HeadLayout ldq, HeadLayout ldkv, HeadLayout lo,
+                         HeadLayout ldo, int* status, cudaStream_t stream, const float* rho_q,
                          const float* rho_k, const float* cos_sin, bool store_ds) {
-  GPT_TRY(check_attn(q, B, H, T, Dh, sbq, shq, stq));
-  GPT_TRY(check_attn(k, B, H, T, Dh, sbq, shq, stq));
-  GPT_TRY(check_attn(v, B, H, T, Dh, sbq, shq, stq));
-  GPT_TRY(check_attn(dq, B, H, T, Dh, sbg, shg, stg));
-  GPT_TRY(check_attn(dk, B, H, T, Dh, sbg, shg, stg));
-  GPT_TRY(check_attn(dv, B, H, T, Dh, sbg, shg, stg));
-  GPT_TRY(check_attn(o, B, H, T, Dh, sbo, sho, sto));
-  GPT_TRY(check_attn(dout, B, H, T, Dh, sbd, shd, std_));
+  if (Hkv <= 0 || H % Hkv) return GPT_ERR_INVALID_ARG;
+  if (Dh == 32 && Hkv != H) return GPT_ERR_UNSUPPORTED_SHAPE;  // the head_dim-32 path is per head
+  GPT_TRY(check_attn(q, B, H, T, Dh, lq.sb, lq.sh, lq.st));
+  GPT_TRY(check_attn(k, B, Hkv, T, Dh, lkv.sb, lkv.sh, lkv.st));
+  GPT_TRY(check_attn(v, B, Hkv, T, Dh, lkv.sb, lkv.sh, lkv.st));
+  GPT_TRY(check_attn(dq, B, H, T, Dh, ldq.sb, ldq.sh, ldq.st));
+  GPT_TRY(check_attn(dk, B, Hkv, T, Dh, ldkv.sb, ldkv.sh, ldkv.st));
+  GPT_TRY(check_attn(dv, B, Hkv, T, Dh, ldkv.sb, ldkv.sh, ldkv.st));
+  GPT_TRY(check_attn(o, B, H, T, Dh, lo.sb, lo.sh, lo.st));
+  GPT_TRY(check_attn(dout, B, H, T, Dh, ldo.sb, ldo.sh, ldo.st));
   if (!lse || !delta) return GPT_ERR_INVALID_ARG;
-  CUtensorMap mq, mk, mv, mdo;
-  if (!make_head_map(&mq, q, B, H, T, Dh, sbq, shq, stq, 64) ||
-      !make_head_map(&mk, k, B, H, T, Dh, sbq, shq, stq, 64) ||
-      !make_head_map(&mv, v, B, H, T, Dh, sbq, shq, stq, 64) ||
-      !make_head_map(&mdo, dout, B, H, T, Dh, sbd, shd, std_, 64))
-    return GPT_ERR_UNSUPPORTED_SHAPE;
   const int Tpad = (T + 63) / 64 * 64;
   // scratch: [2][B·H][Tpad] fp32 (LSE·log2 e, delta), then the dK/dV kernel's extension rows
   // [2][B·H][Tpad][8] bf16, fetched with TMA in 64-row boxes
@@ -1929,11 +1933,12 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
     const long long blocks = (rows * (Dh / 8) + threads - 1) / threads;
     GPT_TRY(launch_kernel(attn_delta_kernel, dim3((unsigned)blocks), dim3(threads), 0, stream,
                           reinterpret_cast<const uint16_t*>(o), reinterpret_cast<const uint16_t*>(dout),
-                          lse, delta, ext, sqrtf((float)Dh), B, H, T, Tpad, Dh, sbo, sho, sto, sbd, shd,
-                          std_));
+                          lse, delta, ext, sqrtf((float)Dh), B, H, T, Tpad, Dh, lo.sb, lo.sh, lo.st,
+                          ldo.sb, ldo.sh, ldo.st));
   }
   AttnArgs a{};
   a.B = B; a.H = H; a.T = T;
+  a.Hkv = Hkv; a.group = H / Hkv;
   a.window = (window > 0 && window < T) ? window : T;
   a.scale = 1.f / sqrtf((float)Dh);
   a.scale_log2 = a.scale * LOG2E;
@@ -1943,23 +1948,31 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   a.ext = ext;
   a.ds_t = ds_t;
   a.status = status;
-  a.sb_o = sbg; a.sh_o = shg; a.st_o = stg;  // strides of the dq/dk/dv outputs
+  a.sb_o = ldq.sb; a.sh_o = ldq.sh; a.st_o = ldq.st;     // dq
+  a.sb_g = ldkv.sb; a.sh_g = ldkv.sh; a.st_g = ldkv.st;  // dk, dv
   a.rho_q = rho_q;
   a.rho_k = rho_k;
   a.cos_sin = cos_sin;
   if (rho_q && (Dh == 32 || !rho_k || !cos_sin)) return GPT_ERR_INVALID_ARG;
-  dim3 grid((T + 63) / 64, H, B);
   a.dk = reinterpret_cast<uint16_t*>(dk);
   a.dv = reinterpret_cast<uint16_t*>(dv);
-  if (Dh == 32) return launch_bwd<32>(grid, mq, mk, mv, mdo, a, dq, stream);
+  if (Dh == 32) {
+    CUtensorMap mq, mk, mv, mdo;
+    if (!make_head_map(&mq, q, B, H, T, Dh, lq.sb, lq.sh, lq.st, 64) ||
+        !make_head_map(&mk, k, B, H, T, Dh, lkv.sb, lkv.sh, lkv.st, 64) ||
+        !make_head_map(&mv, v, B, H, T, Dh, lkv.sb, lkv.sh, lkv.st, 64) ||
+        !make_head_map(&mdo, dout, B, H, T, Dh, ldo.sb, ldo.sh, ldo.st, 64))
+      return GPT_ERR_UNSUPPORTED_SHAPE;
+    dim3 grid((T + 63) / 64, H, B);
+    return launch_bwd<32>(grid, mq, mk, mv, mdo, a, dq, stream);
+  }
   CUtensorMap m128[4], m64[4];
   const void* src[4] = {q, k, v, dout};
+  const HeadLayout lay[4] = {lq, lkv, lkv, ldo};
+  const int heads[4] = {H, Hkv, Hkv, H};
   for (int i = 0; i < 4; ++i) {
-    const bool is_do = (i == 3);
-    if (!make_head_map(&m128[i], src[i], B, H, T, Dh, is_do ? sbd : sbq, is_do ? shd : shq,
-                       is_do ? std_ : stq, 128) ||
-        !make_head_map(&m64[i], src[i], B, H, T, Dh, is_do ? sbd : sbq, is_do ? shd : shq,
-                       is_do ? std_ : stq, 64))
+    if (!make_head_map(&m128[i], src[i], B, heads[i], T, Dh, lay[i].sb, lay[i].sh, lay[i].st, 128) ||
+        !make_head_map(&m64[i], src[i], B, heads[i], T, Dh, lay[i].sb, lay[i].sh, lay[i].st, 64))
       return GPT_ERR_UNSUPPORTED_SHAPE;
   }
   if (Dh == 128) GPT_TRY(launch_bwd_tc<128>(m128, m64, mext, ds_t ? &mds : nullptr, a, dq, stream));
@@ -2006,31 +2019,35 @@ gpt_status attention_bwd_noalloc(const void* q, const void* k, const void* v, co
     return GPT_ERR_UNSUPPORTED_SHAPE;
   float* delta = nullptr;
   GPT_TRY(noalloc_delta_ptr(&delta));
-  return attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, T, Dh, window, sbq, shq, stq,
-                       sbq, shq, stq, sbo, sho, sto, sbo, sho, sto, status, stream, nullptr,
-                       nullptr, nullptr, false);
+  const HeadLayout lq{sbq, shq, stq}, lo{sbo, sho, sto};
+  return attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, H, T, Dh, window, lq, lq, lq, lq,
+                       lo, lo, status, stream, nullptr, nullptr, nullptr, false);
 }
 
 }  // namespace gpt
 
 extern "C" gpt_status gpt_attention_fwd(const void* q, const void* k, const void* v, void* o,
-                                        float* lse, float* kmax, int B, int H, int T, int Dh,
-                                        int window, long long sb_qkv, long long sh_qkv,
-                                        long long st_qkv, long long sb_o, long long sh_o,
+                                        float* lse, float* kmax, int B, int H, int H_kv, int T,
+                                        int Dh, int window, long long sb_q, long long sh_q,
+                                        long long st_q, long long sb_kv, long long sh_kv,
+                                        long long st_kv, long long sb_o, long long sh_o,
                                         long long st_o, int* status, void* stream) {
-  return gpt::attention_fwd(q, k, v, o, lse, B, H, T, Dh, window, sb_qkv, sh_qkv, st_qkv, sb_o,
-                            sh_o, st_o, status, gpt::as_stream(stream), kmax);
+  return gpt::attention_fwd(q, k, v, o, lse, B, H, H_kv, T, Dh, window, {sb_q, sh_q, st_q},
+                            {sb_kv, sh_kv, st_kv}, {sb_o, sh_o, st_o}, status,
+                            gpt::as_stream(stream), kmax);
 }
 
 extern "C" gpt_status gpt_attention_bwd(const void* q, const void* k, const void* v, const void* o,
                                         const void* dout, const float* lse, float* delta, void* dq,
-                                        void* dk, void* dv, int B, int H, int T, int Dh,
-                                        int window, long long sb_qkv, long long sh_qkv,
-                                        long long st_qkv, long long sb_o, long long sh_o,
-                                        long long st_o, int* status, void* stream) {
-  return gpt::attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, T, Dh, window, sb_qkv,
-                            sh_qkv, st_qkv, sb_qkv, sh_qkv, st_qkv, sb_o, sh_o, st_o, sb_o, sh_o,
-                            st_o, status, gpt::as_stream(stream), nullptr, nullptr, nullptr, true);
+                                        void* dk, void* dv, int B, int H, int H_kv, int T, int Dh,
+                                        int window, long long sb_q, long long sh_q, long long st_q,
+                                        long long sb_kv, long long sh_kv, long long st_kv,
+                                        long long sb_o, long long sh_o, long long st_o,
+                                        int* status, void* stream) {
+  const gpt::HeadLayout lq{sb_q, sh_q, st_q}, lkv{sb_kv, sh_kv, st_kv}, lo{sb_o, sh_o, st_o};
+  return gpt::attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, H_kv, T, Dh, window, lq,
+                            lkv, lq, lkv, lo, lo, status, gpt::as_stream(stream), nullptr, nullptr,
+                            nullptr, true);
 }
 
 extern "C" size_t gpt_attention_bwd_scratch_bytes(int B, int H, int T) {

@@ -137,8 +137,8 @@ struct GemmArgs {
   int ldaux;
   int* status;
   CeArgs ce;
-  // head-major outputs (EPI_BF16_HEADS, EPI_QKV_ROPE + Dh)
-  int T, H, Dh, d;
+  // head-major outputs (EPI_BF16_HEADS, EPI_QKV_ROPE + Dh); Hkv key/value heads (QKV)
+  int T, H, Dh, d, Hkv;
   const float* cs;        // [T, Dh/2, 2] cos / sin
   float* rho_q;           // [M, H]
   float* rho_k;
@@ -590,7 +590,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
       if constexpr (EPI > EPI_QKV_ROPE) {
         // one head (DH columns) at a time: q and k heads get RoPE + QK-norm, v heads a plain cast
         constexpr int DH = EPI - EPI_QKV_ROPE, HALF = DH / 2;
-        const long long bhtd = (long long)(args.M / args.T) * args.H * args.T * DH;
+        const long long btd = (long long)(args.M / args.T) * args.T * DH;  // one head of all rows
+        const int dkv = args.Hkv * DH;
         const int b = m / args.T, t = m % args.T;
 #pragma unroll 1
         for (int hh = half * (BN / DH / G); hh < (half + 1) * (BN / DH / G); ++hh) {
@@ -605,8 +606,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
             for (int j = 0; j < 32; ++j) xh[c * 32 + j] = __uint_as_float(r[j]);
           }
           if (m >= args.M || n_head >= args.N) continue;
-          const int region = n_head / args.d;            // 0 q, 1 k, 2 v
-          const int h = (n_head % args.d) / DH;
+          // columns: q (H heads) | k (Hkv heads) | v (Hkv heads)
+          const int region = n_head < args.d ? 0 : (n_head < args.d + dkv ? 1 : 2);
+          const int h = (n_head - (region == 0 ? 0 : args.d + (region - 1) * dkv)) / DH;
+          const int nh = region == 0 ? args.H : args.Hkv;  // heads of this region
           if (region < 2) {
             const float4* cs4 = reinterpret_cast<const float4*>(args.cs + (size_t)t * DH);
             float ss = 0.f;
@@ -624,10 +627,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
             const float rr = rsqrtf(ss / (float)DH + 1e-6f);
 #pragma unroll
             for (int j = 0; j < DH; ++j) xh[j] *= rr;
-            (region == 0 ? args.rho_q : args.rho_k)[(size_t)m * args.H + h] = rr;
+            (region == 0 ? args.rho_q : args.rho_k)[(size_t)m * nh + h] = rr;
           }
-          uint16_t* dst = reinterpret_cast<uint16_t*>(args.C) + region * bhtd +
-                          (((long long)b * args.H + h) * args.T + t) * DH;
+          // q at 0, k after the H query heads, v after the Hkv key heads: [B][heads][T][DH] each
+          const long long base = region == 0 ? 0 : btd * (args.H + (long long)(region - 1) * args.Hkv);
+          uint16_t* dst = reinterpret_cast<uint16_t*>(args.C) + base +
+                          (((long long)b * nh + h) * args.T + t) * DH;
 #pragma unroll
           for (int j = 0; j < DH; j += 8) {
             uint4 o;
@@ -965,8 +970,10 @@ gpt_status gemm_heads_launch(int op, int M, int N, int K, const void* A, int lda
 
 gpt_status gemm_qkv_rope_launch(int M, int d, const void* A, const void* Wqkv, void* heads,
                                 float* rho_q, float* rho_k, const float* cs, int T, int H, int Dh,
-                                int* status, cudaStream_t stream) {
-  const int N = 3 * d, K = d;
+                                int* status, cudaStream_t stream, int Hkv) {
+  if (Hkv <= 0) Hkv = H;
+  if (H % Hkv) return GPT_ERR_INVALID_ARG;
+  const int N = d + 2 * Hkv * Dh, K = d;
   GPT_TRY(check_gemm_args(GPT_GEMM_NT, M, N, K, A, K, Wqkv, K, heads, N));
   if (!rho_q || !rho_k || !cs || T <= 0 || H * Dh != d || (M % T)) return GPT_ERR_INVALID_ARG;
   if (Dh != 32 && Dh != 64 && Dh != 128) return GPT_ERR_UNSUPPORTED_SHAPE;
@@ -976,7 +983,7 @@ gpt_status gemm_qkv_rope_launch(int M, int d, const void* A, const void* Wqkv, v
   GemmArgs a{};
   GPT_TRY(fill_args(a, M, N, K));
   a.C = heads; a.ldc = N; a.status = status;
-  a.T = T; a.H = H; a.Dh = Dh; a.d = d; a.cs = cs; a.rho_q = rho_q; a.rho_k = rho_k;
+  a.T = T; a.H = H; a.Dh = Dh; a.d = d; a.Hkv = Hkv; a.cs = cs; a.rho_q = rho_q; a.rho_k = rho_k;
   if (Dh == 128) return launch_inst<false, false, EPI_QKV_ROPE + 128>(ma, mb, a, stream);
   if (Dh == 64) return launch_inst<false, false, EPI_QKV_ROPE + 64>(ma, mb, a, stream);
   return launch_inst<false, false, EPI_QKV_ROPE + 32>(ma, mb, a, stream);
@@ -1004,10 +1011,10 @@ gpt_status gemm_ce_launch(bool grad, int M, int N, int K, const void* A, int lda
 
 extern "C" gpt_status gpt_qkv_proj_rope(const void* r, const void* w_qkv, void* heads, float* rho_q,
                                         float* rho_k, const float* cos_sin, int B, int T, int H,
-                                        int Dh, int* status, void* stream) {
-  if (B <= 0 || T <= 0 || H <= 0 || Dh <= 0) return GPT_ERR_INVALID_ARG;
+                                        int H_kv, int Dh, int* status, void* stream) {
+  if (B <= 0 || T <= 0 || H <= 0 || Dh <= 0 || H_kv <= 0) return GPT_ERR_INVALID_ARG;
   return gpt::gemm_qkv_rope_launch(B * T, H * Dh, r, w_qkv, heads, rho_q, rho_k, cos_sin, T, H, Dh,
-                                   status, gpt::as_stream(stream));
+                                   status, gpt::as_stream(stream), H_kv);
 }
 
 extern "C" size_t gpt_gemm_scratch_bytes(void) { return gpt::gemm_sk_scratch_bytes(); }

@@ -82,6 +82,11 @@ gpt_status wait_limit_set_gemm(long long cycles);
 gpt_status wait_limit_set_attention(long long cycles);
 gpt_status wait_limit_set_diag(long long cycles);
 
+// Element strides of a [B, heads, T, Dh] tensor: batch, head, position (Dh contiguous).
+struct HeadLayout {
+  long long sb, sh, st;
+};
+
 // Kernel-level launchers used by the step orchestrator (same semantics as the C entry points).
 // sk_scratch (may be null): gemm_sk_scratch_bytes() bytes, 256-byte aligned, whose leading
 // arrival counters are zero; with it, tiles of a partly empty last wave may be split along K.
@@ -125,10 +130,10 @@ int gemm_ce_tile_n();  // vocabulary columns per CE statistics tile
 gpt_status gemm_heads_launch(int op, int M, int N, int K, const void* A, int lda, const void* B,
                              int ldb, void* heads, int T, int H, int Dh, int* status,
                              cudaStream_t stream);
-// [q|k|v] = A·W_qkvᵀ with RoPE + QK-norm applied to q and k, stored head-major as
-// heads[part][b][h][t][j]; rho_q / rho_k [M, H] receive the norm factors.
+// [q|k|v] = A·W_qkvᵀ with RoPE + QK-norm applied to q and k, stored head-major: q [B][H][T][Dh],
+// then k and v [B][Hkv][T][Dh] (Hkv ≤ 0: H); rho_q [M, H] / rho_k [M, Hkv] receive the norm factors.
 gpt_status gemm_qkv_rope_launch(int M, int d, const void* A, const void* Wqkv, void* heads,
                                 float* rho_q, float* rho_k, const float* cs, int T, int H, int Dh,
-                                int* status, cudaStream_t stream);
+                                int* status, cudaStream_t stream, int Hkv = 0);
 
 }  // namespace gpt

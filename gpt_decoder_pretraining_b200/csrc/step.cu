@@ -42,18 +42,20 @@ gpt_status ce_finalize(const float* ell, const int32_t* targets, int M, int V, f
 gpt_status cast_f32_bf16(const float* src, void* dst, size_t n, cudaStream_t s);
 gpt_status add_f32(float* dst, const float* src, size_t n, cudaStream_t s);
 gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                         int H, int T, int Dh, int window, long long sbq, long long shq,
-                         long long stq, long long sbo, long long sho, long long sto, int* status,
-                         cudaStream_t stream, float* kmax_scratch);
+                         int H, int Hkv, int T, int Dh, int window, HeadLayout lq, HeadLayout lkv,
+                         HeadLayout lo, int* status, cudaStream_t stream, float* kmax_scratch);
 gpt_status attention_bwd(const void* q, const void* k, const void* v, const void* o,
                          const void* dout, const float* lse, float* delta, void* dq, void* dk,
-                         void* dv, int B, int H, int T, int Dh, int window, long long sbq,
-                         long long shq, long long stq, long long sbg, long long shg, long long stg,
-                         long long sbo, long long sho, long long sto, long long sbd, long long shd,
-                         long long std_, int* status, cudaStream_t stream, const float* rho_q,
+                         void* dv, int B, int H, int Hkv, int T, int Dh, int window, HeadLayout lq,
+                         HeadLayout lkv, HeadLayout ldq, HeadLayout ldkv, HeadLayout lo,
+                         HeadLayout ldo, int* status, cudaStream_t stream, const float* rho_q,
                          const float* rho_k, const float* cos_sin, bool store_ds);
 
 static inline size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// Key/value heads (grouped-query attention; n_kv_heads = 0 means one per query head) and width.
+static inline int kv_heads(const gpt_config& c) { return c.n_kv_heads > 0 ? c.n_kv_heads : c.n_heads; }
+static inline int kv_dim(const gpt_config& c) { return kv_heads(c) * c.head_dim; }
 
 // ------------------------------------------------------------------------------------------------
 // configuration and packing
@@ -65,6 +67,9 @@ static gpt_status validate(const gpt_config* c) {
     return GPT_ERR_INVALID_ARG;
   if (c->param_dtype != GPT_DTYPE_BF16 && c->param_dtype != GPT_DTYPE_F32) return GPT_ERR_INVALID_ARG;
   if (c->n_heads * c->head_dim != c->d_model) return GPT_ERR_INVALID_ARG;
+  if (c->n_kv_heads < 0 || (c->n_kv_heads > 0 && c->n_heads % c->n_kv_heads)) return GPT_ERR_INVALID_ARG;
+  // the head_dim-32 attention path handles one query head per key/value head only
+  if (c->head_dim == 32 && c->n_kv_heads > 0 && c->n_kv_heads != c->n_heads) return GPT_ERR_UNSUPPORTED_SHAPE;
   if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return GPT_ERR_UNSUPPORTED_SHAPE;
   if ((c->d_model % 64) || (c->d_mlp % 64) || (c->vocab % 64)) return GPT_ERR_UNSUPPORTED_SHAPE;
   if (c->vocab > 65536) return GPT_ERR_UNSUPPORTED_SHAPE;
@@ -84,7 +89,7 @@ static Layout make_layout(const gpt_config& c) {
   size_t pos = 0;
   L.off.push_back(pos); pos += V * d;
   for (int l = 0; l < c.depth; ++l) {
-    L.off.push_back(pos); pos += 3 * d * d;
+    L.off.push_back(pos); pos += (d + 2 * kv_dim(c)) * d;
     L.off.push_back(pos); pos += d * d;
     L.off.push_back(pos); pos += F * d;
     L.off.push_back(pos); pos += d * F;
@@ -172,9 +177,9 @@ static Plan make_plan(const gpt_config& c, size_t n_params) {
   const size_t layer0 = pos;
   p.r1 = take(M * d * 2) - layer0;
   p.rho1 = take(M * 4) - layer0;
-  p.qkv = take(M * 3 * d * 2) - layer0;
+  p.qkv = take(M * (d + 2 * kv_dim(c)) * 2) - layer0;
   p.rq = take(M * H * 4) - layer0;
-  p.rk = take(M * H * 4) - layer0;
+  p.rk = take(M * kv_heads(c) * 4) - layer0;
   p.lse = take(M * H * 4) - layer0;
   p.o = take(M * d * 2) - layer0;
   p.r2 = take(M * d * 2) - layer0;
@@ -203,7 +208,7 @@ static Plan make_plan(const gpt_config& c, size_t n_params) {
   p.du = take(M * F * 2);
   p.dr = take(M * d * 2);
   p.dO = take(M * d * 2);
-  p.dqkv = take(M * 3 * d * 2);
+  p.dqkv = take(M * (d + 2 * kv_dim(c)) * 2);
   p.delta = take(attention_bwd_scratch_bytes(c.batch, H, c.seq_len, true));
   p.emb = take(embedding_bwd_scratch_bytes((int)M, (int)d, (int)V));
   p.sk = take(gemm_sk_scratch_bytes());
@@ -273,10 +278,15 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
   uint16_t* x = reinterpret_cast<uint16_t*>(ws + p.x);
   uint16_t* xf = reinterpret_cast<uint16_t*>(ws + p.xf);
   float* rhof = reinterpret_cast<float*>(ws + p.rhof);
-  const long long qs_b = (long long)T * 3 * d, qs_h = Dh, qs_t = 3 * d;  // dq/dk/dv inside dqkv
+  const int Hkv = kv_heads(c), dkv = kv_dim(c), nqkv = d + 2 * dkv;  // q | k | v widths
+  const long long qs_b = (long long)T * nqkv, qs_h = Dh, qs_t = nqkv;  // dq/dk/dv inside dqkv
   const long long os_b = (long long)T * d, os_h = Dh, os_t = d;          // o (token-major)
   const long long hs_b = (long long)H * T * Dh, hs_h = (long long)T * Dh, hs_t = Dh;  // head-major
-  const long long bhtd = (long long)B * H * T * Dh;
+  const long long bhtd = (long long)B * H * T * Dh, bhktd = (long long)B * Hkv * T * Dh;
+  const HeadLayout lay_q{hs_b, hs_h, hs_t};                            // q̃ head-major
+  const HeadLayout lay_kv{(long long)Hkv * T * Dh, hs_h, hs_t};       // k̃, v head-major
+  const HeadLayout lay_o{os_b, os_h, os_t};                            // o token-major
+  const HeadLayout lay_dqkv{qs_b, qs_h, qs_t};                         // dq, dk, dv in dqkv
 
   // bucket b of the gradient is final: b = 0 W_lm, 1 + (depth − 1 − l) layer l, depth + 1 wte
   auto bucket_done = [&](int b) -> gpt_status {
@@ -301,12 +311,13 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
     float* rho2 = reinterpret_cast<float*>(at(p.rho2, l));
     uint16_t* hsq = reinterpret_cast<uint16_t*>(at(p.hsq, l));
     PROF(PROF_NORM, 0, 4.0 * (double)M * d + 4.0 * M, rmsnorm_fwd(x, r1, rho1, M, d, s));
-    // q̃, k̃, v head-major [3][B][H][T][Dh]; RoPE + QK-norm fused into the projection epilogue
-    PROF(PROF_GEMM, gemm_flops(M, 3.0 * d, d), 0,
-         gemm_qkv_rope_launch(M, d, r1, W(wq), qkv, rq, rk, rope, T, H, Dh, status, s));
+    // q̃ [B][H][T][Dh], k̃ and v [B][Hkv][T][Dh] head-major; RoPE + QK-norm fused into the
+    // projection epilogue
+    PROF(PROF_GEMM, gemm_flops(M, (double)nqkv, d), 0,
+         gemm_qkv_rope_launch(M, d, r1, W(wq), qkv, rq, rk, rope, T, H, Dh, status, s, Hkv));
     PROF(PROF_ATTN_FWD, 4.0 * Dh * H * B * attn_pairs(T, st->window[l]), 0,
-         attention_fwd(qkv, qkv + bhtd, qkv + 2 * bhtd, o, lse, B, H, T, Dh, st->window[l], hs_b,
-                       hs_h, hs_t, os_b, os_h, os_t, status, s, nullptr));
+         attention_fwd(qkv, qkv + bhtd, qkv + bhtd + bhktd, o, lse, B, H, Hkv, T, Dh,
+                       st->window[l], lay_q, lay_kv, lay_o, status, s, nullptr));
     PROF(PROF_GEMM, gemm_flops(M, d, d), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_RESID, M, d, d, o, d, W(wq + 1), d, x, d, nullptr,
                         nullptr, 0, status, s, sk));
     PROF(PROF_NORM, 0, 4.0 * (double)M * d + 4.0 * M, rmsnorm_fwd(x, r2, rho2, M, d, s));
@@ -384,18 +395,18 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
     PROF(PROF_GEMM, gemm_flops(d, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, d, d, M, gxb, d, o, d, G(wq + 1), d, nullptr,
                         nullptr, 0, status, s, sk));
     PROF(PROF_ATTN_BWD, 8.0 * Dh * H * B * attn_pairs(T, st->window[l]), 0,
-         attention_bwd(qkv, qkv + bhtd, qkv + 2 * bhtd, o, dO, lse, delta, dqkv, dqkv + d,
-                       dqkv + 2 * d, B, H, T, Dh, st->window[l], hs_b, hs_h, hs_t, qs_b, qs_h,
-                       qs_t, os_b, os_h, os_t, hs_b, hs_h, hs_t, status, s,
-                       Dh == 32 ? nullptr : rq, rk, rope, true));
+         attention_bwd(qkv, qkv + bhtd, qkv + bhtd + bhktd, o, dO, lse, delta, dqkv, dqkv + d,
+                       dqkv + d + dkv, B, H, Hkv, T, Dh, st->window[l], lay_q, lay_kv, lay_dqkv,
+                       lay_dqkv, lay_o, lay_q, status, s, Dh == 32 ? nullptr : rq, rk, rope,
+                       true));
     if (Dh == 32) {  // the mma.sync path for head_dim 32 has no fused QK-norm/RoPE backward
       PROF(PROF_ROPE, 0, 12.0 * (double)M * d,
            rope_qknorm_bwd_heads(dqkv, qkv, rq, rk, rope, B, T, H, Dh, s));
     }
-    PROF(PROF_GEMM, gemm_flops(3.0 * d, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, 3 * d, d, M, dqkv, 3 * d, r1, d, G(wq), d,
+    PROF(PROF_GEMM, gemm_flops((double)nqkv, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, nqkv, d, M, dqkv, nqkv, r1, d, G(wq), d,
                         nullptr, nullptr, 0, status, s, sk));
     GPT_TRY(bucket_done(1 + (c.depth - 1 - l)));
-    PROF(PROF_GEMM, gemm_flops(M, d, 3.0 * d), 0, gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, 3 * d, dqkv, 3 * d, W(wq), d, dr, d,
+    PROF(PROF_GEMM, gemm_flops(M, d, (double)nqkv), 0, gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, nqkv, dqkv, nqkv, W(wq), d, dr, d,
                         nullptr, nullptr, 0, status, s, sk));
     PROF(PROF_NORM, 0, 14.0 * (double)M * d, rmsnorm_bwd(dr, 0, r1, rho1, gx, gxb, 1, M, d, s));
   }

@@ -62,7 +62,8 @@ class _Config(ctypes.Structure):
     _fields_ = [("depth", ctypes.c_int32), ("d_model", ctypes.c_int32), ("n_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("d_mlp", ctypes.c_int32), ("vocab", ctypes.c_int32),
                 ("seq_len", ctypes.c_int32), ("batch", ctypes.c_int32),
-                ("window", ctypes.POINTER(ctypes.c_int32)), ("param_dtype", ctypes.c_int32)]
+                ("window", ctypes.POINTER(ctypes.c_int32)), ("param_dtype", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32)]
 
 
 def lib():
@@ -96,15 +97,16 @@ def lib():
         L.gpt_gemm.argtypes = [i32, i32, i32, i32, i32, vp, i32, vp, i32, vp, i32, vp, vp, i32, vp, vp, vp]
         L.gpt_gemm_scratch_bytes.argtypes = []
         L.gpt_gemm_scratch_bytes.restype = sz
-        L.gpt_qkv_proj_rope.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp]
+        L.gpt_qkv_proj_rope.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]
         L.gpt_rmsnorm_fwd.argtypes = [vp, vp, vp, i32, i32, vp]
         L.gpt_rmsnorm_bwd.argtypes = [vp, i32, vp, vp, vp, vp, i32, i32, i32, vp]
         L.gpt_rope_qknorm_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.gpt_rope_qknorm_bwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.gpt_rope_table.argtypes = [vp, i32, i32, vp]
-        L.gpt_attention_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, ll, ll, ll, ll, ll, ll, vp, vp]
-        L.gpt_attention_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
-                                        ll, ll, ll, ll, ll, ll, vp, vp]
+        L.gpt_attention_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                        ll, ll, ll, ll, ll, ll, ll, ll, ll, vp, vp]
+        L.gpt_attention_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                        ll, ll, ll, ll, ll, ll, ll, ll, ll, vp, vp]
         L.gpt_attention_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                                 ll, ll, ll, ll, ll, ll, vp, vp]
         L.gpt_embedding_fwd.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp]
@@ -154,7 +156,8 @@ def _stream():
 def _cconfig(cfg: GptConfig):
     win = (ctypes.c_int32 * max(1, cfg.depth))(*cfg.windows)
     c = _Config(cfg.depth, cfg.d_model, cfg.n_heads, cfg.head_dim, cfg.d_mlp, cfg.vocab, cfg.seq_len,
-                cfg.batch, ctypes.cast(win, ctypes.POINTER(ctypes.c_int32)), cfg.param_dtype)
+                cfg.batch, ctypes.cast(win, ctypes.POINTER(ctypes.c_int32)), cfg.param_dtype,
+                int(getattr(cfg, "n_kv_heads", 0) or 0))
     return c, win
 
 
@@ -280,11 +283,12 @@ def gemm(op: int, epi: int, A, B, C, M: int, N: int, K: int, C2=None, aux=None, 
                           _ptr(C2), _ptr(aux), ldaux, _ptr(scratch), _ptr(status), _stream()), "gpt_gemm")
 
 
-def qkv_proj_rope(r, w_qkv, heads, rho_q, rho_k, cs, B, T, H, Dh, status=None):
-    """gpt_qkv_proj_rope: QKV projection + RoPE + QK-norm, head-major output [3][B][H][T][Dh]."""
+def qkv_proj_rope(r, w_qkv, heads, rho_q, rho_k, cs, B, T, H, Dh, status=None, H_kv=None):
+    """gpt_qkv_proj_rope: QKV projection + RoPE + QK-norm, head-major q̃ [B][H][T][Dh] then k̃, v
+    [B][H_kv][T][Dh]."""
     _check(lib().gpt_qkv_proj_rope(r.data_ptr(), w_qkv.data_ptr(), heads.data_ptr(), rho_q.data_ptr(),
-                                   rho_k.data_ptr(), cs.data_ptr(), B, T, H, Dh, _ptr(status), _stream()),
-           "qkv_proj_rope")
+                                   rho_k.data_ptr(), cs.data_ptr(), B, T, H, H_kv or H, Dh, _ptr(status),
+                                   _stream()), "qkv_proj_rope")
 
 
 def rmsnorm_fwd(x, y, rho):
@@ -314,15 +318,18 @@ def rope_qknorm_bwd(dqkv, qkv, rho_q, rho_k, cs, B, T, H, Dh):
 
 
 def attention_fwd(q, k, v, o, lse, window: int, strides_qkv, strides_o, B, H, T, Dh, status=None,
-                  kmax=None, qk_normalized=False):
-    """Causal/window attention forward.  Unless qk_normalized, a B·H float scratch for the per-head
-    key-norm bound is allocated here (or taken from `kmax`)."""
+                  kmax=None, qk_normalized=False, H_kv=None, strides_kv=None):
+    """Causal/window attention forward.  Unless qk_normalized, a B·H_kv float scratch for the
+    per-head key-norm bound is allocated here (or taken from `kmax`).  strides_qkv are q's (and, by
+    default, k's and v's); H_kv / strides_kv describe grouped key/value heads."""
     import torch
+    Hk = H_kv or H
     if not qk_normalized and kmax is None:
-        kmax = torch.empty(B * H, dtype=torch.float32, device=q.device)
+        kmax = torch.empty(B * Hk, dtype=torch.float32, device=q.device)
     _check(lib().gpt_attention_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                   _ptr(None if qk_normalized else kmax), B, H, T, Dh, window,
-                                   *strides_qkv, *strides_o, _ptr(status), _stream()), "attention_fwd")
+                                   _ptr(None if qk_normalized else kmax), B, H, Hk, T, Dh, window,
+                                   *strides_qkv, *(strides_kv or strides_qkv), *strides_o, _ptr(status),
+                                   _stream()), "attention_fwd")
 
 
 def attention_bwd_scratch_bytes(B: int, H: int, T: int) -> int:
@@ -336,11 +343,12 @@ def attention_bwd_scratch(B: int, H: int, T: int, device="cuda"):
 
 
 def attention_bwd(q, k, v, o, do, lse, delta, dq, dk, dv, window: int, strides_qkv, strides_o, B, H, T,
-                  Dh, status=None):
+                  Dh, status=None, H_kv=None, strides_kv=None):
     _check(lib().gpt_attention_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
                                    lse.data_ptr(), delta.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                                   dv.data_ptr(), B, H, T, Dh, window, *strides_qkv, *strides_o,
-                                   _ptr(status), _stream()), "attention_bwd")
+                                   dv.data_ptr(), B, H, H_kv or H, T, Dh, window, *strides_qkv,
+                                   *(strides_kv or strides_qkv), *strides_o, _ptr(status), _stream()),
+           "attention_bwd")
 
 
 def attention_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, window: int, strides_qkv, strides_o, B, H, T,

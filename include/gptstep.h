@@ -58,13 +58,18 @@ typedef struct gpt_config {
   int32_t depth, d_model, n_heads, head_dim, d_mlp, vocab, seq_len, batch;
   const int32_t* window;
   int32_t param_dtype;
+  int32_t n_kv_heads;  /* grouped-query attention: key/value heads, a divisor of n_heads; query
+                          head h reads key/value head h / (n_heads/n_kv_heads) (nanochat User
+                          Guide §10, group-query attention); 0 = n_heads.  head_dim 32 needs 0. */
 } gpt_config;
 
 typedef struct gpt_step gpt_step; /* opaque host-side plan; owns no device memory */
 
 /* Flat parameter packing (element offsets, each a multiple of 64):
  *   offsets[0]            wte   [V, d]
- *   offsets[1 + 4l + 0]   W_qkv [3d, d]   rows q | k | v, row = part·d + head·Dh + j
+ *   offsets[1 + 4l + 0]   W_qkv [d + 2·dkv, d]   rows q (d) | k (dkv) | v (dkv), dkv = n_kv_heads·Dh
+ *                                        (3d without grouping); head h's rows start at h·Dh of
+ *                                        its block
  *   offsets[1 + 4l + 1]   W_o   [d, d]
  *   offsets[1 + 4l + 2]   W_fc  [F, d]
  *   offsets[1 + 4l + 3]   W_proj[d, F]
@@ -198,13 +203,14 @@ gpt_status gpt_quantize_e4m3(const void* x, long long n, void* q, float* dq,
                              unsigned int* amax_scratch, void* stream);
 
 /* Fused QKV projection with RoPE + QK-norm, the step's forward entry into attention:
- * [q | k | v] = r·W_qkvᵀ (r bf16 [B·T, d], W_qkv bf16 [3d, d], d = H·Dh); each q and k head becomes
- * RMS_Dh(RoPE(·, t)) as in gpt_rope_qknorm_fwd; all three are stored head-major in `heads`
- * (bf16 [3][B][H][T][Dh]).  rho_q, rho_k fp32 [B·T, H]; cos_sin from gpt_rope_table.
- * Dh ∈ {32, 64, 128}. */
+ * [q | k | v] = r·W_qkvᵀ (r bf16 [B·T, d], W_qkv bf16 [d + 2·H_kv·Dh, d], d = H·Dh); each q and k
+ * head becomes RMS_Dh(RoPE(·, t)) as in gpt_rope_qknorm_fwd; all three are stored head-major in
+ * `heads`: q̃ bf16 [B][H][T][Dh], then k̃ and v bf16 [B][H_kv][T][Dh].  rho_q fp32 [B·T, H], rho_k
+ * fp32 [B·T, H_kv]; cos_sin from gpt_rope_table.  Dh ∈ {32, 64, 128}; H_kv divides H (H_kv = H:
+ * no grouping). */
 gpt_status gpt_qkv_proj_rope(const void* r, const void* w_qkv, void* heads, float* rho_q,
-                             float* rho_k, const float* cos_sin, int B, int T, int H, int Dh,
-                             int* status, void* stream);
+                             float* rho_k, const float* cos_sin, int B, int T, int H, int H_kv,
+                             int Dh, int* status, void* stream);
 
 /* RMSNorm forward over rows of d (bf16 in/out), y = x·rho, rho = 1/sqrt(mean(x²)+1e-6) (fp32). */
 gpt_status gpt_rmsnorm_fwd(const void* x, void* y, float* rho, int rows, int d, void* stream);
@@ -227,11 +233,14 @@ gpt_status gpt_rope_qknorm_bwd(void* dqkv, const void* qkv, const float* rho_q, 
 /* Fill cos_sin [T, Dh/2, 2] with cos/sin of t·10000^(−2i/Dh), angles computed in fp64. */
 gpt_status gpt_rope_table(float* cos_sin, int T, int Dh, void* stream);
 
-/* Causal / sliding-window flash attention.  q, k, v, o, dq, dk, dv are bf16 tensors addressed as
- * element (b, h, t, j) at base + b·sb + h·sh + t·st + j (strides in elements, j contiguous), one
- * stride set per tensor group: (sb_qkv, sh_qkv, st_qkv) for q/k/v/dq/dk/dv and (sb_o, sh_o, st_o)
- * for o/do.  lse: fp32 [B, H, T], the natural-log logsumexp of the scaled scores.  Dh ∈ {32, 64,
- * 128}.  window ≤ 0 or ≥ T = full causal.  delta: backward scratch of at least
+/* Causal / sliding-window flash attention with grouped-query heads.  q, o, dO, dq have H heads;
+ * k, v, dk, dv have H_kv heads (H a multiple of H_kv); query head h attends with key/value head
+ * h / (H/H_kv), and dk, dv sum over the query heads of their group (H_kv = H: multi-head
+ * attention).  Tensors are bf16, element (b, h, t, j) at base + b·sb + h·sh + t·st + j (strides in
+ * elements, j contiguous), one stride set per tensor group: (sb_q, sh_q, st_q) for q and dq,
+ * (sb_kv, sh_kv, st_kv) for k, v, dk, dv, (sb_o, sh_o, st_o) for o and dO.  lse: fp32 [B, H, T],
+ * the natural-log logsumexp of the scaled scores.  Dh ∈ {32, 64, 128} (32: H_kv = H only).
+ * window ≤ 0 or ≥ T = full causal.  delta: backward scratch of at least
  * gpt_attention_bwd_scratch_bytes(B, H, T) bytes, 16-byte aligned; per row (zero-padded to a
  * multiple of 64 rows per (b, h)) the backward stores LSE·log2(e) and rowsum(dO∘O) in fp32 and,
  * for Dh ≥ 64, both again as bf16 hi/mid/lo triples that its dK/dV kernel adds into the score
@@ -242,11 +251,13 @@ gpt_status gpt_rope_table(float* cos_sin, int T, int Dh, void* stream);
  * instead of a running maximum (softmax is invariant to the shift, so the result is exact); this
  * needs c_t ≤ 40 so that no row underflows, which always holds after QK-norm (c_t ≈ √Dh) — rows
  * beyond it set GPT_ERR_NUMERIC_RANGE in *status. */
-/* kmax: device scratch of B·H floats that receives max_t ‖k_t‖ per (b, h), or NULL when every k row
- * is RMS-normalised over Dh (QK-norm), in which case the bound √Dh·(1 + 2⁻⁹) is used. */
+/* kmax: device scratch of B·H_kv floats that receives max_t ‖k_t‖ per (b, key/value head), or
+ * NULL when every k row is RMS-normalised over Dh (QK-norm), in which case the bound
+ * √Dh·(1 + 2⁻⁹) is used. */
 gpt_status gpt_attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
-                             float* kmax, int B, int H, int T, int Dh, int window, long long sb_qkv,
-                             long long sh_qkv, long long st_qkv, long long sb_o, long long sh_o,
+                             float* kmax, int B, int H, int H_kv, int T, int Dh, int window,
+                             long long sb_q, long long sh_q, long long st_q, long long sb_kv,
+                             long long sh_kv, long long st_kv, long long sb_o, long long sh_o,
                              long long st_o, int* status, void* stream);
 /* Bytes of the `delta` scratch that gpt_attention_bwd needs for (B, H, T): 40 bytes per row of
  * R = B·H·⌈T/64⌉·64, plus 2·T·R bytes of dSᵀ — quadratic in T (1.6 GB for B·H = 192 at T = 2048,
@@ -256,13 +267,15 @@ gpt_status gpt_attention_fwd(const void* q, const void* k, const void* v, void* 
 size_t gpt_attention_bwd_scratch_bytes(int B, int H, int T);
 gpt_status gpt_attention_bwd(const void* q, const void* k, const void* v, const void* o,
                              const void* dout, const float* lse, float* delta, void* dq, void* dk,
-                             void* dv, int B, int H, int T, int Dh, int window, long long sb_qkv,
-                             long long sh_qkv, long long st_qkv, long long sb_o, long long sh_o,
+                             void* dv, int B, int H, int H_kv, int T, int Dh, int window,
+                             long long sb_q, long long sh_q, long long st_q, long long sb_kv,
+                             long long sh_kv, long long st_kv, long long sb_o, long long sh_o,
                              long long st_o, int* status, void* stream);
 
 /* Attention backward that allocates nothing.  The pages have no counterpart: this is a calling
  * convenience, not part of the method.  Arguments and results are those of gpt_attention_bwd
- * without `delta`; the per-row scratch that the backward needs (40 bytes per row of
+ * without `delta`, for multi-head attention (H_kv = H, one stride set (sb_qkv, sh_qkv, st_qkv) for
+ * q/k/v/dq/dk/dv); the per-row scratch that the backward needs (40 bytes per row of
  * B·H·⌈T/64⌉·64) is kept in a static device array inside this library
  * (GPT_ATTN_BWD_NOALLOC_FLOATS fp32 values = 8 MiB), which every GPU that loads the library holds
  * until the process exits.  dSᵀ is not stored: the dQ kernel recomputes the scores instead.

@@ -122,7 +122,11 @@ def test_kernel_entry_points_reject_bad_arguments(lib):
     assert lib.gpt_gemm(5, 0, 64, 64, 64, f, 64, f, 64, f, 64, None, None, 0, None, None, None) == -1
     assert lib.gpt_gemm(0, 0, 64, 64, 64, f, 60, f, 64, f, 64, None, None, 0, None, None, None) == -1
     assert lib.gpt_gemm(0, 0, 64, 64, 64, f + 2, 64, f, 64, f, 64, None, None, 0, None, None, None) == -2
-    assert lib.gpt_attention_fwd(f, f, f, f, f, None, 1, 1, 16, 48, 0, 48, 48, 48, 48, 48, 48, None, None) == -2
+    # head_dim 48 is not supported; 3 query heads cannot share 2 key/value heads
+    assert lib.gpt_attention_fwd(f, f, f, f, f, None, 1, 1, 1, 16, 48, 0, 48, 48, 48, 48, 48, 48, 48, 48, 48,
+                                 None, None) == -2
+    assert lib.gpt_attention_fwd(f, f, f, f, f, None, 1, 3, 2, 16, 64, 0, 64, 64, 64, 64, 64, 64, 64, 64, 64,
+                                 None, None) == -1
     assert lib.gpt_rmsnorm_fwd(None, f, f, 4, 64, None) == -1
     assert lib.gpt_embedding_bwd(f, f, f, 16, 64, 70000, f, None) == -2
 

@@ -217,33 +217,38 @@ def test_rope_qknorm_fwd_bwd(B, T, H, Dh):
             assert_close_rel(gd[b, :, part], ref, rel=1e-2, what=f"bwd part {part}")
 
 
-@pytest.mark.parametrize("B,T,H,Dh", [(1, 130, 2, 128), (2, 64, 3, 64), (1, 96, 4, 32)])
-def test_qkv_proj_rope_matches_gemm_then_rope(B, T, H, Dh):
-    """The fused projection + RoPE + QK-norm equals the oracle's rope/rmsnorm of r·W_qkvᵀ."""
-    rng = np.random.default_rng(B + T + H + Dh)
-    d = H * Dh
+@pytest.mark.parametrize("B,T,H,Hkv,Dh", [(1, 130, 2, 2, 128), (2, 64, 3, 3, 64), (1, 96, 4, 4, 32),
+                                          (2, 70, 4, 2, 64), (1, 130, 6, 1, 128)])
+def test_qkv_proj_rope_matches_gemm_then_rope(B, T, H, Hkv, Dh):
+    """The fused projection + RoPE + QK-norm equals the oracle's rope/rmsnorm of r·W_qkvᵀ; with
+    grouped key/value heads (Hkv < H) the k and v blocks have Hkv heads."""
+    rng = np.random.default_rng(B + T + H + Dh + Hkv)
+    d, dkv = H * Dh, Hkv * Dh
     r = randn(rng, B * T, d)
-    w = randn(rng, 3 * d, d, scale=0.05)
+    w = randn(rng, d + 2 * dkv, d, scale=0.05)
     cs = torch.empty(T * Dh, dtype=torch.float32, device="cuda")
     S.rope_table(cs, T, Dh)
-    heads = torch.zeros(3, B, H, T, Dh, dtype=torch.bfloat16, device="cuda")
+    heads = torch.zeros(B * T * (d + 2 * dkv), dtype=torch.bfloat16, device="cuda")
     rq = torch.zeros(B * T * H, dtype=torch.float32, device="cuda")
-    rk = torch.zeros_like(rq)
-    S.qkv_proj_rope(bf16_tensor(r), bf16_tensor(w), heads, rq, rk, cs, B, T, H, Dh)
+    rk = torch.zeros(B * T * Hkv, dtype=torch.float32, device="cuda")
+    S.qkv_proj_rope(bf16_tensor(r), bf16_tensor(w), heads, rq, rk, cs, B, T, H, Dh, H_kv=Hkv)
     torch.cuda.synchronize()
-    qkv = (r @ w.T).reshape(B, T, 3, H, Dh)
+    qkv = r @ w.T
     cos, sin = O.rope_angles(T, Dh, np.float64)
-    got = to_np(heads)  # [3, B, H, T, Dh]
-    for b in range(B):
-        for part in range(3):
-            x = qkv[b, :, part]  # [T, H, Dh]
-            if part < 2:
-                ref, rho = O.rmsnorm(O.rope(x, cos, sin))
-                r_got = to_np(rq if part == 0 else rk).reshape(B, T, H)[b]
+    flat = to_np(heads)
+    parts = [(0, H, qkv[:, :d]), (B * H * T * Dh, Hkv, qkv[:, d:d + dkv]),
+             (B * (H + Hkv) * T * Dh, Hkv, qkv[:, d + dkv:])]
+    for pi, (base, nh, src) in enumerate(parts):
+        got = flat[base:base + B * nh * T * Dh].reshape(B, nh, T, Dh)
+        x = src.reshape(B, T, nh, Dh)
+        for b in range(B):
+            if pi < 2:
+                ref, rho = O.rmsnorm(O.rope(x[b], cos, sin))
+                r_got = to_np(rq if pi == 0 else rk).reshape(B, T, nh)[b]
                 np.testing.assert_allclose(r_got, rho[..., 0], rtol=2e-2)
             else:
-                ref = x
-            assert_close_rel(got[part, b].transpose(1, 0, 2), ref, rel=2e-2, what=f"part {part}")
+                ref = x[b]
+            assert_close_rel(got[b].transpose(1, 0, 2), ref, rel=2e-2, what=f"part {pi}")
 
 
 # --------------------------------------------------------------------------------------------------
@@ -294,6 +299,36 @@ def test_attention_fwd_bwd(B, H, T, Dh, window, qk_norm):
     # Absolute floor: O is stored in bf16 (relative rounding 2^-9), so delta = rowsum(dO∘O) and
     # hence dS carry ~2^-9·|dO·v| ≈ 2^-9·√Dh of noise even where the exact dq is 0 (T = 1).
     floor = 2.0 ** -9 * math.sqrt(Dh)
+    assert_close_rel(to_np(dq), dq_ref, rel=3e-2, cos=0.999, what="dq", atol=floor)
+    assert_close_rel(to_np(dk), dk_ref, rel=3e-2, cos=0.999, what="dk", atol=floor)
+    assert_close_rel(to_np(dv), dv_ref, rel=3e-2, cos=0.999, what="dv", atol=floor)
+
+
+@pytest.mark.parametrize("B,H,Hkv,T,Dh,window", [(2, 4, 2, 150, 64, 0), (1, 6, 1, 257, 128, 64),
+                                                (1, 8, 2, 300, 128, 0)])
+def test_attention_grouped_query_heads(B, H, Hkv, T, Dh, window):
+    """Query head h reads key/value head h / (H/Hkv); dk, dv sum over each group's query heads."""
+    rng = np.random.default_rng(B + H + Hkv + T + Dh)
+    q, do = (randn(rng, B, H, T, Dh) for _ in range(2))
+    k, v = (randn(rng, B, Hkv, T, Dh) for _ in range(2))
+    o_ref, lse_ref = O.attention_batch_forward(q, k, v, window)
+    dq_ref, dk_ref, dv_ref = O.attention_batch_backward(q, k, v, do, window)
+    tq, tk, tv, tdo = (bf16_tensor(a) for a in (q, k, v, do))
+    sq, skv = (H * T * Dh, T * Dh, Dh), (Hkv * T * Dh, T * Dh, Dh)
+    to = torch.zeros(B, H, T, Dh, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
+    st = _status()
+    S.attention_fwd(tq, tk, tv, to, lse, window, sq, sq, B, H, T, Dh, status=st, H_kv=Hkv, strides_kv=skv)
+    dq = torch.zeros_like(tq)
+    dk, dv = torch.zeros_like(tk), torch.zeros_like(tv)
+    delta = S.attention_bwd_scratch(B, H, T)
+    S.attention_bwd(tq, tk, tv, to, tdo, lse, delta, dq, dk, dv, window, sq, sq, B, H, T, Dh, status=st,
+                    H_kv=Hkv, strides_kv=skv)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    floor = 2.0 ** -9 * math.sqrt(Dh)
+    assert_close_rel(to_np(to), o_ref, rel=2e-2, cos=0.9999, what="o")
+    np.testing.assert_allclose(to_np(lse), lse_ref, atol=2e-3)
     assert_close_rel(to_np(dq), dq_ref, rel=3e-2, cos=0.999, what="dq", atol=floor)
     assert_close_rel(to_np(dk), dk_ref, rel=3e-2, cos=0.999, what="dk", atol=floor)
     assert_close_rel(to_np(dv), dv_ref, rel=3e-2, cos=0.999, what="dv", atol=floor)

@@ -77,6 +77,18 @@ def test_step_small_bf16_configs(T, windows, dh):
     compare(cfg, loss, g, ref)
 
 
+@pytest.mark.parametrize("d,dh,kv,T,windows", [(256, 64, 2, 130, [40, 0]), (512, 128, 1, 200, [0, 77]),
+                                                (384, 64, 3, 96, [0, 0])])
+def test_step_grouped_query_attention(d, dh, kv, T, windows):
+    """Grouped-query attention (kv key/value heads shared by consecutive query heads) through the
+    whole step, against the oracle's grouped attention."""
+    cfg = custom(2, d, dh, 512, T, 2, windows=windows, n_kv_heads=kv)
+    params, tokens, targets = make_config_inputs(cfg)
+    loss, g, _ = run_gpu(cfg, params, tokens, targets)
+    ref = O.step(cfg, params.astype(np.float64), tokens, targets, dtype=np.float64)
+    compare(cfg, loss, g, ref)
+
+
 def test_step_all_targets_ignored():
     cfg = custom(1, 64, 32, 256, 16, 1)
     params, tokens, targets = make_config_inputs(cfg)
