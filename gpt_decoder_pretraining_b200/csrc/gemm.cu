@@ -48,10 +48,9 @@ enum : int {
 };
 
 // TMA warp, MMA warp, then 4 epilogue warps per column group (one per TMEM lane quarter).  Two
-// column groups halve the epilogue time of a tile; the QKV + RoPE epilogue keeps one group, since it
-// holds a whole head per thread and more threads would leave it too few registers.
+// column groups halve the epilogue time of a tile.
 template <int EPI>
-constexpr int gemm_col_groups() { return EPI > EPI_QKV_ROPE ? 1 : 2; }
+constexpr int gemm_col_groups() { return 2; }
 template <int EPI>
 constexpr int gemm_threads() { return 64 + 128 * gemm_col_groups<EPI>(); }
 
@@ -588,59 +587,97 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
         }
       }
       if constexpr (EPI > EPI_QKV_ROPE) {
-        // one head (DH columns) at a time: q and k heads get RoPE + QK-norm, v heads a plain cast
+        // one head (DH columns) at a time: q and k heads get RoPE + QK-norm, v heads a plain cast.
+        // Two passes over tensor memory keep at most 64 values per thread in registers: the sum of
+        // squares first (rotation preserves it), then the rotation pairs (j, j + DH/2) 32 at a time.
         constexpr int DH = EPI - EPI_QKV_ROPE, HALF = DH / 2;
         const long long btd = (long long)(args.M / args.T) * args.T * DH;  // one head of all rows
         const int dkv = args.Hkv * DH;
         const int b = m / args.T, t = m % args.T;
+        const bool row_ok = m < args.M;
 #pragma unroll 1
         for (int hh = half * (BN / DH / G); hh < (half + 1) * (BN / DH / G); ++hh) {
           const int n_head = tn * BN + hh * DH;
-          float xh[DH];
-#pragma unroll
-          for (int c = 0; c < DH / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + hh * DH + c * 32, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) xh[c * 32 + j] = __uint_as_float(r[j]);
-          }
-          if (m >= args.M || n_head >= args.N) continue;
+          if (n_head >= args.N) continue;  // the same for every lane of the warp
+          const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + hh * DH;
           // columns: q (H heads) | k (Hkv heads) | v (Hkv heads)
           const int region = n_head < args.d ? 0 : (n_head < args.d + dkv ? 1 : 2);
           const int h = (n_head - (region == 0 ? 0 : args.d + (region - 1) * dkv)) / DH;
           const int nh = region == 0 ? args.H : args.Hkv;  // heads of this region
-          if (region < 2) {
-            const float4* cs4 = reinterpret_cast<const float4*>(args.cs + (size_t)t * DH);
-            float ss = 0.f;
-#pragma unroll
-            for (int j = 0; j < HALF; j += 2) {
-              const float4 w = cs4[j / 2];  // cos_j, sin_j, cos_{j+1}, sin_{j+1}
-              const float a0 = xh[j], b0 = xh[j + HALF], a1 = xh[j + 1], b1 = xh[j + 1 + HALF];
-              xh[j] = a0 * w.x - b0 * w.y;
-              xh[j + HALF] = a0 * w.y + b0 * w.x;
-              xh[j + 1] = a1 * w.z - b1 * w.w;
-              xh[j + 1 + HALF] = a1 * w.w + b1 * w.z;
-              ss += xh[j] * xh[j] + xh[j + HALF] * xh[j + HALF] + xh[j + 1] * xh[j + 1] +
-                    xh[j + 1 + HALF] * xh[j + 1 + HALF];
-            }
-            const float rr = rsqrtf(ss / (float)DH + 1e-6f);
-#pragma unroll
-            for (int j = 0; j < DH; ++j) xh[j] *= rr;
-            (region == 0 ? args.rho_q : args.rho_k)[(size_t)m * nh + h] = rr;
-          }
           // q at 0, k after the H query heads, v after the Hkv key heads: [B][heads][T][DH] each
           const long long base = region == 0 ? 0 : btd * (args.H + (long long)(region - 1) * args.Hkv);
           uint16_t* dst = reinterpret_cast<uint16_t*>(args.C) + base +
                           (((long long)b * nh + h) * args.T + t) * DH;
+          auto store32 = [&](int col, const float* w) {
+            if (!row_ok) return;
 #pragma unroll
-          for (int j = 0; j < DH; j += 8) {
-            uint4 o;
-            o.x = pack_bf2(xh[j], xh[j + 1]);
-            o.y = pack_bf2(xh[j + 2], xh[j + 3]);
-            o.z = pack_bf2(xh[j + 4], xh[j + 5]);
-            o.w = pack_bf2(xh[j + 6], xh[j + 7]);
-            *reinterpret_cast<uint4*>(dst + j) = o;
+            for (int j = 0; j < 32; j += 8) {
+              uint4 o;
+              o.x = pack_bf2(w[j], w[j + 1]);
+              o.y = pack_bf2(w[j + 2], w[j + 3]);
+              o.z = pack_bf2(w[j + 4], w[j + 5]);
+              o.w = pack_bf2(w[j + 6], w[j + 7]);
+              *reinterpret_cast<uint4*>(dst + col + j) = o;
+            }
+          };
+          if (region == 2) {
+#pragma unroll 1
+            for (int c = 0; c < DH / 32; ++c) {
+              uint32_t r[32];
+              tmem_ld32(tb + 32 * c, r);
+              tmem_ld_wait();
+              store32(32 * c, reinterpret_cast<const float*>(r));
+            }
+            continue;
+          }
+          float ss = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < DH / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tb + 32 * c, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ss = fmaf(__uint_as_float(r[j]), __uint_as_float(r[j]), ss);
+          }
+          const float rr = rsqrtf(ss / (float)DH + 1e-6f);
+          if (row_ok) (region == 0 ? args.rho_q : args.rho_k)[(size_t)m * nh + h] = rr;
+          const float4* cs4 = reinterpret_cast<const float4*>(args.cs + (size_t)(row_ok ? t : 0) * DH);
+          constexpr int PC = HALF < 32 ? HALF : 32;  // rotation pairs per pass
+#pragma unroll 1
+          for (int p0 = 0; p0 < HALF; p0 += PC) {
+            uint32_t ra[32], rb[32];
+            float wa[32], wb[32];
+            if constexpr (HALF >= 32) {
+              tmem_ld32(tb + p0, ra);
+              tmem_ld32(tb + HALF + p0, rb);
+            } else {
+              tmem_ld32(tb, ra);  // DH = 32: one load holds both halves
+#pragma unroll
+              for (int j = 0; j < PC; ++j) rb[j] = ra[HALF + j];
+            }
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < PC; j += 2) {
+              const float4 w = cs4[(p0 + j) / 2];  // cos_j, sin_j, cos_{j+1}, sin_{j+1}
+              const float a0 = __uint_as_float(ra[j]), b0 = __uint_as_float(rb[j]);
+              const float a1 = __uint_as_float(ra[j + 1]), b1 = __uint_as_float(rb[j + 1]);
+              wa[j] = (a0 * w.x - b0 * w.y) * rr;
+              wb[j] = (a0 * w.y + b0 * w.x) * rr;
+              wa[j + 1] = (a1 * w.z - b1 * w.w) * rr;
+              wb[j + 1] = (a1 * w.w + b1 * w.z) * rr;
+            }
+            if constexpr (HALF >= 32) {
+              store32(p0, wa);
+              store32(HALF + p0, wb);
+            } else {
+              float wf[32];
+#pragma unroll
+              for (int j = 0; j < PC; ++j) {
+                wf[j] = wa[j];
+                wf[HALF + j] = wb[j];
+              }
+              store32(0, wf);
+            }
           }
         }
       } else {
