@@ -1378,14 +1378,6 @@ __global__ void attn_kmax_kernel(const uint16_t* __restrict__ k, float* __restri
 // ================================================================================================
 // backward (1): delta = rowsum(dO ∘ O), LSE·log2 e and the extension rows, Dh/8 lanes per row
 // ================================================================================================
-// v as hi + mid + lo in bf16 (each a round-to-nearest-even of the remainder): ~24 significant bits
-__device__ __forceinline__ uint2 split3_bf16(float v) {
-  const uint16_t hi = f2bf(v);
-  const float r1 = v - bf2f(hi);
-  const uint16_t mid = f2bf(r1);
-  const uint16_t lo = f2bf(r1 - bf2f(mid));
-  return make_uint2((uint32_t)hi | ((uint32_t)mid << 16), (uint32_t)lo);
-}
 
 __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                                   const float* __restrict__ lse, float* __restrict__ pad,
@@ -1893,8 +1885,9 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
                          void* dv, int B, int H, int Hkv, int T, int Dh, int window, HeadLayout lq,
                          HeadLayout lkv, HeadLayout ldq, HeadLayout ldkv, HeadLayout lo,
                          HeadLayout ldo, int* status, cudaStream_t stream, const float* rho_q,
-                         const float* rho_k, const float* cos_sin, bool store_ds) {
+                         const float* rho_k, const float* cos_sin, bool store_ds, bool delta_ready) {
   if (Hkv <= 0 || H % Hkv) return GPT_ERR_INVALID_ARG;
+  if (delta_ready && (T % 64)) return GPT_ERR_INVALID_ARG;  // padded rows are the delta pass's job
   if (Dh == 32 && Hkv != H) return GPT_ERR_UNSUPPORTED_SHAPE;  // the head_dim-32 path is per head
   GPT_TRY(check_attn(q, B, H, T, Dh, lq.sb, lq.sh, lq.st));
   GPT_TRY(check_attn(k, B, Hkv, T, Dh, lkv.sb, lkv.sh, lkv.st));
@@ -1928,7 +1921,7 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
         !encode_map_bf16(&mext, ext, 2, dims, strides, box, false))
       return GPT_ERR_UNSUPPORTED_SHAPE;
   }
-  {
+  if (!delta_ready) {  // else the GEMM that produced dO has written these rows
     const int threads = 256;
     const long long blocks = (rows * (Dh / 8) + threads - 1) / threads;
     GPT_TRY(launch_kernel(attn_delta_kernel, dim3((unsigned)blocks), dim3(threads), 0, stream,
@@ -2021,7 +2014,7 @@ gpt_status attention_bwd_noalloc(const void* q, const void* k, const void* v, co
   GPT_TRY(noalloc_delta_ptr(&delta));
   const HeadLayout lq{sbq, shq, stq}, lo{sbo, sho, sto};
   return attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, H, T, Dh, window, lq, lq, lq, lq,
-                       lo, lo, status, stream, nullptr, nullptr, nullptr, false);
+                       lo, lo, status, stream, nullptr, nullptr, nullptr, false, false);
 }
 
 }  // namespace gpt
@@ -2047,7 +2040,7 @@ extern "C" gpt_status gpt_attention_bwd(const void* q, const void* k, const void
   const gpt::HeadLayout lq{sb_q, sh_q, st_q}, lkv{sb_kv, sh_kv, st_kv}, lo{sb_o, sh_o, st_o};
   return gpt::attention_bwd(q, k, v, o, dout, lse, delta, dq, dk, dv, B, H, H_kv, T, Dh, window, lq,
                             lkv, lq, lkv, lo, lo, status, gpt::as_stream(stream), nullptr, nullptr,
-                            nullptr, true);
+                            nullptr, true, false);
 }
 
 extern "C" size_t gpt_attention_bwd_scratch_bytes(int B, int H, int T) {

@@ -141,6 +141,17 @@ struct GemmArgs {
   const float* cs;        // [T, Dh/2, 2] cos / sin
   float* rho_q;           // [M, H]
   float* rho_k;
+  // EPI_BF16_HEADS (optional, dl_pad != null): the attention backward's per-row scratch for the
+  // dO just stored — delta = rowsum(dO∘O) from the bf16-rounded dO, LSE·log2 e, and the two bf16
+  // extension rows — at row (b·H + h)·Tpad + t of [2][B·H·Tpad]
+  const uint16_t* dl_o;   // o, token-major: (b, h, t, j) at b·dl_sb + h·Dh + t·dl_st + j
+  long long dl_sb, dl_st;
+  const float* dl_lse;    // [B, H, T]
+  float* dl_pad;
+  uint16_t* dl_ext;       // may be null
+  int dl_Tpad;
+  long long dl_rows;      // B·H·Tpad
+  float dl_ext_scale;     // √Dh
 };
 
 struct GemmShape {
@@ -151,6 +162,8 @@ struct GemmShape {
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
 };
+
+__device__ __forceinline__ bool j0_end_of_head(int n0, int Dh) { return (n0 % Dh) + 32 == Dh; }
 
 // ------------------------------------------------------------------------------------------------
 // epilogue: one thread owns row m, columns n0 .. n0+31 of the tile (32 fp32 values in v)
@@ -681,6 +694,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
           }
         }
       } else {
+      float dl_dot = 0.f;  // EPI_BF16_HEADS with the fused delta: rowsum(dO∘O) of the current head
 #pragma unroll 1
       for (int c = half * (BN / 32 / G); c < (half + 1) * (BN / 32 / G); ++c) {
         uint32_t r[32];
@@ -723,6 +737,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
             const int b = m / args.T, t = m % args.T, h = n0 / args.Dh, j0 = n0 % args.Dh;
             uint16_t* dst = reinterpret_cast<uint16_t*>(args.C) +
                             (((long long)b * args.H + h) * args.T + t) * args.Dh + j0;
+            const uint16_t* orow = args.dl_pad ? args.dl_o + b * args.dl_sb + (long long)h * args.Dh +
+                                                     (long long)t * args.dl_st + j0
+                                               : nullptr;
 #pragma unroll
             for (int j = 0; j < 32; j += 8) {
               uint4 o;
@@ -731,8 +748,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
               o.z = pack_bf2(v[j + 4], v[j + 5]);
               o.w = pack_bf2(v[j + 6], v[j + 7]);
               *reinterpret_cast<uint4*>(dst + j) = o;
+              if (orow) {  // delta from the dO values as stored
+                const uint4 x = *reinterpret_cast<const uint4*>(orow + j);
+                dl_dot += bf_lo(o.x) * bf_lo(x.x) + bf_hi(o.x) * bf_hi(x.x) + bf_lo(o.y) * bf_lo(x.y) +
+                          bf_hi(o.y) * bf_hi(x.y) + bf_lo(o.z) * bf_lo(x.z) + bf_hi(o.z) * bf_hi(x.z) +
+                          bf_lo(o.w) * bf_lo(x.w) + bf_hi(o.w) * bf_hi(x.w);
+              }
+            }
+            if (orow && j0 + 32 == args.Dh) {  // the head's last chunk: its scratch row
+              const long long r = ((long long)b * args.H + h) * args.dl_Tpad + t;
+              const float l = args.dl_lse[((long long)b * args.H + h) * args.T + t];
+              args.dl_pad[r] = l * 1.4426950408889634f;
+              args.dl_pad[args.dl_rows + r] = dl_dot;
+              if (args.dl_ext) {
+                const uint2 el = split3_bf16(-l * args.dl_ext_scale);
+                const uint2 ed = split3_bf16(-dl_dot);
+                *reinterpret_cast<uint4*>(args.dl_ext + r * 8) = make_uint4(el.x, el.y, 0, 0);
+                *reinterpret_cast<uint4*>(args.dl_ext + (args.dl_rows + r) * 8) = make_uint4(ed.x, ed.y, 0, 0);
+              }
             }
           }
+          if (j0_end_of_head(n0, args.Dh)) dl_dot = 0.f;
         } else {
           if (m < args.M && n0 < args.N) epilogue_store<EPI>(args, 0, m, n0, v);
         }
@@ -989,7 +1025,7 @@ gpt_status gemm_e4m3_launch(int M, int N, int K, const void* A, int lda, const v
 
 gpt_status gemm_heads_launch(int op, int M, int N, int K, const void* A, int lda, const void* B,
                              int ldb, void* heads, int T, int H, int Dh, int* status,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, const AttnDeltaFusion* fuse) {
   GPT_TRY(check_gemm_args(op, M, N, K, A, lda, B, ldb, heads, N));
   if (T <= 0 || H <= 0 || Dh <= 0 || (Dh % 32) || H * Dh != N || (M % T)) return GPT_ERR_INVALID_ARG;
   const bool a_mn = (op == GPT_GEMM_TN), b_mn = (op != GPT_GEMM_NT);
@@ -1000,6 +1036,15 @@ gpt_status gemm_heads_launch(int op, int M, int N, int K, const void* A, int lda
   GPT_TRY(fill_args(a, M, N, K));
   a.C = heads; a.ldc = N; a.status = status;
   a.T = T; a.H = H; a.Dh = Dh;
+  if (fuse) {
+    if (!fuse->o || !fuse->lse || !fuse->pad || fuse->Tpad < T) return GPT_ERR_INVALID_ARG;
+    a.dl_o = reinterpret_cast<const uint16_t*>(fuse->o);
+    a.dl_sb = fuse->sb_o; a.dl_st = fuse->st_o;
+    a.dl_lse = fuse->lse; a.dl_pad = fuse->pad;
+    a.dl_ext = reinterpret_cast<uint16_t*>(fuse->ext);
+    a.dl_Tpad = fuse->Tpad; a.dl_rows = (long long)(M / T) * H * fuse->Tpad;
+    a.dl_ext_scale = sqrtf((float)Dh);
+  }
   if (op == GPT_GEMM_NT) return launch_inst<false, false, EPI_BF16_HEADS>(ma, mb, a, stream);
   if (op == GPT_GEMM_NN) return launch_inst<false, true, EPI_BF16_HEADS>(ma, mb, a, stream);
   return launch_inst<true, true, EPI_BF16_HEADS>(ma, mb, a, stream);

@@ -126,10 +126,22 @@ gpt_status gemm_ce_launch(bool grad, int M, int N, int K, const void* A, int lda
                           cudaStream_t stream);
 int gemm_ce_tile_n();  // vocabulary columns per CE statistics tile
 
+// The attention backward's per-row scratch, computed in the epilogue of the GEMM that produces dO
+// (so that the backward skips its own pass over O and dO): o token-major (b, h, t, j) at
+// b·sb_o + h·Dh + t·st_o + j; lse [B, H, T]; pad = the scratch (fp32 [2][B·H·Tpad]); ext its bf16
+// extension rows (or null).  Only for T a multiple of 64 (no zero-padded rows to fill).
+struct AttnDeltaFusion {
+  const void* o;
+  long long sb_o, st_o;
+  const float* lse;
+  float* pad;
+  void* ext;
+  int Tpad;
+};
 // C (row m = b·T + t, column n = h·Dh + j) stored bf16 head-major at heads[((b·H + h)·T + t)·Dh + j].
 gpt_status gemm_heads_launch(int op, int M, int N, int K, const void* A, int lda, const void* B,
                              int ldb, void* heads, int T, int H, int Dh, int* status,
-                             cudaStream_t stream);
+                             cudaStream_t stream, const AttnDeltaFusion* fuse = nullptr);
 // [q|k|v] = A·W_qkvᵀ with RoPE + QK-norm applied to q and k, stored head-major: q [B][H][T][Dh],
 // then k and v [B][Hkv][T][Dh] (Hkv ≤ 0: H); rho_q [M, H] / rho_k [M, Hkv] receive the norm factors.
 gpt_status gemm_qkv_rope_launch(int M, int d, const void* A, const void* Wqkv, void* heads,

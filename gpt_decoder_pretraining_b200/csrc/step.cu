@@ -49,7 +49,7 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
                          void* dv, int B, int H, int Hkv, int T, int Dh, int window, HeadLayout lq,
                          HeadLayout lkv, HeadLayout ldq, HeadLayout ldkv, HeadLayout lo,
                          HeadLayout ldo, int* status, cudaStream_t stream, const float* rho_q,
-                         const float* rho_k, const float* cos_sin, bool store_ds);
+                         const float* rho_k, const float* cos_sin, bool store_ds, bool delta_ready);
 
 static inline size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
 
@@ -367,6 +367,9 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
   uint16_t* dO = reinterpret_cast<uint16_t*>(ws + p.dO);
   uint16_t* dqkv = reinterpret_cast<uint16_t*>(ws + p.dqkv);
   float* delta = reinterpret_cast<float*>(ws + p.delta);
+  // the delta rows come from the dO GEMM's epilogue when no row of the scratch is padding
+  const bool fuse_delta = (T % 64) == 0;
+  void* delta_ext = (Dh != 32) ? (void*)(delta + 2 * (size_t)B * H * T) : nullptr;
   for (int l = c.depth - 1; l >= 0; --l) {
     const int wq = 1 + 4 * l;
     uint16_t* r1 = reinterpret_cast<uint16_t*>(at(p.r1, l));
@@ -390,15 +393,18 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
                         nullptr, 0, status, s, sk));
     PROF(PROF_NORM, 0, 14.0 * (double)M * d, rmsnorm_bwd(dr, 0, r2, rho2, gx, gxb, 1, M, d, s));
     // attention
+    // dO head-major; its epilogue also forms the attention backward's delta rows (T % 64 == 0)
+    AttnDeltaFusion fuse{o, os_b, os_t, lse, delta, delta_ext, T, };
     PROF(PROF_GEMM, gemm_flops(M, d, d), 0,
-         gemm_heads_launch(GPT_GEMM_NN, M, d, d, gxb, d, W(wq + 1), d, dO, T, H, Dh, status, s));
+         gemm_heads_launch(GPT_GEMM_NN, M, d, d, gxb, d, W(wq + 1), d, dO, T, H, Dh, status, s,
+                           fuse_delta ? &fuse : nullptr));
     PROF(PROF_GEMM, gemm_flops(d, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, d, d, M, gxb, d, o, d, G(wq + 1), d, nullptr,
                         nullptr, 0, status, s, sk));
     PROF(PROF_ATTN_BWD, 8.0 * Dh * H * B * attn_pairs(T, st->window[l]), 0,
          attention_bwd(qkv, qkv + bhtd, qkv + bhtd + bhktd, o, dO, lse, delta, dqkv, dqkv + d,
                        dqkv + d + dkv, B, H, Hkv, T, Dh, st->window[l], lay_q, lay_kv, lay_dqkv,
                        lay_dqkv, lay_o, lay_q, status, s, Dh == 32 ? nullptr : rq, rk, rope,
-                       true));
+                       true, fuse_delta));
     if (Dh == 32) {  // the mma.sync path for head_dim 32 has no fused QK-norm/RoPE backward
       PROF(PROF_ROPE, 0, 12.0 * (double)M * d,
            rope_qknorm_bwd_heads(dqkv, qkv, rq, rk, rope, B, T, H, Dh, s));

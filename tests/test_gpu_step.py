@@ -66,7 +66,8 @@ def test_step_smoke_config():
     compare(cfg, loss, g, ref)
 
 
-@pytest.mark.parametrize("T,windows,dh", [(100, [33, 0], 64), (129, [1, 200], 128), (64, [0, 0], 32)])
+@pytest.mark.parametrize("T,windows,dh", [(100, [33, 0], 64), (129, [1, 200], 128), (64, [0, 0], 32),
+                                          (192, [0, 50], 128), (128, [70, 0], 64)])
 def test_step_small_bf16_configs(T, windows, dh):
     cfg = custom(2, 2 * dh, dh, 512, T, 2, windows=windows)
     params, tokens, targets = make_config_inputs(cfg)
