@@ -358,14 +358,22 @@ struct MuonGroup {
 };
 
 // The pages' grouping: per layer the q, k, v row blocks of W_qkv and W_o (four d×d matrices, each
-// layer's four contiguous), then every W_fc (F×d), then every W_proj (d×F).
+// layer's four contiguous), then every W_fc (F×d), then every W_proj (d×F).  With grouped
+// key/value heads, k and v are (n_kv_heads·Dh)×d: q, the k/v pair and W_o form three groups.
 std::vector<MuonGroup> muon_groups(const gpt_config* cfg, const size_t* off) {
   std::vector<MuonGroup> out;
   const int L = cfg->depth;
   if (L <= 0) return out;
   const long long stride = L > 1 ? (long long)(off[1 + 4] - off[1]) : 0;
   const int d = cfg->d_model, F = cfg->d_mlp;
-  out.push_back({off[1], L, 4, stride, d, d});
+  const int kv = (cfg->n_kv_heads > 0 ? cfg->n_kv_heads : cfg->n_heads) * cfg->head_dim;
+  if (kv == d) {
+    out.push_back({off[1], L, 4, stride, d, d});
+  } else {
+    out.push_back({off[1], L, 1, stride, d, d});
+    out.push_back({off[1] + (size_t)d * d, L, 2, stride, kv, d});
+    out.push_back({off[1 + 1], L, 1, stride, d, d});
+  }
   out.push_back({off[1 + 2], L, 1, stride, F, d});
   out.push_back({off[1 + 3], L, 1, stride, d, F});
   return out;

@@ -87,12 +87,15 @@ def muon_matrices(cfg) -> Dict[str, Tuple[int, int, int]]:
     """Muon's matrices as (offset into the flat packing, rows, cols): per layer q, k, v (the three
     row blocks of W_qkv), o, fc, proj — the grouping the pages print."""
     d, F, V = cfg.d_model, cfg.d_mlp, cfg.vocab
+    # with grouped key/value heads the k and v row blocks of W_qkv have kv_heads·Dh rows
+    kv = getattr(cfg, "kv_heads", cfg.n_heads) * cfg.head_dim
     out = {}
     off = V * d
     for l in range(cfg.depth):
-        for j, name in enumerate("qkv"):
-            out[f"h{l}.w_{name}"] = (off + j * d * d, d, d)
-        off += 3 * d * d
+        out[f"h{l}.w_q"] = (off, d, d)
+        out[f"h{l}.w_k"] = (off + d * d, kv, d)
+        out[f"h{l}.w_v"] = (off + d * d + kv * d, kv, d)
+        off += (d + 2 * kv) * d
         out[f"h{l}.w_o"] = (off, d, d)
         off += d * d
         out[f"h{l}.w_fc"] = (off, F, d)

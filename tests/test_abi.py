@@ -277,3 +277,88 @@ def test_noalloc_attention_backward_row_limit_needs_no_device(lib):
     assert call(*args(1, 3277, 33, 128)) == -2          # T = 33 pads to 64 rows per (b, h)
     assert call(*args(1, 16, 65537, 64)) == -2
     assert call(*args(0, 1, 64, 64)) == -1
+
+
+def test_sharded_optimizer_equals_the_whole_step():
+    """Two gloo ranks split the optimizer step (layers by rank, table rows in halves) and exchange
+    the results: both end with the parameters of the oracle's unsharded optimizer step."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 31500 + (os.getpid() % 1000)
+    procs = [ctx.Process(target=_shard_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = dict(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    from oracle import optim_oracle as Q
+    cfg, params, grads, hp = _shard_case()
+    state = {}
+    ref = Q.optimizer_step(cfg, params, grads, state, 1, hp)
+    ref = Q.optimizer_step(cfg, ref, grads * 0.5, state, 2, hp)
+    for r in range(2):
+        np.testing.assert_array_equal(out[r], ref)
+
+
+def _shard_case():
+    from gpt_decoder_pretraining_b200.config import custom
+    cfg = custom(3, 64, 16, 96, 8, 1, param_dtype=1)
+    rng = np.random.default_rng(4)
+    params = rng.standard_normal(cfg.n_params) * 0.02
+    grads = rng.standard_normal(cfg.n_params) * 0.1
+    hp = {"muon_lr": 0.02, "muon_momentum": 0.95, "ns_steps": 5, "ns_coeffs": (3.4445, -4.7750, 2.0315),
+          "adam_lr_wte": 0.2, "adam_lr_lm": 0.004, "beta1": 0.8, "beta2": 0.95, "eps": 1e-10,
+          "weight_decay": 0.01}
+    return cfg, params, grads, hp
+
+
+def _shard_rank_main(rank, world, port, q):
+    import sys
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from gpt_decoder_pretraining_b200 import dp
+    from oracle import optim_oracle as Q
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    cfg, params, grads, hp = _shard_case()
+    p = torch.from_numpy(params.copy())
+    state = {}
+    muon = Q.muon_matrices(cfg)
+    adam = Q.adamw_tensors(cfg)
+    d = cfg.d_model
+    opt = dp.ShardedOptimizer(cfg, world, rank)
+
+    def run(g, t):
+        def update_layers(layers, t):
+            for l in layers:
+                for name, (off, r, c) in muon.items():
+                    if not name.startswith(f"h{l}."):
+                        continue
+                    w = p.numpy()[off:off + r * c].reshape(r, c)
+                    buf = state.setdefault(name, np.zeros((r, c)))
+                    w2, state[name] = Q.muon_update(w, g[off:off + r * c].reshape(r, c), buf, hp["muon_lr"],
+                                                    hp["muon_momentum"], True, hp["ns_steps"], hp["ns_coeffs"])
+                    p.numpy()[off:off + r * c] = w2.ravel()
+
+        def update_rows(r0, r1, t):
+            scale = 1.0 / np.sqrt(d / 768.0)
+            for name, (off, V, _) in adam.items():
+                lr = (hp["adam_lr_wte"] if name == "wte" else hp["adam_lr_lm"]) * scale
+                a, b = off + r0 * d, off + r1 * d
+                m = state.setdefault(name + ".m", np.zeros(V * d))
+                v = state.setdefault(name + ".v", np.zeros(V * d))
+                w2, m2, v2 = Q.adamw_update(p.numpy()[a:b], g[a:b], m[r0 * d:r1 * d], v[r0 * d:r1 * d], t, lr,
+                                            hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
+                p.numpy()[a:b] = w2
+                m[r0 * d:r1 * d], v[r0 * d:r1 * d] = m2, v2
+
+        opt.step(p, t, update_layers, update_rows)
+
+    run(grads, 1)
+    run(grads * 0.5, 2)
+    dist.destroy_process_group()
+    q.put((rank, p.numpy().copy()))

@@ -133,9 +133,14 @@ def test_muon_group_matches_oracle(rows, cols, groups, per):
                           round_to_bf16(tw.cpu().numpy())[np.setdiff1d(np.arange(total), gap)])
 
 
-@pytest.mark.parametrize("which", ["smoke", "d12_layer"])
+@pytest.mark.parametrize("which", ["smoke", "d12_layer", "gqa"])
 def test_optim_step_matches_oracle(which):
-    cfg = preset("smoke") if which == "smoke" else custom(1, 768, 128, 32768, 2048, 16, name="d12_layer")
+    if which == "smoke":
+        cfg = preset("smoke")
+    elif which == "d12_layer":
+        cfg = custom(1, 768, 128, 32768, 2048, 16, name="d12_layer")
+    else:  # grouped key/value heads: k and v are their own Muon matrices of kv_heads·Dh rows
+        cfg = custom(2, 256, 64, 1024, 64, 2, name="gqa", n_kv_heads=2)
     n = cfg.n_params
     rng = np.random.default_rng(11)
     w0 = make_params(n, keep_fp32=True).astype(np.float64)
@@ -156,8 +161,11 @@ def test_optim_step_matches_oracle(which):
             sl = slice(off, off + a * b)
             off += a * b
             if name.endswith("w_qkv"):
-                for j in range(3):
-                    s2 = slice(sl.start + j * (a // 3) * b, sl.start + (j + 1) * (a // 3) * b)
+                kvr = cfg.kv_heads * cfg.head_dim
+                r0 = sl.start
+                for j, rows in enumerate((cfg.d_model, kvr, kvr)):
+                    s2 = slice(r0, r0 + rows * b)
+                    r0 += rows * b
                     assert_close_rel(after[s2] - before[s2], new_ref[s2] - before[s2], rel=MUON_REL,
                                      cos=MUON_COS, what=f"{name}[{j}] t={t}")
             elif name in ("wte", "w_lm"):
@@ -176,3 +184,30 @@ def test_optim_step_matches_oracle(which):
     # AdamW moments of the embedding (exact fp32 recurrences)
     V, d = cfg.vocab, cfg.d_model
     assert_close_rel(to_np(tv)[:V * d], state["wte.v"], rel=1e-5, cos=0.99999, what="wte v")
+
+
+@pytest.mark.parametrize("world", [1, 2, 3])
+def test_sharded_update_functions_cover_the_whole_step(world):
+    """The per-rank update functions of the sharded optimizer (Muon on layers l ≡ r mod world, AdamW
+    on row ranges), applied for every rank in turn on one GPU, give the same result as
+    gpt_optim_step over the whole model (no collective is needed: the shards are disjoint)."""
+    from gpt_decoder_pretraining_b200 import dp
+    cfg = custom(4, 256, 64, 1024, 64, 2, name="shard")
+    n = cfg.n_params
+    rng = np.random.default_rng(3)
+    w0 = make_params(n, keep_fp32=True)
+    g = torch.from_numpy((rng.standard_normal(n) * 0.05).astype(np.float32)).cuda()
+    ref_w, w = torch.from_numpy(w0).cuda(), torch.from_numpy(w0).cuda()
+    ref_p, p = (torch.zeros(n, dtype=torch.bfloat16, device="cuda") for _ in range(2))
+    ref_m, ref_v, m, v = (torch.zeros(n, device="cuda") for _ in range(4))
+    for t in (1, 2):
+        S.optim_step(cfg, ref_w, ref_p, g, ref_m, ref_v, t, HP)
+        ul, ur = dp.device_update_fns(cfg, w, p, g, m, v, HP, world)
+        for r, sh in dp.optimizer_shards(cfg, world).items():
+            if sh["layers"]:
+                ul(sh["layers"], t)
+            ur(*sh["rows"], t)
+    torch.cuda.synchronize()
+    assert torch.equal(w, ref_w)
+    assert torch.equal(p, ref_p)
+    assert torch.equal(m, ref_m) and torch.equal(v, ref_v)
