@@ -36,6 +36,7 @@ constexpr float LN2 = 0.6931471805599453f;
 
 struct AttnArgs {
   int B, H, T, window;  // window: effective (T for full causal)
+  int Tk, q_off;        // forward: keys, and the absolute position of query row 0 (a cache)
   int Hkv, group;       // key/value heads and query heads per key/value head (H = Hkv·group)
   float scale_log2;     // log2(e)/sqrt(Dh)
   float scale;          // 1/sqrt(Dh)
@@ -367,10 +368,10 @@ __global__ void __launch_bounds__(576, 1)
   const int warp = warp_id(), lane = lane_id();
   const int qt = gridDim.x - 1 - blockIdx.x;  // longest rows first
   const int h = blockIdx.y, b = blockIdx.z;
-  const int T = a.T, W = a.window;
+  const int T = a.T, W = a.window;  // T query rows, at absolute positions q_off .. q_off + T − 1
   const int q0 = qt * 256;
-  const int key_lo = max(0, q0 - W + 1);
-  const int key_hi = min(T, q0 + 256);
+  const int key_lo = max(0, a.q_off + q0 - W + 1);
+  const int key_hi = min(a.Tk, a.q_off + q0 + 256);
   const int kv_first = key_lo / 128;
   const int n_kv = (key_hi - 1) / 128 - kv_first + 1;
 
@@ -480,8 +481,9 @@ __global__ void __launch_bounds__(576, 1)
     const int half = (warp >> 2) & 1;
     const int quarter = warp & 3;
     const int row = 32 * quarter + lane;
-    const int t = q0 + 128 * x + row;
-    const int tile0 = q0 + 128 * x;
+    const int t = q0 + 128 * x + row;            // query row (local)
+    const int ta = a.q_off + t;                  // its position among the keys
+    const int tile0 = a.q_off + q0 + 128 * x;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const uint32_t s_addr = tmem + lane_off + S::TM_S + x * 128 + 64 * half;
     bool ok = mbar_wait_warp(bar_q, 0, abort_flag, a.status);
@@ -521,8 +523,8 @@ __global__ void __launch_bounds__(576, 1)
           }
           if (need_mask) {
             const int key = kv0 + 16 * c + 2 * e;
-            if (!(key <= t && key > t - W)) p0 = 0.f;
-            if (!(key + 1 <= t && key + 1 > t - W)) p1 = 0.f;
+            if (!(key <= ta && key > ta - W)) p0 = 0.f;
+            if (!(key + 1 <= ta && key + 1 > ta - W)) p1 = 0.f;
           }
           add2_acc(l0, l1, p0, p1);
           pk[e] = pack_bf2(p0, p1);
@@ -1829,17 +1831,22 @@ gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[
 // reads key/value head h / (H/Hkv).
 gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                          int H, int Hkv, int T, int Dh, int window, HeadLayout lq, HeadLayout lkv,
-                         HeadLayout lo, int* status, cudaStream_t stream, float* kmax_scratch) {
+                         HeadLayout lo, int* status, cudaStream_t stream, float* kmax_scratch,
+                         int Tk, int q_off) {
   if (Hkv <= 0 || H % Hkv) return GPT_ERR_INVALID_ARG;
+  if (Tk <= 0) Tk = T;
+  if (q_off < 0 || q_off + T > Tk) return GPT_ERR_INVALID_ARG;
+  if ((q_off != 0 || Tk != T) && Dh == 32) return GPT_ERR_UNSUPPORTED_SHAPE;
   GPT_TRY(check_attn(q, B, H, T, Dh, lq.sb, lq.sh, lq.st));
-  GPT_TRY(check_attn(k, B, Hkv, T, Dh, lkv.sb, lkv.sh, lkv.st));
-  GPT_TRY(check_attn(v, B, Hkv, T, Dh, lkv.sb, lkv.sh, lkv.st));
+  GPT_TRY(check_attn(k, B, Hkv, Tk, Dh, lkv.sb, lkv.sh, lkv.st));
+  GPT_TRY(check_attn(v, B, Hkv, Tk, Dh, lkv.sb, lkv.sh, lkv.st));
   GPT_TRY(check_attn(o, B, H, T, Dh, lo.sb, lo.sh, lo.st));
   if (!lse) return GPT_ERR_INVALID_ARG;
   AttnArgs a{};
   a.B = B; a.H = H; a.T = T;
+  a.Tk = Tk; a.q_off = q_off;
   a.Hkv = Hkv; a.group = H / Hkv;
-  a.window = (window > 0 && window < T) ? window : T;
+  a.window = (window > 0 && window < Tk) ? window : Tk;
   a.scale = 1.f / sqrtf((float)Dh);
   a.scale_log2 = a.scale * LOG2E;
   a.o = reinterpret_cast<uint16_t*>(o);
@@ -1857,13 +1864,13 @@ gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, f
   }
   CUtensorMap mq2, mk2, mv2;
   if (!make_head_map(&mq2, q, B, H, T, Dh, lq.sb, lq.sh, lq.st, 128) ||
-      !make_head_map(&mk2, k, B, Hkv, T, Dh, lkv.sb, lkv.sh, lkv.st, 128) ||
-      !make_head_map(&mv2, v, B, Hkv, T, Dh, lkv.sb, lkv.sh, lkv.st, 128))
+      !make_head_map(&mk2, k, B, Hkv, Tk, Dh, lkv.sb, lkv.sh, lkv.st, 128) ||
+      !make_head_map(&mv2, v, B, Hkv, Tk, Dh, lkv.sb, lkv.sh, lkv.st, 128))
     return GPT_ERR_UNSUPPORTED_SHAPE;
   const float kconst = sqrtf((float)Dh) * 1.002f;
   if (kmax_scratch) {
     GPT_TRY(launch_kernel(attn_kmax_kernel, dim3(Hkv, B), dim3(256), 0, stream,
-                          reinterpret_cast<const uint16_t*>(k), kmax_scratch, Hkv, T, Dh, lkv.sb,
+                          reinterpret_cast<const uint16_t*>(k), kmax_scratch, Hkv, Tk, Dh, lkv.sb,
                           lkv.sh, lkv.st));
   }
   if (Dh == 128) return launch_fwd_tc<128>(mq2, mk2, mv2, a, kmax_scratch, kconst, stream);
@@ -1931,6 +1938,7 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   }
   AttnArgs a{};
   a.B = B; a.H = H; a.T = T;
+  a.Tk = T; a.q_off = 0;
   a.Hkv = Hkv; a.group = H / Hkv;
   a.window = (window > 0 && window < T) ? window : T;
   a.scale = 1.f / sqrtf((float)Dh);
@@ -2027,7 +2035,7 @@ extern "C" gpt_status gpt_attention_fwd(const void* q, const void* k, const void
                                         long long st_o, int* status, void* stream) {
   return gpt::attention_fwd(q, k, v, o, lse, B, H, H_kv, T, Dh, window, {sb_q, sh_q, st_q},
                             {sb_kv, sh_kv, st_kv}, {sb_o, sh_o, st_o}, status,
-                            gpt::as_stream(stream), kmax);
+                            gpt::as_stream(stream), kmax, T, 0);
 }
 
 extern "C" gpt_status gpt_attention_bwd(const void* q, const void* k, const void* v, const void* o,

@@ -138,6 +138,11 @@ struct GemmArgs {
   CeArgs ce;
   // head-major outputs (EPI_BF16_HEADS, EPI_QKV_ROPE + Dh); Hkv key/value heads (QKV)
   int T, H, Dh, d, Hkv;
+  // QKV: destination of q, k, v — [B][heads][ts][Dh], row m = b·T + t written at position
+  // t + t_off (which is also the RoPE position); ts ≥ T + t_off (a key/value cache)
+  uint16_t* qkv_dst[3];
+  int qkv_ts[3];
+  int t_off;
   const float* cs;        // [T, Dh/2, 2] cos / sin
   float* rho_q;           // [M, H]
   float* rho_k;
@@ -604,9 +609,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
         // Two passes over tensor memory keep at most 64 values per thread in registers: the sum of
         // squares first (rotation preserves it), then the rotation pairs (j, j + DH/2) 32 at a time.
         constexpr int DH = EPI - EPI_QKV_ROPE, HALF = DH / 2;
-        const long long btd = (long long)(args.M / args.T) * args.T * DH;  // one head of all rows
         const int dkv = args.Hkv * DH;
-        const int b = m / args.T, t = m % args.T;
+        const int b = m / args.T, t = m % args.T + args.t_off;  // position
         const bool row_ok = m < args.M;
 #pragma unroll 1
         for (int hh = half * (BN / DH / G); hh < (half + 1) * (BN / DH / G); ++hh) {
@@ -617,10 +621,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
           const int region = n_head < args.d ? 0 : (n_head < args.d + dkv ? 1 : 2);
           const int h = (n_head - (region == 0 ? 0 : args.d + (region - 1) * dkv)) / DH;
           const int nh = region == 0 ? args.H : args.Hkv;  // heads of this region
-          // q at 0, k after the H query heads, v after the Hkv key heads: [B][heads][T][DH] each
-          const long long base = region == 0 ? 0 : btd * (args.H + (long long)(region - 1) * args.Hkv);
-          uint16_t* dst = reinterpret_cast<uint16_t*>(args.C) + base +
-                          (((long long)b * nh + h) * args.T + t) * DH;
+          uint16_t* dst = args.qkv_dst[region] + (((long long)b * nh + h) * args.qkv_ts[region] + t) * DH;
           auto store32 = [&](int col, const float* w) {
             if (!row_ok) return;
 #pragma unroll
@@ -653,7 +654,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
             for (int j = 0; j < 32; ++j) ss = fmaf(__uint_as_float(r[j]), __uint_as_float(r[j]), ss);
           }
           const float rr = rsqrtf(ss / (float)DH + 1e-6f);
-          if (row_ok) (region == 0 ? args.rho_q : args.rho_k)[(size_t)m * nh + h] = rr;
+          float* rho = region == 0 ? args.rho_q : args.rho_k;
+          if (row_ok && rho) rho[(size_t)m * nh + h] = rr;
           const float4* cs4 = reinterpret_cast<const float4*>(args.cs + (size_t)(row_ok ? t : 0) * DH);
           constexpr int PC = HALF < 32 ? HALF : 32;  // rotation pairs per pass
 #pragma unroll 1
@@ -1052,12 +1054,13 @@ gpt_status gemm_heads_launch(int op, int M, int N, int K, const void* A, int lda
 
 gpt_status gemm_qkv_rope_launch(int M, int d, const void* A, const void* Wqkv, void* heads,
                                 float* rho_q, float* rho_k, const float* cs, int T, int H, int Dh,
-                                int* status, cudaStream_t stream, int Hkv) {
+                                int* status, cudaStream_t stream, int Hkv, const QkvDest* dest) {
   if (Hkv <= 0) Hkv = H;
   if (H % Hkv) return GPT_ERR_INVALID_ARG;
   const int N = d + 2 * Hkv * Dh, K = d;
-  GPT_TRY(check_gemm_args(GPT_GEMM_NT, M, N, K, A, K, Wqkv, K, heads, N));
-  if (!rho_q || !rho_k || !cs || T <= 0 || H * Dh != d || (M % T)) return GPT_ERR_INVALID_ARG;
+  GPT_TRY(check_gemm_args(GPT_GEMM_NT, M, N, K, A, K, Wqkv, K, dest ? dest->q : heads, N));
+  if ((!dest && (!rho_q || !rho_k)) || !cs || T <= 0 || H * Dh != d || (M % T))
+    return GPT_ERR_INVALID_ARG;
   if (Dh != 32 && Dh != 64 && Dh != 128) return GPT_ERR_UNSUPPORTED_SHAPE;
   CUtensorMap ma, mb;
   if (!make_operand_map(&ma, A, false, M, K, K)) return GPT_ERR_UNSUPPORTED_SHAPE;
@@ -1066,6 +1069,25 @@ gpt_status gemm_qkv_rope_launch(int M, int d, const void* A, const void* Wqkv, v
   GPT_TRY(fill_args(a, M, N, K));
   a.C = heads; a.ldc = N; a.status = status;
   a.T = T; a.H = H; a.Dh = Dh; a.d = d; a.Hkv = Hkv; a.cs = cs; a.rho_q = rho_q; a.rho_k = rho_k;
+  if (dest) {
+    if (!dest->k || !dest->v || dest->q_ts < T + dest->t_off || dest->kv_ts < T + dest->t_off ||
+        dest->t_off < 0)
+      return GPT_ERR_INVALID_ARG;
+    a.qkv_dst[0] = reinterpret_cast<uint16_t*>(dest->q);
+    a.qkv_dst[1] = reinterpret_cast<uint16_t*>(dest->k);
+    a.qkv_dst[2] = reinterpret_cast<uint16_t*>(dest->v);
+    a.qkv_ts[0] = dest->q_ts;
+    a.qkv_ts[1] = a.qkv_ts[2] = dest->kv_ts;
+    a.t_off = dest->t_off;
+  } else {  // q̃, k̃, v one after the other in `heads`
+    const long long btd = (long long)(M / T) * T * Dh;
+    uint16_t* h0 = reinterpret_cast<uint16_t*>(heads);
+    a.qkv_dst[0] = h0;
+    a.qkv_dst[1] = h0 + btd * H;
+    a.qkv_dst[2] = h0 + btd * (H + Hkv);
+    a.qkv_ts[0] = a.qkv_ts[1] = a.qkv_ts[2] = T;
+    a.t_off = 0;
+  }
   if (Dh == 128) return launch_inst<false, false, EPI_QKV_ROPE + 128>(ma, mb, a, stream);
   if (Dh == 64) return launch_inst<false, false, EPI_QKV_ROPE + 64>(ma, mb, a, stream);
   return launch_inst<false, false, EPI_QKV_ROPE + 32>(ma, mb, a, stream);

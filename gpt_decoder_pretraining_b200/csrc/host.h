@@ -144,8 +144,18 @@ gpt_status gemm_heads_launch(int op, int M, int N, int K, const void* A, int lda
                              cudaStream_t stream, const AttnDeltaFusion* fuse = nullptr);
 // [q|k|v] = A·W_qkvᵀ with RoPE + QK-norm applied to q and k, stored head-major: q [B][H][T][Dh],
 // then k and v [B][Hkv][T][Dh] (Hkv ≤ 0: H); rho_q [M, H] / rho_k [M, Hkv] receive the norm factors.
+// Optional destination of the QKV projection for inference: q̃ [B][H][q_ts][Dh] and k̃, v
+// [B][Hkv][kv_ts][Dh] (a key/value cache), row m = b·T + t written at position t + t_off, which is
+// also its RoPE position.  rho_q / rho_k may then be null.
+struct QkvDest {
+  void* q;
+  void* k;
+  void* v;
+  int q_ts, kv_ts, t_off;
+};
 gpt_status gemm_qkv_rope_launch(int M, int d, const void* A, const void* Wqkv, void* heads,
                                 float* rho_q, float* rho_k, const float* cs, int T, int H, int Dh,
-                                int* status, cudaStream_t stream, int Hkv = 0);
+                                int* status, cudaStream_t stream, int Hkv = 0,
+                                const QkvDest* dest = nullptr);
 
 }  // namespace gpt

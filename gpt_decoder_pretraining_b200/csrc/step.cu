@@ -43,7 +43,8 @@ gpt_status cast_f32_bf16(const float* src, void* dst, size_t n, cudaStream_t s);
 gpt_status add_f32(float* dst, const float* src, size_t n, cudaStream_t s);
 gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                          int H, int Hkv, int T, int Dh, int window, HeadLayout lq, HeadLayout lkv,
-                         HeadLayout lo, int* status, cudaStream_t stream, float* kmax_scratch);
+                         HeadLayout lo, int* status, cudaStream_t stream, float* kmax_scratch,
+                         int Tk, int q_off);
 gpt_status attention_bwd(const void* q, const void* k, const void* v, const void* o,
                          const void* dout, const float* lse, float* delta, void* dq, void* dk,
                          void* dv, int B, int H, int Hkv, int T, int Dh, int window, HeadLayout lq,
@@ -317,7 +318,7 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
          gemm_qkv_rope_launch(M, d, r1, W(wq), qkv, rq, rk, rope, T, H, Dh, status, s, Hkv));
     PROF(PROF_ATTN_FWD, 4.0 * Dh * H * B * attn_pairs(T, st->window[l]), 0,
          attention_fwd(qkv, qkv + bhtd, qkv + bhtd + bhktd, o, lse, B, H, Hkv, T, Dh,
-                       st->window[l], lay_q, lay_kv, lay_o, status, s, nullptr));
+                       st->window[l], lay_q, lay_kv, lay_o, status, s, nullptr, T, 0));
     PROF(PROF_GEMM, gemm_flops(M, d, d), 0, gemm_launch(GPT_GEMM_NT, GPT_EPI_RESID, M, d, d, o, d, W(wq + 1), d, x, d, nullptr,
                         nullptr, 0, status, s, sk));
     PROF(PROF_NORM, 0, 4.0 * (double)M * d + 4.0 * M, rmsnorm_fwd(x, r2, rho2, M, d, s));

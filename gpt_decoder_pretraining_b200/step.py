@@ -39,6 +39,8 @@ EXPORTED = [
     "gpt_lmhead_ce_fwd_bwd", "gpt_set_wait_limit", "gpt_debug_wait_probe", "gpt_debug_exp2_poly2",
     "gpt_gemm_batched", "gpt_adamw_step", "gpt_muon_scratch_bytes", "gpt_muon_step",
     "gpt_optim_scratch_bytes", "gpt_optim_step", "gpt_gemm_e4m3", "gpt_quantize_e4m3",
+    "gpt_infer_create", "gpt_infer_destroy", "gpt_infer_workspace_bytes", "gpt_infer_kv_cache_bytes",
+    "gpt_prefill", "gpt_decode", "gpt_infer_status",
 ]
 
 
@@ -132,6 +134,15 @@ def lib():
                                      ctypes.POINTER(OptimHparams), vp, sz, vp, vp]
         L.gpt_gemm_e4m3.argtypes = [i32, i32, i32, vp, i32, vp, i32, vp, i32, vp, vp, f32, vp, vp, vp]
         L.gpt_quantize_e4m3.argtypes = [vp, ll, vp, vp, vp, vp]
+        L.gpt_infer_create.argtypes = [ctypes.POINTER(_Config), i32, i32, ctypes.POINTER(vp)]
+        L.gpt_infer_destroy.argtypes = [vp]
+        L.gpt_infer_destroy.restype = None
+        L.gpt_infer_workspace_bytes.argtypes = [vp, ctypes.POINTER(sz)]
+        L.gpt_infer_kv_cache_bytes.argtypes = [vp]
+        L.gpt_infer_kv_cache_bytes.restype = sz
+        L.gpt_prefill.argtypes = [vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
+        L.gpt_decode.argtypes = [vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
+        L.gpt_infer_status.argtypes = [vp, vp, vp]
         L.gpt_set_wait_limit.argtypes = [ll]
         L.gpt_debug_wait_probe.argtypes = [vp, vp]
         L.gpt_debug_exp2_poly2.argtypes = [vp, vp, i32, vp]
@@ -251,6 +262,59 @@ class GptStep:
         by = (ctypes.c_double * n)()
         _check(lib().gpt_step_profile(self._h, ms, calls, fl, by, n), "gpt_step_profile")
         return {c: (ms[i], int(calls[i]), fl[i], by[i]) for i, c in enumerate(PROFILE_CLASSES)}
+
+
+class GptInfer:
+    """Forward-only inference with a KV cache: ``logits = infer.prefill(params, tokens)`` fills
+    positions 0..T−1, ``logits = infer.decode(params, tokens, pos)`` one more position."""
+
+    def __init__(self, cfg: GptConfig, max_batch: int, max_len: int, device=None):
+        import torch
+        self.cfg = cfg
+        c, self._win = _cconfig(cfg)
+        h = ctypes.c_void_p()
+        _check(lib().gpt_infer_create(ctypes.byref(c), max_batch, max_len, ctypes.byref(h)), "gpt_infer_create")
+        self._h = h
+        nbytes = ctypes.c_size_t(0)
+        _check(lib().gpt_infer_workspace_bytes(h, ctypes.byref(nbytes)), "gpt_infer_workspace_bytes")
+        self.device = torch.device(device or "cuda")
+        self.workspace = torch.empty(int(nbytes.value), dtype=torch.uint8, device=self.device)
+        self.kv_cache = torch.zeros(int(lib().gpt_infer_kv_cache_bytes(h)) // 2, dtype=torch.bfloat16,
+                                    device=self.device)
+        self.logits = None
+
+    def __del__(self):
+        try:
+            if getattr(self, "_h", None) is not None and _lib is not None:
+                _lib.gpt_infer_destroy(self._h)
+                self._h = None
+        except Exception:
+            pass
+
+    def _out(self, batch):
+        import torch
+        if self.logits is None or self.logits.shape[0] != batch:
+            self.logits = torch.empty(batch, self.cfg.vocab, dtype=torch.float32, device=self.device)
+        return self.logits
+
+    def prefill(self, params, tokens):
+        B, T = tokens.shape
+        out = self._out(B)
+        _check(lib().gpt_prefill(self._h, params.data_ptr(), tokens.data_ptr(), B, T, out.data_ptr(),
+                                 self.kv_cache.data_ptr(), self.workspace.data_ptr(), self.workspace.numel(),
+                                 _stream()), "gpt_prefill")
+        return out
+
+    def decode(self, params, tokens, pos: int):
+        B = tokens.numel()
+        out = self._out(B)
+        _check(lib().gpt_decode(self._h, params.data_ptr(), tokens.data_ptr(), B, pos, out.data_ptr(),
+                                self.kv_cache.data_ptr(), self.workspace.data_ptr(), self.workspace.numel(),
+                                _stream()), "gpt_decode")
+        return out
+
+    def status(self) -> int:
+        return int(lib().gpt_infer_status(self._h, self.workspace.data_ptr(), _stream()))
 
 
 # ------------------------------------------------------------------------------------------------

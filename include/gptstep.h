@@ -324,6 +324,33 @@ gpt_status gpt_lmhead_ce_fwd_bwd(const void* xf, const void* wlm, const int32_t*
                                  void* scratch, int* status, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * Forward-only inference with a key/value cache (supa beginna nanochat, notes on each stage: the
+ * engine that samples from the trained model keeps a KV cache).  The forward pass is the training
+ * step's (same kernels and numerics); the QKV projection writes k̃ = RMS_Dh(RoPE(k)) and v of every
+ * layer straight into the cache, and the lm-head runs on the last position of each sequence only.
+ *   kv_cache: caller-owned device memory of gpt_infer_kv_cache_bytes() bytes, bf16
+ *             [depth][2][max_batch][n_kv_heads][max_len][head_dim] (k̃ then v per layer).
+ *   gpt_prefill: tokens [batch, T] (positions 0 .. T−1 of every sequence), fills cache positions
+ *             0 .. T−1 and writes logits [batch, V] (fp32) of position T−1.
+ *   gpt_decode: tokens [batch] at position `pos` of every sequence (cache positions 0 .. pos−1
+ *             already filled), fills position pos and writes logits [batch, V] of it.
+ * All sequences of a call share one length.  param_dtype must be BF16 and head_dim 64 or 128.
+ * batch ≤ max_batch, T and pos + 1 ≤ max_len.  Token ids outside [0, V) are clamped and flagged in
+ * the status word (gpt_infer_status).  Host-only: create, destroy, the byte counts. */
+typedef struct gpt_infer gpt_infer;
+gpt_status gpt_infer_create(const gpt_config* cfg, int max_batch, int max_len, gpt_infer** out);
+void gpt_infer_destroy(gpt_infer* inf);
+gpt_status gpt_infer_workspace_bytes(const gpt_infer* inf, size_t* bytes);
+size_t gpt_infer_kv_cache_bytes(const gpt_infer* inf);
+gpt_status gpt_prefill(gpt_infer* inf, const void* params, const int32_t* tokens, int batch, int T,
+                       float* logits, void* kv_cache, void* workspace, size_t workspace_bytes,
+                       void* stream);
+gpt_status gpt_decode(gpt_infer* inf, const void* params, const int32_t* tokens, int batch, int pos,
+                      float* logits, void* kv_cache, void* workspace, size_t workspace_bytes,
+                      void* stream);
+gpt_status gpt_infer_status(const gpt_infer* inf, const void* workspace, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
  * The optimizer step after the training step (Introducing nanochat, Pretraining log: the block
  * matrices go to Muon, grouped by shape — q, k, v, the output projection, W_fc, W_proj — and the
  * embedding and lm-head to AdamW, whose learning rates are scaled by 1/√(d/768)).  The pages print
