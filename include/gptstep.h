@@ -65,7 +65,10 @@ typedef struct gpt_config {
 
 typedef struct gpt_step gpt_step; /* opaque host-side plan; owns no device memory */
 
-/* Flat parameter packing (element offsets, each a multiple of 64):
+/* Flat parameter packing (element offsets, each a multiple of 64).  The tensors are the ones the
+ * pages count (Introducing nanochat, Pretraining: the parameter count 560,988,160 at depth 20 is
+ * 2·V·d for the untied embedding and lm-head plus 12·d² per layer; nanochat User Guide §10: untied
+ * embedding/unembedding, no biases); the order is this library's:
  *   offsets[0]            wte   [V, d]
  *   offsets[1 + 4l + 0]   W_qkv [d + 2·dkv, d]   rows q (d) | k (dkv) | v (dkv), dkv = n_kv_heads·Dh
  *                                        (3d without grouping); head h's rows start at h·Dh of
@@ -78,15 +81,21 @@ typedef struct gpt_step gpt_step; /* opaque host-side plan; owns no device memor
  * Gradients use the same packing in fp32.  Host-only; needs no GPU. */
 gpt_status gpt_param_layout(const gpt_config* cfg, size_t* offsets, size_t* total);
 
-/* Validate cfg and build the host plan.  Host-only; needs no GPU. */
+/* Validate cfg and build the host plan (the window pattern of nanochat User Guide §10 is given
+ * per layer in cfg.window).  Host-only; needs no GPU. */
 gpt_status gpt_step_create(const gpt_config* cfg, gpt_step** out);
 void gpt_step_destroy(gpt_step* step);
 
 /* Bytes of device workspace gpt_step_fwd_bwd needs (activations kept for the backward pass,
- * gradient scratch, statistics).  Host-only. */
+ * gradient scratch, statistics).  The pages give no memory plan; the caller allocates this once
+ * and the library keeps no pointer into it past a call (Porting nanochat to a TPU, §4, the first
+ * lesson: a buffer reused after it was captured corrupted every batch).  Host-only. */
 gpt_status gpt_step_workspace_bytes(const gpt_step* step, size_t* bytes);
 
-/* One training step.
+/* One training step: the forward pass of the model above (nanochat User Guide §10, How It Works),
+ * the mean cross-entropy over targets ≠ −1 (supa beginna nanochat, Troubleshooting) and the backward
+ * pass to the gradients of every parameter (the step whose throughput the pages report as tok/sec and
+ * MFU, Introducing nanochat, Pretraining log).
  *   params    [n_params] bf16 or fp32 (cfg.param_dtype), packing as above
  *   tokens    [batch, seq_len] int32 in [0, V)
  *   targets   [batch, seq_len] int32 in [0, V) or −1 (ignored)
@@ -101,12 +110,16 @@ gpt_status gpt_step_fwd_bwd(gpt_step* step, const void* params, const int32_t* t
                             size_t workspace_bytes, int accumulate, void* stream);
 
 /* Synchronize `stream`, read and clear the device status word that the last step on `workspace`
- * wrote.  Returns GPT_OK, GPT_ERR_TOKEN_OUT_OF_RANGE or GPT_ERR_DEVICE_TIMEOUT (or GPT_ERR_CUDA). */
+ * wrote.  Returns GPT_OK, GPT_ERR_TOKEN_OUT_OF_RANGE or GPT_ERR_DEVICE_TIMEOUT (or GPT_ERR_CUDA).
+ * The pages have no counterpart (errors found on the device instead of a trap or a hang). */
 gpt_status gpt_step_status(const gpt_step* step, const void* workspace, void* stream);
 
+/* A short English description of a status code ("unknown status" for others).  No page
+ * counterpart. */
 const char* gpt_strerror(int status);
 
-/* Number of kernel launches the last gpt_step_fwd_bwd enqueued (host counter, for reporting). */
+/* Number of kernel launches the last gpt_step_fwd_bwd enqueued (host counter, for reporting; the
+ * pages trace idle gaps between device programs, Porting nanochat to a TPU, §4). */
 int64_t gpt_step_last_launch_count(const gpt_step* step);
 
 /* Gradient buckets, for a data-parallel exchange that overlaps the backward pass.  The gradient
