@@ -20,6 +20,7 @@
 // No atomics anywhere: every output element has one writer, so results are bitwise reproducible.
 
 #include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -330,6 +331,29 @@ struct TcFwdShape {
   static constexpr int TM_O = 256;  // O_x at 256 + x·DH
 };
 
+// One query tile per CTA, scores double-buffered in tensor memory: S(j+1) = Q·K(j+1)ᵀ is computed
+// while the softmax warps turn S(j) into P(j), and P(j)·V(j) runs while they work on S(j+1).  The
+// 16 softmax warps form two groups that take alternate key tiles (group g: tiles j ≡ g mod 2, in
+// S buffer g), so each group has two tile-times for one tile's exponentials; within a group a query
+// row is split into two 64-key halves over the four tensor-memory lane quarters.
+template <int DH>
+struct TcFwd1Shape {
+  static constexpr int BQ = 128, BK = 128;
+  static constexpr int K_STAGES = 3, V_STAGES = 2;
+  static constexpr int Q_TILE = BQ * DH * 2;
+  static constexpr int KV_TILE = BK * DH * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = Q_TILE;
+  static constexpr int OFF_V = OFF_K + K_STAGES * KV_TILE;
+  static constexpr int OFF_BAR = OFF_V + V_STAGES * KV_TILE;
+  static constexpr int OFF_RED = OFF_BAR + 256;  // [group][half][row] (l, lb) partial row sums
+  static constexpr int SMEM = OFF_RED + 2 * 2 * 128 * 8 + 1024;
+  static constexpr int THREADS = 576;  // 16 softmax warps, the TMA warp, the MMA warp
+  static constexpr int TMA_WARP = 16, MMA_WARP = 17;
+  static constexpr int TM_S = 0;    // S[g] at g·128
+  static constexpr int TM_O = 256;  // O at 256 (DH columns)
+};
+
 // Row of the [DH/64][128][64] swizzled Q tile as fp32 sum of squares.
 template <int DH>
 __device__ __forceinline__ float q_row_sumsq(const uint8_t* tile, int r) {
@@ -568,6 +592,247 @@ __global__ void __launch_bounds__(576, 1)
         }
       }
       if (t < T && half == 0) a.lse[((long long)b * a.H + h) * T + t] = (c2 + log2f(l)) * LN2;
+    }
+  }
+
+  __syncwarp();
+  if (*abort_flag && threadIdx.x == 0) {
+    for (int i = 0; i < 2000; ++i) __nanosleep(1000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == S::MMA_WARP) tmem_dealloc(tmem, 512);
+}
+
+template <int DH>
+__global__ void __launch_bounds__(576, 1)
+    attn_fwd_tc1_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                        const __grid_constant__ CUtensorMap mv, const AttnArgs a, const float* kmax,
+                        float kmax_const) {
+  using S = TcFwd1Shape<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
+  uint64_t* bar_q = bars;
+  uint64_t* k_full = bars + 1;   // [3]
+  uint64_t* k_empty = bars + 4;  // [3]
+  uint64_t* v_full = bars + 7;   // [2]
+  uint64_t* v_empty = bars + 9;  // [2]
+  uint64_t* s_full = bars + 11;  // [2]
+  uint64_t* p_full = bars + 13;  // [2]
+  uint64_t* o_full = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int qt = gridDim.x - 1 - blockIdx.x;  // longest rows first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int T = a.T, W = a.window;  // T query rows, at absolute positions q_off .. q_off + T − 1
+  const int q0 = qt * 128;
+  const int key_lo = max(0, a.q_off + q0 - W + 1);
+  const int key_hi = min(a.Tk, a.q_off + q0 + 128);
+  const int kv_first = key_lo / 128;
+  const int n_kv = (key_hi - 1) / 128 - kv_first + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 256);
+    }
+    mbar_init(o_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == S::MMA_WARP) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
+
+  if (warp == S::TMA_WARP) {
+    // ---------------- TMA producer: Q; then K(j+1) ahead of V(j) ----------------
+    if (lane == 0) {
+      const int hk = h / a.group;  // the key/value head this query head reads
+      mbar_arrive_expect_tx(bar_q, S::Q_TILE);
+      load_tile<DH, 128>(smem + S::OFF_Q, &mq, bar_q, q0, h, b);
+      auto load_k = [&](int j) -> bool {
+        const int st = j % S::K_STAGES;
+        if (!mbar_wait(&k_empty[st], ((j / S::K_STAGES) & 1) ^ 1, abort_flag, a.status)) return false;
+        mbar_arrive_expect_tx(&k_full[st], S::KV_TILE);
+        load_tile<DH, 128>(smem + S::OFF_K + st * S::KV_TILE, &mk, &k_full[st], (kv_first + j) * 128, hk, b);
+        return true;
+      };
+      bool ok = n_kv > 0 && load_k(0);
+      for (int j = 0; j < n_kv && ok; ++j) {
+        if (j + 1 < n_kv && !load_k(j + 1)) break;
+        const int st = j % S::V_STAGES;
+        if (!mbar_wait(&v_empty[st], ((j / S::V_STAGES) & 1) ^ 1, abort_flag, a.status)) break;
+        mbar_arrive_expect_tx(&v_full[st], S::KV_TILE);
+        load_tile<DH, 128>(smem + S::OFF_V + st * S::KV_TILE, &mv, &v_full[st], (kv_first + j) * 128, hk, b);
+      }
+    }
+  } else if (warp == S::MMA_WARP) {
+    // ---------------- MMA issuer: the warp runs the loop, one elected lane issues ----------------
+    constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
+    constexpr uint32_t id_o = idesc_bf16(128, DH, false, true);
+    const uint64_t qd = sdesc_sw128(smem_u32(smem + S::OFF_Q), 16, 1024);
+    const uint64_t kd = sdesc_sw128(smem_u32(smem + S::OFF_K), 16, 1024);
+    const uint64_t vd = sdesc_sw128(smem_u32(smem + S::OFF_V), 128 * 128, 1024);
+    // S(j) = Q·K(j)ᵀ into buffer j & 1; frees K stage j % 3 and publishes the buffer
+    auto issue_s = [&](int j) -> bool {
+      const int st = j % S::K_STAGES;
+      if (!mbar_wait_warp(&k_full[st], (j / S::K_STAGES) & 1, abort_flag, a.status)) return false;
+      tc_fence_after();
+      const uint64_t k_desc = sdesc_add(kd, st * S::KV_TILE);
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_bf16_ss(tmem + S::TM_S + (j & 1) * 128, sdesc_add(qd, off), sdesc_add(k_desc, off), id_s,
+                      kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&k_empty[st]);
+        tc_commit(&s_full[j & 1]);
+      }
+      __syncwarp();
+      return true;
+    };
+    bool ok = mbar_wait_warp(bar_q, 0, abort_flag, a.status);
+    if (ok && n_kv > 0) ok = issue_s(0);
+    if (ok && n_kv > 1) ok = issue_s(1);
+    for (int j = 0; j < n_kv && ok; ++j) {
+      // P(j) ready (softmax group j & 1), V(j) loaded: O += P(j)·V(j)
+      if (!mbar_wait_warp(&p_full[j & 1], (j >> 1) & 1, abort_flag, a.status)) break;
+      const int vs = j % S::V_STAGES;
+      if (!mbar_wait_warp(&v_full[vs], (j / S::V_STAGES) & 1, abort_flag, a.status)) break;
+      tc_fence_after();
+      const uint64_t v_desc = sdesc_add(vd, vs * S::KV_TILE);
+      const uint32_t p_tmem = tmem + S::TM_S + (j & 1) * 128;
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // key half kk/4 packed in S columns 64·(kk/4) + 8·(kk%4)
+          mma_bf16_ts(tmem + S::TM_O, p_tmem + 64 * (kk >> 2) + 8 * (kk & 3), sdesc_add(v_desc, kk * 2048),
+                      id_o, (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&v_empty[vs]);
+      }
+      __syncwarp();
+      // the next scores of this buffer, issued after P(j)·V(j) has been issued (MMAs run in order)
+      if (j + 2 < n_kv && !issue_s(j + 2)) break;
+    }
+    if (elect_one()) tc_commit(o_full);
+    __syncwarp();
+  } else {
+    // ---------------- softmax warps: group g takes key tiles j ≡ g (mod 2); thread = one query
+    // row × one 64-key half of those tiles
+    const int g = warp >> 3;
+    const int half = (warp >> 2) & 1;
+    const int quarter = warp & 3;
+    const int row = 32 * quarter + lane;
+    const int t = q0 + row;              // query row (local)
+    const int ta = a.q_off + t;          // its position among the keys
+    const int tile0 = a.q_off + q0;
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    const uint32_t s_addr = tmem + lane_off + S::TM_S + g * 128 + 64 * half;
+    bool ok = mbar_wait_warp(bar_q, 0, abort_flag, a.status);
+    // fixed shift c_t (log2 units)
+    const float qn = sqrtf(q_row_sumsq<DH>(smem + S::OFF_Q, row));
+    const float km = kmax ? kmax[(long long)b * a.Hkv + h / a.group] : kmax_const;
+    const float c_nat = qn * km * a.scale * 1.001f + 1e-3f;
+    if (c_nat > 40.f && t < T && half == 0 && g == 0) set_status(a.status, GPT_ERR_NUMERIC_RANGE);
+    const float c2 = c_nat * LOG2E;
+    // l: exact sum of the weights (gives the LSE); lb: sum of the bf16 weights that P·V uses
+    float l0 = 0.f, l1 = 0.f, lb0 = 0.f, lb1 = 0.f;
+    for (int j = g; j < n_kv && ok; j += 2) {
+      if (!mbar_wait_warp(&s_full[g], (j >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+      tc_fence_after();
+      const int kv0 = (kv_first + j) * 128 + 64 * half;  // first key of this thread's half
+      const bool need_mask = (kv0 + 63 > tile0) || (kv0 <= tile0 + 127 - W);
+      uint32_t rbuf[2][16];
+      tmem_ld16(s_addr, rbuf[0]);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t (&r)[16] = rbuf[c & 1];
+        if (c < 3) tmem_ld16(s_addr + 16 * (c + 1), rbuf[(c + 1) & 1]);
+        uint32_t pk[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float x0, x1, p0, p1;
+          fma2_bc(x0, x1, __uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]), a.scale_log2, -c2);
+          if ((e & 3) == 3) {  // one pair in four on the FMA pipe
+            exp2_poly2(p0, p1, x0, x1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          if (need_mask) {
+            const int key = kv0 + 16 * c + 2 * e;
+            if (!(key <= ta && key > ta - W)) p0 = 0.f;
+            if (!(key + 1 <= ta && key + 1 > ta - W)) p1 = 0.f;
+          }
+          add2_acc(l0, l1, p0, p1);
+          pk[e] = pack_bf2(p0, p1);
+          add2_acc(lb0, lb1, bf_lo(pk[e]), bf_hi(pk[e]));
+        }
+        // P of chunk c overwrites this half's S columns 8c..8c+7, all of which have been read
+        tmem_st8(s_addr + 8 * c, pk);
+        if (c < 3) tmem_ld_wait();
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[g]);
+    }
+    // the four partial sums of a row (2 groups × 2 halves) are combined in a fixed order
+    float2* red = reinterpret_cast<float2*>(smem + S::OFF_RED);
+    red[(g * 2 + half) * 128 + row] = make_float2(l0 + l1, lb0 + lb1);
+    named_barrier_sync(1, 512);  // every softmax thread reaches this, whatever its loop did
+    float l = 0.f, lbs = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 v = red[i * 128 + row];
+      l += v.x;
+      lbs += v.y;
+    }
+    const float inv = 1.f / lbs;
+    // epilogue: O / lb, this thread's quarter of the DH columns
+    if (ok) ok = mbar_wait_warp(o_full, 0, abort_flag, a.status);
+    if (ok) {
+      tc_fence_after();
+      uint16_t* orow = a.o + b * a.sb_o + h * a.sh_o + (long long)t * a.st_o;
+      constexpr int QC = DH / 4;  // columns per thread
+      const int c0 = (g * 2 + half) * QC;
+      uint32_t r[QC];
+      if constexpr (QC == 32) {
+        tmem_ld32(tmem + lane_off + S::TM_O + c0, r);
+      } else {
+        tmem_ld16(tmem + lane_off + S::TM_O + c0, r);
+      }
+      tmem_ld_wait();
+      if (t < T) {
+#pragma unroll
+        for (int u = 0; u < QC / 8; ++u) {
+          uint4 w;
+          w.x = pack_bf2(__uint_as_float(r[8 * u + 0]) * inv, __uint_as_float(r[8 * u + 1]) * inv);
+          w.y = pack_bf2(__uint_as_float(r[8 * u + 2]) * inv, __uint_as_float(r[8 * u + 3]) * inv);
+          w.z = pack_bf2(__uint_as_float(r[8 * u + 4]) * inv, __uint_as_float(r[8 * u + 5]) * inv);
+          w.w = pack_bf2(__uint_as_float(r[8 * u + 6]) * inv, __uint_as_float(r[8 * u + 7]) * inv);
+          *reinterpret_cast<uint4*>(orow + c0 + 8 * u) = w;
+        }
+        if (half == 0 && g == 0) a.lse[((long long)b * a.H + h) * T + t] = (c2 + log2f(l)) * LN2;
+      }
     }
   }
 
@@ -1775,9 +2040,26 @@ gpt_status launch_fwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, c
   return launch_kernel(attn_fwd_kernel<DH>, grid, dim3(256), FwdShape<DH>::SMEM, stream, mq, mk, mv, a);
 }
 
+// Forward kernel choice: one query tile per CTA with double-buffered scores (default) or two query
+// tiles per CTA sharing each K/V tile (GPTSTEP_ATTN_FWD=2).
+static bool fwd_one_tile() {
+  static const bool one = [] {
+    const char* v = std::getenv("GPTSTEP_ATTN_FWD");
+    return !(v && v[0] == '2');
+  }();
+  return one;
+}
+
 template <int DH>
 gpt_status launch_fwd_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const AttnArgs& a, const float* kmax, float kmax_const, cudaStream_t stream) {
+  if (fwd_one_tile()) {
+    using S1 = TcFwd1Shape<DH>;
+    GPT_TRY(ensure_smem(attn_fwd_tc1_kernel<DH>, S1::SMEM));
+    dim3 grid((a.T + 127) / 128, a.H, a.B);
+    return launch_kernel(attn_fwd_tc1_kernel<DH>, grid, dim3(S1::THREADS), S1::SMEM, stream, mq, mk, mv, a,
+                         kmax, kmax_const);
+  }
   using S = TcFwdShape<DH>;
   GPT_TRY(ensure_smem(attn_fwd_tc_kernel<DH>, S::SMEM));
   dim3 grid((a.T + 255) / 256, a.H, a.B);
