@@ -362,3 +362,50 @@ def _shard_rank_main(rank, world, port, q):
     run(grads * 0.5, 2)
     dist.destroy_process_group()
     q.put((rank, p.numpy().copy()))
+
+
+def test_a_failed_rank_ends_the_others_exchange_with_an_error():
+    """Rank 1 raises before its gradient exchange and exits; rank 0's bucketed average must end with
+    an error (connection closed or the short process-group timeout), not wait for good."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 31700 + (os.getpid() % 1000)
+    procs = [ctx.Process(target=_failing_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+    assert out[1] == "raised"
+    assert out[0].startswith("error:"), out[0]
+
+
+def _failing_rank_main(rank, world, port, q):
+    import sys
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from gpt_decoder_pretraining_b200 import dp
+    from gpt_decoder_pretraining_b200.config import custom
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    cfg = custom(2, 32, 16, 64, 12, 1, param_dtype=1)
+    g = torch.ones(cfg.n_params, dtype=torch.float32)
+    if rank == 1:
+        try:
+            raise RuntimeError("rank 1 fails before its exchange")
+        except RuntimeError:
+            q.put((rank, "raised"))
+            q.close()
+            q.join_thread()
+            os._exit(0)  # leaves without destroying the process group, as a crashed rank would
+    try:
+        dp.average_in_buckets(g, dp.grad_buckets(cfg), world)
+        q.put((rank, "completed"))
+    except Exception as e:  # noqa: BLE001 - any error ends the wait, which is what is checked
+        q.put((rank, "error: " + type(e).__name__))
+    q.close()
+    q.join_thread()
+    os._exit(0)
