@@ -55,62 +55,53 @@ template <int EPI>
 constexpr int gemm_threads() { return 64 + 128 * gemm_col_groups<EPI>(); }
 
 // Persistent schedule over the CTA pairs.  Output tiles 0 .. dp_tiles−1 are dealt round-robin and
-// computed whole; the sk_tiles after them are computed "stream-K": their sk_tiles·k_tiles K-steps,
-// in tile-major order, are cut into num_pairs contiguous ranges (sk_base steps each, one more for
-// the first sk_rem pairs), one per pair.  sk_smax is the most pieces any such tile is cut into.
+// computed whole; dp_tiles is a whole number of waves, so every pair walks K in step with the others
+// and the operand rows / columns that tiles of one wave share are read from L2, not HBM.  The
+// sk_tiles after them (the last, partly empty wave) are each cut along K into sk_split equal
+// pieces, all starting together: pair p takes piece p mod sk_split of tail tile p / sk_split,
+// k-tiles [⌊j·k_tiles/sk_split⌋, ⌊(j+1)·k_tiles/sk_split⌋).  At any moment the tail pieces sit at
+// sk_split K offsets, so L2 reuse across the tail tiles survives the split.
 struct Sched {
   int num_pairs, k_tiles;
   int dp_tiles, sk_tiles;
-  long long sk_base;
-  int sk_rem;
-  int sk_smax;
+  int sk_split;  // pieces per tail tile (1: no split)
 };
 
-__host__ __device__ inline long long sk_begin(const Sched& s, int p) {
-  return (long long)p * s.sk_base + (p < s.sk_rem ? p : s.sk_rem);
-}
-// The pair whose range holds stream-K step i.
-__host__ __device__ inline int sk_pair_of(const Sched& s, long long i) {
-  const long long cut = (long long)s.sk_rem * (s.sk_base + 1);
-  if (i < cut) return (int)(i / (s.sk_base + 1));
-  return s.sk_rem + (int)((i - cut) / s.sk_base);
-}
-
-// One unit of a pair's work: k-tiles [k0, k1) of output tile `tile`.
+// One unit of a pair's work: k-tiles [k0, k1) of output tile `tile`; `piece` is the piece index of
+// a split tail tile, −1 for a whole tile.
 struct Work {
-  int tile, k0, k1;
+  int tile, k0, k1, piece;
 };
 struct WorkIter {
   int dp_next;
-  long long sk_i, sk_end;
-  __device__ WorkIter(const Sched& s, int p)
-      : dp_next(p), sk_i(sk_begin(s, p)), sk_end(sk_begin(s, p + 1)) {}
+  bool tail_done;
+  __device__ WorkIter(const Sched& s, int p) : dp_next(p), tail_done(false) {}
   __device__ bool next(const Sched& s, Work& w) {
     if (dp_next < s.dp_tiles) {
       w.tile = dp_next;
       w.k0 = 0;
       w.k1 = s.k_tiles;
+      w.piece = -1;
       dp_next += s.num_pairs;
       return true;
     }
-    if (sk_i < sk_end) {
-      const long long t = sk_i / s.k_tiles;
-      const int k0 = (int)(sk_i - t * s.k_tiles);
-      const long long lim = k0 + (sk_end - sk_i);
-      const int k1 = lim < s.k_tiles ? (int)lim : s.k_tiles;
-      w.tile = s.dp_tiles + (int)t;
-      w.k0 = k0;
-      w.k1 = k1;
-      sk_i += k1 - k0;
+    const int p = dp_next - s.dp_tiles;  // this pair's index in the tail phase
+    if (!tail_done && p < s.sk_tiles * s.sk_split) {
+      tail_done = true;
+      const int j = p % s.sk_split;
+      w.tile = s.dp_tiles + p / s.sk_split;
+      w.k0 = (int)((long long)j * s.k_tiles / s.sk_split);
+      w.k1 = (int)((long long)(j + 1) * s.k_tiles / s.sk_split);
+      w.piece = s.sk_split > 1 ? j : -1;
       return true;
     }
     return false;
   }
 };
 
-// Stream-K piece exchange: each piece of a split tile writes its fp32 partial tile to its own slot
-// (256 × 256 floats, slot = tile·sk_smax + piece), then counts itself in one counter per epilogue
-// warp (32 rows × 128 columns: 16 per tile).
+// Piece exchange of a split tail tile: each piece writes its fp32 partial tile to its own slot
+// (256 × 256 floats, slot = tail tile·sk_split + piece), then counts itself in one counter per
+// epilogue warp (32 rows × 128 columns: 16 per tile).
 constexpr int SK_WARPS_PER_TILE = 16;
 constexpr int SK_MAX_TILES = 320;
 constexpr int SK_MAX_SLOTS = 320;
@@ -122,7 +113,7 @@ struct GemmArgs {
   int M, N, K;
   int tiles_m, tiles_n, k_tiles;  // tiles_m counts 256-row pair tiles
   Sched sched;
-  float* sk_part;                  // [sk_tiles·sk_smax][256][256] partial tiles
+  float* sk_part;                  // [sk_tiles·sk_split][256][256] partial tiles
   int* sk_cnt;                     // [sk_tiles·16] arrival counters, zero between launches
   int batch;                       // independent matrices; tile t belongs to matrix t / (tiles_m·tiles_n)
   long long c_bstride, aux_bstride;  // elements between consecutive matrices of C and aux
@@ -138,8 +129,8 @@ struct GemmArgs {
   CeArgs ce;
   // head-major outputs (EPI_BF16_HEADS, EPI_QKV_ROPE + Dh); Hkv key/value heads (QKV)
   int T, H, Dh, d, Hkv;
-  // QKV: destination of q, k, v — [B][heads][ts][Dh], row m = b·T + t written at position
-  // t + t_off (which is also the RoPE position); ts ≥ T + t_off (a key/value cache)
+  // QKV: destination of q, k, v — [B][heads][ts][Dh]; row m = b·T + t has RoPE position t + t_off,
+  // q is written at position t (q_ts ≥ T), k and v at t + t_off (kv_ts ≥ T + t_off: a cache)
   uint16_t* qkv_dst[3];
   int qkv_ts[3];
   int t_off;
@@ -325,7 +316,7 @@ __device__ __forceinline__ bool plain_epilogue(const GemmArgs& a, const Work& w,
                                                volatile int* abort_flag) {
   constexpr int NC = BN / 32 / 2;  // 32-column chunks per thread
   const Sched& sch = a.sched;
-  const bool piece = w.tile >= sch.dp_tiles && !(w.k0 == 0 && w.k1 == sch.k_tiles);
+  const bool piece = w.piece >= 0;
   const int nbase = tn * BN + half * (BN / 2);
   constexpr bool kPre = (EPI == GPT_EPI_RESID || EPI == GPT_EPI_DRELU2);
   // The residual / saved activation does not depend on the accumulator: chunk 0 is fetched before
@@ -367,12 +358,9 @@ __device__ __forceinline__ bool plain_epilogue(const GemmArgs& a, const Work& w,
   }
   // ---- stream-K piece ----
   const int st = w.tile - sch.dp_tiles;
-  const long long s0 = (long long)st * sch.k_tiles;
-  const int first = sk_pair_of(sch, s0);
-  const int nseg = sk_pair_of(sch, s0 + sch.k_tiles - 1) - first + 1;
-  const int seg = sk_pair_of(sch, s0 + w.k0) - first;
+  const int nseg = sch.sk_split, seg = w.piece;
   const size_t row_off = (size_t)(rank * BM + q * 32 + lane) * BN + half * (BN / 2);
-  float* mine = a.sk_part + (size_t)(st * sch.sk_smax + seg) * SK_SLOT_FLOATS + row_off;
+  float* mine = a.sk_part + (size_t)(st * nseg + seg) * SK_SLOT_FLOATS + row_off;
 #pragma unroll 1
   for (int c = 0; c < NC; ++c) {
     uint32_t r[32];
@@ -391,7 +379,7 @@ __device__ __forceinline__ bool plain_epilogue(const GemmArgs& a, const Work& w,
   if (old != nseg - 1) return true;
   // last piece: every other piece's partial is visible; sum in ascending K (= slot) order
   __threadfence();
-  const float* slot0 = a.sk_part + (size_t)st * sch.sk_smax * SK_SLOT_FLOATS + row_off;
+  const float* slot0 = a.sk_part + (size_t)st * nseg * SK_SLOT_FLOATS + row_off;
 #pragma unroll 1
   for (int c = 0; c < NC; ++c) {
     uint32_t r[32];
@@ -610,7 +598,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
         // squares first (rotation preserves it), then the rotation pairs (j, j + DH/2) 32 at a time.
         constexpr int DH = EPI - EPI_QKV_ROPE, HALF = DH / 2;
         const int dkv = args.Hkv * DH;
-        const int b = m / args.T, t = m % args.T + args.t_off;  // position
+        const int b = m / args.T, tl = m % args.T, t = tl + args.t_off;  // local row, position
         const bool row_ok = m < args.M;
 #pragma unroll 1
         for (int hh = half * (BN / DH / G); hh < (half + 1) * (BN / DH / G); ++hh) {
@@ -621,7 +609,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
           const int region = n_head < args.d ? 0 : (n_head < args.d + dkv ? 1 : 2);
           const int h = (n_head - (region == 0 ? 0 : args.d + (region - 1) * dkv)) / DH;
           const int nh = region == 0 ? args.H : args.Hkv;  // heads of this region
-          uint16_t* dst = args.qkv_dst[region] + (((long long)b * nh + h) * args.qkv_ts[region] + t) * DH;
+          uint16_t* dst = args.qkv_dst[region] +
+                          (((long long)b * nh + h) * args.qkv_ts[region] + (region == 0 ? tl : t)) * DH;
           auto store32 = [&](int col, const float* w) {
             if (!row_ok) return;
 #pragma unroll
@@ -888,34 +877,31 @@ static gpt_status fill_args(GemmArgs& a, int M, int N, int K, int batch = 1, int
   return GPT_OK;
 }
 
-// Stream-K plan for the tail of the tile list, or false when the round-robin schedule is as good.
-// Cost model, in k-step times of one CTA pair: round robin takes ⌈tiles/P⌉·k_tiles; stream-K takes
-// (dp waves)·k_tiles + ⌈sk steps/P⌉ plus the piece exchange, ≈ 8 k-steps per extra piece that the
-// last piece reads back (a 128 KB partial per CTA at its share of HBM bandwidth) + 4 for writing.
+// Split plan for the tail of the tile list, or false when the round-robin schedule is as good.
+// Cost model, in k-step times of one CTA pair: round robin takes ⌈tiles/P⌉·k_tiles; the split takes
+// ⌊tiles/P⌋·k_tiles + ⌈k_tiles/s⌉ plus the piece exchange, ≈ 8 k-steps per extra piece that the
+// last piece reads back (a 128 KB partial per CTA) + 4 for writing its own.  s ≤ P / tail tiles,
+// and the split must save at least 5%.
 bool plan_stream_k(int tiles, int k_tiles, int pairs, Sched* out) {
-  if (pairs < 2 || tiles <= 0 || k_tiles <= 0 || tiles % pairs == 0) return false;
-  const long long rr_cost = (long long)((tiles + pairs - 1) / pairs) * k_tiles;
-  const int sk_tiles = tiles < pairs ? tiles : tiles % pairs + pairs;
-  const int dp_tiles = tiles - sk_tiles;
-  Sched s{};
-  s.num_pairs = pairs;
-  s.k_tiles = k_tiles;
-  s.dp_tiles = dp_tiles;
-  s.sk_tiles = sk_tiles;
-  const long long total = (long long)sk_tiles * k_tiles;
-  s.sk_base = total / pairs;
-  s.sk_rem = (int)(total % pairs);
-  if (s.sk_base < 1) return false;
-  int smax = 1;
-  for (int t = 0; t < sk_tiles; ++t) {
-    const long long s0 = (long long)t * k_tiles;
-    smax = std::max(smax, sk_pair_of(s, s0 + k_tiles - 1) - sk_pair_of(s, s0) + 1);
+  if (pairs < 2 || tiles <= 0 || k_tiles < 2 || tiles % pairs == 0) return false;
+  const int waves = tiles / pairs, tail = tiles % pairs;
+  const long long rr_cost = (long long)(waves + 1) * k_tiles;
+  int best_s = 1;
+  long long best = k_tiles;
+  for (int sp = 2; sp <= pairs / tail && sp <= k_tiles; ++sp) {
+    if (tail > SK_MAX_TILES || (long long)tail * sp > SK_MAX_SLOTS) break;
+    const long long c = (k_tiles + sp - 1) / sp + 8 * (sp - 1) + 4;
+    if (c < best) { best = c; best_s = sp; }
   }
-  s.sk_smax = smax;
-  if (sk_tiles > SK_MAX_TILES || (long long)sk_tiles * smax > SK_MAX_SLOTS) return false;
-  const long long sk_cost = (long long)(dp_tiles / pairs) * k_tiles + (total + pairs - 1) / pairs +
-                            8 * (smax - 1) + 4;
-  if (100 * sk_cost > 97 * rr_cost) return false;
+  if (best_s == 1) return false;
+  const long long cost = (long long)waves * k_tiles + best;
+  if (100 * cost > 95 * rr_cost) return false;
+  Sched s{};
+  s.num_pairs = waves > 0 ? pairs : tail * best_s;  // with no whole wave, launch only the pieces
+  s.k_tiles = k_tiles;
+  s.dp_tiles = waves * pairs;
+  s.sk_tiles = tail;
+  s.sk_split = best_s;
   *out = s;
   return true;
 }
@@ -1070,7 +1056,7 @@ gpt_status gemm_qkv_rope_launch(int M, int d, const void* A, const void* Wqkv, v
   a.C = heads; a.ldc = N; a.status = status;
   a.T = T; a.H = H; a.Dh = Dh; a.d = d; a.Hkv = Hkv; a.cs = cs; a.rho_q = rho_q; a.rho_k = rho_k;
   if (dest) {
-    if (!dest->k || !dest->v || dest->q_ts < T + dest->t_off || dest->kv_ts < T + dest->t_off ||
+    if (!dest->k || !dest->v || dest->q_ts < T || dest->kv_ts < T + dest->t_off ||
         dest->t_off < 0)
       return GPT_ERR_INVALID_ARG;
     a.qkv_dst[0] = reinterpret_cast<uint16_t*>(dest->q);

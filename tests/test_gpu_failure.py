@@ -88,7 +88,9 @@ def test_wait_probe_times_out_and_the_context_survives():
 
 @pytest.mark.parametrize("op", [0, 2])
 def test_gemm_wait_timeout_returns_status_then_recovers(op):
-    A, B, ref = _gemm_case(seed=4 + op)
+    # one 256×256 tile with a long K: the epilogue warps wait for the accumulator through 512
+    # k-steps, far longer than the time one mbarrier.try_wait may suspend before it reports "not yet"
+    A, B, ref = _gemm_case(seed=4 + op, M=256, N=256, K=32768)
     M, N = ref.shape
     K = A.shape[1]
     tA = bf16_tensor(A if op == 0 else np.ascontiguousarray(A.T))   # TN takes A as [K, M]
@@ -97,14 +99,14 @@ def test_gemm_wait_timeout_returns_status_then_recovers(op):
     st = _status()
     try:
         S.set_wait_limit(TINY_LIMIT)
-        S.gemm(op, S.EPI_F32, tA, tB, C, M, N, K, status=st)
+        S.gemm(op, S.EPI_F32, tA, tB, C, M, N, K, status=st, scratch=None)
         torch.cuda.synchronize()
     finally:
         S.set_wait_limit(0)
     assert int(st.item()) == TIMEOUT
     st2 = _status()
     C.zero_()
-    S.gemm(op, S.EPI_F32, tA, tB, C, M, N, K, status=st2)
+    S.gemm(op, S.EPI_F32, tA, tB, C, M, N, K, status=st2, scratch=None)
     torch.cuda.synchronize()
     assert int(st2.item()) == 0
     assert_close_rel(to_np(C), ref, rel=1e-5, cos=0.9999999, what="gemm after recovery")

@@ -42,7 +42,7 @@ def test_quantize_codes_bit_exact(n, scale):
     assert np.float32(dq.item()) == ref_dq
 
 
-@pytest.mark.parametrize("M,N,K", [(300, 200, 136), (1024, 768, 2048), (3000, 1700, 2560)])
+@pytest.mark.parametrize("M,N,K", [(300, 200, 144), (1024, 768, 2048), (3000, 1700, 2560)])
 def test_gemm_e4m3_matches_oracle(M, N, K):
     rng = np.random.default_rng(M + N + K)
     a = randn(rng, M, K)
@@ -63,3 +63,14 @@ def test_gemm_e4m3_matches_oracle(M, N, K):
     assert torch.equal(C, C2)
     # and the 8-bit product approximates the bf16 one to the quantisation error
     assert_close_rel(to_np(C), 0.5 * a @ b.T, rel=0.15, cos=0.99, what="vs bf16 product")
+
+
+def test_gemm_e4m3_rejects_rows_that_break_16_byte_alignment():
+    # K = 136 one-byte codes per row: the row stride is not a multiple of 16 bytes (TMA)
+    M, N, K = 64, 64, 136
+    qa = torch.zeros(M, K, dtype=torch.uint8, device="cuda")
+    qb = torch.zeros(N, K, dtype=torch.uint8, device="cuda")
+    one = torch.ones(1, dtype=torch.float32, device="cuda")
+    C = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(S.GptError, match="UNSUPPORTED_SHAPE"):
+        S.gemm_e4m3(qa, qb, C, one, one, M, N, K)

@@ -87,8 +87,8 @@ def test_gemm_epilogues(M, N, K):
 
 
 # Shapes whose tile count leaves the last wave of CTA pairs partly empty, so that the GEMM splits
-# the tail tiles along K (stream-K): fewer tiles than CTA pairs (every tile in pieces, up to four
-# per tile), a weight-gradient shape of 100 tiles, and 84 ragged tiles.
+# the tail tiles along K: fewer tiles than CTA pairs (every tile in two pieces), a weight-gradient
+# shape of 100 tiles (one whole wave, 26 tail tiles in two pieces), and 84 ragged tiles.
 SK_SHAPES = [(1536, 1536, 16384, 2), (1280, 5120, 8192, 2), (3000, 1700, 2560, 0), (3000, 1700, 2560, 1)]
 
 
@@ -110,7 +110,9 @@ def test_gemm_stream_k_tail_matches_fp64_and_is_reproducible(M, N, K, op):
     assert int(st.item()) == 0
     assert_close_rel(to_np(C1), ref, rel=1e-5, cos=0.9999999, what="f32 stream-K")
     assert torch.equal(C1, C2)  # bitwise reproducible
-    assert_close_rel(to_np(C1), to_np(Cn), rel=1e-5, cos=0.9999999, what="stream-K vs whole tiles")
+    assert_close_rel(to_np(Cn), ref, rel=1e-5, cos=0.9999999, what="f32 whole tiles")
+    # both within 1e-5 of the fp64 product: they differ from each other only by fp32 summation order
+    assert_close_rel(to_np(C1), to_np(Cn), rel=2e-5, cos=0.9999999, what="stream-K vs whole tiles")
     if op == 2:
         return
     # the element-wise epilogues on the same split schedule

@@ -43,7 +43,7 @@ def setup_module(module):
 @pytest.mark.parametrize("op", [0, 1, 2])
 def test_gemm_batched_axpby(op):
     rng = np.random.default_rng(70 + op)
-    nb, M, N, K = 5, 300, 200, 136
+    nb, M, N, K = 5, 296, 200, 136  # ragged against the 256-row tiles; M·2 bytes a 16-byte multiple (TN)
     a_shape = (K, M) if op == 2 else (M, K)
     b_shape = (N, K) if op == 0 else (K, N)
     pad = 64  # matrices further apart than their size
