@@ -331,28 +331,6 @@ struct TcFwdShape {
   static constexpr int TM_O = 256;  // O_x at 256 + x·DH
 };
 
-// One query tile per CTA, scores double-buffered in tensor memory: S(j+1) = Q·K(j+1)ᵀ is computed
-// while the softmax warps turn S(j) into P(j), and P(j)·V(j) runs while they work on S(j+1).  The
-// 16 softmax warps form two groups that take alternate key tiles (group g: tiles j ≡ g mod 2, in
-// S buffer g), so each group has two tile-times for one tile's exponentials; within a group a query
-// row is split into two 64-key halves over the four tensor-memory lane quarters.
-template <int DH>
-struct TcFwd1Shape {
-  static constexpr int BQ = 128, BK = 128;
-  static constexpr int K_STAGES = 3, V_STAGES = 2;
-  static constexpr int Q_TILE = BQ * DH * 2;
-  static constexpr int KV_TILE = BK * DH * 2;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = Q_TILE;
-  static constexpr int OFF_V = OFF_K + K_STAGES * KV_TILE;
-  static constexpr int OFF_BAR = OFF_V + V_STAGES * KV_TILE;
-  static constexpr int OFF_RED = OFF_BAR + 256;  // [group][half][row] (l, lb) partial row sums
-  static constexpr int SMEM = OFF_RED + 2 * 2 * 128 * 8 + 1024;
-  static constexpr int THREADS = 576;  // 16 softmax warps, the TMA warp, the MMA warp
-  static constexpr int TMA_WARP = 16, MMA_WARP = 17;
-  static constexpr int TM_S = 0;    // S[g] at g·128
-  static constexpr int TM_O = 256;  // O at 256 (DH columns)
-};
 
 // Row of the [DH/64][128][64] swizzled Q tile as fp32 sum of squares.
 template <int DH>
@@ -605,246 +583,6 @@ __global__ void __launch_bounds__(576, 1)
   if (warp == S::MMA_WARP) tmem_dealloc(tmem, 512);
 }
 
-template <int DH>
-__global__ void __launch_bounds__(576, 1)
-    attn_fwd_tc1_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-                        const __grid_constant__ CUtensorMap mv, const AttnArgs a, const float* kmax,
-                        float kmax_const) {
-  using S = TcFwd1Shape<DH>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
-  uint64_t* bar_q = bars;
-  uint64_t* k_full = bars + 1;   // [3]
-  uint64_t* k_empty = bars + 4;  // [3]
-  uint64_t* v_full = bars + 7;   // [2]
-  uint64_t* v_empty = bars + 9;  // [2]
-  uint64_t* s_full = bars + 11;  // [2]
-  uint64_t* p_full = bars + 13;  // [2]
-  uint64_t* o_full = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = warp_id(), lane = lane_id();
-  const int qt = gridDim.x - 1 - blockIdx.x;  // longest rows first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int T = a.T, W = a.window;  // T query rows, at absolute positions q_off .. q_off + T − 1
-  const int q0 = qt * 128;
-  const int key_lo = max(0, a.q_off + q0 - W + 1);
-  const int key_hi = min(a.Tk, a.q_off + q0 + 128);
-  const int kv_first = key_lo / 128;
-  const int n_kv = (key_hi - 1) / 128 - kv_first + 1;
-
-  if (threadIdx.x == 0) {
-    mbar_init(bar_q, 1);
-    for (int i = 0; i < 3; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 256);
-    }
-    mbar_init(o_full, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == S::MMA_WARP) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  pdl_wait();
-  pdl_trigger();
-
-  if (warp == S::TMA_WARP) {
-    // ---------------- TMA producer: Q; then K(j+1) ahead of V(j) ----------------
-    if (lane == 0) {
-      const int hk = h / a.group;  // the key/value head this query head reads
-      mbar_arrive_expect_tx(bar_q, S::Q_TILE);
-      load_tile<DH, 128>(smem + S::OFF_Q, &mq, bar_q, q0, h, b);
-      auto load_k = [&](int j) -> bool {
-        const int st = j % S::K_STAGES;
-        if (!mbar_wait(&k_empty[st], ((j / S::K_STAGES) & 1) ^ 1, abort_flag, a.status)) return false;
-        mbar_arrive_expect_tx(&k_full[st], S::KV_TILE);
-        load_tile<DH, 128>(smem + S::OFF_K + st * S::KV_TILE, &mk, &k_full[st], (kv_first + j) * 128, hk, b);
-        return true;
-      };
-      bool ok = n_kv > 0 && load_k(0);
-      for (int j = 0; j < n_kv && ok; ++j) {
-        if (j + 1 < n_kv && !load_k(j + 1)) break;
-        const int st = j % S::V_STAGES;
-        if (!mbar_wait(&v_empty[st], ((j / S::V_STAGES) & 1) ^ 1, abort_flag, a.status)) break;
-        mbar_arrive_expect_tx(&v_full[st], S::KV_TILE);
-        load_tile<DH, 128>(smem + S::OFF_V + st * S::KV_TILE, &mv, &v_full[st], (kv_first + j) * 128, hk, b);
-      }
-    }
-  } else if (warp == S::MMA_WARP) {
-    // ---------------- MMA issuer: the warp runs the loop, one elected lane issues ----------------
-    constexpr uint32_t id_s = idesc_bf16(128, 128, false, false);
-    constexpr uint32_t id_o = idesc_bf16(128, DH, false, true);
-    const uint64_t qd = sdesc_sw128(smem_u32(smem + S::OFF_Q), 16, 1024);
-    const uint64_t kd = sdesc_sw128(smem_u32(smem + S::OFF_K), 16, 1024);
-    const uint64_t vd = sdesc_sw128(smem_u32(smem + S::OFF_V), 128 * 128, 1024);
-    // S(j) = Q·K(j)ᵀ into buffer j & 1; frees K stage j % 3 and publishes the buffer
-    auto issue_s = [&](int j) -> bool {
-      const int st = j % S::K_STAGES;
-      if (!mbar_wait_warp(&k_full[st], (j / S::K_STAGES) & 1, abort_flag, a.status)) return false;
-      tc_fence_after();
-      const uint64_t k_desc = sdesc_add(kd, st * S::KV_TILE);
-      if (elect_one()) {
-#pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_bf16_ss(tmem + S::TM_S + (j & 1) * 128, sdesc_add(qd, off), sdesc_add(k_desc, off), id_s,
-                      kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&k_empty[st]);
-        tc_commit(&s_full[j & 1]);
-      }
-      __syncwarp();
-      return true;
-    };
-    bool ok = mbar_wait_warp(bar_q, 0, abort_flag, a.status);
-    if (ok && n_kv > 0) ok = issue_s(0);
-    if (ok && n_kv > 1) ok = issue_s(1);
-    for (int j = 0; j < n_kv && ok; ++j) {
-      // P(j) ready (softmax group j & 1), V(j) loaded: O += P(j)·V(j)
-      if (!mbar_wait_warp(&p_full[j & 1], (j >> 1) & 1, abort_flag, a.status)) break;
-      const int vs = j % S::V_STAGES;
-      if (!mbar_wait_warp(&v_full[vs], (j / S::V_STAGES) & 1, abort_flag, a.status)) break;
-      tc_fence_after();
-      const uint64_t v_desc = sdesc_add(vd, vs * S::KV_TILE);
-      const uint32_t p_tmem = tmem + S::TM_S + (j & 1) * 128;
-      if (elect_one()) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // key half kk/4 packed in S columns 64·(kk/4) + 8·(kk%4)
-          mma_bf16_ts(tmem + S::TM_O, p_tmem + 64 * (kk >> 2) + 8 * (kk & 3), sdesc_add(v_desc, kk * 2048),
-                      id_o, (j > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&v_empty[vs]);
-      }
-      __syncwarp();
-      // the next scores of this buffer, issued after P(j)·V(j) has been issued (MMAs run in order)
-      if (j + 2 < n_kv && !issue_s(j + 2)) break;
-    }
-    if (elect_one()) tc_commit(o_full);
-    __syncwarp();
-  } else {
-    // ---------------- softmax warps: group g takes key tiles j ≡ g (mod 2); thread = one query
-    // row × one 64-key half of those tiles
-    const int g = warp >> 3;
-    const int half = (warp >> 2) & 1;
-    const int quarter = warp & 3;
-    const int row = 32 * quarter + lane;
-    const int t = q0 + row;              // query row (local)
-    const int ta = a.q_off + t;          // its position among the keys
-    const int tile0 = a.q_off + q0;
-    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
-    const uint32_t s_addr = tmem + lane_off + S::TM_S + g * 128 + 64 * half;
-    bool ok = mbar_wait_warp(bar_q, 0, abort_flag, a.status);
-    // fixed shift c_t (log2 units)
-    const float qn = sqrtf(q_row_sumsq<DH>(smem + S::OFF_Q, row));
-    const float km = kmax ? kmax[(long long)b * a.Hkv + h / a.group] : kmax_const;
-    const float c_nat = qn * km * a.scale * 1.001f + 1e-3f;
-    if (c_nat > 40.f && t < T && half == 0 && g == 0) set_status(a.status, GPT_ERR_NUMERIC_RANGE);
-    const float c2 = c_nat * LOG2E;
-    // l: exact sum of the weights (gives the LSE); lb: sum of the bf16 weights that P·V uses
-    float l0 = 0.f, l1 = 0.f, lb0 = 0.f, lb1 = 0.f;
-    for (int j = g; j < n_kv && ok; j += 2) {
-      if (!mbar_wait_warp(&s_full[g], (j >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
-      tc_fence_after();
-      const int kv0 = (kv_first + j) * 128 + 64 * half;  // first key of this thread's half
-      const bool need_mask = (kv0 + 63 > tile0) || (kv0 <= tile0 + 127 - W);
-      uint32_t rbuf[2][16];
-      tmem_ld16(s_addr, rbuf[0]);
-      tmem_ld_wait();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t (&r)[16] = rbuf[c & 1];
-        if (c < 3) tmem_ld16(s_addr + 16 * (c + 1), rbuf[(c + 1) & 1]);
-        uint32_t pk[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float x0, x1, p0, p1;
-          fma2_bc(x0, x1, __uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]), a.scale_log2, -c2);
-          if ((e & 3) == 3) {  // one pair in four on the FMA pipe
-            exp2_poly2(p0, p1, x0, x1);
-          } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
-          if (need_mask) {
-            const int key = kv0 + 16 * c + 2 * e;
-            if (!(key <= ta && key > ta - W)) p0 = 0.f;
-            if (!(key + 1 <= ta && key + 1 > ta - W)) p1 = 0.f;
-          }
-          add2_acc(l0, l1, p0, p1);
-          pk[e] = pack_bf2(p0, p1);
-          add2_acc(lb0, lb1, bf_lo(pk[e]), bf_hi(pk[e]));
-        }
-        // P of chunk c overwrites this half's S columns 8c..8c+7, all of which have been read
-        tmem_st8(s_addr + 8 * c, pk);
-        if (c < 3) tmem_ld_wait();
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[g]);
-    }
-    // the four partial sums of a row (2 groups × 2 halves) are combined in a fixed order
-    float2* red = reinterpret_cast<float2*>(smem + S::OFF_RED);
-    red[(g * 2 + half) * 128 + row] = make_float2(l0 + l1, lb0 + lb1);
-    named_barrier_sync(1, 512);  // every softmax thread reaches this, whatever its loop did
-    float l = 0.f, lbs = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 v = red[i * 128 + row];
-      l += v.x;
-      lbs += v.y;
-    }
-    const float inv = 1.f / lbs;
-    // epilogue: O / lb, this thread's quarter of the DH columns
-    if (ok) ok = mbar_wait_warp(o_full, 0, abort_flag, a.status);
-    if (ok) {
-      tc_fence_after();
-      uint16_t* orow = a.o + b * a.sb_o + h * a.sh_o + (long long)t * a.st_o;
-      constexpr int QC = DH / 4;  // columns per thread
-      const int c0 = (g * 2 + half) * QC;
-      uint32_t r[QC];
-      if constexpr (QC == 32) {
-        tmem_ld32(tmem + lane_off + S::TM_O + c0, r);
-      } else {
-        tmem_ld16(tmem + lane_off + S::TM_O + c0, r);
-      }
-      tmem_ld_wait();
-      if (t < T) {
-#pragma unroll
-        for (int u = 0; u < QC / 8; ++u) {
-          uint4 w;
-          w.x = pack_bf2(__uint_as_float(r[8 * u + 0]) * inv, __uint_as_float(r[8 * u + 1]) * inv);
-          w.y = pack_bf2(__uint_as_float(r[8 * u + 2]) * inv, __uint_as_float(r[8 * u + 3]) * inv);
-          w.z = pack_bf2(__uint_as_float(r[8 * u + 4]) * inv, __uint_as_float(r[8 * u + 5]) * inv);
-          w.w = pack_bf2(__uint_as_float(r[8 * u + 6]) * inv, __uint_as_float(r[8 * u + 7]) * inv);
-          *reinterpret_cast<uint4*>(orow + c0 + 8 * u) = w;
-        }
-        if (half == 0 && g == 0) a.lse[((long long)b * a.H + h) * T + t] = (c2 + log2f(l)) * LN2;
-      }
-    }
-  }
-
-  __syncwarp();
-  if (*abort_flag && threadIdx.x == 0) {
-    for (int i = 0; i < 2000; ++i) __nanosleep(1000);
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == S::MMA_WARP) tmem_dealloc(tmem, 512);
-}
 
 // ================================================================================================
 // backward on the tcgen05 tensor cores (head_dim 64 or 128), deterministic kernels
@@ -1239,6 +977,332 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 9) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------------------------------------
+// dK/dV, two softmax groups.  The same products as attn_bwd_dkdv_tc_kernel per (128-key tile,
+// 64-query tile): Sᵀ = K·Qᵀ and dPᵀ = V·dOᵀ into a double-buffered pair of tensor-memory tiles,
+// then dV += Pᵀ·dO and dK += dSᵀ·Q from tensor memory.  Differences:
+//  * 16 softmax-backward warps in two groups; group g takes the query tiles i ≡ g (mod 2), so each
+//    group has two tile-times of tensor work to turn its Sᵀ / dPᵀ into Pᵀ / dSᵀ;
+//  * −LSE and −delta are applied in the softmax arithmetic (one fused multiply-add and one
+//    subtraction per element, fp32 values staged per query tile by a bulk copy) instead of two
+//    K = 16 extension products per tile, which cost as much tensor time as a K = 64 one at N = 64;
+//  * every group works in 16-column chunks (registers for 576 threads);
+//  * the epilogue splits dV (group 0) and dK (group 1) by column halves.
+// ------------------------------------------------------------------------------------------------
+template <int DH>
+struct TcBwd2Shape {
+  static constexpr int BIG_TILE = 128 * DH * 2;
+  static constexpr int SMALL_TILE = 64 * DH * 2;
+  static constexpr int STAGES = 4;
+  static constexpr int OFF_A = 0;                  // K
+  static constexpr int OFF_B = BIG_TILE;           // V
+  static constexpr int OFF_STAGE = 2 * BIG_TILE;   // stages of (Q, dO)
+  static constexpr int STAGE_BYTES = 2 * SMALL_TILE;
+  static constexpr int OFF_LD = OFF_STAGE + STAGES * STAGE_BYTES;  // [stage][LSE·log2 e | delta][64] fp32
+  static constexpr int LD_BYTES = 2 * 64 * 4;
+  static constexpr int OFF_BAR = OFF_LD + STAGES * LD_BYTES;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int THREADS = 576;  // 16 softmax warps (two groups of 8), TMA, MMA
+  static constexpr int W_TMA = 16, W_MMA = 17;
+  static constexpr int TM_S = 0, TM_P = 128, TM_ACC = 256;  // S[b] at b·64, dP[b] at 128 + b·64
+};
+
+// QK-norm + RoPE backward of one key row held in tensor memory (columns taddr .. taddr+DH−1 of this
+// thread's lane, times `scale`), writing rotation pairs [part·DH/4, (part+1)·DH/4) and their partners
+// + DH/2: the dot product with ŷ runs over the whole row, the output over this part only, in
+// 16-column chunks.  Whole warps only (tcgen05.ld is warp-wide).
+template <int DH, int ROWS>
+__device__ __forceinline__ void qknorm_rope_bwd_tmem_part(uint32_t taddr, float scale, const uint8_t* tile,
+                                                          int r, float rho, const float* cs_t,
+                                                          uint16_t* dst, bool store, int part) {
+  constexpr int HALF = DH / 2, QUART = DH / 4;
+  float dot = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < DH / 16; ++c) {
+    uint32_t v[16];
+    tmem_ld16(taddr + 16 * c, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int jj = 0; jj < 2; ++jj) {
+      float y[8];
+      load_y8<ROWS>(tile, r, 16 * c + 8 * jj, y);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dot += __uint_as_float(v[8 * jj + e]) * y[e];
+    }
+  }
+  dot = dot * scale / (float)DH;
+  const float4* cs4 = reinterpret_cast<const float4*>(cs_t);
+#pragma unroll 1
+  for (int c = 0; c < QUART / 16; ++c) {
+    const int j0 = part * QUART + 16 * c;
+    uint32_t va[16], vb[16];
+    tmem_ld16(taddr + j0, va);
+    tmem_ld16(taddr + HALF + j0, vb);
+    tmem_ld_wait();
+#pragma unroll
+    for (int jj = 0; jj < 2; ++jj) {
+      const int j = j0 + 8 * jj;
+      float ya[8], yb[8], oa[8], ob[8];
+      load_y8<ROWS>(tile, r, j, ya);
+      load_y8<ROWS>(tile, r, j + HALF, yb);
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const float4 w = cs4[(j + e) / 2];  // cos_j, sin_j, cos_{j+1}, sin_{j+1}
+        const float a0 = rho * (__uint_as_float(va[8 * jj + e]) * scale - ya[e] * dot);
+        const float b0 = rho * (__uint_as_float(vb[8 * jj + e]) * scale - yb[e] * dot);
+        const float a1 = rho * (__uint_as_float(va[8 * jj + e + 1]) * scale - ya[e + 1] * dot);
+        const float b1 = rho * (__uint_as_float(vb[8 * jj + e + 1]) * scale - yb[e + 1] * dot);
+        oa[e] = a0 * w.x + b0 * w.y;
+        ob[e] = -a0 * w.y + b0 * w.x;
+        oa[e + 1] = a1 * w.z + b1 * w.w;
+        ob[e + 1] = -a1 * w.w + b1 * w.z;
+      }
+      if (store) {
+        uint4 pa, pb;
+        pa.x = pack_bf2(oa[0], oa[1]); pa.y = pack_bf2(oa[2], oa[3]);
+        pa.z = pack_bf2(oa[4], oa[5]); pa.w = pack_bf2(oa[6], oa[7]);
+        pb.x = pack_bf2(ob[0], ob[1]); pb.y = pack_bf2(ob[2], ob[3]);
+        pb.z = pack_bf2(ob[4], ob[5]); pb.w = pack_bf2(ob[6], ob[7]);
+        *reinterpret_cast<uint4*>(dst + j) = pa;
+        *reinterpret_cast<uint4*>(dst + j + HALF) = pb;
+      }
+    }
+  }
+}
+
+template <int DH>
+__global__ void __launch_bounds__(576, 1)
+    attn_bwd_dkdv2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                          const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
+                          const AttnArgs a) {
+  using S = TcBwd2Shape<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
+  uint64_t* kv_bar = bars;
+  uint64_t* q_full = bars + 1;                // [STAGES]
+  uint64_t* q_empty = q_full + S::STAGES;     // [STAGES]
+  uint64_t* s_full = q_empty + S::STAGES;     // [2]
+  uint64_t* p_full = s_full + 2;              // [2]
+  uint64_t* done = p_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int hk = blockIdx.y, b = blockIdx.z;  // one key/value head; its group's query heads in turn
+  const int T = a.T, W = a.window;
+  const int kv0 = blockIdx.x * 128;
+  const int q_first = kv0 / 64;
+  // with dSᵀ stored, cover every 128-query tile that reads one of these keys (tiles beyond the
+  // window are fully masked and store zeros)
+  const int q_reach = a.ds_t ? ((kv0 + 126 + W) / 128) * 128 + 127 : kv0 + 127 + W - 1;
+  const int q_last = min(T - 1, q_reach) / 64;
+  const int n_qt = q_last - q_first + 1;  // query tiles per query head
+  const int n_q = n_qt * a.group;         // iterations: query head hk·group + i / n_qt, tile i % n_qt
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_bar, 1);
+    for (int i = 0; i < S::STAGES; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 256);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == S::W_MMA) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
+
+  if (warp == S::W_TMA) {
+    // ---------------- TMA producer: K, V once; per query tile Q, dO and the LSE / delta values ----------------
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_bar, 2 * S::BIG_TILE);
+      load_tile<DH, 128>(smem + S::OFF_A, &mk, kv_bar, kv0, hk, b);
+      load_tile<DH, 128>(smem + S::OFF_B, &mv, kv_bar, kv0, hk, b);
+      const long long rows = (long long)a.B * a.H * a.Tpad;
+      for (int i = 0; i < n_q; ++i) {
+        const int st = i % S::STAGES;
+        if (!mbar_wait(&q_empty[st], ((i / S::STAGES) & 1) ^ 1, abort_flag, a.status)) break;
+        const int h = hk * a.group + i / n_qt;
+        const long long bh = (long long)b * a.H + h;
+        const int t0 = (q_first + i % n_qt) * 64;
+        mbar_arrive_expect_tx(&q_full[st], S::STAGE_BYTES + S::LD_BYTES);
+        uint8_t* dst = smem + S::OFF_STAGE + st * S::STAGE_BYTES;
+        load_tile<DH, 64>(dst, &mq, &q_full[st], t0, h, b);
+        load_tile<DH, 64>(dst + S::SMALL_TILE, &mdo, &q_full[st], t0, h, b);
+        uint8_t* ld = smem + S::OFF_LD + st * S::LD_BYTES;
+        const long long row = bh * a.Tpad + t0;
+        bulk_load(ld, a.delta + row, 256, &q_full[st]);               // LSE·log2 e
+        bulk_load(ld + 256, a.delta + rows + row, 256, &q_full[st]);  // delta
+      }
+    }
+  } else if (warp == S::W_MMA) {
+    // ---------------- MMA issuer: the warp runs the loop, one elected lane issues ----------------
+    constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
+    constexpr uint32_t id_acc = idesc_bf16(128, DH, false, true);
+    const uint64_t kd = sdesc_sw128(smem_u32(smem + S::OFF_A), 16, 1024);
+    const uint64_t vd = sdesc_sw128(smem_u32(smem + S::OFF_B), 16, 1024);
+    const uint32_t stage0 = smem_u32(smem + S::OFF_STAGE);
+    const uint64_t q_k = sdesc_sw128(stage0, 16, 1024);                          // Q, K-major
+    const uint64_t do_k = sdesc_sw128(stage0 + S::SMALL_TILE, 16, 1024);         // dO, K-major
+    const uint64_t q_mn = sdesc_sw128(stage0, 64 * 128, 1024);                   // Q, MN-major
+    const uint64_t do_mn = sdesc_sw128(stage0 + S::SMALL_TILE, 64 * 128, 1024);  // dO, MN-major
+    bool ok = mbar_wait_warp(kv_bar, 0, abort_flag, a.status);
+    auto issue_acc = [&](int i) {  // dV += Pᵀ·dOᵢ, dK += dSᵀ·Qᵢ
+      const int bf = i & 1;
+      const uint32_t so = (i % S::STAGES) * S::STAGE_BYTES;
+      if (elect_one()) {
+        mma_acc_from_tmem<DH>(tmem + S::TM_ACC, tmem + S::TM_S + bf * 64, sdesc_add(do_mn, so), id_acc, i == 0);
+        mma_acc_from_tmem<DH>(tmem + S::TM_ACC + DH, tmem + S::TM_P + bf * 64, sdesc_add(q_mn, so), id_acc, i == 0);
+        tc_commit(&q_empty[i % S::STAGES]);
+      }
+      __syncwarp();
+    };
+    for (int i = 0; i < n_q && ok; ++i) {
+      const int st = i % S::STAGES, bf = i & 1;
+      if (!mbar_wait_warp(&q_full[st], (i / S::STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t so = st * S::STAGE_BYTES;
+      if (elect_one()) {
+        mma_rows_128x64<DH>(tmem + S::TM_S + bf * 64, kd, sdesc_add(q_k, so), id_s);    // Sᵀ
+        mma_rows_128x64<DH>(tmem + S::TM_P + bf * 64, vd, sdesc_add(do_k, so), id_s);   // dPᵀ
+        tc_commit(&s_full[bf]);
+      }
+      __syncwarp();
+      if (i >= 1) {
+        if (!mbar_wait_warp(&p_full[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
+        issue_acc(i - 1);
+      }
+    }
+    if (ok && n_q >= 1) {
+      if (mbar_wait_warp(&p_full[(n_q - 1) & 1], ((n_q - 1) >> 1) & 1, abort_flag, a.status)) {
+        tc_fence_after();
+        issue_acc(n_q - 1);
+      }
+    }
+    if (elect_one()) tc_commit(done);
+    __syncwarp();
+  } else {
+    // ---------------- softmax-backward warps: thread = key row, warp half = 32 of the 64 queries,
+    // group = parity of the query tiles it takes
+    const int quarter = warp & 3, half = (warp >> 2) & 1, grp = warp >> 3;
+    const int kr = 32 * quarter + lane;
+    const int key = kv0 + kr;
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    const int kmin = kv0 + 32 * quarter, kmax_ = kmin + 31;  // this warp's keys
+    bool ok = true;
+    for (int i = grp; i < n_q && ok; i += 2) {
+      const int st = i % S::STAGES;
+      if (!mbar_wait_warp(&s_full[grp], (i >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+      tc_fence_after();
+      const long long bh = (long long)b * a.H + hk * a.group + i / n_qt;  // the query head
+      const int qh = (q_first + i % n_qt) * 64 + 32 * half;  // first query of this warp's 32 columns
+      const float* ldl = reinterpret_cast<const float*>(smem + S::OFF_LD + st * S::LD_BYTES) + 32 * half;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        const int qc = qh + 16 * c;
+        uint32_t rs[16], rp[16];
+        tmem_ld16(tmem + lane_off + S::TM_S + grp * 64 + 32 * half + 16 * c, rs);
+        tmem_ld16(tmem + lane_off + S::TM_P + grp * 64 + 32 * half + 16 * c, rp);
+        tmem_ld_wait();
+        // every (key, query) of the chunk visible: no per-element mask
+        const bool full = (kmax_ <= qc) && (kmin > qc + 15 - W) && (qc + 15 < T);
+        uint32_t pk[8], dk[8];
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(ldl + 16 * c + 4 * g4);        // LSE·log2 e
+          const float4 d4 = *reinterpret_cast<const float4*>(ldl + 64 + 16 * c + 4 * g4);   // delta
+#pragma unroll
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const int j = 4 * g4 + 2 * e2;
+            const float la = e2 ? l4.z : l4.x, lb = e2 ? l4.w : l4.y;
+            const float da = e2 ? d4.z : d4.x, db = e2 ? d4.w : d4.y;
+            float x0, x1, u0, u1, s0, s1;
+            fma2(x0, x1, __uint_as_float(rs[j]), __uint_as_float(rs[j + 1]), a.scale_log2, a.scale_log2, -la, -lb);
+            float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            if (!full) {
+              const int qq = qc + j;
+              if (!((qq < T) && (key <= qq) && (key > qq - W))) p0 = 0.f;
+              if (!((qq + 1 < T) && (key <= qq + 1) && (key > qq + 1 - W))) p1 = 0.f;
+            }
+            sub2(u0, u1, __uint_as_float(rp[j]), __uint_as_float(rp[j + 1]), da, db);
+            mul2(s0, s1, p0, p1, u0, u1);
+            pk[j / 2] = pack_bf2(p0, p1);
+            dk[j / 2] = pack_bf2(s0, s1);
+          }
+        }
+        if (a.ds_t != nullptr && key < T) {
+          uint4* dst = reinterpret_cast<uint4*>(a.ds_t + ((size_t)bh * T + key) * a.Tpad + qc);
+          dst[0] = make_uint4(dk[0], dk[1], dk[2], dk[3]);
+          dst[1] = make_uint4(dk[4], dk[5], dk[6], dk[7]);
+        }
+        // packed: chunk c of half h fills columns 32h + 8c .. +7, inside what this warp has read
+        tmem_st8(tmem + lane_off + S::TM_S + grp * 64 + 32 * half + 8 * c, pk);
+        tmem_st8(tmem + lane_off + S::TM_P + grp * 64 + 32 * half + 8 * c, dk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[grp]);
+    }
+    // epilogue: group 0 writes dV, group 1 dK, each warp half one part of the row
+    if (ok) ok = mbar_wait_warp(done, 0, abort_flag, a.status);
+    if (ok) {
+      tc_fence_after();
+      const long long off = b * a.sb_g + hk * a.sh_g + (long long)key * a.st_g;
+      if (grp == 1 && a.rho_k != nullptr) {
+        const bool valid = key < T;
+        const float rho = valid ? a.rho_k[((long long)b * T + key) * a.Hkv + hk] : 0.f;
+        qknorm_rope_bwd_tmem_part<DH, 128>(tmem + lane_off + S::TM_ACC + DH, a.scale, smem + S::OFF_A, kr,
+                                           rho, a.cos_sin + (size_t)(valid ? key : 0) * DH, a.dk + off,
+                                           valid, half);
+      } else {
+        uint16_t* dst = (grp == 0 ? a.dv : a.dk) + off;
+        const float sc = (grp == 0) ? 1.f : a.scale;
+#pragma unroll 1
+        for (int c = 0; c < DH / 32; ++c) {
+          const int col = half * (DH / 2) + 16 * c;
+          uint32_t r[16];
+          tmem_ld16(tmem + lane_off + S::TM_ACC + grp * DH + col, r);
+          tmem_ld_wait();
+          if (key < T) {
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              uint4 w;
+              w.x = pack_bf2(__uint_as_float(r[8 * u + 0]) * sc, __uint_as_float(r[8 * u + 1]) * sc);
+              w.y = pack_bf2(__uint_as_float(r[8 * u + 2]) * sc, __uint_as_float(r[8 * u + 3]) * sc);
+              w.z = pack_bf2(__uint_as_float(r[8 * u + 4]) * sc, __uint_as_float(r[8 * u + 5]) * sc);
+              w.w = pack_bf2(__uint_as_float(r[8 * u + 6]) * sc, __uint_as_float(r[8 * u + 7]) * sc);
+              *reinterpret_cast<uint4*>(dst + col + 8 * u) = w;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  if (*abort_flag && threadIdx.x == 0) {
+    for (int i = 0; i < 2000; ++i) __nanosleep(1000);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == S::W_MMA) tmem_dealloc(tmem, 512);
 }
 
 template <int DH>
@@ -2040,26 +2104,9 @@ gpt_status launch_fwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, c
   return launch_kernel(attn_fwd_kernel<DH>, grid, dim3(256), FwdShape<DH>::SMEM, stream, mq, mk, mv, a);
 }
 
-// Forward kernel choice: one query tile per CTA with double-buffered scores (default) or two query
-// tiles per CTA sharing each K/V tile (GPTSTEP_ATTN_FWD=2).
-static bool fwd_one_tile() {
-  static const bool one = [] {
-    const char* v = std::getenv("GPTSTEP_ATTN_FWD");
-    return !(v && v[0] == '2');
-  }();
-  return one;
-}
-
 template <int DH>
 gpt_status launch_fwd_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const AttnArgs& a, const float* kmax, float kmax_const, cudaStream_t stream) {
-  if (fwd_one_tile()) {
-    using S1 = TcFwd1Shape<DH>;
-    GPT_TRY(ensure_smem(attn_fwd_tc1_kernel<DH>, S1::SMEM));
-    dim3 grid((a.T + 127) / 128, a.H, a.B);
-    return launch_kernel(attn_fwd_tc1_kernel<DH>, grid, dim3(S1::THREADS), S1::SMEM, stream, mq, mk, mv, a,
-                         kmax, kmax_const);
-  }
   using S = TcFwdShape<DH>;
   GPT_TRY(ensure_smem(attn_fwd_tc_kernel<DH>, S::SMEM));
   dim3 grid((a.T + 255) / 256, a.H, a.B);
@@ -2078,6 +2125,16 @@ gpt_status launch_bwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, c
   return launch_kernel(attn_bwd_dq_kernel<DH>, grid, dim3(128), smem, stream, mq, mk, mv, mdo, a);
 }
 
+// dK/dV kernel choice: two softmax groups with −LSE / −delta in the softmax arithmetic (default) or
+// one group with the extension products (GPTSTEP_ATTN_BWD=1).
+static bool bwd_two_groups() {
+  static const bool two = [] {
+    const char* v = std::getenv("GPTSTEP_ATTN_BWD");
+    return !(v && v[0] == '1');
+  }();
+  return two;
+}
+
 // tcgen05 backward: maps with 128-row boxes (outer tiles) and 64-row boxes (inner tiles), and the
 // [2·B·H·Tpad][8] bf16 extension rows in 64-row boxes.
 template <int DH>
@@ -2085,14 +2142,21 @@ gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[
                          const CUtensorMap& mext, const CUtensorMap* mds, AttnArgs a, void* dq,
                          cudaStream_t stream) {
   using S = TcBwdShape<DH>;
+  using S2 = TcBwd2Shape<DH>;
   using SD = DqDsShape<DH>;
-  GPT_TRY(ensure_smem(attn_bwd_dkdv_tc_kernel<DH>, S::SMEM));
   GPT_TRY(ensure_smem(attn_bwd_dq_tc_kernel<DH>, S::SMEM));
   GPT_TRY(ensure_smem(attn_bwd_dq_ds_kernel<DH>, SD::SMEM));
   // dK/dV: outer 128-key tiles (K, V with 128-row boxes), inner 64-query tiles (Q, dO 64-row boxes)
   dim3 g1((a.T + 127) / 128, a.Hkv, a.B);  // one CTA per key tile of each key/value head
-  GPT_TRY(launch_kernel(attn_bwd_dkdv_tc_kernel<DH>, g1, dim3(S::THREADS), S::SMEM, stream, m64[0],
-                        m128[1], m128[2], m64[3], mext, a));
+  if (bwd_two_groups()) {
+    GPT_TRY(ensure_smem(attn_bwd_dkdv2_kernel<DH>, S2::SMEM));
+    GPT_TRY(launch_kernel(attn_bwd_dkdv2_kernel<DH>, g1, dim3(S2::THREADS), S2::SMEM, stream, m64[0],
+                          m128[1], m128[2], m64[3], a));
+  } else {
+    GPT_TRY(ensure_smem(attn_bwd_dkdv_tc_kernel<DH>, S::SMEM));
+    GPT_TRY(launch_kernel(attn_bwd_dkdv_tc_kernel<DH>, g1, dim3(S::THREADS), S::SMEM, stream, m64[0],
+                          m128[1], m128[2], m64[3], mext, a));
+  }
   a.o = reinterpret_cast<uint16_t*>(dq);
   dim3 g2((a.T + 127) / 128, a.H, a.B);
   if (mds != nullptr) {

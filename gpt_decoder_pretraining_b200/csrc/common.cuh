@@ -149,6 +149,16 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Contiguous bytes from global to shared memory (no tensor map): both addresses 16-byte aligned,
+// `bytes` a multiple of 16; completes `bytes` of transaction count on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ------------------------------------------------------------------------------------------------
 // tcgen05: tensor memory allocation, MMA, commit, loads
 // ------------------------------------------------------------------------------------------------
@@ -461,6 +471,18 @@ __device__ __forceinline__ void fma2_b(float& d0, float& d1, float a0, float a1,
       "mov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b), "f"(c0), "f"(c1));
+}
+// (d0, d1) = (a0·b + c0, a1·b + c1) is fma2_b; (d0, d1) = (a0·b0 + c0, a1·b1 + c1):
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                     float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
 // (d0, d1) = (a0 − b0, a1 − b1)
 __device__ __forceinline__ void sub2(float& d0, float& d1, float a0, float a1, float b0, float b1) {

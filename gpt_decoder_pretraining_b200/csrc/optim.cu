@@ -238,8 +238,7 @@ gpt_status muon_step(float* w, void* params, int param_dtype, const float* g, fl
   if (groups <= 0 || per <= 0 || rows <= 0 || cols <= 0 || ns_steps < 0) return GPT_ERR_INVALID_ARG;
   if (param_dtype != GPT_DTYPE_BF16 && param_dtype != GPT_DTYPE_F32) return GPT_ERR_INVALID_ARG;
   const long long mat = (long long)rows * cols;
-  if (per > 1 && gstride < per * mat) return GPT_ERR_INVALID_ARG;
-  if (groups > 1 && gstride < mat) return GPT_ERR_INVALID_ARG;
+  if (groups > 1 && gstride < per * mat) return GPT_ERR_INVALID_ARG;  // groups must not overlap
   if ((rows % 8) || (cols % 8)) return GPT_ERR_UNSUPPORTED_SHAPE;  // 16-byte rows for TMA
   const int nb = groups * per;
   if (scratch_bytes < muon_scratch_bytes(nb, rows, cols)) return GPT_ERR_WORKSPACE_TOO_SMALL;

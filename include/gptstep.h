@@ -391,7 +391,8 @@ gpt_status gpt_adamw_step(float* master, void* params, int param_dtype, const fl
  *   W ← W − lr·√max(1, rows/cols)·X
  * The Newton–Schulz products are batched tcgen05 GEMMs over the group in bf16 with fp32
  * accumulation (the precision the method is published with); ‖u‖ is summed in a fixed order.
- * rows, cols multiples of 8.  scratch ≥ gpt_muon_scratch_bytes(n, rows, cols), 256-byte aligned. */
+ * rows, cols multiples of 8; with groups > 1, group_stride ≥ per_group·rows·cols (ignored for one
+ * group).  scratch ≥ gpt_muon_scratch_bytes(n, rows, cols), 256-byte aligned. */
 size_t gpt_muon_scratch_bytes(int n_matrices, int rows, int cols);
 gpt_status gpt_muon_step(float* master, void* params, int param_dtype, const float* grads,
                          float* momentum_buf, int groups, int per_group, long long group_stride,

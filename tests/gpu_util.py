@@ -42,3 +42,12 @@ def assert_close_rel(got, ref, rel=1e-2, cos=0.9999, what="", atol=1e-6):
     if scale > 100 * atol:
         c = cosine(got, ref)
         assert c >= cos, f"{what}: cosine {c:.6f} < {cos}"
+
+
+def f32_accum_rel(K: int) -> float:
+    """Relative tolerance (of max |C|) for an fp32-accumulated product over K exactly representable
+    bf16 terms.  Each partial sum is rounded to 2^-24 of its size; with terms of random sign the
+    rounding errors add like a random walk, so the error of C grows like √K · 2^-24 times the
+    typical partial sum, which is about max |C| / 3 for these inputs.  5e-7·√K is about 25× that
+    estimate; the products of a tile's K loop accumulate in the tensor core in its own order."""
+    return max(1e-5, 5e-7 * float(np.sqrt(K)))

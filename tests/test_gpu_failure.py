@@ -16,7 +16,7 @@ import pytest
 import torch
 
 from oracle import gpt_oracle as O
-from tests.gpu_util import assert_close_rel, bf16_tensor, randn, to_np
+from tests.gpu_util import f32_accum_rel, assert_close_rel, bf16_tensor, randn, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -109,7 +109,7 @@ def test_gemm_wait_timeout_returns_status_then_recovers(op):
     S.gemm(op, S.EPI_F32, tA, tB, C, M, N, K, status=st2, scratch=None)
     torch.cuda.synchronize()
     assert int(st2.item()) == 0
-    assert_close_rel(to_np(C), ref, rel=1e-5, cos=0.9999999, what="gemm after recovery")
+    assert_close_rel(to_np(C), ref, rel=f32_accum_rel(K), cos=0.9999999, what="gemm after recovery")
 
 
 def test_attention_wait_timeout_returns_status_then_recovers():

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 from oracle import gpt_oracle as O
-from tests.gpu_util import assert_close_rel, bf16_tensor, cosine, randn, to_np
+from tests.gpu_util import f32_accum_rel, assert_close_rel, bf16_tensor, cosine, randn, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -89,7 +89,7 @@ def test_gemm_epilogues(M, N, K):
 # Shapes whose tile count leaves the last wave of CTA pairs partly empty, so that the GEMM splits
 # the tail tiles along K: fewer tiles than CTA pairs (every tile in two pieces), a weight-gradient
 # shape of 100 tiles (one whole wave, 26 tail tiles in two pieces), and 84 ragged tiles.
-SK_SHAPES = [(1536, 1536, 16384, 2), (1280, 5120, 8192, 2), (3000, 1700, 2560, 0), (3000, 1700, 2560, 1)]
+SK_SHAPES = [(1536, 1536, 16384, 2), (1280, 5120, 8192, 2), (3000, 1704, 2560, 0), (3000, 1704, 2560, 1)]
 
 
 @pytest.mark.parametrize("M,N,K,op", SK_SHAPES)
@@ -108,11 +108,12 @@ def test_gemm_stream_k_tail_matches_fp64_and_is_reproducible(M, N, K, op):
     S.gemm(op, S.EPI_F32, tA, tB, Cn, M, N, K, status=st, scratch=None)  # every tile whole
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    assert_close_rel(to_np(C1), ref, rel=1e-5, cos=0.9999999, what="f32 stream-K")
+    tol = f32_accum_rel(K)
+    assert_close_rel(to_np(C1), ref, rel=tol, cos=0.9999999, what="f32 split tail")
     assert torch.equal(C1, C2)  # bitwise reproducible
-    assert_close_rel(to_np(Cn), ref, rel=1e-5, cos=0.9999999, what="f32 whole tiles")
-    # both within 1e-5 of the fp64 product: they differ from each other only by fp32 summation order
-    assert_close_rel(to_np(C1), to_np(Cn), rel=2e-5, cos=0.9999999, what="stream-K vs whole tiles")
+    assert_close_rel(to_np(Cn), ref, rel=tol, cos=0.9999999, what="f32 whole tiles")
+    # both within tol of the fp64 product: they differ from each other only by fp32 summation order
+    assert_close_rel(to_np(C1), to_np(Cn), rel=2 * tol, cos=0.9999999, what="split vs whole tiles")
     if op == 2:
         return
     # the element-wise epilogues on the same split schedule
