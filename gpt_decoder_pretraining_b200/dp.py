@@ -149,7 +149,7 @@ def device_update_fns(cfg, master, params, grads, state_m, state_v, hp: dict, wo
     the owned layers are `world` layers apart, which is the group stride — and AdamW
     (gpt_adamw_step) on row ranges of wte and W_lm with learning rates × 1/√(d/768).  Buffers are
     the full flat packing (master, grads, state fp32; params in the step's dtype)."""
-    import math
+    import numpy as np
 
     from . import step as S
     layers_rng, offs, total = _layer_ranges(cfg)
@@ -184,11 +184,14 @@ def device_update_fns(cfg, master, params, grads, state_m, state_v, hp: dict, wo
     def update_rows(r0, r1, t):
         if r1 <= r0:
             return
-        scale = 1.0 / math.sqrt(d / 768.0)
+        # the learning-rate scale in fp32, formed as gpt_optim_step forms it, so that both give
+        # bitwise the same update
+        scale = np.float32(1.0) / np.sqrt(np.float32(d) / np.float32(768.0))
         for base, lr_t in ((offs[0], hp["adam_lr_wte"]), (offs[-1], hp["adam_lr_lm"])):
             a, b = base + r0 * d, base + r1 * d
+            lr32 = float(np.float32(lr_t) * scale)
             S.adamw_step(master[a:b], sl(params, a, b), grads[a:b], state_m[a:b], state_v[a:b], t,
-                         lr_t * scale, hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"],
+                         lr32, hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"],
                          param_dtype=cfg.param_dtype)
 
     return update_layers, update_rows
