@@ -11,10 +11,11 @@
 //   forward     grid (256-query blocks, H, B): 2 query tiles of 128, 16 softmax warps.  Each row's
 //               exponentials are shifted by the Cauchy–Schwarz bound ‖q‖·max‖k‖/√Dh rather than a
 //               running maximum (softmax is shift-invariant), so O needs no rescaling.
-//   backward    (1) delta pre-pass: rowsum(dO∘O), LSE, and their bf16 "extension rows";
+//   backward    (1) delta pre-pass: rowsum(dO∘O) and LSE·log2 e per row (or formed by the GEMM
+//                   that produces dO);
 //               (2) dK, dV: grid over 128-key tiles, loop over 64-query tiles; −LSE and −delta enter
-//                   the score accumulators through one extra K = 16 MMA each; dSᵀ is stored;
-//               (3) dQ = dS·K from the stored dSᵀ (or, for the allocation-free entry, with the scores
+//                   the softmax arithmetic; dS is stored query-major;
+//               (3) dQ = dS·K from the stored dS (or, for the allocation-free entry, with the scores
 //                   recomputed).
 // head_dim 32 (small test configurations): m16n8k16 mma.sync kernels with an online softmax.
 // No atomics anywhere: every output element has one writer, so results are bitwise reproducible.
@@ -52,8 +53,8 @@ struct AttnArgs {
   float* lse;
   float* delta;  // backward: [2][B·H][Tpad] fp32 — LSE·log2(e), then rowsum(dO∘O); zero-padded
   int Tpad;      // T rounded up to a multiple of 64
-  uint16_t* ext; // backward: [2][B·H][Tpad][8] bf16 rows [hi, mid, lo, 0…] of −LSE·√Dh, −delta
-  uint16_t* ds_t; // backward (optional): dSᵀ [B·H][T][Tpad] bf16, written by the dK/dV kernel
+  uint16_t* ds;  // backward (optional): dS [B·H][T][Tpad] bf16 (query rows, key columns), written
+                 // by the dK/dV kernel and read by the dQ kernel
   int* status;
   // optional QK-norm + RoPE backward fused into the dq / dk epilogues (rho_q == nullptr: off):
   // q̃ = RMS_Dh(RoPE(q)), so dq = Rᵀ·rho·(dq̃ − q̃·mean(q̃·dq̃)), likewise for k
@@ -587,14 +588,14 @@ __global__ void __launch_bounds__(576, 1)
 // ================================================================================================
 // backward on the tcgen05 tensor cores (head_dim 64 or 128), deterministic kernels
 //
-// dK/dV kernel: one CTA per 128-key tile; loops over the 64-query tiles that see it.
-//   Sᵀ = K·Qᵢᵀ and dPᵀ = V·dOᵢᵀ (128 keys × 64 queries, A and B from shared memory) go to tensor
-//   memory, each followed by a K = 16 extension MMA that adds −LSE·√Dh resp. −delta per query
-//   column; the softmax warps (one key row per thread) form Pᵀ = 2^(Sᵀ·log2 e/√Dh) and
-//   dSᵀ = Pᵀ∘dPᵀ, write both back over Sᵀ / dPᵀ as packed bf16 (and dSᵀ to global memory when the
-//   caller's scratch holds it), and the MMA warp accumulates dV += Pᵀ·dOᵢ and dK += dSᵀ·Qᵢ with A
-//   read from tensor memory.
-// dQ: from the stored dSᵀ (attn_bwd_dq_ds_kernel, below), or with the scores recomputed: one CTA
+// dK/dV kernel (attn_bwd_dkdv_tc_kernel): one CTA per 128-key tile of a key/value head; loops over
+//   the 64-query tiles of its group's query heads that see those keys.  Sᵀ = K·Qᵢᵀ and
+//   dPᵀ = V·dOᵢᵀ (128 keys × 64 queries, A and B from shared memory) go to tensor memory; the softmax
+//   warps (one key row per thread) form Pᵀ = 2^(Sᵀ·log2 e/√Dh − LSE·log2 e) and
+//   dSᵀ = Pᵀ∘(dPᵀ − delta), write both back over Sᵀ / dPᵀ as packed bf16 (and dS to global memory
+//   when the caller's scratch holds it), and the MMA warp accumulates dV += Pᵀ·dOᵢ and
+//   dK += dSᵀ·Qᵢ with A read from tensor memory.
+// dQ: from the stored dS (attn_bwd_dq_ds_kernel, below), or with the scores recomputed: one CTA
 //   per 128-query tile looping over its 64-key tiles, S = Q·Kⱼᵀ, dP = dO·Vⱼᵀ, the softmax warps
 //   (one query row per thread) write dS over S and the MMA warp accumulates dQ += dS·Kⱼ.
 // S/dP buffers are double-buffered in tensor memory, so tile i+1's products run while the softmax
@@ -611,15 +612,7 @@ struct TcBwdShape {
   static constexpr int OFF_B = BIG_TILE;               // V (dkdv) or dO (dq)
   static constexpr int OFF_STAGE = 2 * BIG_TILE;       // stages of (Q, dO) or (K, V)
   static constexpr int STAGE_BYTES = 2 * SMALL_TILE;
-  // dK/dV kernel only: the K = 16 extension operands that fold −LSE and −delta into the Sᵀ / dPᵀ
-  // accumulators (unswizzled core-matrix layout, 16-byte rows).  A_EXT: 128 key rows of
-  // [1, 1, 1, 0, …]; per stage the query tile's [hi, mid, lo, 0, …] rows of −LSE·√Dh and −delta;
-  // ZERO: the second K core column of every extension operand.
-  static constexpr int EXT_ROWS_BYTES = 64 * 16;                     // one 64-row extension tile
-  static constexpr int OFF_A_EXT = OFF_STAGE + STAGES * STAGE_BYTES;  // 128 rows × 16 B
-  static constexpr int OFF_EXT = OFF_A_EXT + 128 * 16;                 // [stage][lse | delta] tiles
-  static constexpr int OFF_ZERO = OFF_EXT + STAGES * 2 * EXT_ROWS_BYTES;
-  static constexpr int OFF_BAR = OFF_ZERO + 128 * 16;
+  static constexpr int OFF_BAR = OFF_STAGE + STAGES * STAGE_BYTES;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr int THREADS = 320;  // 8 softmax warps (two per TMEM lane quarter), TMA, MMA
   static constexpr int TM_S = 0, TM_P = 128, TM_ACC = 256;  // S[b] at b·64, dP[b] at 128 + b·64
@@ -724,275 +717,17 @@ __device__ __forceinline__ void qknorm_rope_bwd_tmem(uint32_t taddr, float scale
   }
 }
 
-template <int DH>
-__global__ void __launch_bounds__(320, 1)
-    attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-                            const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
-                            const __grid_constant__ CUtensorMap mext, const AttnArgs a) {
-  using S = TcBwdShape<DH>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
-  uint64_t* kv_bar = bars;
-  uint64_t* q_full = bars + 1;                // [STAGES]
-  uint64_t* q_empty = q_full + S::STAGES;     // [STAGES]
-  uint64_t* s_full = q_empty + S::STAGES;     // [2]
-  uint64_t* p_full = s_full + 2;              // [2]
-  uint64_t* done = p_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = warp_id(), lane = lane_id();
-  const int hk = blockIdx.y, b = blockIdx.z;  // one key/value head; its group's query heads in turn
-  const int T = a.T, W = a.window;
-  const int kv0 = blockIdx.x * 128;
-  const int q_first = kv0 / 64;
-  // with dSᵀ stored, cover every 128-query tile that reads one of these keys (tiles beyond the
-  // window are fully masked and store zeros)
-  const int q_reach = a.ds_t ? ((kv0 + 126 + W) / 128) * 128 + 127 : kv0 + 127 + W - 1;
-  const int q_last = min(T - 1, q_reach) / 64;
-  const int n_qt = q_last - q_first + 1;  // query tiles per query head
-  const int n_q = n_qt * a.group;         // iterations: query head hk·group + i / n_qt, tile i % n_qt
-
-  if (threadIdx.x == 0) {
-    mbar_init(kv_bar, 1);
-    for (int i = 0; i < S::STAGES; ++i) {
-      mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 256);
-    }
-    mbar_init(done, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  // constant extension operands: A_EXT rows [1, 1, 1, 0, 0, 0, 0, 0] (bf16), ZERO all zeros
-  for (int r = threadIdx.x; r < 128; r += blockDim.x) {
-    *reinterpret_cast<uint4*>(smem + S::OFF_A_EXT + 16 * r) = make_uint4(0x3F803F80u, 0x3F80u, 0u, 0u);
-    *reinterpret_cast<uint4*>(smem + S::OFF_ZERO + 16 * r) = make_uint4(0u, 0u, 0u, 0u);
-  }
-  fence_proxy_async_smem();
-  if (warp == 9) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  pdl_wait();
-  pdl_trigger();
-
-  if (warp == 8) {
-    // ---------------- TMA producer: K, V once; per query tile Q, dO and the LSE / delta rows ----------------
-    if (lane == 0) {
-      mbar_arrive_expect_tx(kv_bar, 2 * S::BIG_TILE);
-      load_tile<DH, 128>(smem + S::OFF_A, &mk, kv_bar, kv0, hk, b);
-      load_tile<DH, 128>(smem + S::OFF_B, &mv, kv_bar, kv0, hk, b);
-      const int rows = a.B * a.H * a.Tpad;
-      for (int i = 0; i < n_q; ++i) {
-        const int st = i % S::STAGES;
-        if (!mbar_wait(&q_empty[st], ((i / S::STAGES) & 1) ^ 1, abort_flag, a.status)) break;
-        const int h = hk * a.group + i / n_qt;
-        const long long bh = (long long)b * a.H + h;
-        const int t0 = (q_first + i % n_qt) * 64;
-        mbar_arrive_expect_tx(&q_full[st], S::STAGE_BYTES + 2 * S::EXT_ROWS_BYTES);
-        uint8_t* dst = smem + S::OFF_STAGE + st * S::STAGE_BYTES;
-        load_tile<DH, 64>(dst, &mq, &q_full[st], t0, h, b);
-        load_tile<DH, 64>(dst + S::SMALL_TILE, &mdo, &q_full[st], t0, h, b);
-        uint8_t* ext = smem + S::OFF_EXT + st * 2 * S::EXT_ROWS_BYTES;
-        const int row = (int)bh * a.Tpad + t0;
-        tma_load_2d(ext, &mext, &q_full[st], 0, row);                              // −LSE·√Dh
-        tma_load_2d(ext + S::EXT_ROWS_BYTES, &mext, &q_full[st], 0, rows + row);  // −delta
-      }
-    }
-  } else if (warp == 9) {
-    // ---------------- MMA issuer: the warp runs the loop, one elected lane issues ----------------
-    {
-      constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
-      constexpr uint32_t id_acc = idesc_bf16(128, DH, false, true);
-      const uint64_t kd = sdesc_sw128(smem_u32(smem + S::OFF_A), 16, 1024);
-      const uint64_t vd = sdesc_sw128(smem_u32(smem + S::OFF_B), 16, 1024);
-      const uint32_t stage0 = smem_u32(smem + S::OFF_STAGE);
-      const uint64_t q_k = sdesc_sw128(stage0, 16, 1024);                          // Q, K-major
-      const uint64_t do_k = sdesc_sw128(stage0 + S::SMALL_TILE, 16, 1024);         // dO, K-major
-      const uint64_t q_mn = sdesc_sw128(stage0, 64 * 128, 1024);                   // Q, MN-major
-      const uint64_t do_mn = sdesc_sw128(stage0 + S::SMALL_TILE, 64 * 128, 1024);  // dO, MN-major
-      // extension operands (K = 16, unswizzled): core matrices 128 B apart along M/N, the second
-      // K core column read from the zero block
-      const uint32_t a_ext = smem_u32(smem + S::OFF_A_EXT);
-      const uint64_t a_ext_d = sdesc_plain(a_ext, S::OFF_ZERO - S::OFF_A_EXT, 128);
-      const uint32_t ext0 = smem_u32(smem + S::OFF_EXT);
-      const uint64_t el_d = sdesc_plain(ext0, S::OFF_ZERO - S::OFF_EXT, 128);
-      const uint64_t ed_d = sdesc_plain(ext0 + S::EXT_ROWS_BYTES, S::OFF_ZERO - S::OFF_EXT - S::EXT_ROWS_BYTES, 128);
-      bool ok = mbar_wait_warp(kv_bar, 0, abort_flag, a.status);
-      auto issue_acc = [&](int i) {  // dV += Pᵀ·dOᵢ, dK += dSᵀ·Qᵢ
-        const int bf = i & 1;
-        const uint32_t so = (i % S::STAGES) * S::STAGE_BYTES;
-        if (elect_one()) {
-          mma_acc_from_tmem<DH>(tmem + S::TM_ACC, tmem + S::TM_S + bf * 64, sdesc_add(do_mn, so), id_acc, i == 0);
-          mma_acc_from_tmem<DH>(tmem + S::TM_ACC + DH, tmem + S::TM_P + bf * 64, sdesc_add(q_mn, so), id_acc, i == 0);
-          tc_commit(&q_empty[i % S::STAGES]);
-        }
-        __syncwarp();
-      };
-      for (int i = 0; i < n_q && ok; ++i) {
-        const int st = i % S::STAGES, bf = i & 1;
-        if (!mbar_wait_warp(&q_full[st], (i / S::STAGES) & 1, abort_flag, a.status)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t so = st * S::STAGE_BYTES;
-        // the extension tiles of stage st sit st·2 tiles further from the zero block: their K
-        // core stride shrinks by the same amount (descriptor bits 16..29 hold it in 16-byte units)
-        const uint64_t lbo_fix = (uint64_t)((st * 2 * S::EXT_ROWS_BYTES) >> 4) << 16;
-        const uint32_t eo = st * 2 * S::EXT_ROWS_BYTES;
-        const uint64_t el_st = sdesc_add(el_d, eo) - lbo_fix, ed_st = sdesc_add(ed_d, eo) - lbo_fix;
-        const uint64_t q_st = sdesc_add(q_k, so), do_st = sdesc_add(do_k, so);
-        if (elect_one()) {
-          mma_rows_128x64<DH>(tmem + S::TM_S + bf * 64, kd, q_st, id_s);    // Sᵀ
-          mma_bf16_ss(tmem + S::TM_S + bf * 64, a_ext_d, el_st, id_s, 1u);
-          mma_rows_128x64<DH>(tmem + S::TM_P + bf * 64, vd, do_st, id_s);   // dPᵀ
-          mma_bf16_ss(tmem + S::TM_P + bf * 64, a_ext_d, ed_st, id_s, 1u);
-          tc_commit(&s_full[bf]);
-        }
-        __syncwarp();
-        if (i >= 1) {
-          if (!mbar_wait_warp(&p_full[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
-          tc_fence_after();
-          issue_acc(i - 1);
-        }
-      }
-      if (ok && n_q >= 1) {
-        if (mbar_wait_warp(&p_full[(n_q - 1) & 1], ((n_q - 1) >> 1) & 1, abort_flag, a.status)) {
-          tc_fence_after();
-          issue_acc(n_q - 1);
-        }
-      }
-      if (elect_one()) tc_commit(done);
-      __syncwarp();
-    }
-  } else {
-    // ---------------- softmax-backward warps: thread = key row, warp half = 32 of the 64 queries
-    const int quarter = warp & 3, half = warp >> 2;
-    const int kr = 32 * quarter + lane;
-    const int key = kv0 + kr;
-    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
-    bool ok = true;
-    uint32_t rs[32], rp[32];
-    if (n_q > 0) {
-      ok = mbar_wait_warp(&s_full[0], 0, abort_flag, a.status);
-      if (ok) {
-        tc_fence_after();
-        tmem_ld32(tmem + lane_off + S::TM_S + 32 * half, rs);
-        tmem_ld32(tmem + lane_off + S::TM_P + 32 * half, rp);
-        tmem_ld_wait();
-      }
-    }
-    for (int i = 0; i < n_q && ok; ++i) {
-      const int bf = i & 1;
-      const long long bh = (long long)b * a.H + hk * a.group + i / n_qt;  // the query head
-      const int qc = (q_first + i % n_qt) * 64 + 32 * half;  // first query of this warp's 32 columns
-      // every (key, query) of the warp visible: no per-element mask
-      const int kmin = kv0 + 32 * quarter, kmax_ = kmin + 31;
-      const bool full = (kmax_ <= qc) && (kmin > qc + 31 - W) && (qc + 31 < T);
-      // the accumulators already hold Sᵀ − LSE/scale and dPᵀ − delta (extension MMAs)
-      uint32_t pk[16], dk[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int j = 2 * e;
-        float x0, x1, s0, s1;
-        mul2_b(x0, x1, __uint_as_float(rs[j]), __uint_as_float(rs[j + 1]), a.scale_log2);
-        float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-        if (!full) {
-          const int qq = qc + j;
-          if (!((qq < T) && (key <= qq) && (key > qq - W))) p0 = 0.f;
-          if (!((qq + 1 < T) && (key <= qq + 1) && (key > qq + 1 - W))) p1 = 0.f;
-        }
-        mul2(s0, s1, p0, p1, __uint_as_float(rp[j]), __uint_as_float(rp[j + 1]));
-        pk[e] = pack_bf2(p0, p1);
-        dk[e] = pack_bf2(s0, s1);
-      }
-      if (a.ds_t != nullptr && key < T) {
-        uint4* dst = reinterpret_cast<uint4*>(a.ds_t + ((size_t)bh * T + key) * a.Tpad + qc);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) dst[u] = make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
-      }
-      // packed halves stay inside the columns this warp just read (see mma_acc_from_tmem)
-      tmem_st16(tmem + lane_off + S::TM_S + bf * 64 + 32 * half, pk);
-      tmem_st16(tmem + lane_off + S::TM_P + bf * 64 + 32 * half, dk);
-      // release this tile to the MMA warp first, then fetch the next one's columns
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[bf]);
-      if (i + 1 < n_q) {
-        const int nb = (i + 1) & 1;
-        if (!mbar_wait_warp(&s_full[nb], ((i + 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
-        tc_fence_after();
-        tmem_ld32(tmem + lane_off + S::TM_S + nb * 64 + 32 * half, rs);
-        tmem_ld32(tmem + lane_off + S::TM_P + nb * 64 + 32 * half, rp);
-        tmem_ld_wait();
-      }
-    }
-    // epilogue: half 0 writes the dV row, half 1 the dK row of each key
-    if (ok) ok = mbar_wait_warp(done, 0, abort_flag, a.status);
-    if (ok) {
-      tc_fence_after();
-      const long long off = b * a.sb_g + hk * a.sh_g + (long long)key * a.st_g;
-      if (half == 1 && a.rho_k != nullptr) {
-        const bool valid = key < T;
-        const float rho = valid ? a.rho_k[((long long)b * T + key) * a.Hkv + hk] : 0.f;
-        qknorm_rope_bwd_tmem<DH, 128>(tmem + lane_off + S::TM_ACC + DH, a.scale, smem + S::OFF_A, kr,
-                                      rho, a.cos_sin + (size_t)(valid ? key : 0) * DH, a.dk + off, valid);
-      } else {
-        const int part = half;
-        uint16_t* dst = (part == 0 ? a.dv : a.dk) + off;
-        const float sc = (part == 0) ? 1.f : a.scale;
-#pragma unroll 1
-        for (int c = 0; c < DH / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_off + S::TM_ACC + part * DH + 32 * c, r);
-          tmem_ld_wait();
-          if (key < T) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              uint4 w;
-              w.x = pack_bf2(__uint_as_float(r[8 * u + 0]) * sc, __uint_as_float(r[8 * u + 1]) * sc);
-              w.y = pack_bf2(__uint_as_float(r[8 * u + 2]) * sc, __uint_as_float(r[8 * u + 3]) * sc);
-              w.z = pack_bf2(__uint_as_float(r[8 * u + 4]) * sc, __uint_as_float(r[8 * u + 5]) * sc);
-              w.w = pack_bf2(__uint_as_float(r[8 * u + 6]) * sc, __uint_as_float(r[8 * u + 7]) * sc);
-              *reinterpret_cast<uint4*>(dst + 32 * c + 8 * u) = w;
-            }
-          }
-        }
-      }
-    }
-  }
-
-  __syncwarp();
-  if (*abort_flag && threadIdx.x == 0) {
-    for (int i = 0; i < 2000; ++i) __nanosleep(1000);
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 9) tmem_dealloc(tmem, 512);
-}
-
 // ------------------------------------------------------------------------------------------------
-// dK/dV, two softmax groups.  The same products as attn_bwd_dkdv_tc_kernel per (128-key tile,
-// 64-query tile): Sᵀ = K·Qᵀ and dPᵀ = V·dOᵀ into a double-buffered pair of tensor-memory tiles,
-// then dV += Pᵀ·dO and dK += dSᵀ·Q from tensor memory.  Differences:
-//  * 16 softmax-backward warps in two groups; group g takes the query tiles i ≡ g (mod 2), so each
-//    group has two tile-times of tensor work to turn its Sᵀ / dPᵀ into Pᵀ / dSᵀ;
-//  * −LSE and −delta are applied in the softmax arithmetic (one fused multiply-add and one
-//    subtraction per element, fp32 values staged per query tile by a bulk copy) instead of two
-//    K = 16 extension products per tile, which cost as much tensor time as a K = 64 one at N = 64;
-//  * every group works in 16-column chunks (registers for 576 threads);
-//  * the epilogue splits dV (group 0) and dK (group 1) by column halves.
+// dK/dV kernel.  16 softmax-backward warps in two groups; group g takes the query tiles
+// i ≡ g (mod 2), so each group has two tile-times of tensor work to turn its Sᵀ / dPᵀ into
+// Pᵀ / dSᵀ.  −LSE and −delta enter the softmax arithmetic (one fused multiply-add and one
+// subtraction per element, fp32 values staged per query tile by a bulk copy).  Each warp works in
+// 16-column chunks (registers for 576 threads); the epilogue splits dV (group 0) and dK (group 1)
+// by column halves.  dS goes to global memory query-major: for one query the 32 lanes of a warp
+// hold 32 consecutive keys, so every store instruction writes 64 contiguous bytes.
 // ------------------------------------------------------------------------------------------------
 template <int DH>
-struct TcBwd2Shape {
+struct TcDkdvShape {
   static constexpr int BIG_TILE = 128 * DH * 2;
   static constexpr int SMALL_TILE = 64 * DH * 2;
   static constexpr int STAGES = 4;
@@ -1074,10 +809,10 @@ __device__ __forceinline__ void qknorm_rope_bwd_tmem_part(uint32_t taddr, float 
 
 template <int DH>
 __global__ void __launch_bounds__(576, 1)
-    attn_bwd_dkdv2_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+    attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                           const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
                           const AttnArgs a) {
-  using S = TcBwd2Shape<DH>;
+  using S = TcDkdvShape<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
@@ -1095,9 +830,9 @@ __global__ void __launch_bounds__(576, 1)
   const int T = a.T, W = a.window;
   const int kv0 = blockIdx.x * 128;
   const int q_first = kv0 / 64;
-  // with dSᵀ stored, cover every 128-query tile that reads one of these keys (tiles beyond the
+  // with dS stored, cover every 128-query tile that reads one of these keys (tiles beyond the
   // window are fully masked and store zeros)
-  const int q_reach = a.ds_t ? ((kv0 + 126 + W) / 128) * 128 + 127 : kv0 + 127 + W - 1;
+  const int q_reach = a.ds ? ((kv0 + 126 + W) / 128) * 128 + 127 : kv0 + 127 + W - 1;
   const int q_last = min(T - 1, q_reach) / 64;
   const int n_qt = q_last - q_first + 1;  // query tiles per query head
   const int n_q = n_qt * a.group;         // iterations: query head hk·group + i / n_qt, tile i % n_qt
@@ -1246,10 +981,14 @@ __global__ void __launch_bounds__(576, 1)
             dk[j / 2] = pack_bf2(s0, s1);
           }
         }
-        if (a.ds_t != nullptr && key < T) {
-          uint4* dst = reinterpret_cast<uint4*>(a.ds_t + ((size_t)bh * T + key) * a.Tpad + qc);
-          dst[0] = make_uint4(dk[0], dk[1], dk[2], dk[3]);
-          dst[1] = make_uint4(dk[4], dk[5], dk[6], dk[7]);
+        if (a.ds != nullptr && key < T) {
+          // dS[q][key]: lanes hold consecutive keys, so each store covers 64 contiguous bytes
+          uint16_t* dst = a.ds + ((size_t)bh * T + qc) * a.Tpad + key;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (qc + 2 * e < T) dst[(size_t)(2 * e) * a.Tpad] = (uint16_t)(dk[e] & 0xFFFFu);
+            if (qc + 2 * e + 1 < T) dst[(size_t)(2 * e + 1) * a.Tpad] = (uint16_t)(dk[e] >> 16);
+          }
         }
         // packed: chunk c of half h fills columns 32h + 8c .. +7, inside what this warp has read
         tmem_st8(tmem + lane_off + S::TM_S + grp * 64 + 32 * half + 8 * c, pk);
@@ -1519,18 +1258,19 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 // ================================================================================================
-// backward (3'): dQ from the dSᵀ tiles the dK/dV kernel stored — one CTA per 128-query tile, loop
-// over its 64-key tiles: dQ += dS·Kⱼ with A = dS read MN-major from the [64 keys][128 queries] dSᵀ
-// tile and B = Kⱼ (MN-major).  No scores are recomputed; the epilogue is the dQ kernel's.
+// backward (3'): dQ from the dS tiles the dK/dV kernel stored — one CTA per 128-query tile, loop
+// over its 64-key tiles: dQ += dS·Kⱼ with A = dS read K-major from the [128 queries][64 keys] dS
+// tile (one TMA box) and B = Kⱼ (MN-major).  No scores are recomputed; the epilogue is the dQ
+// kernel's.
 // ================================================================================================
 // Two CTAs share an SM (two stages each, ≈97 KB of shared memory and DH tensor-memory columns per
-// CTA), so that one CTA's prologue (Q tile, first dSᵀ tiles) and epilogue (QK-norm + RoPE backward)
-// overlap the other's stream of dSᵀ tiles: the kernel is bound by reading dSᵀ from HBM.
+// CTA), so that one CTA's prologue (Q tile, first dS tiles) and epilogue (QK-norm + RoPE backward)
+// overlap the other's stream of dS tiles: the kernel is bound by reading dS from HBM.
 template <int DH>
 struct DqDsShape {
   static constexpr int STAGES = 2;
   static constexpr int Q_TILE = 128 * DH * 2;   // q̃ tile (the QK-norm + RoPE backward reads it)
-  static constexpr int DS_TILE = 64 * 128 * 2;  // [2 query chunks][64 keys][64 queries]
+  static constexpr int DS_TILE = 128 * 64 * 2;  // [128 queries][64 keys]
   static constexpr int K_TILE = 64 * DH * 2;
   static constexpr int STAGE_BYTES = DS_TILE + K_TILE;
   static constexpr int OFF_Q = 0;
@@ -1599,16 +1339,15 @@ __global__ void __launch_bounds__(192, 2)
         mbar_arrive_expect_tx(&full[st], S::STAGE_BYTES);
         uint8_t* dst = smem + S::OFF_STAGE + st * S::STAGE_BYTES;
         const int k0 = (kv_first + j) * 64;
-        tma_load_3d(dst, &mds, &full[st], q0, k0, bh);                  // queries q0 .. q0+63
-        tma_load_3d(dst + S::DS_TILE / 2, &mds, &full[st], q0 + 64, k0, bh);  // q0+64 .. q0+127
+        tma_load_3d(dst, &mds, &full[st], k0, q0, bh);  // dS rows q0 .. q0+127, keys k0 .. k0+63
         load_tile<DH, 64>(dst + S::DS_TILE, &mk, &full[st], k0, h / a.group, b);
       }
     }
   } else if (warp == 5) {
     // ---------------- MMA issuer: the warp runs the loop, one elected lane issues ----------------
-    constexpr uint32_t id_acc = idesc_bf16(128, DH, true, true);
+    constexpr uint32_t id_acc = idesc_bf16(128, DH, false, true);
     const uint32_t stage0 = smem_u32(smem + S::OFF_STAGE);
-    const uint64_t ds_d = sdesc_sw128(stage0, S::DS_TILE / 2, 1024);       // dS, MN-major (queries)
+    const uint64_t ds_d = sdesc_sw128(stage0, 16, 1024);                   // dS, K-major (keys)
     const uint64_t k_d = sdesc_sw128(stage0 + S::DS_TILE, 64 * 128, 1024);  // K, MN-major (Dh)
     bool ok = true;
     for (int j = 0; j < n_kv && ok; ++j) {
@@ -1620,7 +1359,7 @@ __global__ void __launch_bounds__(192, 2)
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ss(tmem, sdesc_add(a_st, kk * 2048), sdesc_add(b_st, kk * 2048), id_acc,
+          mma_bf16_ss(tmem, sdesc_add(a_st, kk * 32), sdesc_add(b_st, kk * 2048), id_acc,
                       (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&empty[st]);
       }
@@ -1707,13 +1446,12 @@ __global__ void attn_kmax_kernel(const uint16_t* __restrict__ k, float* __restri
 }
 
 // ================================================================================================
-// backward (1): delta = rowsum(dO ∘ O), LSE·log2 e and the extension rows, Dh/8 lanes per row
+// backward (1): delta = rowsum(dO ∘ O) and LSE·log2 e, Dh/8 lanes per row
 // ================================================================================================
 
 __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
-                                  const float* __restrict__ lse, float* __restrict__ pad,
-                                  uint16_t* __restrict__ ext, float ext_scale, int B, int H, int T,
-                                  int Tpad, int Dh, long long sb, long long sh, long long st,
+                                  const float* __restrict__ lse, float* __restrict__ pad, int B, int H,
+                                  int T, int Tpad, int Dh, long long sb, long long sh, long long st,
                                   long long sbd, long long shd, long long std_) {
   pdl_wait();
   pdl_trigger();
@@ -1742,13 +1480,6 @@ __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t
     const float l = (t < T) ? lse[bh * T + t] : 0.f;
     pad[r] = l * LOG2E;
     pad[rows + r] = acc;
-    if (ext != nullptr) {
-      // (Sᵀ + ext)·scale·log2 e = s·scale·log2 e − LSE·log2 e  and  dPᵀ + ext = dP − delta
-      const uint2 el = (t < T) ? split3_bf16(-l * ext_scale) : make_uint2(0, 0);
-      const uint2 ed = split3_bf16(-acc);
-      *reinterpret_cast<uint4*>(ext + r * 8) = make_uint4(el.x, el.y, 0, 0);
-      *reinterpret_cast<uint4*>(ext + (rows + r) * 8) = make_uint4(ed.x, ed.y, 0, 0);
-    }
   }
 }
 
@@ -2125,42 +1856,24 @@ gpt_status launch_bwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, c
   return launch_kernel(attn_bwd_dq_kernel<DH>, grid, dim3(128), smem, stream, mq, mk, mv, mdo, a);
 }
 
-// dK/dV kernel choice: two softmax groups with −LSE / −delta in the softmax arithmetic (default) or
-// one group with the extension products (GPTSTEP_ATTN_BWD=1).
-static bool bwd_two_groups() {
-  static const bool two = [] {
-    const char* v = std::getenv("GPTSTEP_ATTN_BWD");
-    return !(v && v[0] == '1');
-  }();
-  return two;
-}
-
-// tcgen05 backward: maps with 128-row boxes (outer tiles) and 64-row boxes (inner tiles), and the
-// [2·B·H·Tpad][8] bf16 extension rows in 64-row boxes.
+// tcgen05 backward: maps with 128-row boxes (outer tiles) and 64-row boxes (inner tiles).
 template <int DH>
 gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[4],
-                         const CUtensorMap& mext, const CUtensorMap* mds, AttnArgs a, void* dq,
-                         cudaStream_t stream) {
+                         const CUtensorMap* mds, AttnArgs a, void* dq, cudaStream_t stream) {
   using S = TcBwdShape<DH>;
-  using S2 = TcBwd2Shape<DH>;
+  using SK = TcDkdvShape<DH>;
   using SD = DqDsShape<DH>;
+  GPT_TRY(ensure_smem(attn_bwd_dkdv_tc_kernel<DH>, SK::SMEM));
   GPT_TRY(ensure_smem(attn_bwd_dq_tc_kernel<DH>, S::SMEM));
   GPT_TRY(ensure_smem(attn_bwd_dq_ds_kernel<DH>, SD::SMEM));
   // dK/dV: outer 128-key tiles (K, V with 128-row boxes), inner 64-query tiles (Q, dO 64-row boxes)
   dim3 g1((a.T + 127) / 128, a.Hkv, a.B);  // one CTA per key tile of each key/value head
-  if (bwd_two_groups()) {
-    GPT_TRY(ensure_smem(attn_bwd_dkdv2_kernel<DH>, S2::SMEM));
-    GPT_TRY(launch_kernel(attn_bwd_dkdv2_kernel<DH>, g1, dim3(S2::THREADS), S2::SMEM, stream, m64[0],
-                          m128[1], m128[2], m64[3], a));
-  } else {
-    GPT_TRY(ensure_smem(attn_bwd_dkdv_tc_kernel<DH>, S::SMEM));
-    GPT_TRY(launch_kernel(attn_bwd_dkdv_tc_kernel<DH>, g1, dim3(S::THREADS), S::SMEM, stream, m64[0],
-                          m128[1], m128[2], m64[3], mext, a));
-  }
+  GPT_TRY(launch_kernel(attn_bwd_dkdv_tc_kernel<DH>, g1, dim3(SK::THREADS), SK::SMEM, stream, m64[0],
+                        m128[1], m128[2], m64[3], a));
   a.o = reinterpret_cast<uint16_t*>(dq);
   dim3 g2((a.T + 127) / 128, a.H, a.B);
   if (mds != nullptr) {
-    // dQ = dS·K from the stored dSᵀ tiles: outer 128-query tiles, inner 64-key tiles
+    // dQ = dS·K from the stored dS tiles: outer 128-query tiles, inner 64-key tiles
     return launch_kernel(attn_bwd_dq_ds_kernel<DH>, g2, dim3(SD::THREADS), SD::SMEM, stream, m128[0],
                          m64[1], *mds, a);
   } else {
@@ -2223,12 +1936,12 @@ gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, f
   return launch_fwd_tc<64>(mq2, mk2, mv2, a, kmax_scratch, kconst, stream);
 }
 
-// Backward scratch per padded row (b, h, t < ⌈T/64⌉·64): LSE·log2 e and delta (fp32), and the two
-// 16-byte extension rows of the dK/dV kernel.
+// Backward scratch per padded row (b, h, t < ⌈T/64⌉·64): LSE·log2 e and delta (fp32); then, when
+// stored, dS [B·H][T][⌈T/64⌉·64] bf16.
 size_t attention_bwd_scratch_bytes(int B, int H, int T, bool store_ds) {
   if (B <= 0 || H <= 0 || T <= 0) return 0;
   const size_t rows = (size_t)B * H * ((T + 63) / 64 * 64);
-  return rows * (2 * sizeof(float) + 2 * 16) + (store_ds ? rows * (size_t)T * 2 : 0);
+  return rows * 2 * sizeof(float) + (store_ds ? rows * (size_t)T * 2 : 0);
 }
 
 // Layouts: lq for q, lkv for k and v (Hkv heads), ldq for dq, ldkv for dk and dv, lo for o, ldo for
@@ -2252,34 +1965,25 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   GPT_TRY(check_attn(dout, B, H, T, Dh, ldo.sb, ldo.sh, ldo.st));
   if (!lse || !delta) return GPT_ERR_INVALID_ARG;
   const int Tpad = (T + 63) / 64 * 64;
-  // scratch: [2][B·H][Tpad] fp32 (LSE·log2 e, delta), then the dK/dV kernel's extension rows
-  // [2][B·H][Tpad][8] bf16, fetched with TMA in 64-row boxes
+  // scratch: [2][B·H][Tpad] fp32 (LSE·log2 e, delta), then, when the scratch holds it, dS
+  // [B·H][T][Tpad] bf16 (query rows, key columns)
   const long long rows = (long long)B * H * Tpad;
-  uint16_t* ext = (Dh != 32) ? reinterpret_cast<uint16_t*>(delta + 2 * rows) : nullptr;
-  // dSᵀ [B·H][T][Tpad] bf16 after the extension rows, when the scratch holds it
-  uint16_t* ds_t = (Dh != 32 && store_ds) ? ext + 2 * rows * 8 : nullptr;
+  if ((reinterpret_cast<uintptr_t>(delta) & 15) != 0) return GPT_ERR_UNSUPPORTED_SHAPE;
+  uint16_t* ds = (Dh != 32 && store_ds) ? reinterpret_cast<uint16_t*>(delta + 2 * rows) : nullptr;
   CUtensorMap mds;
-  if (ds_t != nullptr) {
-    const uint64_t dims[3] = {(uint64_t)Tpad, (uint64_t)T, (uint64_t)B * H};
+  if (ds != nullptr) {
+    // keys ≥ T lie outside the map (read as zero), as do query rows ≥ T
+    const uint64_t dims[3] = {(uint64_t)T, (uint64_t)T, (uint64_t)B * H};
     const uint64_t strides[2] = {(uint64_t)Tpad * 2, (uint64_t)T * Tpad * 2};
-    const uint32_t box[3] = {64, 64, 1};
-    if (!encode_map_bf16(&mds, ds_t, 3, dims, strides, box, true)) return GPT_ERR_UNSUPPORTED_SHAPE;
-  }
-  CUtensorMap mext;
-  if (Dh != 32) {
-    const uint64_t dims[2] = {8, (uint64_t)(2 * rows)};
-    const uint64_t strides[1] = {16};
-    const uint32_t box[2] = {8, 64};
-    if ((reinterpret_cast<uintptr_t>(delta) & 15) != 0 || 2 * rows >= (1ll << 31) ||
-        !encode_map_bf16(&mext, ext, 2, dims, strides, box, false))
-      return GPT_ERR_UNSUPPORTED_SHAPE;
+    const uint32_t box[3] = {64, 128, 1};
+    if (!encode_map_bf16(&mds, ds, 3, dims, strides, box, false)) return GPT_ERR_UNSUPPORTED_SHAPE;
   }
   if (!delta_ready) {  // else the GEMM that produced dO has written these rows
     const int threads = 256;
     const long long blocks = (rows * (Dh / 8) + threads - 1) / threads;
     GPT_TRY(launch_kernel(attn_delta_kernel, dim3((unsigned)blocks), dim3(threads), 0, stream,
                           reinterpret_cast<const uint16_t*>(o), reinterpret_cast<const uint16_t*>(dout),
-                          lse, delta, ext, sqrtf((float)Dh), B, H, T, Tpad, Dh, lo.sb, lo.sh, lo.st,
+                          lse, delta, B, H, T, Tpad, Dh, lo.sb, lo.sh, lo.st,
                           ldo.sb, ldo.sh, ldo.st));
   }
   AttnArgs a{};
@@ -2292,8 +1996,7 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   a.lse = const_cast<float*>(lse);
   a.delta = delta;
   a.Tpad = Tpad;
-  a.ext = ext;
-  a.ds_t = ds_t;
+  a.ds = ds;
   a.status = status;
   a.sb_o = ldq.sb; a.sh_o = ldq.sh; a.st_o = ldq.st;     // dq
   a.sb_g = ldkv.sb; a.sh_g = ldkv.sh; a.st_g = ldkv.st;  // dk, dv
@@ -2322,16 +2025,15 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
         !make_head_map(&m64[i], src[i], B, heads[i], T, Dh, lay[i].sb, lay[i].sh, lay[i].st, 64))
       return GPT_ERR_UNSUPPORTED_SHAPE;
   }
-  if (Dh == 128) GPT_TRY(launch_bwd_tc<128>(m128, m64, mext, ds_t ? &mds : nullptr, a, dq, stream));
-  else GPT_TRY(launch_bwd_tc<64>(m128, m64, mext, ds_t ? &mds : nullptr, a, dq, stream));
+  if (Dh == 128) GPT_TRY(launch_bwd_tc<128>(m128, m64, ds ? &mds : nullptr, a, dq, stream));
+  else GPT_TRY(launch_bwd_tc<64>(m128, m64, ds ? &mds : nullptr, a, dq, stream));
   return GPT_OK;
 }
 
 // ------------------------------------------------------------------------------------------------
 // Allocation-free attention backward: the backward's per-row scratch (LSE·log2 e and
-// delta = rowsum(dO∘O) in fp32, then the two 16-byte bf16 extension rows: 40 bytes = 10 floats per
-// row of B·H·⌈T/64⌉·64) lives in this fixed array instead of a caller-supplied buffer.  Every GPU
-// that loads the library holds it until exit.
+// delta = rowsum(dO∘O) in fp32: 8 bytes = 2 floats per row of B·H·⌈T/64⌉·64) lives in this fixed
+// array instead of a caller-supplied buffer.  Every GPU that loads the library holds it until exit.
 // ------------------------------------------------------------------------------------------------
 constexpr long long NOALLOC_FLOATS = GPT_ATTN_BWD_NOALLOC_FLOATS;
 static __device__ __align__(256) float g_noalloc_delta[NOALLOC_FLOATS];
@@ -2361,7 +2063,7 @@ gpt_status attention_bwd_noalloc(const void* q, const void* k, const void* v, co
                                  long long sto, int* status, cudaStream_t stream) {
   if (B <= 0 || H <= 0 || T <= 0) return GPT_ERR_INVALID_ARG;
   // the fixed array holds the per-row scratch only: dQ recomputes the scores instead of reading
-  // a stored dSᵀ
+  // a stored dS
   if ((long long)attention_bwd_scratch_bytes(B, H, T, false) > NOALLOC_FLOATS * 4)
     return GPT_ERR_UNSUPPORTED_SHAPE;
   float* delta = nullptr;

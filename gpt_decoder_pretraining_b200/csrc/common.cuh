@@ -28,15 +28,6 @@ __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
 }
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-// v as hi + mid + lo in bf16 (each a round-to-nearest-even of the remainder): ~24 significant bits
-// (the attention backward adds such triples into fp32 accumulators with one K = 16 MMA).
-__device__ __forceinline__ uint2 split3_bf16(float v) {
-  const uint16_t hi = f2bf(v);
-  const float r1 = v - bf2f(hi);
-  const uint16_t mid = f2bf(r1);
-  const uint16_t lo = f2bf(r1 - bf2f(mid));
-  return make_uint2((uint32_t)hi | ((uint32_t)mid << 16), (uint32_t)lo);
-}
 
 // ------------------------------------------------------------------------------------------------
 // device status word: first nonzero code wins

@@ -138,16 +138,14 @@ struct GemmArgs {
   float* rho_q;           // [M, H]
   float* rho_k;
   // EPI_BF16_HEADS (optional, dl_pad != null): the attention backward's per-row scratch for the
-  // dO just stored — delta = rowsum(dO∘O) from the bf16-rounded dO, LSE·log2 e, and the two bf16
-  // extension rows — at row (b·H + h)·Tpad + t of [2][B·H·Tpad]
+  // dO just stored — delta = rowsum(dO∘O) from the bf16-rounded dO and LSE·log2 e — at row
+  // (b·H + h)·Tpad + t of [2][B·H·Tpad]
   const uint16_t* dl_o;   // o, token-major: (b, h, t, j) at b·dl_sb + h·Dh + t·dl_st + j
   long long dl_sb, dl_st;
   const float* dl_lse;    // [B, H, T]
   float* dl_pad;
-  uint16_t* dl_ext;       // may be null
   int dl_Tpad;
   long long dl_rows;      // B·H·Tpad
-  float dl_ext_scale;     // √Dh
 };
 
 struct GemmShape {
@@ -751,12 +749,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
               const float l = args.dl_lse[((long long)b * args.H + h) * args.T + t];
               args.dl_pad[r] = l * 1.4426950408889634f;
               args.dl_pad[args.dl_rows + r] = dl_dot;
-              if (args.dl_ext) {
-                const uint2 el = split3_bf16(-l * args.dl_ext_scale);
-                const uint2 ed = split3_bf16(-dl_dot);
-                *reinterpret_cast<uint4*>(args.dl_ext + r * 8) = make_uint4(el.x, el.y, 0, 0);
-                *reinterpret_cast<uint4*>(args.dl_ext + (args.dl_rows + r) * 8) = make_uint4(ed.x, ed.y, 0, 0);
-              }
             }
           }
           if (j0_end_of_head(n0, args.Dh)) dl_dot = 0.f;
@@ -1029,9 +1021,7 @@ gpt_status gemm_heads_launch(int op, int M, int N, int K, const void* A, int lda
     a.dl_o = reinterpret_cast<const uint16_t*>(fuse->o);
     a.dl_sb = fuse->sb_o; a.dl_st = fuse->st_o;
     a.dl_lse = fuse->lse; a.dl_pad = fuse->pad;
-    a.dl_ext = reinterpret_cast<uint16_t*>(fuse->ext);
     a.dl_Tpad = fuse->Tpad; a.dl_rows = (long long)(M / T) * H * fuse->Tpad;
-    a.dl_ext_scale = sqrtf((float)Dh);
   }
   if (op == GPT_GEMM_NT) return launch_inst<false, false, EPI_BF16_HEADS>(ma, mb, a, stream);
   if (op == GPT_GEMM_NN) return launch_inst<false, true, EPI_BF16_HEADS>(ma, mb, a, stream);

@@ -128,14 +128,13 @@ int gemm_ce_tile_n();  // vocabulary columns per CE statistics tile
 
 // The attention backward's per-row scratch, computed in the epilogue of the GEMM that produces dO
 // (so that the backward skips its own pass over O and dO): o token-major (b, h, t, j) at
-// b·sb_o + h·Dh + t·st_o + j; lse [B, H, T]; pad = the scratch (fp32 [2][B·H·Tpad]); ext its bf16
-// extension rows (or null).  Only for T a multiple of 64 (no zero-padded rows to fill).
+// b·sb_o + h·Dh + t·st_o + j; lse [B, H, T]; pad = the scratch (fp32 [2][B·H·Tpad]).  Only for T a
+// multiple of 64 (no zero-padded rows to fill).
 struct AttnDeltaFusion {
   const void* o;
   long long sb_o, st_o;
   const float* lse;
   float* pad;
-  void* ext;
   int Tpad;
 };
 // C (row m = b·T + t, column n = h·Dh + j) stored bf16 head-major at heads[((b·H + h)·T + t)·Dh + j].

@@ -370,7 +370,6 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
   float* delta = reinterpret_cast<float*>(ws + p.delta);
   // the delta rows come from the dO GEMM's epilogue when no row of the scratch is padding
   const bool fuse_delta = (T % 64) == 0;
-  void* delta_ext = (Dh != 32) ? (void*)(delta + 2 * (size_t)B * H * T) : nullptr;
   for (int l = c.depth - 1; l >= 0; --l) {
     const int wq = 1 + 4 * l;
     uint16_t* r1 = reinterpret_cast<uint16_t*>(at(p.r1, l));
@@ -395,7 +394,7 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
     PROF(PROF_NORM, 0, 14.0 * (double)M * d, rmsnorm_bwd(dr, 0, r2, rho2, gx, gxb, 1, M, d, s));
     // attention
     // dO head-major; its epilogue also forms the attention backward's delta rows (T % 64 == 0)
-    AttnDeltaFusion fuse{o, os_b, os_t, lse, delta, delta_ext, T, };
+    AttnDeltaFusion fuse{o, os_b, os_t, lse, delta, T};
     PROF(PROF_GEMM, gemm_flops(M, d, d), 0,
          gemm_heads_launch(GPT_GEMM_NN, M, d, d, gxb, d, W(wq + 1), d, dO, T, H, Dh, status, s,
                            fuse_delta ? &fuse : nullptr));

@@ -255,11 +255,9 @@ gpt_status gpt_rope_table(float* cos_sin, int T, int Dh, void* stream);
  * the natural-log logsumexp of the scaled scores.  Dh ∈ {32, 64, 128} (32: H_kv = H only).
  * window ≤ 0 or ≥ T = full causal.  delta: backward scratch of at least
  * gpt_attention_bwd_scratch_bytes(B, H, T) bytes, 16-byte aligned; per row (zero-padded to a
- * multiple of 64 rows per (b, h)) the backward stores LSE·log2(e) and rowsum(dO∘O) in fp32 and,
- * for Dh ≥ 64, both again as bf16 hi/mid/lo triples that its dK/dV kernel adds into the score
- * accumulators with one extra K = 16 tensor-core step; after these rows, for Dh ≥ 64, the dK/dV
- * kernel stores dSᵀ (bf16 [B·H][T][⌈T/64⌉·64], causal band / window only) and the dQ kernel
- * contracts it with K.
+ * multiple of 64 rows per (b, h)) the backward stores LSE·log2(e) and rowsum(dO∘O) in fp32; after
+ * these rows, for Dh ≥ 64, the dK/dV kernel stores dS (bf16 [B·H][T][⌈T/64⌉·64], query rows and
+ * key columns, causal band / window only) and the dQ kernel contracts it with K.
  * The forward shifts each row's exponentials by the Cauchy–Schwarz bound c_t = ‖q_t‖·max_j‖k_j‖/√Dh
  * instead of a running maximum (softmax is invariant to the shift, so the result is exact); this
  * needs c_t ≤ 40 so that no row underflows, which always holds after QK-norm (c_t ≈ √Dh) — rows
@@ -272,8 +270,8 @@ gpt_status gpt_attention_fwd(const void* q, const void* k, const void* v, void* 
                              long long sb_q, long long sh_q, long long st_q, long long sb_kv,
                              long long sh_kv, long long st_kv, long long sb_o, long long sh_o,
                              long long st_o, int* status, void* stream);
-/* Bytes of the `delta` scratch that gpt_attention_bwd needs for (B, H, T): 40 bytes per row of
- * R = B·H·⌈T/64⌉·64, plus 2·T·R bytes of dSᵀ — quadratic in T (1.6 GB for B·H = 192 at T = 2048,
+/* Bytes of the `delta` scratch that gpt_attention_bwd needs for (B, H, T): 8 bytes per row of
+ * R = B·H·⌈T/64⌉·64, plus 2·T·R bytes of dS — quadratic in T (1.6 GB for B·H = 192 at T = 2048,
  * 34 GB for B·H·T = 2^21 at T = 8192).  Callers short of memory can use, within its row limit,
  * gpt_attention_bwd_noalloc, which recomputes the scores instead.  Returns 0 for a non-positive
  * size. */
@@ -288,25 +286,25 @@ gpt_status gpt_attention_bwd(const void* q, const void* k, const void* v, const 
 /* Attention backward that allocates nothing.  The pages have no counterpart: this is a calling
  * convenience, not part of the method.  Arguments and results are those of gpt_attention_bwd
  * without `delta`, for multi-head attention (H_kv = H, one stride set (sb_qkv, sh_qkv, st_qkv) for
- * q/k/v/dq/dk/dv); the per-row scratch that the backward needs (40 bytes per row of
+ * q/k/v/dq/dk/dv); the per-row scratch that the backward needs (8 bytes per row of
  * B·H·⌈T/64⌉·64) is kept in a static device array inside this library
  * (GPT_ATTN_BWD_NOALLOC_FLOATS fp32 values = 8 MiB), which every GPU that loads the library holds
- * until the process exits.  dSᵀ is not stored: the dQ kernel recomputes the scores instead.
+ * until the process exits.  dS is not stored: the dQ kernel recomputes the scores instead.
  * It serves callers that cannot obtain device memory where they call the backward — for example
  * code running under a device-memory budget fixed at start-up, or inside a host framework whose own
  * allocator owns all device memory and allows no side allocations — and therefore cannot hand
  * gpt_attention_bwd its scratch buffer.  It calls no cudaMalloc, cudaFree or allocating routine.
- *   - The array holds GPT_ATTN_BWD_NOALLOC_FLOATS fp32 values; at 40 bytes (10 floats) per padded
- *     row it serves B·H·⌈T/64⌉·64 ≤ GPT_ATTN_BWD_NOALLOC_MAX_ROWS rows (209,715; the largest
- *     multiple of 64 below it, 209,664, is the largest accepted).  Larger shapes return
- *     GPT_ERR_UNSUPPORTED_SHAPE before anything is enqueued or any CUDA call is made.
+ *   - The array holds GPT_ATTN_BWD_NOALLOC_FLOATS fp32 values; at 8 bytes (2 floats) per padded
+ *     row it serves B·H·⌈T/64⌉·64 ≤ GPT_ATTN_BWD_NOALLOC_MAX_ROWS rows (1,048,576, itself a
+ *     multiple of 64).  Larger shapes return GPT_ERR_UNSUPPORTED_SHAPE before anything is enqueued
+ *     or any CUDA call is made.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
  *     that device current); make that first call before any stream capture.
  *   - All calls share the one array.  Each call writes the rows it uses before reading them, so
  *     nothing needs clearing, but calls that overlap on the GPU (unordered streams, several host
  *     threads) race on it and give wrong results: order them on one stream. */
 #define GPT_ATTN_BWD_NOALLOC_FLOATS (1ll << 21)
-#define GPT_ATTN_BWD_NOALLOC_MAX_ROWS (GPT_ATTN_BWD_NOALLOC_FLOATS / 10)
+#define GPT_ATTN_BWD_NOALLOC_MAX_ROWS (GPT_ATTN_BWD_NOALLOC_FLOATS / 2)
 gpt_status gpt_attention_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                                      const void* dout, const float* lse, void* dq, void* dk,
                                      void* dv, int B, int H, int T, int Dh, int window,

@@ -253,29 +253,29 @@ def test_bucketed_data_parallel_average_equals_the_full_batch_step():
 
 
 def test_attention_backward_scratch_size(lib):
-    """Per padded row 40 bytes (LSE·log2 e and delta in fp32, two 16-byte extension rows), then
-    dSᵀ: 2·T bytes per padded row."""
+    """Per padded row 8 bytes (LSE·log2 e and delta in fp32), then dS: 2·T bytes per padded row."""
     f = lib.gpt_attention_bwd_scratch_bytes
     f.restype = ctypes.c_size_t
     for B, H, T in [(1, 1, 1), (2, 3, 200), (16, 12, 2048), (4, 8, 130)]:
         rows = B * H * ((T + 63) // 64 * 64)
-        assert f(B, H, T) == rows * 40 + rows * T * 2
+        assert f(B, H, T) == rows * 8 + rows * T * 2
     assert f(0, 1, 1) == 0 and f(1, 1, 0) == 0
 
 
 def test_noalloc_attention_backward_row_limit_needs_no_device(lib):
-    """The allocation-free backward keeps 40 bytes per padded row in a static array of 2^21 floats
-    (209,715 rows).  One 64-row pad beyond the largest accepted shape (B·H·⌈T/64⌉·64 = 209,664)
-    is refused with GPT_ERR_UNSUPPORTED_SHAPE before any CUDA call, so no device is needed here
-    (the pointers are never dereferenced).  The accepted side runs in tests/test_zz_no_alloc.py."""
+    """The allocation-free backward keeps 8 bytes per padded row in a static array of 2^21 floats
+    (1,048,576 rows).  One 64-row pad beyond the largest accepted shape (B·H·⌈T/64⌉·64 =
+    1,048,576) is refused with GPT_ERR_UNSUPPORTED_SHAPE before any CUDA call, so no device is
+    needed here (the pointers are never dereferenced).  The accepted side runs in
+    tests/test_zz_no_alloc.py."""
     f = 1 << 20
     call = lib.gpt_attention_bwd_noalloc
-    assert (1 << 21) * 4 // 40 == 209715 and 3276 * 64 == 209664
+    assert (1 << 21) * 4 // 8 == 1048576 and 16384 * 64 == 1048576
     args = lambda B, H, T, Dh: (f, f, f, f, f, f, f, f, f, B, H, T, Dh, 0,  # noqa: E731
                                 H * T * Dh, T * Dh, Dh, H * T * Dh, T * Dh, Dh, None, None)
-    assert call(*args(3277, 1, 64, 64)) == -2           # 209,728 padded rows
-    assert call(*args(1, 3277, 33, 128)) == -2          # T = 33 pads to 64 rows per (b, h)
-    assert call(*args(1, 16, 65537, 64)) == -2
+    assert call(*args(16385, 1, 64, 64)) == -2          # 1,048,640 padded rows
+    assert call(*args(1, 16385, 33, 128)) == -2         # T = 33 pads to 64 rows per (b, h)
+    assert call(*args(1, 16, 65537 * 2, 64)) == -2
     assert call(*args(0, 1, 64, 64)) == -1
 
 

@@ -21,8 +21,8 @@ pytestmark = pytest.mark.gpu
 
 # (B, H, T, Dh, window): each call has fewer rows than the one before it
 CALLS = [(2, 3, 200, 128, 0), (1, 2, 97, 64, 33), (1, 2, 77, 32, 9)]
-# the largest shape the static array serves: B·H·⌈T/64⌉·64 = 209,664 rows of 40 bytes
-LIMIT_CASE = (3276, 1, 64, 64, 0)
+# the largest shape the static array serves: B·H·⌈T/64⌉·64 = 1,048,576 rows of 8 bytes
+LIMIT_CASE = (16384, 1, 64, 64, 0)
 
 
 def _inputs(B, H, T, Dh, seed):
@@ -73,7 +73,7 @@ def test_noalloc_attention_bwd_serves_its_largest_shape():
         pytest.skip("no CUDA device")
     from gpt_decoder_pretraining_b200 import step as S
     B, H, T, Dh, window = LIMIT_CASE
-    assert B * H * ((T + 63) // 64 * 64) * 40 <= 4 * (1 << 21)
+    assert B * H * ((T + 63) // 64 * 64) * 8 <= 4 * (1 << 21)
     arrays = _inputs(B, H, T, Dh, seed=77)
     ref = _run(S, B, H, T, Dh, window, arrays, noalloc=False)
     got = _run(S, B, H, T, Dh, window, arrays, noalloc=True)
