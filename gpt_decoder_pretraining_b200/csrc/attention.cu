@@ -730,14 +730,17 @@ template <int DH>
 struct TcDkdvShape {
   static constexpr int BIG_TILE = 128 * DH * 2;
   static constexpr int SMALL_TILE = 64 * DH * 2;
-  static constexpr int STAGES = 4;
+  static constexpr int STAGES = 3;
   static constexpr int OFF_A = 0;                  // K
   static constexpr int OFF_B = BIG_TILE;           // V
   static constexpr int OFF_STAGE = 2 * BIG_TILE;   // stages of (Q, dO)
   static constexpr int STAGE_BYTES = 2 * SMALL_TILE;
   static constexpr int OFF_LD = OFF_STAGE + STAGES * STAGE_BYTES;  // [stage][LSE·log2 e | delta][64] fp32
   static constexpr int LD_BYTES = 2 * 64 * 4;
-  static constexpr int OFF_BAR = OFF_LD + STAGES * LD_BYTES;
+  // per softmax warp, its [32 queries][32 keys] bf16 block of dS, written out by one TMA store
+  static constexpr int DS_WARP_BYTES = 32 * 32 * 2;
+  static constexpr int OFF_DS = (OFF_LD + STAGES * LD_BYTES + 1023) / 1024 * 1024;
+  static constexpr int OFF_BAR = OFF_DS + 16 * DS_WARP_BYTES;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr int THREADS = 576;  // 16 softmax warps (two groups of 8), TMA, MMA
   static constexpr int W_TMA = 16, W_MMA = 17;
@@ -755,14 +758,15 @@ __device__ __forceinline__ void qknorm_rope_bwd_tmem_part(uint32_t taddr, float 
   constexpr int HALF = DH / 2, QUART = DH / 4;
   float dot = 0.f;
 #pragma unroll 1
-  for (int c = 0; c < DH / 16; ++c) {
-    uint32_t v[16];
-    tmem_ld16(taddr + 16 * c, v);
+  for (int c = 0; c < DH / 32; ++c) {  // two 16-column loads per wait
+    uint32_t v[32];
+    tmem_ld16(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[16]>(v));
+    tmem_ld16(taddr + 32 * c + 16, *reinterpret_cast<uint32_t(*)[16]>(v + 16));
     tmem_ld_wait();
 #pragma unroll
-    for (int jj = 0; jj < 2; ++jj) {
+    for (int jj = 0; jj < 4; ++jj) {
       float y[8];
-      load_y8<ROWS>(tile, r, 16 * c + 8 * jj, y);
+      load_y8<ROWS>(tile, r, 32 * c + 8 * jj, y);
 #pragma unroll
       for (int e = 0; e < 8; ++e) dot += __uint_as_float(v[8 * jj + e]) * y[e];
     }
@@ -811,7 +815,7 @@ template <int DH>
 __global__ void __launch_bounds__(576, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                           const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
-                          const AttnArgs a) {
+                          const __grid_constant__ CUtensorMap mds_st, const AttnArgs a) {
   using S = TcDkdvShape<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -941,10 +945,15 @@ __global__ void __launch_bounds__(576, 1)
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const int kmin = kv0 + 32 * quarter, kmax_ = kmin + 31;  // this warp's keys
     bool ok = true;
+    uint8_t* ds_stage = smem + S::OFF_DS + warp * S::DS_WARP_BYTES;  // [32 queries][32 keys]
     for (int i = grp; i < n_q && ok; i += 2) {
       const int st = i % S::STAGES;
       if (!mbar_wait_warp(&s_full[grp], (i >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
       tc_fence_after();
+      if (a.ds != nullptr) {  // the previous tile's dS block has been read out of the staging area
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+      }
       const long long bh = (long long)b * a.H + hk * a.group + i / n_qt;  // the query head
       const int qh = (q_first + i % n_qt) * 64 + 32 * half;  // first query of this warp's 32 columns
       const float* ldl = reinterpret_cast<const float*>(smem + S::OFF_LD + st * S::LD_BYTES) + 32 * half;
@@ -981,13 +990,13 @@ __global__ void __launch_bounds__(576, 1)
             dk[j / 2] = pack_bf2(s0, s1);
           }
         }
-        if (a.ds != nullptr && key < T) {
-          // dS[q][key]: lanes hold consecutive keys, so each store covers 64 contiguous bytes
-          uint16_t* dst = a.ds + ((size_t)bh * T + qc) * a.Tpad + key;
+        if (a.ds != nullptr) {
+          // staging row = query, column = key (this lane): every row write is 64 contiguous bytes
+          uint16_t* row0 = reinterpret_cast<uint16_t*>(ds_stage) + (16 * c) * 32 + lane;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            if (qc + 2 * e < T) dst[(size_t)(2 * e) * a.Tpad] = (uint16_t)(dk[e] & 0xFFFFu);
-            if (qc + 2 * e + 1 < T) dst[(size_t)(2 * e + 1) * a.Tpad] = (uint16_t)(dk[e] >> 16);
+            row0[(2 * e) * 32] = (uint16_t)(dk[e] & 0xFFFFu);
+            row0[(2 * e + 1) * 32] = (uint16_t)(dk[e] >> 16);
           }
         }
         // packed: chunk c of half h fills columns 32h + 8c .. +7, inside what this warp has read
@@ -997,7 +1006,17 @@ __global__ void __launch_bounds__(576, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[grp]);
+      if (a.ds != nullptr) {
+        // dS[q][key] block of 32 queries × 32 keys; rows ≥ T and keys ≥ T fall outside the map
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&mds_st, ds_stage, kmin, qh, (int)bh);
+          bulk_commit();
+        }
+      }
     }
+    if (a.ds != nullptr && lane == 0) bulk_wait_all();
     // epilogue: group 0 writes dV, group 1 dK, each warp half one part of the row
     if (ok) ok = mbar_wait_warp(done, 0, abort_flag, a.status);
     if (ok) {
@@ -1013,14 +1032,15 @@ __global__ void __launch_bounds__(576, 1)
         uint16_t* dst = (grp == 0 ? a.dv : a.dk) + off;
         const float sc = (grp == 0) ? 1.f : a.scale;
 #pragma unroll 1
-        for (int c = 0; c < DH / 32; ++c) {
-          const int col = half * (DH / 2) + 16 * c;
-          uint32_t r[16];
-          tmem_ld16(tmem + lane_off + S::TM_ACC + grp * DH + col, r);
+        for (int c = 0; c < DH / 64; ++c) {  // two 16-column loads per wait
+          const int col = half * (DH / 2) + 32 * c;
+          uint32_t r[32];
+          tmem_ld16(tmem + lane_off + S::TM_ACC + grp * DH + col, *reinterpret_cast<uint32_t(*)[16]>(r));
+          tmem_ld16(tmem + lane_off + S::TM_ACC + grp * DH + col + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
           tmem_ld_wait();
           if (key < T) {
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
+            for (int u = 0; u < 4; ++u) {
               uint4 w;
               w.x = pack_bf2(__uint_as_float(r[8 * u + 0]) * sc, __uint_as_float(r[8 * u + 1]) * sc);
               w.y = pack_bf2(__uint_as_float(r[8 * u + 2]) * sc, __uint_as_float(r[8 * u + 3]) * sc);
@@ -1860,6 +1880,8 @@ gpt_status launch_bwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, c
 template <int DH>
 gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[4],
                          const CUtensorMap* mds, AttnArgs a, void* dq, cudaStream_t stream) {
+  // mds: null, or the stored dS's maps — [0] 128-query × 64-key boxes (128-byte swizzle) for the dQ
+  // kernel's loads, [1] 32 × 32 boxes (no swizzle) for the dK/dV kernel's per-warp stores
   using S = TcBwdShape<DH>;
   using SK = TcDkdvShape<DH>;
   using SD = DqDsShape<DH>;
@@ -1869,13 +1891,13 @@ gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[
   // dK/dV: outer 128-key tiles (K, V with 128-row boxes), inner 64-query tiles (Q, dO 64-row boxes)
   dim3 g1((a.T + 127) / 128, a.Hkv, a.B);  // one CTA per key tile of each key/value head
   GPT_TRY(launch_kernel(attn_bwd_dkdv_tc_kernel<DH>, g1, dim3(SK::THREADS), SK::SMEM, stream, m64[0],
-                        m128[1], m128[2], m64[3], a));
+                        m128[1], m128[2], m64[3], mds ? mds[1] : m64[0], a));
   a.o = reinterpret_cast<uint16_t*>(dq);
   dim3 g2((a.T + 127) / 128, a.H, a.B);
   if (mds != nullptr) {
     // dQ = dS·K from the stored dS tiles: outer 128-query tiles, inner 64-key tiles
     return launch_kernel(attn_bwd_dq_ds_kernel<DH>, g2, dim3(SD::THREADS), SD::SMEM, stream, m128[0],
-                         m64[1], *mds, a);
+                         m64[1], mds[0], a);
   } else {
     // dQ with S and dP recomputed: outer 128-query tiles (Q, dO 128-row boxes), inner 64-key tiles
     return launch_kernel(attn_bwd_dq_tc_kernel<DH>, g2, dim3(S::THREADS), S::SMEM, stream, m128[0],
@@ -1970,13 +1992,15 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   const long long rows = (long long)B * H * Tpad;
   if ((reinterpret_cast<uintptr_t>(delta) & 15) != 0) return GPT_ERR_UNSUPPORTED_SHAPE;
   uint16_t* ds = (Dh != 32 && store_ds) ? reinterpret_cast<uint16_t*>(delta + 2 * rows) : nullptr;
-  CUtensorMap mds;
+  CUtensorMap mds[2];
   if (ds != nullptr) {
-    // keys ≥ T lie outside the map (read as zero), as do query rows ≥ T
+    // keys ≥ T lie outside the maps (read as zero, never written), as do query rows ≥ T
     const uint64_t dims[3] = {(uint64_t)T, (uint64_t)T, (uint64_t)B * H};
     const uint64_t strides[2] = {(uint64_t)Tpad * 2, (uint64_t)T * Tpad * 2};
-    const uint32_t box[3] = {64, 128, 1};
-    if (!encode_map_bf16(&mds, ds, 3, dims, strides, box, false)) return GPT_ERR_UNSUPPORTED_SHAPE;
+    const uint32_t box_ld[3] = {64, 128, 1}, box_st[3] = {32, 32, 1};
+    if (!encode_map_bf16(&mds[0], ds, 3, dims, strides, box_ld, true) ||
+        !encode_map_bf16(&mds[1], ds, 3, dims, strides, box_st, false))
+      return GPT_ERR_UNSUPPORTED_SHAPE;
   }
   if (!delta_ready) {  // else the GEMM that produced dO has written these rows
     const int threads = 256;
@@ -2025,8 +2049,8 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
         !make_head_map(&m64[i], src[i], B, heads[i], T, Dh, lay[i].sb, lay[i].sh, lay[i].st, 64))
       return GPT_ERR_UNSUPPORTED_SHAPE;
   }
-  if (Dh == 128) GPT_TRY(launch_bwd_tc<128>(m128, m64, ds ? &mds : nullptr, a, dq, stream));
-  else GPT_TRY(launch_bwd_tc<64>(m128, m64, ds ? &mds : nullptr, a, dq, stream));
+  if (Dh == 128) GPT_TRY(launch_bwd_tc<128>(m128, m64, ds ? mds : nullptr, a, dq, stream));
+  else GPT_TRY(launch_bwd_tc<64>(m128, m64, ds ? mds : nullptr, a, dq, stream));
   return GPT_OK;
 }
 
