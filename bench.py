@@ -70,6 +70,16 @@ def load_traffic(workload: str):
         return None
 
 
+def traffic_fields(workload: str):
+    """roofline.traffic: DRAM bytes (read + write) per step of the GEMM family from the committed ncu
+    launch list of this workload (null when there is none), with the algorithmic bytes beside it."""
+    t = load_traffic(workload)
+    if not t:
+        return {"traffic": None}
+    return {"traffic": t.get("dram_bytes_per_step"), "traffic_unit": "bytes per step",
+            "traffic_algorithmic": t.get("algorithmic_bytes_per_step"), "traffic_source": t.get("source")}
+
+
 # ------------------------------------------------------------------------------------------------
 # clocks sampled during the timed region
 # ------------------------------------------------------------------------------------------------
@@ -454,7 +464,7 @@ def run_ours(args, cfg):
                      "executed_tflops": executed,
                      "executed_basis": "all launched GEMM FLOPs, including the lm-head logit recompute "
                                        "of the backward pass (2·B·T·d·V per step)",
-                     "traffic": load_traffic(workload)},
+                     **traffic_fields(workload)},
         "kernels": r["kernels"],
         "clocks": r["clocks"],
     }

@@ -1435,33 +1435,43 @@ __global__ void __launch_bounds__(192, 2)
 }
 
 // max_t ‖k_t‖ for each (batch, head): one CTA per (h, b).
-__global__ void attn_kmax_kernel(const uint16_t* __restrict__ k, float* __restrict__ kmax, int H,
-                                 int T, int Dh, long long sb, long long sh, long long st) {
+__global__ void __launch_bounds__(256) attn_kmax_kernel(const uint16_t* __restrict__ k, float* __restrict__ kmax,
+                                                        int H, int T, int Dh, long long sb, long long sh,
+                                                        long long st) {
   pdl_wait();
   pdl_trigger();
-  const int h = blockIdx.x, b = blockIdx.y;
+  // block (row chunk, h, b): Dh/8 lanes per row, one 16-byte load each; the block's largest ‖k_t‖
+  // goes to kmax[b][h] by an atomic maximum on the bit pattern (order-free for non-negative floats;
+  // kmax is zeroed before the launch)
+  const int G = Dh >> 3;  // lanes per row (4, 8 or 16; divides 32)
+  const int rows_per_pass = blockDim.x / G;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int t0 = blockIdx.x * 64;
   const uint16_t* base = k + b * sb + h * sh;
+  const int sub = threadIdx.x / G, part = threadIdx.x % G;
   float m = 0.f;
-  for (int t = threadIdx.x; t < T; t += blockDim.x) {
-    const uint4* row = reinterpret_cast<const uint4*>(base + (long long)t * st);
+  // the same trip count for every lane (the shuffles below involve the whole warp)
+  for (int it = 0; it < 64 / rows_per_pass; ++it) {
+    const int t = t0 + sub + it * rows_per_pass;
     float ss = 0.f;
-    for (int u = 0; u < Dh / 8; ++u) {
-      const uint4 v = row[u];
+    if (t < T) {
+      const uint4 v = *reinterpret_cast<const uint4*>(base + (long long)t * st + 8 * part);
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) ss += bf_lo(w[e]) * bf_lo(w[e]) + bf_hi(w[e]) * bf_hi(w[e]);
     }
+    for (int o = G >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     m = fmaxf(m, ss);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  __shared__ float red[32];
+  __shared__ float red[8];
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
   if (threadIdx.x == 0) {
     float r = 0.f;
     for (int i = 0; i < (int)(blockDim.x >> 5); ++i) r = fmaxf(r, red[i]);
-    kmax[(long long)b * H + h] = sqrtf(r);
+    atomicMax(reinterpret_cast<unsigned int*>(kmax) + (long long)b * H + h, __float_as_uint(sqrtf(r)));
   }
 }
 
@@ -1950,7 +1960,8 @@ gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, f
     return GPT_ERR_UNSUPPORTED_SHAPE;
   const float kconst = sqrtf((float)Dh) * 1.002f;
   if (kmax_scratch) {
-    GPT_TRY(launch_kernel(attn_kmax_kernel, dim3(Hkv, B), dim3(256), 0, stream,
+    GPT_CUDA_TRY(cudaMemsetAsync(kmax_scratch, 0, (size_t)B * Hkv * sizeof(float), stream));
+    GPT_TRY(launch_kernel(attn_kmax_kernel, dim3((Tk + 63) / 64, Hkv, B), dim3(256), 0, stream,
                           reinterpret_cast<const uint16_t*>(k), kmax_scratch, Hkv, Tk, Dh, lkv.sb,
                           lkv.sh, lkv.st));
   }

@@ -99,6 +99,25 @@ struct WorkIter {
   }
 };
 
+// Output tile order within one matrix: groups of `group` row tiles, column by column inside a
+// group (group 1: row by row).  With groups of 8 the tiles that run at the same time share a few row
+// blocks of A and the column blocks of B they read, so a B larger than L2 (the lm-head's vocabulary
+// matrix) is streamed once per group of row tiles instead of once per row tile.  Any order gives the
+// same results: every tile is computed whole (or by its own pieces) and written once.
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int group, int& tm, int& tn) {
+  const int per_group = group * tiles_n;
+  const int g = t / per_group, r = t - g * per_group;
+  const int rows = min(group, tiles_m - g * group);
+  tm = g * group + r % rows;
+  tn = r / rows;
+}
+// Row-by-row order everywhere except the lm-head's NT products against the vocabulary matrix (its
+// B, 100–168 MB, does not fit in L2); the projection weights (≤ 19 MB at d24) stay in L2 either way.
+constexpr long long RASTER_B_BYTES = 32ll << 20;
+inline int raster_for(int op, int N, int K) {
+  return (op == GPT_GEMM_NT && (long long)N * K * 2 > RASTER_B_BYTES) ? 8 : 1;
+}
+
 // Piece exchange of a split tail tile: each piece writes its fp32 partial tile to its own slot
 // (256 × 256 floats, slot = tail tile·sk_split + piece), then counts itself in one counter per
 // epilogue warp (32 rows × 128 columns: 16 per tile).
@@ -112,6 +131,7 @@ static_assert(GEMM_SK_COUNTER_BYTES == (size_t)SK_MAX_TILES * SK_WARPS_PER_TILE 
 struct GemmArgs {
   int M, N, K;
   int tiles_m, tiles_n, k_tiles;  // tiles_m counts 256-row pair tiles
+  int raster;                     // row tiles per group of the tile order (tile_coords)
   Sched sched;
   float* sk_part;                  // [sk_tiles·sk_split][256][256] partial tiles
   int* sk_cnt;                     // [sk_tiles·16] arrival counters, zero between launches
@@ -471,7 +491,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
       const int per_mat = args.tiles_m * args.tiles_n;
       while (it.next(sch, w)) {
         const int bb = w.tile / per_mat, tr = w.tile % per_mat;
-        const int tm = tr / args.tiles_n, tn = tr % args.tiles_n;
+        int tm, tn;
+        tile_coords(tr, args.tiles_m, args.tiles_n, args.raster, tm, tn);
         const int kt0 = w.k0, kt1 = w.k1;
         const int arow = tm * 2 * BM + rank * BM;        // this CTA's 128 rows of A
         const int brow = tn * BN + rank * (BN / 2);      // this CTA's 128 rows of B
@@ -564,7 +585,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
     const int per_mat = args.tiles_m * args.tiles_n;
     while (it.next(sch, w)) {
       const int bb = w.tile / per_mat, tr = w.tile % per_mat;
-      const int tm = tr / args.tiles_n, tn = tr % args.tiles_n;
+      int tm, tn;
+      tile_coords(tr, args.tiles_m, args.tiles_n, args.raster, tm, tn);
       const int m = tm * 2 * BM + rank * BM + row_in_tile;
       if constexpr (epi_plain<EPI>()) {
         if (!plain_epilogue<EPI>(args, w, bb, m, tn, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN,
@@ -855,6 +877,7 @@ static gpt_status fill_args(GemmArgs& a, int M, int N, int K, int batch = 1, int
   a.tiles_m = (M + 2 * BM - 1) / (2 * BM);
   a.tiles_n = (N + BN - 1) / BN;
   a.k_tiles = (K + k_per_tile - 1) / k_per_tile;
+  a.raster = 1;
   a.batch = batch;
   a.alpha = 1.f;
   a.beta = 0.f;
@@ -929,6 +952,7 @@ gpt_status gemm_launch_batched(const GemmBatch& g, cudaStream_t stream, void* sk
   if (!make_operand_map(&mb, g.B, b_mn, N, K, g.ldb, g.batch, g.b_bstride)) return GPT_ERR_UNSUPPORTED_SHAPE;
   GemmArgs a{};
   GPT_TRY(fill_args(a, M, N, K, g.batch));
+  a.raster = raster_for(op, N, K);
   a.C = g.C; a.ldc = g.ldc; a.C2 = nullptr;
   a.aux = reinterpret_cast<const uint16_t*>(g.aux); a.ldaux = g.ldaux;
   a.c_bstride = g.batch > 1 ? g.c_bstride : 0;
@@ -1080,6 +1104,7 @@ gpt_status gemm_ce_launch(bool grad, int M, int N, int K, const void* A, int lda
   if (!make_operand_map(&mb, B, false, N, K, ldb)) return GPT_ERR_UNSUPPORTED_SHAPE;
   GemmArgs a{};
   GPT_TRY(fill_args(a, M, N, K));
+  a.raster = raster_for(GPT_GEMM_NT, N, K);
   a.C = C; a.ldc = ldc;
   a.status = status;
   a.ce = ce;
