@@ -298,43 +298,95 @@ __global__ void embedding_fwd_kernel(const int32_t* __restrict__ tok, const uint
   for (int i = lane; i < (d >> 3); i += 32) dst[i] = src[i];
 }
 
-// Single-CTA bitonic sort of the keys (id << 16 | local index) of one segment of ≤ 32768 tokens,
-// then the run heads (first position of every distinct id) are compacted in ascending order.
+// Single-CTA stable sort of the keys (id << 16 | local index) of one segment of ≤ 32768 tokens by
+// id: a least-significant-digit radix sort over the 16 id bits in four 4-bit passes.  Thread t owns
+// the 32 keys at positions 32t .. 32t+31 of the current order; per pass it counts its digits, a
+// block-wide exclusive scan over (digit, thread) gives every thread its first slot per digit, and
+// the thread writes its keys there in order — so equal ids keep their position order (stable), and
+// since positions start in increasing order the keys end sorted by (id, position).  Then the run
+// heads (first position of every distinct id) are compacted in ascending order.
 // Outputs: sorted keys [n], run starts [nruns + 1] (last = n), *nruns.
 constexpr int EMB_SEG = 32768;
-__global__ void __launch_bounds__(1024) embedding_sort_kernel(const int32_t* __restrict__ tok, int n,
-                                                              int V, uint32_t* __restrict__ keys_out,
-                                                              int* __restrict__ run_start,
-                                                              int* __restrict__ nruns) {
+constexpr int EMB_SORT_THREADS = 1024;
+constexpr int EMB_SORT_PER_THREAD = EMB_SEG / EMB_SORT_THREADS;                     // 32
+constexpr int EMB_SORT_SMEM = EMB_SEG * 4 + 16 * EMB_SORT_THREADS * 4;                // keys + counts
+__global__ void __launch_bounds__(EMB_SORT_THREADS) embedding_sort_kernel(const int32_t* __restrict__ tok, int n,
+                                                                          int V, uint32_t* __restrict__ keys_out,
+                                                                          int* __restrict__ run_start,
+                                                                          int* __restrict__ nruns) {
   pdl_wait();
   pdl_trigger();
-  extern __shared__ uint32_t sk[];  // [P] keys, then [P/1024 + 1] scan scratch
-  int P = 1;
-  while (P < n) P <<= 1;
-  for (int i = threadIdx.x; i < P; i += blockDim.x) {
+  extern __shared__ uint32_t sk[];                  // [EMB_SEG] keys
+  int* cnt = reinterpret_cast<int*>(sk + EMB_SEG);  // [16][EMB_SORT_THREADS] digit counts, then offsets
+  __shared__ int warp_sum[EMB_SORT_THREADS / 32];
+  const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
+  uint32_t key[EMB_SORT_PER_THREAD];
+#pragma unroll
+  for (int j = 0; j < EMB_SORT_PER_THREAD; ++j) {
+    const int i = t * EMB_SORT_PER_THREAD + j;
     if (i < n) {
       int id = tok[i];
       id = min(max(id, 0), V - 1);
-      sk[i] = ((uint32_t)id << 16) | (uint32_t)i;
+      key[j] = ((uint32_t)id << 16) | (uint32_t)i;
     } else {
-      sk[i] = 0xFFFFFFFFu;
+      key[j] = 0xFFFFFFFFu;  // after every real key of id 0xFFFF too: it starts later and the sort is stable
     }
   }
-  __syncthreads();
-  for (int k = 2; k <= P; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < P; i += blockDim.x) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const uint32_t a = sk[i], b = sk[ixj];
-          const bool up = ((i & k) == 0);
-          if ((a > b) == up) { sk[i] = b; sk[ixj] = a; }
-        }
+#pragma unroll 1
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 16 + 4 * pass;
+    int c[16];
+#pragma unroll
+    for (int dg = 0; dg < 16; ++dg) c[dg] = 0;
+#pragma unroll
+    for (int j = 0; j < EMB_SORT_PER_THREAD; ++j) {
+      const int dg = (key[j] >> shift) & 15;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) c[e] += (dg == e);
+    }
+#pragma unroll
+    for (int dg = 0; dg < 16; ++dg) cnt[dg * EMB_SORT_THREADS + t] = c[dg];
+    __syncthreads();
+    // exclusive scan of cnt in (digit, thread) order: thread t scans elements 16t .. 16t+15
+    int local[16], sum = 0;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      local[e] = sum;
+      sum += cnt[16 * t + e];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_sum[wid] = incl;
+    __syncthreads();
+    int base = incl - sum;
+    for (int w = 0; w < wid; ++w) base += warp_sum[w];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) cnt[16 * t + e] = base + local[e];
+    __syncthreads();
+    // scatter this thread's keys, in order, from its first slot per digit
+    int off[16];
+#pragma unroll
+    for (int dg = 0; dg < 16; ++dg) off[dg] = cnt[dg * EMB_SORT_THREADS + t];
+#pragma unroll
+    for (int j = 0; j < EMB_SORT_PER_THREAD; ++j) {
+      const int dg = (key[j] >> shift) & 15;
+      int slot = 0;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        if (dg == e) { slot = off[e]; off[e] = slot + 1; }
       }
-      __syncthreads();
+      sk[slot] = key[j];
     }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < EMB_SORT_PER_THREAD; ++j) key[j] = sk[t * EMB_SORT_PER_THREAD + j];
+    __syncthreads();
   }
-  for (int i = threadIdx.x; i < n; i += blockDim.x) keys_out[i] = sk[i];
+  for (int i = t; i < n; i += blockDim.x) keys_out[i] = sk[i];
   __syncthreads();
   // run heads: a stable compaction with a block-wide scan over chunks of blockDim.x
   __shared__ int warp_tot[32];
@@ -655,13 +707,11 @@ gpt_status embedding_bwd(const int32_t* tok, const float* gx, float* dwte, int M
   int* nruns = reinterpret_cast<int*>(p + al((size_t)seg * 4) + al((size_t)(seg + 1) * 4));
   float* partial = reinterpret_cast<float*>(p + al((size_t)seg * 4) + al((size_t)(seg + 1) * 4) + al(4));
   GPT_CUDA_TRY(cudaMemsetAsync(dwte, 0, (size_t)V * d * sizeof(float), s));
-  GPT_TRY(ensure_smem(embedding_sort_kernel, EMB_SEG * 4));
+  GPT_TRY(ensure_smem(embedding_sort_kernel, EMB_SORT_SMEM));
   const int threads = std::min(512, std::max(32, ((d / 4) + 31) / 32 * 32));
   for (int s0 = 0; s0 < M; s0 += EMB_SEG) {
     const int n = std::min(EMB_SEG, M - s0);
-    int P = 1;
-    while (P < n) P <<= 1;
-    embedding_sort_kernel<<<1, 1024, (size_t)P * 4, s>>>(tok + s0, n, V, keys, run_start, nruns);
+    embedding_sort_kernel<<<1, EMB_SORT_THREADS, EMB_SORT_SMEM, s>>>(tok + s0, n, V, keys, run_start, nruns);
     count_launch();
     GPT_CUDA_TRY(cudaGetLastError());
     const int pieces = (n + EMB_PIECE - 1) / EMB_PIECE;
