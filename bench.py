@@ -281,6 +281,23 @@ def measure_step(args, cfg, dev, world, rank, barrier, exchange, with_e2e=True):
         raise RuntimeError(f"device status {st} after warm-up ({cfg.name})")
     loss0 = float(step.loss.item())
 
+    # the step as one CUDA graph (its launches recorded once), unless disabled or not capturable
+    graph = None
+    if not getattr(args, "no_graph", False) and world == 1:
+        try:
+            graph = step.capture(params, tokens, targets)
+            torch.cuda.synchronize(dev)
+        except Exception as e:  # noqa: BLE001 - the eager launches below are the same kernels
+            print(f"step graph not captured ({type(e).__name__}: {e}); timing eager launches",
+                  file=sys.stderr)
+            graph = None
+
+    def run_step():
+        if graph is not None:
+            return graph.replay(), graph.launches
+        out = step(params, tokens, targets)
+        return out, step.last_launch_count()
+
     # ---------------- timed region (device-resident inputs) ----------------
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     clocks = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
@@ -292,9 +309,9 @@ def measure_step(args, cfg, dev, world, rank, barrier, exchange, with_e2e=True):
     launches = 0
     e0.record(stream)
     for _ in range(args.steps):
-        _, grads = step(params, tokens, targets)
+        (_, grads), n_launch = run_step()
         exchange(grads)
-        launches += step.last_launch_count()
+        launches += n_launch
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -316,7 +333,9 @@ def measure_step(args, cfg, dev, world, rank, barrier, exchange, with_e2e=True):
         tok_h = torch.from_numpy(tok_np).pin_memory()
         tgt_h = torch.from_numpy(tgt_np).pin_memory()
         loss_h = torch.zeros(1, dtype=torch.float32).pin_memory()
-        tok_d, tgt_d = torch.empty_like(tokens), torch.empty_like(targets)
+        # the graph reads tokens/targets from the buffers it was captured with: copy into those
+        tok_d, tgt_d = (tokens, targets) if graph is not None else (torch.empty_like(tokens),
+                                                                     torch.empty_like(targets))
         barrier()
         torch.cuda.synchronize(dev)
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -324,7 +343,10 @@ def measure_step(args, cfg, dev, world, rank, barrier, exchange, with_e2e=True):
         for _ in range(args.steps):
             tok_d.copy_(tok_h, non_blocking=True)
             tgt_d.copy_(tgt_h, non_blocking=True)
-            loss, grads = step(params, tok_d, tgt_d)
+            if graph is not None:
+                loss, grads = graph.replay()
+            else:
+                loss, grads = step(params, tok_d, tgt_d)
             exchange(grads)
             loss_h.copy_(loss, non_blocking=True)
         f1.record(stream)
@@ -345,9 +367,10 @@ def measure_step(args, cfg, dev, world, rank, barrier, exchange, with_e2e=True):
         kernels[name] = ent
     out = {"ms": ms, "ms_e2e": ms_e2e_m if ms_e2e is not None else None, "clocks": clk,
            "launches": launches, "loss0": loss0, "prof": prof, "prof_steps": prof_steps,
+           "step_launch": "one CUDA graph per step" if graph is not None else "kernel launches from the host",
            "kernels": kernels, "params_np": params_np,
            "h2d": int(tok_np.nbytes + tgt_np.nbytes)}
-    del step, params, tokens, targets, grads
+    del graph, step, params, tokens, targets, grads
     torch.cuda.empty_cache()
     return out
 
@@ -453,6 +476,7 @@ def run_ours(args, cfg):
         "e2e": {"value": value_e2e, "unit": "tokens/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": 4},
         "gpu_launches": int(r["launches"]),
+        "step_launch": r["step_launch"],
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
                      "frac": (achieved / peak_sus) if achieved else None,
                      "peak_source": f"bf16_tflops_sustained of {peak_src}",
@@ -629,6 +653,8 @@ def main():
     ap.add_argument("--also", default="d20", help="second configuration measured in the same run")
     ap.add_argument("--no-also", action="store_true")
     ap.add_argument("--no-optim", action="store_true", help="skip the optimizer-step measurement")
+    ap.add_argument("--no-graph", action="store_true", help="launch the step's kernels from the host "
+                    "instead of replaying it as one CUDA graph")
     ap.add_argument("--rows-d", default="65536,1536", help="rmsnorm workload: rows,d")
     ap.add_argument("--norm-pass", default="fwd", choices=["fwd", "bwd"])
     ap.add_argument("--emb", default="32768,1536,32768", help="embedding workload: M,d,V")

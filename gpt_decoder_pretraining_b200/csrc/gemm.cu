@@ -13,13 +13,14 @@
 //   warps 2..   epilogue (both CTAs): 4 warps per column group (one per tensor-memory lane
 //               quarter; two groups split the 256 columns, one for the QKV + RoPE epilogue);
 //               tcgen05.ld one accumulator row per thread, fused epilogue (bf16 cast, residual add,
-//               ReLU², dReLU², fp32 store / add, split-K reduction, QKV + RoPE + QK-norm, or the
+//               ReLU², dReLU², fp32 store / add, axpby, head-major stores, QKV + RoPE + QK-norm, or the
 //               cross-entropy statistics / gradient of the fused lm-head), global store; then
 //               release the accumulator buffer to the leader.
 // Tiles are distributed persistently over the CTA pairs.  When the tile count leaves the last wave
-// partly empty, the tail tiles are split along K into equal ranges per pair ("stream-K"): every pair
-// then finishes at the same time, and a tile whose K range is split is summed from its pieces,
-// in ascending K order, by the piece that finishes last (no waiting, no atomics on the output,
+// partly empty, each tail tile is split along K into equal ranges that start together on several
+// pairs (the whole waves before them keep every pair's K in step, so operands shared by
+// concurrent tiles come from L2); a tile whose K range is split is summed from its pieces, in
+// ascending K order, by the piece that finishes last (no waiting, no atomics on the output,
 // bitwise reproducible).
 //
 // Operand majors: A and B may each be K-contiguous ("K-major") or M/N-contiguous ("MN-major"),
@@ -315,7 +316,7 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, int b, int m, 
 }
 
 // Epilogues that write each accumulator element on its own (bf16 cast, residual add, ReLU²,
-// dReLU², fp32 store / add): these are the ones whose tiles may be split stream-K.
+// dReLU², fp32 store / add, axpby): these are the ones whose tiles may be split along K.
 template <int EPI>
 constexpr bool epi_plain() {
   return EPI == GPT_EPI_BF16 || EPI == GPT_EPI_RESID || EPI == GPT_EPI_RELU2 ||
@@ -324,7 +325,7 @@ constexpr bool epi_plain() {
 
 // One epilogue warp's share of a work unit: rows 32q .. 32q+31 of this CTA's 128, columns
 // 128·half .. +127 of the tile.  Waits for the accumulator (`tfull`), then either stores the tile
-// (a whole-K unit) or, for a stream-K piece, publishes its partial sums and — if it is the last
+// (a whole-K unit) or, for a piece of a split tile, publishes its partial sums and — if it is the last
 // piece of the tile to arrive — adds all pieces in ascending K order and stores the sum.
 // Returns false if the wait gave up.
 template <int EPI>
@@ -374,7 +375,7 @@ __device__ __forceinline__ bool plain_epilogue(const GemmArgs& a, const Work& w,
     }
     return true;
   }
-  // ---- stream-K piece ----
+  // ---- piece of a split tile ----
   const int st = w.tile - sch.dp_tiles;
   const int nseg = sch.sk_split, seg = w.piece;
   const size_t row_off = (size_t)(rank * BM + q * 32 + lane) * BN + half * (BN / 2);

@@ -106,7 +106,7 @@ struct GemmBatch {
   int* status;
 };
 gpt_status gemm_launch_batched(const GemmBatch& g, cudaStream_t stream, void* sk_scratch);
-// Bytes at the start of the stream-K scratch holding the arrival counters (zeroed per step).
+// Bytes at the start of the split-tile scratch holding the arrival counters (zeroed per step).
 constexpr size_t GEMM_SK_COUNTER_BYTES = 320 * 16 * sizeof(int);
 
 struct CeArgs {

@@ -265,7 +265,7 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
   int* status = reinterpret_cast<int*>(ws + p.status);
   float* rope = reinterpret_cast<float*>(ws + p.rope);
   GPT_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
-  // stream-K arrival counters of the GEMMs: zero here, and every GEMM leaves them at zero
+  // arrival counters of the GEMMs' split tiles: zero here, and every GEMM leaves them at zero
   void* sk = ws + p.sk;
   GPT_CUDA_TRY(cudaMemsetAsync(sk, 0, GEMM_SK_COUNTER_BYTES, s));
   const uint16_t* P = reinterpret_cast<const uint16_t*>(params);

@@ -182,6 +182,20 @@ def param_layout(cfg: GptConfig):
     return list(offs), int(total.value)
 
 
+class StepGraph:
+    """A captured training step (GptStep.capture): replay() enqueues it on the current stream and
+    returns (loss, grads), the buffers the captured step writes."""
+
+    def __init__(self, graph, outputs, launches: int):
+        self._g = graph
+        self.outputs = outputs
+        self.launches = launches  # kernel launches recorded in the graph
+
+    def replay(self):
+        self._g.replay()
+        return self.outputs
+
+
 class GptStep:
     """One training step on the GPU: ``loss, grads = step(params, tokens, targets)``."""
 
@@ -224,6 +238,19 @@ class GptStep:
                                     self.workspace_bytes, 1 if accumulate else 0, _stream())
         _check(st, "gpt_step_fwd_bwd")
         return loss, grads
+
+    def capture(self, params, tokens, targets, grads=None, loss=None, accumulate=False):
+        """Record one step with these buffers into a CUDA graph (one launch of the whole step instead
+        of ~500 kernel launches from the host).  Returns a StepGraph; its replay() enqueues the step
+        again on the current stream, reading whatever the same buffers then hold.  A plain step runs
+        first, so that first-call work (kernel attributes) happens outside the capture."""
+        import torch
+        self(params, tokens, targets, grads, loss, accumulate)
+        torch.cuda.synchronize(self.device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            out = self(params, tokens, targets, grads, loss, accumulate)
+        return StepGraph(g, out, self.last_launch_count())
 
     def grad_buckets(self):
         """[(begin, end)] element ranges of the gradient buckets, in the order the backward pass
@@ -324,7 +351,7 @@ _gemm_scratch = {}
 
 
 def gemm_scratch(device):
-    """A device buffer for gpt_gemm's stream-K scratch, one per device, kept for reuse."""
+    """A device buffer for gpt_gemm's split-tile scratch, one per device, kept for reuse."""
     import torch
     dev = torch.device(device)
     key = dev.index if dev.index is not None else torch.cuda.current_device()
@@ -336,7 +363,8 @@ def gemm_scratch(device):
 def gemm(op: int, epi: int, A, B, C, M: int, N: int, K: int, C2=None, aux=None, status=None,
          lda=None, ldb=None, ldc=None, scratch="auto"):
     """C (op) A·B as defined for gpt_gemm; row strides default to the tensors' last dimension.
-    scratch: "auto" (a cached per-device buffer, so that stream-K may be used), None, or a tensor."""
+    scratch: "auto" (a cached per-device buffer, so that a partly empty last wave may be split along
+    K), None, or a tensor."""
     lda = lda or A.shape[-1]
     ldb = ldb or B.shape[-1]
     ldc = ldc or C.shape[-1]

@@ -172,10 +172,11 @@ gpt_status gpt_step_profile(gpt_step* step, double* ms, int64_t* calls, double* 
  *                                                       through gpt_gemm_batched)
  * Sizes: M, N ≥ 1; K ≥ 1 (tails are zero-filled).  Pointers 16-byte aligned.
  * scratch: NULL, or gpt_gemm_scratch_bytes() bytes of device memory (256-byte aligned) that the
- * call may use to split the tiles of a partly empty last wave along K across all CTA pairs
- * ("stream-K": each pair gets an equal share of the K-steps; the pieces of a split tile are summed
- * in ascending K order by the piece that finishes last, so results are bitwise reproducible and no
- * output is zeroed or updated atomically).  The call zeroes the scratch's counters on `stream`
+ * call may use to split the tiles of a partly empty last wave along K: after the whole waves, each
+ * remaining tile is cut into s equal K ranges that run at the same time on s CTA pairs (s chosen
+ * by a cost model, at most pairs / tail tiles); the pieces of a split tile are summed in ascending K
+ * order by the piece that finishes last, so results are bitwise reproducible and no output is
+ * zeroed or updated atomically.  The call zeroes the scratch's counters on `stream`
  * first; concurrent calls need separate scratch buffers.  With NULL every tile is computed whole. */
 enum { GPT_GEMM_NT = 0, GPT_GEMM_NN = 1, GPT_GEMM_TN = 2 };
 enum {

@@ -1,7 +1,7 @@
 """Parity of the 8-bit path (needs a B200): gpt_quantize_e4m3 gives bit-identical codes and the same
 dequantisation factor as the oracle (both decide every code in fp32), and gpt_gemm_e4m3 (tcgen05
 kind::f8f6f4) matches the oracle's exact product of the decoded codes within the bf16 rounding of
-its output, on ragged shapes and on a shape whose tail is split along K (stream-K)."""
+its output, on ragged shapes and on a shape whose tail is split along K."""
 import numpy as np
 import pytest
 import torch

@@ -138,3 +138,32 @@ def test_step_accumulates_gradients_across_micro_batches():
     torch.cuda.synchronize()
     assert st.status() == 0
     assert np.array_equal(acc.cpu().numpy(), (g_a + g_b).astype(np.float32))
+
+
+def test_step_graph_replay_matches_eager_launches():
+    """The step captured as one CUDA graph (GptStep.capture) gives bitwise the eager step's loss and
+    gradients, and a replay after the token buffers change computes the new batch."""
+    from gpt_decoder_pretraining_b200.step import GptStep
+    cfg = custom(2, 256, 128, 512, 256, 2, windows=[100, 0])
+    params, tokens, targets = make_config_inputs(cfg)
+    p = torch.from_numpy(params.astype(np.float32)).cuda().to(torch.bfloat16)
+    t = torch.from_numpy(tokens.astype(np.int32)).cuda()
+    y = torch.from_numpy(targets.astype(np.int32)).cuda()
+    st = GptStep(cfg)
+    graph = st.capture(p, t, y)
+    assert graph.launches > 0
+    loss_g, grads_g = graph.replay()
+    torch.cuda.synchronize()
+    loss_g, grads_g = loss_g.clone(), grads_g.clone()
+    eager = GptStep(cfg)
+    loss_e, grads_e = eager(p, t, y)
+    torch.cuda.synchronize()
+    assert torch.equal(loss_g, loss_e) and torch.equal(grads_g, grads_e)
+    # new tokens in the captured buffers: the replay computes them
+    t2 = torch.roll(t, 7, dims=1).contiguous()
+    t.copy_(t2)
+    loss_g2, grads_g2 = graph.replay()
+    loss_e2, grads_e2 = eager(p, t2, y)
+    torch.cuda.synchronize()
+    assert torch.equal(loss_g2, loss_e2) and torch.equal(grads_g2, grads_e2)
+    assert not torch.equal(loss_g2, loss_g)
