@@ -1,6 +1,7 @@
 // Host utilities: device properties, TMA tensor-map encoding, status strings.
 #include <cudaTypedefs.h>
 
+#include <cstdio>
 #include <cstdlib>
 #include <mutex>
 #include <unordered_map>
@@ -36,6 +37,9 @@ gpt_status device_info(int* num_sms) {
   *num_sms = cached_sms[dev];
   return GPT_OK;
 }
+
+static thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+void note_cuda_error(cudaError_t e) { g_last_cuda_error = e; }
 
 gpt_status ensure_smem_limit(const void* kernel, int bytes) {
   static std::mutex mu;
@@ -117,4 +121,11 @@ extern "C" const char* gpt_strerror(int status) {
     case GPT_ERR_NUMERIC_RANGE: return "attention score bound out of the supported range";
     default: return "unknown status";
   }
+}
+
+extern "C" const char* gpt_last_cuda_error(void) {
+  static thread_local char buf[256];
+  const cudaError_t e = gpt::g_last_cuda_error;
+  snprintf(buf, sizeof(buf), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return buf;
 }

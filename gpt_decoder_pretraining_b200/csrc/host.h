@@ -12,10 +12,16 @@
 
 namespace gpt {
 
+// The CUDA error behind the last GPT_ERR_CUDA of this thread (gpt_last_cuda_error reports it).
+void note_cuda_error(cudaError_t e);
+
 #define GPT_CUDA_TRY(expr)                           \
   do {                                               \
     cudaError_t e_ = (expr);                         \
-    if (e_ != cudaSuccess) return GPT_ERR_CUDA;      \
+    if (e_ != cudaSuccess) {                         \
+      ::gpt::note_cuda_error(e_);                    \
+      return GPT_ERR_CUDA;                           \
+    }                                                \
   } while (0)
 
 #define GPT_TRY(expr)                                \
@@ -72,7 +78,11 @@ inline gpt_status launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, s
   attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) return GPT_ERR_CUDA;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  if (e != cudaSuccess) {
+    note_cuda_error(e);
+    return GPT_ERR_CUDA;
+  }
   count_launch();
   return GPT_OK;
 }

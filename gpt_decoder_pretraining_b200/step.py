@@ -29,7 +29,7 @@ EPI_BF16, EPI_RESID, EPI_RELU2, EPI_DRELU2, EPI_F32, EPI_F32_ADD = 0, 1, 2, 3, 4
 
 EXPORTED = [
     "gpt_param_layout", "gpt_step_create", "gpt_step_destroy", "gpt_step_workspace_bytes",
-    "gpt_step_fwd_bwd", "gpt_step_status", "gpt_strerror", "gpt_step_last_launch_count",
+    "gpt_step_fwd_bwd", "gpt_step_status", "gpt_strerror", "gpt_last_cuda_error", "gpt_step_last_launch_count",
     "gpt_step_set_profiling", "gpt_step_profile", "gpt_step_grad_buckets", "gpt_step_grad_bucket",
     "gpt_step_enable_grad_events", "gpt_step_wait_grad_bucket",
     "gpt_gemm", "gpt_gemm_scratch_bytes", "gpt_qkv_proj_rope", "gpt_rmsnorm_fwd", "gpt_rmsnorm_bwd", "gpt_rope_qknorm_fwd", "gpt_rope_qknorm_bwd",
@@ -57,7 +57,10 @@ class OptimHparams(ctypes.Structure):
 class GptError(RuntimeError):
     def __init__(self, status: int, what: str = ""):
         self.status = status
-        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+        msg = f"{what}: {STATUS_NAMES.get(status, status)}"
+        if status == -4 and _lib is not None:  # GPT_ERR_CUDA: add the CUDA error behind it
+            msg += f" ({_lib.gpt_last_cuda_error().decode()})"
+        super().__init__(msg)
 
 
 class _Config(ctypes.Structure):
@@ -87,6 +90,8 @@ def lib():
         L.gpt_step_status.argtypes = [vp, vp, vp]
         L.gpt_strerror.argtypes = [i32]
         L.gpt_strerror.restype = ctypes.c_char_p
+        L.gpt_last_cuda_error.argtypes = []
+        L.gpt_last_cuda_error.restype = ctypes.c_char_p
         L.gpt_step_last_launch_count.argtypes = [vp]
         L.gpt_step_last_launch_count.restype = ctypes.c_int64
         L.gpt_step_set_profiling.argtypes = [vp, i32]

@@ -117,6 +117,9 @@ gpt_status gpt_step_status(const gpt_step* step, const void* workspace, void* st
 /* A short English description of a status code ("unknown status" for others).  No page
  * counterpart. */
 const char* gpt_strerror(int status);
+/* The name and text of the CUDA error behind this thread's last GPT_ERR_CUDA (a per-thread buffer,
+ * valid until the next call on the thread; "cudaSuccess: …" when there was none). */
+const char* gpt_last_cuda_error(void);
 
 /* Number of kernel launches the last gpt_step_fwd_bwd enqueued (host counter, for reporting; the
  * pages trace idle gaps between device programs, Porting nanochat to a TPU, §4). */

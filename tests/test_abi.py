@@ -409,3 +409,11 @@ def _failing_rank_main(rank, world, port, q):
     q.close()
     q.join_thread()
     os._exit(0)
+
+
+def test_last_cuda_error_names_the_error_behind_gpt_err_cuda(lib):
+    """gpt_last_cuda_error: the CUDA error name and text of this thread's last GPT_ERR_CUDA."""
+    f = lib.gpt_last_cuda_error
+    f.restype = ctypes.c_char_p
+    msg = f().decode()
+    assert msg.startswith("cuda") and ": " in msg
