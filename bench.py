@@ -560,6 +560,22 @@ def run_kernel(args):
         run = lambda: S.gemm(op, epi, A, B, C, M, N, K, aux=aux, scratch=scratch)  # noqa: E731
         flops = 2.0 * M * N * K
         unit_desc = f"GEMM {args.gemm_op} M={M} N={N} K={K}"
+    elif args.kernel == "qkv":
+        # QKV projection with the RoPE + QK-norm epilogue: r [M, d] · W_qkv [3d, d]ᵀ → q̃, k̃, v head-major
+        M, d, H = (int(x) for x in args.qkv.split(","))
+        Dh, T = d // H, 2048
+        Bq = max(1, M // T)
+        M = Bq * T
+        r = torch.randn(M, d, device=dev, generator=g).to(torch.bfloat16)
+        w = (torch.randn(3 * d, d, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+        heads = torch.empty(3 * M * d, device=dev, dtype=torch.bfloat16)
+        rq = torch.empty(M * H, device=dev)
+        rk = torch.empty(M * H, device=dev)
+        cs = torch.empty(T * Dh, device=dev)
+        S.rope_table(cs, T, Dh)
+        run = lambda: S.qkv_proj_rope(r, w, heads, rq, rk, cs, Bq, T, H, Dh)  # noqa: E731
+        flops = 2.0 * M * 3 * d * d
+        unit_desc = f"QKV projection + RoPE + QK-norm M={M} d={d} H={H}"
     elif args.kernel == "rmsnorm":
         # RMSNorm forward and backward (bf16 dy, fp32 accumulate + bf16 copy) on [rows, d]
         rows, d = (int(x) for x in args.rows_d.split(","))
@@ -658,7 +674,8 @@ def main():
     ap.add_argument("--rows-d", default="65536,1536", help="rmsnorm workload: rows,d")
     ap.add_argument("--norm-pass", default="fwd", choices=["fwd", "bwd"])
     ap.add_argument("--emb", default="32768,1536,32768", help="embedding workload: M,d,V")
-    ap.add_argument("--kernel", choices=["gemm", "attention", "rmsnorm", "embedding"], default=None,
+    ap.add_argument("--qkv", default="8192,1536,12", help="QKV projection workload: tokens,d,heads")
+    ap.add_argument("--kernel", choices=["gemm", "attention", "rmsnorm", "embedding", "qkv"], default=None,
                     help="time one kernel-level workload instead of the step")
     ap.add_argument("--gemm-shape", default="32768,6144,1536")
     ap.add_argument("--gemm-op", default="nt", choices=["nt", "nn", "tn"])

@@ -340,9 +340,10 @@ __device__ __forceinline__ bool plain_epilogue(const GemmArgs& a, const Work& w,
   constexpr bool kPre = (EPI == GPT_EPI_RESID || EPI == GPT_EPI_DRELU2);
   // The residual / saved activation does not depend on the accumulator: chunk 0 is fetched before
   // the wait for the tile, and chunk c+1 before chunk c is read from tensor memory, so that one
-  // 64-byte row segment per thread is always in flight (within the epilogue warps' registers).
+  // 64-byte row segment per thread is always in flight (within the epilogue warps' registers).  Two
+  // buffers alternate, chunk pairs per loop trip, so no register copy waits on a load in flight.
   const bool pre_ok = kPre && !piece && m < a.M;
-  uint4 cur[4], nxt[4];
+  uint4 bufa[4], bufb[4];
   auto fetch = [&](int c, uint4 (&dst)[4]) {
     const int n0 = nbase + 32 * c;
     if (pre_ok && n0 + 32 <= a.N) {
@@ -353,25 +354,27 @@ __device__ __forceinline__ bool plain_epilogue(const GemmArgs& a, const Work& w,
       for (int e = 0; e < 4; ++e) dst[e] = *reinterpret_cast<const uint4*>(src + 8 * e);
     }
   };
-  if (kPre) fetch(0, cur);
+  if (kPre) fetch(0, bufa);
   if (!mbar_wait_warp(tfull, parity, abort_flag, a.status)) return false;
   tc_fence_after();
   const uint32_t t0 = tm_addr + half * (BN / 2);
   if (!piece) {
-#pragma unroll 1
-    for (int c = 0; c < NC; ++c) {
-      if (kPre && c + 1 < NC) fetch(c + 1, nxt);
+    auto chunk = [&](int c, const uint4 (&pre)[4]) {
       uint32_t r[32];
       tmem_ld32(t0 + 32 * c, r);
       tmem_ld_wait();
       const int n0 = nbase + 32 * c;
       const bool use_pre = pre_ok && n0 + 32 <= a.N;
       if (m < a.M && n0 < a.N)
-        epilogue_store<EPI>(a, bb, m, n0, reinterpret_cast<const float*>(r), use_pre, cur);
-      if (kPre) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) cur[e] = nxt[e];
-      }
+        epilogue_store<EPI>(a, bb, m, n0, reinterpret_cast<const float*>(r), use_pre, pre);
+    };
+    static_assert(NC % 2 == 0, "chunk pairs");
+#pragma unroll 1
+    for (int c = 0; c < NC; c += 2) {
+      if (kPre) fetch(c + 1, bufb);
+      chunk(c, bufa);
+      if (kPre && c + 2 < NC) fetch(c + 2, bufa);
+      chunk(c + 1, bufb);
     }
     return true;
   }
