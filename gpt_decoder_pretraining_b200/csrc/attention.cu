@@ -720,8 +720,9 @@ __device__ __forceinline__ void qknorm_rope_bwd_tmem(uint32_t taddr, float scale
 // ------------------------------------------------------------------------------------------------
 // dK/dV kernel.  16 softmax-backward warps in two groups; group g takes the query tiles
 // i ≡ g (mod 2), so each group has two tile-times of tensor work to turn its Sᵀ / dPᵀ into
-// Pᵀ / dSᵀ.  −LSE and −delta enter the softmax arithmetic (one fused multiply-add and one
-// subtraction per element, fp32 values staged per query tile by a bulk copy).  Each warp works in
+// Pᵀ / dSᵀ.  Sᵀ and dPᵀ are signalled separately: the exponentials run while dPᵀ is computed.
+// −LSE and −delta enter the softmax arithmetic (one fused multiply-add and one subtraction per
+// element, fp32 values staged per query tile by a bulk copy).  Each warp works in
 // 16-column chunks (registers for 576 threads); the epilogue splits dV (group 0) and dK (group 1)
 // by column halves.  dS goes to global memory query-major: for one query the 32 lanes of a warp
 // hold 32 consecutive keys, so every store instruction writes 64 contiguous bytes.
@@ -823,8 +824,9 @@ __global__ void __launch_bounds__(576, 1)
   uint64_t* kv_bar = bars;
   uint64_t* q_full = bars + 1;                // [STAGES]
   uint64_t* q_empty = q_full + S::STAGES;     // [STAGES]
-  uint64_t* s_full = q_empty + S::STAGES;     // [2]
-  uint64_t* p_full = s_full + 2;              // [2]
+  uint64_t* s_full = q_empty + S::STAGES;     // [2] Sᵀ of a tile in tensor memory
+  uint64_t* dp_full = s_full + 2;             // [2] dPᵀ of a tile in tensor memory
+  uint64_t* p_full = dp_full + 2;             // [2] Pᵀ and dSᵀ written back
   uint64_t* done = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -849,6 +851,7 @@ __global__ void __launch_bounds__(576, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
+      mbar_init(&dp_full[i], 1);
       mbar_init(&p_full[i], 256);
     }
     mbar_init(done, 1);
@@ -918,8 +921,9 @@ __global__ void __launch_bounds__(576, 1)
       const uint32_t so = st * S::STAGE_BYTES;
       if (elect_one()) {
         mma_rows_128x64<DH>(tmem + S::TM_S + bf * 64, kd, sdesc_add(q_k, so), id_s);    // Sᵀ
+        tc_commit(&s_full[bf]);  // the exponentials can start while dPᵀ runs
         mma_rows_128x64<DH>(tmem + S::TM_P + bf * 64, vd, sdesc_add(do_k, so), id_s);   // dPᵀ
-        tc_commit(&s_full[bf]);
+        tc_commit(&dp_full[bf]);
       }
       __syncwarp();
       if (i >= 1) {
@@ -957,36 +961,59 @@ __global__ void __launch_bounds__(576, 1)
       const long long bh = (long long)b * a.H + hk * a.group + i / n_qt;  // the query head
       const int qh = (q_first + i % n_qt) * 64 + 32 * half;  // first query of this warp's 32 columns
       const float* ldl = reinterpret_cast<const float*>(smem + S::OFF_LD + st * S::LD_BYTES) + 32 * half;
-#pragma unroll 1
+      // phase 1 (needs Sᵀ only): Pᵀ = 2^(Sᵀ·scale·log2 e − LSE·log2 e) for the 32 queries, kept in
+      // fp32 for phase 2 and written back packed
+      float p[32];
+#pragma unroll
       for (int c = 0; c < 2; ++c) {
         const int qc = qh + 16 * c;
-        uint32_t rs[16], rp[16];
+        uint32_t rs[16];
         tmem_ld16(tmem + lane_off + S::TM_S + grp * 64 + 32 * half + 16 * c, rs);
-        tmem_ld16(tmem + lane_off + S::TM_P + grp * 64 + 32 * half + 16 * c, rp);
         tmem_ld_wait();
         // every (key, query) of the chunk visible: no per-element mask
         const bool full = (kmax_ <= qc) && (kmin > qc + 15 - W) && (qc + 15 < T);
-        uint32_t pk[8], dk[8];
+        uint32_t pk[8];
 #pragma unroll
         for (int g4 = 0; g4 < 4; ++g4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(ldl + 16 * c + 4 * g4);        // LSE·log2 e
-          const float4 d4 = *reinterpret_cast<const float4*>(ldl + 64 + 16 * c + 4 * g4);   // delta
+          const float4 l4 = *reinterpret_cast<const float4*>(ldl + 16 * c + 4 * g4);  // LSE·log2 e
 #pragma unroll
           for (int e2 = 0; e2 < 2; ++e2) {
             const int j = 4 * g4 + 2 * e2;
-            const float la = e2 ? l4.z : l4.x, lb = e2 ? l4.w : l4.y;
-            const float da = e2 ? d4.z : d4.x, db = e2 ? d4.w : d4.y;
-            float x0, x1, u0, u1, s0, s1;
-            fma2(x0, x1, __uint_as_float(rs[j]), __uint_as_float(rs[j + 1]), a.scale_log2, a.scale_log2, -la, -lb);
+            float x0, x1;
+            fma2(x0, x1, __uint_as_float(rs[j]), __uint_as_float(rs[j + 1]), a.scale_log2, a.scale_log2,
+                 -(e2 ? l4.z : l4.x), -(e2 ? l4.w : l4.y));
             float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
             if (!full) {
               const int qq = qc + j;
               if (!((qq < T) && (key <= qq) && (key > qq - W))) p0 = 0.f;
               if (!((qq + 1 < T) && (key <= qq + 1) && (key > qq + 1 - W))) p1 = 0.f;
             }
-            sub2(u0, u1, __uint_as_float(rp[j]), __uint_as_float(rp[j + 1]), da, db);
-            mul2(s0, s1, p0, p1, u0, u1);
+            p[16 * c + j] = p0;
+            p[16 * c + j + 1] = p1;
             pk[j / 2] = pack_bf2(p0, p1);
+          }
+        }
+        // packed: chunk c of half h fills columns 32h + 8c .. +7, inside what this warp has read
+        tmem_st8(tmem + lane_off + S::TM_S + grp * 64 + 32 * half + 8 * c, pk);
+      }
+      // phase 2: dSᵀ = Pᵀ∘(dPᵀ − delta)
+      if (!mbar_wait_warp(&dp_full[grp], (i >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t rp[16];
+        tmem_ld16(tmem + lane_off + S::TM_P + grp * 64 + 32 * half + 16 * c, rp);
+        tmem_ld_wait();
+        uint32_t dk[8];
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(ldl + 64 + 16 * c + 4 * g4);  // delta
+#pragma unroll
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const int j = 4 * g4 + 2 * e2;
+            float u0, u1, s0, s1;
+            sub2(u0, u1, __uint_as_float(rp[j]), __uint_as_float(rp[j + 1]), e2 ? d4.z : d4.x, e2 ? d4.w : d4.y);
+            mul2(s0, s1, p[16 * c + j], p[16 * c + j + 1], u0, u1);
             dk[j / 2] = pack_bf2(s0, s1);
           }
         }
@@ -999,8 +1026,6 @@ __global__ void __launch_bounds__(576, 1)
             row0[(2 * e + 1) * 32] = (uint16_t)(dk[e] >> 16);
           }
         }
-        // packed: chunk c of half h fills columns 32h + 8c .. +7, inside what this warp has read
-        tmem_st8(tmem + lane_off + S::TM_S + grp * 64 + 32 * half + 8 * c, pk);
         tmem_st8(tmem + lane_off + S::TM_P + grp * 64 + 32 * half + 8 * c, dk);
       }
       tmem_st_wait();
