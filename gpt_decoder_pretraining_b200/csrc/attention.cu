@@ -53,8 +53,9 @@ struct AttnArgs {
   float* lse;
   float* delta;  // backward: [2][B·H][Tpad] fp32 — LSE·log2(e), then rowsum(dO∘O); zero-padded
   int Tpad;      // T rounded up to a multiple of 64
-  uint16_t* ds;  // backward (optional): dS [B·H][T][Tpad] bf16 (query rows, key columns), written
-                 // by the dK/dV kernel and read by the dQ kernel
+  uint16_t* ds;  // backward (optional): dS [nb·H][T][Tpad] bf16 (query rows, key columns) of the
+                 // batches b0 .. b0+nb−1, written by the dK/dV kernel and read by the dQ kernel
+  int b0;        // backward with dS stored: batch of blockIdx.z = 0 (the batch chunk's first)
   int* status;
   // optional QK-norm + RoPE backward fused into the dq / dk epilogues (rho_q == nullptr: off):
   // q̃ = RMS_Dh(RoPE(q)), so dq = Rᵀ·rho·(dq̃ − q̃·mean(q̃·dq̃)), likewise for k
@@ -832,7 +833,7 @@ __global__ void __launch_bounds__(576, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = warp_id(), lane = lane_id();
-  const int hk = blockIdx.y, b = blockIdx.z;  // one key/value head; its group's query heads in turn
+  const int hk = blockIdx.y, b = blockIdx.z + a.b0;  // one key/value head; its group's query heads in turn
   const int T = a.T, W = a.window;
   const int kv0 = blockIdx.x * 128;
   const int q_first = kv0 / 64;
@@ -1036,7 +1037,7 @@ __global__ void __launch_bounds__(576, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_3d(&mds_st, ds_stage, kmin, qh, (int)bh);
+          tma_store_3d(&mds_st, ds_stage, kmin, qh, (int)(bh - (long long)a.b0 * a.H));
           bulk_commit();
         }
       }
@@ -1343,14 +1344,14 @@ __global__ void __launch_bounds__(192, 2)
 
   const int warp = warp_id(), lane = lane_id();
   const int qt = gridDim.x - 1 - blockIdx.x;  // longest rows first
-  const int h = blockIdx.y, b = blockIdx.z;
+  const int h = blockIdx.y, b = blockIdx.z + a.b0;
   const int T = a.T, W = a.window;
   const int q0 = qt * 128;
   const int key_lo = max(0, q0 - W + 1);
   const int key_hi = min(T, q0 + 128);
   const int kv_first = key_lo / 64;
   const int n_kv = (key_hi - 1) / 64 - kv_first + 1;
-  const int bh = b * a.H + h;
+  const int bh_ds = (int)blockIdx.z * a.H + h;  // the dS block of this (b, h) within the chunk
 
   if (threadIdx.x == 0) {
     mbar_init(q_bar, 1);
@@ -1384,7 +1385,7 @@ __global__ void __launch_bounds__(192, 2)
         mbar_arrive_expect_tx(&full[st], S::STAGE_BYTES);
         uint8_t* dst = smem + S::OFF_STAGE + st * S::STAGE_BYTES;
         const int k0 = (kv_first + j) * 64;
-        tma_load_3d(dst, &mds, &full[st], k0, q0, bh);  // dS rows q0 .. q0+127, keys k0 .. k0+63
+        tma_load_3d(dst, &mds, &full[st], k0, q0, bh_ds);  // dS rows q0 .. q0+127, keys k0 .. k0+63
         load_tile<DH, 64>(dst + S::DS_TILE, &mk, &full[st], k0, h / a.group, b);
       }
     }
@@ -1914,7 +1915,10 @@ gpt_status launch_bwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, c
 // tcgen05 backward: maps with 128-row boxes (outer tiles) and 64-row boxes (inner tiles).
 template <int DH>
 gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[4],
-                         const CUtensorMap* mds, AttnArgs a, void* dq, cudaStream_t stream) {
+                         const CUtensorMap* mds, AttnArgs a, void* dq, cudaStream_t stream,
+                         int batches = -1) {
+  // batches: the grids cover batches a.b0 .. a.b0 + batches − 1 (−1: all of a.B)
+  const int nb = batches < 0 ? a.B : batches;
   // mds: null, or the stored dS's maps — [0] 128-query × 64-key boxes (128-byte swizzle) for the dQ
   // kernel's loads, [1] 32 × 32 boxes (no swizzle) for the dK/dV kernel's per-warp stores
   using S = TcBwdShape<DH>;
@@ -1924,11 +1928,11 @@ gpt_status launch_bwd_tc(const CUtensorMap (&m128)[4], const CUtensorMap (&m64)[
   GPT_TRY(ensure_smem(attn_bwd_dq_tc_kernel<DH>, S::SMEM));
   GPT_TRY(ensure_smem(attn_bwd_dq_ds_kernel<DH>, SD::SMEM));
   // dK/dV: outer 128-key tiles (K, V with 128-row boxes), inner 64-query tiles (Q, dO 64-row boxes)
-  dim3 g1((a.T + 127) / 128, a.Hkv, a.B);  // one CTA per key tile of each key/value head
+  dim3 g1((a.T + 127) / 128, a.Hkv, nb);  // one CTA per key tile of each key/value head
   GPT_TRY(launch_kernel(attn_bwd_dkdv_tc_kernel<DH>, g1, dim3(SK::THREADS), SK::SMEM, stream, m64[0],
                         m128[1], m128[2], m64[3], mds ? mds[1] : m64[0], a));
   a.o = reinterpret_cast<uint16_t*>(dq);
-  dim3 g2((a.T + 127) / 128, a.H, a.B);
+  dim3 g2((a.T + 127) / 128, a.H, nb);
   if (mds != nullptr) {
     // dQ = dS·K from the stored dS tiles: outer 128-query tiles, inner 64-key tiles
     return launch_kernel(attn_bwd_dq_ds_kernel<DH>, g2, dim3(SD::THREADS), SD::SMEM, stream, m128[0],
@@ -1994,12 +1998,22 @@ gpt_status attention_fwd(const void* q, const void* k, const void* v, void* o, f
   return launch_fwd_tc<64>(mq2, mk2, mv2, a, kmax_scratch, kconst, stream);
 }
 
+// Batches whose dS the backward holds at once: as many as fit GPT_ATTN_BWD_DS_MAX_BYTES (at most B);
+// 0 when one batch's dS alone exceeds it, and then dQ recomputes the scores instead.
+static int ds_batch_chunk(int B, int H, int T) {
+  const size_t per_batch = (size_t)H * T * ((T + 63) / 64 * 64) * 2;
+  const size_t fit = (size_t)GPT_ATTN_BWD_DS_MAX_BYTES / per_batch;
+  return (int)std::min<size_t>((size_t)B, fit);
+}
+
 // Backward scratch per padded row (b, h, t < ⌈T/64⌉·64): LSE·log2 e and delta (fp32); then, when
-// stored, dS [B·H][T][⌈T/64⌉·64] bf16.
+// stored, dS [nb·H][T][⌈T/64⌉·64] bf16 for one chunk of nb batches (the chunks reuse it in turn).
 size_t attention_bwd_scratch_bytes(int B, int H, int T, bool store_ds) {
   if (B <= 0 || H <= 0 || T <= 0) return 0;
-  const size_t rows = (size_t)B * H * ((T + 63) / 64 * 64);
-  return rows * 2 * sizeof(float) + (store_ds ? rows * (size_t)T * 2 : 0);
+  const size_t Tpad = (T + 63) / 64 * 64;
+  const size_t rows = (size_t)B * H * Tpad;
+  const size_t nb = store_ds ? (size_t)ds_batch_chunk(B, H, T) : 0;
+  return rows * 2 * sizeof(float) + nb * H * (size_t)T * Tpad * 2;
 }
 
 // Layouts: lq for q, lkv for k and v (Hkv heads), ldq for dq, ldkv for dk and dv, lo for o, ldo for
@@ -2027,17 +2041,9 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
   // [B·H][T][Tpad] bf16 (query rows, key columns)
   const long long rows = (long long)B * H * Tpad;
   if ((reinterpret_cast<uintptr_t>(delta) & 15) != 0) return GPT_ERR_UNSUPPORTED_SHAPE;
-  uint16_t* ds = (Dh != 32 && store_ds) ? reinterpret_cast<uint16_t*>(delta + 2 * rows) : nullptr;
-  CUtensorMap mds[2];
-  if (ds != nullptr) {
-    // keys ≥ T lie outside the maps (read as zero, never written), as do query rows ≥ T
-    const uint64_t dims[3] = {(uint64_t)T, (uint64_t)T, (uint64_t)B * H};
-    const uint64_t strides[2] = {(uint64_t)Tpad * 2, (uint64_t)T * Tpad * 2};
-    const uint32_t box_ld[3] = {64, 128, 1}, box_st[3] = {32, 32, 1};
-    if (!encode_map_bf16(&mds[0], ds, 3, dims, strides, box_ld, true) ||
-        !encode_map_bf16(&mds[1], ds, 3, dims, strides, box_st, false))
-      return GPT_ERR_UNSUPPORTED_SHAPE;
-  }
+  // dS is held for nb batches at a time (nb = 0: not stored, dQ recomputes the scores)
+  const int nb = (Dh != 32 && store_ds) ? ds_batch_chunk(B, H, T) : 0;
+  uint16_t* ds = nb > 0 ? reinterpret_cast<uint16_t*>(delta + 2 * rows) : nullptr;
   if (!delta_ready) {  // else the GEMM that produced dO has written these rows
     const int threads = 256;
     const long long blocks = (rows * (Dh / 8) + threads - 1) / threads;
@@ -2085,8 +2091,27 @@ gpt_status attention_bwd(const void* q, const void* k, const void* v, const void
         !make_head_map(&m64[i], src[i], B, heads[i], T, Dh, lay[i].sb, lay[i].sh, lay[i].st, 64))
       return GPT_ERR_UNSUPPORTED_SHAPE;
   }
-  if (Dh == 128) GPT_TRY(launch_bwd_tc<128>(m128, m64, ds ? mds : nullptr, a, dq, stream));
-  else GPT_TRY(launch_bwd_tc<64>(m128, m64, ds ? mds : nullptr, a, dq, stream));
+  if (ds == nullptr) {
+    if (Dh == 128) return launch_bwd_tc<128>(m128, m64, nullptr, a, dq, stream);
+    return launch_bwd_tc<64>(m128, m64, nullptr, a, dq, stream);
+  }
+  // batch chunks b0 .. b0+n−1 in turn, each through the same dS buffer: the next chunk's dK/dV
+  // kernel writes it only after the previous dQ kernel has finished (stream order)
+  for (int b0 = 0; b0 < B; b0 += nb) {
+    const int n = std::min(nb, B - b0);
+    CUtensorMap mds[2];
+    // keys ≥ T lie outside the maps (read as zero, never written), as do query rows ≥ T
+    const uint64_t dims[3] = {(uint64_t)T, (uint64_t)T, (uint64_t)n * H};
+    const uint64_t strides[2] = {(uint64_t)Tpad * 2, (uint64_t)T * Tpad * 2};
+    const uint32_t box_ld[3] = {64, 128, 1}, box_st[3] = {32, 32, 1};
+    if (!encode_map_bf16(&mds[0], ds, 3, dims, strides, box_ld, true) ||
+        !encode_map_bf16(&mds[1], ds, 3, dims, strides, box_st, false))
+      return GPT_ERR_UNSUPPORTED_SHAPE;
+    a.b0 = b0;
+    a.B = B;
+    if (Dh == 128) GPT_TRY(launch_bwd_tc<128>(m128, m64, mds, a, dq, stream, n));
+    else GPT_TRY(launch_bwd_tc<64>(m128, m64, mds, a, dq, stream, n));
+  }
   return GPT_OK;
 }
 

@@ -260,8 +260,10 @@ gpt_status gpt_rope_table(float* cos_sin, int T, int Dh, void* stream);
  * window ≤ 0 or ≥ T = full causal.  delta: backward scratch of at least
  * gpt_attention_bwd_scratch_bytes(B, H, T) bytes, 16-byte aligned; per row (zero-padded to a
  * multiple of 64 rows per (b, h)) the backward stores LSE·log2(e) and rowsum(dO∘O) in fp32; after
- * these rows, for Dh ≥ 64, the dK/dV kernel stores dS (bf16 [B·H][T][⌈T/64⌉·64], query rows and
- * key columns, causal band / window only) and the dQ kernel contracts it with K.
+ * these rows, for Dh ≥ 64, the dK/dV kernel stores dS (bf16 [nb·H][T][⌈T/64⌉·64], query rows and
+ * key columns, causal band / window only) for a chunk of nb batches and the dQ kernel contracts it
+ * with K, chunk after chunk; nb is the largest count whose dS fits GPT_ATTN_BWD_DS_MAX_BYTES, and
+ * when not even one batch fits, dS is not stored and the dQ kernel recomputes the scores.
  * The forward shifts each row's exponentials by the Cauchy–Schwarz bound c_t = ‖q_t‖·max_j‖k_j‖/√Dh
  * instead of a running maximum (softmax is invariant to the shift, so the result is exact); this
  * needs c_t ≤ 40 so that no row underflows, which always holds after QK-norm (c_t ≈ √Dh) — rows
@@ -275,10 +277,12 @@ gpt_status gpt_attention_fwd(const void* q, const void* k, const void* v, void* 
                              long long sh_kv, long long st_kv, long long sb_o, long long sh_o,
                              long long st_o, int* status, void* stream);
 /* Bytes of the `delta` scratch that gpt_attention_bwd needs for (B, H, T): 8 bytes per row of
- * R = B·H·⌈T/64⌉·64, plus 2·T·R bytes of dS — quadratic in T (1.6 GB for B·H = 192 at T = 2048,
- * 34 GB for B·H·T = 2^21 at T = 8192).  Callers short of memory can use, within its row limit,
- * gpt_attention_bwd_noalloc, which recomputes the scores instead.  Returns 0 for a non-positive
- * size. */
+ * R = B·H·⌈T/64⌉·64, plus the dS of one batch chunk, nb·H·T·⌈T/64⌉·64·2 bytes ≤
+ * GPT_ATTN_BWD_DS_MAX_BYTES (1.6 GB for B 16 × H 12 at T = 2048, one chunk; 8.6 GB for B 32 × H 8
+ * at T = 8192, which runs as four chunks of 8 batches).  Callers short of memory can use, within
+ * its row limit, gpt_attention_bwd_noalloc, which recomputes the scores instead.  Returns 0 for a
+ * non-positive size. */
+#define GPT_ATTN_BWD_DS_MAX_BYTES (8ll << 30)
 size_t gpt_attention_bwd_scratch_bytes(int B, int H, int T);
 gpt_status gpt_attention_bwd(const void* q, const void* k, const void* v, const void* o,
                              const void* dout, const float* lse, float* delta, void* dq, void* dk,

@@ -253,12 +253,19 @@ def test_bucketed_data_parallel_average_equals_the_full_batch_step():
 
 
 def test_attention_backward_scratch_size(lib):
-    """Per padded row 8 bytes (LSE·log2 e and delta in fp32), then dS: 2·T bytes per padded row."""
+    """Per padded row 8 bytes (LSE·log2 e and delta in fp32), then dS for one chunk of batches:
+    2·T bytes per padded row of the chunk, the chunk being as many batches as fit 8 GiB of dS (all
+    of them at the training shapes; 8 of 32 at H 8 × T 8192; none at T 32768, where one batch's
+    dS alone is 16 GiB and the dQ kernel recomputes the scores instead)."""
     f = lib.gpt_attention_bwd_scratch_bytes
     f.restype = ctypes.c_size_t
-    for B, H, T in [(1, 1, 1), (2, 3, 200), (16, 12, 2048), (4, 8, 130)]:
-        rows = B * H * ((T + 63) // 64 * 64)
-        assert f(B, H, T) == rows * 8 + rows * T * 2
+    cap = 8 << 30
+    for B, H, T, nb in [(1, 1, 1, 1), (2, 3, 200, 2), (16, 12, 2048, 16), (4, 8, 130, 4),
+                        (32, 8, 8192, 8), (9, 8, 8192, 8), (1, 8, 32768, 0), (3, 1, 65536, 1), (3, 2, 65536, 0)]:
+        tpad = (T + 63) // 64 * 64
+        rows = B * H * tpad
+        assert nb * H * T * tpad * 2 <= cap < (nb + 1) * H * T * tpad * 2 or nb == B
+        assert f(B, H, T) == rows * 8 + nb * H * T * tpad * 2, (B, H, T)
     assert f(0, 1, 1) == 0 and f(1, 1, 0) == 0
 
 

@@ -9,7 +9,11 @@ a few (batch, head) slices — the first, one in the middle and the last — sin
 T×T probabilities do not fit the whole batch.  Every other slice is checked for finiteness, and
 both status words must stay 0.
 
-A second test raises the norms of q and k until the fixed softmax shift ‖q‖·max‖k‖/√Dh exceeds 40
+A long-sequence test runs T = 32768 with a 1024-key window, where one batch's dS would exceed the
+backward's dS bound, so dQ recomputes the scores: outputs are compared with the oracle on
+sub-sequences that hold every key a checked output depends on.
+
+Another test raises the norms of q and k until the fixed softmax shift ‖q‖·max‖k‖/√Dh exceeds 40
 (where exp of the shifted scores may underflow in fp32): the forward must report
 GPT_ERR_NUMERIC_RANGE instead of passing wrong values off as valid.
 """
@@ -104,3 +108,49 @@ def test_scores_beyond_the_shift_bound_are_reported(Dh):
     assert int(st2.item()) == 0
     o_ref, _ = O.attention_batch_forward(q2, k2, v, 0)
     assert_close_rel(to_np(o), o_ref, rel=2e-2, cos=0.9999, what="o below the bound")
+
+
+def test_long_sequence_backward_without_stored_ds():
+    """T = 32768, H 8, Dh 128, window W = 1024: dS for one batch would be 16 GiB, above the 8 GiB
+    bound, so the backward stores none and the dQ kernel recomputes the scores.  With a window, the
+    outputs of query t depend only on positions (t − W, t], so the oracle on the sub-sequence
+    [t0 − W + 1, t0 + R) reproduces o, LSE and dq of queries [t0, t0 + R) exactly, and dk, dv of keys
+    [t0, t0 + R − W + 1), whose queries all lie in that range; the sub-sequence [0, R) needs no
+    left margin.  Checked on the first and last head, R = 2W, at both ends of the sequence."""
+    B, H, T, Dh, W = 1, HEADS, 32768, 128, 1024
+    assert S.attention_bwd_scratch_bytes(B, H, T) == B * H * T * 8  # no dS held
+    q, k, v, do = make_attention_inputs(B, H, T, Dh, seed=5)
+    tq, tk, tv, tdo = (torch.from_numpy(a).cuda().to(torch.bfloat16) for a in (q, k, v, do))
+    strides = (H * T * Dh, T * Dh, Dh)
+    delta = S.attention_bwd_scratch(B, H, T)
+    o = torch.zeros_like(tq)
+    lse = torch.zeros(B, H, T, dtype=torch.float32, device="cuda")
+    dq, dk, dv = (torch.full_like(tq, float("nan")) for _ in range(3))
+    st_f = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st_b = torch.zeros(1, dtype=torch.int32, device="cuda")
+    S.attention_fwd(tq, tk, tv, o, lse, W, strides, strides, B, H, T, Dh, status=st_f)
+    S.attention_bwd(tq, tk, tv, o, tdo, lse, delta, dq, dk, dv, W, strides, strides, B, H, T, Dh,
+                    status=st_b)
+    torch.cuda.synchronize()
+    assert int(st_f.item()) == 0 and int(st_b.item()) == 0
+    for t in (o, lse, dq, dk, dv):
+        assert bool(torch.isfinite(t).all())
+    R = 2 * W
+    floor = 2.0 ** -9 * math.sqrt(Dh)
+    for h in (0, H - 1):
+        for t0 in (0, T - R):
+            lo = max(0, t0 - W + 1)
+            sl = (slice(0, 1), slice(h, h + 1), slice(lo, t0 + R))
+            qs, ks, vs, dos = (a[sl].astype(np.float64) for a in (q, k, v, do))
+            o_ref, lse_ref = O.attention_batch_forward(qs, ks, vs, W)
+            dq_ref, dk_ref, dv_ref = O.attention_batch_backward(qs, ks, vs, dos, W)
+            rq = slice(t0 - lo, t0 - lo + R)            # queries checked, within the sub-sequence
+            rk = slice(t0 - lo, t0 - lo + R - W + 1)    # keys checked
+            gq = (slice(0, 1), slice(h, h + 1), slice(t0, t0 + R))
+            gk = (slice(0, 1), slice(h, h + 1), slice(t0, t0 + R - W + 1))
+            what = f"T={T} w={W} h={h} t0={t0}"
+            assert_close_rel(to_np(o[gq]), o_ref[:, :, rq], rel=2e-2, cos=0.9999, what="o " + what)
+            np.testing.assert_allclose(to_np(lse[gq]), lse_ref[:, :, rq], atol=2e-3, err_msg="lse " + what)
+            assert_close_rel(to_np(dq[gq]), dq_ref[:, :, rq], rel=3e-2, cos=0.999, what="dq " + what, atol=floor)
+            assert_close_rel(to_np(dk[gk]), dk_ref[:, :, rk], rel=3e-2, cos=0.999, what="dk " + what, atol=floor)
+            assert_close_rel(to_np(dv[gk]), dv_ref[:, :, rk], rel=3e-2, cos=0.999, what="dv " + what, atol=floor)
