@@ -137,6 +137,14 @@ struct GemmArgs {
   float* sk_part;                  // [sk_tiles·sk_split][256][256] partial tiles
   int* sk_cnt;                     // [sk_tiles·16] arrival counters, zero between launches
   int batch;                       // independent matrices; tile t belongs to matrix t / (tiles_m·tiles_n)
+  // grouped launch (groups > 1, a kernel built for that): tiles g_tile0[g] .. g_tile0[g+1]−1 belong
+  // to problem g — its own operand maps, output g_C[g] (row stride g_ldc[g]) of g_M[g] × g_N[g] in
+  // g_tiles_m[g] × g_tiles_n[g] tiles; every problem has the same K
+  int groups;
+  int g_tile0[GEMM_MAX_GROUPS + 1];
+  int g_M[GEMM_MAX_GROUPS], g_N[GEMM_MAX_GROUPS], g_tiles_m[GEMM_MAX_GROUPS], g_tiles_n[GEMM_MAX_GROUPS];
+  int g_ldc[GEMM_MAX_GROUPS];
+  void* g_C[GEMM_MAX_GROUPS];
   long long c_bstride, aux_bstride;  // elements between consecutive matrices of C and aux
   float alpha, beta;               // GPT_EPI_AXPBY
   const float* dq_a;               // e4m3 operands: device dequantisation factors (else null)
@@ -168,6 +176,30 @@ struct GemmArgs {
   int dl_Tpad;
   long long dl_rows;      // B·H·Tpad
 };
+
+// Operand maps of the NG problems of one launch (NG = 1: an ordinary or batched GEMM).
+template <int NG>
+struct GemmMaps {
+  CUtensorMap a[NG];
+  CUtensorMap b[NG];
+};
+
+// Output tile t of the launch → problem g, matrix bb of a batch, pair-tile row tm and column tn.
+template <int NG>
+__device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, int& g, int& bb, int& tm, int& tn) {
+  if constexpr (NG == 1) {
+    const int per_mat = a.tiles_m * a.tiles_n;
+    g = 0;
+    bb = t / per_mat;
+    tile_coords(t - bb * per_mat, a.tiles_m, a.tiles_n, a.raster, tm, tn);
+  } else {
+    g = 0;
+#pragma unroll
+    for (int i = 1; i < NG; ++i) g += (i < a.groups && t >= a.g_tile0[i]) ? 1 : 0;
+    bb = 0;
+    tile_coords(t - a.g_tile0[g], a.g_tiles_m[g], a.g_tiles_n[g], 1, tm, tn);
+  }
+}
 
 struct GemmShape {
   static constexpr int A_BYTES = BM * BK * 2;        // 16 KB
@@ -438,10 +470,11 @@ __device__ __forceinline__ bool plain_epilogue(const GemmArgs& a, const Work& w,
 // ------------------------------------------------------------------------------------------------
 // F8: A and B are e4m3 (one byte per element): a k-tile is 128 elements (the same 128-byte rows as
 // 64 bf16), one MMA instruction covers K = 32, and the accumulator is scaled in the epilogue.
-template <bool A_MN, bool B_MN, int EPI, bool F8 = false>
+// NG > 1: a grouped launch of NG problems (plain epilogues only), see GemmArgs::groups.
+template <bool A_MN, bool B_MN, int EPI, bool F8 = false, int NG = 1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(), 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const GemmArgs args) {
+    gemm_kernel(const __grid_constant__ GemmMaps<NG> maps, const GemmArgs args) {
+  static_assert(NG == 1 || epi_plain<EPI>(), "grouped launches use the plain epilogues");
   constexpr int KE = F8 ? 2 * BK : BK;  // elements per k-tile
   using S = GemmShape;
   extern __shared__ uint8_t smem_raw[];
@@ -468,8 +501,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
     }
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      tma_prefetch_desc(&maps.a[g]);
+      tma_prefetch_desc(&maps.b[g]);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, S::TMEM_COLS);
@@ -492,11 +528,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
       uint32_t phase = 0;
       WorkIter it(sch, pair);
       Work w;
-      const int per_mat = args.tiles_m * args.tiles_n;
       while (it.next(sch, w)) {
-        const int bb = w.tile / per_mat, tr = w.tile % per_mat;
-        int tm, tn;
-        tile_coords(tr, args.tiles_m, args.tiles_n, args.raster, tm, tn);
+        int g, bb, tm, tn;
+        decode_tile<NG>(args, w.tile, g, bb, tm, tn);
+        const CUtensorMap* tmA = &maps.a[g];
+        const CUtensorMap* tmB = &maps.b[g];
         const int kt0 = w.k0, kt1 = w.k1;
         const int arow = tm * 2 * BM + rank * BM;        // this CTA's 128 rows of A
         const int brow = tn * BN + rank * (BN / 2);      // this CTA's 128 rows of B
@@ -508,18 +544,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * S::STAGE_BYTES);
           const int k0 = kt * KE;
           if (!A_MN) {
-            tma_load_3d_pair(sa, &tmA, &full[stage], k0, arow, bb);
+            tma_load_3d_pair(sa, tmA, &full[stage], k0, arow, bb);
           } else {
 #pragma unroll
             for (int c = 0; c < BM / 64; ++c)
-              tma_load_3d_pair(sa + c * 8192, &tmA, &full[stage], arow + c * 64, k0, bb);
+              tma_load_3d_pair(sa + c * 8192, tmA, &full[stage], arow + c * 64, k0, bb);
           }
           if (!B_MN) {
-            tma_load_3d_pair(sb, &tmB, &full[stage], k0, brow, bb);
+            tma_load_3d_pair(sb, tmB, &full[stage], k0, brow, bb);
           } else {
 #pragma unroll
             for (int c = 0; c < (BN / 2) / 64; ++c)
-              tma_load_3d_pair(sb + c * 8192, &tmB, &full[stage], brow + c * 64, k0, bb);
+              tma_load_3d_pair(sb + c * 8192, tmB, &full[stage], brow + c * 64, k0, bb);
           }
           if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
         }
@@ -586,16 +622,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads<EPI>(),
     uint32_t acc_phase = 0;
     WorkIter it(sch, pair);
     Work w;
-    const int per_mat = args.tiles_m * args.tiles_n;
     while (it.next(sch, w)) {
-      const int bb = w.tile / per_mat, tr = w.tile % per_mat;
-      int tm, tn;
-      tile_coords(tr, args.tiles_m, args.tiles_n, args.raster, tm, tn);
+      int g, bb, tm, tn;
+      decode_tile<NG>(args, w.tile, g, bb, tm, tn);
       const int m = tm * 2 * BM + rank * BM + row_in_tile;
       if constexpr (epi_plain<EPI>()) {
-        if (!plain_epilogue<EPI>(args, w, bb, m, tn, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN,
-                                 rank, q, half, lane, &tfull[acc], acc_phase, abort_flag))
-          break;
+        bool ok_tile;
+        if constexpr (NG == 1) {
+          ok_tile = plain_epilogue<EPI>(args, w, bb, m, tn, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN,
+                                        rank, q, half, lane, &tfull[acc], acc_phase, abort_flag);
+        } else {
+          GemmArgs ga = args;  // problem g's output
+          ga.M = args.g_M[g];
+          ga.N = args.g_N[g];
+          ga.C = args.g_C[g];
+          ga.ldc = args.g_ldc[g];
+          ok_tile = plain_epilogue<EPI>(ga, w, 0, m, tn, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN,
+                                        rank, q, half, lane, &tfull[acc], acc_phase, abort_flag);
+        }
+        if (!ok_tile) break;
         tc_fence_before();
         mbar_arrive_leader(&tempty[acc]);
         acc ^= 1;
@@ -813,10 +858,13 @@ template <bool A_MN, bool B_MN, int EPI, bool F8 = false>
 static gpt_status launch_inst(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& a,
                               cudaStream_t stream) {
   using S = GemmShape;
-  auto kern = gemm_kernel<A_MN, B_MN, EPI, F8>;
+  auto kern = gemm_kernel<A_MN, B_MN, EPI, F8, 1>;
   GPT_TRY(ensure_smem(kern, S::SMEM_BYTES));
+  GemmMaps<1> maps;
+  maps.a[0] = ma;
+  maps.b[0] = mb;
   return launch_kernel(kern, dim3(2 * a.sched.num_pairs), dim3(gemm_threads<EPI>()), S::SMEM_BYTES,
-                       stream, ma, mb, a);
+                       stream, maps, a);
 }
 
 template <bool A_MN, bool B_MN>
@@ -978,6 +1026,67 @@ gpt_status gemm_launch_batched(const GemmBatch& g, cudaStream_t stream, void* sk
   if (op == GPT_GEMM_NT) return dispatch_epi<false, false>(epi, ma, mb, a, stream);
   if (op == GPT_GEMM_NN) return dispatch_epi<false, true>(epi, ma, mb, a, stream);
   return dispatch_epi<true, true>(epi, ma, mb, a, stream);
+}
+
+gpt_status gemm_group_tn_launch(int n, const GemmTnProblem* p, int K, int epi, int* status,
+                                cudaStream_t stream, void* sk_scratch) {
+  if (n < 1 || n > GEMM_MAX_GROUPS || !p) return GPT_ERR_INVALID_ARG;
+  if (epi != GPT_EPI_F32 && epi != GPT_EPI_F32_ADD) return GPT_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(sk_scratch) & 255) return GPT_ERR_UNSUPPORTED_SHAPE;
+  GemmMaps<GEMM_MAX_GROUPS> maps;
+  GemmArgs a{};
+  long long tiles = 0;
+  for (int g = 0; g < n; ++g)  // every argument is checked before any map is encoded
+    GPT_TRY(check_gemm_args(GPT_GEMM_TN, p[g].M, p[g].N, K, p[g].A, p[g].lda, p[g].B, p[g].ldb, p[g].C,
+                            p[g].ldc));
+  for (int g = 0; g < n; ++g) {
+    const GemmTnProblem& q = p[g];
+    if (!make_operand_map(&maps.a[g], q.A, true, q.M, K, q.lda) ||
+        !make_operand_map(&maps.b[g], q.B, true, q.N, K, q.ldb))
+      return GPT_ERR_UNSUPPORTED_SHAPE;
+    a.g_tile0[g] = (int)tiles;
+    a.g_M[g] = q.M;
+    a.g_N[g] = q.N;
+    a.g_tiles_m[g] = (q.M + 2 * BM - 1) / (2 * BM);
+    a.g_tiles_n[g] = (q.N + BN - 1) / BN;
+    a.g_C[g] = q.C;
+    a.g_ldc[g] = q.ldc;
+    tiles += (long long)a.g_tiles_m[g] * a.g_tiles_n[g];
+  }
+  for (int g = n; g < GEMM_MAX_GROUPS; ++g) maps.a[g] = maps.b[g] = maps.a[0];  // never read
+  if (tiles > (1 << 30)) return GPT_ERR_UNSUPPORTED_SHAPE;
+  a.g_tile0[n] = (int)tiles;
+  a.groups = n;
+  int sms = 0;
+  GPT_TRY(device_info(&sms));
+  // one schedule over the whole tile list (tiles_m / tiles_n / M / N are per problem here)
+  a.M = p[0].M; a.N = p[0].N; a.K = K;
+  a.tiles_m = a.tiles_n = 1;
+  a.k_tiles = (K + BK - 1) / BK;
+  a.raster = 1;
+  a.batch = 1;
+  a.alpha = 1.f;
+  a.beta = 0.f;
+  a.sched = Sched{};
+  a.sched.num_pairs = std::max(1, std::min((int)tiles, sms / 2));
+  a.sched.k_tiles = a.k_tiles;
+  a.sched.dp_tiles = (int)tiles;
+  a.status = status;
+  if (sk_scratch) {
+    Sched sk;
+    if (plan_stream_k((int)tiles, a.k_tiles, std::max(1, sms / 2), &sk)) {
+      a.sched = sk;
+      a.sk_cnt = reinterpret_cast<int*>(sk_scratch);
+      a.sk_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sk_scratch) +
+                                           ((GEMM_SK_COUNTER_BYTES + 255) & ~(size_t)255));
+    }
+  }
+  using S = GemmShape;
+  auto kern = (epi == GPT_EPI_F32) ? gemm_kernel<true, true, GPT_EPI_F32, false, GEMM_MAX_GROUPS>
+                                   : gemm_kernel<true, true, GPT_EPI_F32_ADD, false, GEMM_MAX_GROUPS>;
+  GPT_TRY(ensure_smem(kern, S::SMEM_BYTES));
+  return launch_kernel(kern, dim3(2 * a.sched.num_pairs), dim3(gemm_threads<GPT_EPI_F32>()),
+                       S::SMEM_BYTES, stream, maps, a);
 }
 
 gpt_status gemm_launch(int op, int epi, int M, int N, int K, const void* A, int lda, const void* B,
@@ -1155,6 +1264,22 @@ extern "C" gpt_status gpt_gemm_batched(int op, int epilogue, int batch, int M, i
   g.alpha = alpha; g.beta = beta; g.status = status;
   if (epilogue != GPT_EPI_AXPBY) { g.alpha = 1.f; g.beta = 0.f; }
   return gpt::gemm_launch_batched(g, gpt::as_stream(stream), nullptr);
+}
+
+extern "C" gpt_status gpt_gemm_group_tn(int n, const gpt_gemm_tn_problem* problems, int K, int epilogue,
+                                        void* scratch, int* status, void* stream) {
+  if (n < 1 || n > gpt::GEMM_MAX_GROUPS || !problems) return GPT_ERR_INVALID_ARG;
+  gpt::GemmTnProblem p[gpt::GEMM_MAX_GROUPS];
+  for (int g = 0; g < n; ++g) {
+    const gpt_gemm_tn_problem& q = problems[g];
+    p[g] = gpt::GemmTnProblem{q.M, q.N, q.A, q.lda, q.B, q.ldb, q.C, q.ldc};
+  }
+  cudaStream_t s = gpt::as_stream(stream);
+  if (scratch) {
+    if (reinterpret_cast<uintptr_t>(scratch) & 255) return GPT_ERR_UNSUPPORTED_SHAPE;
+    GPT_CUDA_TRY(cudaMemsetAsync(scratch, 0, gpt::GEMM_SK_COUNTER_BYTES, s));
+  }
+  return gpt::gemm_group_tn_launch(n, p, K, epilogue, status, s, scratch);
 }
 
 extern "C" gpt_status gpt_gemm(int op, int epilogue, int M, int N, int K, const void* A, int lda,

@@ -118,6 +118,20 @@ struct GemmBatch {
 gpt_status gemm_launch_batched(const GemmBatch& g, cudaStream_t stream, void* sk_scratch);
 // Bytes at the start of the split-tile scratch holding the arrival counters (zeroed per step).
 constexpr size_t GEMM_SK_COUNTER_BYTES = 320 * 16 * sizeof(int);
+// Grouped weight gradients: up to GEMM_MAX_GROUPS products C_g[M_g, N_g] = A_gᵀ·B_g with one K
+// (A_g [K, M_g] and B_g [K, N_g] bf16, rows lda / ldb apart; C_g fp32, rows ldc apart) in one
+// launch, their tiles dealt over the CTA pairs as one list, so that a layer's small weight
+// gradients share whole waves instead of each ending in a partly empty one.  epi: GPT_EPI_F32 or
+// GPT_EPI_F32_ADD.
+constexpr int GEMM_MAX_GROUPS = 4;
+struct GemmTnProblem {
+  int M, N;
+  const void* A; int lda;
+  const void* B; int ldb;
+  float* C; int ldc;
+};
+gpt_status gemm_group_tn_launch(int n, const GemmTnProblem* p, int K, int epi, int* status,
+                                cudaStream_t stream, void* sk_scratch);
 
 struct CeArgs {
   const int32_t* targets;

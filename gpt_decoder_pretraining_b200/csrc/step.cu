@@ -111,7 +111,7 @@ struct Plan {
   // CE
   size_t stats, zt, lse_ce, ell, inv_n, dz, dxf;
   // backward transients
-  size_t gx, gxb, du, dr, dO, dqkv, delta, emb, sk;
+  size_t gx, gxb, gxb2, du, dr, dO, dqkv, delta, emb, sk;
   size_t gacc;  // this micro-batch's gradients when the call accumulates into the caller's
   size_t total;
   int vc;  // vocabulary chunk of the backward lm-head
@@ -206,6 +206,7 @@ static Plan make_plan(const gpt_config& c, size_t n_params) {
   // backward transients
   p.gx = take(M * d * 4);
   p.gxb = take(M * d * 2);
+  p.gxb2 = take(M * d * 2);
   p.du = take(M * F * 2);
   p.dr = take(M * d * 2);
   p.dO = take(M * d * 2);
@@ -365,6 +366,7 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
   // ---------------- backward ----------------
   uint16_t* du = reinterpret_cast<uint16_t*>(ws + p.du);
   uint16_t* dr = reinterpret_cast<uint16_t*>(ws + p.dr);
+  uint16_t* gxb2 = reinterpret_cast<uint16_t*>(ws + p.gxb2);  // bf16 residual gradient at the attention branch
   uint16_t* dO = reinterpret_cast<uint16_t*>(ws + p.dO);
   uint16_t* dqkv = reinterpret_cast<uint16_t*>(ws + p.dqkv);
   float* delta = reinterpret_cast<float*>(ws + p.delta);
@@ -382,24 +384,18 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
     uint16_t* r2 = reinterpret_cast<uint16_t*>(at(p.r2, l));
     float* rho2 = reinterpret_cast<float*>(at(p.rho2, l));
     uint16_t* hsq = reinterpret_cast<uint16_t*>(at(p.hsq, l));
-    // MLP
+    // MLP (its weight gradients are formed with the attention ones, below)
     PROF(PROF_GEMM, gemm_flops(M, F, d), 0, gemm_launch(GPT_GEMM_NN, GPT_EPI_DRELU2, M, F, d, gxb, d, W(wq + 3), F, du, F, nullptr,
                         hsq, F, status, s, sk));
-    PROF(PROF_GEMM, gemm_flops(d, F, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, d, F, M, gxb, d, hsq, F, G(wq + 3), F, nullptr,
-                        nullptr, 0, status, s, sk));
-    PROF(PROF_GEMM, gemm_flops(F, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, F, d, M, du, F, r2, d, G(wq + 2), d, nullptr,
-                        nullptr, 0, status, s, sk));
     PROF(PROF_GEMM, gemm_flops(M, d, F), 0, gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, F, du, F, W(wq + 2), d, dr, d, nullptr,
                         nullptr, 0, status, s, sk));
-    PROF(PROF_NORM, 0, 14.0 * (double)M * d, rmsnorm_bwd(dr, 0, r2, rho2, gx, gxb, 1, M, d, s));
+    PROF(PROF_NORM, 0, 14.0 * (double)M * d, rmsnorm_bwd(dr, 0, r2, rho2, gx, gxb2, 1, M, d, s));
     // attention
     // dO head-major; its epilogue also forms the attention backward's delta rows (T % 64 == 0)
     AttnDeltaFusion fuse{o, os_b, os_t, lse, delta, T};
     PROF(PROF_GEMM, gemm_flops(M, d, d), 0,
-         gemm_heads_launch(GPT_GEMM_NN, M, d, d, gxb, d, W(wq + 1), d, dO, T, H, Dh, status, s,
+         gemm_heads_launch(GPT_GEMM_NN, M, d, d, gxb2, d, W(wq + 1), d, dO, T, H, Dh, status, s,
                            fuse_delta ? &fuse : nullptr));
-    PROF(PROF_GEMM, gemm_flops(d, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, d, d, M, gxb, d, o, d, G(wq + 1), d, nullptr,
-                        nullptr, 0, status, s, sk));
     PROF(PROF_ATTN_BWD, 8.0 * Dh * H * B * attn_pairs(T, st->window[l]), 0,
          attention_bwd(qkv, qkv + bhtd, qkv + bhtd + bhktd, o, dO, lse, delta, dqkv, dqkv + d,
                        dqkv + d + dkv, B, H, Hkv, T, Dh, st->window[l], lay_q, lay_kv, lay_dqkv,
@@ -409,8 +405,17 @@ static gpt_status run_step(gpt_step* st, const void* params, const int32_t* toke
       PROF(PROF_ROPE, 0, 12.0 * (double)M * d,
            rope_qknorm_bwd_heads(dqkv, qkv, rq, rk, rope, B, T, H, Dh, s));
     }
-    PROF(PROF_GEMM, gemm_flops((double)nqkv, d, M), 0, gemm_launch(GPT_GEMM_TN, GPT_EPI_F32, nqkv, d, M, dqkv, nqkv, r1, d, G(wq), d,
-                        nullptr, nullptr, 0, status, s, sk));
+    // the layer's four weight gradients in one launch: dW_proj = dyᵀ·h, dW_fc = duᵀ·r₂,
+    // dW_o = dyᵀ·o, dW_qkv = dqkvᵀ·r₁ (their tiles share whole waves instead of four partly
+    // empty last ones)
+    {
+      const GemmTnProblem wg[4] = {{(int)d, (int)F, gxb, (int)d, hsq, (int)F, G(wq + 3), (int)F},
+                                   {(int)F, (int)d, du, (int)F, r2, (int)d, G(wq + 2), (int)d},
+                                   {(int)d, (int)d, gxb2, (int)d, o, (int)d, G(wq + 1), (int)d},
+                                   {(int)nqkv, (int)d, dqkv, (int)nqkv, r1, (int)d, G(wq), (int)d}};
+      PROF(PROF_GEMM, gemm_flops(d, F, M) + gemm_flops(F, d, M) + gemm_flops(d, d, M) + gemm_flops((double)nqkv, d, M), 0,
+           gemm_group_tn_launch(4, wg, (int)M, GPT_EPI_F32, status, s, sk));
+    }
     GPT_TRY(bucket_done(1 + (c.depth - 1 - l)));
     PROF(PROF_GEMM, gemm_flops(M, d, (double)nqkv), 0, gemm_launch(GPT_GEMM_NN, GPT_EPI_BF16, M, d, nqkv, dqkv, nqkv, W(wq), d, dr, d,
                         nullptr, nullptr, 0, status, s, sk));

@@ -37,7 +37,7 @@ EXPORTED = [
     "gpt_embedding_fwd",
     "gpt_attention_bwd_scratch_bytes", "gpt_embedding_bwd_scratch_bytes", "gpt_embedding_bwd", "gpt_lmhead_ce_scratch_bytes",
     "gpt_lmhead_ce_fwd_bwd", "gpt_set_wait_limit", "gpt_debug_wait_probe", "gpt_debug_exp2_poly2",
-    "gpt_gemm_batched", "gpt_adamw_step", "gpt_muon_scratch_bytes", "gpt_muon_step",
+    "gpt_gemm_batched", "gpt_gemm_group_tn", "gpt_adamw_step", "gpt_muon_scratch_bytes", "gpt_muon_step",
     "gpt_optim_scratch_bytes", "gpt_optim_step", "gpt_gemm_e4m3", "gpt_quantize_e4m3",
     "gpt_infer_create", "gpt_infer_destroy", "gpt_infer_workspace_bytes", "gpt_infer_kv_cache_bytes",
     "gpt_prefill", "gpt_decode", "gpt_infer_status",
@@ -128,6 +128,7 @@ def lib():
         f32 = ctypes.c_float
         L.gpt_gemm_batched.argtypes = [i32, i32, i32, i32, i32, i32, vp, i32, ll, vp, i32, ll, vp, i32, ll,
                                        vp, i32, ll, f32, f32, vp, vp]
+        L.gpt_gemm_group_tn.argtypes = [i32, vp, i32, i32, vp, vp, vp]
         L.gpt_adamw_step.argtypes = [vp, vp, i32, vp, vp, vp, ll, i32, f32, f32, f32, f32, f32, vp]
         L.gpt_muon_scratch_bytes.argtypes = [i32, i32, i32]
         L.gpt_muon_scratch_bytes.restype = sz
@@ -378,6 +379,25 @@ def gemm(op: int, epi: int, A, B, C, M: int, N: int, K: int, C2=None, aux=None, 
         scratch = gemm_scratch(C.device)
     _check(lib().gpt_gemm(op, epi, M, N, K, A.data_ptr(), lda, B.data_ptr(), ldb, C.data_ptr(), ldc,
                           _ptr(C2), _ptr(aux), ldaux, _ptr(scratch), _ptr(status), _stream()), "gpt_gemm")
+
+
+class GemmTnProblem(ctypes.Structure):
+    """gpt_gemm_tn_problem: C[M, N] (fp32) (+)= Aᵀ·B with A [K, M] and B [K, N] bf16."""
+    _fields_ = [("M", ctypes.c_int), ("N", ctypes.c_int), ("A", ctypes.c_void_p), ("lda", ctypes.c_int),
+                ("B", ctypes.c_void_p), ("ldb", ctypes.c_int), ("C", ctypes.c_void_p), ("ldc", ctypes.c_int)]
+
+
+def gemm_group_tn(problems, K: int, epi: int, status=None, scratch="auto"):
+    """gpt_gemm_group_tn over [(A, B, C), …]: C = Aᵀ·B (GPT_EPI_F32) or C += Aᵀ·B (GPT_EPI_F32_ADD),
+    A [K, M], B [K, N] bf16 and C [M, N] fp32, row strides from the tensors' last dimension."""
+    arr = (GemmTnProblem * max(1, len(problems)))()
+    for i, (A, B, C) in enumerate(problems):
+        arr[i] = GemmTnProblem(C.shape[0], C.shape[1], A.data_ptr(), A.shape[-1], B.data_ptr(), B.shape[-1],
+                               C.data_ptr(), C.shape[-1])
+    if isinstance(scratch, str):
+        scratch = gemm_scratch(problems[0][2].device)
+    _check(lib().gpt_gemm_group_tn(len(problems), ctypes.addressof(arr), K, epi, _ptr(scratch), _ptr(status),
+                                   _stream()), "gpt_gemm_group_tn")
 
 
 def qkv_proj_rope(r, w_qkv, heads, rho_q, rho_k, cs, B, T, H, Dh, status=None, H_kv=None):

@@ -191,6 +191,26 @@ gpt_status gpt_gemm(int op, int epilogue, int M, int N, int K, const void* A, in
                     const void* B, int ldb, void* C, int ldc, void* C2, const void* aux,
                     int ldaux, void* scratch, int* status, void* stream);
 
+/* Grouped weight gradients ("Introducing nanochat", Pretraining: the gradients of every block
+ * matrix, which the optimizer then updates): for g < n (1 ≤ n ≤ 4), C_g[M_g, N_g] = A_gᵀ·B_g
+ * (epilogue GPT_EPI_F32) or C_g += A_gᵀ·B_g (GPT_EPI_F32_ADD), with A_g [K, M_g] and B_g [K, N_g]
+ * bf16 (row strides lda ≥ M_g, ldb ≥ N_g, multiples of 8) and C_g fp32 (ldc ≥ N_g), one K for all.
+ * The output tiles of all n products are dealt to the CTA pairs as one list, so the products of one
+ * layer (at d20: 75, 25, 100 and 100 tiles) fill whole waves together instead of each ending in a
+ * partly empty one.  scratch, status and stream as for gpt_gemm; argument errors return
+ * GPT_ERR_INVALID_ARG / GPT_ERR_UNSUPPORTED_SHAPE before anything is launched. */
+typedef struct {
+  int M, N;
+  const void* A;
+  int lda;
+  const void* B;
+  int ldb;
+  float* C;
+  int ldc;
+} gpt_gemm_tn_problem;
+gpt_status gpt_gemm_group_tn(int n, const gpt_gemm_tn_problem* problems, int K, int epilogue,
+                             void* scratch, int* status, void* stream);
+
 /* `batch` independent GEMMs of one shape and op (as gpt_gemm): matrix i of A, B, C and aux starts
  * i·*_bstride elements after matrix 0 (multiples of 8; the matrices must not overlap).  Any
  * epilogue of gpt_gemm, plus GPT_EPI_AXPBY (alpha, beta are ignored by the others).  One launch

@@ -129,6 +129,21 @@ def test_kernel_entry_points_reject_bad_arguments(lib):
                                  None, None) == -1
     assert lib.gpt_rmsnorm_fwd(None, f, f, 4, 64, None) == -1
     assert lib.gpt_embedding_bwd(f, f, f, 16, 64, 70000, f, None) == -2
+    # grouped weight gradients: 1..4 problems, fp32 epilogues only, each problem checked like gpt_gemm
+    from gpt_decoder_pretraining_b200.step import GemmTnProblem
+    probs = (GemmTnProblem * 5)(*[GemmTnProblem(64, 64, f, 64, f, 64, f, 64) for _ in range(5)])
+    grp = lib.gpt_gemm_group_tn
+    grp.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                    ctypes.c_void_p, ctypes.c_void_p]
+    p0 = ctypes.addressof(probs)
+    assert grp(0, p0, 64, 4, None, None, None) == -1      # no problem
+    assert grp(5, p0, 64, 4, None, None, None) == -1      # more than four
+    assert grp(2, p0, 64, 0, None, None, None) == -1      # bf16 epilogue
+    assert grp(2, None, 64, 4, None, None, None) == -1
+    probs[1] = GemmTnProblem(64, 64, f, 60, f, 64, f, 64)  # lda < M
+    assert grp(2, p0, 64, 4, None, None, None) == -1
+    probs[1] = GemmTnProblem(64, 64, f + 2, 64, f, 64, f, 64)  # misaligned A
+    assert grp(2, p0, 64, 5, None, None, None) == -2
 
 
 def test_multi_rank_timing_uses_the_slowest_rank():

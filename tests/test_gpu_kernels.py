@@ -139,6 +139,46 @@ def test_gemm_stream_k_tail_matches_fp64_and_is_reproducible(M, N, K, op):
     assert_close_rel(to_np(Cf), base + acc, rel=1e-5, cos=0.9999999, what="f32 add")
 
 
+# the four weight gradients of one layer in one launch: small ragged sizes; the d20 layer shapes
+# (75 + 25 + 100 + 100 tiles of 256 × 256, every tile whole at K = 4096); and 32 + 16 + 24 + 6 = 78
+# tiles at K = 16384, one whole wave of 74 pairs and 4 tail tiles split along K
+GROUP_CASES = [
+    (512, [(296, 200), (136, 384), (520, 256), (64, 64)]),
+    (4096, [(3840, 1280), (1280, 1280), (5120, 1280), (1280, 5120)]),
+    (16384, [(2048, 1024), (1024, 1024), (1536, 1024), (768, 512)]),
+]
+
+
+@pytest.mark.parametrize("K,shapes", GROUP_CASES)
+def test_gemm_group_tn_matches_fp64_and_single_products(K, shapes):
+    rng = np.random.default_rng(K + len(shapes))
+    probs, refs = [], []
+    for M, N in shapes:
+        A, B = randn(rng, K, M), randn(rng, K, N)
+        refs.append(A.T @ B)
+        probs.append((bf16_tensor(A), bf16_tensor(B), torch.full((M, N), float("nan"), device="cuda")))
+    st = _status()
+    S.gemm_group_tn(probs, K, S.EPI_F32, status=st)
+    again = [torch.full_like(c, float("nan")) for _, _, c in probs]
+    S.gemm_group_tn([(a, b, c) for (a, b, _), c in zip(probs, again)], K, S.EPI_F32, status=st)
+    # accumulate form on a base
+    bases = [rng.standard_normal(r.shape).astype(np.float32) for r in refs]
+    accs = [torch.from_numpy(b).cuda() for b in bases]
+    S.gemm_group_tn([(a, b, c) for (a, b, _), c in zip(probs, accs)], K, S.EPI_F32_ADD, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    tol = f32_accum_rel(K)
+    for (a, b, c), c2, acc, base, ref, (M, N) in zip(probs, again, accs, bases, refs, shapes):
+        assert_close_rel(to_np(c), ref, rel=tol, cos=0.9999999, what=f"grouped {M}x{N}")
+        assert torch.equal(c, c2)  # bitwise reproducible
+        assert_close_rel(to_np(acc), base + ref, rel=tol, cos=0.9999999, what=f"grouped add {M}x{N}")
+        one = torch.zeros_like(c)
+        S.gemm(2, S.EPI_F32, a, b, one, M, N, K, status=st)
+        torch.cuda.synchronize()
+        # the same products on their own differ only in fp32 summation order (split tiles)
+        assert_close_rel(to_np(c), to_np(one), rel=2 * tol, cos=0.9999999, what=f"grouped vs single {M}x{N}")
+
+
 def test_gemm_rejects_bad_arguments():
     t = torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(S.GptError):
