@@ -560,6 +560,20 @@ def run_kernel(args):
         run = lambda: S.gemm(op, epi, A, B, C, M, N, K, aux=aux, scratch=scratch)  # noqa: E731
         flops = 2.0 * M * N * K
         unit_desc = f"GEMM {args.gemm_op} M={M} N={N} K={K}"
+    elif args.kernel == "wgrad":
+        # one layer's four weight gradients in one grouped launch: dW_proj [d, 4d], dW_fc [4d, d],
+        # dW_o [d, d], dW_qkv [3d, d], all over K = tokens
+        K, d = (int(x) for x in args.wgrad.split(","))
+        shapes = [(d, 4 * d), (4 * d, d), (d, d), (3 * d, d)]
+        probs = []
+        for Mw, Nw in shapes:
+            A = torch.randn(K, Mw, device=dev, generator=g).to(torch.bfloat16)
+            B = torch.randn(K, Nw, device=dev, generator=g).to(torch.bfloat16)
+            probs.append((A, B, torch.empty(Mw, Nw, device=dev)))
+        scratch = None if args.no_stream_k else "auto"
+        run = lambda: S.gemm_group_tn(probs, K, S.EPI_F32, scratch=scratch)  # noqa: E731
+        flops = 2.0 * K * sum(Mw * Nw for Mw, Nw in shapes)
+        unit_desc = f"grouped weight gradients K={K} d={d} (d x 4d, 4d x d, d x d, 3d x d)"
     elif args.kernel == "qkv":
         # QKV projection with the RoPE + QK-norm epilogue: r [M, d] · W_qkv [3d, d]ᵀ → q̃, k̃, v head-major
         M, d, H = (int(x) for x in args.qkv.split(","))
@@ -675,7 +689,8 @@ def main():
     ap.add_argument("--norm-pass", default="fwd", choices=["fwd", "bwd"])
     ap.add_argument("--emb", default="32768,1536,32768", help="embedding workload: M,d,V")
     ap.add_argument("--qkv", default="8192,1536,12", help="QKV projection workload: tokens,d,heads")
-    ap.add_argument("--kernel", choices=["gemm", "attention", "rmsnorm", "embedding", "qkv"], default=None,
+    ap.add_argument("--wgrad", default="32768,1536", help="grouped weight-gradient workload: tokens,d")
+    ap.add_argument("--kernel", choices=["gemm", "attention", "rmsnorm", "embedding", "qkv", "wgrad"], default=None,
                     help="time one kernel-level workload instead of the step")
     ap.add_argument("--gemm-shape", default="32768,6144,1536")
     ap.add_argument("--gemm-op", default="nt", choices=["nt", "nn", "tn"])
