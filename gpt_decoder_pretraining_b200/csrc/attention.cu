@@ -966,17 +966,17 @@ __global__ void __launch_bounds__(576, 1)
       // fp32 for phase 2 and written back packed
       float p[32];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int qc = qh + 16 * c;
-        uint32_t rs[16];
-        tmem_ld16(tmem + lane_off + S::TM_S + grp * 64 + 32 * half + 16 * c, rs);
+      for (int c = 0; c < 4; ++c) {  // 8-column chunks
+        const int qc = qh + 8 * c;
+        uint32_t rs[8];
+        tmem_ld8(tmem + lane_off + S::TM_S + grp * 64 + 32 * half + 8 * c, rs);
         tmem_ld_wait();
         // every (key, query) of the chunk visible: no per-element mask
-        const bool full = (kmax_ <= qc) && (kmin > qc + 15 - W) && (qc + 15 < T);
-        uint32_t pk[8];
+        const bool full = (kmax_ <= qc) && (kmin > qc + 7 - W) && (qc + 7 < T);
+        uint32_t pk[4];
 #pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(ldl + 16 * c + 4 * g4);  // LSE·log2 e
+        for (int g4 = 0; g4 < 2; ++g4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(ldl + 8 * c + 4 * g4);  // LSE·log2 e
 #pragma unroll
           for (int e2 = 0; e2 < 2; ++e2) {
             const int j = 4 * g4 + 2 * e2;
@@ -989,45 +989,45 @@ __global__ void __launch_bounds__(576, 1)
               if (!((qq < T) && (key <= qq) && (key > qq - W))) p0 = 0.f;
               if (!((qq + 1 < T) && (key <= qq + 1) && (key > qq + 1 - W))) p1 = 0.f;
             }
-            p[16 * c + j] = p0;
-            p[16 * c + j + 1] = p1;
+            p[8 * c + j] = p0;
+            p[8 * c + j + 1] = p1;
             pk[j / 2] = pack_bf2(p0, p1);
           }
         }
-        // packed: chunk c of half h fills columns 32h + 8c .. +7, inside what this warp has read
-        tmem_st8(tmem + lane_off + S::TM_S + grp * 64 + 32 * half + 8 * c, pk);
+        // packed: chunk c of half h fills columns 32h + 4c .. +3, inside what this warp has read
+        tmem_st4(tmem + lane_off + S::TM_S + grp * 64 + 32 * half + 4 * c, pk);
       }
       // phase 2: dSᵀ = Pᵀ∘(dPᵀ − delta)
       if (!mbar_wait_warp(&dp_full[grp], (i >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t rp[16];
-        tmem_ld16(tmem + lane_off + S::TM_P + grp * 64 + 32 * half + 16 * c, rp);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rp[8];
+        tmem_ld8(tmem + lane_off + S::TM_P + grp * 64 + 32 * half + 8 * c, rp);
         tmem_ld_wait();
-        uint32_t dk[8];
+        uint32_t dk[4];
 #pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
-          const float4 d4 = *reinterpret_cast<const float4*>(ldl + 64 + 16 * c + 4 * g4);  // delta
+        for (int g4 = 0; g4 < 2; ++g4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(ldl + 64 + 8 * c + 4 * g4);  // delta
 #pragma unroll
           for (int e2 = 0; e2 < 2; ++e2) {
             const int j = 4 * g4 + 2 * e2;
             float u0, u1, s0, s1;
             sub2(u0, u1, __uint_as_float(rp[j]), __uint_as_float(rp[j + 1]), e2 ? d4.z : d4.x, e2 ? d4.w : d4.y);
-            mul2(s0, s1, p[16 * c + j], p[16 * c + j + 1], u0, u1);
+            mul2(s0, s1, p[8 * c + j], p[8 * c + j + 1], u0, u1);
             dk[j / 2] = pack_bf2(s0, s1);
           }
         }
         if (a.ds != nullptr) {
           // staging row = query, column = key (this lane): every row write is 64 contiguous bytes
-          uint16_t* row0 = reinterpret_cast<uint16_t*>(ds_stage) + (16 * c) * 32 + lane;
+          uint16_t* row0 = reinterpret_cast<uint16_t*>(ds_stage) + (8 * c) * 32 + lane;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
+          for (int e = 0; e < 4; ++e) {
             row0[(2 * e) * 32] = (uint16_t)(dk[e] & 0xFFFFu);
             row0[(2 * e + 1) * 32] = (uint16_t)(dk[e] >> 16);
           }
         }
-        tmem_st8(tmem + lane_off + S::TM_P + grp * 64 + 32 * half + 8 * c, dk);
+        tmem_st4(tmem + lane_off + S::TM_P + grp * 64 + 32 * half + 4 * c, dk);
       }
       tmem_st_wait();
       tc_fence_before();
