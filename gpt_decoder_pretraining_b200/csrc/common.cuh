@@ -115,14 +115,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
-                                            int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
-      "%4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
-      : "memory");
-}
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
                                             int y, int z) {
   asm volatile(
@@ -294,18 +286,6 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return d;
 }
 
-// Shared-memory descriptor for an unswizzled K-major tile of 8-row × 16-byte core matrices:
-// lbo_bytes = distance between core matrices adjacent along K, sbo_bytes = along M/N.
-__device__ __forceinline__ uint64_t sdesc_plain(uint32_t saddr, uint32_t lbo_bytes,
-                                                uint32_t sbo_bytes) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;  // descriptor version for tcgen05; layout type 0 = no swizzle
-  return d;
-}
-
 // A descriptor advanced by `bytes` (a multiple of 16 that keeps the address inside shared memory):
 // the start address sits in the low 14 bits as address >> 4, so this is one integer add.  Issue
 // loops form their descriptors this way from bases computed once, keeping the MMA thread's
@@ -391,18 +371,8 @@ __device__ __forceinline__ void mbar_arrive_leader(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(smem_u32(bar) & PAIR_LEADER_MASK)
                : "memory");
 }
-// TMA tile load into this CTA's shared memory whose completion is counted on the leader CTA's
-// barrier (no multicast).
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                                 int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(smem_u32(bar) & PAIR_LEADER_MASK), "r"(x), "r"(y)
-      : "memory");
-}
-
-// Same, for a 3-d tensor map (the third coordinate selects the matrix of a batch).
+// TMA tile load (3-d tensor map; the third coordinate selects the matrix of a batch) into this
+// CTA's shared memory whose completion is counted on the leader CTA's barrier (no multicast).
 __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint64_t* bar,
                                                  int x, int y, int z) {
   asm volatile(
@@ -458,16 +428,6 @@ __device__ __forceinline__ void add2_bc(float& d0, float& d1, float a0, float a1
       "mov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(c));
-}
-// (d0, d1) = (a0·b, a1·b)
-__device__ __forceinline__ void mul2_b(float& d0, float& d1, float a0, float a1, float b) {
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\t"
-      "mov.b64 rb, {%4, %4};\n\t"
-      "mul.rn.f32x2 rd, ra, rb;\n\t"
-      "mov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b));
 }
 // (d0, d1) = (a0·b0, a1·b1)
 __device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
