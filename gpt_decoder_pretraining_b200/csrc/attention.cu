@@ -1314,13 +1314,15 @@ __global__ void __launch_bounds__(320, 1)
 // overlap the other's stream of dS tiles: the kernel is bound by reading dS from HBM.
 template <int DH>
 struct DqDsShape {
-  static constexpr int STAGES = 2;
+  static constexpr int STAGES = 3;
   static constexpr int Q_TILE = 128 * DH * 2;   // q̃ tile (the QK-norm + RoPE backward reads it)
   static constexpr int DS_TILE = 128 * 64 * 2;  // [128 queries][64 keys]
   static constexpr int K_TILE = 64 * DH * 2;
   static constexpr int STAGE_BYTES = DS_TILE + K_TILE;
+  // the q̃ tile is loaded over ring stage 0 once its last product is done (only the epilogue reads it)
+  static constexpr int OFF_STAGE = 0;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_STAGE = Q_TILE;
+  static_assert(Q_TILE <= STAGE_BYTES, "q tile inside ring stage 0");
   static constexpr int OFF_BAR = OFF_STAGE + STAGES * STAGE_BYTES;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr int THREADS = 192;  // 4 epilogue warps, TMA warp, MMA warp
@@ -1377,16 +1379,22 @@ __global__ void __launch_bounds__(192, 2)
   if (warp == 4) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_bar, S::Q_TILE);
-      load_tile<DH, 128>(smem + S::OFF_Q, &mq, q_bar, q0, h, b);
+      bool ok = true;
       for (int j = 0; j < n_kv; ++j) {
         const int st = j % S::STAGES;
-        if (!mbar_wait(&empty[st], ((j / S::STAGES) & 1) ^ 1, abort_flag, a.status)) break;
+        if (!mbar_wait(&empty[st], ((j / S::STAGES) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
         mbar_arrive_expect_tx(&full[st], S::STAGE_BYTES);
         uint8_t* dst = smem + S::OFF_STAGE + st * S::STAGE_BYTES;
         const int k0 = (kv_first + j) * 64;
         tma_load_3d(dst, &mds, &full[st], k0, q0, bh_ds);  // dS rows q0 .. q0+127, keys k0 .. k0+63
         load_tile<DH, 64>(dst + S::DS_TILE, &mk, &full[st], k0, h / a.group, b);
+      }
+      // q̃ over stage 0 once its last product (tile j0) has read it; the products of the last
+      // tiles in stages 1 and 2 may still run
+      const int j0 = ((n_kv - 1) / S::STAGES) * S::STAGES;
+      if (ok && a.rho_q != nullptr && mbar_wait(&empty[0], (j0 / S::STAGES) & 1, abort_flag, a.status)) {
+        mbar_arrive_expect_tx(q_bar, S::Q_TILE);
+        load_tile<DH, 128>(smem + S::OFF_Q, &mq, q_bar, q0, h, b);
       }
     }
   } else if (warp == 5) {
@@ -1418,8 +1426,8 @@ __global__ void __launch_bounds__(192, 2)
     const int row = 32 * warp + lane;
     const int t = q0 + row;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
-    bool ok = mbar_wait_warp(q_bar, 0, abort_flag, a.status);
-    if (ok) ok = mbar_wait_warp(done, 0, abort_flag, a.status);
+    bool ok = mbar_wait_warp(done, 0, abort_flag, a.status);
+    if (ok && a.rho_q != nullptr) ok = mbar_wait_warp(q_bar, 0, abort_flag, a.status);
     if (ok) {
       tc_fence_after();
       uint16_t* dst = a.o + b * a.sb_o + h * a.sh_o + (long long)t * a.st_o;
